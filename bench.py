@@ -1,0 +1,483 @@
+#!/usr/bin/env python
+"""Benchmark of the fused matmul-sample (FMMS) step; prints one JSON line.
+
+One step = one fused LM-head matmul + temperature + Gumbel noise + argmax call
+(fs_sample_ex) over one batch of B rows of a Qwen3-8B-shaped head
+(d=4096, V=151936, bf16, T=0.7, per-row seeds) with inputs resident in HBM.
+Weights (1.24 GB) exceed the 126 MB L2, so no flush is needed between steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--batch B]
+  python bench.py --impl reference ...   # the CPU oracle, timed the same way
+
+Under torchrun each rank runs an independent replica (the path has no
+data-path exchange at one GPU per replica); timings are the max over ranks.
+"""
+import argparse
+import hashlib
+import json
+import os
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "FMMS µs/call & HBM GB/s (% roofline), d=4096 V=151936 bf16, B=1–256"
+UNIT = "us/call"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+KERNEL_SOURCES = ["lm_head_exact_fmms_b200/csrc/fmms_kernel.cu",
+                  "lm_head_exact_fmms_b200/csrc/noise.cuh",
+                  "lm_head_exact_fmms_b200/csrc/sm100.cuh",
+                  "lm_head_exact_fmms_b200/csrc/fmms_common.cuh"]
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--batch", type=int, default=64)
+    ap.add_argument("--workload", default="qwen3-8b")
+    ap.add_argument("--impl", default="fmms", choices=["fmms", "reference"])
+    ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------- helpers
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(workload_key):
+    """Per-launch DRAM bytes from the committed ncu summary, if it was taken
+    on the current kernel source for this workload; else None."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    with open(TRAFFIC_FILE) as f:
+        t = json.load(f)
+    if t.get("kernel_source_sha") != kernel_source_hash():
+        return None
+    entry = t.get("workloads", {}).get(workload_key)
+    return None if entry is None else entry.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons while the timed region runs
+    (NVML, the library nvidia-smi reads; nvidia-smi itself as fallback)."""
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, index, period=0.01):
+        self.index, self.period = index, period
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        self._nvml = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nvml = None
+
+    def _reasons(self):
+        n = self._nvml
+        fn = getattr(n, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            getattr(n, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        return fn(self._h)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self._nvml.nvmlDeviceGetClockInfo(self._h, self._nvml.NVML_CLOCK_SM))
+                bits = self._reasons()
+                for b, name in self.REASONS.items():
+                    if bits & b:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self._nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        else:
+            import subprocess
+            self._proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index),
+                 "--query-gpu=clocks.sm,clocks.max.sm,clocks_event_reasons.active",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+
+    def stop(self):
+        if self._nvml is not None:
+            self._stop.set()
+            self._thread.join()
+        elif getattr(self, "_proc", None) is not None:
+            self._proc.terminate()
+            out, _ = self._proc.communicate()
+            for line in out.strip().splitlines():
+                try:
+                    sm, mx, act = [x.strip() for x in line.split(",")]
+                    self.samples.append(int(sm))
+                    self.max_mhz = int(mx)
+                    bits = int(act, 16)
+                    for b, name in self.REASONS.items():
+                        if bits & b:
+                            self.reasons.add(name)
+                except Exception:
+                    pass
+
+    def summary(self):
+        s = sorted(self.samples)
+        med = s[len(s) // 2] if s else None
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(s)}
+
+
+def dist_setup():
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def algorithmic(B, d, V, masked):
+    """Bytes that must cross HBM and flops of one call."""
+    nbytes = V * d * 2 + B * d * 2 + B * 4
+    if masked:
+        nbytes += B * ((V + 31) // 32) * 4
+    return nbytes, 2.0 * B * V * d
+
+
+def roofline(B, d, V, masked, kernel_us, peaks, peak_kind, traffic):
+    nbytes, flops = algorithmic(B, d, V, masked)
+    t_mem = nbytes / (peaks["hbm_gbs"] * 1e9)
+    t_tc = flops / (peaks["bf16_tflops_sustained"] * 1e12)
+    if t_mem >= t_tc:
+        achieved = nbytes / (kernel_us * 1e-6) / 1e9
+        r = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    else:
+        achieved = flops / (kernel_us * 1e-6) / 1e12
+        r = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops_sustained"],
+             "unit": "TFLOP/s"}
+    r["frac"] = r["achieved"] / r["peak"]
+    r["traffic"] = traffic
+    r["peak_source"] = "%s (MEASURED_PEAKS.json)" % peak_kind if peak_kind == "measured" else "fallback"
+    r["algorithmic_bytes"] = nbytes
+    r["algorithmic_flops"] = flops
+    return r
+
+
+# ------------------------------------------------------------ the GPU arm
+def time_calls(fn, steps, warmup, stream, world=1, sampler=None):
+    """Times exactly `steps` calls after `warmup` untimed ones.  Returns
+    (region ms, per-call event durations in us)."""
+    import torch
+    for i in range(warmup):
+        fn(i)
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    r0 = torch.cuda.Event(enable_timing=True)
+    r1 = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+    r0.record(stream)
+    for i in range(steps):
+        starts[i].record(stream)
+        fn(warmup + i)
+        ends[i].record(stream)
+    r1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    if sampler:
+        sampler.stop()
+    per = [s.elapsed_time(e) * 1e3 for s, e in zip(starts, ends)]
+    return r0.elapsed_time(r1), per
+
+
+def median(xs):
+    s = sorted(xs)
+    return s[len(s) // 2]
+
+
+def cpu_baseline(H, W, wl, B, rs, budget_s=12.0, max_rows=64):
+    """The oracle as it stands, on this host's cores, over a bounded sample of
+    the workload's rows; scaled to us per B-row call."""
+    import numpy as np
+    import oracle
+    Hc, Wc = H.cpu(), W.cpu()
+    rsc = rs.cpu() if rs is not None else None
+    times = []
+    t_start = time.time()
+    for r in range(min(B, max_rows)):
+        t0 = time.perf_counter()
+        oracle.sample(Hc, Wc, T=wl.temperature, seed=0, row_seeds=rsc, step=0,
+                      rows=np.array([r], dtype=np.int32))
+        times.append(time.perf_counter() - t0)
+        if time.time() - t_start > budget_s:
+            break
+    per_row = sum(times) / len(times)
+    return {"value": per_row * B * 1e6, "unit": UNIT, "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": "%d of the %d rows of one B=%d call (full vocabulary each), fp64 oracle; "
+                      "value = mean row time x %d rows" % (len(times), B, B, B),
+            "seconds": round(sum(times), 2)}
+
+
+def run_gpu(args, world, rank, local):
+    import torch
+
+    from lm_head_exact_fmms_b200 import binding, synth
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    binding.load_library()
+    wl = synth.WORKLOADS[args.workload]
+    B = args.batch
+    stream = torch.cuda.current_stream()
+    peaks, peak_kind = load_peaks()
+
+    W = synth.make_weight(wl.V, wl.d, wl.w_std, device=dev)
+    H = synth.make_hidden(B, wl.d, device=dev)
+    rs = synth.make_row_seeds(B, device=dev) if wl.per_row_seeds else None
+    out = torch.empty(B, dtype=torch.int32, device=dev)
+    ws = torch.zeros(binding.fs_workspace_bytes(B, wl.V, 0), dtype=torch.uint8, device=dev)
+
+    def step(i):
+        binding.fs_sample_ex(H, W, temperature=wl.temperature, seed=0, row_seeds=rs, step=i,
+                             out_idx=out, workspace=ws, stream=stream)
+
+    sampler = ClockSampler(local)
+    region_ms, per_call = time_calls(step, args.steps, args.warmup, stream, world, sampler)
+    region_ms = max_over_ranks(region_ms, world)
+    kernel_us = sum(per_call) / len(per_call)
+    kernel_us = max_over_ranks(kernel_us, world)
+    us_per_call = region_ms * 1e3 / args.steps
+    nbytes, flops = algorithmic(B, wl.d, wl.V, False)
+    launches_per_call = (B + 255) // 256
+
+    # e2e: host buffers through the public C entry point (H2D + kernel + D2H).
+    Hh = H.cpu().pin_memory()
+    Oh = torch.empty(B, dtype=torch.int32).pin_memory()
+
+    def step_host(i):
+        binding.fs_sample_host(Hh, W, temperature=wl.temperature, seed=0, row_seeds=rs, step=i,
+                               out_idx_host=Oh, stream=stream)
+
+    e2e_ms, _ = time_calls(step_host, args.steps, args.warmup, stream, world)
+    e2e_ms = max_over_ranks(e2e_ms, world)
+
+    result = {
+        "metric": METRIC, "value": round(us_per_call, 3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(region_ms / args.steps, 6),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: seeded H ~ N(0,1), W ~ N(0, %g^2) bf16 (random-init %s head)"
+                % (wl.w_std, wl.name),
+        "config": {"workload": "%s LM head, d=%d V=%d B=%d T=%g%s, fused fs_sample_ex"
+                               % (wl.name, wl.d, wl.V, B, wl.temperature,
+                                  ", per-row seeds" if wl.per_row_seeds else ""),
+                   "batch_per_gpu": B, "global_batch": B * world, "d": wl.d, "V": wl.V,
+                   "parallelism": "replicas x%d" % world,
+                   "l2": "no flush: W (%.2f GB) exceeds the 126 MB L2" % (wl.V * wl.d * 2 / 1e9)},
+        "samples_per_s": round(B * world / (us_per_call * 1e-6), 1),
+        "hbm_gbs_per_gpu": round(nbytes / (us_per_call * 1e-6) / 1e9, 1),
+        "kernel_us": round(kernel_us, 3),
+        "roofline": roofline(B, wl.d, wl.V, False, kernel_us, peaks, peak_kind,
+                             committed_traffic("%s/B%d" % (wl.name, B))),
+        "e2e": {"value": round(e2e_ms * 1e3 / args.steps, 3), "unit": UNIT,
+                "h2d_bytes_per_step": B * wl.d * 2, "d2h_bytes_per_step": B * 4,
+                "entry_point": "fs_sample_host (pinned host H in, host tokens out)"},
+        "gpu_launches": args.steps * launches_per_call,
+        "clocks": sampler.summary(),
+    }
+
+    if rank == 0 and not args.no_sweep:
+        result["sweep"] = sweep(torch, binding, synth, W, wl, dev, stream, peaks, peak_kind)
+        result["grouped_masked"] = grouped_point(torch, binding, synth, dev, stream, peaks,
+                                                 peak_kind, W)
+        result["unfused"] = unfused_point(torch, binding, synth, W, wl, dev, stream, B)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(H, W, wl, B, rs)
+    return result
+
+
+def sweep(torch, binding, synth, W, wl, dev, stream, peaks, peak_kind, steps=200, warmup=10):
+    rows = []
+    for B in wl.batches:
+        H = synth.make_hidden(B, wl.d, device=dev)
+        rs = synth.make_row_seeds(B, device=dev) if wl.per_row_seeds else None
+        out = torch.empty(B, dtype=torch.int32, device=dev)
+
+        def step(i):
+            binding.fs_sample_ex(H, W, temperature=wl.temperature, seed=0, row_seeds=rs, step=i,
+                                 out_idx=out, stream=stream)
+
+        region_ms, per = time_calls(step, steps, warmup, stream)
+        kus = sum(per) / len(per)
+        rf = roofline(B, wl.d, wl.V, False, kus, peaks, peak_kind,
+                      committed_traffic("%s/B%d" % (wl.name, B)))
+        rows.append({"B": B, "us_per_call": round(region_ms * 1e3 / steps, 3),
+                     "kernel_us": round(kus, 3), "bound": rf["bound"],
+                     "achieved": round(rf["achieved"], 1), "unit": rf["unit"],
+                     "frac": round(rf["frac"], 4)})
+    return rows
+
+
+def grouped_point(torch, binding, synth, dev, stream, peaks, peak_kind, W8, B=64, steps=100):
+    wl = synth.WORKLOADS["grouped-masked"]
+    H = synth.make_hidden(B, wl.d, device=dev)
+    mask = synth.make_mask(B, wl.V, wl.mask_allowed).to(dev)
+    out = torch.empty(B, dtype=torch.int32, device=dev)
+    W = W8 if (W8.shape[0] == wl.V and W8.shape[1] == wl.d) else \
+        synth.make_weight(wl.V, wl.d, wl.w_std, device=dev)
+
+    def step(i):
+        binding.fs_sample_grouped(H, W, wl.groups, temperature=wl.temperature, seed=0, step=i,
+                                  mask_bits=mask, out_idx=out, stream=stream)
+
+    region_ms, per = time_calls(step, steps, 10, stream)
+    us = region_ms * 1e3 / steps
+    rf = roofline(B, wl.d, wl.V, True, us, peaks, peak_kind, None)
+    return {"workload": "grouped-masked d=%d V=%d G=%d B=%d 50%% mask T=%g (2 kernels per call)"
+                        % (wl.d, wl.V, wl.groups, B, wl.temperature),
+            "us_per_call": round(us, 3), "bound": rf["bound"], "achieved": round(rf["achieved"], 1),
+            "unit": rf["unit"], "frac": round(rf["frac"], 4)}
+
+
+def unfused_point(torch, binding, synth, W, wl, dev, stream, B, steps=100):
+    H = synth.make_hidden(B, wl.d, device=dev)
+    rs = synth.make_row_seeds(B, device=dev) if wl.per_row_seeds else None
+    out = torch.empty(B, dtype=torch.int32, device=dev)
+    logits = torch.empty(B, wl.V, dtype=torch.float32, device=dev)
+
+    def step(i):
+        binding.fs_sample_unfused(H, W, temperature=wl.temperature, seed=0, row_seeds=rs, step=i,
+                                  out_idx=out, logits=logits, stream=stream)
+
+    region_ms, _ = time_calls(step, steps, 10, stream)
+    return {"us_per_call": round(region_ms * 1e3 / steps, 3),
+            "extra_hbm_bytes_per_call": 2 * B * wl.V * 4,
+            "note": "matmul writes fp32 logits [B,V], a second kernel reads them back"}
+
+
+# ------------------------------------------------------ the reference arm
+def run_reference(args, world, rank):
+    """The CPU oracle timed on this host's cores, on the same workload, metric
+    and unit; each step is a bounded sample (one row over a vocabulary slice)."""
+    if rank != 0:
+        return None
+    import numpy as np
+    import torch
+
+    import oracle
+    from lm_head_exact_fmms_b200 import synth
+    wl = synth.WORKLOADS[args.workload]
+    B = args.batch
+    H = synth.make_hidden(B, wl.d)
+    # a vocabulary slice of the head; the full head would take minutes per step
+    total = args.steps + args.warmup
+    budget = 120.0 / max(total, 1)
+    probe_V = 4096
+    Wp = synth.make_weight(probe_V, wl.d, wl.w_std)
+    rs = synth.make_row_seeds(B) if wl.per_row_seeds else None
+    t0 = time.perf_counter()
+    oracle.sample(H, Wp, T=wl.temperature, row_seeds=rs, rows=np.array([0], dtype=np.int32))
+    t_probe = max(time.perf_counter() - t0, 1e-6)
+    Vs = int(max(64, min(wl.V, probe_V * budget / t_probe)))
+    Ws = synth.make_weight(Vs, wl.d, wl.w_std)
+    times = []
+    for i in range(total):
+        r = np.array([i % B], dtype=np.int32)
+        t0 = time.perf_counter()
+        oracle.sample(H, Ws, T=wl.temperature, row_seeds=rs, step=i, rows=r)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            times.append(dt)
+    scale = (wl.V / Vs) * B
+    value = sum(times) / len(times) * scale * 1e6
+    cores = oracle.num_threads()
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 1), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(sum(times) / len(times) * 1e3, 3), "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "%s LM head, d=%d V=%d B=%d T=%g" % (wl.name, wl.d, wl.V, B,
+                                                                   wl.temperature),
+                   "global_batch": B, "parallelism": "CPU oracle, %d threads" % cores},
+        "cpu_baseline": {"value": round(value, 1), "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": "each step: 1 row x %d-token vocabulary slice; value scaled "
+                                   "by (V/%d) x B" % (Vs, Vs)},
+        "e2e": {"value": round(value, 1), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        res = run_reference(args, world, rank)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    world, rank, local = dist_setup()
+    res = run_gpu(args, world, rank, local)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

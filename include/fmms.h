@@ -1,0 +1,197 @@
+/*
+ * fmms.h -- C ABI of the FlashSampling fused matmul-sample (FMMS) library for
+ * NVIDIA B200 (sm_100a), libfmms.so.
+ *
+ * The method (FlashSampling: Fast and Memory-Efficient Exact Sampling,
+ * Ruiz et al., arXiv:2603.15854, abstract): the LM-head logits
+ * l = h W^T are computed tile by tile on chip, Gumbel noise is added, only
+ * one maximiser per row and per vocabulary tile is kept, and a small
+ * reduction over tiles returns one sampled token per row.  The B x V logits
+ * tensor never reaches HBM.  It is exact because argmax decomposes over a
+ * partition of the vocabulary (Gumbel-Max theorem, readus.org page, section
+ * "Gumbel Max Trick").
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  H      hidden states, bf16 [B, d], row-major (row b is contiguous).
+ *  W      LM-head weight, bf16 [V, d], row-major (the nn.Linear layout).
+ *         Both base addresses must be 16-byte aligned and d % 8 == 0 (rows
+ *         are read by TMA with 16-byte strides).  B >= 1, V >= 1.
+ *  temperature  T > 0 and finite; scores are x = l / T.  The Gumbel noise is
+ *         not scaled by T (readus.org page, "API": temperature is an argument
+ *         of the sampling call).
+ *  mask_bits  optional per-row vocab bitmask, uint32 [B][ceil(V/32)]: bit
+ *         (v & 31) of word [b][v >> 5] is 1 when token v is allowed.
+ *         Forbidden tokens get score -inf before the noise, so they are never
+ *         sampled (readus.org page, "Top-K and masking").  NULL = all allowed.
+ *  seed, row_seeds, step  the noise for (row b, token v) is word (v & 3) of
+ *         Philox4x32-10 (Salmon et al., SC'11) with key = (k lo32, k hi32),
+ *         k = row_seeds[b] if row_seeds is non-NULL else seed, and counter
+ *         (v >> 2, b, step, 0).  The noise is therefore a pure function of
+ *         (seed, step, row, token): the same call gives the same tokens on
+ *         any device, stream or tiling (readus.org page, "seed management").
+ *  noise  g = -log(-log u), u = (r + 1) / (2^32 + 1) for the noise word r
+ *         (readus.org page, "floating point precision"); u never reaches 0
+ *         or 1, so g is always finite.
+ *  out_idx  int32 [B]: the sampled token of each row, the smallest v
+ *         attaining max_v (x[b,v] + g[b,v]); -1 when every token of the row is
+ *         masked (a per-row result, not an error).
+ *  stream  a cudaStream_t passed as an opaque pointer; NULL is the legacy
+ *         default stream.  Every entry point is asynchronous on `stream`
+ *         unless stated otherwise: it validates its arguments, enqueues its
+ *         kernels and returns.  Output buffers are valid once the stream has
+ *         reached that point; the caller keeps every buffer alive until then.
+ *  memory  unless stated otherwise every array pointer is a DEVICE pointer on
+ *         the current device, owned by the caller.  The library keeps no
+ *         pointer past the call.
+ *  workspace  entry points that take (workspace, workspace_bytes) use the
+ *         caller's device buffer of at least fs_workspace_bytes(B, V, G) bytes,
+ *         256-byte aligned, which must be zero-filled before its first use
+ *         (cudaMemset) and is left zeroed by every call that completes.
+ *         Calls that share a workspace must be ordered on one stream.  With
+ *         workspace == NULL the library uses its own per-device workspace,
+ *         allocated on first use; such calls must not run concurrently on
+ *         different streams.
+ *  errors  argument errors are detected on the host before anything is
+ *         enqueued and returned synchronously; launch failures return
+ *         FS_ERR_CUDA.  A device-side wait that exceeds its time limit (about
+ *         one second) makes the kernel record FS_ERR_DEVICE_TIMEOUT in the
+ *         workspace and exit early; fs_device_status() reports it.
+ */
+#ifndef FMMS_H_
+#define FMMS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FS_OK = 0,
+  FS_ERR_INVALID_ARG = 1,    /* a pointer, size, alignment or value is invalid */
+  FS_ERR_UNSUPPORTED = 2,    /* no sm_100 device, or a shape outside the supported range */
+  FS_ERR_CUDA = 3,           /* a CUDA runtime/driver call or a launch failed */
+  FS_ERR_WORKSPACE = 4,      /* the workspace is too small or misaligned */
+  FS_ERR_DEVICE_TIMEOUT = 5  /* a kernel gave up on a bounded wait (see fs_device_status) */
+} fs_status;
+
+/* A cudaStream_t, passed without the CUDA headers. */
+typedef void *fs_stream_t;
+
+/* Per-(row, group) summary of the grouped sampler. */
+typedef struct {
+  float max_score; /* max over the group of x + g (-inf if the group is fully masked) */
+  int32_t argmax;  /* the token attaining it (smallest index on ties), -1 if none */
+  float lse;       /* log sum_{v in group, allowed} exp(x[v]), -inf if none */
+} fs_group_summary;
+
+/* Flat FMMS sample of B rows with one scalar seed and the library-owned
+ * workspace (fused LM-head matmul + temperature + optional mask + Gumbel
+ * noise + per-tile argmax + cross-tile reduction; abstract of the paper).
+ * One kernel launch for B <= 256; larger B is processed in chunks of 256
+ * rows.  Not safe for concurrent calls on different streams. */
+fs_status fs_sample(const void *H, const void *W, int B, int d, int V,
+                    float temperature, uint64_t seed, uint32_t step,
+                    const uint32_t *mask_bits, int32_t *out_idx,
+                    fs_stream_t stream);
+
+/* fs_sample with optional per-row seeds (row_seeds: device uint64 [B] or
+ * NULL) and an optional caller workspace (see "workspace" above). */
+fs_status fs_sample_ex(const void *H, const void *W, int B, int d, int V,
+                       float temperature, uint64_t seed,
+                       const uint64_t *row_seeds, uint32_t step,
+                       const uint32_t *mask_bits, int32_t *out_idx,
+                       void *workspace, size_t workspace_bytes,
+                       fs_stream_t stream);
+
+/* Grouped sampling (Group-Gumbel-Max; readus.org page, section "Group Gumbel
+ * Max"; abstract: grouped variants are exact by hierarchical factorisation
+ * of the categorical distribution).  The vocabulary is split into G
+ * contiguous groups, group g = [floor(g V / G), floor((g+1) V / G)),
+ * 1 <= G <= V.  Per row and group the fused kernel keeps (max x + g, argmax,
+ * lse = log sum exp(x) over allowed tokens); a merge kernel then picks
+ * g* = argmax_g (lse_g + gumbel_g), where gumbel_g uses the noise word
+ * (g & 3) of Philox(key, (g >> 2, b, step, 1)), and returns the argmax of
+ * group g*.  The result equals flat sampling in distribution (not bitwise).
+ * out_summary: optional device fs_group_summary [B][G] (NULL to skip). */
+fs_status fs_sample_grouped(const void *H, const void *W, int B, int d, int V,
+                            int G, float temperature, uint64_t seed,
+                            const uint64_t *row_seeds, uint32_t step,
+                            const uint32_t *mask_bits, int32_t *out_idx,
+                            fs_group_summary *out_summary, void *workspace,
+                            size_t workspace_bytes, fs_stream_t stream);
+
+/* Unfused two-kernel mode, kept to measure the HBM traffic the fused kernel
+ * saves: the matmul writes fp32 logits l (before temperature) to
+ * logits [B][V] (device, caller-owned, row-major), then a second kernel
+ * applies temperature, mask and noise and reduces to out_idx.  Returns the
+ * same tokens as fs_sample_ex up to fp32 rounding of the logits. */
+fs_status fs_sample_unfused(const void *H, const void *W, int B, int d, int V,
+                            float temperature, uint64_t seed,
+                            const uint64_t *row_seeds, uint32_t step,
+                            const uint32_t *mask_bits, int32_t *out_idx,
+                            float *logits, void *workspace,
+                            size_t workspace_bytes, fs_stream_t stream);
+
+/* End-to-end call with HOST buffers: H_host (bf16 [B, d]) and out_idx_host
+ * (int32 [B]) are host pointers (page-locked for the copies to be
+ * asynchronous); W and row_seeds/mask_bits stay device pointers.  Enqueues
+ * the host-to-device copy of H into a library-owned device buffer, the
+ * fused sample, and the device-to-host copy of the tokens on `stream`; the
+ * tokens are valid once the stream is synchronised. */
+fs_status fs_sample_host(const void *H_host, const void *W, int B, int d,
+                         int V, float temperature, uint64_t seed,
+                         const uint64_t *row_seeds, uint32_t step,
+                         const uint32_t *mask_bits, int32_t *out_idx_host,
+                         fs_stream_t stream);
+
+/* Bytes of caller workspace needed by the calls above for these sizes on the
+ * current device (G = 0 or 1 for flat sampling).  Returns 0 on invalid sizes. */
+size_t fs_workspace_bytes(int B, int V, int G);
+
+/* Reads (synchronously, after the stream drains) and clears the device-side
+ * status word of a workspace (NULL = the library-owned one on the current
+ * device).  Returns FS_OK or FS_ERR_DEVICE_TIMEOUT; after a timeout the
+ * workspace is zero-filled again so it can be reused. */
+fs_status fs_device_status(void *workspace, size_t workspace_bytes,
+                           fs_stream_t stream);
+
+/* Human-readable name of a status code (static storage). */
+const char *fs_status_string(fs_status status);
+
+/* ---- Test entry points: the device noise primitives the kernels use ---- */
+
+/* out[i][0..3] = Philox4x32-10(counter = ctr[i][0..3], key = key[i][0..1]),
+ * n >= 0 counters; all pointers device uint32 arrays. */
+fs_status fs_philox4x32_10(const uint32_t *ctr, const uint32_t *key,
+                           uint32_t *out, int64_t n, fs_stream_t stream);
+
+/* g[i] = fp32 Gumbel transform of the noise word r[i] (the same device
+ * function the sampling kernels use); device arrays of n elements. */
+fs_status fs_gumbel(const uint32_t *r, float *g, int64_t n,
+                    fs_stream_t stream);
+
+/* ---- Host-only schedule query (no GPU needed) ---- */
+
+/* The vocabulary schedule of the fused kernel for V tokens, G groups
+ * (0 or 1: flat) and `num_ctas` persistent CTAs (0: the value the library
+ * would launch on `num_sms` SMs, returned in *num_ctas_out).  Writes up to
+ * max_tiles rows of int32 [5] = (tile start, first valid token, end of valid
+ * tokens, partial slot, last-tile-of-segment flag) for CTA `cta` and returns
+ * the count in *ntiles.  Tiles are 128 tokens; a CTA's range is a multiple
+ * of 8 tokens (except at V); a tile never crosses a group boundary. */
+fs_status fs_plan_tiles(int V, int G, int num_sms, int cta, int32_t *tiles,
+                        int max_tiles, int *ntiles, int *num_ctas_out);
+
+/* The CTAs whose vocabulary range meets group g (0 <= g < G), as the grouped
+ * merge kernel enumerates them: [*first, *last].  Host-only. */
+fs_status fs_plan_group_ctas(int V, int G, int num_sms, int g, int *first,
+                             int *last);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FMMS_H_ */

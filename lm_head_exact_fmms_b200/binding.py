@@ -1,0 +1,274 @@
+"""Thin ctypes binding of libfmms.so (include/fmms.h).
+
+Argument marshalling only: tensors are checked for dtype, device, shape and
+contiguity and passed as raw pointers; every step of the sampling path runs in
+the library's CUDA kernels.  torch supplies device memory and the current
+stream.  There is no fallback: if the library is missing, every call raises.
+"""
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libfmms.so")
+
+FS_OK = 0
+_STATUS = {0: "FS_OK", 1: "FS_ERR_INVALID_ARG", 2: "FS_ERR_UNSUPPORTED", 3: "FS_ERR_CUDA",
+           4: "FS_ERR_WORKSPACE", 5: "FS_ERR_DEVICE_TIMEOUT"}
+
+# Every symbol include/fmms.h declares.
+EXPORTED = ("fs_sample", "fs_sample_ex", "fs_sample_grouped", "fs_sample_unfused",
+            "fs_sample_host", "fs_workspace_bytes", "fs_device_status", "fs_status_string",
+            "fs_philox4x32_10", "fs_gumbel", "fs_plan_tiles", "fs_plan_group_ctas")
+
+
+class FmmsError(RuntimeError):
+    def __init__(self, status, what):
+        super().__init__("%s failed: %s" % (what, _STATUS.get(status, str(status))))
+        self.status = status
+
+
+class GroupSummary(ctypes.Structure):
+    _fields_ = [("max_score", ctypes.c_float), ("argmax", ctypes.c_int32), ("lse", ctypes.c_float)]
+
+
+_lib = None
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Loads libfmms.so (once).  Raises FmmsError if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise FmmsError(-1, "loading %s (build it with python -m lm_head_exact_fmms_b200.build)"
+                        % _LIB_PATH)
+    lib = ctypes.CDLL(_LIB_PATH)
+    vp, i32, u32, u64, f32, sz = (ctypes.c_void_p, ctypes.c_int, ctypes.c_uint32, ctypes.c_uint64,
+                                  ctypes.c_float, ctypes.c_size_t)
+    common = [vp, vp, i32, i32, i32]
+    lib.fs_sample.argtypes = common + [f32, u64, u32, vp, vp, vp]
+    lib.fs_sample_ex.argtypes = common + [f32, u64, vp, u32, vp, vp, vp, sz, vp]
+    lib.fs_sample_grouped.argtypes = common + [i32, f32, u64, vp, u32, vp, vp, vp, vp, sz, vp]
+    lib.fs_sample_unfused.argtypes = common + [f32, u64, vp, u32, vp, vp, vp, vp, sz, vp]
+    lib.fs_sample_host.argtypes = common + [f32, u64, vp, u32, vp, vp, vp]
+    lib.fs_workspace_bytes.argtypes = [i32, i32, i32]
+    lib.fs_workspace_bytes.restype = sz
+    lib.fs_device_status.argtypes = [vp, sz, vp]
+    lib.fs_status_string.argtypes = [i32]
+    lib.fs_status_string.restype = ctypes.c_char_p
+    lib.fs_philox4x32_10.argtypes = [vp, vp, vp, ctypes.c_int64, vp]
+    lib.fs_gumbel.argtypes = [vp, vp, ctypes.c_int64, vp]
+    lib.fs_plan_tiles.argtypes = [i32, i32, i32, i32, vp, i32, ctypes.POINTER(ctypes.c_int),
+                                  ctypes.POINTER(ctypes.c_int)]
+    lib.fs_plan_group_ctas.argtypes = [i32, i32, i32, i32, ctypes.POINTER(ctypes.c_int),
+                                       ctypes.POINTER(ctypes.c_int)]
+    for name in EXPORTED:
+        if name not in ("fs_workspace_bytes", "fs_status_string"):
+            getattr(lib, name).restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+# ------------------------------------------------------------------ helpers
+def _check(status, what):
+    if status != FS_OK:
+        raise FmmsError(status, what)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check_operands(H, W):
+    if H.dtype != torch.bfloat16 or W.dtype != torch.bfloat16:
+        raise TypeError("H and W must be bfloat16")
+    if H.dim() != 2 or W.dim() != 2 or H.shape[1] != W.shape[1]:
+        raise ValueError("H must be [B, d] and W [V, d]")
+    if not (H.is_cuda and W.is_cuda) or H.device != W.device:
+        raise ValueError("H and W must be CUDA tensors on the same device")
+    if not (H.is_contiguous() and W.is_contiguous()):
+        raise ValueError("H and W must be contiguous")
+    return H.shape[0], H.shape[1], W.shape[0]
+
+
+def _opt_dev(t, dtype, n, name, device):
+    if t is None:
+        return None
+    if t.dtype != dtype or not t.is_cuda or t.device != device or not t.is_contiguous():
+        raise ValueError("%s must be a contiguous %s CUDA tensor on %s" % (name, dtype, device))
+    if t.numel() < n:
+        raise ValueError("%s has %d elements, needs %d" % (name, t.numel(), n))
+    return t
+
+
+def _out(out, B, device):
+    if out is None:
+        return torch.empty(B, dtype=torch.int32, device=device)
+    _opt_dev(out, torch.int32, B, "out_idx", device)
+    return out
+
+
+def _seed(seed):
+    return ctypes.c_uint64(int(seed) & 0xFFFFFFFFFFFFFFFF)
+
+
+# ------------------------------------------------------------- entry points
+def fs_sample(H, W, temperature=1.0, seed=0, step=0, mask_bits=None, out_idx=None, stream=None):
+    """Flat FMMS sample (scalar seed, library workspace).  Returns out_idx [B] int32."""
+    lib = load_library()
+    B, d, V = _check_operands(H, W)
+    mask_bits = _opt_dev(mask_bits, torch.int32, B * ((V + 31) // 32), "mask_bits", H.device)
+    out_idx = _out(out_idx, B, H.device)
+    _check(lib.fs_sample(_ptr(H), _ptr(W), B, d, V, float(temperature), _seed(seed), int(step),
+                         _ptr(mask_bits), _ptr(out_idx), _stream(stream)), "fs_sample")
+    return out_idx
+
+
+def fs_sample_ex(H, W, temperature=1.0, seed=0, row_seeds=None, step=0, mask_bits=None,
+                 out_idx=None, workspace=None, stream=None):
+    """Flat FMMS sample with optional per-row seeds ([B] int64) and caller workspace (uint8)."""
+    lib = load_library()
+    B, d, V = _check_operands(H, W)
+    row_seeds = _opt_dev(row_seeds, torch.int64, B, "row_seeds", H.device)
+    mask_bits = _opt_dev(mask_bits, torch.int32, B * ((V + 31) // 32), "mask_bits", H.device)
+    out_idx = _out(out_idx, B, H.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.fs_sample_ex(_ptr(H), _ptr(W), B, d, V, float(temperature), _seed(seed),
+                            _ptr(row_seeds), int(step), _ptr(mask_bits), _ptr(out_idx),
+                            _ptr(workspace), ws_bytes, _stream(stream)), "fs_sample_ex")
+    return out_idx
+
+
+def fs_sample_grouped(H, W, G, temperature=1.0, seed=0, row_seeds=None, step=0, mask_bits=None,
+                      out_idx=None, out_summary=None, workspace=None, stream=None):
+    """Group-Gumbel-Max sample.  out_summary, if given, is a float32 CUDA tensor
+    [B, G, 3] receiving (max score, argmax bits as int32, lse)."""
+    lib = load_library()
+    B, d, V = _check_operands(H, W)
+    row_seeds = _opt_dev(row_seeds, torch.int64, B, "row_seeds", H.device)
+    mask_bits = _opt_dev(mask_bits, torch.int32, B * ((V + 31) // 32), "mask_bits", H.device)
+    out_idx = _out(out_idx, B, H.device)
+    if out_summary is not None:
+        _opt_dev(out_summary, torch.float32, B * G * 3, "out_summary", H.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.fs_sample_grouped(_ptr(H), _ptr(W), B, d, V, int(G), float(temperature),
+                                 _seed(seed), _ptr(row_seeds), int(step), _ptr(mask_bits),
+                                 _ptr(out_idx), _ptr(out_summary), _ptr(workspace), ws_bytes,
+                                 _stream(stream)), "fs_sample_grouped")
+    return out_idx
+
+
+def fs_sample_unfused(H, W, temperature=1.0, seed=0, row_seeds=None, step=0, mask_bits=None,
+                      out_idx=None, logits=None, workspace=None, stream=None):
+    """Unfused two-kernel mode (measurement only): fp32 logits [B, V] go through HBM."""
+    lib = load_library()
+    B, d, V = _check_operands(H, W)
+    row_seeds = _opt_dev(row_seeds, torch.int64, B, "row_seeds", H.device)
+    mask_bits = _opt_dev(mask_bits, torch.int32, B * ((V + 31) // 32), "mask_bits", H.device)
+    out_idx = _out(out_idx, B, H.device)
+    if logits is None:
+        logits = torch.empty(B, V, dtype=torch.float32, device=H.device)
+    _opt_dev(logits, torch.float32, B * V, "logits", H.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.fs_sample_unfused(_ptr(H), _ptr(W), B, d, V, float(temperature), _seed(seed),
+                                 _ptr(row_seeds), int(step), _ptr(mask_bits), _ptr(out_idx),
+                                 _ptr(logits), _ptr(workspace), ws_bytes, _stream(stream)),
+           "fs_sample_unfused")
+    return out_idx
+
+
+def fs_sample_host(H_host, W, temperature=1.0, seed=0, row_seeds=None, step=0, mask_bits=None,
+                   out_idx_host=None, stream=None):
+    """End-to-end call with host buffers: H_host (pinned CPU bf16 [B, d]) in,
+    out_idx_host (pinned CPU int32 [B]) out, asynchronous on the stream."""
+    lib = load_library()
+    if H_host.dtype != torch.bfloat16 or H_host.is_cuda or not H_host.is_contiguous():
+        raise ValueError("H_host must be a contiguous CPU bfloat16 tensor")
+    if W.dtype != torch.bfloat16 or not W.is_cuda or not W.is_contiguous():
+        raise ValueError("W must be a contiguous CUDA bfloat16 tensor")
+    B, d = H_host.shape
+    V = W.shape[0]
+    row_seeds = _opt_dev(row_seeds, torch.int64, B, "row_seeds", W.device)
+    mask_bits = _opt_dev(mask_bits, torch.int32, B * ((V + 31) // 32), "mask_bits", W.device)
+    if out_idx_host is None:
+        out_idx_host = torch.empty(B, dtype=torch.int32, pin_memory=True)
+    _check(lib.fs_sample_host(_ptr(H_host), _ptr(W), B, d, V, float(temperature), _seed(seed),
+                              _ptr(row_seeds), int(step), _ptr(mask_bits), _ptr(out_idx_host),
+                              _stream(stream)), "fs_sample_host")
+    return out_idx_host
+
+
+def fs_workspace_bytes(B, V, G=0):
+    return int(load_library().fs_workspace_bytes(int(B), int(V), int(G)))
+
+
+def fs_device_status(workspace=None, stream=None):
+    lib = load_library()
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    return int(lib.fs_device_status(_ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def fs_status_string(status):
+    return load_library().fs_status_string(int(status)).decode()
+
+
+def fs_philox4x32_10(ctr, key, stream=None):
+    """Device Philox4x32-10 of int32-viewed [n, 4] counters with [n, 2] keys."""
+    lib = load_library()
+    n = ctr.shape[0]
+    out = torch.empty_like(ctr)
+    _check(lib.fs_philox4x32_10(_ptr(ctr), _ptr(key), _ptr(out), n, _stream(stream)),
+           "fs_philox4x32_10")
+    return out
+
+
+def fs_gumbel(r, stream=None):
+    """Device fp32 Gumbel transform of int32-viewed u32 words."""
+    lib = load_library()
+    out = torch.empty(r.shape, dtype=torch.float32, device=r.device)
+    _check(lib.fs_gumbel(_ptr(r), _ptr(out), r.numel(), _stream(stream)), "fs_gumbel")
+    return out
+
+
+def fs_plan_tiles(V, G, num_sms, cta, max_tiles=4096):
+    """Host-only schedule query: (tiles int32 [n, 5], num_ctas)."""
+    import numpy as np
+    lib = load_library()
+    buf = np.zeros((max_tiles, 5), dtype=np.int32)
+    n = ctypes.c_int(0)
+    nc = ctypes.c_int(0)
+    _check(lib.fs_plan_tiles(int(V), int(G), int(num_sms), int(cta),
+                             buf.ctypes.data_as(ctypes.c_void_p), max_tiles, ctypes.byref(n),
+                             ctypes.byref(nc)), "fs_plan_tiles")
+    return buf[: min(n.value, max_tiles)].copy(), nc.value
+
+
+def plan_num_ctas(V, G, num_sms):
+    lib = load_library()
+    n = ctypes.c_int(0)
+    nc = ctypes.c_int(0)
+    _check(lib.fs_plan_tiles(int(V), int(G), int(num_sms), 0, None, 0, ctypes.byref(n),
+                             ctypes.byref(nc)), "fs_plan_tiles")
+    return nc.value
+
+
+def fs_plan_group_ctas(V, G, num_sms, g):
+    """Host-only: (first, last) CTA whose range meets group g."""
+    lib = load_library()
+    a = ctypes.c_int(0)
+    z = ctypes.c_int(0)
+    _check(lib.fs_plan_group_ctas(int(V), int(G), int(num_sms), int(g), ctypes.byref(a),
+                                  ctypes.byref(z)), "fs_plan_group_ctas")
+    return a.value, z.value

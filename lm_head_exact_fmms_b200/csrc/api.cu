@@ -1,0 +1,444 @@
+// api.cu -- the C ABI of libfmms (declared in include/fmms.h): argument
+// validation, workspace management, TMA tensor maps and kernel dispatch.
+// Nothing here computes a sampling step; every step runs in the kernels.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "../../include/fmms.h"
+#include "fmms_common.cuh"
+#include "launch.h"
+
+namespace {
+
+using fmms::FmmsParams;
+using fmms::Schedule;
+
+// ------------------------------------------------------------- device state
+struct DeviceState {
+  bool init = false;
+  int sms = 0;
+  int cc_major = 0;
+  void *ws = nullptr;       // library-owned workspace
+  size_t ws_bytes = 0;
+  void *h_stage = nullptr;  // fs_sample_host: device copy of H
+  size_t h_stage_bytes = 0;
+  void *o_stage = nullptr;  // fs_sample_host: device tokens
+  size_t o_stage_bytes = 0;
+};
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+
+fs_status get_device(DeviceState **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FS_ERR_CUDA;
+  DeviceState &st = g_dev[dev];
+  if (!st.init) {
+    if (cudaDeviceGetAttribute(&st.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return FS_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&st.cc_major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+      return FS_ERR_CUDA;
+    st.init = true;
+  }
+  if (st.cc_major != 10) return FS_ERR_UNSUPPORTED;  // built for sm_100a only
+  *out = &st;
+  return FS_OK;
+}
+
+// Grows a library-owned device buffer; new memory is zero-filled.
+fs_status grow(void **buf, size_t *have, size_t need) {
+  if (*have >= need) return FS_OK;
+  if (*buf) {
+    cudaDeviceSynchronize();
+    cudaFree(*buf);
+    *buf = nullptr;
+    *have = 0;
+  }
+  if (cudaMalloc(buf, need) != cudaSuccess) return FS_ERR_CUDA;
+  if (cudaMemset(*buf, 0, need) != cudaSuccess) return FS_ERR_CUDA;
+  *have = need;
+  return FS_OK;
+}
+
+// ----------------------------------------------------------- tensor maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// A bf16 matrix [rows][inner] read in boxes of [box_rows][64] with the
+// 128-byte swizzle; out-of-range elements read as zero.
+struct TmapKey {
+  const void *ptr;
+  uint64_t inner, rows;
+  uint32_t box_rows;
+  int dev;
+};
+
+struct TmapEntry {
+  TmapKey key;
+  CUtensorMap map;
+  bool used = false;
+};
+
+constexpr int kTmapCache = 64;
+TmapEntry g_tmaps[kTmapCache];
+int g_tmap_next = 0;
+
+fs_status tensor_map(CUtensorMap *out, const void *ptr, uint64_t inner, uint64_t rows,
+                     uint32_t box_rows) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  for (auto &e : g_tmaps) {
+    if (e.used && e.key.ptr == ptr && e.key.inner == inner && e.key.rows == rows &&
+        e.key.box_rows == box_rows && e.key.dev == dev) {
+      *out = e.map;
+      return FS_OK;
+    }
+  }
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return FS_ERR_CUDA;
+  CUtensorMap m;
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {inner * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(fmms::kBlockK), box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return FS_ERR_CUDA;
+  TmapEntry &e = g_tmaps[g_tmap_next];
+  g_tmap_next = (g_tmap_next + 1) % kTmapCache;
+  e.key = TmapKey{ptr, inner, rows, box_rows, dev};
+  e.map = m;
+  e.used = true;
+  *out = m;
+  return FS_OK;
+}
+
+// ------------------------------------------------------------ validation
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+fs_status validate(const void *H, const void *W, int B, int d, int V, float T, const void *out) {
+  if (!H || !W || !out) return FS_ERR_INVALID_ARG;
+  if (B < 1 || V < 1 || d < 8 || (d % 8) != 0) return FS_ERR_INVALID_ARG;
+  if (!(T > 0.f) || !isfinite(T)) return FS_ERR_INVALID_ARG;
+  if (!aligned16(H) || !aligned16(W)) return FS_ERR_INVALID_ARG;
+  return FS_OK;
+}
+
+struct Workspace {
+  int *err;
+  unsigned int *ticket;
+  unsigned long long *keys;
+  fmms::GroupPartial *partials;
+};
+
+Workspace carve(void *ws) {
+  char *b = static_cast<char *>(ws);
+  Workspace w;
+  w.err = reinterpret_cast<int *>(b);
+  w.ticket = reinterpret_cast<unsigned int *>(b + 4);
+  w.keys = reinterpret_cast<unsigned long long *>(b + fmms::kWsHeader);
+  w.partials = reinterpret_cast<fmms::GroupPartial *>(b + fmms::kWsHeader + fmms::kWsKeys);
+  return w;
+}
+
+fs_status resolve_workspace(DeviceState *st, const Schedule &sch, int B, void *ws, size_t ws_bytes,
+                            void **out) {
+  const size_t need = static_cast<size_t>(fmms::workspace_bytes_for(B, sch.G, sch.num_ctas));
+  if (ws == nullptr) {
+    fs_status s = grow(&st->ws, &st->ws_bytes, need);
+    if (s != FS_OK) return s;
+    *out = st->ws;
+    return FS_OK;
+  }
+  if (ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return FS_ERR_WORKSPACE;
+  *out = ws;
+  return FS_OK;
+}
+
+// The fused path in all three modes, chunked over 256 batch rows.
+fs_status run(int mode, const void *H, const void *W, int B, int d, int V, int G, float T,
+              uint64_t seed, const uint64_t *row_seeds, uint32_t step, const uint32_t *mask,
+              int32_t *out_idx, fs_group_summary *summary, float *logits, void *ws,
+              size_t ws_bytes, cudaStream_t stream) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState *st = nullptr;
+  fs_status s = get_device(&st);
+  if (s != FS_OK) return s;
+  const Schedule sch = fmms::make_schedule(V, mode == fmms::kModeGrouped ? G : 1, st->sms);
+  void *wsp = nullptr;
+  s = resolve_workspace(st, sch, B, ws, ws_bytes, &wsp);
+  if (s != FS_OK) return s;
+  const Workspace w = carve(wsp);
+
+  CUtensorMap tw, tw8;
+  if ((s = tensor_map(&tw, W, d, V, fmms::kTileM)) != FS_OK) return s;
+  if ((s = tensor_map(&tw8, W, d, V, fmms::kGranule)) != FS_OK) return s;
+
+  for (int b0 = 0; b0 < B; b0 += fmms::kMaxBN) {
+    const int Bc = fmms::imin(fmms::kMaxBN, B - b0);
+    const int BN = fmms::fmms_batch_tile(Bc);
+    CUtensorMap th;
+    if ((s = tensor_map(&th, H, d, B, BN)) != FS_OK) return s;
+    FmmsParams p;
+    memset(&p, 0, sizeof p);
+    p.B = Bc;
+    p.b_off = b0;
+    p.d = d;
+    p.V = V;
+    p.G = sch.G;
+    p.num_ctas = sch.num_ctas;
+    p.ngran = sch.ngran;
+    p.nk = (d + fmms::kBlockK - 1) / fmms::kBlockK;
+    p.inv_temp = 1.0f / T;
+    p.step = step;
+    p.seed = seed;
+    p.row_seeds = row_seeds;
+    p.mask = mask;
+    p.mask_words = (V + 31) / 32;
+    p.out_idx = out_idx + b0;
+    p.keys = w.keys;
+    p.ticket = w.ticket;
+    p.err = w.err;
+    p.partials = w.partials;
+    p.logits = logits ? logits + static_cast<size_t>(b0) * V : nullptr;
+    if (fmms::launch_fmms(mode, BN, tw, tw8, th, p, stream) != cudaSuccess) return FS_ERR_CUDA;
+
+    if (mode == fmms::kModeGrouped) {
+      fmms::MergeParams m;
+      m.partials = w.partials;
+      m.B = Bc;
+      m.b_off = b0;
+      m.V = V;
+      m.G = sch.G;
+      m.num_ctas = sch.num_ctas;
+      m.ngran = sch.ngran;
+      m.seed = seed;
+      m.row_seeds = row_seeds;
+      m.step = step;
+      m.out_idx = out_idx + b0;
+      m.summary = summary ? static_cast<void *>(summary + static_cast<size_t>(b0) * sch.G) : nullptr;
+      if (fmms::launch_group_merge(m, stream) != cudaSuccess) return FS_ERR_CUDA;
+    } else if (mode == fmms::kModeLogits) {
+      fmms::SampleLogitsParams sp;
+      sp.logits = p.logits;
+      sp.B = Bc;
+      sp.b_off = b0;
+      sp.V = V;
+      sp.inv_temp = p.inv_temp;
+      sp.seed = seed;
+      sp.row_seeds = row_seeds;
+      sp.step = step;
+      sp.mask = mask;
+      sp.mask_words = p.mask_words;
+      sp.keys = w.keys;
+      sp.ticket = w.ticket;
+      sp.out_idx = out_idx + b0;
+      sp.num_sms = st->sms;
+      if (fmms::launch_sample_logits(sp, stream) != cudaSuccess) return FS_ERR_CUDA;
+    }
+  }
+  return FS_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+fs_status fs_sample(const void *H, const void *W, int B, int d, int V, float temperature,
+                    uint64_t seed, uint32_t step, const uint32_t *mask_bits, int32_t *out_idx,
+                    fs_stream_t stream) {
+  fs_status s = validate(H, W, B, d, V, temperature, out_idx);
+  if (s != FS_OK) return s;
+  return run(fmms::kModeFlat, H, W, B, d, V, 1, temperature, seed, nullptr, step, mask_bits,
+             out_idx, nullptr, nullptr, nullptr, 0, static_cast<cudaStream_t>(stream));
+}
+
+fs_status fs_sample_ex(const void *H, const void *W, int B, int d, int V, float temperature,
+                       uint64_t seed, const uint64_t *row_seeds, uint32_t step,
+                       const uint32_t *mask_bits, int32_t *out_idx, void *workspace,
+                       size_t workspace_bytes, fs_stream_t stream) {
+  fs_status s = validate(H, W, B, d, V, temperature, out_idx);
+  if (s != FS_OK) return s;
+  return run(fmms::kModeFlat, H, W, B, d, V, 1, temperature, seed, row_seeds, step, mask_bits,
+             out_idx, nullptr, nullptr, workspace, workspace_bytes,
+             static_cast<cudaStream_t>(stream));
+}
+
+fs_status fs_sample_grouped(const void *H, const void *W, int B, int d, int V, int G,
+                            float temperature, uint64_t seed, const uint64_t *row_seeds,
+                            uint32_t step, const uint32_t *mask_bits, int32_t *out_idx,
+                            fs_group_summary *out_summary, void *workspace, size_t workspace_bytes,
+                            fs_stream_t stream) {
+  fs_status s = validate(H, W, B, d, V, temperature, out_idx);
+  if (s != FS_OK) return s;
+  if (G < 1 || G > V) return FS_ERR_INVALID_ARG;
+  return run(fmms::kModeGrouped, H, W, B, d, V, G, temperature, seed, row_seeds, step, mask_bits,
+             out_idx, out_summary, nullptr, workspace, workspace_bytes,
+             static_cast<cudaStream_t>(stream));
+}
+
+fs_status fs_sample_unfused(const void *H, const void *W, int B, int d, int V, float temperature,
+                            uint64_t seed, const uint64_t *row_seeds, uint32_t step,
+                            const uint32_t *mask_bits, int32_t *out_idx, float *logits,
+                            void *workspace, size_t workspace_bytes, fs_stream_t stream) {
+  fs_status s = validate(H, W, B, d, V, temperature, out_idx);
+  if (s != FS_OK) return s;
+  if (!logits) return FS_ERR_INVALID_ARG;
+  return run(fmms::kModeLogits, H, W, B, d, V, 1, temperature, seed, row_seeds, step, mask_bits,
+             out_idx, nullptr, logits, workspace, workspace_bytes,
+             static_cast<cudaStream_t>(stream));
+}
+
+fs_status fs_sample_host(const void *H_host, const void *W, int B, int d, int V,
+                         float temperature, uint64_t seed, const uint64_t *row_seeds,
+                         uint32_t step, const uint32_t *mask_bits, int32_t *out_idx_host,
+                         fs_stream_t stream) {
+  if (!H_host || !out_idx_host) return FS_ERR_INVALID_ARG;
+  if (B < 1 || V < 1 || d < 8 || (d % 8) != 0) return FS_ERR_INVALID_ARG;
+  if (!(temperature > 0.f) || !isfinite(temperature) || !W || !aligned16(W))
+    return FS_ERR_INVALID_ARG;
+  cudaStream_t st_ = static_cast<cudaStream_t>(stream);
+  void *hdev = nullptr, *odev = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceState *st = nullptr;
+    fs_status s = get_device(&st);
+    if (s != FS_OK) return s;
+    const size_t hbytes = static_cast<size_t>(B) * d * 2;
+    if ((s = grow(&st->h_stage, &st->h_stage_bytes, hbytes)) != FS_OK) return s;
+    if ((s = grow(&st->o_stage, &st->o_stage_bytes, static_cast<size_t>(B) * 4)) != FS_OK) return s;
+    hdev = st->h_stage;
+    odev = st->o_stage;
+    if (cudaMemcpyAsync(hdev, H_host, hbytes, cudaMemcpyHostToDevice, st_) != cudaSuccess)
+      return FS_ERR_CUDA;
+  }
+  fs_status s = run(fmms::kModeFlat, hdev, W, B, d, V, 1, temperature, seed, row_seeds, step,
+                    mask_bits, static_cast<int32_t *>(odev), nullptr, nullptr, nullptr, 0, st_);
+  if (s != FS_OK) return s;
+  if (cudaMemcpyAsync(out_idx_host, odev, static_cast<size_t>(B) * 4, cudaMemcpyDeviceToHost,
+                      st_) != cudaSuccess)
+    return FS_ERR_CUDA;
+  return FS_OK;
+}
+
+size_t fs_workspace_bytes(int B, int V, int G) {
+  if (B < 1 || V < 1 || G < 0 || G > V) return 0;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 0;
+  const Schedule sch = fmms::make_schedule(V, G, sms);
+  return static_cast<size_t>(fmms::workspace_bytes_for(B, sch.G, sch.num_ctas));
+}
+
+fs_status fs_device_status(void *workspace, size_t workspace_bytes, fs_stream_t stream) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  void *ws = workspace;
+  size_t bytes = workspace_bytes;
+  if (!ws) {
+    DeviceState *st = nullptr;
+    fs_status s = get_device(&st);
+    if (s != FS_OK) return s;
+    ws = st->ws;
+    bytes = st->ws_bytes;
+    if (!ws) return FS_OK;
+  }
+  if (bytes < static_cast<size_t>(fmms::kWsHeader)) return FS_ERR_WORKSPACE;
+  cudaStream_t st_ = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st_) != cudaSuccess) return FS_ERR_CUDA;
+  int err = 0;
+  if (cudaMemcpy(&err, ws, sizeof err, cudaMemcpyDeviceToHost) != cudaSuccess) return FS_ERR_CUDA;
+  if (err == 0) return FS_OK;
+  if (cudaMemset(ws, 0, bytes) != cudaSuccess) return FS_ERR_CUDA;
+  return FS_ERR_DEVICE_TIMEOUT;
+}
+
+const char *fs_status_string(fs_status status) {
+  switch (status) {
+    case FS_OK: return "FS_OK";
+    case FS_ERR_INVALID_ARG: return "FS_ERR_INVALID_ARG";
+    case FS_ERR_UNSUPPORTED: return "FS_ERR_UNSUPPORTED";
+    case FS_ERR_CUDA: return "FS_ERR_CUDA";
+    case FS_ERR_WORKSPACE: return "FS_ERR_WORKSPACE";
+    case FS_ERR_DEVICE_TIMEOUT: return "FS_ERR_DEVICE_TIMEOUT";
+  }
+  return "FS_ERR_UNKNOWN";
+}
+
+fs_status fs_philox4x32_10(const uint32_t *ctr, const uint32_t *key, uint32_t *out, int64_t n,
+                           fs_stream_t stream) {
+  if (n < 0 || (n > 0 && (!ctr || !key || !out))) return FS_ERR_INVALID_ARG;
+  DeviceState *st = nullptr;
+  fs_status s = get_device(&st);
+  if (s != FS_OK) return s;
+  return fmms::launch_philox_test(ctr, key, out, n, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? FS_OK
+             : FS_ERR_CUDA;
+}
+
+fs_status fs_gumbel(const uint32_t *r, float *g, int64_t n, fs_stream_t stream) {
+  if (n < 0 || (n > 0 && (!r || !g))) return FS_ERR_INVALID_ARG;
+  DeviceState *st = nullptr;
+  fs_status s = get_device(&st);
+  if (s != FS_OK) return s;
+  return fmms::launch_gumbel_test(r, g, n, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? FS_OK
+             : FS_ERR_CUDA;
+}
+
+fs_status fs_plan_tiles(int V, int G, int num_sms, int cta, int32_t *tiles, int max_tiles,
+                        int *ntiles, int *num_ctas_out) {
+  if (V < 1 || G < 0 || G > V || num_sms < 1 || !ntiles) return FS_ERR_INVALID_ARG;
+  const Schedule sch = fmms::make_schedule(V, G, num_sms);
+  if (num_ctas_out) *num_ctas_out = sch.num_ctas;
+  if (cta < 0 || cta >= sch.num_ctas) return FS_ERR_INVALID_ARG;
+  fmms::TileIter it(sch, cta);
+  fmms::Tile t;
+  int n = 0;
+  while (it.next(t)) {
+    if (tiles && n < max_tiles) {
+      tiles[5 * n + 0] = t.start;
+      tiles[5 * n + 1] = t.lo;
+      tiles[5 * n + 2] = t.hi;
+      tiles[5 * n + 3] = t.slot;
+      tiles[5 * n + 4] = t.last;
+    }
+    ++n;
+  }
+  *ntiles = n;
+  return FS_OK;
+}
+
+fs_status fs_plan_group_ctas(int V, int G, int num_sms, int g, int *first, int *last) {
+  if (V < 1 || G < 1 || G > V || num_sms < 1 || g < 0 || g >= G || !first || !last)
+    return FS_ERR_INVALID_ARG;
+  const Schedule sch = fmms::make_schedule(V, G, num_sms);
+  *first = fmms::cta_of(fmms::group_begin(g, V, G), sch);
+  *last = fmms::cta_of(fmms::group_begin(g + 1, V, G) - 1, sch);
+  return FS_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,218 @@
+// aux_kernels.cu -- the small kernels around the fused one:
+//  * the Group-Gumbel-Max merge of per-(segment, row) partials (readus.org
+//    page, "Group Gumbel Max": pick a group with Gumbel noise on the group
+//    log-masses, then take the sample inside the winning group);
+//  * the second kernel of the unfused mode, sampling from fp32 logits in HBM;
+//  * test kernels exposing the device Philox and Gumbel primitives.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "../../include/fmms.h"
+#include "fmms_common.cuh"
+#include "launch.h"
+#include "noise.cuh"
+
+namespace fmms {
+
+// ---------------------------------------------------------------------------
+// Group merge: one warp per row; lanes stride over the groups.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(128) group_merge_kernel(const MergeParams m) {
+  const int b = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+  const int lane = threadIdx.x & 31;
+  if (b >= m.B) return;
+  Schedule sch;
+  sch.V = m.V;
+  sch.G = m.G;
+  sch.num_ctas = m.num_ctas;
+  sch.ngran = m.ngran;
+  const uint32_t bg = static_cast<uint32_t>(m.b_off + b);
+  const uint64_t k64 = m.row_seeds ? m.row_seeds[bg] : m.seed;
+  fs_group_summary *summary = static_cast<fs_group_summary *>(m.summary);
+
+  float best_key = -INFINITY;
+  int best_g = -1;
+  unsigned long long best_tok = 0ull;
+  for (int g = lane; g < m.G; g += 32) {
+    const int lo = group_begin(g, m.V, m.G);
+    const int hi = group_begin(g + 1, m.V, m.G);
+    const int c_first = cta_of(lo, sch);
+    const int c_last = cta_of(hi - 1, sch);
+    unsigned long long kmax = 0ull;
+    float M = -INFINITY, S = 0.f;
+    for (int c = c_first; c <= c_last; ++c) {
+      const GroupPartial gp = m.partials[static_cast<size_t>(c + g) * m.B + b];
+      kmax = gp.key > kmax ? gp.key : kmax;
+      if (gp.m != -INFINITY) {
+        if (M == -INFINITY) {
+          M = gp.m;
+          S = gp.sum;
+        } else {
+          const float mx = fmaxf(M, gp.m);
+          S = S * expf(M - mx) + gp.sum * expf(gp.m - mx);
+          M = mx;
+        }
+      }
+    }
+    const float lse = (M == -INFINITY) ? -INFINITY : M + logf(S);
+    if (summary != nullptr) {
+      fs_group_summary gs;
+      gs.max_score = kmax ? __uint_as_float(key_score_bits(kmax)) : -INFINITY;
+      gs.argmax = key_token(kmax);
+      gs.lse = lse;
+      summary[static_cast<size_t>(b) * m.G + g] = gs;
+    }
+    if (lse != -INFINITY) {
+      const Philox4 ph = philox4x32_10(static_cast<uint32_t>(g) >> 2, bg, m.step, 1u,
+                                       static_cast<uint32_t>(k64), static_cast<uint32_t>(k64 >> 32));
+      const uint32_t w = (g & 3) == 0 ? ph.w0 : (g & 3) == 1 ? ph.w1 : (g & 3) == 2 ? ph.w2 : ph.w3;
+      const float kg = lse + gumbel_from_u32(w);
+      if (best_g < 0 || kg > best_key) {  // g rises within a lane: ties keep the smaller g
+        best_key = kg;
+        best_g = g;
+        best_tok = kmax;
+      }
+    }
+  }
+  // Warp argmax over (key, group): larger key first, then the smaller group.
+  uint64_t packed = best_g < 0 ? 0ull : pack_key(__float_as_uint(best_key), best_g);
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+    const uint64_t o = __shfl_xor_sync(0xffffffffu, packed, off);
+    packed = o > packed ? o : packed;
+  }
+  const int gwin = key_token(packed);
+  const unsigned long long tok =
+      __shfl_sync(0xffffffffu, best_tok, gwin < 0 ? 0 : (gwin & 31));
+  if (lane == 0) m.out_idx[b] = gwin < 0 ? -1 : key_token(tok);
+}
+
+cudaError_t launch_group_merge(const MergeParams &m, cudaStream_t stream) {
+  const int threads = 128;
+  const int blocks = (m.B * 32 + threads - 1) / threads;
+  group_merge_kernel<<<blocks, threads, 0, stream>>>(m);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Unfused mode, kernel 2: temperature, mask, noise and argmax over fp32
+// logits [B][V].  Each thread takes four consecutive tokens (one Philox
+// call); blocks publish a packed max per row with atomicMax and the last
+// block decodes.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) sample_logits_kernel(const SampleLogitsParams s) {
+  const int b = blockIdx.y;
+  const uint32_t bg = static_cast<uint32_t>(s.b_off + b);
+  const uint64_t k64 = s.row_seeds ? s.row_seeds[bg] : s.seed;
+  const float *row = s.logits + static_cast<size_t>(b) * s.V;
+  const int nquads = (s.V + 3) / 4;
+  const bool vec = (s.V & 3) == 0;
+  uint64_t best = 0ull;
+  for (int qd = blockIdx.x * blockDim.x + threadIdx.x; qd < nquads; qd += gridDim.x * blockDim.x) {
+    const Philox4 ph = philox4x32_10(static_cast<uint32_t>(qd), bg, s.step, 0u,
+                                     static_cast<uint32_t>(k64), static_cast<uint32_t>(k64 >> 32));
+    const uint32_t w[4] = {ph.w0, ph.w1, ph.w2, ph.w3};
+    float l[4];
+    const int v0 = 4 * qd;
+    if (vec) {
+      const float4 l4 = *reinterpret_cast<const float4 *>(row + v0);
+      l[0] = l4.x;
+      l[1] = l4.y;
+      l[2] = l4.z;
+      l[3] = l4.w;
+    } else {
+#pragma unroll
+      for (int m = 0; m < 4; ++m) l[m] = (v0 + m < s.V) ? row[v0 + m] : 0.f;
+    }
+    uint32_t mword = 0xFFFFFFFFu;
+    if (s.mask) mword = s.mask[static_cast<size_t>(bg) * s.mask_words + (v0 >> 5)];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int v = v0 + m;
+      const bool ok = v < s.V && ((mword >> (v & 31)) & 1u);
+      const float sc = l[m] * s.inv_temp + gumbel_from_u32(w[m]);
+      const uint64_t k = ok ? pack_key(__float_as_uint(sc), v) : 0ull;
+      best = k > best ? k : best;
+    }
+  }
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+    const uint64_t o = __shfl_xor_sync(0xffffffffu, best, off);
+    best = o > best ? o : best;
+  }
+  __shared__ uint64_t warp_best[8];
+  __shared__ int is_last;
+  if ((threadIdx.x & 31) == 0) warp_best[threadIdx.x >> 5] = best;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint64_t r = 0ull;
+    for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) r = warp_best[i] > r ? warp_best[i] : r;
+    if (r) atomicMax(s.keys + b, static_cast<unsigned long long>(r));
+    __threadfence();
+    const unsigned total = gridDim.x * gridDim.y;
+    is_last = (atomicAdd(s.ticket, 1u) == total - 1) ? 1 : 0;
+  }
+  __syncthreads();
+  if (is_last) {
+    __threadfence();
+    for (int r = threadIdx.x; r < s.B; r += blockDim.x)
+      s.out_idx[r] = key_token(atomicExch(s.keys + r, 0ull));
+    if (threadIdx.x == 0) atomicExch(s.ticket, 0u);
+  }
+}
+
+cudaError_t launch_sample_logits(const SampleLogitsParams &s, cudaStream_t stream) {
+  const int threads = 256;
+  const int nquads = (s.V + 3) / 4;
+  int per_row = (nquads + threads - 1) / threads;
+  const int target = (4 * s.num_sms + s.B - 1) / s.B;  // about four blocks per SM in total
+  if (per_row > target) per_row = target;
+  if (per_row < 1) per_row = 1;
+  dim3 grid(per_row, s.B);
+  sample_logits_kernel<<<grid, threads, 0, stream>>>(s);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Test kernels
+// ---------------------------------------------------------------------------
+__global__ void philox_test_kernel(const uint32_t *ctr, const uint32_t *key, uint32_t *out,
+                                   int64_t n) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const Philox4 ph = philox4x32_10(ctr[4 * i], ctr[4 * i + 1], ctr[4 * i + 2], ctr[4 * i + 3],
+                                     key[2 * i], key[2 * i + 1]);
+    out[4 * i] = ph.w0;
+    out[4 * i + 1] = ph.w1;
+    out[4 * i + 2] = ph.w2;
+    out[4 * i + 3] = ph.w3;
+  }
+}
+
+__global__ void gumbel_test_kernel(const uint32_t *r, float *g, int64_t n) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    g[i] = gumbel_from_u32(r[i]);
+}
+
+static int test_grid(int64_t n) {
+  int64_t blocks = (n + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  return blocks < 1 ? 1 : static_cast<int>(blocks);
+}
+
+cudaError_t launch_philox_test(const uint32_t *ctr, const uint32_t *key, uint32_t *out, int64_t n,
+                               cudaStream_t stream) {
+  if (n <= 0) return cudaSuccess;
+  philox_test_kernel<<<test_grid(n), 256, 0, stream>>>(ctr, key, out, n);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gumbel_test(const uint32_t *r, float *g, int64_t n, cudaStream_t stream) {
+  if (n <= 0) return cudaSuccess;
+  gumbel_test_kernel<<<test_grid(n), 256, 0, stream>>>(r, g, n);
+  return cudaGetLastError();
+}
+
+}  // namespace fmms

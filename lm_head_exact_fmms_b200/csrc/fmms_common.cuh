@@ -1,0 +1,186 @@
+// fmms_common.cuh -- host/device definitions shared by the FMMS kernels and
+// the C ABI: tile geometry, the split-V schedule, kernel parameters and the
+// packed (score, token) key used by every reduction.
+#pragma once
+
+#include <stdint.h>
+
+#if defined(__CUDACC__)
+#define FS_HD __host__ __device__ __forceinline__
+#else
+#define FS_HD inline
+#endif
+
+namespace fmms {
+
+// Tile geometry (swap-AB orientation: vocabulary rows on the MMA M axis and
+// TMEM lanes, batch rows on the MMA N axis and TMEM columns).
+constexpr int kTileM = 128;   // vocabulary rows per tile (tcgen05 M)
+constexpr int kBlockK = 64;   // K elements per pipeline stage: one 128-byte swizzle row
+constexpr int kGranule = 8;   // vocabulary granule of the per-CTA split: one 8-row swizzle atom
+constexpr int kMaxBN = 256;   // batch rows per launch (tcgen05 N limit)
+constexpr int kNumEpiWarps = 8;
+constexpr int kThreads = 32 * (2 + kNumEpiWarps);  // TMA warp + MMA warp + epilogue
+constexpr int kEpiThreads = 32 * kNumEpiWarps;
+
+FS_HD int imin(int a, int b) { return a < b ? a : b; }
+FS_HD int imax(int a, int b) { return a > b ? a : b; }
+
+// ---------------------------------------------------------------------------
+// Split-V schedule.  The vocabulary is cut into ceil(V/8) granules; CTA c of
+// num_ctas owns granules [floor(c n / C), floor((c+1) n / C)), so every CTA
+// streams the same number of W rows to within one granule.  Group g of G
+// covers [floor(g V / G), floor((g+1) V / G)).  A CTA's range is cut at group
+// boundaries into segments; each segment is walked in 128-row tiles whose
+// start is rounded down to a multiple of 8 (rows before the segment are
+// loaded but ignored).  Segment (c, g) owns partial slot c + g, which is
+// unique because c and g never both stay put from one segment to the next.
+// ---------------------------------------------------------------------------
+struct Schedule {
+  int V;
+  int G;         // number of groups (1 = flat)
+  int num_ctas;
+  int ngran;     // ceil(V / 8)
+};
+
+FS_HD Schedule make_schedule(int V, int G, int num_sms) {
+  Schedule s;
+  s.V = V;
+  s.G = G < 1 ? 1 : G;
+  s.ngran = (V + kGranule - 1) / kGranule;
+  s.num_ctas = imin(num_sms, s.ngran);
+  return s;
+}
+
+FS_HD int group_begin(int g, int V, int G) { return (int)(((int64_t)g * V) / G); }
+
+// The group containing token v: the largest g with floor(g V / G) <= v.
+FS_HD int group_of(int v, int V, int G) {
+  return (int)((((int64_t)v + 1) * G - 1) / V);
+}
+
+FS_HD int cta_begin(int c, const Schedule &s) {
+  int64_t gran = ((int64_t)c * s.ngran) / s.num_ctas;
+  int64_t v = gran * kGranule;
+  return v < s.V ? (int)v : s.V;
+}
+
+// The CTA whose range contains token v.
+FS_HD int cta_of(int v, const Schedule &s) {
+  int64_t q = v / kGranule;
+  return (int)(((q + 1) * s.num_ctas - 1) / s.ngran);
+}
+
+struct Tile {
+  int start;  // first vocabulary row of the tile (multiple of 8)
+  int lo;     // first valid row
+  int hi;     // one past the last valid row (hi - start <= 128)
+  int slot;   // partial slot of the segment
+  int last;   // 1 on the last tile of a segment
+};
+
+// Walks the tiles of one CTA.  All three kernel roles and the host-side
+// schedule query run this same code.
+struct TileIter {
+  int V, G, cta, cta_hi;
+  int v;       // first token of the current segment
+  int seg_hi;  // end of the current segment
+  int t;       // start of the next tile
+  int slot;
+
+  FS_HD TileIter(const Schedule &s, int c) {
+    V = s.V;
+    G = s.G;
+    cta = c;
+    v = cta_begin(c, s);
+    cta_hi = cta_begin(c + 1, s);
+    seg_hi = v;
+    t = v;
+    slot = c;
+  }
+
+  FS_HD bool next(Tile &tile) {
+    if (t >= seg_hi) {
+      v = seg_hi;
+      if (v >= cta_hi) return false;
+      int g = G > 1 ? group_of(v, V, G) : 0;
+      int gend = G > 1 ? group_begin(g + 1, V, G) : V;
+      seg_hi = imin(cta_hi, gend);
+      slot = cta + g;
+      t = v & ~(kGranule - 1);
+    }
+    tile.start = t;
+    tile.lo = imax(t, v);
+    tile.hi = imin(t + kTileM, seg_hi);
+    tile.slot = slot;
+    t += kTileM;
+    tile.last = (t >= seg_hi) ? 1 : 0;
+    return true;
+  }
+};
+
+// ---------------------------------------------------------------------------
+// Packed (score, token) key.  Unsigned 64-bit order on
+//   (order_bits(s) << 32) | (0xFFFFFFFF - v)
+// is "larger score first, then smaller token", the tie rule of every argmax
+// here.  0 means "no candidate" (a masked or out-of-range entry).
+// ---------------------------------------------------------------------------
+FS_HD uint32_t order_bits(uint32_t f) {
+  return (f & 0x80000000u) ? ~f : (f | 0x80000000u);
+}
+FS_HD uint32_t order_bits_inv(uint32_t o) {
+  return (o & 0x80000000u) ? (o & 0x7FFFFFFFu) : ~o;
+}
+FS_HD uint64_t pack_key(uint32_t score_bits, int v) {
+  return ((uint64_t)order_bits(score_bits) << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)v);
+}
+FS_HD int key_token(uint64_t k) { return k == 0 ? -1 : (int)(0xFFFFFFFFu - (uint32_t)k); }
+FS_HD uint32_t key_score_bits(uint64_t k) { return order_bits_inv((uint32_t)(k >> 32)); }
+
+// Per-(slot, row) partial of the grouped kernel.
+struct __align__(16) GroupPartial {
+  unsigned long long key;  // packed best (score, token)
+  float m;                 // max of allowed x in the segment (-inf if none)
+  float sum;               // sum of exp(x - m) over allowed x
+};
+
+enum Mode { kModeFlat = 0, kModeGrouped = 1, kModeLogits = 2 };
+
+struct FmmsParams {
+  int B;            // rows in this launch (<= BN)
+  int b_off;        // global index of this launch's row 0 (noise, mask, seeds)
+  int d;
+  int V;
+  int G;
+  int num_ctas;
+  int ngran;
+  int nk;           // ceil(d / 64) pipeline stages per tile
+  float inv_temp;
+  uint32_t step;
+  uint64_t seed;
+  const uint64_t *row_seeds;   // [global rows] or null
+  const uint32_t *mask;        // [global rows][mask_words] or null
+  int mask_words;
+  int32_t *out_idx;            // [B] (already offset to this launch)
+  unsigned long long *keys;    // workspace [B]: running packed maxima (flat)
+  unsigned int *ticket;        // workspace: CTAs finished (flat)
+  int *err;                    // workspace: device status word
+  GroupPartial *partials;      // workspace [slots][B] (grouped)
+  float *logits;               // [B][V] (logits mode; already offset)
+};
+
+// Workspace layout (bytes): [0, 256) status word and ticket; [256, 256 + 2048)
+// packed keys of up to 256 rows; then grouped partials [slots][256].
+constexpr int kWsHeader = 256;
+constexpr int kWsKeys = 8 * kMaxBN;
+
+FS_HD int64_t workspace_bytes_for(int B, int G, int num_ctas) {
+  int64_t bytes = kWsHeader + kWsKeys;
+  if (G > 1) {
+    int64_t rows = B < kMaxBN ? B : kMaxBN;
+    bytes += (int64_t)(num_ctas + G - 1) * rows * (int64_t)sizeof(GroupPartial);
+  }
+  return (bytes + 255) / 256 * 256;
+}
+
+}  // namespace fmms

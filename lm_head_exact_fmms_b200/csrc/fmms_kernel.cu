@@ -1,0 +1,592 @@
+// fmms_kernel.cu -- the fused matmul-sample (FMMS) kernel for sm_100a.
+//
+// What it computes (FlashSampling, arXiv:2603.15854, abstract): logits of a
+// vocabulary tile are formed on chip, scaled by 1/T, masked, perturbed with
+// Gumbel noise, and only one (score, token) maximiser per row and tile
+// survives; a reduction over tiles gives one token per row.  The B x V
+// logits never reach HBM (except in the logits mode kept for measurement).
+//
+// How (B200 design; the Triton kernel the pages describe is prior art only):
+//  * one persistent CTA per SM; each CTA owns a contiguous, 8-row-granular
+//    slice of the vocabulary (split-V), so small batches still keep all 148
+//    SMs streaming W and no W row is read twice;
+//  * swap-AB MMA: A = 128 vocabulary rows of W (M = 128), B = the batch of
+//    hidden states (N = 16..256), D = a 128-lane x N-column fp32 accumulator
+//    in tensor memory; the tile's vocabulary rows land on TMEM lanes, i.e. on
+//    epilogue threads;
+//  * warp roles: warp 0 issues TMA loads of W (evict-first) and H
+//    (evict-last) into a multi-stage 128-byte-swizzled shared-memory ring;
+//    warp 1 allocates TMEM and issues tcgen05.mma; warps 2-9 drain the
+//    double-buffered accumulator while the next tile is being multiplied;
+//  * epilogue per element: x = acc / T, Philox4x32-10 noise word for
+//    (seed, step, row, token) (one Philox call serves four consecutive
+//    tokens; four lanes exchange words with a 4x4 shuffle transpose), the
+//    Gumbel transform, s = x + g, then a 32-lane "transpose-reduce" leaves
+//    lane j with the packed max of column j;
+//  * flat mode: per CTA, one atomicMax of a packed (score, token) key per row
+//    into the workspace; the last CTA to finish (atomic ticket, no waiting)
+//    decodes the tokens and re-zeroes the workspace;
+//  * grouped mode: per (segment, row) partial (max key, lse pieces) for the
+//    Group-Gumbel-Max merge kernel;
+//  * logits mode: raw fp32 logits to HBM for the unfused measurement path.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "fmms_common.cuh"
+#include "launch.h"
+#include "noise.cuh"
+#include "sm100.cuh"
+
+namespace fmms {
+
+template <int BN>
+struct KCfg {
+  static constexpr int kStageW = kTileM * kBlockK * 2;  // 16 KB of W per stage
+  static constexpr int kStageH = BN * kBlockK * 2;      // BN rows of H per stage
+  static constexpr int kStageBytes = kStageW + kStageH;
+  static constexpr int kStagesFit = 196608 / kStageBytes;
+  static constexpr int kStages = kStagesFit < 10 ? kStagesFit : 10;
+  static constexpr int kCW = BN >= 64 ? 32 : 16;        // columns per epilogue chunk
+  static constexpr int kChunks = BN / kCW;
+  static constexpr int kChunksPerHalf = kChunks >= 2 ? kChunks / 2 : 1;
+  static constexpr int kTmemCols = 2 * BN < 32 ? 32 : 2 * BN;  // two accumulators
+  static constexpr uint32_t kIdesc = sm100::idesc_bf16_f32(kTileM, BN);
+  static constexpr int kBarBytes = 256;
+  static constexpr int kCombBytes = 4 * BN * 16;
+  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBarBytes + kCombBytes;
+  static_assert(kStageH % 1024 == 0, "H stage must keep 1024-byte atom alignment");
+  static_assert((2 * kStages + 5) * 8 + 16 <= kBarBytes, "barrier area too small");
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+};
+
+// ---------------------------------------------------------------------------
+// Epilogue helpers
+// ---------------------------------------------------------------------------
+
+// Four lanes with the same token >> 2 each hold the four Philox words of one
+// column (lane i: column c + i, words for tokens 4q..4q+3).  Afterwards lane
+// i holds, in w[m], the word of token 4q + i for column c + m.
+__device__ __forceinline__ void quad_transpose(uint32_t (&w)[4], int lane) {
+  const bool b0 = (lane & 1) != 0;
+  const bool b1 = (lane & 2) != 0;
+  const uint32_t s01 = b0 ? w[0] : w[1];
+  const uint32_t s23 = b0 ? w[2] : w[3];
+  const uint32_t r01 = __shfl_xor_sync(0xffffffffu, s01, 1);
+  const uint32_t r23 = __shfl_xor_sync(0xffffffffu, s23, 1);
+  if (b0) {
+    w[0] = r01;
+    w[2] = r23;
+  } else {
+    w[1] = r01;
+    w[3] = r23;
+  }
+  const uint32_t s02 = b1 ? w[0] : w[2];
+  const uint32_t s13 = b1 ? w[1] : w[3];
+  const uint32_t r02 = __shfl_xor_sync(0xffffffffu, s02, 2);
+  const uint32_t r13 = __shfl_xor_sync(0xffffffffu, s13, 2);
+  if (b1) {
+    w[0] = r02;
+    w[1] = r13;
+  } else {
+    w[2] = r02;
+    w[3] = r13;
+  }
+}
+
+// Lane that ends up holding column j of a CW-column transpose-reduce.
+template <int CW>
+__device__ __forceinline__ int column_of_lane(int lane) {
+  return CW == 32 ? lane : (lane >> 1);
+}
+template <int CW>
+__device__ __forceinline__ int lane_of_column(int j) {
+  return CW == 32 ? j : 2 * j;
+}
+
+// Transpose-reduce: every lane holds CW values (one per column); afterwards
+// lane l holds the reduction over all 32 lanes of column column_of_lane(l).
+// Each halving round keeps one half of the columns and trades the other half
+// with the partner lane, so CW=32 costs 31 exchanges instead of 32 x 5.
+struct OpMaxU64 {
+  __device__ __forceinline__ static uint64_t apply(uint64_t a, uint64_t b) { return a > b ? a : b; }
+};
+struct OpMaxF {
+  __device__ __forceinline__ static float apply(float a, float b) { return fmaxf(a, b); }
+};
+struct OpAddF {
+  __device__ __forceinline__ static float apply(float a, float b) { return a + b; }
+};
+
+template <int CW, class Op, class T>
+__device__ __forceinline__ T transpose_reduce(T (&k)[CW], int lane) {
+#pragma unroll
+  for (int half = CW / 2, off = 16; half >= 1; half /= 2, off /= 2) {
+    const bool upper = (lane & off) != 0;
+#pragma unroll
+    for (int i = 0; i < half; ++i) {
+      const T send = upper ? k[i] : k[i + half];
+      const T keep = upper ? k[i + half] : k[i];
+      const T recv = __shfl_xor_sync(0xffffffffu, send, off);
+      k[i] = Op::apply(keep, recv);
+    }
+  }
+  if (CW == 16) k[0] = Op::apply(k[0], __shfl_xor_sync(0xffffffffu, k[0], 1));
+  return k[0];
+}
+
+// Folds (m2, s2) into the running log-sum-exp pieces (m, s): sum exp(x - m) = s.
+__device__ __forceinline__ void lse_merge(float &m, float &s, float m2, float s2) {
+  if (m2 == -INFINITY) return;
+  if (m == -INFINITY) {
+    m = m2;
+    s = s2;
+    return;
+  }
+  const float mx = fmaxf(m, m2);
+  s = s * __expf(m - mx) + s2 * __expf(m2 - mx);
+  m = mx;
+}
+
+// One chunk of CW columns for one tile row v (one per thread): scores,
+// transpose-reduce, fold into the lane's running best of its column.
+template <int CW, int MODE>
+__device__ __forceinline__ void epi_chunk(const uint32_t (&acc)[CW], const FmmsParams &p, int v,
+                                          bool v_ok, int col0, int lane, uint64_t &best,
+                                          float &m_run, float &s_run) {
+  uint64_t key[CW];
+  float xs[CW];
+#pragma unroll
+  for (int q4 = 0; q4 < CW / 4; ++q4) {
+    const int colp = col0 + 4 * q4 + (lane & 3);  // column of this lane's Philox call
+    const uint32_t bg = static_cast<uint32_t>(p.b_off + colp);
+    uint64_t k64 = p.seed;
+    if (p.row_seeds != nullptr && colp < p.B) k64 = __ldg(p.row_seeds + bg);
+    const Philox4 ph = philox4x32_10(static_cast<uint32_t>(v) >> 2, bg, p.step, 0u,
+                                     static_cast<uint32_t>(k64), static_cast<uint32_t>(k64 >> 32));
+    uint32_t w[4] = {ph.w0, ph.w1, ph.w2, ph.w3};
+    quad_transpose(w, lane);
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int j = 4 * q4 + m;
+      const int col = col0 + j;
+      bool ok = v_ok && col < p.B;
+      if (ok && p.mask != nullptr) {
+        const uint32_t word =
+            __ldg(p.mask + static_cast<size_t>(p.b_off + col) * p.mask_words + (v >> 5));
+        ok = ((word >> (v & 31)) & 1u) != 0;
+      }
+      const float x = __uint_as_float(acc[j]) * p.inv_temp;
+      const float s = x + gumbel_from_u32(w[m]);
+      key[j] = ok ? pack_key(__float_as_uint(s), v) : 0ull;
+      if (MODE == kModeGrouped) xs[j] = ok ? x : -INFINITY;
+    }
+  }
+  const uint64_t cmax = transpose_reduce<CW, OpMaxU64>(key, lane);
+  best = cmax > best ? cmax : best;
+  if (MODE == kModeGrouped) {
+    float t[CW];
+#pragma unroll
+    for (int j = 0; j < CW; ++j) t[j] = xs[j];
+    const float colmax = transpose_reduce<CW, OpMaxF>(t, lane);
+    float e[CW];
+#pragma unroll
+    for (int j = 0; j < CW; ++j) {
+      const float cm = __shfl_sync(0xffffffffu, colmax, lane_of_column<CW>(j));
+      e[j] = (xs[j] == -INFINITY) ? 0.f : __expf(xs[j] - cm);
+    }
+    const float colsum = transpose_reduce<CW, OpAddF>(e, lane);
+    lse_merge(m_run, s_run, colmax, colsum);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Roles
+// ---------------------------------------------------------------------------
+
+template <int BN>
+__device__ __forceinline__ void role_producer(const CUtensorMap *tw, const CUtensorMap *tw8,
+                                              const CUtensorMap *th, const FmmsParams &p,
+                                              const Schedule &sch, uint8_t *stages,
+                                              uint64_t *full, uint64_t *empty,
+                                              volatile int *abort_flag) {
+  using C = KCfg<BN>;
+  const uint64_t pol_w = sm100::l2_policy_evict_first();
+  const uint64_t pol_h = sm100::l2_policy_evict_last();
+  TileIter it(sch, blockIdx.x);
+  Tile tile;
+  int stage = 0;
+  uint32_t phase = 0;
+  long long issued = 0;
+  bool ok = true;
+  while (ok && it.next(tile)) {
+    const int rows = tile.hi - tile.start;
+    const bool whole = rows == kTileM;
+    const int nbox8 = (rows + kGranule - 1) / kGranule;
+    const uint32_t bytes = (whole ? C::kStageW : nbox8 * 1024) + C::kStageH;
+    for (int kb = 0; kb < p.nk; ++kb) {
+      if (!sm100::wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.err)) {
+        ok = false;
+        break;
+      }
+      uint8_t *sw = stages + stage * C::kStageBytes;
+      uint8_t *sh = sw + C::kStageW;
+      sm100::mbar_arrive_expect_tx(&full[stage], bytes);
+      const int x = kb * kBlockK;
+      if (whole) {
+        sm100::tma_load_2d(sw, tw, &full[stage], x, tile.start, pol_w);
+      } else {
+        for (int i = 0; i < nbox8; ++i)
+          sm100::tma_load_2d(sw + i * 1024, tw8, &full[stage], x, tile.start + kGranule * i, pol_w);
+      }
+      sm100::tma_load_2d(sh, th, &full[stage], x, p.b_off, pol_h);
+      ++issued;
+      if (++stage == C::kStages) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    }
+  }
+  if (!ok) {
+    // Gave up: let the copies already in flight land before the CTA exits.
+    const long long first = issued > C::kStages ? issued - C::kStages : 0;
+    for (long long n = first; n < issued; ++n) {
+      const int s = static_cast<int>(n % C::kStages);
+      const uint32_t ph = static_cast<uint32_t>((n / C::kStages) & 1);
+      const long long t0 = clock64();
+      while (!sm100::mbar_try_wait(&full[s], ph) && clock64() - t0 < sm100::kWaitLimitCycles) {
+      }
+    }
+  }
+}
+
+template <int BN>
+__device__ __forceinline__ void role_mma(const FmmsParams &p, const Schedule &sch,
+                                         uint8_t *stages, uint64_t *full, uint64_t *empty,
+                                         uint64_t *acc_full, uint64_t *acc_empty,
+                                         uint64_t *drain_bar, uint32_t tmem_base,
+                                         volatile int *abort_flag) {
+  using C = KCfg<BN>;
+  TileIter it(sch, blockIdx.x);
+  Tile tile;
+  int stage = 0;
+  uint32_t phase = 0;
+  int buf = 0;
+  uint32_t acc_phase = 0;
+  bool ok = true;
+  while (ok && it.next(tile)) {
+    if (!sm100::wait_bounded(&acc_empty[buf], acc_phase ^ 1u, abort_flag, p.err)) break;
+    sm100::tc_fence_after();
+    const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
+    for (int kb = 0; kb < p.nk; ++kb) {
+      if (!sm100::wait_bounded(&full[stage], phase, abort_flag, p.err)) {
+        ok = false;
+        break;
+      }
+      sm100::tc_fence_after();
+      const uint32_t a_addr = sm100::smem_addr(stages + stage * C::kStageBytes);
+      const uint32_t b_addr = a_addr + C::kStageW;
+#pragma unroll
+      for (int kk = 0; kk < kBlockK / 16; ++kk) {
+        sm100::mma_bf16_ss(d_tmem, sm100::smem_desc_sw128(a_addr + kk * 32),
+                           sm100::smem_desc_sw128(b_addr + kk * 32), C::kIdesc,
+                           (kb | kk) != 0 ? 1u : 0u);
+      }
+      sm100::mma_commit(&empty[stage]);  // frees the stage once these MMAs finish
+      if (++stage == C::kStages) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    }
+    if (!ok) break;
+    sm100::mma_commit(&acc_full[buf]);   // accumulator ready for the epilogue
+    buf ^= 1;
+    if (buf == 0) acc_phase ^= 1u;
+  }
+  // Drain: every MMA issued above has completed once this arrives.
+  sm100::mma_commit(drain_bar);
+  const long long t0 = clock64();
+  while (!sm100::mbar_try_wait(drain_bar, 0) && clock64() - t0 < sm100::kWaitLimitCycles) {
+  }
+}
+
+template <int BN, int MODE>
+__device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedule &sch,
+                                              uint32_t tmem_base, uint64_t *acc_full,
+                                              uint64_t *acc_empty, volatile int *abort_flag,
+                                              int *last_flag, uint64_t *comb_key, float *comb_m,
+                                              float *comb_s, int warp, int lane) {
+  using C = KCfg<BN>;
+  constexpr int CW = C::kCW;
+  const int q = warp & 3;          // TMEM lane quarter this warp may access
+  const int h = (warp - 2) >> 2;   // which half of the column chunks
+  const int etid = (warp - 2) * 32 + lane;
+
+  uint64_t best[C::kChunksPerHalf];
+  float m_run[C::kChunksPerHalf], s_run[C::kChunksPerHalf];
+#pragma unroll
+  for (int i = 0; i < C::kChunksPerHalf; ++i) {
+    best[i] = 0ull;
+    m_run[i] = -INFINITY;
+    s_run[i] = 0.f;
+  }
+
+  TileIter it(sch, blockIdx.x);
+  Tile tile;
+  int buf = 0;
+  uint32_t phase = 0;
+  bool aborted = false;
+  while (it.next(tile)) {
+    // After an abort the loop keeps walking the tiles without touching TMEM,
+    // so that every epilogue warp reaches the same named barriers.  The
+    // decision is made warp-uniform because the TMEM loads below are
+    // warp-collective.
+    const bool got = aborted ? false : sm100::wait_bounded(&acc_full[buf], phase, abort_flag, p.err);
+    aborted = __any_sync(0xffffffffu, !got);
+    if (!aborted) {
+      sm100::tc_fence_after();
+      const int v = tile.start + 32 * q + lane;
+      const bool v_ok = v >= tile.lo && v < tile.hi;
+      const uint32_t tbase =
+          tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(buf * BN);
+#pragma unroll
+      for (int kk = 0; kk < C::kChunksPerHalf; ++kk) {
+        if (C::kChunks < 2 && h == 1) continue;
+        const int k = C::kChunks >= 2 ? 2 * kk + h : kk;
+        const int col0 = k * CW;
+        if (col0 >= p.B) continue;  // warp-uniform
+        uint32_t acc[CW];
+        if constexpr (CW == 32) {
+          sm100::tmem_ld_32(tbase + col0, acc);
+        } else {
+          sm100::tmem_ld_16(tbase + col0, acc);
+        }
+        sm100::tmem_wait_ld();
+        if constexpr (MODE == kModeLogits) {
+          if (v_ok) {
+#pragma unroll
+            for (int j = 0; j < CW; ++j)
+              if (col0 + j < p.B)
+                p.logits[static_cast<size_t>(col0 + j) * p.V + v] = __uint_as_float(acc[j]);
+          }
+        } else {
+          epi_chunk<CW, MODE>(acc, p, v, v_ok, col0, lane, best[kk], m_run[kk], s_run[kk]);
+        }
+      }
+      sm100::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) sm100::mbar_arrive(&acc_empty[buf]);
+    }
+    buf ^= 1;
+    if (buf == 0) phase ^= 1u;
+
+    if constexpr (MODE == kModeGrouped) {
+      if (tile.last) {
+        // Segment done: combine the four lane quarters and write the partial.
+#pragma unroll
+        for (int kk = 0; kk < C::kChunksPerHalf; ++kk) {
+          if (C::kChunks < 2 && h == 1) continue;
+          const int k = C::kChunks >= 2 ? 2 * kk + h : kk;
+          const int col = k * CW + column_of_lane<CW>(lane);
+          if (k * CW < p.B) {
+            comb_key[q * BN + col] = best[kk];
+            comb_m[q * BN + col] = m_run[kk];
+            comb_s[q * BN + col] = s_run[kk];
+          }
+          best[kk] = 0ull;
+          m_run[kk] = -INFINITY;
+          s_run[kk] = 0.f;
+        }
+        sm100::epi_sync(kEpiThreads);
+        if (!*abort_flag) {
+          for (int b = etid; b < p.B; b += kEpiThreads) {
+            uint64_t kb = 0ull;
+            float m = -INFINITY, s = 0.f;
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq) {
+              const uint64_t kq = comb_key[qq * BN + b];
+              kb = kq > kb ? kq : kb;
+              lse_merge(m, s, comb_m[qq * BN + b], comb_s[qq * BN + b]);
+            }
+            GroupPartial gp;
+            gp.key = kb;
+            gp.m = m;
+            gp.sum = s;
+            p.partials[static_cast<size_t>(tile.slot) * p.B + b] = gp;
+          }
+        }
+        sm100::epi_sync(kEpiThreads);
+      }
+    }
+  }
+
+  if constexpr (MODE == kModeFlat) {
+#pragma unroll
+    for (int kk = 0; kk < C::kChunksPerHalf; ++kk) {
+      if (C::kChunks < 2 && h == 1) continue;
+      const int k = C::kChunks >= 2 ? 2 * kk + h : kk;
+      if (k * CW < p.B) comb_key[q * BN + k * CW + column_of_lane<CW>(lane)] = best[kk];
+    }
+    sm100::epi_sync(kEpiThreads);
+    const bool ok = !*abort_flag;
+    if (ok) {
+      for (int b = etid; b < p.B; b += kEpiThreads) {
+        uint64_t kb = 0ull;
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq) {
+          const uint64_t kq = comb_key[qq * BN + b];
+          kb = kq > kb ? kq : kb;
+        }
+        if (kb != 0ull) atomicMax(p.keys + b, static_cast<unsigned long long>(kb));
+      }
+      __threadfence();
+    }
+    sm100::epi_sync(kEpiThreads);
+    if (etid == 0) {
+      int last = 0;
+      if (ok) last = (atomicAdd(p.ticket, 1u) == static_cast<unsigned>(p.num_ctas - 1)) ? 1 : 0;
+      *last_flag = last;
+    }
+    sm100::epi_sync(kEpiThreads);
+    if (*last_flag) {
+      // Every other CTA has published its maxima: decode and re-zero.
+      __threadfence();
+      for (int b = etid; b < p.B; b += kEpiThreads) {
+        const unsigned long long kb = atomicExch(p.keys + b, 0ull);
+        p.out_idx[b] = key_token(kb);
+      }
+      if (etid == 0) atomicExch(p.ticket, 0u);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Kernel
+// ---------------------------------------------------------------------------
+template <int BN, int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+    fmms_kernel(const __grid_constant__ CUtensorMap tmap_w,
+                const __grid_constant__ CUtensorMap tmap_w8,
+                const __grid_constant__ CUtensorMap tmap_h, const FmmsParams p) {
+  using C = KCfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t *stages = smem;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kStages * C::kStageBytes);
+  uint64_t *full = bars;
+  uint64_t *empty = full + C::kStages;
+  uint64_t *acc_full = empty + C::kStages;
+  uint64_t *acc_empty = acc_full + 2;
+  uint64_t *drain_bar = acc_empty + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain_bar + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  int *last_flag = reinterpret_cast<int *>(tmem_slot + 2);
+  uint8_t *comb = reinterpret_cast<uint8_t *>(bars) + C::kBarBytes;
+  uint64_t *comb_key = reinterpret_cast<uint64_t *>(comb);
+  float *comb_m = reinterpret_cast<float *>(comb_key + 4 * BN);
+  float *comb_s = comb_m + 4 * BN;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  Schedule sch;
+  sch.V = p.V;
+  sch.G = p.G;
+  sch.num_ctas = p.num_ctas;
+  sch.ngran = p.ngran;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      sm100::mbar_init(&full[s], 1);
+      sm100::mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      sm100::mbar_init(&acc_full[b], 1);
+      sm100::mbar_init(&acc_empty[b], kNumEpiWarps);
+    }
+    sm100::mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    *last_flag = 0;
+    sm100::fence_mbar_init();
+    sm100::fence_async_smem();
+    sm100::prefetch_tensormap(&tmap_w);
+    sm100::prefetch_tensormap(&tmap_w8);
+    sm100::prefetch_tensormap(&tmap_h);
+  }
+  if (warp == 1) {
+    sm100::tmem_alloc(tmem_slot, C::kTmemCols);
+    sm100::tmem_relinquish();
+  }
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0)
+      role_producer<BN>(&tmap_w, &tmap_w8, &tmap_h, p, sch, stages, full, empty, abort_flag);
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0)
+      role_mma<BN>(p, sch, stages, full, empty, acc_full, acc_empty, drain_bar, tmem_base,
+                   abort_flag);
+    __syncwarp();
+  } else {
+    role_epilogue<BN, MODE>(p, sch, tmem_base, acc_full, acc_empty, abort_flag, last_flag,
+                            comb_key, comb_m, comb_s, warp, lane);
+  }
+
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::tc_fence_after();
+  if (warp == 1) sm100::tmem_dealloc(tmem_base, C::kTmemCols);
+}
+
+// ---------------------------------------------------------------------------
+// Host launchers
+// ---------------------------------------------------------------------------
+template <int BN, int MODE>
+static cudaError_t launch_t(const CUtensorMap &tw, const CUtensorMap &tw8, const CUtensorMap &th,
+                            const FmmsParams &p, cudaStream_t stream) {
+  using C = KCfg<BN>;
+  auto kern = fmms_kernel<BN, MODE>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  kern<<<p.num_ctas, kThreads, C::kSmemBytes, stream>>>(tw, tw8, th, p);
+  return cudaGetLastError();
+}
+
+template <int MODE>
+static cudaError_t launch_mode(int BN, const CUtensorMap &tw, const CUtensorMap &tw8,
+                               const CUtensorMap &th, const FmmsParams &p, cudaStream_t stream) {
+  switch (BN) {
+    case 16: return launch_t<16, MODE>(tw, tw8, th, p, stream);
+    case 32: return launch_t<32, MODE>(tw, tw8, th, p, stream);
+    case 64: return launch_t<64, MODE>(tw, tw8, th, p, stream);
+    case 128: return launch_t<128, MODE>(tw, tw8, th, p, stream);
+    case 256: return launch_t<256, MODE>(tw, tw8, th, p, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_fmms(int mode, int BN, const CUtensorMap &tw, const CUtensorMap &tw8,
+                        const CUtensorMap &th, const FmmsParams &p, cudaStream_t stream) {
+  switch (mode) {
+    case kModeFlat: return launch_mode<kModeFlat>(BN, tw, tw8, th, p, stream);
+    case kModeGrouped: return launch_mode<kModeGrouped>(BN, tw, tw8, th, p, stream);
+    case kModeLogits: return launch_mode<kModeLogits>(BN, tw, tw8, th, p, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+int fmms_batch_tile(int rows) {
+  if (rows <= 16) return 16;
+  if (rows <= 32) return 32;
+  if (rows <= 64) return 64;
+  if (rows <= 128) return 128;
+  return 256;
+}
+
+}  // namespace fmms

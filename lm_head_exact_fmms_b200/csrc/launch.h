@@ -1,0 +1,53 @@
+// launch.h -- host-side launchers of the FMMS kernels (internal to libfmms).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "fmms_common.cuh"
+
+namespace fmms {
+
+// Smallest supported MMA N (16, 32, 64, 128, 256) holding `rows` batch rows.
+int fmms_batch_tile(int rows);
+
+// The fused kernel in mode kModeFlat / kModeGrouped / kModeLogits with batch
+// tile BN, grid p.num_ctas x 320 threads.
+cudaError_t launch_fmms(int mode, int BN, const CUtensorMap &tw, const CUtensorMap &tw8,
+                        const CUtensorMap &th, const FmmsParams &p, cudaStream_t stream);
+
+// Group-Gumbel-Max merge of the grouped partials of one launch (B rows).
+struct MergeParams {
+  const GroupPartial *partials;  // [num_ctas + G - 1][B]
+  int B, b_off, V, G, num_ctas, ngran;
+  uint64_t seed;
+  const uint64_t *row_seeds;
+  uint32_t step;
+  int32_t *out_idx;              // [B], offset to this launch
+  void *summary;                 // fs_group_summary [B][G] offset to this launch, or null
+};
+cudaError_t launch_group_merge(const MergeParams &m, cudaStream_t stream);
+
+// Second kernel of the unfused mode: samples from fp32 logits [B][V].
+struct SampleLogitsParams {
+  const float *logits;           // [B][V], offset to this launch
+  int B, b_off, V;
+  float inv_temp;
+  uint64_t seed;
+  const uint64_t *row_seeds;
+  uint32_t step;
+  const uint32_t *mask;
+  int mask_words;
+  unsigned long long *keys;      // workspace [B]
+  unsigned int *ticket;
+  int32_t *out_idx;
+  int num_sms;
+};
+cudaError_t launch_sample_logits(const SampleLogitsParams &s, cudaStream_t stream);
+
+cudaError_t launch_philox_test(const uint32_t *ctr, const uint32_t *key, uint32_t *out, int64_t n,
+                               cudaStream_t stream);
+cudaError_t launch_gumbel_test(const uint32_t *r, float *g, int64_t n, cudaStream_t stream);
+
+}  // namespace fmms

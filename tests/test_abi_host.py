@@ -1,0 +1,124 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads and
+exports every symbol include/fmms.h declares, arguments are validated before
+anything touches CUDA, and the split-V schedule the kernels walk covers the
+vocabulary exactly once with tiles that never cross a group boundary."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from lm_head_exact_fmms_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fmms.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from lm_head_exact_fmms_b200 import build
+    build.build()
+    return binding.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fs_\w+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 12
+    for name in names:
+        assert hasattr(lib, name), name
+    assert set(names) == set(binding.EXPORTED)
+
+
+def test_status_strings(lib):
+    for code, name in binding._STATUS.items():
+        assert binding.fs_status_string(code) == name
+
+
+FAKE = ctypes.c_void_p(0x10000)      # never dereferenced: validation fails first
+FAKE_ODD = ctypes.c_void_p(0x10008)  # not 16-byte aligned
+
+
+def _sample(lib, H=FAKE, W=FAKE, B=4, d=64, V=100, T=1.0, out=FAKE):
+    return lib.fs_sample(H, W, B, d, V, T, 0, 0, None, out, None)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(H=None), dict(W=None), dict(out=None), dict(B=0), dict(V=0), dict(d=0), dict(d=4),
+    dict(d=12), dict(T=0.0), dict(T=-1.0), dict(T=float("nan")), dict(T=float("inf")),
+    dict(H=FAKE_ODD), dict(W=FAKE_ODD),
+])
+def test_invalid_arguments_rejected_on_host(lib, kw):
+    assert _sample(lib, **kw) == 1
+
+
+def test_grouped_and_unfused_validation(lib):
+    g = lambda G: lib.fs_sample_grouped(FAKE, FAKE, 4, 64, 100, G, 1.0, 0, None, 0, None, FAKE,
+                                        None, None, 0, None)
+    assert g(0) == 1 and g(101) == 1 and g(-3) == 1
+    assert lib.fs_sample_unfused(FAKE, FAKE, 4, 64, 100, 1.0, 0, None, 0, None, FAKE, None, None,
+                                 0, None) == 1
+    assert lib.fs_sample_host(None, FAKE, 4, 64, 100, 1.0, 0, None, 0, None, FAKE, None) == 1
+    assert lib.fs_philox4x32_10(None, None, None, 5, None) == 1
+    assert lib.fs_gumbel(None, None, -1, None) == 1
+
+
+def _all_tiles(V, G, sms):
+    _, nc = binding.fs_plan_tiles(V, G, sms, 0)
+    return nc, [binding.fs_plan_tiles(V, G, sms, c)[0] for c in range(nc)]
+
+
+@pytest.mark.parametrize("V,G,sms", [
+    (1, 0, 148), (7, 1, 148), (12, 3, 148), (129, 0, 148), (4096, 0, 148), (4097, 5, 148),
+    (151936, 0, 148), (151936, 8, 148), (151937, 8, 148), (128256, 0, 148), (1000, 1000, 148),
+    (64, 64, 148), (5003, 7, 13), (100000, 97, 148),
+])
+def test_schedule_covers_vocab_once(lib, V, G, sms):
+    nc, per_cta = _all_tiles(V, G, sms)
+    Geff = max(G, 1)
+    assert nc == min(sms, (V + 7) // 8)
+    bounds = [(g * V) // Geff for g in range(Geff + 1)]
+    owner = np.full(V, -1)
+    slots = set()
+    rows_per_cta = []
+    for c, tiles in enumerate(per_cta):
+        assert len(tiles) > 0
+        rows = 0
+        for i, (start, lo, hi, slot, last) in enumerate(tiles):
+            assert start % 8 == 0 and start <= lo < hi <= start + 128
+            g = np.searchsorted(bounds, lo, side="right") - 1
+            assert bounds[g] <= lo and hi <= bounds[g + 1], "tile crosses a group boundary"
+            assert slot == c + g and slot < nc + Geff - 1
+            assert np.all(owner[lo:hi] == -1), "token covered twice"
+            owner[lo:hi] = c
+            rows += hi - lo
+            nxt = tiles[i + 1] if i + 1 < len(tiles) else None
+            assert last == (1 if nxt is None or nxt[3] != slot else 0)
+            slots.add((c, g, slot))
+        rows_per_cta.append(rows)
+    assert np.all(owner >= 0), "token never covered"
+    assert np.all(np.diff(owner) >= 0), "CTA ranges are not contiguous and ordered"
+    assert len({s for _, _, s in slots}) == len(slots), "slot reused by two segments"
+    # balance: every CTA streams the same number of rows to within one granule
+    full = rows_per_cta[:-1] if V % 8 else rows_per_cta
+    if full:
+        assert max(full) - min(full) <= 8
+    # the grouped merge enumerates exactly the CTAs that met the group
+    if G >= 1:
+        for g in range(Geff):
+            first, last = binding.fs_plan_group_ctas(V, G, sms, g)
+            met = sorted({c for c, gg, _ in slots if gg == g})
+            assert met == list(range(first, last + 1))
+
+
+def test_flagship_schedule_balance(lib):
+    """Qwen3 heads: 148 CTAs stream 1026-1027 rows each (8.02 tiles), not 8 or 9 tiles."""
+    nc, per_cta = _all_tiles(151936, 0, 148)
+    rows = [int(sum(t[2] - t[1] for t in tiles)) for tiles in per_cta]
+    assert nc == 148 and min(rows) >= 1024 and max(rows) <= 1032

@@ -1,0 +1,333 @@
+"""GPU parity of the sm_100a path against the CPU oracle, through the C ABI.
+
+Tolerance (stated for the method's floating-point result): the noise words
+and the (row, token) indexing are bit-exact; a sampled token may differ from
+the oracle's only where the oracle's best and second-best perturbed scores lie
+within 2e-3 * (1 + |best|), and such rows must stay below 1e-4 of all rows
+(checked in aggregate by test_mismatch_rate_bound).  Everything else must
+match exactly, including -1 for fully masked rows.
+"""
+import numpy as np
+import pytest
+import torch
+
+from lm_head_exact_fmms_b200 import binding, synth
+
+pytestmark = pytest.mark.gpu
+
+TIE_REL = 2e-3
+
+
+@pytest.fixture(scope="module")
+def dev():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from lm_head_exact_fmms_b200 import build
+    build.build()
+    binding.load_library()
+    return torch.device("cuda:0")
+
+
+def near_tie(best, second):
+    return (best - second) <= TIE_REL * (1.0 + np.abs(best))
+
+
+def assert_parity(gpu, o_idx, o_best, o_second, what=""):
+    gpu = np.asarray(gpu)
+    bad = gpu != o_idx
+    if bad.any():
+        allowed = near_tie(o_best, o_second)
+        hard = bad & ~allowed
+        assert not hard.any(), "%s: %d rows differ outside the tie tolerance: rows %s gpu %s oracle %s" % (
+            what, hard.sum(), np.flatnonzero(hard)[:8], gpu[hard][:8], o_idx[hard][:8])
+    return int(bad.sum())
+
+
+def rand_inputs(B, d, V, seed, w_std=None, device="cuda"):
+    H = synth.make_hidden(B, d, device="cpu", seed=seed)
+    W = synth.make_weight(V, d, w_std if w_std is not None else 1.0 / np.sqrt(d), device="cpu",
+                          seed=seed + 1)
+    return H, W, H.to(device), W.to(device)
+
+
+# ---------------------------------------------------------------- noise
+def test_philox_bitwise(dev, oracle):
+    rng = np.random.default_rng(1)
+    n = 1 << 20
+    ctr = rng.integers(0, 2 ** 32, size=(n, 4), dtype=np.uint64).astype(np.uint32)
+    key = rng.integers(0, 2 ** 32, size=(n, 2), dtype=np.uint64).astype(np.uint32)
+    ctr[:4096, 1:] = 0
+    ref = oracle.philox4x32_10(ctr, key)
+    t_ctr = torch.from_numpy(ctr.view(np.int32)).to(dev)
+    t_key = torch.from_numpy(key.view(np.int32)).to(dev)
+    got = binding.fs_philox4x32_10(t_ctr, t_key).cpu().numpy().view(np.uint32)
+    assert np.array_equal(got, ref)
+
+
+def gumbel_rs():
+    lo = np.arange(0, 1 << 20, dtype=np.uint64)
+    hi = np.arange((1 << 32) - (1 << 20), 1 << 32, dtype=np.uint64)
+    mid = np.linspace(1 << 20, (1 << 32) - (1 << 20) - 1, 1 << 22).astype(np.uint64)
+    edge = np.arange((1 << 31) - 4096, (1 << 31) + 4096, dtype=np.uint64)
+    return np.unique(np.concatenate([lo, mid, edge, hi])).astype(np.uint32)
+
+
+def test_gumbel_transform_accuracy(dev, oracle):
+    """fp32 g(r) within 3 ulp(g) + 2^-22 of the fp64 value on both tails, the
+    branch boundary and a stratified sample; finite and non-decreasing in r.
+    Derivation: the fp32 inputs u or 1-u carry 2^-24 relative rounding, which
+    reaches g as at most ~1.5 * 2^-24 absolute after two logs; logf/log1pf add
+    about one ulp each, the outer log's ulp being ulp(g)."""
+    r = gumbel_rs()
+    ref = oracle.gumbel(r)
+    got = binding.fs_gumbel(torch.from_numpy(r.view(np.int32)).to(dev)).cpu().numpy()
+    assert np.all(np.isfinite(got))
+    ulp = np.spacing(np.abs(ref).astype(np.float32)).astype(np.float64)
+    err = np.abs(got.astype(np.float64) - ref)
+    assert np.all(err <= 3 * ulp + 2.0 ** -22), (err / ulp).max()
+    assert np.all(np.diff(got) >= 0)
+
+
+# ------------------------------------------------------------ flat sampling
+def test_tiny_workload_matches_golden(dev, oracle):
+    from tests.test_golden import load_golden
+    wl = synth.WORKLOADS["tiny"]
+    H = synth.make_hidden(1, wl.d).to(dev)
+    W = synth.make_weight(wl.V, wl.d, wl.w_std).to(dev)
+    for step, tok, best, second in load_golden():
+        got = binding.fs_sample(H, W, temperature=1.0, seed=0, step=step).item()
+        assert_parity([got], np.array([tok]), np.array([best]), np.array([second]), "tiny")
+
+
+@pytest.mark.parametrize("B,d,V", [
+    (1, 256, 4096), (3, 64, 129), (17, 24, 1000), (64, 128, 4097), (65, 256, 777),
+    (128, 8, 300), (200, 96, 5000), (256, 256, 4096), (257, 64, 2048), (300, 40, 64),
+    (16, 64, 1), (16, 64, 7), (33, 64, 8), (2, 64, 9), (5, 512, 127), (5, 512, 128),
+    (4, 72, 1183),
+])
+def test_flat_parity_shapes(dev, oracle, B, d, V):
+    H, W, Hd, Wd = rand_inputs(B, d, V, seed=B * 1000 + V)
+    T = 0.9
+    got = binding.fs_sample(Hd, Wd, temperature=T, seed=77, step=3).cpu().numpy()
+    idx, best, second = oracle.sample(H, W, T=T, seed=77, step=3)
+    assert_parity(got, idx, best, second, "B=%d d=%d V=%d" % (B, d, V))
+
+
+def test_flat_parity_large_vocab_small_d(dev, oracle):
+    B, d, V = 6, 64, 151937
+    H, W, Hd, Wd = rand_inputs(B, d, V, seed=5, w_std=0.2)
+    got = binding.fs_sample(Hd, Wd, temperature=1.0, seed=1, step=0).cpu().numpy()
+    assert_parity(got, *oracle.sample(H, W, T=1.0, seed=1, step=0), "V=151937")
+
+
+def test_row_seeds_and_temperatures(dev, oracle):
+    B, d, V = 32, 128, 3000
+    H, W, Hd, Wd = rand_inputs(B, d, V, seed=11)
+    rs = synth.make_row_seeds(B)
+    for T in (0.5, 0.7, 2.0):
+        for step in (0, 1, 2 ** 31 + 5):
+            got = binding.fs_sample_ex(Hd, Wd, temperature=T, seed=99, row_seeds=rs.to(dev),
+                                       step=step).cpu().numpy()
+            assert_parity(got, *oracle.sample(H, W, T=T, seed=99, row_seeds=rs, step=step),
+                          "T=%g step=%d" % (T, step))
+
+
+def test_masks(dev, oracle):
+    B, d, V = 8, 64, 5000
+    H, W, Hd, Wd = rand_inputs(B, d, V, seed=21)
+    allowed = torch.rand(B, V, generator=torch.Generator().manual_seed(5)) < 0.5
+    allowed[0] = False
+    allowed[0, 4321] = True          # single allowed token
+    allowed[1] = False               # fully masked -> -1
+    allowed[2] = False
+    allowed[2, V - 1] = True         # only the last token
+    allowed[3] = True
+    mask = synth.mask_from_bool(allowed)
+    for step in range(6):
+        got = binding.fs_sample(Hd, Wd, temperature=1.0, seed=3, step=step,
+                                mask_bits=mask.to(dev)).cpu().numpy()
+        idx, best, second = oracle.sample(H, W, T=1.0, seed=3, step=step, mask=mask)
+        assert got[0] == 4321 and got[1] == -1 and got[2] == V - 1
+        assert allowed[np.arange(B)[got >= 0], got[got >= 0]].all()
+        assert_parity(got, idx, best, second, "mask step %d" % step)
+
+
+def test_peaked_head(dev, oracle):
+    """Low-entropy rows: one token per row gets +8 on its logit."""
+    B, d, V = 16, 64, 2000
+    H, W, _, _ = rand_inputs(B, d, V, seed=31)
+    W = W.clone()
+    W[123] = (H[0].float() * 8.0 / (H[0].float() ** 2).sum()).to(torch.bfloat16)
+    got = binding.fs_sample(H.to(dev), W.to(dev), temperature=1.0, seed=4, step=0).cpu().numpy()
+    assert_parity(got, *oracle.sample(H, W, T=1.0, seed=4, step=0), "peaked")
+
+
+def test_determinism_streams_and_batch_invariance(dev):
+    B, d, V = 64, 128, 10000
+    _, _, Hd, Wd = rand_inputs(B, d, V, seed=41)
+    a = binding.fs_sample(Hd, Wd, temperature=0.8, seed=5, step=9)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())   # the library workspace is shared
+    with torch.cuda.stream(s):
+        b = binding.fs_sample(Hd, Wd, temperature=0.8, seed=5, step=9, stream=s)
+    s.synchronize()
+    torch.cuda.current_stream().wait_stream(s)
+    assert torch.equal(a, b)
+    c = binding.fs_sample(Hd[:5].contiguous(), Wd, temperature=0.8, seed=5, step=9)
+    assert torch.equal(a[:5], c)
+    d2 = binding.fs_sample(Hd, Wd, temperature=0.8, seed=5, step=10)
+    assert not torch.equal(a, d2)
+
+
+def test_caller_workspace_and_status(dev):
+    B, d, V = 40, 64, 9000
+    _, _, Hd, Wd = rand_inputs(B, d, V, seed=51)
+    nbytes = binding.fs_workspace_bytes(B, V, 0)
+    assert nbytes > 0
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
+    ref = binding.fs_sample_ex(Hd, Wd, temperature=1.0, seed=8, step=1)
+    for _ in range(3):
+        got = binding.fs_sample_ex(Hd, Wd, temperature=1.0, seed=8, step=1, workspace=ws)
+        assert torch.equal(got, ref)
+    assert binding.fs_device_status(ws) == 0
+    assert int(ws.count_nonzero()) == 0          # left zeroed for the next call
+    with pytest.raises(binding.FmmsError):
+        binding.fs_sample_ex(Hd, Wd, workspace=ws[:128])
+
+
+def test_host_entry_point(dev):
+    B, d, V = 24, 128, 7000
+    H, _, Hd, Wd = rand_inputs(B, d, V, seed=61)
+    ref = binding.fs_sample_ex(Hd, Wd, temperature=1.0, seed=2, step=4).cpu()
+    Hp = H.pin_memory()
+    out = torch.empty(B, dtype=torch.int32).pin_memory()
+    binding.fs_sample_host(Hp, Wd, temperature=1.0, seed=2, step=4, out_idx_host=out)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
+
+
+def test_gumbel_max_is_softmax_on_gpu(dev, oracle):
+    """Draws of identical rows (noise differs per row index) follow the exact
+    softmax of l / T (chi-square)."""
+    from tests.test_oracle_pins import _chi2_pvalue, _softmax
+    V, d, B, T = 64, 32, 256, 1.3
+    h = synth.make_hidden(1, d, seed=71)
+    W = synth.make_weight(V, d, 0.35, seed=72)
+    Hd = h.to(dev).repeat(B, 1).contiguous()
+    Wd = W.to(dev)
+    counts = torch.zeros(V, dtype=torch.int64, device=dev)
+    for step in range(400):
+        out = binding.fs_sample(Hd, Wd, temperature=T, seed=13, step=step)
+        counts += torch.bincount(out.long(), minlength=V)
+    p = _softmax(oracle.logits(h, W)[0] / T)
+    assert _chi2_pvalue(counts.cpu().numpy(), p) > 1e-3
+
+
+def test_mismatch_rate_bound(dev, oracle):
+    """Aggregate: tokens that differ from the oracle (all near ties) stay
+    below 1e-4 of 25,600 rows."""
+    B, d, V = 256, 64, 4096
+    H, W, Hd, Wd = rand_inputs(B, d, V, seed=81)
+    total = mism = 0
+    for step in range(100):
+        got = binding.fs_sample(Hd, Wd, temperature=1.0, seed=6, step=step).cpu().numpy()
+        idx, best, second = oracle.sample(H, W, T=1.0, seed=6, step=step)
+        mism += assert_parity(got, idx, best, second, "step %d" % step)
+        total += B
+    assert mism / total < 1e-4, (mism, total)
+
+
+# --------------------------------------------------------- grouped sampling
+@pytest.mark.parametrize("G,masked", [(1, False), (2, False), (3, True), (8, True), (64, False),
+                                      (1000, True)])
+def test_grouped_parity(dev, oracle, G, masked):
+    B, d, V = 20, 64, 6007
+    H, W, Hd, Wd = rand_inputs(B, d, V, seed=G + 90)
+    mask = synth.make_mask(B, V, 0.5, seed=G) if masked else None
+    md = mask.to(dev) if masked else None
+    summ = torch.empty(B, G, 3, dtype=torch.float32, device=dev)
+    got = binding.fs_sample_grouped(Hd, Wd, G, temperature=0.8, seed=12, step=2, mask_bits=md,
+                                    out_summary=summ).cpu().numpy()
+    idx, o_summ, margin = oracle.sample_grouped(H, W, G, T=0.8, seed=12, step=2, mask=mask)
+    s = summ.cpu()
+    g_lse = s[:, :, 2].numpy().astype(np.float64)
+    g_arg = s[:, :, 1].contiguous().view(torch.int32).numpy()
+    fin = np.isfinite(o_summ[:, :, 2])
+    assert np.array_equal(np.isfinite(g_lse), fin)
+    assert np.allclose(g_lse[fin], o_summ[:, :, 2][fin], rtol=1e-5, atol=1e-4)
+    ok_arg = g_arg == o_summ[:, :, 1]
+    # per-group argmax: may differ only at a within-group near tie
+    for b in range(B):
+        for g in range(G):
+            if not ok_arg[b, g]:
+                sc = oracle.scores(H, W, T=0.8, seed=12, step=2, mask=mask, rows=[b])[0]
+                lo, hi = (g * V) // G, ((g + 1) * V) // G
+                top = np.sort(sc[lo:hi])[-2:]
+                assert near_tie(top[1], top[0]), (b, g, g_arg[b, g], o_summ[b, g, 1])
+    bad = got != idx
+    for b in np.flatnonzero(bad):
+        assert margin[b, 0] <= TIE_REL * (1 + abs(o_summ[b].max())) or \
+            margin[b, 1] <= TIE_REL * (1 + abs(o_summ[b, :, 0].max())), (b, got[b], idx[b])
+    if G == 1:
+        flat = binding.fs_sample_ex(Hd, Wd, temperature=0.8, seed=12, step=2, mask_bits=md)
+        assert np.array_equal(flat.cpu().numpy(), got)
+
+
+# ------------------------------------------------------------ unfused mode
+@pytest.mark.parametrize("B,V", [(1, 4096), (37, 5001), (256, 3000)])
+def test_unfused_parity(dev, oracle, B, V):
+    d = 128
+    H, W, Hd, Wd = rand_inputs(B, d, V, seed=B + V)
+    mask = synth.make_mask(B, V, 0.7, seed=3)
+    logits = torch.empty(B, V, dtype=torch.float32, device=dev)
+    got = binding.fs_sample_unfused(Hd, Wd, temperature=1.1, seed=9, step=1,
+                                    mask_bits=mask.to(dev), logits=logits).cpu().numpy()
+    assert_parity(got, *oracle.sample(H, W, T=1.1, seed=9, step=1, mask=mask), "unfused")
+    ref_l = oracle.logits(H, W)
+    assert np.allclose(logits.cpu().numpy(), ref_l, rtol=1e-4, atol=1e-4 * np.abs(ref_l).max())
+    fused = binding.fs_sample_ex(Hd, Wd, temperature=1.1, seed=9, step=1, mask_bits=mask.to(dev))
+    assert (fused.cpu().numpy() == got).mean() > 0.99
+
+
+# ----------------------------------------------- full-size workloads (sampled)
+def _sampled_rows(B, rng):
+    rows = {0, B - 1}
+    while len(rows) < min(B, 3):
+        rows.add(int(rng.integers(0, B)))
+    return np.array(sorted(rows), dtype=np.int32)
+
+
+@pytest.mark.parametrize("name", ["qwen3-1.7b", "qwen3-8b", "large", "grouped-masked"])
+def test_full_size_workloads(dev, oracle, name):
+    """Every batch size of each LM-head workload in the launch configuration
+    the benchmark times; oracle on sampled rows."""
+    wl = synth.WORKLOADS[name]
+    rng = np.random.default_rng(0)
+    Wd = synth.make_weight(wl.V, wl.d, wl.w_std, device=dev)
+    W = Wd.cpu()
+    for B in wl.batches:
+        Hd = synth.make_hidden(B, wl.d, device=dev)
+        H = Hd.cpu()
+        rs = synth.make_row_seeds(B) if wl.per_row_seeds else None
+        mask = synth.make_mask(B, wl.V, wl.mask_allowed) if wl.mask_allowed else None
+        rows = _sampled_rows(B, rng)
+        kw = dict(temperature=wl.temperature, seed=0, step=0,
+                  row_seeds=rs.to(dev) if rs is not None else None,
+                  mask_bits=mask.to(dev) if mask is not None else None)
+        if wl.groups:
+            got = binding.fs_sample_grouped(Hd, Wd, wl.groups, **kw).cpu().numpy()
+            idx, summ, margin = oracle.sample_grouped(H, W, wl.groups, T=wl.temperature, seed=0,
+                                                      row_seeds=rs, step=0, mask=mask, rows=rows)
+            for i, b in enumerate(rows):
+                if got[b] != idx[i]:
+                    scale = TIE_REL * (1 + abs(summ[i, :, 0].max()))
+                    assert margin[i, 0] <= scale or margin[i, 1] <= scale, (name, B, b)
+        else:
+            got = binding.fs_sample_ex(Hd, Wd, **kw).cpu().numpy()
+            idx, best, second = oracle.sample(H, W, T=wl.temperature, seed=0, row_seeds=rs,
+                                              step=0, mask=mask, rows=rows)
+            assert_parity(got[rows], idx, best, second, "%s B=%d" % (name, B))
+        assert np.all((got >= 0) & (got < wl.V))
+        del Hd
+    del Wd
+    torch.cuda.empty_cache()
