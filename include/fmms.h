@@ -147,6 +147,30 @@ fs_status fs_sample_host(const void *H_host, const void *W, int B, int d,
                          const uint32_t *mask_bits, int32_t *out_idx_host,
                          fs_stream_t stream);
 
+/* Allocation-free flat sampling: the same computation and arguments as
+ * fs_sample_ex without a workspace.  It exists for callers that must not
+ * call cudaMalloc: a serving engine or framework that owns all device memory
+ * through its own pool and hands a plug-in only its inputs and outputs, or a
+ * decode loop that cannot afford an allocation's latency and device-wide
+ * synchronisation.  The other entry points either allocate a workspace on
+ * their first call or need one from the caller; this one keeps its scratch
+ * (status word, ticket counter, one packed key per row: 2,304 bytes) in a
+ * fixed array inside the library's device memory, which every GPU that
+ * loads the library holds until the process exits.  The paper has no
+ * counterpart for this entry point.
+ * Limit: B <= 256 rows per call; a larger B returns FS_ERR_UNSUPPORTED
+ * (split the batch into several calls).  The first call on each device
+ * looks up the array's device address and may load the library's device
+ * code; make that first call before any stream capture.  Each call clears
+ * the array on `stream` before using it, and every call on a device shares
+ * the same array: calls that overlap on the GPU (different streams or
+ * threads) race, so the caller must order them. */
+fs_status fs_sample_noalloc(const void *H, const void *W, int B, int d, int V,
+                            float temperature, uint64_t seed,
+                            const uint64_t *row_seeds, uint32_t step,
+                            const uint32_t *mask_bits, int32_t *out_idx,
+                            fs_stream_t stream);
+
 /* Bytes of caller workspace needed by the calls above for these sizes on the
  * current device (G = 0 or 1 for flat sampling).  Returns 0 on invalid sizes. */
 size_t fs_workspace_bytes(int B, int V, int G);

@@ -20,7 +20,8 @@ _STATUS = {0: "FS_OK", 1: "FS_ERR_INVALID_ARG", 2: "FS_ERR_UNSUPPORTED", 3: "FS_
 # Every symbol include/fmms.h declares.
 EXPORTED = ("fs_sample", "fs_sample_ex", "fs_sample_grouped", "fs_sample_unfused",
             "fs_sample_host", "fs_workspace_bytes", "fs_device_status", "fs_status_string",
-            "fs_philox4x32_10", "fs_gumbel", "fs_plan_tiles", "fs_plan_group_ctas")
+            "fs_philox4x32_10", "fs_gumbel", "fs_plan_tiles", "fs_plan_group_ctas",
+            "fs_sample_noalloc")
 
 
 class FmmsError(RuntimeError):
@@ -57,6 +58,7 @@ def load_library():
     lib.fs_sample_grouped.argtypes = common + [i32, f32, u64, vp, u32, vp, vp, vp, vp, sz, vp]
     lib.fs_sample_unfused.argtypes = common + [f32, u64, vp, u32, vp, vp, vp, vp, sz, vp]
     lib.fs_sample_host.argtypes = common + [f32, u64, vp, u32, vp, vp, vp]
+    lib.fs_sample_noalloc.argtypes = common + [f32, u64, vp, u32, vp, vp, vp]
     lib.fs_workspace_bytes.argtypes = [i32, i32, i32]
     lib.fs_workspace_bytes.restype = sz
     lib.fs_device_status.argtypes = [vp, sz, vp]
@@ -272,3 +274,19 @@ def fs_plan_group_ctas(V, G, num_sms, g):
     _check(lib.fs_plan_group_ctas(int(V), int(G), int(num_sms), int(g), ctypes.byref(a),
                                   ctypes.byref(z)), "fs_plan_group_ctas")
     return a.value, z.value
+
+
+def fs_sample_noalloc(H, W, temperature=1.0, seed=0, row_seeds=None, step=0, mask_bits=None,
+                      out_idx=None, stream=None):
+    """Allocation-free flat sample (B <= 256) for callers that may not allocate
+    device memory: the library keeps the scratch in a fixed device array.
+    Calls on one device share that array, so they must not overlap on the GPU."""
+    lib = load_library()
+    B, d, V = _check_operands(H, W)
+    row_seeds = _opt_dev(row_seeds, torch.int64, B, "row_seeds", H.device)
+    mask_bits = _opt_dev(mask_bits, torch.int32, B * ((V + 31) // 32), "mask_bits", H.device)
+    out_idx = _out(out_idx, B, H.device)
+    _check(lib.fs_sample_noalloc(_ptr(H), _ptr(W), B, d, V, float(temperature), _seed(seed),
+                                 _ptr(row_seeds), int(step), _ptr(mask_bits), _ptr(out_idx),
+                                 _stream(stream)), "fs_sample_noalloc")
+    return out_idx

@@ -442,3 +442,47 @@ fs_status fs_plan_group_ctas(int V, int G, int num_sms, int g, int *first, int *
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free entry point: scratch in a fixed device array of this file.
+// ---------------------------------------------------------------------------
+namespace {
+
+// Status word + ticket (256 bytes) and packed keys of up to 256 rows.
+constexpr size_t kNoAllocScratchBytes = fmms::kWsHeader + fmms::kWsKeys;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch on each device (null until looked up).
+// In host code the array's name is only a host-side stand-in.
+void *g_noalloc_addr[kMaxDevices];
+
+}  // namespace
+
+extern "C" fs_status fs_sample_noalloc(const void *H, const void *W, int B, int d, int V,
+                                       float temperature, uint64_t seed,
+                                       const uint64_t *row_seeds, uint32_t step,
+                                       const uint32_t *mask_bits, int32_t *out_idx,
+                                       fs_stream_t stream) {
+  fs_status s = validate(H, W, B, d, V, temperature, out_idx);
+  if (s != FS_OK) return s;
+  if (B > fmms::kMaxBN) return FS_ERR_UNSUPPORTED;  // keys for at most 256 rows
+  if (static_cast<size_t>(fmms::workspace_bytes_for(B, 1, 1)) > kNoAllocScratchBytes)
+    return FS_ERR_WORKSPACE;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FS_ERR_CUDA;
+  void *scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (g_noalloc_addr[dev] == nullptr) {
+      void *p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+        return FS_ERR_CUDA;
+      g_noalloc_addr[dev] = p;
+    }
+    scratch = g_noalloc_addr[dev];
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(scratch, 0, kNoAllocScratchBytes, st) != cudaSuccess) return FS_ERR_CUDA;
+  return run(fmms::kModeFlat, H, W, B, d, V, 1, temperature, seed, row_seeds, step, mask_bits,
+             out_idx, nullptr, nullptr, scratch, kNoAllocScratchBytes, st);
+}
