@@ -58,7 +58,7 @@ __global__ void __launch_bounds__(128) group_merge_kernel(const MergeParams m) {
     const float lse = (M == -INFINITY) ? -INFINITY : M + logf(S);
     if (summary != nullptr) {
       fs_group_summary gs;
-      gs.max_score = kmax ? __uint_as_float(key_score_bits(kmax)) : -INFINITY;
+      gs.max_score = key_valid(kmax) ? __uint_as_float(key_score_bits(kmax)) : -INFINITY;
       gs.argmax = key_token(kmax);
       gs.lse = lse;
       summary[static_cast<size_t>(b) * m.G + g] = gs;
@@ -148,7 +148,7 @@ __global__ void __launch_bounds__(256) sample_logits_kernel(const SampleLogitsPa
   if (threadIdx.x == 0) {
     uint64_t r = 0ull;
     for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) r = warp_best[i] > r ? warp_best[i] : r;
-    if (r) atomicMax(s.keys + b, static_cast<unsigned long long>(r));
+    if (key_valid(r)) atomicMax(s.keys + b, static_cast<unsigned long long>(r));
     __threadfence();
     const unsigned total = gridDim.x * gridDim.y;
     is_last = (atomicAdd(s.ticket, 1u) == total - 1) ? 1 : 0;

@@ -123,10 +123,13 @@ struct TileIter {
 // Packed (score, token) key.  Unsigned 64-bit order on
 //   (order_bits(s) << 32) | (0xFFFFFFFF - v)
 // is "larger score first, then smaller token", the tie rule of every argmax
-// here.  0 means "no candidate" (a masked or out-of-range entry).
+// here.  A key whose high word is 0 means "no candidate" (a masked or
+// out-of-range entry): every finite or infinite score maps to a nonzero
+// high word.
 // ---------------------------------------------------------------------------
 FS_HD uint32_t order_bits(uint32_t f) {
-  return (f & 0x80000000u) ? ~f : (f | 0x80000000u);
+  // negative: flip every bit; non-negative: set the sign bit
+  return f ^ (static_cast<uint32_t>(static_cast<int32_t>(f) >> 31) | 0x80000000u);
 }
 FS_HD uint32_t order_bits_inv(uint32_t o) {
   return (o & 0x80000000u) ? (o & 0x7FFFFFFFu) : ~o;
@@ -134,7 +137,8 @@ FS_HD uint32_t order_bits_inv(uint32_t o) {
 FS_HD uint64_t pack_key(uint32_t score_bits, int v) {
   return ((uint64_t)order_bits(score_bits) << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)v);
 }
-FS_HD int key_token(uint64_t k) { return k == 0 ? -1 : (int)(0xFFFFFFFFu - (uint32_t)k); }
+FS_HD bool key_valid(uint64_t k) { return (k >> 32) != 0; }
+FS_HD int key_token(uint64_t k) { return key_valid(k) ? (int)(0xFFFFFFFFu - (uint32_t)k) : -1; }
 FS_HD uint32_t key_score_bits(uint64_t k) { return order_bits_inv((uint32_t)(k >> 32)); }
 
 // Per-(slot, row) partial of the grouped kernel.

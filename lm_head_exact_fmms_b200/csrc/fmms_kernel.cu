@@ -157,6 +157,7 @@ __device__ __forceinline__ void epi_chunk(const uint32_t (&acc)[CW], const FmmsP
                                           float &m_run, float &s_run) {
   uint64_t key[CW];
   float xs[CW];
+  const uint64_t low = 0xFFFFFFFFu - static_cast<uint32_t>(v);  // token part of the key
 #pragma unroll
   for (int q4 = 0; q4 < CW / 4; ++q4) {
     const int colp = col0 + 4 * q4 + (lane & 3);  // column of this lane's Philox call
@@ -177,10 +178,10 @@ __device__ __forceinline__ void epi_chunk(const uint32_t (&acc)[CW], const FmmsP
             __ldg(p.mask + static_cast<size_t>(p.b_off + col) * p.mask_words + (v >> 5));
         ok = ((word >> (v & 31)) & 1u) != 0;
       }
-      const float x = __uint_as_float(acc[j]) * p.inv_temp;
-      const float s = x + gumbel_from_u32(w[m]);
-      key[j] = ok ? pack_key(__float_as_uint(s), v) : 0ull;
-      if (MODE == kModeGrouped) xs[j] = ok ? x : -INFINITY;
+      const float s = fmaf(__uint_as_float(acc[j]), p.inv_temp, gumbel_from_u32(w[m]));
+      const uint32_t hi = ok ? order_bits(__float_as_uint(s)) : 0u;
+      key[j] = (static_cast<uint64_t>(hi) << 32) | low;
+      if (MODE == kModeGrouped) xs[j] = ok ? __uint_as_float(acc[j]) * p.inv_temp : -INFINITY;
     }
   }
   const uint64_t cmax = transpose_reduce<CW, OpMaxU64>(key, lane);
@@ -438,7 +439,7 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
           const uint64_t kq = comb_key[qq * BN + b];
           kb = kq > kb ? kq : kb;
         }
-        if (kb != 0ull) atomicMax(p.keys + b, static_cast<unsigned long long>(kb));
+        if (key_valid(kb)) atomicMax(p.keys + b, static_cast<unsigned long long>(kb));
       }
       __threadfence();
     }

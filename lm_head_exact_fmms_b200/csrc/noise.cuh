@@ -12,13 +12,21 @@
 // The Gumbel transform maps a word r to g = -log(-log u) with
 // u = (r + 1) / (2^32 + 1) (readus.org page, "floating point precision").
 // In fp32, (float)(r + 1) / (2^32 + 1) rounds to 1.0 for the top 256 words,
-// which would make g infinite; so the inner log is taken on whichever of u
-// and 1 - u is below one half, both of which are exact-enough fp32 values:
-//   r <  2^31:  t = -log(u),        u     = (r + 1) 2^-32 (1 - 2^-32 ...)
-//   r >= 2^31:  t = -log1p(-z),     z = 1 - u = (2^32 - r) 2^-32 (...)
-// then g = -log(t).  Dropping the factor 2^32 / (2^32 + 1) changes u by a
-// relative 2.3e-10, far below fp32 rounding.  logf and log1pf are CUDA's
-// accurate library functions (this file must not be built with fast-math).
+// which would make g infinite; so the transform works from
+//   a = q 2^-32,  q = r + 1 (r < 2^31, then a = u) or 2^32 - r (then a = 1 - u),
+// a value in (0, 1/2] that fp32 holds to 2^-24 relative (the neglected factor
+// 2^32 / (2^32 + 1) is 1 - 2.3e-10).  The inner value t = -ln u is then
+//   lower half:  t = -ln a,       with |ln a| >= ln 2, so the hardware log2
+//                                 (__log2f, at most 2 ulp off away from 1)
+//                                 keeps t to about 2^-22 relative;
+//   upper half:  t = -ln(1 - a) = 2 atanh(w) = 2 (w + w^3/3 + w^5/5 + ...),
+//                w = a / (2 - a) in (0, 1/3]: seven terms leave a relative
+//                remainder below (1/9)^7 / 15 < 2e-8, with no cancellation
+//                however small a is;
+// and g = -ln t through __log2f again.  Both halves are evaluated and one is
+// selected, so lanes never diverge.  The error of g against the exact value
+// stays within 2 ulp(g) plus about 2^-21 absolute (the GPU test checks it
+// against the fp64 oracle over both 2^20-word tails and a stratified sample).
 #pragma once
 
 #include <stdint.h>
@@ -51,15 +59,23 @@ __device__ __forceinline__ Philox4 philox4x32_10(uint32_t c0, uint32_t c1, uint3
 
 __device__ __forceinline__ float gumbel_from_u32(uint32_t r) {
   const float kTwoPowM32 = 2.3283064365386963e-10f;  // 2^-32
-  float t;
-  if (r >= 0x80000000u) {
-    const float z = __uint2float_rn(0u - r) * kTwoPowM32;  // 1 - u, in (0, 1/2]
-    t = -log1pf(-z);
-  } else {
-    const float u = __uint2float_rn(r + 1u) * kTwoPowM32;  // u, in (0, 1/2]
-    t = -logf(u);
-  }
-  return -logf(t);
+  const float kMinusLn2 = -0.69314718055994531f;
+  const bool upper = r >= 0x80000000u;
+  const uint32_t q = upper ? (0u - r) : (r + 1u);     // in [1, 2^31]
+  const float a = __uint2float_rn(q) * kTwoPowM32;    // in (0, 1/2]
+  const float t_lower = __log2f(a) * kMinusLn2;       // -ln a
+  const float w = __fdividef(a, 2.0f - a);            // atanh argument, (0, 1/3]
+  const float w2 = w * w;
+  float p = 2.0f / 13.0f;
+  p = fmaf(p, w2, 2.0f / 11.0f);
+  p = fmaf(p, w2, 2.0f / 9.0f);
+  p = fmaf(p, w2, 2.0f / 7.0f);
+  p = fmaf(p, w2, 2.0f / 5.0f);
+  p = fmaf(p, w2, 2.0f / 3.0f);
+  p = fmaf(p, w2, 2.0f);
+  const float t_upper = w * p;                        // -ln(1 - a)
+  const float t = upper ? t_upper : t_lower;
+  return __log2f(t) * kMinusLn2;
 }
 
 }  // namespace fmms

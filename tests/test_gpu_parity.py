@@ -72,20 +72,28 @@ def gumbel_rs():
     return np.unique(np.concatenate([lo, mid, edge, hi])).astype(np.uint32)
 
 
+GUMBEL_ULPS, GUMBEL_ABS = 3.0, 1e-6
+
+
 def test_gumbel_transform_accuracy(dev, oracle):
-    """fp32 g(r) within 3 ulp(g) + 2^-22 of the fp64 value on both tails, the
-    branch boundary and a stratified sample; finite and non-decreasing in r.
-    Derivation: the fp32 inputs u or 1-u carry 2^-24 relative rounding, which
-    reaches g as at most ~1.5 * 2^-24 absolute after two logs; logf/log1pf add
-    about one ulp each, the outer log's ulp being ulp(g)."""
+    """fp32 g(r) within 3 ulp(g) + 1e-6 of the fp64 value on both 2^20-word
+    tails, the branch boundary and a stratified sample; always finite.
+    Derivation of the bound: a = q 2^-32 carries 2^-24 relative rounding; the
+    inner value t = -ln u then carries at most ~5e-7 relative error (hardware
+    log2 within 2 ulp on the lower half; a / (2 - a) with a fast division and a
+    seven-term series, remainder < 2e-8, on the upper half), which reaches g
+    as the same absolute error; the outer hardware log2 adds at most 2 ulp(g)
+    (2^-22 absolute for t in [0.5, 2]) and the final scaling half an ulp.
+    g must also rise with r up to that error."""
     r = gumbel_rs()
     ref = oracle.gumbel(r)
     got = binding.fs_gumbel(torch.from_numpy(r.view(np.int32)).to(dev)).cpu().numpy()
     assert np.all(np.isfinite(got))
     ulp = np.spacing(np.abs(ref).astype(np.float32)).astype(np.float64)
+    tol = GUMBEL_ULPS * ulp + GUMBEL_ABS
     err = np.abs(got.astype(np.float64) - ref)
-    assert np.all(err <= 3 * ulp + 2.0 ** -22), (err / ulp).max()
-    assert np.all(np.diff(got) >= 0)
+    assert np.all(err <= tol), ((err / ulp).max(), err.max())
+    assert np.all(np.diff(got.astype(np.float64)) >= -2 * tol[1:])
 
 
 # ------------------------------------------------------------ flat sampling
