@@ -9,7 +9,7 @@
 
 #include <mutex>
 
-#include "../../include/fmms.h"
+#include "fmms.h"
 #include "fmms_common.cuh"
 #include "launch.h"
 

@@ -8,7 +8,7 @@
 #include <math.h>
 #include <stdint.h>
 
-#include "../../include/fmms.h"
+#include "fmms.h"
 #include "fmms_common.cuh"
 #include "launch.h"
 #include "noise.cuh"

@@ -19,7 +19,7 @@ constexpr int kTileM = 128;   // vocabulary rows per tile (tcgen05 M)
 constexpr int kBlockK = 64;   // K elements per pipeline stage: one 128-byte swizzle row
 constexpr int kGranule = 8;   // vocabulary granule of the per-CTA split: one 8-row swizzle atom
 constexpr int kMaxBN = 256;   // batch rows per launch (tcgen05 N limit)
-constexpr int kNumEpiWarps = 8;
+constexpr int kNumEpiWarps = 16;  // four per TMEM lane quarter
 constexpr int kThreads = 32 * (2 + kNumEpiWarps);  // TMA warp + MMA warp + epilogue
 constexpr int kEpiThreads = 32 * kNumEpiWarps;
 

@@ -48,16 +48,19 @@ struct KCfg {
   static constexpr int kStageBytes = kStageW + kStageH;
   static constexpr int kStagesFit = 196608 / kStageBytes;
   static constexpr int kStages = kStagesFit < 10 ? kStagesFit : 10;
-  static constexpr int kCW = BN >= 64 ? 32 : 16;        // columns per epilogue chunk
+  static constexpr int kCW = 16;                        // columns per epilogue chunk
   static constexpr int kChunks = BN / kCW;
-  static constexpr int kChunksPerHalf = kChunks >= 2 ? kChunks / 2 : 1;
-  static constexpr int kTmemCols = 2 * BN < 32 ? 32 : 2 * BN;  // two accumulators
+  static constexpr int kWarpsPerQuarter = kNumEpiWarps / 4;
+  static constexpr int kChunksPerWarp = kChunks >= kWarpsPerQuarter ? kChunks / kWarpsPerQuarter : 1;
+  static constexpr int kAccBufs = BN <= 128 ? 4 : 2;     // accumulators in flight
+  static constexpr int kTmemCols = kAccBufs * BN < 32 ? 32 : kAccBufs * BN;
   static constexpr uint32_t kIdesc = sm100::idesc_bf16_f32(kTileM, BN);
   static constexpr int kBarBytes = 256;
   static constexpr int kCombBytes = 4 * BN * 16;
   static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBarBytes + kCombBytes;
   static_assert(kStageH % 1024 == 0, "H stage must keep 1024-byte atom alignment");
-  static_assert((2 * kStages + 5) * 8 + 16 <= kBarBytes, "barrier area too small");
+  static_assert((2 * kStages + 2 * kAccBufs + 1) * 8 + 16 <= kBarBytes, "barrier area too small");
+  static_assert(kTmemCols <= 512, "tensor memory holds 512 columns");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
@@ -302,8 +305,10 @@ __device__ __forceinline__ void role_mma(const FmmsParams &p, const Schedule &sc
     }
     if (!ok) break;
     sm100::mma_commit(&acc_full[buf]);   // accumulator ready for the epilogue
-    buf ^= 1;
-    if (buf == 0) acc_phase ^= 1u;
+    if (++buf == C::kAccBufs) {
+      buf = 0;
+      acc_phase ^= 1u;
+    }
   }
   // Drain: every MMA issued above has completed once this arrives.
   sm100::mma_commit(drain_bar);
@@ -321,13 +326,14 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
   using C = KCfg<BN>;
   constexpr int CW = C::kCW;
   const int q = warp & 3;          // TMEM lane quarter this warp may access
-  const int h = (warp - 2) >> 2;   // which half of the column chunks
+  const int h = (warp - 2) >> 2;   // which of the quarter's warps: chunks h, h+4, ...
   const int etid = (warp - 2) * 32 + lane;
+  const bool has_chunks = h < C::kChunks;
 
-  uint64_t best[C::kChunksPerHalf];
-  float m_run[C::kChunksPerHalf], s_run[C::kChunksPerHalf];
+  uint64_t best[C::kChunksPerWarp];
+  float m_run[C::kChunksPerWarp], s_run[C::kChunksPerWarp];
 #pragma unroll
-  for (int i = 0; i < C::kChunksPerHalf; ++i) {
+  for (int i = 0; i < C::kChunksPerWarp; ++i) {
     best[i] = 0ull;
     m_run[i] = -INFINITY;
     s_run[i] = 0.f;
@@ -352,9 +358,9 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
       const uint32_t tbase =
           tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(buf * BN);
 #pragma unroll
-      for (int kk = 0; kk < C::kChunksPerHalf; ++kk) {
-        if (C::kChunks < 2 && h == 1) continue;
-        const int k = C::kChunks >= 2 ? 2 * kk + h : kk;
+      for (int kk = 0; kk < C::kChunksPerWarp; ++kk) {
+        if (!has_chunks) continue;
+        const int k = kk * C::kWarpsPerQuarter + h;
         const int col0 = k * CW;
         if (col0 >= p.B) continue;  // warp-uniform
         uint32_t acc[CW];
@@ -379,16 +385,18 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
       __syncwarp();
       if (lane == 0) sm100::mbar_arrive(&acc_empty[buf]);
     }
-    buf ^= 1;
-    if (buf == 0) phase ^= 1u;
+    if (++buf == C::kAccBufs) {
+      buf = 0;
+      phase ^= 1u;
+    }
 
     if constexpr (MODE == kModeGrouped) {
       if (tile.last) {
         // Segment done: combine the four lane quarters and write the partial.
 #pragma unroll
-        for (int kk = 0; kk < C::kChunksPerHalf; ++kk) {
-          if (C::kChunks < 2 && h == 1) continue;
-          const int k = C::kChunks >= 2 ? 2 * kk + h : kk;
+        for (int kk = 0; kk < C::kChunksPerWarp; ++kk) {
+          if (!has_chunks) continue;
+          const int k = kk * C::kWarpsPerQuarter + h;
           const int col = k * CW + column_of_lane<CW>(lane);
           if (k * CW < p.B) {
             comb_key[q * BN + col] = best[kk];
@@ -424,9 +432,9 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
 
   if constexpr (MODE == kModeFlat) {
 #pragma unroll
-    for (int kk = 0; kk < C::kChunksPerHalf; ++kk) {
-      if (C::kChunks < 2 && h == 1) continue;
-      const int k = C::kChunks >= 2 ? 2 * kk + h : kk;
+    for (int kk = 0; kk < C::kChunksPerWarp; ++kk) {
+      if (!has_chunks) continue;
+      const int k = kk * C::kWarpsPerQuarter + h;
       if (k * CW < p.B) comb_key[q * BN + k * CW + column_of_lane<CW>(lane)] = best[kk];
     }
     sm100::epi_sync(kEpiThreads);
@@ -479,8 +487,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *full = bars;
   uint64_t *empty = full + C::kStages;
   uint64_t *acc_full = empty + C::kStages;
-  uint64_t *acc_empty = acc_full + 2;
-  uint64_t *drain_bar = acc_empty + 2;
+  uint64_t *acc_empty = acc_full + C::kAccBufs;
+  uint64_t *drain_bar = acc_empty + C::kAccBufs;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain_bar + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   int *last_flag = reinterpret_cast<int *>(tmem_slot + 2);
@@ -502,7 +510,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       sm100::mbar_init(&full[s], 1);
       sm100::mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < C::kAccBufs; ++b) {
       sm100::mbar_init(&acc_full[b], 1);
       sm100::mbar_init(&acc_empty[b], kNumEpiWarps);
     }
