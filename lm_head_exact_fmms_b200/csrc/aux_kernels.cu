@@ -131,7 +131,7 @@ __global__ void __launch_bounds__(256) sample_logits_kernel(const SampleLogitsPa
     for (int m = 0; m < 4; ++m) {
       const int v = v0 + m;
       const bool ok = v < s.V && ((mword >> (v & 31)) & 1u);
-      const float sc = l[m] * s.inv_temp + gumbel_from_u32(w[m]);
+      const float sc = fmaf(l[m], s.inv_temp, gumbel_from_u32(w[m]));  // as the fused kernel
       const uint64_t k = ok ? pack_key(__float_as_uint(sc), v) : 0ull;
       best = k > best ? k : best;
     }

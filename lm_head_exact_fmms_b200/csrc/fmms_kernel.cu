@@ -152,15 +152,12 @@ __device__ __forceinline__ void lse_merge(float &m, float &s, float m2, float s2
   m = mx;
 }
 
-// One chunk of CW columns for one tile row v (one per thread): scores,
-// transpose-reduce, fold into the lane's running best of its column.
-template <int CW, int MODE>
-__device__ __forceinline__ void epi_chunk(const uint32_t (&acc)[CW], const FmmsParams &p, int v,
-                                          bool v_ok, int col0, int lane, uint64_t &best,
-                                          float &m_run, float &s_run) {
-  uint64_t key[CW];
-  float xs[CW];
-  const uint64_t low = 0xFFFFFFFFu - static_cast<uint32_t>(v);  // token part of the key
+// Noise words of one chunk: afterwards words[j] is the word of (row col0 + j,
+// token v) for this lane's tile row v.  One Philox call per lane serves four
+// consecutive tokens of one row; the quad transpose hands each lane its word.
+template <int CW>
+__device__ __forceinline__ void chunk_noise(const FmmsParams &p, int v, int col0, int lane,
+                                            uint32_t (&words)[CW]) {
 #pragma unroll
   for (int q4 = 0; q4 < CW / 4; ++q4) {
     const int colp = col0 + 4 * q4 + (lane & 3);  // column of this lane's Philox call
@@ -172,20 +169,33 @@ __device__ __forceinline__ void epi_chunk(const uint32_t (&acc)[CW], const FmmsP
     uint32_t w[4] = {ph.w0, ph.w1, ph.w2, ph.w3};
     quad_transpose(w, lane);
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const int j = 4 * q4 + m;
-      const int col = col0 + j;
-      bool ok = v_ok && col < p.B;
-      if (ok && p.mask != nullptr) {
-        const uint32_t word =
-            __ldg(p.mask + static_cast<size_t>(p.b_off + col) * p.mask_words + (v >> 5));
-        ok = ((word >> (v & 31)) & 1u) != 0;
-      }
-      const float s = fmaf(__uint_as_float(acc[j]), p.inv_temp, gumbel_from_u32(w[m]));
-      const uint32_t hi = ok ? order_bits(__float_as_uint(s)) : 0u;
-      key[j] = (static_cast<uint64_t>(hi) << 32) | low;
-      if (MODE == kModeGrouped) xs[j] = ok ? __uint_as_float(acc[j]) * p.inv_temp : -INFINITY;
+    for (int m = 0; m < 4; ++m) words[4 * q4 + m] = w[m];
+  }
+}
+
+// Exact scores of one chunk: mask, s = x + g, packed keys, transpose-reduce,
+// fold into the lane's running best of its column (and, grouped, the
+// running log-sum-exp pieces of the allowed x).
+template <int CW, int MODE>
+__device__ __forceinline__ void chunk_exact(const uint32_t (&acc)[CW], const uint32_t (&words)[CW],
+                                            const FmmsParams &p, int v, bool v_ok, int col0,
+                                            int lane, uint64_t &best, float &m_run, float &s_run) {
+  uint64_t key[CW];
+  float xs[CW];
+  const uint64_t low = 0xFFFFFFFFu - static_cast<uint32_t>(v);  // token part of the key
+#pragma unroll
+  for (int j = 0; j < CW; ++j) {
+    const int col = col0 + j;
+    bool ok = v_ok && col < p.B;
+    if (ok && p.mask != nullptr) {
+      const uint32_t word =
+          __ldg(p.mask + static_cast<size_t>(p.b_off + col) * p.mask_words + (v >> 5));
+      ok = ((word >> (v & 31)) & 1u) != 0;
     }
+    const float s = fmaf(__uint_as_float(acc[j]), p.inv_temp, gumbel_from_u32(words[j]));
+    const uint32_t hi = ok ? order_bits(__float_as_uint(s)) : 0u;
+    key[j] = (static_cast<uint64_t>(hi) << 32) | low;
+    if (MODE == kModeGrouped) xs[j] = ok ? __uint_as_float(acc[j]) * p.inv_temp : -INFINITY;
   }
   const uint64_t cmax = transpose_reduce<CW, OpMaxU64>(key, lane);
   best = cmax > best ? cmax : best;
@@ -203,6 +213,39 @@ __device__ __forceinline__ void epi_chunk(const uint32_t (&acc)[CW], const FmmsP
     const float colsum = transpose_reduce<CW, OpAddF>(e, lane);
     lse_merge(m_run, s_run, colmax, colsum);
   }
+}
+
+// Flat mode: skip the exact scores of a chunk when no element can reach its
+// row's threshold.  The threshold of a row is the score of an element already
+// computed exactly (the best this lane's column has seen, or the best any CTA
+// has published to the workspace keys), so an element whose upper bound
+// x + gumbel_upper_bound(r) is below it can be neither the maximum nor tied
+// with it: the sampled tokens are the same as without the filter.  Returns
+// true when the exact path ran.
+template <int CW>
+__device__ __forceinline__ bool chunk_filtered(const uint32_t (&acc)[CW], const FmmsParams &p,
+                                               int v, bool v_ok, int col0, int lane,
+                                               uint64_t &best) {
+  const int c = col0 + column_of_lane<CW>(lane);
+  uint64_t k = best;
+  if (c < p.B) {
+    const uint64_t g = __ldcg(reinterpret_cast<const unsigned long long *>(p.keys + c));
+    k = g > k ? g : k;
+  }
+  const float t_col = key_valid(k) ? __uint_as_float(key_score_bits(k)) : -INFINITY;
+  uint32_t words[CW];
+  chunk_noise<CW>(p, v, col0, lane, words);
+  bool cand = false;
+#pragma unroll
+  for (int j = 0; j < CW; ++j) {
+    const float thr = __shfl_sync(0xffffffffu, t_col, lane_of_column<CW>(j));
+    const float ub = fmaf(__uint_as_float(acc[j]), p.inv_temp, gumbel_upper_bound(words[j]));
+    cand = cand || (v_ok && col0 + j < p.B && ub >= thr);
+  }
+  if (!__any_sync(0xffffffffu, cand)) return false;
+  float m_unused = -INFINITY, s_unused = 0.f;
+  chunk_exact<CW, kModeFlat>(acc, words, p, v, v_ok, col0, lane, best, m_unused, s_unused);
+  return true;
 }
 
 // ---------------------------------------------------------------------------
@@ -378,7 +421,19 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
                 p.logits[static_cast<size_t>(col0 + j) * p.V + v] = __uint_as_float(acc[j]);
           }
         } else {
-          epi_chunk<CW, MODE>(acc, p, v, v_ok, col0, lane, best[kk], m_run[kk], s_run[kk]);
+          if constexpr (MODE == kModeFlat) {
+            if (chunk_filtered<CW>(acc, p, v, v_ok, col0, lane, best[kk])) {
+              // publish the improved maximum so every CTA's filter sharpens
+              const int c = col0 + column_of_lane<CW>(lane);
+              if ((lane & 1) == 0 && c < p.B && key_valid(best[kk]))
+                atomicMax(p.keys + c, static_cast<unsigned long long>(best[kk]));
+            }
+          } else {
+            uint32_t words[CW];
+            chunk_noise<CW>(p, v, col0, lane, words);
+            chunk_exact<CW, MODE>(acc, words, p, v, v_ok, col0, lane, best[kk], m_run[kk],
+                                  s_run[kk]);
+          }
         }
       }
       sm100::tc_fence_before();

@@ -78,4 +78,22 @@ __device__ __forceinline__ float gumbel_from_u32(uint32_t r) {
   return __log2f(t) * kMinusLn2;
 }
 
+// A cheap upper bound of gumbel_from_u32(r), with no logarithm, for the
+// epilogue's filter.  Lower half (u < 1/2): t = -ln u > ln 2, so
+// g < -ln(ln 2) = 0.36651.  Upper half: with z = 1 - u = q / (2^32 + 1),
+// q = 2^32 - r, t = -ln(1 - z) >= z gives g <= -ln z <= 32 ln 2 - ln q, and
+// log2 q >= e + m for q = 2^e (1 + m) (log2(1 + m) >= m on [0, 1]); the
+// float bits of q hold e + m as bits / 2^23 - 127, so
+//   g <= ln 2 * (159 - bits(float(q)) / 2^23).
+// The constant 1e-4 covers the fp32 rounding of this expression (< 2e-5) and
+// the error of gumbel_from_u32 itself (< 3 ulp + 1e-6), so the bound holds
+// for the computed value, not only the exact one.
+__device__ __forceinline__ float gumbel_upper_bound(uint32_t r) {
+  const float kSlope = -0.69314718055994531f * 1.1920928955078125e-07f;  // -ln2 / 2^23
+  const float kOffset = 0.69314718055994531f * 159.0f + 1e-4f;
+  const float fq = __uint2float_rn(0u - r);
+  const float upper = fmaf(__uint2float_rn(__float_as_uint(fq)), kSlope, kOffset);
+  return r >= 0x80000000u ? upper : 0.36661f;
+}
+
 }  // namespace fmms
