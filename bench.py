@@ -342,8 +342,8 @@ def run_gpu(args, world, rank, local):
 
     if rank == 0 and not args.no_sweep:
         result["sweep"] = sweep(torch, binding, synth, W, wl, dev, stream, peaks, peak_kind)
-        result["grouped_masked"] = grouped_point(torch, binding, synth, dev, stream, peaks,
-                                                 peak_kind, W)
+        result["grouped_masked"] = grouped_points(torch, binding, synth, dev, stream, peaks,
+                                                  peak_kind, W)
         result["unfused"] = unfused_point(torch, binding, synth, W, wl, dev, stream, B)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(H, W, wl, B, rs)
@@ -372,25 +372,30 @@ def sweep(torch, binding, synth, W, wl, dev, stream, peaks, peak_kind, steps=200
     return rows
 
 
-def grouped_point(torch, binding, synth, dev, stream, peaks, peak_kind, W8, B=64, steps=100):
+def grouped_points(torch, binding, synth, dev, stream, peaks, peak_kind, W8, steps=100):
+    """The grouped + masked workload at each of its batch sizes."""
     wl = synth.WORKLOADS["grouped-masked"]
-    H = synth.make_hidden(B, wl.d, device=dev)
-    mask = synth.make_mask(B, wl.V, wl.mask_allowed).to(dev)
-    out = torch.empty(B, dtype=torch.int32, device=dev)
     W = W8 if (W8.shape[0] == wl.V and W8.shape[1] == wl.d) else \
         synth.make_weight(wl.V, wl.d, wl.w_std, device=dev)
+    rows = []
+    for B in wl.batches:
+        H = synth.make_hidden(B, wl.d, device=dev)
+        mask = synth.make_mask(B, wl.V, wl.mask_allowed).to(dev)
+        out = torch.empty(B, dtype=torch.int32, device=dev)
 
-    def step(i):
-        binding.fs_sample_grouped(H, W, wl.groups, temperature=wl.temperature, seed=0, step=i,
-                                  mask_bits=mask, out_idx=out, stream=stream)
+        def step(i):
+            binding.fs_sample_grouped(H, W, wl.groups, temperature=wl.temperature, seed=0, step=i,
+                                      mask_bits=mask, out_idx=out, stream=stream)
 
-    region_ms, per = time_calls(step, steps, 10, stream)
-    us = region_ms * 1e3 / steps
-    rf = roofline(B, wl.d, wl.V, True, us, peaks, peak_kind, None)
-    return {"workload": "grouped-masked d=%d V=%d G=%d B=%d 50%% mask T=%g (2 kernels per call)"
-                        % (wl.d, wl.V, wl.groups, B, wl.temperature),
-            "us_per_call": round(us, 3), "bound": rf["bound"], "achieved": round(rf["achieved"], 1),
-            "unit": rf["unit"], "frac": round(rf["frac"], 4)}
+        region_ms, _ = time_calls(step, steps, 10, stream)
+        us = region_ms * 1e3 / steps
+        rf = roofline(B, wl.d, wl.V, True, us, peaks, peak_kind, None)
+        rows.append({"B": B, "us_per_call": round(us, 3), "bound": rf["bound"],
+                     "achieved": round(rf["achieved"], 1), "unit": rf["unit"],
+                     "frac": round(rf["frac"], 4),
+                     "launches_per_call": 2 * ((B + 255) // 256)})
+    return {"workload": "grouped-masked d=%d V=%d G=%d, 50%% mask, T=%g (fused kernel + merge)"
+                        % (wl.d, wl.V, wl.groups, wl.temperature), "points": rows}
 
 
 def unfused_point(torch, binding, synth, W, wl, dev, stream, B, steps=100):

@@ -152,15 +152,20 @@ struct Workspace {
   unsigned int *ticket;
   unsigned long long *keys;
   fmms::GroupPartial *partials;
+  unsigned long long *gkeys;
 };
 
-Workspace carve(void *ws) {
+Workspace carve(void *ws, int B, int G, int num_ctas) {
   char *b = static_cast<char *>(ws);
   Workspace w;
   w.err = reinterpret_cast<int *>(b);
   w.ticket = reinterpret_cast<unsigned int *>(b + 4);
   w.keys = reinterpret_cast<unsigned long long *>(b + fmms::kWsHeader);
   w.partials = reinterpret_cast<fmms::GroupPartial *>(b + fmms::kWsHeader + fmms::kWsKeys);
+  w.gkeys = fmms::ws_gkeys_bytes(B, G) > 0
+                ? reinterpret_cast<unsigned long long *>(
+                      b + fmms::kWsHeader + fmms::kWsKeys + fmms::ws_partials_bytes(B, G, num_ctas))
+                : nullptr;
   return w;
 }
 
@@ -191,7 +196,7 @@ fs_status run(int mode, const void *H, const void *W, int B, int d, int V, int G
   void *wsp = nullptr;
   s = resolve_workspace(st, sch, B, ws, ws_bytes, &wsp);
   if (s != FS_OK) return s;
-  const Workspace w = carve(wsp);
+  const Workspace w = carve(wsp, B, sch.G, sch.num_ctas);
 
   CUtensorMap tw, tw8;
   if ((s = tensor_map(&tw, W, d, V, fmms::kTileM)) != FS_OK) return s;
@@ -223,12 +228,14 @@ fs_status run(int mode, const void *H, const void *W, int B, int d, int V, int G
     p.ticket = w.ticket;
     p.err = w.err;
     p.partials = w.partials;
+    p.gkeys = mode == fmms::kModeGrouped ? w.gkeys : nullptr;
     p.logits = logits ? logits + static_cast<size_t>(b0) * V : nullptr;
     if (fmms::launch_fmms(mode, BN, tw, tw8, th, p, stream) != cudaSuccess) return FS_ERR_CUDA;
 
     if (mode == fmms::kModeGrouped) {
       fmms::MergeParams m;
       m.partials = w.partials;
+      m.gkeys = w.gkeys;
       m.B = Bc;
       m.b_off = b0;
       m.V = V;

@@ -55,6 +55,7 @@ __global__ void __launch_bounds__(128) group_merge_kernel(const MergeParams m) {
         }
       }
     }
+    if (m.gkeys != nullptr) m.gkeys[static_cast<size_t>(g) * m.B + b] = 0ull;  // left zeroed
     const float lse = (M == -INFINITY) ? -INFINITY : M + logf(S);
     if (summary != nullptr) {
       fs_group_summary gs;

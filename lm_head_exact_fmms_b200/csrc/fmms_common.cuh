@@ -170,20 +170,31 @@ struct FmmsParams {
   unsigned int *ticket;        // workspace: CTAs finished (flat)
   int *err;                    // workspace: device status word
   GroupPartial *partials;      // workspace [slots][B] (grouped)
+  unsigned long long *gkeys;   // workspace [G][B] published per-group maxima, or null
   float *logits;               // [B][V] (logits mode; already offset)
 };
 
 // Workspace layout (bytes): [0, 256) status word and ticket; [256, 256 + 2048)
-// packed keys of up to 256 rows; then grouped partials [slots][256].
+// packed keys of up to 256 rows; then, grouped, the partials [slots][rows]
+// and, for G <= kMaxPublishedGroups, the published per-group maxima
+// [G][rows] that sharpen the exact-score filter (re-zeroed by the merge).
 constexpr int kWsHeader = 256;
 constexpr int kWsKeys = 8 * kMaxBN;
+constexpr int kMaxPublishedGroups = 4096;
+
+FS_HD int64_t ws_partials_bytes(int B, int G, int num_ctas) {
+  const int64_t rows = B < kMaxBN ? B : kMaxBN;
+  return G > 1 ? (int64_t)(num_ctas + G - 1) * rows * (int64_t)sizeof(GroupPartial) : 0;
+}
+
+FS_HD int64_t ws_gkeys_bytes(int B, int G) {
+  const int64_t rows = B < kMaxBN ? B : kMaxBN;
+  return (G > 1 && G <= kMaxPublishedGroups) ? (int64_t)G * rows * 8 : 0;
+}
 
 FS_HD int64_t workspace_bytes_for(int B, int G, int num_ctas) {
-  int64_t bytes = kWsHeader + kWsKeys;
-  if (G > 1) {
-    int64_t rows = B < kMaxBN ? B : kMaxBN;
-    bytes += (int64_t)(num_ctas + G - 1) * rows * (int64_t)sizeof(GroupPartial);
-  }
+  const int64_t bytes =
+      kWsHeader + kWsKeys + ws_partials_bytes(B, G, num_ctas) + ws_gkeys_bytes(B, G);
   return (bytes + 255) / 256 * 256;
 }
 

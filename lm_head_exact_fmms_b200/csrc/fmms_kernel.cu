@@ -152,6 +152,11 @@ __device__ __forceinline__ void lse_merge(float &m, float &s, float m2, float s2
   m = mx;
 }
 
+// Reads a published key from global memory, bypassing L1 (other CTAs update it).
+__device__ __forceinline__ uint64_t ld_key(const unsigned long long *ptr) {
+  return __ldcg(ptr);
+}
+
 // Noise words of one chunk: afterwards words[j] is the word of (row col0 + j,
 // token v) for this lane's tile row v.  One Philox call per lane serves four
 // consecutive tokens of one row; the quad transpose hands each lane its word.
@@ -173,16 +178,12 @@ __device__ __forceinline__ void chunk_noise(const FmmsParams &p, int v, int col0
   }
 }
 
-// Exact scores of one chunk: mask, s = x + g, packed keys, transpose-reduce,
-// fold into the lane's running best of its column (and, grouped, the
-// running log-sum-exp pieces of the allowed x).
-template <int CW, int MODE>
-__device__ __forceinline__ void chunk_exact(const uint32_t (&acc)[CW], const uint32_t (&words)[CW],
-                                            const FmmsParams &p, int v, bool v_ok, int col0,
-                                            int lane, uint64_t &best, float &m_run, float &s_run) {
-  uint64_t key[CW];
-  float xs[CW];
-  const uint64_t low = 0xFFFFFFFFu - static_cast<uint32_t>(v);  // token part of the key
+// Bit j set when (row col0 + j, token v) is in range and, with a mask,
+// allowed for that row.
+template <int CW>
+__device__ __forceinline__ uint32_t chunk_allowed(const FmmsParams &p, int v, bool v_ok,
+                                                  int col0) {
+  uint32_t bits = 0;
 #pragma unroll
   for (int j = 0; j < CW; ++j) {
     const int col = col0 + j;
@@ -192,60 +193,80 @@ __device__ __forceinline__ void chunk_exact(const uint32_t (&acc)[CW], const uin
           __ldg(p.mask + static_cast<size_t>(p.b_off + col) * p.mask_words + (v >> 5));
       ok = ((word >> (v & 31)) & 1u) != 0;
     }
+    bits |= (ok ? 1u : 0u) << j;
+  }
+  return bits;
+}
+
+// Bit j set when (row col0 + j, token v) is in range, mask not consulted.
+template <int CW>
+__device__ __forceinline__ uint32_t chunk_in_range(const FmmsParams &p, bool v_ok, int col0) {
+  if (!v_ok) return 0u;
+  const int n = p.B - col0;
+  return n >= CW ? ((1u << CW) - 1u) : ((1u << n) - 1u);
+}
+
+// Exact scores s = x + g of the allowed elements as packed keys,
+// transpose-reduced into the lane's running best of its column.
+template <int CW>
+__device__ __forceinline__ void chunk_keys(const uint32_t (&acc)[CW], const uint32_t (&words)[CW],
+                                           const FmmsParams &p, int v, uint32_t allowed, int lane,
+                                           uint64_t &best) {
+  uint64_t key[CW];
+  const uint64_t low = 0xFFFFFFFFu - static_cast<uint32_t>(v);  // token part of the key
+#pragma unroll
+  for (int j = 0; j < CW; ++j) {
     const float s = fmaf(__uint_as_float(acc[j]), p.inv_temp, gumbel_from_u32(words[j]));
-    const uint32_t hi = ok ? order_bits(__float_as_uint(s)) : 0u;
+    const uint32_t hi = ((allowed >> j) & 1u) ? order_bits(__float_as_uint(s)) : 0u;
     key[j] = (static_cast<uint64_t>(hi) << 32) | low;
-    if (MODE == kModeGrouped) xs[j] = ok ? __uint_as_float(acc[j]) * p.inv_temp : -INFINITY;
   }
   const uint64_t cmax = transpose_reduce<CW, OpMaxU64>(key, lane);
   best = cmax > best ? cmax : best;
-  if (MODE == kModeGrouped) {
-    float t[CW];
-#pragma unroll
-    for (int j = 0; j < CW; ++j) t[j] = xs[j];
-    const float colmax = transpose_reduce<CW, OpMaxF>(t, lane);
-    float e[CW];
-#pragma unroll
-    for (int j = 0; j < CW; ++j) {
-      const float cm = __shfl_sync(0xffffffffu, colmax, lane_of_column<CW>(j));
-      e[j] = (xs[j] == -INFINITY) ? 0.f : __expf(xs[j] - cm);
-    }
-    const float colsum = transpose_reduce<CW, OpAddF>(e, lane);
-    lse_merge(m_run, s_run, colmax, colsum);
-  }
 }
 
-// Flat mode: skip the exact scores of a chunk when no element can reach its
-// row's threshold.  The threshold of a row is the score of an element already
-// computed exactly (the best this lane's column has seen, or the best any CTA
-// has published to the workspace keys), so an element whose upper bound
-// x + gumbel_upper_bound(r) is below it can be neither the maximum nor tied
-// with it: the sampled tokens are the same as without the filter.  Returns
-// true when the exact path ran.
+// Log-sum-exp pieces of the allowed x = acc / T of one chunk, folded into the
+// lane's running (m, s) of its column.
 template <int CW>
-__device__ __forceinline__ bool chunk_filtered(const uint32_t (&acc)[CW], const FmmsParams &p,
-                                               int v, bool v_ok, int col0, int lane,
-                                               uint64_t &best) {
-  const int c = col0 + column_of_lane<CW>(lane);
-  uint64_t k = best;
-  if (c < p.B) {
-    const uint64_t g = __ldcg(reinterpret_cast<const unsigned long long *>(p.keys + c));
-    k = g > k ? g : k;
+__device__ __forceinline__ void chunk_lse(const uint32_t (&acc)[CW], const FmmsParams &p,
+                                          uint32_t allowed, int lane, float &m_run, float &s_run) {
+  float xs[CW], t[CW];
+#pragma unroll
+  for (int j = 0; j < CW; ++j) {
+    xs[j] = ((allowed >> j) & 1u) ? __uint_as_float(acc[j]) * p.inv_temp : -INFINITY;
+    t[j] = xs[j];
   }
+  const float colmax = transpose_reduce<CW, OpMaxF>(t, lane);
+  float e[CW];
+#pragma unroll
+  for (int j = 0; j < CW; ++j) {
+    const float cm = __shfl_sync(0xffffffffu, colmax, lane_of_column<CW>(j));
+    e[j] = (xs[j] == -INFINITY) ? 0.f : __expf(xs[j] - cm);
+  }
+  const float colsum = transpose_reduce<CW, OpAddF>(e, lane);
+  lse_merge(m_run, s_run, colmax, colsum);
+}
+
+// The filter: may any element of the chunk (bit set in `cand`) reach its
+// column's threshold?  The threshold of a column is the score of an element
+// already computed exactly (the lane's own best, or the best any CTA has
+// published for this row), so an element whose upper bound
+// x + gumbel_upper_bound(r) is below it can be neither the maximum nor tied
+// with it: skipping its exact score leaves the sampled token unchanged.
+template <int CW>
+__device__ __forceinline__ bool chunk_any_candidate(const uint32_t (&acc)[CW],
+                                                    const uint32_t (&words)[CW],
+                                                    const FmmsParams &p, uint32_t cand,
+                                                    uint64_t best, uint64_t published, int lane) {
+  const uint64_t k = published > best ? published : best;
   const float t_col = key_valid(k) ? __uint_as_float(key_score_bits(k)) : -INFINITY;
-  uint32_t words[CW];
-  chunk_noise<CW>(p, v, col0, lane, words);
-  bool cand = false;
+  bool any = false;
 #pragma unroll
   for (int j = 0; j < CW; ++j) {
     const float thr = __shfl_sync(0xffffffffu, t_col, lane_of_column<CW>(j));
     const float ub = fmaf(__uint_as_float(acc[j]), p.inv_temp, gumbel_upper_bound(words[j]));
-    cand = cand || (v_ok && col0 + j < p.B && ub >= thr);
+    any = any || (((cand >> j) & 1u) && ub >= thr);
   }
-  if (!__any_sync(0xffffffffu, cand)) return false;
-  float m_unused = -INFINITY, s_unused = 0.f;
-  chunk_exact<CW, kModeFlat>(acc, words, p, v, v_ok, col0, lane, best, m_unused, s_unused);
-  return true;
+  return __any_sync(0xffffffffu, any);
 }
 
 // ---------------------------------------------------------------------------
@@ -421,18 +442,35 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
                 p.logits[static_cast<size_t>(col0 + j) * p.V + v] = __uint_as_float(acc[j]);
           }
         } else {
+          const int c = col0 + column_of_lane<CW>(lane);  // this lane's column
           if constexpr (MODE == kModeFlat) {
-            if (chunk_filtered<CW>(acc, p, v, v_ok, col0, lane, best[kk])) {
+            // The mask is consulted only on the exact path.
+            const uint64_t pub = c < p.B ? ld_key(p.keys + c) : 0ull;  // in flight during Philox
+            uint32_t words[CW];
+            chunk_noise<CW>(p, v, col0, lane, words);
+            if (chunk_any_candidate<CW>(acc, words, p, chunk_in_range<CW>(p, v_ok, col0),
+                                        best[kk], pub, lane)) {
+              chunk_keys<CW>(acc, words, p, v, chunk_allowed<CW>(p, v, v_ok, col0), lane,
+                             best[kk]);
               // publish the improved maximum so every CTA's filter sharpens
-              const int c = col0 + column_of_lane<CW>(lane);
-              if ((lane & 1) == 0 && c < p.B && key_valid(best[kk]))
+              if ((lane & 1) == 0 && c < p.B && key_valid(best[kk]) && best[kk] > pub)
                 atomicMax(p.keys + c, static_cast<unsigned long long>(best[kk]));
             }
           } else {
+            unsigned long long *gk =
+                p.gkeys ? p.gkeys + static_cast<size_t>(tile.slot - blockIdx.x) * p.B + c
+                        : nullptr;
+            const uint64_t pub = (gk != nullptr && c < p.B) ? ld_key(gk) : 0ull;
+            const uint32_t allowed = chunk_allowed<CW>(p, v, v_ok, col0);
             uint32_t words[CW];
             chunk_noise<CW>(p, v, col0, lane, words);
-            chunk_exact<CW, MODE>(acc, words, p, v, v_ok, col0, lane, best[kk], m_run[kk],
-                                  s_run[kk]);
+            chunk_lse<CW>(acc, p, allowed, lane, m_run[kk], s_run[kk]);
+            if (chunk_any_candidate<CW>(acc, words, p, allowed, best[kk], pub, lane)) {
+              chunk_keys<CW>(acc, words, p, v, allowed, lane, best[kk]);
+              if (gk != nullptr && (lane & 1) == 0 && c < p.B && key_valid(best[kk]) &&
+                  best[kk] > pub)
+                atomicMax(gk, static_cast<unsigned long long>(best[kk]));
+            }
           }
         }
       }

@@ -20,6 +20,7 @@ cudaError_t launch_fmms(int mode, int BN, const CUtensorMap &tw, const CUtensorM
 // Group-Gumbel-Max merge of the grouped partials of one launch (B rows).
 struct MergeParams {
   const GroupPartial *partials;  // [num_ctas + G - 1][B]
+  unsigned long long *gkeys;     // [G][B] published maxima to re-zero, or null
   int B, b_off, V, G, num_ctas, ngran;
   uint64_t seed;
   const uint64_t *row_seeds;
