@@ -43,6 +43,9 @@ def parse_args():
     ap.add_argument("--impl", default="fmms", choices=["fmms", "reference"])
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tp", action="store_true",
+                    help="split the vocabulary across the ranks (one int64 MAX all-reduce of "
+                         "8 bytes per row per step) instead of running independent replicas")
     return ap.parse_args()
 
 
@@ -215,10 +218,14 @@ def roofline(B, d, V, masked, kernel_us, peaks, peak_kind, traffic):
 
 
 # ------------------------------------------------------------ the GPU arm
-def time_calls(fn, steps, warmup, stream, world=1, sampler=None):
+def time_calls(fn, steps, warmup, stream, world=1, sampler=None, cooldown_s=1.0):
     """Times exactly `steps` calls after `warmup` untimed ones.  Returns
-    (region ms, per-call event durations in us)."""
+    (region ms, per-call event durations in us).  A short idle period first
+    lets the clocks recover from the power limit a previous heavy section may
+    have left them at."""
     import torch
+    torch.cuda.synchronize()
+    time.sleep(cooldown_s)
     for i in range(warmup):
         fn(i)
     torch.cuda.synchronize()
@@ -291,10 +298,26 @@ def run_gpu(args, world, rank, local):
     rs = synth.make_row_seeds(B, device=dev) if wl.per_row_seeds else None
     out = torch.empty(B, dtype=torch.int32, device=dev)
     ws = torch.zeros(binding.fs_workspace_bytes(B, wl.V, 0), dtype=torch.uint8, device=dev)
+    tp = args.tp and world > 1
+    if tp:
+        from lm_head_exact_fmms_b200 import tp as tpmod
+        lo, hi = tpmod.shard_bounds(wl.V, world)[rank]
+        W_full = W
+        W = W_full[lo:hi].contiguous()
+        del W_full
+        torch.cuda.empty_cache()
+        keys = torch.empty(B, dtype=torch.int64, device=dev)
 
-    def step(i):
-        binding.fs_sample_ex(H, W, temperature=wl.temperature, seed=0, row_seeds=rs, step=i,
-                             out_idx=out, workspace=ws, stream=stream)
+        def step(i):
+            binding.fs_sample_shard_keys(H, W, lo, wl.V, temperature=wl.temperature, seed=0,
+                                         row_seeds=rs, step=i, out_keys=keys, workspace=ws,
+                                         stream=stream)
+            tpmod.reduce_keys(keys)
+            binding.fs_keys_to_tokens(keys, out_idx=out, stream=stream)
+    else:
+        def step(i):
+            binding.fs_sample_ex(H, W, temperature=wl.temperature, seed=0, row_seeds=rs, step=i,
+                                 out_idx=out, workspace=ws, stream=stream)
 
     sampler = ClockSampler(local)
     region_ms, per_call = time_calls(step, args.steps, args.warmup, stream, world, sampler)
@@ -303,7 +326,10 @@ def run_gpu(args, world, rank, local):
     kernel_us = max_over_ranks(kernel_us, world)
     us_per_call = region_ms * 1e3 / args.steps
     nbytes, flops = algorithmic(B, wl.d, wl.V, False)
-    launches_per_call = (B + 255) // 256
+    launches_per_call = (B + 255) // 256 + (1 if tp else 0)
+    if tp:
+        # each rank streams its shard; the roofline below is per rank
+        nbytes = nbytes * W.shape[0] // wl.V
 
     # e2e: host buffers through the public C entry point (H2D + kernel + D2H).
     Hh = H.cpu().pin_memory()
@@ -313,26 +339,34 @@ def run_gpu(args, world, rank, local):
         binding.fs_sample_host(Hh, W, temperature=wl.temperature, seed=0, row_seeds=rs, step=i,
                                out_idx_host=Oh, stream=stream)
 
+    if tp:
+        # the host-buffer entry point is single-GPU: time H2D + the sharded step + D2H here
+        def step_host(i):
+            H.copy_(Hh, non_blocking=True)
+            step(i)
+            Oh.copy_(out, non_blocking=True)
     e2e_ms, _ = time_calls(step_host, args.steps, args.warmup, stream, world)
     e2e_ms = max_over_ranks(e2e_ms, world)
 
     result = {
         "metric": METRIC, "value": round(us_per_call, 3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(region_ms / args.steps, 6),
-        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": False, "scaling": "strong" if tp else "weak", "vs_baseline": None,
+        "dtype": "bf16",
         "data": "synthetic: seeded H ~ N(0,1), W ~ N(0, %g^2) bf16 (random-init %s head)"
                 % (wl.w_std, wl.name),
         "config": {"workload": "%s LM head, d=%d V=%d B=%d T=%g%s, fused fs_sample_ex"
                                % (wl.name, wl.d, wl.V, B, wl.temperature,
                                   ", per-row seeds" if wl.per_row_seeds else ""),
                    "batch_per_gpu": B, "global_batch": B * world, "d": wl.d, "V": wl.V,
-                   "parallelism": "replicas x%d" % world,
+                   "parallelism": ("tensor-parallel vocabulary x%d" % world) if tp
+                   else ("replicas x%d" % world),
                    "l2": "no flush: W (%.2f GB) exceeds the 126 MB L2" % (wl.V * wl.d * 2 / 1e9)},
         "samples_per_s": round(B * world / (us_per_call * 1e-6), 1),
         "hbm_gbs_per_gpu": round(nbytes / (us_per_call * 1e-6) / 1e9, 1),
         "kernel_us": round(kernel_us, 3),
-        "roofline": roofline(B, wl.d, wl.V, False, kernel_us, peaks, peak_kind,
-                             committed_traffic("%s/B%d" % (wl.name, B))),
+        "roofline": roofline(B, wl.d, W.shape[0], False, kernel_us, peaks, peak_kind,
+                             None if tp else committed_traffic("%s/B%d" % (wl.name, B))),
         "e2e": {"value": round(e2e_ms * 1e3 / args.steps, 3), "unit": UNIT,
                 "h2d_bytes_per_step": B * wl.d * 2, "d2h_bytes_per_step": B * 4,
                 "entry_point": "fs_sample_host (pinned host H in, host tokens out)"},

@@ -135,6 +135,34 @@ fs_status fs_sample_unfused(const void *H, const void *W, int B, int d, int V,
                             float *logits, void *workspace,
                             size_t workspace_bytes, fs_stream_t stream);
 
+/* One vocabulary shard of a tensor-parallel LM head (readus.org page,
+ * "distributed FlashSampling": each GPU is one group of the vocabulary and
+ * contributes only its winning index and score; abstract: the argmax
+ * decomposes over any partition).  W_shard holds rows
+ * [vocab_offset, vocab_offset + V_shard) of a head with V_total rows;
+ * vocab_offset must be a multiple of 8.  Noise, mask and token indices are
+ * global, so the shard's candidates are exactly those of the full head.
+ * Writes, per row, the shard's best (score, global token) as a packed key in
+ * out_keys (device int64 [B]) encoded so that the signed 64-bit maximum over
+ * shards is the full head's key: reduce with an int64 MAX all-reduce (8 bytes
+ * per row), then decode with fs_keys_to_tokens.  The result is bitwise the
+ * single-GPU fs_sample_ex result.  mask_bits, if given, covers the full
+ * vocabulary, uint32 [B][ceil(V_total/32)].  Other arguments as fs_sample_ex;
+ * a row with no allowed token in the shard gets the smallest key. */
+fs_status fs_sample_shard_keys(const void *H, const void *W_shard, int B, int d,
+                               int V_shard, int vocab_offset, int V_total,
+                               float temperature, uint64_t seed,
+                               const uint64_t *row_seeds, uint32_t step,
+                               const uint32_t *mask_bits, int64_t *out_keys,
+                               void *workspace, size_t workspace_bytes,
+                               fs_stream_t stream);
+
+/* Decodes reduced keys (device int64 [B], from fs_sample_shard_keys and a
+ * MAX reduction) into tokens out_idx (device int32 [B]); -1 where no shard
+ * had an allowed token. */
+fs_status fs_keys_to_tokens(const int64_t *keys, int B, int32_t *out_idx,
+                            fs_stream_t stream);
+
 /* End-to-end call with HOST buffers: H_host (bf16 [B, d]) and out_idx_host
  * (int32 [B]) are host pointers (page-locked for the copies to be
  * asynchronous); W and row_seeds/mask_bits stay device pointers.  Enqueues
@@ -196,6 +224,17 @@ fs_status fs_philox4x32_10(const uint32_t *ctr, const uint32_t *key,
  * function the sampling kernels use); device arrays of n elements. */
 fs_status fs_gumbel(const uint32_t *r, float *g, int64_t n,
                     fs_stream_t stream);
+
+/* Failure-detection test: launches the flat kernel on these arguments with
+ * its load-issuing warp told to issue nothing, so the MMA warp's wait for
+ * data runs out after about one second; every CTA then records
+ * FS_ERR_DEVICE_TIMEOUT in the workspace, drains, frees its tensor memory and
+ * exits, leaving the context usable.  fs_device_status() on the same
+ * workspace afterwards returns FS_ERR_DEVICE_TIMEOUT (and re-zeroes it).
+ * out_idx is left unwritten.  Same argument rules as fs_sample_ex. */
+fs_status fs_test_stalled_sample(const void *H, const void *W, int B, int d,
+                                 int V, int32_t *out_idx, void *workspace,
+                                 size_t workspace_bytes, fs_stream_t stream);
 
 /* ---- Host-only schedule query (no GPU needed) ---- */
 

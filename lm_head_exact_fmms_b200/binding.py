@@ -21,7 +21,8 @@ _STATUS = {0: "FS_OK", 1: "FS_ERR_INVALID_ARG", 2: "FS_ERR_UNSUPPORTED", 3: "FS_
 EXPORTED = ("fs_sample", "fs_sample_ex", "fs_sample_grouped", "fs_sample_unfused",
             "fs_sample_host", "fs_workspace_bytes", "fs_device_status", "fs_status_string",
             "fs_philox4x32_10", "fs_gumbel", "fs_plan_tiles", "fs_plan_group_ctas",
-            "fs_sample_noalloc")
+            "fs_sample_noalloc", "fs_test_stalled_sample", "fs_sample_shard_keys",
+            "fs_keys_to_tokens")
 
 
 class FmmsError(RuntimeError):
@@ -59,6 +60,9 @@ def load_library():
     lib.fs_sample_unfused.argtypes = common + [f32, u64, vp, u32, vp, vp, vp, vp, sz, vp]
     lib.fs_sample_host.argtypes = common + [f32, u64, vp, u32, vp, vp, vp]
     lib.fs_sample_noalloc.argtypes = common + [f32, u64, vp, u32, vp, vp, vp]
+    lib.fs_test_stalled_sample.argtypes = common + [vp, vp, sz, vp]
+    lib.fs_sample_shard_keys.argtypes = common + [i32, i32, f32, u64, vp, u32, vp, vp, vp, sz, vp]
+    lib.fs_keys_to_tokens.argtypes = [vp, i32, vp, vp]
     lib.fs_workspace_bytes.argtypes = [i32, i32, i32]
     lib.fs_workspace_bytes.restype = sz
     lib.fs_device_status.argtypes = [vp, sz, vp]
@@ -289,4 +293,47 @@ def fs_sample_noalloc(H, W, temperature=1.0, seed=0, row_seeds=None, step=0, mas
     _check(lib.fs_sample_noalloc(_ptr(H), _ptr(W), B, d, V, float(temperature), _seed(seed),
                                  _ptr(row_seeds), int(step), _ptr(mask_bits), _ptr(out_idx),
                                  _stream(stream)), "fs_sample_noalloc")
+    return out_idx
+
+
+def fs_test_stalled_sample(H, W, workspace, out_idx=None, stream=None):
+    """Failure-detection test hook: launches a sampling kernel whose waits run
+    out (about one second); the workspace then holds FS_ERR_DEVICE_TIMEOUT."""
+    lib = load_library()
+    B, d, V = _check_operands(H, W)
+    out_idx = _out(out_idx, B, H.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib.fs_test_stalled_sample(_ptr(H), _ptr(W), B, d, V, _ptr(out_idx), _ptr(workspace),
+                                      ws_bytes, _stream(stream)), "fs_test_stalled_sample")
+    return out_idx
+
+
+def fs_sample_shard_keys(H, W_shard, vocab_offset, V_total, temperature=1.0, seed=0,
+                         row_seeds=None, step=0, mask_bits=None, out_keys=None, workspace=None,
+                         stream=None):
+    """Packed (score, global token) keys [B] int64 of one vocabulary shard;
+    their int64 maximum over shards is the full head's key."""
+    lib = load_library()
+    B, d, Vs = _check_operands(H, W_shard)
+    row_seeds = _opt_dev(row_seeds, torch.int64, B, "row_seeds", H.device)
+    mask_bits = _opt_dev(mask_bits, torch.int32, B * ((V_total + 31) // 32), "mask_bits",
+                         H.device)
+    if out_keys is None:
+        out_keys = torch.empty(B, dtype=torch.int64, device=H.device)
+    _opt_dev(out_keys, torch.int64, B, "out_keys", H.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.fs_sample_shard_keys(_ptr(H), _ptr(W_shard), B, d, Vs, int(vocab_offset),
+                                    int(V_total), float(temperature), _seed(seed), _ptr(row_seeds),
+                                    int(step), _ptr(mask_bits), _ptr(out_keys), _ptr(workspace),
+                                    ws_bytes, _stream(stream)), "fs_sample_shard_keys")
+    return out_keys
+
+
+def fs_keys_to_tokens(keys, out_idx=None, stream=None):
+    """Tokens [B] int32 from reduced keys [B] int64."""
+    lib = load_library()
+    B = keys.numel()
+    out_idx = _out(out_idx, B, keys.device)
+    _check(lib.fs_keys_to_tokens(_ptr(keys), B, _ptr(out_idx), _stream(stream)),
+           "fs_keys_to_tokens")
     return out_idx

@@ -183,12 +183,37 @@ fs_status resolve_workspace(DeviceState *st, const Schedule &sch, int B, void *w
   return FS_OK;
 }
 
+// Set only for the duration of fs_test_stalled_sample (under g_mu).
+bool g_test_no_loads = false;
+
+// Options of a vocabulary-shard call (fs_sample_shard_keys).
+struct ShardOpts {
+  int vocab_offset = 0;         // global token index of W row 0
+  int V_total = 0;              // full vocabulary (0: V); sets the mask row length
+  long long *out_keys = nullptr;  // write packed keys instead of tokens
+};
+
 // The fused path in all three modes, chunked over 256 batch rows.
+fs_status run_locked(int mode, const void *H, const void *W, int B, int d, int V, int G,
+                     float T, uint64_t seed, const uint64_t *row_seeds, uint32_t step,
+                     const uint32_t *mask, int32_t *out_idx, fs_group_summary *summary,
+                     float *logits, void *ws, size_t ws_bytes, cudaStream_t stream,
+                     const ShardOpts &shard = ShardOpts());
+
 fs_status run(int mode, const void *H, const void *W, int B, int d, int V, int G, float T,
               uint64_t seed, const uint64_t *row_seeds, uint32_t step, const uint32_t *mask,
               int32_t *out_idx, fs_group_summary *summary, float *logits, void *ws,
               size_t ws_bytes, cudaStream_t stream) {
   std::lock_guard<std::mutex> lock(g_mu);
+  return run_locked(mode, H, W, B, d, V, G, T, seed, row_seeds, step, mask, out_idx, summary,
+                    logits, ws, ws_bytes, stream);
+}
+
+fs_status run_locked(int mode, const void *H, const void *W, int B, int d, int V, int G,
+                     float T, uint64_t seed, const uint64_t *row_seeds, uint32_t step,
+                     const uint32_t *mask, int32_t *out_idx, fs_group_summary *summary,
+                     float *logits, void *ws, size_t ws_bytes, cudaStream_t stream,
+                     const ShardOpts &shard) {
   DeviceState *st = nullptr;
   fs_status s = get_device(&st);
   if (s != FS_OK) return s;
@@ -222,7 +247,7 @@ fs_status run(int mode, const void *H, const void *W, int B, int d, int V, int G
     p.seed = seed;
     p.row_seeds = row_seeds;
     p.mask = mask;
-    p.mask_words = (V + 31) / 32;
+    p.mask_words = ((shard.V_total > 0 ? shard.V_total : V) + 31) / 32;
     p.out_idx = out_idx + b0;
     p.keys = w.keys;
     p.ticket = w.ticket;
@@ -230,6 +255,9 @@ fs_status run(int mode, const void *H, const void *W, int B, int d, int V, int G
     p.partials = w.partials;
     p.gkeys = mode == fmms::kModeGrouped ? w.gkeys : nullptr;
     p.logits = logits ? logits + static_cast<size_t>(b0) * V : nullptr;
+    p.test_no_loads = g_test_no_loads ? 1 : 0;
+    p.vocab_offset = shard.vocab_offset;
+    p.out_keys = shard.out_keys ? shard.out_keys + b0 : nullptr;
     if (fmms::launch_fmms(mode, BN, tw, tw8, th, p, stream) != cudaSuccess) return FS_ERR_CUDA;
 
     if (mode == fmms::kModeGrouped) {
@@ -349,6 +377,50 @@ fs_status fs_sample_host(const void *H_host, const void *W, int B, int d, int V,
                       st_) != cudaSuccess)
     return FS_ERR_CUDA;
   return FS_OK;
+}
+
+fs_status fs_test_stalled_sample(const void *H, const void *W, int B, int d, int V,
+                                 int32_t *out_idx, void *workspace, size_t workspace_bytes,
+                                 fs_stream_t stream) {
+  fs_status s = validate(H, W, B, d, V, 1.0f, out_idx);
+  if (s != FS_OK) return s;
+  std::lock_guard<std::mutex> lock(g_mu);
+  g_test_no_loads = true;
+  s = run_locked(fmms::kModeFlat, H, W, B, d, V, 1, 1.0f, 0, nullptr, 0, nullptr, out_idx,
+                 nullptr, nullptr, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+  g_test_no_loads = false;
+  return s;
+}
+
+fs_status fs_sample_shard_keys(const void *H, const void *W_shard, int B, int d, int V_shard,
+                               int vocab_offset, int V_total, float temperature, uint64_t seed,
+                               const uint64_t *row_seeds, uint32_t step, const uint32_t *mask_bits,
+                               int64_t *out_keys, void *workspace, size_t workspace_bytes,
+                               fs_stream_t stream) {
+  fs_status s = validate(H, W_shard, B, d, V_shard, temperature, out_keys);
+  if (s != FS_OK) return s;
+  if (vocab_offset < 0 || (vocab_offset % fmms::kGranule) != 0 || V_total < 1 ||
+      static_cast<int64_t>(vocab_offset) + V_shard > V_total)
+    return FS_ERR_INVALID_ARG;
+  ShardOpts opts;
+  opts.vocab_offset = vocab_offset;
+  opts.V_total = V_total;
+  opts.out_keys = reinterpret_cast<long long *>(out_keys);
+  std::lock_guard<std::mutex> lock(g_mu);
+  return run_locked(fmms::kModeFlat, H, W_shard, B, d, V_shard, 1, temperature, seed, row_seeds,
+                    step, mask_bits, reinterpret_cast<int32_t *>(out_keys), nullptr, nullptr,
+                    workspace, workspace_bytes, static_cast<cudaStream_t>(stream), opts);
+}
+
+fs_status fs_keys_to_tokens(const int64_t *keys, int B, int32_t *out_idx, fs_stream_t stream) {
+  if (!keys || !out_idx || B < 1) return FS_ERR_INVALID_ARG;
+  DeviceState *st = nullptr;
+  fs_status s = get_device(&st);
+  if (s != FS_OK) return s;
+  return fmms::launch_keys_to_tokens(reinterpret_cast<const long long *>(keys), B, out_idx,
+                                     static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? FS_OK
+             : FS_ERR_CUDA;
 }
 
 size_t fs_workspace_bytes(int B, int V, int G) {

@@ -176,6 +176,20 @@ cudaError_t launch_sample_logits(const SampleLogitsParams &s, cudaStream_t strea
 }
 
 // ---------------------------------------------------------------------------
+// Vocabulary shards: tokens from the reduced keys.
+// ---------------------------------------------------------------------------
+__global__ void keys_to_tokens_kernel(const long long *keys, int B, int32_t *out_idx) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b < B) out_idx[b] = key_token(static_cast<uint64_t>(keys[b]) ^ 0x8000000000000000ull);
+}
+
+cudaError_t launch_keys_to_tokens(const long long *keys, int B, int32_t *out_idx,
+                                  cudaStream_t stream) {
+  keys_to_tokens_kernel<<<(B + 255) / 256, 256, 0, stream>>>(keys, B, out_idx);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
 // Test kernels
 // ---------------------------------------------------------------------------
 __global__ void philox_test_kernel(const uint32_t *ctr, const uint32_t *key, uint32_t *out,

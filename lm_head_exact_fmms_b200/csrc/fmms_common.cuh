@@ -172,6 +172,9 @@ struct FmmsParams {
   GroupPartial *partials;      // workspace [slots][B] (grouped)
   unsigned long long *gkeys;   // workspace [G][B] published per-group maxima, or null
   float *logits;               // [B][V] (logits mode; already offset)
+  int test_no_loads;           // test hook: the producer issues no loads, so waits time out
+  int vocab_offset;            // global token index of W row 0 (a vocabulary shard), % 8 == 0
+  long long *out_keys;         // if set: per-row packed keys XOR 2^63 instead of tokens
 };
 
 // Workspace layout (bytes): [0, 256) status word and ticket; [256, 256 + 2048)

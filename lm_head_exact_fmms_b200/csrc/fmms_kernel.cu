@@ -287,7 +287,7 @@ __device__ __forceinline__ void role_producer(const CUtensorMap *tw, const CUten
   int stage = 0;
   uint32_t phase = 0;
   long long issued = 0;
-  bool ok = true;
+  bool ok = p.test_no_loads == 0;
   while (ok && it.next(tile)) {
     const int rows = tile.hi - tile.start;
     const bool whole = rows == kTileM;
@@ -316,7 +316,7 @@ __device__ __forceinline__ void role_producer(const CUtensorMap *tw, const CUten
       }
     }
   }
-  if (!ok) {
+  if (!ok && issued > 0) {
     // Gave up: let the copies already in flight land before the CTA exits.
     const long long first = issued > C::kStages ? issued - C::kStages : 0;
     for (long long n = first; n < issued; ++n) {
@@ -417,8 +417,9 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
     aborted = __any_sync(0xffffffffu, !got);
     if (!aborted) {
       sm100::tc_fence_after();
-      const int v = tile.start + 32 * q + lane;
+      const int v = tile.start + 32 * q + lane;           // row of W in this launch
       const bool v_ok = v >= tile.lo && v < tile.hi;
+      const int vg = v + p.vocab_offset;                  // global token index
       const uint32_t tbase =
           tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(buf * BN);
 #pragma unroll
@@ -447,10 +448,10 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
             // The mask is consulted only on the exact path.
             const uint64_t pub = c < p.B ? ld_key(p.keys + c) : 0ull;  // in flight during Philox
             uint32_t words[CW];
-            chunk_noise<CW>(p, v, col0, lane, words);
+            chunk_noise<CW>(p, vg, col0, lane, words);
             if (chunk_any_candidate<CW>(acc, words, p, chunk_in_range<CW>(p, v_ok, col0),
                                         best[kk], pub, lane)) {
-              chunk_keys<CW>(acc, words, p, v, chunk_allowed<CW>(p, v, v_ok, col0), lane,
+              chunk_keys<CW>(acc, words, p, vg, chunk_allowed<CW>(p, vg, v_ok, col0), lane,
                              best[kk]);
               // publish the improved maximum so every CTA's filter sharpens
               if ((lane & 1) == 0 && c < p.B && key_valid(best[kk]) && best[kk] > pub)
@@ -461,12 +462,12 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
                 p.gkeys ? p.gkeys + static_cast<size_t>(tile.slot - blockIdx.x) * p.B + c
                         : nullptr;
             const uint64_t pub = (gk != nullptr && c < p.B) ? ld_key(gk) : 0ull;
-            const uint32_t allowed = chunk_allowed<CW>(p, v, v_ok, col0);
+            const uint32_t allowed = chunk_allowed<CW>(p, vg, v_ok, col0);
             uint32_t words[CW];
-            chunk_noise<CW>(p, v, col0, lane, words);
+            chunk_noise<CW>(p, vg, col0, lane, words);
             chunk_lse<CW>(acc, p, allowed, lane, m_run[kk], s_run[kk]);
             if (chunk_any_candidate<CW>(acc, words, p, allowed, best[kk], pub, lane)) {
-              chunk_keys<CW>(acc, words, p, v, allowed, lane, best[kk]);
+              chunk_keys<CW>(acc, words, p, vg, allowed, lane, best[kk]);
               if (gk != nullptr && (lane & 1) == 0 && c < p.B && key_valid(best[kk]) &&
                   best[kk] > pub)
                 atomicMax(gk, static_cast<unsigned long long>(best[kk]));
@@ -556,7 +557,10 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
       __threadfence();
       for (int b = etid; b < p.B; b += kEpiThreads) {
         const unsigned long long kb = atomicExch(p.keys + b, 0ull);
-        p.out_idx[b] = key_token(kb);
+        if (p.out_keys != nullptr)
+          p.out_keys[b] = static_cast<long long>(kb ^ 0x8000000000000000ull);  // signed order
+        else
+          p.out_idx[b] = key_token(kb);
       }
       if (etid == 0) atomicExch(p.ticket, 0u);
     }

@@ -47,6 +47,10 @@ struct SampleLogitsParams {
 };
 cudaError_t launch_sample_logits(const SampleLogitsParams &s, cudaStream_t stream);
 
+// Decodes packed keys (XOR 2^63, as fs_sample_shard_keys writes them) to tokens.
+cudaError_t launch_keys_to_tokens(const long long *keys, int B, int32_t *out_idx,
+                                  cudaStream_t stream);
+
 cudaError_t launch_philox_test(const uint32_t *ctr, const uint32_t *key, uint32_t *out, int64_t n,
                                cudaStream_t stream);
 cudaError_t launch_gumbel_test(const uint32_t *r, float *g, int64_t n, cudaStream_t stream);

@@ -66,6 +66,8 @@ def test_grouped_and_unfused_validation(lib):
                                  0, None) == 1
     assert lib.fs_sample_host(None, FAKE, 4, 64, 100, 1.0, 0, None, 0, None, FAKE, None) == 1
     assert lib.fs_philox4x32_10(None, None, None, 5, None) == 1
+    assert lib.fs_test_stalled_sample(None, FAKE, 4, 64, 100, FAKE, None, 0, None) == 1
+    assert lib.fs_sample_noalloc(FAKE, FAKE, 4, 64, 100, 0.0, 0, None, 0, None, FAKE, None) == 1
     assert lib.fs_gumbel(None, None, -1, None) == 1
 
 

@@ -371,3 +371,26 @@ def test_full_size_workloads(dev, oracle, name):
         del Hd
     del Wd
     torch.cuda.empty_cache()
+
+
+# --------------------------------------------- tensor-parallel vocabulary shards
+@pytest.mark.parametrize("world,B", [(2, 8), (3, 64), (4, 256), (5, 300)])
+def test_vocab_shards_equal_single_gpu(dev, world, B):
+    """Shards of the head on one GPU, reduced with an int64 max as the
+    all-reduce does, give the single-GPU tokens bit for bit."""
+    from lm_head_exact_fmms_b200.tp import shard_bounds
+    d, V = 256, 30011
+    H, W, Hd, Wd = rand_inputs(B, d, V, seed=world * 7 + B)
+    rs = synth.make_row_seeds(B).to(dev)
+    mask = synth.make_mask(B, V, 0.5, seed=world).to(dev)
+    for step in range(2):
+        ref = binding.fs_sample_ex(Hd, Wd, temperature=0.9, seed=4, row_seeds=rs, step=step,
+                                   mask_bits=mask)
+        keys = []
+        for lo, hi in shard_bounds(V, world):
+            keys.append(binding.fs_sample_shard_keys(Hd, Wd[lo:hi].contiguous(), lo, V,
+                                                     temperature=0.9, seed=4, row_seeds=rs,
+                                                     step=step, mask_bits=mask))
+        red = torch.stack(keys).max(dim=0).values.contiguous()
+        got = binding.fs_keys_to_tokens(red)
+        assert torch.equal(got, ref)
