@@ -243,6 +243,8 @@ def time_calls(fn, steps, warmup, stream, world=1, sampler=None, cooldown_s=1.0)
         fn(warmup + i)
         ends[i].record(stream)
     r1.record(stream)
+    while not r1.query():     # poll (releasing the GIL) so the clock sampler keeps running
+        time.sleep(0.0005)
     torch.cuda.synchronize()
     barrier(world)
     if sampler:
@@ -379,6 +381,7 @@ def run_gpu(args, world, rank, local):
         result["grouped_masked"] = grouped_points(torch, binding, synth, dev, stream, peaks,
                                                   peak_kind, W)
         result["unfused"] = unfused_point(torch, binding, synth, W, wl, dev, stream, B)
+        result["multi_sample"] = multi_point(torch, binding, synth, W, wl, dev, stream, B)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(H, W, wl, B, rs)
     return result
@@ -430,6 +433,22 @@ def grouped_points(torch, binding, synth, dev, stream, peaks, peak_kind, W8, ste
                      "launches_per_call": 2 * ((B + 255) // 256)})
     return {"workload": "grouped-masked d=%d V=%d G=%d, 50%% mask, T=%g (fused kernel + merge)"
                         % (wl.d, wl.V, wl.groups, wl.temperature), "points": rows}
+
+
+def multi_point(torch, binding, synth, W, wl, dev, stream, B, S=4, steps=100):
+    """num_samples > 1: S exact draws per row from one pass over W."""
+    H = synth.make_hidden(B, wl.d, device=dev)
+    rs = synth.make_row_seeds(B, device=dev) if wl.per_row_seeds else None
+    out = torch.empty(B, S, dtype=torch.int32, device=dev)
+    ws = torch.zeros(binding.fs_workspace_bytes_multi(B, wl.V, S), dtype=torch.uint8, device=dev)
+
+    def step(i):
+        binding.fs_sample_multi(H, W, S, temperature=wl.temperature, seed=0, row_seeds=rs, step=i,
+                                out_idx=out, workspace=ws, stream=stream)
+
+    region_ms, _ = time_calls(step, steps, 10, stream)
+    return {"B": B, "num_samples": S, "us_per_call": round(region_ms * 1e3 / steps, 3),
+            "samples_per_s": round(B * S / (region_ms * 1e-3 / steps), 1)}
 
 
 def unfused_point(torch, binding, synth, W, wl, dev, stream, B, steps=100):

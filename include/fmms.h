@@ -47,8 +47,11 @@
  *  workspace  entry points that take (workspace, workspace_bytes) use the
  *         caller's device buffer of at least fs_workspace_bytes(B, V, G) bytes,
  *         256-byte aligned, which must be zero-filled before its first use
- *         (cudaMemset) and is left zeroed by every call that completes.
- *         Calls that share a workspace must be ordered on one stream.  With
+ *         (cudaMemset).  Every call that completes leaves the parts that must
+ *         start at zero (status, ticket, per-row keys, published maxima)
+ *         zeroed again; the grouped calls' partials are per-call scratch.  One
+ *         workspace may serve calls of any kind and size it is large enough
+ *         for.  Calls that share a workspace must be ordered on one stream.  With
  *         workspace == NULL the library uses its own per-device workspace,
  *         allocated on first use; such calls must not run concurrently on
  *         different streams.
@@ -135,6 +138,20 @@ fs_status fs_sample_unfused(const void *H, const void *W, int B, int d, int V,
                             float *logits, void *workspace,
                             size_t workspace_bytes, fs_stream_t stream);
 
+/* Several samples per row from one pass over W (readus.org page, API: the
+ * number of samples is an argument of the sampling call).  Sample k of row b
+ * uses token noise with counter tag 2k, so the samples are independent exact
+ * draws from softmax(l/T) (with replacement) and sample 0 is the fs_sample_ex
+ * token.  out_idx is device int32 [B][num_samples] (row-major), 1 <= num_samples
+ * <= 64.  The workspace needs fs_workspace_bytes_multi(B, V, num_samples)
+ * bytes; other arguments as fs_sample_ex. */
+fs_status fs_sample_multi(const void *H, const void *W, int B, int d, int V,
+                          int num_samples, float temperature, uint64_t seed,
+                          const uint64_t *row_seeds, uint32_t step,
+                          const uint32_t *mask_bits, int32_t *out_idx,
+                          void *workspace, size_t workspace_bytes,
+                          fs_stream_t stream);
+
 /* One vocabulary shard of a tensor-parallel LM head (readus.org page,
  * "distributed FlashSampling": each GPU is one group of the vocabulary and
  * contributes only its winning index and score; abstract: the argmax
@@ -202,6 +219,10 @@ fs_status fs_sample_noalloc(const void *H, const void *W, int B, int d, int V,
 /* Bytes of caller workspace needed by the calls above for these sizes on the
  * current device (G = 0 or 1 for flat sampling).  Returns 0 on invalid sizes. */
 size_t fs_workspace_bytes(int B, int V, int G);
+
+/* Workspace bytes of fs_sample_multi on the current device (0 on invalid
+ * sizes). */
+size_t fs_workspace_bytes_multi(int B, int V, int num_samples);
 
 /* Reads (synchronously, after the stream drains) and clears the device-side
  * status word of a workspace (NULL = the library-owned one on the current

@@ -22,7 +22,7 @@ EXPORTED = ("fs_sample", "fs_sample_ex", "fs_sample_grouped", "fs_sample_unfused
             "fs_sample_host", "fs_workspace_bytes", "fs_device_status", "fs_status_string",
             "fs_philox4x32_10", "fs_gumbel", "fs_plan_tiles", "fs_plan_group_ctas",
             "fs_sample_noalloc", "fs_test_stalled_sample", "fs_sample_shard_keys",
-            "fs_keys_to_tokens")
+            "fs_keys_to_tokens", "fs_sample_multi", "fs_workspace_bytes_multi")
 
 
 class FmmsError(RuntimeError):
@@ -63,6 +63,9 @@ def load_library():
     lib.fs_test_stalled_sample.argtypes = common + [vp, vp, sz, vp]
     lib.fs_sample_shard_keys.argtypes = common + [i32, i32, f32, u64, vp, u32, vp, vp, vp, sz, vp]
     lib.fs_keys_to_tokens.argtypes = [vp, i32, vp, vp]
+    lib.fs_sample_multi.argtypes = common + [i32, f32, u64, vp, u32, vp, vp, vp, sz, vp]
+    lib.fs_workspace_bytes_multi.argtypes = [i32, i32, i32]
+    lib.fs_workspace_bytes_multi.restype = sz
     lib.fs_workspace_bytes.argtypes = [i32, i32, i32]
     lib.fs_workspace_bytes.restype = sz
     lib.fs_device_status.argtypes = [vp, sz, vp]
@@ -75,7 +78,7 @@ def load_library():
     lib.fs_plan_group_ctas.argtypes = [i32, i32, i32, i32, ctypes.POINTER(ctypes.c_int),
                                        ctypes.POINTER(ctypes.c_int)]
     for name in EXPORTED:
-        if name not in ("fs_workspace_bytes", "fs_status_string"):
+        if name not in ("fs_workspace_bytes", "fs_workspace_bytes_multi", "fs_status_string"):
             getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -337,3 +340,25 @@ def fs_keys_to_tokens(keys, out_idx=None, stream=None):
     _check(lib.fs_keys_to_tokens(_ptr(keys), B, _ptr(out_idx), _stream(stream)),
            "fs_keys_to_tokens")
     return out_idx
+
+
+def fs_sample_multi(H, W, num_samples, temperature=1.0, seed=0, row_seeds=None, step=0,
+                    mask_bits=None, out_idx=None, workspace=None, stream=None):
+    """num_samples exact draws per row from one pass over W: int32 [B, num_samples]."""
+    lib = load_library()
+    B, d, V = _check_operands(H, W)
+    row_seeds = _opt_dev(row_seeds, torch.int64, B, "row_seeds", H.device)
+    mask_bits = _opt_dev(mask_bits, torch.int32, B * ((V + 31) // 32), "mask_bits", H.device)
+    if out_idx is None:
+        out_idx = torch.empty(B, int(num_samples), dtype=torch.int32, device=H.device)
+    _opt_dev(out_idx, torch.int32, B * int(num_samples), "out_idx", H.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.fs_sample_multi(_ptr(H), _ptr(W), B, d, V, int(num_samples), float(temperature),
+                               _seed(seed), _ptr(row_seeds), int(step), _ptr(mask_bits),
+                               _ptr(out_idx), _ptr(workspace), ws_bytes, _stream(stream)),
+           "fs_sample_multi")
+    return out_idx
+
+
+def fs_workspace_bytes_multi(B, V, num_samples):
+    return int(load_library().fs_workspace_bytes_multi(int(B), int(V), int(num_samples)))

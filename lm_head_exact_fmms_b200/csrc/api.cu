@@ -155,23 +155,26 @@ struct Workspace {
   unsigned long long *gkeys;
 };
 
-Workspace carve(void *ws, int B, int G, int num_ctas) {
+Workspace carve(void *ws, int B, int G, int num_ctas, int samples) {
   char *b = static_cast<char *>(ws);
+  (void)samples;
+  const size_t keys_bytes = static_cast<size_t>(fmms::kWsKeysRegion);  // fixed layout
   Workspace w;
   w.err = reinterpret_cast<int *>(b);
   w.ticket = reinterpret_cast<unsigned int *>(b + 4);
   w.keys = reinterpret_cast<unsigned long long *>(b + fmms::kWsHeader);
-  w.partials = reinterpret_cast<fmms::GroupPartial *>(b + fmms::kWsHeader + fmms::kWsKeys);
+  w.partials = reinterpret_cast<fmms::GroupPartial *>(b + fmms::kWsHeader + keys_bytes);
   w.gkeys = fmms::ws_gkeys_bytes(B, G) > 0
                 ? reinterpret_cast<unsigned long long *>(
-                      b + fmms::kWsHeader + fmms::kWsKeys + fmms::ws_partials_bytes(B, G, num_ctas))
+                      b + fmms::kWsHeader + keys_bytes + fmms::ws_partials_bytes(B, G, num_ctas))
                 : nullptr;
   return w;
 }
 
-fs_status resolve_workspace(DeviceState *st, const Schedule &sch, int B, void *ws, size_t ws_bytes,
-                            void **out) {
-  const size_t need = static_cast<size_t>(fmms::workspace_bytes_for(B, sch.G, sch.num_ctas));
+fs_status resolve_workspace(DeviceState *st, const Schedule &sch, int B, int samples, void *ws,
+                            size_t ws_bytes, void **out) {
+  const size_t need =
+      static_cast<size_t>(fmms::workspace_bytes_for(B, sch.G, sch.num_ctas, samples));
   if (ws == nullptr) {
     fs_status s = grow(&st->ws, &st->ws_bytes, need);
     if (s != FS_OK) return s;
@@ -186,11 +189,12 @@ fs_status resolve_workspace(DeviceState *st, const Schedule &sch, int B, void *w
 // Set only for the duration of fs_test_stalled_sample (under g_mu).
 bool g_test_no_loads = false;
 
-// Options of a vocabulary-shard call (fs_sample_shard_keys).
+// Options of vocabulary-shard and multi-sample calls.
 struct ShardOpts {
   int vocab_offset = 0;         // global token index of W row 0
   int V_total = 0;              // full vocabulary (0: V); sets the mask row length
   long long *out_keys = nullptr;  // write packed keys instead of tokens
+  int num_samples = 1;          // samples per row (flat mode)
 };
 
 // The fused path in all three modes, chunked over 256 batch rows.
@@ -219,9 +223,10 @@ fs_status run_locked(int mode, const void *H, const void *W, int B, int d, int V
   if (s != FS_OK) return s;
   const Schedule sch = fmms::make_schedule(V, mode == fmms::kModeGrouped ? G : 1, st->sms);
   void *wsp = nullptr;
-  s = resolve_workspace(st, sch, B, ws, ws_bytes, &wsp);
+  const int S = shard.num_samples;
+  s = resolve_workspace(st, sch, B, S, ws, ws_bytes, &wsp);
   if (s != FS_OK) return s;
-  const Workspace w = carve(wsp, B, sch.G, sch.num_ctas);
+  const Workspace w = carve(wsp, B, sch.G, sch.num_ctas, S);
 
   CUtensorMap tw, tw8;
   if ((s = tensor_map(&tw, W, d, V, fmms::kTileM)) != FS_OK) return s;
@@ -248,7 +253,7 @@ fs_status run_locked(int mode, const void *H, const void *W, int B, int d, int V
     p.row_seeds = row_seeds;
     p.mask = mask;
     p.mask_words = ((shard.V_total > 0 ? shard.V_total : V) + 31) / 32;
-    p.out_idx = out_idx + b0;
+    p.out_idx = out_idx + static_cast<size_t>(b0) * S;
     p.keys = w.keys;
     p.ticket = w.ticket;
     p.err = w.err;
@@ -257,7 +262,8 @@ fs_status run_locked(int mode, const void *H, const void *W, int B, int d, int V
     p.logits = logits ? logits + static_cast<size_t>(b0) * V : nullptr;
     p.test_no_loads = g_test_no_loads ? 1 : 0;
     p.vocab_offset = shard.vocab_offset;
-    p.out_keys = shard.out_keys ? shard.out_keys + b0 : nullptr;
+    p.out_keys = shard.out_keys ? shard.out_keys + static_cast<size_t>(b0) * S : nullptr;
+    p.num_samples = S;
     if (fmms::launch_fmms(mode, BN, tw, tw8, th, p, stream) != cudaSuccess) return FS_ERR_CUDA;
 
     if (mode == fmms::kModeGrouped) {
@@ -410,6 +416,31 @@ fs_status fs_sample_shard_keys(const void *H, const void *W_shard, int B, int d,
   return run_locked(fmms::kModeFlat, H, W_shard, B, d, V_shard, 1, temperature, seed, row_seeds,
                     step, mask_bits, reinterpret_cast<int32_t *>(out_keys), nullptr, nullptr,
                     workspace, workspace_bytes, static_cast<cudaStream_t>(stream), opts);
+}
+
+fs_status fs_sample_multi(const void *H, const void *W, int B, int d, int V, int num_samples,
+                          float temperature, uint64_t seed, const uint64_t *row_seeds,
+                          uint32_t step, const uint32_t *mask_bits, int32_t *out_idx,
+                          void *workspace, size_t workspace_bytes, fs_stream_t stream) {
+  fs_status s = validate(H, W, B, d, V, temperature, out_idx);
+  if (s != FS_OK) return s;
+  if (num_samples < 1 || num_samples > fmms::kMaxSamples) return FS_ERR_INVALID_ARG;
+  ShardOpts opts;
+  opts.num_samples = num_samples;
+  std::lock_guard<std::mutex> lock(g_mu);
+  return run_locked(fmms::kModeFlat, H, W, B, d, V, 1, temperature, seed, row_seeds, step,
+                    mask_bits, out_idx, nullptr, nullptr, workspace, workspace_bytes,
+                    static_cast<cudaStream_t>(stream), opts);
+}
+
+size_t fs_workspace_bytes_multi(int B, int V, int num_samples) {
+  if (B < 1 || V < 1 || num_samples < 1 || num_samples > fmms::kMaxSamples) return 0;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 0;
+  const Schedule sch = fmms::make_schedule(V, 1, sms);
+  return static_cast<size_t>(fmms::workspace_bytes_for(B, 1, sch.num_ctas, num_samples));
 }
 
 fs_status fs_keys_to_tokens(const int64_t *keys, int B, int32_t *out_idx, fs_stream_t stream) {

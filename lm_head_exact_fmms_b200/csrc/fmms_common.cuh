@@ -175,15 +175,22 @@ struct FmmsParams {
   int test_no_loads;           // test hook: the producer issues no loads, so waits time out
   int vocab_offset;            // global token index of W row 0 (a vocabulary shard), % 8 == 0
   long long *out_keys;         // if set: per-row packed keys XOR 2^63 instead of tokens
+  int num_samples;             // samples per row (flat mode), 1..kMaxSamples
 };
 
-// Workspace layout (bytes): [0, 256) status word and ticket; [256, 256 + 2048)
-// packed keys of up to 256 rows; then, grouped, the partials [slots][rows]
-// and, for G <= kMaxPublishedGroups, the published per-group maxima
-// [G][rows] that sharpen the exact-score filter (re-zeroed by the merge).
+// Workspace layout (bytes), fixed so that calls of different kinds can share
+// one workspace: [0, 256) status word and ticket; [256, 256 + 64 * 2048)
+// packed keys [sample][256 rows], of which a flat call uses (and needs) only
+// its samples' part; then, grouped only, the partials [slots][rows] and, for
+// G <= kMaxPublishedGroups, the published per-group maxima [G][rows] that
+// sharpen the exact-score filter (re-zeroed by the merge kernel).  Keys, the
+// ticket and the published maxima are left zeroed by every completed call;
+// partials are per-call scratch, each written before it is read.
 constexpr int kWsHeader = 256;
 constexpr int kWsKeys = 8 * kMaxBN;
 constexpr int kMaxPublishedGroups = 4096;
+constexpr int kMaxSamples = 64;
+constexpr int kWsKeysRegion = kMaxSamples * kWsKeys;
 
 FS_HD int64_t ws_partials_bytes(int B, int G, int num_ctas) {
   const int64_t rows = B < kMaxBN ? B : kMaxBN;
@@ -195,9 +202,11 @@ FS_HD int64_t ws_gkeys_bytes(int B, int G) {
   return (G > 1 && G <= kMaxPublishedGroups) ? (int64_t)G * rows * 8 : 0;
 }
 
-FS_HD int64_t workspace_bytes_for(int B, int G, int num_ctas) {
+FS_HD int64_t workspace_bytes_for(int B, int G, int num_ctas, int samples = 1) {
   const int64_t bytes =
-      kWsHeader + kWsKeys + ws_partials_bytes(B, G, num_ctas) + ws_gkeys_bytes(B, G);
+      G > 1 ? (int64_t)kWsHeader + kWsKeysRegion + ws_partials_bytes(B, G, num_ctas) +
+                  ws_gkeys_bytes(B, G)
+            : (int64_t)kWsHeader + (int64_t)kWsKeys * (samples < 1 ? 1 : samples);
   return (bytes + 255) / 256 * 256;
 }
 

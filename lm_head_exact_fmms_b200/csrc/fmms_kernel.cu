@@ -162,14 +162,14 @@ __device__ __forceinline__ uint64_t ld_key(const unsigned long long *ptr) {
 // consecutive tokens of one row; the quad transpose hands each lane its word.
 template <int CW>
 __device__ __forceinline__ void chunk_noise(const FmmsParams &p, int v, int col0, int lane,
-                                            uint32_t (&words)[CW]) {
+                                            uint32_t tag, uint32_t (&words)[CW]) {
 #pragma unroll
   for (int q4 = 0; q4 < CW / 4; ++q4) {
     const int colp = col0 + 4 * q4 + (lane & 3);  // column of this lane's Philox call
     const uint32_t bg = static_cast<uint32_t>(p.b_off + colp);
     uint64_t k64 = p.seed;
     if (p.row_seeds != nullptr && colp < p.B) k64 = __ldg(p.row_seeds + bg);
-    const Philox4 ph = philox4x32_10(static_cast<uint32_t>(v) >> 2, bg, p.step, 0u,
+    const Philox4 ph = philox4x32_10(static_cast<uint32_t>(v) >> 2, bg, p.step, tag,
                                      static_cast<uint32_t>(k64), static_cast<uint32_t>(k64 >> 32));
     uint32_t w[4] = {ph.w0, ph.w1, ph.w2, ph.w3};
     quad_transpose(w, lane);
@@ -445,17 +445,29 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
         } else {
           const int c = col0 + column_of_lane<CW>(lane);  // this lane's column
           if constexpr (MODE == kModeFlat) {
+            // Sample smp draws with token-noise tag 2 smp and keeps its running
+            // per-row maximum in the published keys [smp][row]: every exact
+            // chunk raises it at once, which also sharpens every CTA's filter.
             // The mask is consulted only on the exact path.
-            const uint64_t pub = c < p.B ? ld_key(p.keys + c) : 0ull;  // in flight during Philox
-            uint32_t words[CW];
-            chunk_noise<CW>(p, vg, col0, lane, words);
-            if (chunk_any_candidate<CW>(acc, words, p, chunk_in_range<CW>(p, v_ok, col0),
-                                        best[kk], pub, lane)) {
-              chunk_keys<CW>(acc, words, p, vg, chunk_allowed<CW>(p, vg, v_ok, col0), lane,
-                             best[kk]);
-              // publish the improved maximum so every CTA's filter sharpens
-              if ((lane & 1) == 0 && c < p.B && key_valid(best[kk]) && best[kk] > pub)
-                atomicMax(p.keys + c, static_cast<unsigned long long>(best[kk]));
+            const uint32_t in_range = chunk_in_range<CW>(p, v_ok, col0);
+            uint32_t allowed = 0u;
+            bool have_allowed = false;
+#pragma unroll 1
+            for (int smp = 0; smp < p.num_samples; ++smp) {
+              unsigned long long *kp = p.keys + smp * kMaxBN + c;
+              const uint64_t pub = c < p.B ? ld_key(kp) : 0ull;  // in flight during Philox
+              uint32_t words[CW];
+              chunk_noise<CW>(p, vg, col0, lane, 2u * static_cast<uint32_t>(smp), words);
+              if (chunk_any_candidate<CW>(acc, words, p, in_range, 0ull, pub, lane)) {
+                if (!have_allowed) {
+                  allowed = chunk_allowed<CW>(p, vg, v_ok, col0);
+                  have_allowed = true;
+                }
+                uint64_t cbest = 0ull;
+                chunk_keys<CW>(acc, words, p, vg, allowed, lane, cbest);
+                if ((lane & 1) == 0 && c < p.B && key_valid(cbest) && cbest > pub)
+                  atomicMax(kp, static_cast<unsigned long long>(cbest));
+              }
             }
           } else {
             unsigned long long *gk =
@@ -464,7 +476,7 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
             const uint64_t pub = (gk != nullptr && c < p.B) ? ld_key(gk) : 0ull;
             const uint32_t allowed = chunk_allowed<CW>(p, vg, v_ok, col0);
             uint32_t words[CW];
-            chunk_noise<CW>(p, vg, col0, lane, words);
+            chunk_noise<CW>(p, vg, col0, lane, 0u, words);
             chunk_lse<CW>(acc, p, allowed, lane, m_run[kk], s_run[kk]);
             if (chunk_any_candidate<CW>(acc, words, p, allowed, best[kk], pub, lane)) {
               chunk_keys<CW>(acc, words, p, vg, allowed, lane, best[kk]);
@@ -525,42 +537,28 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
   }
 
   if constexpr (MODE == kModeFlat) {
-#pragma unroll
-    for (int kk = 0; kk < C::kChunksPerWarp; ++kk) {
-      if (!has_chunks) continue;
-      const int k = kk * C::kWarpsPerQuarter + h;
-      if (k * CW < p.B) comb_key[q * BN + k * CW + column_of_lane<CW>(lane)] = best[kk];
-    }
-    sm100::epi_sync(kEpiThreads);
-    const bool ok = !*abort_flag;
-    if (ok) {
-      for (int b = etid; b < p.B; b += kEpiThreads) {
-        uint64_t kb = 0ull;
-#pragma unroll
-        for (int qq = 0; qq < 4; ++qq) {
-          const uint64_t kq = comb_key[qq * BN + b];
-          kb = kq > kb ? kq : kb;
-        }
-        if (key_valid(kb)) atomicMax(p.keys + b, static_cast<unsigned long long>(kb));
-      }
-      __threadfence();
-    }
+    // Every maximum is already published; take a ticket, and the last CTA
+    // decodes the keys and re-zeroes them for the next call.
+    __threadfence();
     sm100::epi_sync(kEpiThreads);
     if (etid == 0) {
       int last = 0;
-      if (ok) last = (atomicAdd(p.ticket, 1u) == static_cast<unsigned>(p.num_ctas - 1)) ? 1 : 0;
+      if (!*abort_flag)
+        last = (atomicAdd(p.ticket, 1u) == static_cast<unsigned>(p.num_ctas - 1)) ? 1 : 0;
       *last_flag = last;
     }
     sm100::epi_sync(kEpiThreads);
     if (*last_flag) {
-      // Every other CTA has published its maxima: decode and re-zero.
       __threadfence();
-      for (int b = etid; b < p.B; b += kEpiThreads) {
-        const unsigned long long kb = atomicExch(p.keys + b, 0ull);
+      const int total = p.B * p.num_samples;
+      for (int i = etid; i < total; i += kEpiThreads) {
+        const int b = i / p.num_samples;
+        const int smp = i - b * p.num_samples;
+        const unsigned long long kb = atomicExch(p.keys + smp * kMaxBN + b, 0ull);
         if (p.out_keys != nullptr)
-          p.out_keys[b] = static_cast<long long>(kb ^ 0x8000000000000000ull);  // signed order
+          p.out_keys[i] = static_cast<long long>(kb ^ 0x8000000000000000ull);  // signed order
         else
-          p.out_idx[b] = key_token(kb);
+          p.out_idx[i] = key_token(kb);
       }
       if (etid == 0) atomicExch(p.ticket, 0u);
     }

@@ -180,19 +180,28 @@ static uint64_t row_key(uint64_t seed, const uint64_t *row_seeds, int b) {
   return row_seeds ? row_seeds[b] : seed;
 }
 
-/* s[v] for row b given its logits l[v]. */
-static void scores_from_logits(const double *l, int V, double T, uint64_t key,
-                               uint32_t step, int b, const uint32_t *mask,
-                               double *s) {
+/* s[v] for row b given its logits l[v], with token noise of counter tag
+ * `tag` (0 for the first sample of a row; sample k of a multi-sample call
+ * uses 2k, keeping odd tags for group noise). */
+static void scores_from_logits_tag(const double *l, int V, double T,
+                                   uint64_t key, uint32_t step, int b,
+                                   uint32_t tag, const uint32_t *mask,
+                                   double *s) {
 #pragma omp parallel for schedule(static)
   for (int v = 0; v < V; ++v) {
     if (!token_allowed(mask, V, b, v)) {
       s[v] = -INFINITY;
     } else {
-      uint32_t r = oracle_noise_word(key, step, (uint32_t)b, (uint32_t)v, 0u);
+      uint32_t r = oracle_noise_word(key, step, (uint32_t)b, (uint32_t)v, tag);
       s[v] = l[v] / T + oracle_gumbel_from_u32(r);
     }
   }
+}
+
+static void scores_from_logits(const double *l, int V, double T, uint64_t key,
+                               uint32_t step, int b, const uint32_t *mask,
+                               double *s) {
+  scores_from_logits_tag(l, V, T, key, step, b, 0u, mask, s);
 }
 
 /* Perturbed scores of the listed rows: out[i*V + v] = s[rows[i], v]. */
@@ -252,6 +261,35 @@ void oracle_sample(const uint16_t *H, const uint16_t *W, int B, int d, int V,
     out_idx[i] = argmax_scan(s, 0, V, &b1, &b2);
     if (out_best) out_best[i] = b1;
     if (out_second) out_second[i] = b2;
+  }
+  free(s);
+  free(l);
+}
+
+/* Several samples per row: sample k draws with token-noise tag 2k, so the
+ * samples are independent draws from the same softmax and sample 0 is the
+ * single-sample result.  out_idx[i*S + k], out_best / out_second likewise
+ * (readus.org page, API: the number of samples is an argument of the call). */
+void oracle_sample_multi(const uint16_t *H, const uint16_t *W, int B, int d,
+                         int V, int S, double T, uint64_t seed,
+                         const uint64_t *row_seeds, uint32_t step,
+                         const uint32_t *mask, const int32_t *rows, int nrows,
+                         int32_t *out_idx, double *out_best,
+                         double *out_second) {
+  (void)B;
+  double *l = (double *)malloc(sizeof(double) * (size_t)V);
+  double *s = (double *)malloc(sizeof(double) * (size_t)V);
+  for (int i = 0; i < nrows; ++i) {
+    int b = rows[i];
+    logits_row(H + (int64_t)b * d, W, d, V, l);
+    for (int k = 0; k < S; ++k) {
+      scores_from_logits_tag(l, V, T, row_key(seed, row_seeds, b), step, b,
+                             2u * (uint32_t)k, mask, s);
+      double b1, b2;
+      out_idx[(int64_t)i * S + k] = argmax_scan(s, 0, V, &b1, &b2);
+      if (out_best) out_best[(int64_t)i * S + k] = b1;
+      if (out_second) out_second[(int64_t)i * S + k] = b2;
+    }
   }
   free(s);
   free(l);

@@ -394,3 +394,53 @@ def test_vocab_shards_equal_single_gpu(dev, world, B):
         red = torch.stack(keys).max(dim=0).values.contiguous()
         got = binding.fs_keys_to_tokens(red)
         assert torch.equal(got, ref)
+
+
+# ----------------------------------------------------- several samples per row
+@pytest.mark.parametrize("B,d,V,S", [(1, 64, 4096, 8), (17, 96, 3001, 3), (64, 128, 9000, 4),
+                                     (300, 64, 2048, 2)])
+def test_multi_sample_parity(dev, oracle, B, d, V, S):
+    H, W, Hd, Wd = rand_inputs(B, d, V, seed=B + S)
+    rs = synth.make_row_seeds(B)
+    mask = synth.make_mask(B, V, 0.7, seed=S)
+    got = binding.fs_sample_multi(Hd, Wd, S, temperature=0.9, seed=3, row_seeds=rs.to(dev),
+                                  step=2, mask_bits=mask.to(dev)).cpu().numpy()
+    idx, best, second = oracle.sample_multi(H, W, S, T=0.9, seed=3, row_seeds=rs, step=2,
+                                            mask=mask)
+    assert_parity(got.ravel(), idx.ravel(), best.ravel(), second.ravel(), "multi S=%d" % S)
+    first = binding.fs_sample_ex(Hd, Wd, temperature=0.9, seed=3, row_seeds=rs.to(dev), step=2,
+                                 mask_bits=mask.to(dev)).cpu().numpy()
+    assert np.array_equal(got[:, 0], first)
+
+
+def test_multi_sample_full_vocab(dev, oracle):
+    wl = synth.WORKLOADS["qwen3-8b"]
+    B, S = 64, 4
+    Wd = synth.make_weight(wl.V, wl.d, wl.w_std, device=dev)
+    Hd = synth.make_hidden(B, wl.d, device=dev)
+    rs = synth.make_row_seeds(B)
+    got = binding.fs_sample_multi(Hd, Wd, S, temperature=wl.temperature, row_seeds=rs.to(dev),
+                                  step=7).cpu().numpy()
+    rows = np.array([0, 31, 63], dtype=np.int32)
+    idx, best, second = oracle.sample_multi(Hd.cpu(), Wd.cpu(), S, T=wl.temperature,
+                                            row_seeds=rs, step=7, rows=rows)
+    assert_parity(got[rows].ravel(), idx.ravel(), best.ravel(), second.ravel(), "multi full")
+    del Wd
+    torch.cuda.empty_cache()
+
+
+def test_one_workspace_serves_every_kind_of_call(dev, oracle):
+    """Grouped, multi-sample and flat calls in any order on one workspace."""
+    B, d, V = 32, 64, 5000
+    H, W, Hd, Wd = rand_inputs(B, d, V, seed=99)
+    ws = torch.zeros(max(binding.fs_workspace_bytes(B, V, 64), binding.fs_workspace_bytes_multi(B, V, 64)),
+                     dtype=torch.uint8, device=dev)
+    for rep in range(2):
+        g = binding.fs_sample_grouped(Hd, Wd, 64, temperature=1.0, seed=1, step=rep, workspace=ws)
+        m = binding.fs_sample_multi(Hd, Wd, 64, temperature=1.0, seed=1, step=rep, workspace=ws)
+        f = binding.fs_sample_ex(Hd, Wd, temperature=1.0, seed=1, step=rep, workspace=ws)
+        assert torch.equal(m[:, 0], f)
+        idx, best, second = oracle.sample_multi(H, W, 64, T=1.0, seed=1, step=rep, rows=[0, 31])
+        assert_parity(m.cpu().numpy()[[0, 31]].ravel(), idx.ravel(), best.ravel(), second.ravel(),
+                      "multi after grouped")
+        assert g.shape == (B,)

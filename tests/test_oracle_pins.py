@@ -423,3 +423,31 @@ def test_same_seed_same_tokens_and_steps_differ(oracle):
     rows = np.array([5, 0, 31], dtype=np.int32)
     sub, _, _ = oracle.sample(H, W, T=0.7, row_seeds=rs, step=17, rows=rows)
     assert np.array_equal(sub, a[rows])
+
+
+# --------------------------------------------------------------------------
+# Several samples per row (readus.org page, API: number of samples)
+# --------------------------------------------------------------------------
+
+def test_multi_sample_first_is_single_sample(oracle):
+    B, d, V = 12, 32, 300
+    H = synth.make_hidden(B, d, seed=121)
+    W = synth.make_weight(V, d, 0.5, seed=122)
+    single, b1, _ = oracle.sample(H, W, T=0.8, seed=5, step=3)
+    multi, mb, _ = oracle.sample_multi(H, W, 6, T=0.8, seed=5, step=3)
+    assert np.array_equal(multi[:, 0], single) and np.array_equal(mb[:, 0], b1)
+    # the samples use distinct noise: they are not all equal
+    assert (multi != multi[:, :1]).any()
+
+
+def test_multi_samples_are_softmax_draws(oracle):
+    """All S samples of one row over many steps follow the exact softmax."""
+    V, d, S, steps = 64, 32, 16, 4000
+    H = synth.make_hidden(1, d, seed=131)
+    W = synth.make_weight(V, d, 0.35, seed=132)
+    counts = np.zeros(V, dtype=np.int64)
+    for step in range(0, steps, 1):
+        idx, _, _ = oracle.sample_multi(H, W, S, T=1.2, seed=9, step=step)
+        counts += np.bincount(idx.ravel(), minlength=V)
+    p = _softmax(oracle.logits(H, W)[0] / 1.2)
+    assert _chi2_pvalue(counts, p) > 1e-3
