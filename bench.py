@@ -382,6 +382,7 @@ def run_gpu(args, world, rank, local):
                                                   peak_kind, W)
         result["unfused"] = unfused_point(torch, binding, synth, W, wl, dev, stream, B)
         result["multi_sample"] = multi_point(torch, binding, synth, W, wl, dev, stream, B)
+        result["cuda_graph"] = graph_point(torch, binding, synth, W, wl, dev, B)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(H, W, wl, B, rs)
     return result
@@ -449,6 +450,45 @@ def multi_point(torch, binding, synth, W, wl, dev, stream, B, S=4, steps=100):
     region_ms, _ = time_calls(step, steps, 10, stream)
     return {"B": B, "num_samples": S, "us_per_call": round(region_ms * 1e3 / steps, 3),
             "samples_per_s": round(B * S / (region_ms * 1e-3 / steps), 1)}
+
+
+def graph_point(torch, binding, synth, W, wl, dev, B, calls=10, replays=30):
+    """The same step captured ten calls at a time in a CUDA graph, to separate
+    the kernel from per-call launch overhead."""
+    try:
+        H = synth.make_hidden(B, wl.d, device=dev)
+        rs = synth.make_row_seeds(B, device=dev) if wl.per_row_seeds else None
+        out = torch.empty(B, dtype=torch.int32, device=dev)
+        ws = torch.zeros(binding.fs_workspace_bytes(B, wl.V, 0), dtype=torch.uint8, device=dev)
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            for i in range(3):
+                binding.fs_sample_ex(H, W, temperature=wl.temperature, row_seeds=rs, step=i,
+                                     out_idx=out, workspace=ws, stream=s)
+        s.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            for i in range(calls):
+                binding.fs_sample_ex(H, W, temperature=wl.temperature, row_seeds=rs, step=i,
+                                     out_idx=out, workspace=ws, stream=s)
+        torch.cuda.synchronize()
+        time.sleep(1.0)
+        for _ in range(2):
+            g.replay()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(replays):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / (replays * calls)
+        del g
+        return {"B": B, "us_per_call": round(us, 3), "calls_per_graph": calls}
+    except Exception as exc:   # report, do not break the bench line
+        return {"B": B, "us_per_call": None, "error": str(exc)[:200]}
 
 
 def unfused_point(torch, binding, synth, W, wl, dev, stream, B, steps=100):

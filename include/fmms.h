@@ -152,6 +152,35 @@ fs_status fs_sample_multi(const void *H, const void *W, int B, int d, int V,
                           void *workspace, size_t workspace_bytes,
                           fs_stream_t stream);
 
+/* Online grouped sampling, one group at a time (readus.org page, "Group
+ * Gumbel Max": only one group of the vocabulary needs to be on chip at a
+ * time, its "captain" kept and the rest discarded; abstract: grouped variants
+ * for online settings are exact by hierarchical factorisation).  W_g holds
+ * rows [vocab_offset, vocab_offset + V_g) of a head with V_total rows
+ * (vocab_offset % 8 == 0), delivered separately from the other groups.
+ * Writes per row b the group's summary (max x + g, its global token, lse of
+ * the allowed x = l / T) to out_summary[b] (device fs_group_summary [B]).
+ * Token noise, mask and indices are global, as in fs_sample_grouped.  The
+ * workspace needs fs_workspace_bytes_summary(B, V_g) bytes. */
+fs_status fs_summarize_group(const void *H, const void *W_g, int B, int d,
+                           int V_g, int vocab_offset, int V_total,
+                           float temperature, uint64_t seed,
+                           const uint64_t *row_seeds, uint32_t step,
+                           const uint32_t *mask_bits,
+                           fs_group_summary *out_summary, void *workspace,
+                           size_t workspace_bytes, fs_stream_t stream);
+
+/* Merges G group summaries (device fs_group_summary [G][B]: the summaries of
+ * group g at [g][0..B)) by Group-Gumbel-Max: g* = argmax_g (lse_g + gumbel_g)
+ * with gumbel_g from noise word (g & 3) of Philox(key, (g >> 2, b, step, 1)),
+ * ties to the smaller g; out_idx[b] = the argmax of group g*, or -1 when every
+ * group of the row is fully masked.  With the contiguous groups
+ * [floor(g V/G), floor((g+1) V/G)) this is fs_sample_grouped (the group lse
+ * may differ in the last fp32 bits, which can change g* only at near ties). */
+fs_status fs_merge_groups(const fs_group_summary *summaries, int G, int B,
+                          uint64_t seed, const uint64_t *row_seeds,
+                          uint32_t step, int32_t *out_idx, fs_stream_t stream);
+
 /* One vocabulary shard of a tensor-parallel LM head (readus.org page,
  * "distributed FlashSampling": each GPU is one group of the vocabulary and
  * contributes only its winning index and score; abstract: the argmax
@@ -223,6 +252,9 @@ size_t fs_workspace_bytes(int B, int V, int G);
 /* Workspace bytes of fs_sample_multi on the current device (0 on invalid
  * sizes). */
 size_t fs_workspace_bytes_multi(int B, int V, int num_samples);
+
+/* Workspace bytes of fs_summarize_group for a group of V_g rows. */
+size_t fs_workspace_bytes_summary(int B, int V_g);
 
 /* Reads (synchronously, after the stream drains) and clears the device-side
  * status word of a workspace (NULL = the library-owned one on the current

@@ -11,7 +11,8 @@ _BINDING_NAMES = ("FmmsError", "fs_sample", "fs_sample_ex", "fs_sample_grouped",
                   "fs_status_string", "fs_philox4x32_10", "fs_gumbel", "fs_plan_tiles",
                   "library_path", "load_library", "fs_sample_noalloc",
                   "fs_test_stalled_sample", "fs_sample_shard_keys", "fs_keys_to_tokens",
-                  "fs_sample_multi", "fs_workspace_bytes_multi")
+                  "fs_sample_multi", "fs_workspace_bytes_multi", "fs_summarize_group",
+                  "fs_merge_groups", "fs_workspace_bytes_summary")
 
 
 def __getattr__(name):

@@ -22,7 +22,8 @@ EXPORTED = ("fs_sample", "fs_sample_ex", "fs_sample_grouped", "fs_sample_unfused
             "fs_sample_host", "fs_workspace_bytes", "fs_device_status", "fs_status_string",
             "fs_philox4x32_10", "fs_gumbel", "fs_plan_tiles", "fs_plan_group_ctas",
             "fs_sample_noalloc", "fs_test_stalled_sample", "fs_sample_shard_keys",
-            "fs_keys_to_tokens", "fs_sample_multi", "fs_workspace_bytes_multi")
+            "fs_keys_to_tokens", "fs_sample_multi", "fs_workspace_bytes_multi",
+            "fs_summarize_group", "fs_merge_groups", "fs_workspace_bytes_summary")
 
 
 class FmmsError(RuntimeError):
@@ -66,6 +67,10 @@ def load_library():
     lib.fs_sample_multi.argtypes = common + [i32, f32, u64, vp, u32, vp, vp, vp, sz, vp]
     lib.fs_workspace_bytes_multi.argtypes = [i32, i32, i32]
     lib.fs_workspace_bytes_multi.restype = sz
+    lib.fs_summarize_group.argtypes = common + [i32, i32, f32, u64, vp, u32, vp, vp, vp, sz, vp]
+    lib.fs_merge_groups.argtypes = [vp, i32, i32, u64, vp, u32, vp, vp]
+    lib.fs_workspace_bytes_summary.argtypes = [i32, i32]
+    lib.fs_workspace_bytes_summary.restype = sz
     lib.fs_workspace_bytes.argtypes = [i32, i32, i32]
     lib.fs_workspace_bytes.restype = sz
     lib.fs_device_status.argtypes = [vp, sz, vp]
@@ -78,7 +83,8 @@ def load_library():
     lib.fs_plan_group_ctas.argtypes = [i32, i32, i32, i32, ctypes.POINTER(ctypes.c_int),
                                        ctypes.POINTER(ctypes.c_int)]
     for name in EXPORTED:
-        if name not in ("fs_workspace_bytes", "fs_workspace_bytes_multi", "fs_status_string"):
+        if name not in ("fs_workspace_bytes", "fs_workspace_bytes_multi",
+                        "fs_workspace_bytes_summary", "fs_status_string"):
             getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -362,3 +368,39 @@ def fs_sample_multi(H, W, num_samples, temperature=1.0, seed=0, row_seeds=None, 
 
 def fs_workspace_bytes_multi(B, V, num_samples):
     return int(load_library().fs_workspace_bytes_multi(int(B), int(V), int(num_samples)))
+
+
+def fs_summarize_group(H, W_g, vocab_offset, V_total, temperature=1.0, seed=0, row_seeds=None,
+                     step=0, mask_bits=None, out_summary=None, workspace=None, stream=None):
+    """Summary of one group (rows [vocab_offset, vocab_offset + V_g) of the head):
+    float32 [B, 3] records (max score, argmax as int32 bits, lse)."""
+    lib = load_library()
+    B, d, Vg = _check_operands(H, W_g)
+    row_seeds = _opt_dev(row_seeds, torch.int64, B, "row_seeds", H.device)
+    mask_bits = _opt_dev(mask_bits, torch.int32, B * ((V_total + 31) // 32), "mask_bits",
+                         H.device)
+    if out_summary is None:
+        out_summary = torch.empty(B, 3, dtype=torch.float32, device=H.device)
+    _opt_dev(out_summary, torch.float32, B * 3, "out_summary", H.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.fs_summarize_group(_ptr(H), _ptr(W_g), B, d, Vg, int(vocab_offset), int(V_total),
+                                float(temperature), _seed(seed), _ptr(row_seeds), int(step),
+                                _ptr(mask_bits), _ptr(out_summary), _ptr(workspace), ws_bytes,
+                                _stream(stream)), "fs_summarize_group")
+    return out_summary
+
+
+def fs_merge_groups(summaries, seed=0, row_seeds=None, step=0, out_idx=None, stream=None):
+    """Tokens [B] from group summaries [G, B, 3] (float32 records)."""
+    lib = load_library()
+    G, B = summaries.shape[0], summaries.shape[1]
+    row_seeds = _opt_dev(row_seeds, torch.int64, B, "row_seeds", summaries.device)
+    out_idx = _out(out_idx, B, summaries.device)
+    _check(lib.fs_merge_groups(_ptr(summaries.contiguous()), int(G), int(B), _seed(seed),
+                               _ptr(row_seeds), int(step), _ptr(out_idx), _stream(stream)),
+           "fs_merge_groups")
+    return out_idx
+
+
+def fs_workspace_bytes_summary(B, V_g):
+    return int(load_library().fs_workspace_bytes_summary(int(B), int(V_g)))

@@ -155,7 +155,7 @@ struct Workspace {
   unsigned long long *gkeys;
 };
 
-Workspace carve(void *ws, int B, int G, int num_ctas, int samples) {
+Workspace carve(void *ws, int B, int G, int num_ctas, int samples, bool grouped) {
   char *b = static_cast<char *>(ws);
   (void)samples;
   const size_t keys_bytes = static_cast<size_t>(fmms::kWsKeysRegion);  // fixed layout
@@ -164,17 +164,17 @@ Workspace carve(void *ws, int B, int G, int num_ctas, int samples) {
   w.ticket = reinterpret_cast<unsigned int *>(b + 4);
   w.keys = reinterpret_cast<unsigned long long *>(b + fmms::kWsHeader);
   w.partials = reinterpret_cast<fmms::GroupPartial *>(b + fmms::kWsHeader + keys_bytes);
-  w.gkeys = fmms::ws_gkeys_bytes(B, G) > 0
+  w.gkeys = (grouped && fmms::ws_gkeys_bytes(B, G) > 0)
                 ? reinterpret_cast<unsigned long long *>(
                       b + fmms::kWsHeader + keys_bytes + fmms::ws_partials_bytes(B, G, num_ctas))
                 : nullptr;
   return w;
 }
 
-fs_status resolve_workspace(DeviceState *st, const Schedule &sch, int B, int samples, void *ws,
-                            size_t ws_bytes, void **out) {
+fs_status resolve_workspace(DeviceState *st, const Schedule &sch, int B, int samples,
+                            bool grouped, void *ws, size_t ws_bytes, void **out) {
   const size_t need =
-      static_cast<size_t>(fmms::workspace_bytes_for(B, sch.G, sch.num_ctas, samples));
+      static_cast<size_t>(fmms::workspace_bytes_for(B, sch.G, sch.num_ctas, samples, grouped));
   if (ws == nullptr) {
     fs_status s = grow(&st->ws, &st->ws_bytes, need);
     if (s != FS_OK) return s;
@@ -224,9 +224,10 @@ fs_status run_locked(int mode, const void *H, const void *W, int B, int d, int V
   const Schedule sch = fmms::make_schedule(V, mode == fmms::kModeGrouped ? G : 1, st->sms);
   void *wsp = nullptr;
   const int S = shard.num_samples;
-  s = resolve_workspace(st, sch, B, S, ws, ws_bytes, &wsp);
+  const bool grouped = mode == fmms::kModeGrouped;
+  s = resolve_workspace(st, sch, B, S, grouped, ws, ws_bytes, &wsp);
   if (s != FS_OK) return s;
-  const Workspace w = carve(wsp, B, sch.G, sch.num_ctas, S);
+  const Workspace w = carve(wsp, B, sch.G, sch.num_ctas, S, grouped);
 
   CUtensorMap tw, tw8;
   if ((s = tensor_map(&tw, W, d, V, fmms::kTileM)) != FS_OK) return s;
@@ -279,7 +280,7 @@ fs_status run_locked(int mode, const void *H, const void *W, int B, int d, int V
       m.seed = seed;
       m.row_seeds = row_seeds;
       m.step = step;
-      m.out_idx = out_idx + b0;
+      m.out_idx = out_idx ? out_idx + b0 : nullptr;
       m.summary = summary ? static_cast<void *>(summary + static_cast<size_t>(b0) * sch.G) : nullptr;
       if (fmms::launch_group_merge(m, stream) != cudaSuccess) return FS_ERR_CUDA;
     } else if (mode == fmms::kModeLogits) {
@@ -461,7 +462,49 @@ size_t fs_workspace_bytes(int B, int V, int G) {
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return 0;
   const Schedule sch = fmms::make_schedule(V, G, sms);
-  return static_cast<size_t>(fmms::workspace_bytes_for(B, sch.G, sch.num_ctas));
+  return static_cast<size_t>(fmms::workspace_bytes_for(B, sch.G, sch.num_ctas, 1, G >= 2));
+}
+
+size_t fs_workspace_bytes_summary(int B, int V_g) {
+  if (B < 1 || V_g < 1) return 0;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 0;
+  const Schedule sch = fmms::make_schedule(V_g, 1, sms);
+  return static_cast<size_t>(fmms::workspace_bytes_for(B, 1, sch.num_ctas, 1, true));
+}
+
+fs_status fs_summarize_group(const void *H, const void *W_g, int B, int d, int V_g,
+                           int vocab_offset, int V_total, float temperature, uint64_t seed,
+                           const uint64_t *row_seeds, uint32_t step, const uint32_t *mask_bits,
+                           fs_group_summary *out_summary, void *workspace, size_t workspace_bytes,
+                           fs_stream_t stream) {
+  fs_status s = validate(H, W_g, B, d, V_g, temperature, out_summary);
+  if (s != FS_OK) return s;
+  if (vocab_offset < 0 || (vocab_offset % fmms::kGranule) != 0 || V_total < 1 ||
+      static_cast<int64_t>(vocab_offset) + V_g > V_total)
+    return FS_ERR_INVALID_ARG;
+  ShardOpts opts;
+  opts.vocab_offset = vocab_offset;
+  opts.V_total = V_total;
+  std::lock_guard<std::mutex> lock(g_mu);
+  return run_locked(fmms::kModeGrouped, H, W_g, B, d, V_g, 1, temperature, seed, row_seeds, step,
+                    mask_bits, nullptr, out_summary, nullptr, workspace, workspace_bytes,
+                    static_cast<cudaStream_t>(stream), opts);
+}
+
+fs_status fs_merge_groups(const fs_group_summary *summaries, int G, int B, uint64_t seed,
+                          const uint64_t *row_seeds, uint32_t step, int32_t *out_idx,
+                          fs_stream_t stream) {
+  if (!summaries || !out_idx || G < 1 || B < 1) return FS_ERR_INVALID_ARG;
+  DeviceState *st = nullptr;
+  fs_status s = get_device(&st);
+  if (s != FS_OK) return s;
+  return fmms::launch_merge_summaries(summaries, G, B, seed, row_seeds, step, out_idx,
+                                      static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? FS_OK
+             : FS_ERR_CUDA;
 }
 
 fs_status fs_device_status(void *workspace, size_t workspace_bytes, fs_stream_t stream) {

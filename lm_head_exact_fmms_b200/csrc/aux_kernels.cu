@@ -86,7 +86,54 @@ __global__ void __launch_bounds__(128) group_merge_kernel(const MergeParams m) {
   const int gwin = key_token(packed);
   const unsigned long long tok =
       __shfl_sync(0xffffffffu, best_tok, gwin < 0 ? 0 : (gwin & 31));
-  if (lane == 0) m.out_idx[b] = gwin < 0 ? -1 : key_token(tok);
+  if (lane == 0 && m.out_idx != nullptr) m.out_idx[b] = gwin < 0 ? -1 : key_token(tok);
+}
+
+// Online grouped sampling: Group-Gumbel-Max over summaries [G][B] produced
+// one group at a time; the same group noise (tag 1) as the fused grouped path.
+__global__ void __launch_bounds__(128)
+    merge_summaries_kernel(const fs_group_summary *summaries, int G, int B, uint64_t seed,
+                           const uint64_t *row_seeds, uint32_t step, int32_t *out_idx) {
+  const int b = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+  const int lane = threadIdx.x & 31;
+  if (b >= B) return;
+  const uint32_t bg = static_cast<uint32_t>(b);
+  const uint64_t k64 = row_seeds ? row_seeds[bg] : seed;
+  float best_key = -INFINITY;
+  int best_g = -1;
+  int best_tok = -1;
+  for (int g = lane; g < G; g += 32) {
+    const fs_group_summary sm = summaries[static_cast<size_t>(g) * B + b];
+    if (sm.lse == -INFINITY || sm.argmax < 0) continue;
+    const Philox4 ph = philox4x32_10(static_cast<uint32_t>(g) >> 2, bg, step, 1u,
+                                     static_cast<uint32_t>(k64), static_cast<uint32_t>(k64 >> 32));
+    const uint32_t w = (g & 3) == 0 ? ph.w0 : (g & 3) == 1 ? ph.w1 : (g & 3) == 2 ? ph.w2 : ph.w3;
+    const float kg = sm.lse + gumbel_from_u32(w);
+    if (best_g < 0 || kg > best_key) {
+      best_key = kg;
+      best_g = g;
+      best_tok = sm.argmax;
+    }
+  }
+  uint64_t packed = best_g < 0 ? 0ull : pack_key(__float_as_uint(best_key), best_g);
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+    const uint64_t o = __shfl_xor_sync(0xffffffffu, packed, off);
+    packed = o > packed ? o : packed;
+  }
+  const int gwin = key_token(packed);
+  const int tok = __shfl_sync(0xffffffffu, best_tok, gwin < 0 ? 0 : (gwin & 31));
+  if (lane == 0) out_idx[b] = gwin < 0 ? -1 : tok;
+}
+
+cudaError_t launch_merge_summaries(const void *summaries, int G, int B, uint64_t seed,
+                                   const uint64_t *row_seeds, uint32_t step, int32_t *out_idx,
+                                   cudaStream_t stream) {
+  const int threads = 128;
+  const int blocks = (B * 32 + threads - 1) / threads;
+  merge_summaries_kernel<<<blocks, threads, 0, stream>>>(
+      static_cast<const fs_group_summary *>(summaries), G, B, seed, row_seeds, step, out_idx);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_group_merge(const MergeParams &m, cudaStream_t stream) {

@@ -194,19 +194,22 @@ constexpr int kWsKeysRegion = kMaxSamples * kWsKeys;
 
 FS_HD int64_t ws_partials_bytes(int B, int G, int num_ctas) {
   const int64_t rows = B < kMaxBN ? B : kMaxBN;
-  return G > 1 ? (int64_t)(num_ctas + G - 1) * rows * (int64_t)sizeof(GroupPartial) : 0;
+  return (int64_t)(num_ctas + G - 1) * rows * (int64_t)sizeof(GroupPartial);
 }
 
 FS_HD int64_t ws_gkeys_bytes(int B, int G) {
   const int64_t rows = B < kMaxBN ? B : kMaxBN;
-  return (G > 1 && G <= kMaxPublishedGroups) ? (int64_t)G * rows * 8 : 0;
+  return G <= kMaxPublishedGroups ? (int64_t)G * rows * 8 : 0;
 }
 
-FS_HD int64_t workspace_bytes_for(int B, int G, int num_ctas, int samples = 1) {
+// Bytes of workspace for a flat call with `samples` samples, or a grouped call
+// (grouped = true) with G >= 1 groups.
+FS_HD int64_t workspace_bytes_for(int B, int G, int num_ctas, int samples = 1,
+                                  bool grouped = false) {
   const int64_t bytes =
-      G > 1 ? (int64_t)kWsHeader + kWsKeysRegion + ws_partials_bytes(B, G, num_ctas) +
-                  ws_gkeys_bytes(B, G)
-            : (int64_t)kWsHeader + (int64_t)kWsKeys * (samples < 1 ? 1 : samples);
+      grouped ? (int64_t)kWsHeader + kWsKeysRegion + ws_partials_bytes(B, G, num_ctas) +
+                    ws_gkeys_bytes(B, G)
+              : (int64_t)kWsHeader + (int64_t)kWsKeys * (samples < 1 ? 1 : samples);
   return (bytes + 255) / 256 * 256;
 }
 

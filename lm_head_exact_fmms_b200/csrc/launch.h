@@ -47,6 +47,11 @@ struct SampleLogitsParams {
 };
 cudaError_t launch_sample_logits(const SampleLogitsParams &s, cudaStream_t stream);
 
+// Group-Gumbel-Max over per-group summaries [G][B] (fs_group_summary records).
+cudaError_t launch_merge_summaries(const void *summaries, int G, int B, uint64_t seed,
+                                   const uint64_t *row_seeds, uint32_t step, int32_t *out_idx,
+                                   cudaStream_t stream);
+
 // Decodes packed keys (XOR 2^63, as fs_sample_shard_keys writes them) to tokens.
 cudaError_t launch_keys_to_tokens(const long long *keys, int B, int32_t *out_idx,
                                   cudaStream_t stream);

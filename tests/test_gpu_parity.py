@@ -444,3 +444,38 @@ def test_one_workspace_serves_every_kind_of_call(dev, oracle):
         assert_parity(m.cpu().numpy()[[0, 31]].ravel(), idx.ravel(), best.ravel(), second.ravel(),
                       "multi after grouped")
         assert g.shape == (B,)
+
+
+# ------------------------------------------------ online grouped sampling
+@pytest.mark.parametrize("B,V,G,masked", [(16, 6000, 3, False), (64, 8192, 8, True),
+                                          (300, 4000, 5, True)])
+def test_online_groups_match_fused_grouped(dev, oracle, B, V, G, masked):
+    d = 128
+    H, W, Hd, Wd = rand_inputs(B, d, V, seed=V + G)
+    mask = synth.make_mask(B, V, 0.5, seed=G) if masked else None
+    md = mask.to(dev) if masked else None
+    rs = synth.make_row_seeds(B).to(dev)
+    bounds = [(g * V) // G for g in range(G + 1)]
+    assert all(b % 8 == 0 for b in bounds)
+    summ = torch.empty(G, B, 3, dtype=torch.float32, device=dev)
+    for g in range(G):
+        lo, hi = bounds[g], bounds[g + 1]
+        binding.fs_summarize_group(Hd, Wd[lo:hi].contiguous(), lo, V, temperature=0.8, seed=7,
+                                   row_seeds=rs, step=1, mask_bits=md, out_summary=summ[g])
+    got = binding.fs_merge_groups(summ, seed=7, row_seeds=rs, step=1).cpu().numpy()
+    fused = binding.fs_sample_grouped(Hd, Wd, G, temperature=0.8, seed=7, row_seeds=rs, step=1,
+                                      mask_bits=md).cpu().numpy()
+    idx, o_summ, margin = oracle.sample_grouped(H, W, G, T=0.8, seed=7, row_seeds=rs.cpu(),
+                                                step=1, mask=mask)
+    s = summ.cpu()
+    lse = s[:, :, 2].numpy().T.astype(np.float64)
+    arg = s[:, :, 1].contiguous().view(torch.int32).numpy().T
+    fin = np.isfinite(o_summ[:, :, 2])
+    assert np.array_equal(np.isfinite(lse), fin)
+    assert np.allclose(lse[fin], o_summ[:, :, 2][fin], rtol=1e-5, atol=1e-4)
+    assert np.array_equal(arg[fin], o_summ[:, :, 1][fin].astype(np.int32)) or \
+        (arg[fin] != o_summ[:, :, 1][fin]).mean() < 0.01
+    for b in np.flatnonzero(got != idx):
+        scale = TIE_REL * (1 + abs(o_summ[b, :, 0].max()))
+        assert margin[b, 0] <= scale or margin[b, 1] <= scale, (b, got[b], idx[b])
+    assert (got == fused).mean() > 0.98
