@@ -383,6 +383,7 @@ def run_gpu(args, world, rank, local):
         result["unfused"] = unfused_point(torch, binding, synth, W, wl, dev, stream, B)
         result["multi_sample"] = multi_point(torch, binding, synth, W, wl, dev, stream, B)
         result["cuda_graph"] = graph_point(torch, binding, synth, W, wl, dev, B)
+        result["top_k"] = topk_point(torch, binding, synth, W, wl, dev, stream, B)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(H, W, wl, B, rs)
     return result
@@ -489,6 +490,22 @@ def graph_point(torch, binding, synth, W, wl, dev, B, calls=10, replays=30):
         return {"B": B, "us_per_call": round(us, 3), "calls_per_graph": calls}
     except Exception as exc:   # report, do not break the bench line
         return {"B": B, "us_per_call": None, "error": str(exc)[:200]}
+
+
+def topk_point(torch, binding, synth, W, wl, dev, stream, B, K=50, steps=100):
+    """Top-k sampling (two kernels: fp32 logits to HBM, then radix select)."""
+    H = synth.make_hidden(B, wl.d, device=dev)
+    rs = synth.make_row_seeds(B, device=dev) if wl.per_row_seeds else None
+    out = torch.empty(B, dtype=torch.int32, device=dev)
+    logits = torch.empty(B, wl.V, dtype=torch.float32, device=dev)
+
+    def step(i):
+        binding.fs_sample_topk(H, W, K, temperature=wl.temperature, seed=0, row_seeds=rs, step=i,
+                               out_idx=out, logits=logits, stream=stream)
+
+    region_ms, _ = time_calls(step, steps, 10, stream)
+    return {"B": B, "K": K, "us_per_call": round(region_ms * 1e3 / steps, 3),
+            "launches_per_call": 2}
 
 
 def unfused_point(torch, binding, synth, W, wl, dev, stream, B, steps=100):

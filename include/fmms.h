@@ -209,6 +209,23 @@ fs_status fs_sample_shard_keys(const void *H, const void *W_shard, int B, int d,
 fs_status fs_keys_to_tokens(const int64_t *keys, int B, int32_t *out_idx,
                             fs_stream_t stream);
 
+/* Top-k sampling (readus.org page, "Top-K and masking": a fast prefilter
+ * isolates the candidates, then exact Gumbel-max runs on that subset).  The
+ * candidates of row b are its K allowed tokens with the largest logits l
+ * (ties toward the smaller index; every allowed token if there are fewer),
+ * and the token is the argmax over them of x + g with the same noise as
+ * fs_sample_ex, so K >= V gives the fs_sample_ex token.  Two kernels: the
+ * matmul writes fp32 logits to `logits` (device [B][V], caller-owned, as in
+ * fs_sample_unfused), then one block per row selects the K-th largest logit
+ * exactly (radix select over the order-preserving bits) and samples.  K >= 1;
+ * other arguments as fs_sample_ex. */
+fs_status fs_sample_topk(const void *H, const void *W, int B, int d, int V,
+                         int K, float temperature, uint64_t seed,
+                         const uint64_t *row_seeds, uint32_t step,
+                         const uint32_t *mask_bits, int32_t *out_idx,
+                         float *logits, void *workspace, size_t workspace_bytes,
+                         fs_stream_t stream);
+
 /* End-to-end call with HOST buffers: H_host (bf16 [B, d]) and out_idx_host
  * (int32 [B]) are host pointers (page-locked for the copies to be
  * asynchronous); W and row_seeds/mask_bits stay device pointers.  Enqueues

@@ -23,7 +23,8 @@ EXPORTED = ("fs_sample", "fs_sample_ex", "fs_sample_grouped", "fs_sample_unfused
             "fs_philox4x32_10", "fs_gumbel", "fs_plan_tiles", "fs_plan_group_ctas",
             "fs_sample_noalloc", "fs_test_stalled_sample", "fs_sample_shard_keys",
             "fs_keys_to_tokens", "fs_sample_multi", "fs_workspace_bytes_multi",
-            "fs_summarize_group", "fs_merge_groups", "fs_workspace_bytes_summary")
+            "fs_summarize_group", "fs_merge_groups", "fs_workspace_bytes_summary",
+            "fs_sample_topk")
 
 
 class FmmsError(RuntimeError):
@@ -71,6 +72,7 @@ def load_library():
     lib.fs_merge_groups.argtypes = [vp, i32, i32, u64, vp, u32, vp, vp]
     lib.fs_workspace_bytes_summary.argtypes = [i32, i32]
     lib.fs_workspace_bytes_summary.restype = sz
+    lib.fs_sample_topk.argtypes = common + [i32, f32, u64, vp, u32, vp, vp, vp, vp, sz, vp]
     lib.fs_workspace_bytes.argtypes = [i32, i32, i32]
     lib.fs_workspace_bytes.restype = sz
     lib.fs_device_status.argtypes = [vp, sz, vp]
@@ -404,3 +406,22 @@ def fs_merge_groups(summaries, seed=0, row_seeds=None, step=0, out_idx=None, str
 
 def fs_workspace_bytes_summary(B, V_g):
     return int(load_library().fs_workspace_bytes_summary(int(B), int(V_g)))
+
+
+def fs_sample_topk(H, W, K, temperature=1.0, seed=0, row_seeds=None, step=0, mask_bits=None,
+                   out_idx=None, logits=None, workspace=None, stream=None):
+    """Top-k sample: Gumbel-max over each row's K largest allowed logits."""
+    lib = load_library()
+    B, d, V = _check_operands(H, W)
+    row_seeds = _opt_dev(row_seeds, torch.int64, B, "row_seeds", H.device)
+    mask_bits = _opt_dev(mask_bits, torch.int32, B * ((V + 31) // 32), "mask_bits", H.device)
+    out_idx = _out(out_idx, B, H.device)
+    if logits is None:
+        logits = torch.empty(B, V, dtype=torch.float32, device=H.device)
+    _opt_dev(logits, torch.float32, B * V, "logits", H.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.fs_sample_topk(_ptr(H), _ptr(W), B, d, V, int(K), float(temperature), _seed(seed),
+                              _ptr(row_seeds), int(step), _ptr(mask_bits), _ptr(out_idx),
+                              _ptr(logits), _ptr(workspace), ws_bytes, _stream(stream)),
+           "fs_sample_topk")
+    return out_idx

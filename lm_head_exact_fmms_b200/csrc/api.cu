@@ -195,6 +195,7 @@ struct ShardOpts {
   int V_total = 0;              // full vocabulary (0: V); sets the mask row length
   long long *out_keys = nullptr;  // write packed keys instead of tokens
   int num_samples = 1;          // samples per row (flat mode)
+  int top_k = 0;                // logits mode: top-k selection instead of full sampling
 };
 
 // The fused path in all three modes, chunked over 256 batch rows.
@@ -299,7 +300,9 @@ fs_status run_locked(int mode, const void *H, const void *W, int B, int d, int V
       sp.ticket = w.ticket;
       sp.out_idx = out_idx + b0;
       sp.num_sms = st->sms;
-      if (fmms::launch_sample_logits(sp, stream) != cudaSuccess) return FS_ERR_CUDA;
+      const cudaError_t e = shard.top_k > 0 ? fmms::launch_topk_sample(sp, shard.top_k, stream)
+                                            : fmms::launch_sample_logits(sp, stream);
+      if (e != cudaSuccess) return FS_ERR_CUDA;
     }
   }
   return FS_OK;
@@ -463,6 +466,22 @@ size_t fs_workspace_bytes(int B, int V, int G) {
     return 0;
   const Schedule sch = fmms::make_schedule(V, G, sms);
   return static_cast<size_t>(fmms::workspace_bytes_for(B, sch.G, sch.num_ctas, 1, G >= 2));
+}
+
+fs_status fs_sample_topk(const void *H, const void *W, int B, int d, int V, int K,
+                         float temperature, uint64_t seed, const uint64_t *row_seeds,
+                         uint32_t step, const uint32_t *mask_bits, int32_t *out_idx,
+                         float *logits, void *workspace, size_t workspace_bytes,
+                         fs_stream_t stream) {
+  fs_status s = validate(H, W, B, d, V, temperature, out_idx);
+  if (s != FS_OK) return s;
+  if (!logits || K < 1) return FS_ERR_INVALID_ARG;
+  ShardOpts opts;
+  opts.top_k = K;
+  std::lock_guard<std::mutex> lock(g_mu);
+  return run_locked(fmms::kModeLogits, H, W, B, d, V, 1, temperature, seed, row_seeds, step,
+                    mask_bits, out_idx, nullptr, logits, workspace, workspace_bytes,
+                    static_cast<cudaStream_t>(stream), opts);
 }
 
 size_t fs_workspace_bytes_summary(int B, int V_g) {

@@ -223,6 +223,176 @@ cudaError_t launch_sample_logits(const SampleLogitsParams &s, cudaStream_t strea
 }
 
 // ---------------------------------------------------------------------------
+// Top-k sampling over fp32 logits [B][V] (readus.org page, "Top-K and
+// masking": a prefilter isolates the candidates, exact Gumbel-max runs on
+// them).  One block per row: an exact radix select finds the k-th largest
+// order-preserving key of the allowed logits (passes over bits 31-21, 20-10,
+// 9-0), then the candidates -- keys above it, and as many keys equal to it as
+// k allows, in index order -- get their noise and the Gumbel-max.
+// ---------------------------------------------------------------------------
+constexpr int kTopkThreads = 1024;
+constexpr int kTopkBins = 2048;
+
+__device__ __forceinline__ bool topk_allowed(const SampleLogitsParams &s, uint32_t bg, int v) {
+  if (s.mask == nullptr) return true;
+  return ((s.mask[static_cast<size_t>(bg) * s.mask_words + (v >> 5)] >> (v & 31)) & 1u) != 0;
+}
+
+// Block-wide exclusive scan of one int per thread (1024 threads); returns the
+// thread's prefix and writes the total to *total.
+__device__ __forceinline__ int block_exclusive_scan(int x, int *warp_sums, int *total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = x;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += y;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = warp_sums[lane];
+    int wi = w;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, wi, off);
+      if (lane >= off) wi += y;
+    }
+    warp_sums[lane] = wi - w;  // exclusive prefix of the warp totals
+    if (lane == 31) *total = wi;
+  }
+  __syncthreads();
+  const int r = warp_sums[warp] + incl - x;
+  __syncthreads();
+  return r;
+}
+
+__global__ void __launch_bounds__(kTopkThreads) topk_sample_kernel(const SampleLogitsParams s,
+                                                                   int K) {
+  __shared__ int hist[kTopkBins];
+  __shared__ int warp_sums[32];
+  __shared__ int sh_digit, sh_above, sh_total;
+  __shared__ uint64_t warp_best[32];
+  const int b = blockIdx.x;
+  const uint32_t bg = static_cast<uint32_t>(s.b_off + b);
+  const float *row = s.logits + static_cast<size_t>(b) * s.V;
+  const int lane = threadIdx.x & 31;
+
+  // ---- radix select of the k-th largest key among allowed logits
+  uint32_t prefix = 0, pmask = 0;
+  int k_rem = K;         // rank still to find inside the current prefix
+  int n_allowed = 0;
+  const int shifts[3] = {21, 10, 0};
+  const int widths[3] = {11, 11, 10};
+  for (int pass = 0; pass < 3; ++pass) {
+    const int shift = shifts[pass];
+    const uint32_t dmask = (1u << widths[pass]) - 1u;
+    for (int i = threadIdx.x; i < kTopkBins; i += kTopkThreads) hist[i] = 0;
+    __syncthreads();
+    for (int base = 0; base < s.V; base += kTopkThreads) {
+      const int v = base + threadIdx.x;
+      bool take = false;
+      uint32_t bin = 0;
+      if (v < s.V && topk_allowed(s, bg, v)) {
+        const uint32_t key = order_bits(__float_as_uint(row[v]));
+        if ((key & pmask) == prefix) {
+          take = true;
+          bin = (key >> shift) & dmask;
+        }
+      }
+      // warp-aggregated increments: lanes with the same bin add once
+      const unsigned active = __ballot_sync(0xffffffffu, take);
+      if (take) {
+        const unsigned same = __match_any_sync(active, bin);
+        if ((__ffs(same) - 1) == lane) atomicAdd(&hist[bin], __popc(same));
+      }
+    }
+    __syncthreads();
+    if (pass == 0) {
+      // allowed tokens in total
+      int c = 0;
+      for (int i = threadIdx.x; i < kTopkBins; i += kTopkThreads) c += hist[i];
+      int total;
+      block_exclusive_scan(c, warp_sums, &sh_total);
+      total = sh_total;
+      n_allowed = total;
+      if (n_allowed <= K) break;   // every allowed token is a candidate
+    }
+    // find the digit holding the k_rem-th largest: suffix sums from the top bin
+    {
+      // each thread owns two adjacent bins, scanned from the top
+      const int t = kTopkThreads - 1 - threadIdx.x;   // thread 0 holds the top bins
+      const int hi_bin = 2 * t + 1, lo_bin = 2 * t;
+      const int c_hi = hist[hi_bin], c_lo = hist[lo_bin];
+      int total;
+      const int above = block_exclusive_scan(c_hi + c_lo, warp_sums, &total);  // bins above mine
+      if (above < k_rem && above + c_hi >= k_rem) {
+        sh_digit = hi_bin;
+        sh_above = above;
+      } else if (above + c_hi < k_rem && above + c_hi + c_lo >= k_rem) {
+        sh_digit = lo_bin;
+        sh_above = above + c_hi;
+      }
+      __syncthreads();
+    }
+    prefix |= static_cast<uint32_t>(sh_digit) << shift;
+    pmask |= dmask << shift;
+    k_rem -= sh_above;
+    __syncthreads();
+  }
+  const bool all_allowed = n_allowed <= K;
+  // prefix is now the k-th largest key; k_rem of the keys equal to it are in.
+
+  // ---- candidates and Gumbel-max
+  const uint64_t k64 = s.row_seeds ? s.row_seeds[bg] : s.seed;
+  uint64_t best = 0ull;
+  int eq_seen = 0;   // keys equal to the threshold already passed, in index order
+  for (int base = 0; base < s.V; base += kTopkThreads) {
+    const int v = base + threadIdx.x;
+    bool ok = v < s.V && topk_allowed(s, bg, v);
+    uint32_t key = 0;
+    float l = 0.f;
+    if (ok) {
+      l = row[v];
+      key = order_bits(__float_as_uint(l));
+    }
+    bool cand = ok && (all_allowed || key > prefix);
+    const bool eq = ok && !all_allowed && key == prefix;
+    int n_eq;
+    const int rank = block_exclusive_scan(eq ? 1 : 0, warp_sums, &sh_total);
+    n_eq = sh_total;
+    if (eq && eq_seen + rank < k_rem) cand = true;
+    eq_seen += n_eq;
+    if (cand) {
+      const Philox4 ph = philox4x32_10(static_cast<uint32_t>(v) >> 2, bg, s.step, 0u,
+                                       static_cast<uint32_t>(k64), static_cast<uint32_t>(k64 >> 32));
+      const uint32_t w = (v & 3) == 0 ? ph.w0 : (v & 3) == 1 ? ph.w1 : (v & 3) == 2 ? ph.w2 : ph.w3;
+      const float sc = fmaf(l, s.inv_temp, gumbel_from_u32(w));
+      const uint64_t k = pack_key(__float_as_uint(sc), v);
+      best = k > best ? k : best;
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+    const uint64_t o = __shfl_xor_sync(0xffffffffu, best, off);
+    best = o > best ? o : best;
+  }
+  if (lane == 0) warp_best[threadIdx.x >> 5] = best;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint64_t r = 0ull;
+    for (int i = 0; i < kTopkThreads / 32; ++i) r = warp_best[i] > r ? warp_best[i] : r;
+    s.out_idx[b] = key_token(r);
+  }
+}
+
+cudaError_t launch_topk_sample(const SampleLogitsParams &s, int K, cudaStream_t stream) {
+  topk_sample_kernel<<<s.B, kTopkThreads, 0, stream>>>(s, K);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
 // Vocabulary shards: tokens from the reduced keys.
 // ---------------------------------------------------------------------------
 __global__ void keys_to_tokens_kernel(const long long *keys, int B, int32_t *out_idx) {

@@ -47,6 +47,9 @@ struct SampleLogitsParams {
 };
 cudaError_t launch_sample_logits(const SampleLogitsParams &s, cudaStream_t stream);
 
+// Top-k sampling over the fp32 logits: one block per row.
+cudaError_t launch_topk_sample(const SampleLogitsParams &s, int K, cudaStream_t stream);
+
 // Group-Gumbel-Max over per-group summaries [G][B] (fs_group_summary records).
 cudaError_t launch_merge_summaries(const void *summaries, int G, int B, uint64_t seed,
                                    const uint64_t *row_seeds, uint32_t step, int32_t *out_idx,

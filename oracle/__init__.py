@@ -52,6 +52,7 @@ def _load():
     lib.oracle_sample.argtypes = common + sample_args + [_i32p, _f64p, _f64p]
     lib.oracle_sample_grouped.argtypes = common + [ctypes.c_int] + sample_args + [_i32p, _f64p, _f64p]
     lib.oracle_sample_multi.argtypes = common + [ctypes.c_int] + sample_args + [_i32p, _f64p, _f64p]
+    lib.oracle_sample_topk.argtypes = common + [ctypes.c_int] + sample_args + [_i32p, _f64p, _f64p]
     lib.oracle_histogram.argtypes = common + [ctypes.c_int, ctypes.c_double, ctypes.c_uint64, _u64p,
                                               ctypes.c_int, _u32p, ctypes.c_uint32, ctypes.c_int64,
                                               _i64p]
@@ -180,6 +181,23 @@ def sample_multi(H, W, S, T=1.0, seed=0, row_seeds=None, step=0, mask=None, rows
                             int(seed), _ptr(rs, _u64p), int(step), _ptr(mk, _u32p),
                             _ptr(rows, _i32p), rows.size, _ptr(idx, _i32p), _ptr(best, _f64p),
                             _ptr(second, _f64p))
+    return idx, best, second
+
+
+def sample_topk(H, W, K, T=1.0, seed=0, row_seeds=None, step=0, mask=None, rows=None):
+    """Top-k sample of the listed rows: Gumbel-max over each row's k allowed
+    tokens with the largest logits (ties toward the smaller index).
+
+    Returns (idx int32 [n], best f64 [n], second f64 [n])."""
+    lib = _load()
+    H16, W16, B, d, V, rs, mk, rows = _sample_common(H, W, T, seed, row_seeds, step, mask, rows)
+    idx = np.empty(rows.size, dtype=np.int32)
+    best = np.empty(rows.size, dtype=np.float64)
+    second = np.empty(rows.size, dtype=np.float64)
+    lib.oracle_sample_topk(_ptr(H16, _u16p), _ptr(W16, _u16p), B, d, V, int(K), float(T),
+                           int(seed), _ptr(rs, _u64p), int(step), _ptr(mk, _u32p),
+                           _ptr(rows, _i32p), rows.size, _ptr(idx, _i32p), _ptr(best, _f64p),
+                           _ptr(second, _f64p))
     return idx, best, second
 
 

@@ -296,6 +296,73 @@ void oracle_sample_multi(const uint16_t *H, const uint16_t *W, int B, int d,
 }
 
 /* ------------------------------------------------------------------------ */
+/* Top-k sampling.                                                           */
+/* ------------------------------------------------------------------------ */
+
+/* Order of the candidate selection: larger logit first, then smaller index. */
+typedef struct {
+  double l;
+  int v;
+} oracle_lv;
+
+static int cmp_lv_desc(const void *a, const void *b) {
+  const oracle_lv *x = (const oracle_lv *)a, *y = (const oracle_lv *)b;
+  if (x->l > y->l) return -1;
+  if (x->l < y->l) return 1;
+  return (x->v < y->v) ? -1 : (x->v > y->v);
+}
+
+/* Top-k sampling (readus.org page, "Top-K and masking": a prefilter isolates
+ * the candidates, then exact Gumbel-max runs on that subset): the candidates
+ * of row b are its k allowed tokens with the largest logits (ties broken
+ * toward the smaller index; all allowed tokens if fewer than k), and the
+ * sample is the smallest-index argmax of x + g over them, with the same noise
+ * as flat sampling.  The logit l orders the candidates (T > 0 keeps the order
+ * of x = l / T). */
+void oracle_sample_topk(const uint16_t *H, const uint16_t *W, int B, int d,
+                        int V, int K, double T, uint64_t seed,
+                        const uint64_t *row_seeds, uint32_t step,
+                        const uint32_t *mask, const int32_t *rows, int nrows,
+                        int32_t *out_idx, double *out_best, double *out_second) {
+  (void)B;
+  double *l = (double *)malloc(sizeof(double) * (size_t)V);
+  double *s = (double *)malloc(sizeof(double) * (size_t)V);
+  oracle_lv *cand = (oracle_lv *)malloc(sizeof(oracle_lv) * (size_t)V);
+  for (int i = 0; i < nrows; ++i) {
+    int b = rows[i];
+    logits_row(H + (int64_t)b * d, W, d, V, l);
+    scores_from_logits(l, V, T, row_key(seed, row_seeds, b), step, b, mask, s);
+    int n = 0;
+    for (int v = 0; v < V; ++v)
+      if (token_allowed(mask, V, b, v)) {
+        cand[n].l = l[v];
+        cand[n].v = v;
+        ++n;
+      }
+    qsort(cand, (size_t)n, sizeof(oracle_lv), cmp_lv_desc);
+    int keep = n < K ? n : K;
+    int arg = -1;
+    double b1 = -INFINITY, b2 = -INFINITY;
+    for (int j = 0; j < keep; ++j) {
+      int v = cand[j].v;
+      if (arg < 0 || s[v] > b1 || (s[v] == b1 && v < arg)) {
+        if (arg >= 0) b2 = b1 > b2 ? b1 : b2;
+        b1 = s[v];
+        arg = v;
+      } else if (s[v] > b2) {
+        b2 = s[v];
+      }
+    }
+    out_idx[i] = arg;
+    if (out_best) out_best[i] = b1;
+    if (out_second) out_second[i] = b2;
+  }
+  free(cand);
+  free(s);
+  free(l);
+}
+
+/* ------------------------------------------------------------------------ */
 /* Grouped (Group-Gumbel-Max) sampling.                                      */
 /* ------------------------------------------------------------------------ */
 

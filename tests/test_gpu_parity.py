@@ -479,3 +479,56 @@ def test_online_groups_match_fused_grouped(dev, oracle, B, V, G, masked):
         scale = TIE_REL * (1 + abs(o_summ[b, :, 0].max()))
         assert margin[b, 0] <= scale or margin[b, 1] <= scale, (b, got[b], idx[b])
     assert (got == fused).mean() > 0.98
+
+
+# --------------------------------------------------------------- top-k
+@pytest.mark.parametrize("B,d,V,K,masked", [(1, 64, 4096, 1, False), (7, 64, 3001, 5, True),
+                                            (64, 128, 9000, 50, False), (33, 64, 1000, 1000, True),
+                                            (300, 32, 2048, 20, True), (4, 64, 700, 9999, False)])
+def test_topk_parity(dev, oracle, B, d, V, K, masked):
+    H, W, Hd, Wd = rand_inputs(B, d, V, seed=K + V)
+    mask = synth.make_mask(B, V, 0.6, seed=K) if masked else None
+    md = mask.to(dev) if masked else None
+    rs = synth.make_row_seeds(B)
+    got = binding.fs_sample_topk(Hd, Wd, K, temperature=0.8, seed=2, row_seeds=rs.to(dev), step=3,
+                                 mask_bits=md).cpu().numpy()
+    idx, best, second = oracle.sample_topk(H, W, K, T=0.8, seed=2, row_seeds=rs, step=3, mask=mask)
+    assert_parity(got, idx, best, second, "topk K=%d" % K)
+    if K >= V:
+        flat = binding.fs_sample_ex(Hd, Wd, temperature=0.8, seed=2, row_seeds=rs.to(dev), step=3,
+                                    mask_bits=md).cpu().numpy()
+        assert np.array_equal(got, flat)
+
+
+def test_topk_ties_at_the_boundary(dev, oracle):
+    """41 duplicated W rows hold the largest logit of every row, so the k-th
+    place falls inside the tie and the smallest indices must be kept."""
+    B, d, V, K = 8, 64, 512, 6
+    _, W, _, _ = rand_inputs(B, d, V, seed=5)
+    h = synth.make_hidden(1, d, seed=6)
+    H = h.repeat(B, 1).contiguous()
+    W = W.clone()
+    hf = h[0].float()
+    W[7] = (hf * 8.0 / (hf * hf).sum()).to(torch.bfloat16)
+    W[100:140] = W[7]
+    keep = {7, 100, 101, 102, 103, 104}
+    Hd, Wd = H.to(dev), W.to(dev)
+    for step in range(6):
+        got = binding.fs_sample_topk(Hd, Wd, K, temperature=1.0, seed=1, step=step).cpu().numpy()
+        idx, best, second = oracle.sample_topk(H, W, K, T=1.0, seed=1, step=step)
+        assert set(idx.tolist()) <= keep and set(got.tolist()) <= keep
+        assert_parity(got, idx, best, second, "topk ties")
+
+
+def test_topk_full_vocab(dev, oracle):
+    wl = synth.WORKLOADS["qwen3-8b"]
+    B, K = 64, 40
+    Wd = synth.make_weight(wl.V, wl.d, wl.w_std, device=dev)
+    Hd = synth.make_hidden(B, wl.d, device=dev)
+    got = binding.fs_sample_topk(Hd, Wd, K, temperature=wl.temperature, step=1).cpu().numpy()
+    rows = np.array([0, 40, 63], dtype=np.int32)
+    idx, best, second = oracle.sample_topk(Hd.cpu(), Wd.cpu(), K, T=wl.temperature, step=1,
+                                           rows=rows)
+    assert_parity(got[rows], idx, best, second, "topk full")
+    del Wd
+    torch.cuda.empty_cache()

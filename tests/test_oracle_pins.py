@@ -451,3 +451,54 @@ def test_multi_samples_are_softmax_draws(oracle):
         counts += np.bincount(idx.ravel(), minlength=V)
     p = _softmax(oracle.logits(H, W)[0] / 1.2)
     assert _chi2_pvalue(counts, p) > 1e-3
+
+
+# --------------------------------------------------------------------------
+# Top-k (readus.org page, "Top-K and masking": prefilter, then exact Gumbel-max)
+# --------------------------------------------------------------------------
+
+def test_topk_degenerate_cases(oracle):
+    B, d, V = 10, 32, 257
+    H = synth.make_hidden(B, d, seed=141)
+    W = synth.make_weight(V, d, 0.5, seed=142)
+    for step in range(4):
+        flat, fb, _ = oracle.sample(H, W, T=0.9, seed=2, step=step)
+        all_k, ab, _ = oracle.sample_topk(H, W, V, T=0.9, seed=2, step=step)
+        more, _, _ = oracle.sample_topk(H, W, 10 * V, T=0.9, seed=2, step=step)
+        assert np.array_equal(all_k, flat) and np.array_equal(ab, fb) and np.array_equal(more, flat)
+        one, _, _ = oracle.sample_topk(H, W, 1, T=0.9, seed=2, step=step)
+        assert np.array_equal(one, np.argmax(oracle.logits(H, W), axis=1))   # greedy
+
+
+def test_topk_respects_mask_and_set(oracle):
+    B, d, V, K = 6, 32, 300, 7
+    H = synth.make_hidden(B, d, seed=151)
+    W = synth.make_weight(V, d, 0.5, seed=152)
+    allowed = torch.rand(B, V, generator=torch.Generator().manual_seed(8)) < 0.5
+    allowed[0] = False
+    mask = synth.mask_from_bool(allowed)
+    l = oracle.logits(H, W)
+    for step in range(8):
+        idx, _, _ = oracle.sample_topk(H, W, K, seed=3, step=step, mask=mask)
+        assert idx[0] == -1
+        for b in range(1, B):
+            a = np.flatnonzero(allowed[b].numpy())
+            top = a[np.lexsort((a, -l[b, a]))][:K]
+            assert idx[b] in top
+
+
+def test_topk_matches_truncated_softmax(oracle):
+    V, d, K, N, T = 64, 32, 9, 200_000, 1.1
+    H = synth.make_hidden(1, d, seed=161)
+    W = synth.make_weight(V, d, 0.35, seed=162)
+    l = oracle.logits(H, W)[0]
+    counts = np.zeros(V, dtype=np.int64)
+    # 2000 rows of the same hidden state, 100 steps: 200k draws
+    Hr = H.repeat(2000, 1)
+    for step in range(N // 2000):
+        idx, _, _ = oracle.sample_topk(Hr, W, K, T=T, seed=4, step=step)
+        counts += np.bincount(idx, minlength=V)
+    top = np.argsort(-l, kind="stable")[:K]
+    assert counts[np.setdiff1d(np.arange(V), top)].sum() == 0
+    p = _softmax(l[top] / T)
+    assert _chi2_pvalue(counts[top], p) > 1e-3
