@@ -232,6 +232,8 @@ cudaError_t launch_sample_logits(const SampleLogitsParams &s, cudaStream_t strea
 // ---------------------------------------------------------------------------
 constexpr int kTopkThreads = 1024;
 constexpr int kTopkBins = 2048;
+constexpr int kTopkItems = 8;     // consecutive elements per thread per iteration
+constexpr int kTopkSubHists = 4;  // warp-interleaved copies of the histogram
 
 __device__ __forceinline__ bool topk_allowed(const SampleLogitsParams &s, uint32_t bg, int v) {
   if (s.mask == nullptr) return true;
@@ -267,9 +269,38 @@ __device__ __forceinline__ int block_exclusive_scan(int x, int *warp_sums, int *
   return r;
 }
 
+// Loads this thread's kTopkItems consecutive logits starting at v0 and their
+// order-preserving keys; ok[i] is false past V or for a masked token.
+__device__ __forceinline__ void topk_load(const SampleLogitsParams &s, const float *row,
+                                          uint32_t bg, int v0, bool vec, float (&l)[kTopkItems],
+                                          uint32_t (&key)[kTopkItems], bool (&ok)[kTopkItems]) {
+  if (vec && v0 + kTopkItems <= s.V) {
+    const float4 a = *reinterpret_cast<const float4 *>(row + v0);
+    const float4 c = *reinterpret_cast<const float4 *>(row + v0 + 4);
+    l[0] = a.x; l[1] = a.y; l[2] = a.z; l[3] = a.w;
+    l[4] = c.x; l[5] = c.y; l[6] = c.z; l[7] = c.w;
+#pragma unroll
+    for (int i = 0; i < kTopkItems; ++i) ok[i] = true;
+  } else {
+#pragma unroll
+    for (int i = 0; i < kTopkItems; ++i) {
+      ok[i] = v0 + i < s.V;
+      l[i] = ok[i] ? row[v0 + i] : 0.f;
+    }
+  }
+  uint32_t mword = 0xFFFFFFFFu;
+  if (s.mask != nullptr && v0 < s.V)   // 8 consecutive tokens share one mask word
+    mword = s.mask[static_cast<size_t>(bg) * s.mask_words + (v0 >> 5)];
+#pragma unroll
+  for (int i = 0; i < kTopkItems; ++i) {
+    ok[i] = ok[i] && ((mword >> ((v0 + i) & 31)) & 1u);
+    key[i] = order_bits(__float_as_uint(l[i]));
+  }
+}
+
 __global__ void __launch_bounds__(kTopkThreads) topk_sample_kernel(const SampleLogitsParams s,
                                                                    int K) {
-  __shared__ int hist[kTopkBins];
+  __shared__ int hist[kTopkSubHists * kTopkBins];
   __shared__ int warp_sums[32];
   __shared__ int sh_digit, sh_above, sh_total;
   __shared__ uint64_t warp_best[32];
@@ -277,55 +308,52 @@ __global__ void __launch_bounds__(kTopkThreads) topk_sample_kernel(const SampleL
   const uint32_t bg = static_cast<uint32_t>(s.b_off + b);
   const float *row = s.logits + static_cast<size_t>(b) * s.V;
   const int lane = threadIdx.x & 31;
+  const bool vec = (s.V & 3) == 0;
+  const int span = kTopkThreads * kTopkItems;
+  int *my_hist = hist + ((threadIdx.x >> 5) & (kTopkSubHists - 1)) * kTopkBins;
 
-  // ---- radix select of the k-th largest key among allowed logits
+  // ---- radix select of the K-th largest key among allowed logits
   uint32_t prefix = 0, pmask = 0;
-  int k_rem = K;         // rank still to find inside the current prefix
+  int k_rem = K;   // rank still to find among keys matching the prefix
   int n_allowed = 0;
   const int shifts[3] = {21, 10, 0};
   const int widths[3] = {11, 11, 10};
   for (int pass = 0; pass < 3; ++pass) {
     const int shift = shifts[pass];
     const uint32_t dmask = (1u << widths[pass]) - 1u;
-    for (int i = threadIdx.x; i < kTopkBins; i += kTopkThreads) hist[i] = 0;
+    for (int i = threadIdx.x; i < kTopkSubHists * kTopkBins; i += kTopkThreads) hist[i] = 0;
     __syncthreads();
-    for (int base = 0; base < s.V; base += kTopkThreads) {
-      const int v = base + threadIdx.x;
-      bool take = false;
-      uint32_t bin = 0;
-      if (v < s.V && topk_allowed(s, bg, v)) {
-        const uint32_t key = order_bits(__float_as_uint(row[v]));
-        if ((key & pmask) == prefix) {
-          take = true;
-          bin = (key >> shift) & dmask;
-        }
-      }
-      // warp-aggregated increments: lanes with the same bin add once
-      const unsigned active = __ballot_sync(0xffffffffu, take);
-      if (take) {
-        const unsigned same = __match_any_sync(active, bin);
-        if ((__ffs(same) - 1) == lane) atomicAdd(&hist[bin], __popc(same));
-      }
+    for (int base = 0; base < s.V; base += span) {
+      float l[kTopkItems];
+      uint32_t key[kTopkItems];
+      bool ok[kTopkItems];
+      topk_load(s, row, bg, base + threadIdx.x * kTopkItems, vec, l, key, ok);
+#pragma unroll
+      for (int i = 0; i < kTopkItems; ++i)
+        if (ok[i] && (key[i] & pmask) == prefix) atomicAdd(&my_hist[(key[i] >> shift) & dmask], 1);
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < kTopkBins; i += kTopkThreads) {   // fold the copies
+      int c = 0;
+#pragma unroll
+      for (int h = 0; h < kTopkSubHists; ++h) c += hist[h * kTopkBins + i];
+      hist[i] = c;
     }
     __syncthreads();
     if (pass == 0) {
-      // allowed tokens in total
       int c = 0;
       for (int i = threadIdx.x; i < kTopkBins; i += kTopkThreads) c += hist[i];
-      int total;
       block_exclusive_scan(c, warp_sums, &sh_total);
-      total = sh_total;
-      n_allowed = total;
+      n_allowed = sh_total;
       if (n_allowed <= K) break;   // every allowed token is a candidate
     }
-    // find the digit holding the k_rem-th largest: suffix sums from the top bin
     {
-      // each thread owns two adjacent bins, scanned from the top
-      const int t = kTopkThreads - 1 - threadIdx.x;   // thread 0 holds the top bins
+      // suffix sums from the top bin: thread 0 holds bins 2047 and 2046
+      const int t = kTopkThreads - 1 - threadIdx.x;
       const int hi_bin = 2 * t + 1, lo_bin = 2 * t;
       const int c_hi = hist[hi_bin], c_lo = hist[lo_bin];
       int total;
-      const int above = block_exclusive_scan(c_hi + c_lo, warp_sums, &total);  // bins above mine
+      const int above = block_exclusive_scan(c_hi + c_lo, warp_sums, &total);
       if (above < k_rem && above + c_hi >= k_rem) {
         sh_digit = hi_bin;
         sh_above = above;
@@ -341,37 +369,46 @@ __global__ void __launch_bounds__(kTopkThreads) topk_sample_kernel(const SampleL
     __syncthreads();
   }
   const bool all_allowed = n_allowed <= K;
-  // prefix is now the k-th largest key; k_rem of the keys equal to it are in.
+  // prefix is the K-th largest key; the first k_rem keys equal to it (in
+  // index order) are candidates, as is every larger key.
 
   // ---- candidates and Gumbel-max
   const uint64_t k64 = s.row_seeds ? s.row_seeds[bg] : s.seed;
   uint64_t best = 0ull;
-  int eq_seen = 0;   // keys equal to the threshold already passed, in index order
-  for (int base = 0; base < s.V; base += kTopkThreads) {
-    const int v = base + threadIdx.x;
-    bool ok = v < s.V && topk_allowed(s, bg, v);
-    uint32_t key = 0;
-    float l = 0.f;
-    if (ok) {
-      l = row[v];
-      key = order_bits(__float_as_uint(l));
+  int eq_seen = 0;
+  for (int base = 0; base < s.V; base += span) {
+    const int v0 = base + threadIdx.x * kTopkItems;
+    float l[kTopkItems];
+    uint32_t key[kTopkItems];
+    bool ok[kTopkItems];
+    topk_load(s, row, bg, v0, vec, l, key, ok);
+    int n_eq_mine = 0;
+#pragma unroll
+    for (int i = 0; i < kTopkItems; ++i)
+      n_eq_mine += (ok[i] && !all_allowed && key[i] == prefix) ? 1 : 0;
+    const int rank0 = eq_seen + block_exclusive_scan(n_eq_mine, warp_sums, &sh_total);
+    eq_seen += sh_total;
+    int r = rank0;
+#pragma unroll
+    for (int i = 0; i < kTopkItems; ++i) {
+      if (!ok[i]) continue;
+      bool cand = all_allowed || key[i] > prefix;
+      if (!all_allowed && key[i] == prefix) {
+        cand = r < k_rem;
+        ++r;
+      }
+      if (cand) {
+        const int v = v0 + i;
+        const Philox4 ph = philox4x32_10(static_cast<uint32_t>(v) >> 2, bg, s.step, 0u,
+                                         static_cast<uint32_t>(k64),
+                                         static_cast<uint32_t>(k64 >> 32));
+        const uint32_t w =
+            (v & 3) == 0 ? ph.w0 : (v & 3) == 1 ? ph.w1 : (v & 3) == 2 ? ph.w2 : ph.w3;
+        const float sc = fmaf(l[i], s.inv_temp, gumbel_from_u32(w));
+        const uint64_t k = pack_key(__float_as_uint(sc), v);
+        best = k > best ? k : best;
+      }
     }
-    bool cand = ok && (all_allowed || key > prefix);
-    const bool eq = ok && !all_allowed && key == prefix;
-    int n_eq;
-    const int rank = block_exclusive_scan(eq ? 1 : 0, warp_sums, &sh_total);
-    n_eq = sh_total;
-    if (eq && eq_seen + rank < k_rem) cand = true;
-    eq_seen += n_eq;
-    if (cand) {
-      const Philox4 ph = philox4x32_10(static_cast<uint32_t>(v) >> 2, bg, s.step, 0u,
-                                       static_cast<uint32_t>(k64), static_cast<uint32_t>(k64 >> 32));
-      const uint32_t w = (v & 3) == 0 ? ph.w0 : (v & 3) == 1 ? ph.w1 : (v & 3) == 2 ? ph.w2 : ph.w3;
-      const float sc = fmaf(l, s.inv_temp, gumbel_from_u32(w));
-      const uint64_t k = pack_key(__float_as_uint(sc), v);
-      best = k > best ? k : best;
-    }
-    __syncthreads();
   }
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) {

@@ -41,12 +41,13 @@
 
 namespace fmms {
 
-template <int BN>
+template <int BN, int MODE>
 struct KCfg {
   static constexpr int kStageW = kTileM * kBlockK * 2;  // 16 KB of W per stage
   static constexpr int kStageH = BN * kBlockK * 2;      // BN rows of H per stage
   static constexpr int kStageBytes = kStageW + kStageH;
-  static constexpr int kStagesFit = 196608 / kStageBytes;
+  static constexpr int kCombBytes = MODE == kModeGrouped ? 4 * BN * 16 : 0;  // grouped only
+  static constexpr int kStagesFit = (232448 - 1024 - 256 - kCombBytes) / kStageBytes;
   static constexpr int kStages = kStagesFit < 10 ? kStagesFit : 10;
   static constexpr int kCW = 16;                        // columns per epilogue chunk
   static constexpr int kChunks = BN / kCW;
@@ -56,7 +57,6 @@ struct KCfg {
   static constexpr int kTmemCols = kAccBufs * BN < 32 ? 32 : kAccBufs * BN;
   static constexpr uint32_t kIdesc = sm100::idesc_bf16_f32(kTileM, BN);
   static constexpr int kBarBytes = 256;
-  static constexpr int kCombBytes = 4 * BN * 16;
   static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBarBytes + kCombBytes;
   static_assert(kStageH % 1024 == 0, "H stage must keep 1024-byte atom alignment");
   static_assert((2 * kStages + 2 * kAccBufs + 1) * 8 + 16 <= kBarBytes, "barrier area too small");
@@ -273,13 +273,13 @@ __device__ __forceinline__ bool chunk_any_candidate(const uint32_t (&acc)[CW],
 // Roles
 // ---------------------------------------------------------------------------
 
-template <int BN>
+template <int BN, int MODE>
 __device__ __forceinline__ void role_producer(const CUtensorMap *tw, const CUtensorMap *tw8,
                                               const CUtensorMap *th, const FmmsParams &p,
                                               const Schedule &sch, uint8_t *stages,
                                               uint64_t *full, uint64_t *empty,
                                               volatile int *abort_flag) {
-  using C = KCfg<BN>;
+  using C = KCfg<BN, MODE>;
   const uint64_t pol_w = sm100::l2_policy_evict_first();
   const uint64_t pol_h = sm100::l2_policy_evict_last();
   TileIter it(sch, blockIdx.x);
@@ -329,13 +329,13 @@ __device__ __forceinline__ void role_producer(const CUtensorMap *tw, const CUten
   }
 }
 
-template <int BN>
+template <int BN, int MODE>
 __device__ __forceinline__ void role_mma(const FmmsParams &p, const Schedule &sch,
                                          uint8_t *stages, uint64_t *full, uint64_t *empty,
                                          uint64_t *acc_full, uint64_t *acc_empty,
                                          uint64_t *drain_bar, uint32_t tmem_base,
                                          volatile int *abort_flag) {
-  using C = KCfg<BN>;
+  using C = KCfg<BN, MODE>;
   TileIter it(sch, blockIdx.x);
   Tile tile;
   int stage = 0;
@@ -387,7 +387,7 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
                                               uint64_t *acc_empty, volatile int *abort_flag,
                                               int *last_flag, uint64_t *comb_key, float *comb_m,
                                               float *comb_s, int warp, int lane) {
-  using C = KCfg<BN>;
+  using C = KCfg<BN, MODE>;
   constexpr int CW = C::kCW;
   const int q = warp & 3;          // TMEM lane quarter this warp may access
   const int h = (warp - 2) >> 2;   // which of the quarter's warps: chunks h, h+4, ...
@@ -573,7 +573,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fmms_kernel(const __grid_constant__ CUtensorMap tmap_w,
                 const __grid_constant__ CUtensorMap tmap_w8,
                 const __grid_constant__ CUtensorMap tmap_h, const FmmsParams p) {
-  using C = KCfg<BN>;
+  using C = KCfg<BN, MODE>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -629,11 +629,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     if (lane == 0)
-      role_producer<BN>(&tmap_w, &tmap_w8, &tmap_h, p, sch, stages, full, empty, abort_flag);
+      role_producer<BN, MODE>(&tmap_w, &tmap_w8, &tmap_h, p, sch, stages, full, empty, abort_flag);
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0)
-      role_mma<BN>(p, sch, stages, full, empty, acc_full, acc_empty, drain_bar, tmem_base,
+      role_mma<BN, MODE>(p, sch, stages, full, empty, acc_full, acc_empty, drain_bar, tmem_base,
                    abort_flag);
     __syncwarp();
   } else {
@@ -653,7 +653,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int BN, int MODE>
 static cudaError_t launch_t(const CUtensorMap &tw, const CUtensorMap &tw8, const CUtensorMap &th,
                             const FmmsParams &p, cudaStream_t stream) {
-  using C = KCfg<BN>;
+  using C = KCfg<BN, MODE>;
   auto kern = fmms_kernel<BN, MODE>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
