@@ -306,6 +306,20 @@ fs_status fs_test_stalled_sample(const void *H, const void *W, int B, int d,
                                  int V, int32_t *out_idx, void *workspace,
                                  size_t workspace_bytes, fs_stream_t stream);
 
+/* ---- Kernel choice ---- */
+
+/* Whether flat-mode calls (fs_sample, fs_sample_ex, fs_sample_host,
+ * fs_sample_noalloc, fs_sample_multi, fs_sample_shard_keys) run the fused
+ * kernel on CTA pairs: clusters of two CTAs on two SMs that share one
+ * M = 256 tensor-core MMA (tcgen05 cta_group::2), each SM staging 128 rows
+ * of W and half of the batch rows of H per pipeline stage.  This is a B200
+ * design choice, not part of the method: the sampled tokens are the same
+ * either way.  policy: -1 automatic (the default: pairs for launches of more
+ * than 64 batch rows), 0 never, 1 always.  Process-wide; applies to calls
+ * made after it returns.  FS_ERR_INVALID_ARG for any other value.  When the
+ * device cannot co-schedule a pair, the single-CTA kernel runs. */
+fs_status fs_set_cta_pairs(int policy);
+
 /* ---- Host-only schedule query (no GPU needed) ---- */
 
 /* The vocabulary schedule of the fused kernel for V tokens, G groups

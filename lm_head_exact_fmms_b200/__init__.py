@@ -12,7 +12,8 @@ _BINDING_NAMES = ("FmmsError", "fs_sample", "fs_sample_ex", "fs_sample_grouped",
                   "library_path", "load_library", "fs_sample_noalloc",
                   "fs_test_stalled_sample", "fs_sample_shard_keys", "fs_keys_to_tokens",
                   "fs_sample_multi", "fs_workspace_bytes_multi", "fs_summarize_group",
-                  "fs_merge_groups", "fs_workspace_bytes_summary", "fs_sample_topk")
+                  "fs_merge_groups", "fs_workspace_bytes_summary", "fs_sample_topk",
+                  "fs_set_cta_pairs")
 
 
 def __getattr__(name):

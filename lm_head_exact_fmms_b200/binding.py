@@ -24,7 +24,7 @@ EXPORTED = ("fs_sample", "fs_sample_ex", "fs_sample_grouped", "fs_sample_unfused
             "fs_sample_noalloc", "fs_test_stalled_sample", "fs_sample_shard_keys",
             "fs_keys_to_tokens", "fs_sample_multi", "fs_workspace_bytes_multi",
             "fs_summarize_group", "fs_merge_groups", "fs_workspace_bytes_summary",
-            "fs_sample_topk")
+            "fs_sample_topk", "fs_set_cta_pairs")
 
 
 class FmmsError(RuntimeError):
@@ -317,6 +317,12 @@ def fs_test_stalled_sample(H, W, workspace, out_idx=None, stream=None):
     _check(lib.fs_test_stalled_sample(_ptr(H), _ptr(W), B, d, V, _ptr(out_idx), _ptr(workspace),
                                       ws_bytes, _stream(stream)), "fs_test_stalled_sample")
     return out_idx
+
+
+def fs_set_cta_pairs(policy):
+    """Kernel choice for flat-mode calls: -1 automatic, 0 single-CTA kernel
+    only, 1 CTA-pair (cta_group::2) kernel whenever possible.  Process-wide."""
+    _check(load_library().fs_set_cta_pairs(int(policy)), "fs_set_cta_pairs")
 
 
 def fs_sample_shard_keys(H, W_shard, vocab_offset, V_total, temperature=1.0, seed=0,

@@ -29,6 +29,7 @@ struct DeviceState {
   size_t h_stage_bytes = 0;
   void *o_stage = nullptr;  // fs_sample_host: device tokens
   size_t o_stage_bytes = 0;
+  int pair_units[5] = {-1, -1, -1, -1, -1};  // resident CTA pairs per batch tile (-1: unknown)
 };
 
 constexpr int kMaxDevices = 64;
@@ -189,6 +190,35 @@ fs_status resolve_workspace(DeviceState *st, const Schedule &sch, int B, int sam
 // Set only for the duration of fs_test_stalled_sample (under g_mu).
 bool g_test_no_loads = false;
 
+// fs_set_cta_pairs: -1 automatic, 0 never, 1 whenever the call allows it.
+int g_pair_policy = -1;
+
+int bn_index(int BN) {
+  return BN <= 16 ? 0 : BN <= 32 ? 1 : BN <= 64 ? 2 : BN <= 128 ? 3 : 4;
+}
+
+// CTA pairs of the BN pair kernel that fit on the device at once (0: none).
+int pair_units(DeviceState *st, int BN) {
+  int &u = st->pair_units[bn_index(BN)];
+  if (u < 0) {
+    int n = 0;
+    if (fmms::fmms_pair_units(BN, &n) != cudaSuccess) {
+      cudaGetLastError();  // clear the error; the single-CTA kernel is used
+      n = 0;
+    }
+    u = fmms::imin(n, st->sms / 2);
+  }
+  return u;
+}
+
+// Flat calls with a batch tile of 128 or more rows run on CTA pairs: each SM
+// then stages half of H per stage, which halves the batch operand's L2
+// traffic where it matters.
+bool use_pairs(int mode, int BN) {
+  if (mode != fmms::kModeFlat || g_pair_policy == 0) return false;
+  return g_pair_policy == 1 || BN >= 128;
+}
+
 // Options of vocabulary-shard and multi-sample calls.
 struct ShardOpts {
   int vocab_offset = 0;         // global token index of W row 0
@@ -237,8 +267,10 @@ fs_status run_locked(int mode, const void *H, const void *W, int B, int d, int V
   for (int b0 = 0; b0 < B; b0 += fmms::kMaxBN) {
     const int Bc = fmms::imin(fmms::kMaxBN, B - b0);
     const int BN = fmms::fmms_batch_tile(Bc);
+    const int units = use_pairs(mode, BN) ? pair_units(st, BN) : 0;
+    const bool pair = units > 0;
     CUtensorMap th;
-    if ((s = tensor_map(&th, H, d, B, BN)) != FS_OK) return s;
+    if ((s = tensor_map(&th, H, d, B, pair ? BN / 2 : BN)) != FS_OK) return s;
     FmmsParams p;
     memset(&p, 0, sizeof p);
     p.B = Bc;
@@ -266,7 +298,12 @@ fs_status run_locked(int mode, const void *H, const void *W, int B, int d, int V
     p.vocab_offset = shard.vocab_offset;
     p.out_keys = shard.out_keys ? shard.out_keys + static_cast<size_t>(b0) * S : nullptr;
     p.num_samples = S;
-    if (fmms::launch_fmms(mode, BN, tw, tw8, th, p, stream) != cudaSuccess) return FS_ERR_CUDA;
+    if (pair) {
+      p.num_ctas = 2 * fmms::make_schedule(V, 1, units).num_ctas;
+      if (fmms::launch_fmms_pair(BN, tw, tw8, th, p, stream) != cudaSuccess) return FS_ERR_CUDA;
+    } else {
+      if (fmms::launch_fmms(mode, BN, tw, tw8, th, p, stream) != cudaSuccess) return FS_ERR_CUDA;
+    }
 
     if (mode == fmms::kModeGrouped) {
       fmms::MergeParams m;
@@ -579,6 +616,13 @@ fs_status fs_gumbel(const uint32_t *r, float *g, int64_t n, fs_stream_t stream) 
   return fmms::launch_gumbel_test(r, g, n, static_cast<cudaStream_t>(stream)) == cudaSuccess
              ? FS_OK
              : FS_ERR_CUDA;
+}
+
+fs_status fs_set_cta_pairs(int policy) {
+  if (policy < -1 || policy > 1) return FS_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(g_mu);
+  g_pair_policy = policy;
+  return FS_OK;
 }
 
 fs_status fs_plan_tiles(int V, int G, int num_sms, int cta, int32_t *tiles, int max_tiles,

@@ -27,6 +27,7 @@ __global__ void __launch_bounds__(128) group_merge_kernel(const MergeParams m) {
   sch.G = m.G;
   sch.num_ctas = m.num_ctas;
   sch.ngran = m.ngran;
+  sch.tile_rows = kTileM;
   const uint32_t bg = static_cast<uint32_t>(m.b_off + b);
   const uint64_t k64 = m.row_seeds ? m.row_seeds[bg] : m.seed;
   fs_group_summary *summary = static_cast<fs_group_summary *>(m.summary);

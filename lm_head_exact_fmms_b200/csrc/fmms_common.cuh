@@ -38,9 +38,10 @@ FS_HD int imax(int a, int b) { return a > b ? a : b; }
 // ---------------------------------------------------------------------------
 struct Schedule {
   int V;
-  int G;         // number of groups (1 = flat)
-  int num_ctas;
-  int ngran;     // ceil(V / 8)
+  int G;          // number of groups (1 = flat)
+  int num_ctas;   // schedule units: CTAs, or CTA pairs in pair mode
+  int ngran;      // ceil(V / 8)
+  int tile_rows;  // vocabulary rows per tile: 128, or 256 for a CTA pair
 };
 
 FS_HD Schedule make_schedule(int V, int G, int num_sms) {
@@ -49,6 +50,7 @@ FS_HD Schedule make_schedule(int V, int G, int num_sms) {
   s.G = G < 1 ? 1 : G;
   s.ngran = (V + kGranule - 1) / kGranule;
   s.num_ctas = imin(num_sms, s.ngran);
+  s.tile_rows = kTileM;
   return s;
 }
 
@@ -74,15 +76,25 @@ FS_HD int cta_of(int v, const Schedule &s) {
 struct Tile {
   int start;  // first vocabulary row of the tile (multiple of 8)
   int lo;     // first valid row
-  int hi;     // one past the last valid row (hi - start <= 128)
+  int hi;     // one past the last valid row (hi - start <= tile rows)
   int slot;   // partial slot of the segment
   int last;   // 1 on the last tile of a segment
 };
 
+// The 128-row half of a 256-row pair tile that CTA `rank` of the pair
+// multiplies; hi <= lo when the half holds no valid row.
+FS_HD Tile pair_half(const Tile &t, int rank) {
+  Tile h = t;
+  h.start = t.start + rank * kTileM;
+  h.lo = imax(t.lo, h.start);
+  h.hi = imin(t.hi, h.start + kTileM);
+  return h;
+}
+
 // Walks the tiles of one CTA.  All three kernel roles and the host-side
 // schedule query run this same code.
 struct TileIter {
-  int V, G, cta, cta_hi;
+  int V, G, cta, cta_hi, rows;
   int v;       // first token of the current segment
   int seg_hi;  // end of the current segment
   int t;       // start of the next tile
@@ -91,6 +103,7 @@ struct TileIter {
   FS_HD TileIter(const Schedule &s, int c) {
     V = s.V;
     G = s.G;
+    rows = s.tile_rows;
     cta = c;
     v = cta_begin(c, s);
     cta_hi = cta_begin(c + 1, s);
@@ -111,9 +124,9 @@ struct TileIter {
     }
     tile.start = t;
     tile.lo = imax(t, v);
-    tile.hi = imin(t + kTileM, seg_hi);
+    tile.hi = imin(t + rows, seg_hi);
     tile.slot = slot;
-    t += kTileM;
+    t += rows;
     tile.last = (t >= seg_hi) ? 1 : 0;
     return true;
   }

@@ -41,13 +41,36 @@
 
 namespace fmms {
 
-template <int BN, int MODE>
+// Shared memory a kernel may use beyond the stages: alignment slack,
+// barriers and (grouped mode) the combine area.
+constexpr int kSmemBudget = 232448 - 1024 - 256;
+
+// K sub-blocks of 64 elements per pipeline stage.  Two sub-blocks halve the
+// per-stage handshake (full wait, tcgen05 fence, commit, empty wait) per byte
+// of W and let W be fetched 256 bytes of a row at a time, but they halve the
+// number of stages.  Measured on the Qwen3-8B-shaped head: a ten-stage ring of
+// single sub-blocks is best while it fits (batch tiles up to 32 rows per
+// CTA); where H is large enough to shorten the ring below ten stages, two
+// sub-blocks win as long as four stages remain (64 rows; 128 rows per pair).
+constexpr int ksub_for(int h_rows, int comb_bytes) {
+  const int stage1 = (kTileM + h_rows) * kBlockK * 2;
+  const int fit1 = (kSmemBudget - comb_bytes) / stage1;
+  const int fit2 = (kSmemBudget - comb_bytes) / (2 * stage1);
+  return (fit1 < 10 && fit2 >= 4) ? 2 : 1;
+}
+
+template <int BN, int MODE, bool PAIR = false>
 struct KCfg {
-  static constexpr int kStageW = kTileM * kBlockK * 2;  // 16 KB of W per stage
-  static constexpr int kStageH = BN * kBlockK * 2;      // BN rows of H per stage
-  static constexpr int kStageBytes = kStageW + kStageH;
+  static_assert(!PAIR || MODE == kModeFlat, "CTA pairs run the flat mode only");
+  static constexpr int kHRows = PAIR ? BN / 2 : BN;     // H rows this CTA stages
   static constexpr int kCombBytes = MODE == kModeGrouped ? 4 * BN * 16 : 0;  // grouped only
-  static constexpr int kStagesFit = (232448 - 1024 - 256 - kCombBytes) / kStageBytes;
+  static constexpr int kSub = ksub_for(kHRows, kCombBytes);  // 64-wide K blocks per stage
+  static constexpr int kSubW = kTileM * kBlockK * 2;    // 16 KB of W per sub-block
+  static constexpr int kSubH = kHRows * kBlockK * 2;    // this CTA's H rows per sub-block
+  static constexpr int kStageW = kSub * kSubW;
+  static constexpr int kStageH = kSub * kSubH;
+  static constexpr int kStageBytes = kStageW + kStageH;
+  static constexpr int kStagesFit = (kSmemBudget - kCombBytes) / kStageBytes;
   static constexpr int kStages = kStagesFit < 10 ? kStagesFit : 10;
   static constexpr int kCW = 16;                        // columns per epilogue chunk
   static constexpr int kChunks = BN / kCW;
@@ -55,10 +78,11 @@ struct KCfg {
   static constexpr int kChunksPerWarp = kChunks >= kWarpsPerQuarter ? kChunks / kWarpsPerQuarter : 1;
   static constexpr int kAccBufs = BN <= 128 ? 4 : 2;     // accumulators in flight
   static constexpr int kTmemCols = kAccBufs * BN < 32 ? 32 : kAccBufs * BN;
-  static constexpr uint32_t kIdesc = sm100::idesc_bf16_f32(kTileM, BN);
+  static constexpr uint32_t kIdesc = sm100::idesc_bf16_f32(PAIR ? 2 * kTileM : kTileM, BN);
+  static constexpr int kEpiArrivals = PAIR ? 2 * kNumEpiWarps : kNumEpiWarps;
   static constexpr int kBarBytes = 256;
   static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBarBytes + kCombBytes;
-  static_assert(kStageH % 1024 == 0, "H stage must keep 1024-byte atom alignment");
+  static_assert(kSubH % 1024 == 0, "H sub-block must keep 1024-byte atom alignment");
   static_assert((2 * kStages + 2 * kAccBufs + 1) * 8 + 16 <= kBarBytes, "barrier area too small");
   static_assert(kTmemCols <= 512, "tensor memory holds 512 columns");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -273,42 +297,84 @@ __device__ __forceinline__ bool chunk_any_candidate(const uint32_t (&acc)[CW],
 // Roles
 // ---------------------------------------------------------------------------
 
-template <int BN, int MODE>
+// Bytes of W a CTA loads per 64-wide K sub-block for `rows` rows from the
+// tile start (whole tile: one 128-row box; otherwise 8-row boxes).
+__device__ __forceinline__ uint32_t w_sub_bytes(int rows) {
+  if (rows <= 0) return 0u;
+  if (rows >= kTileM) return static_cast<uint32_t>(kTileM * kBlockK * 2);
+  return static_cast<uint32_t>((rows + kGranule - 1) / kGranule) * 1024u;
+}
+
+// TMA producer (one thread).  In pair mode both CTAs load their own half of
+// every stage (128 W rows, BN/2 H rows) and count the bytes on the even
+// CTA's full barrier; the even CTA also hands each freed stage on to the odd
+// CTA, whose MMA reads happen in the even CTA's tcgen05 pipeline.
+template <int BN, int MODE, bool PAIR>
 __device__ __forceinline__ void role_producer(const CUtensorMap *tw, const CUtensorMap *tw8,
                                               const CUtensorMap *th, const FmmsParams &p,
                                               const Schedule &sch, uint8_t *stages,
                                               uint64_t *full, uint64_t *empty,
-                                              volatile int *abort_flag) {
-  using C = KCfg<BN, MODE>;
+                                              volatile int *abort_flag, int unit, int rank) {
+  using C = KCfg<BN, MODE, PAIR>;
   const uint64_t pol_w = sm100::l2_policy_evict_first();
   const uint64_t pol_h = sm100::l2_policy_evict_last();
-  TileIter it(sch, blockIdx.x);
+  TileIter it(sch, unit);
   Tile tile;
   int stage = 0;
   uint32_t phase = 0;
   long long issued = 0;
   bool ok = p.test_no_loads == 0;
   while (ok && it.next(tile)) {
-    const int rows = tile.hi - tile.start;
-    const bool whole = rows == kTileM;
-    const int nbox8 = (rows + kGranule - 1) / kGranule;
-    const uint32_t bytes = (whole ? C::kStageW : nbox8 * 1024) + C::kStageH;
-    for (int kb = 0; kb < p.nk; ++kb) {
-      if (!sm100::wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.err)) {
+    const Tile mine = PAIR ? pair_half(tile, rank) : tile;
+    const int rows = mine.hi - mine.start;
+    const bool whole = rows >= kTileM;
+    const int nbox8 = rows > 0 ? (rows + kGranule - 1) / kGranule : 0;
+    uint32_t sub_bytes = w_sub_bytes(rows) + C::kSubH;  // counted on this CTA's barrier
+    if (PAIR) {
+      const Tile other = pair_half(tile, 1 - rank);
+      sub_bytes += w_sub_bytes(other.hi - other.start) + C::kSubH;
+    }
+    const int nks = (p.nk + C::kSub - 1) / C::kSub;
+    for (int ks = 0; ks < nks; ++ks) {
+      const int sub0 = ks * C::kSub;
+      const int nsub = imin(C::kSub, p.nk - sub0);
+      const uint32_t bytes = sub_bytes * static_cast<uint32_t>(nsub);
+      if (!sm100::wait_bounded<PAIR>(&empty[stage], phase ^ 1u, abort_flag, p.err)) {
         ok = false;
         break;
       }
-      uint8_t *sw = stages + stage * C::kStageBytes;
-      uint8_t *sh = sw + C::kStageW;
-      sm100::mbar_arrive_expect_tx(&full[stage], bytes);
-      const int x = kb * kBlockK;
-      if (whole) {
-        sm100::tma_load_2d(sw, tw, &full[stage], x, tile.start, pol_w);
-      } else {
-        for (int i = 0; i < nbox8; ++i)
-          sm100::tma_load_2d(sw + i * 1024, tw8, &full[stage], x, tile.start + kGranule * i, pol_w);
+      if (PAIR && rank == 0 && issued >= C::kStages)
+        sm100::mbar_arrive_cluster(sm100::cluster_addr(&empty[stage], 1));
+      uint8_t *sw0 = stages + stage * C::kStageBytes;
+      uint8_t *sh0 = sw0 + C::kStageW;
+      if (!PAIR || rank == 0) sm100::mbar_arrive_expect_tx(&full[stage], bytes);
+      const uint32_t bar = PAIR ? sm100::cluster_addr(&full[stage], 0) : 0u;
+#pragma unroll
+      for (int j = 0; j < C::kSub; ++j) {
+        if (j >= nsub) break;
+        uint8_t *sw = sw0 + j * C::kSubW;
+        uint8_t *sh = sh0 + j * C::kSubH;
+        const int x = (sub0 + j) * kBlockK;
+        if constexpr (PAIR) {
+          if (whole) {
+            sm100::tma_load_2d_pair(sw, tw, bar, x, mine.start, pol_w);
+          } else {
+            for (int i = 0; i < nbox8; ++i)
+              sm100::tma_load_2d_pair(sw + i * 1024, tw8, bar, x, mine.start + kGranule * i,
+                                      pol_w);
+          }
+          sm100::tma_load_2d_pair(sh, th, bar, x, p.b_off + rank * C::kHRows, pol_h);
+        } else {
+          if (whole) {
+            sm100::tma_load_2d(sw, tw, &full[stage], x, mine.start, pol_w);
+          } else {
+            for (int i = 0; i < nbox8; ++i)
+              sm100::tma_load_2d(sw + i * 1024, tw8, &full[stage], x, mine.start + kGranule * i,
+                                 pol_w);
+          }
+          sm100::tma_load_2d(sh, th, &full[stage], x, p.b_off, pol_h);
+        }
       }
-      sm100::tma_load_2d(sh, th, &full[stage], x, p.b_off, pol_h);
       ++issued;
       if (++stage == C::kStages) {
         stage = 0;
@@ -316,27 +382,32 @@ __device__ __forceinline__ void role_producer(const CUtensorMap *tw, const CUten
       }
     }
   }
-  if (!ok && issued > 0) {
+  if (!ok && issued > 0 && (!PAIR || rank == 0)) {
     // Gave up: let the copies already in flight land before the CTA exits.
+    // (The odd CTA of a pair cannot observe its copies, which complete on the
+    // even CTA's barriers; it exits only after the cluster barrier at the end
+    // of the kernel, which the even CTA reaches after this drain.)
+    // One time limit covers the whole drain.
     const long long first = issued > C::kStages ? issued - C::kStages : 0;
+    const long long t0 = clock64();
     for (long long n = first; n < issued; ++n) {
       const int s = static_cast<int>(n % C::kStages);
       const uint32_t ph = static_cast<uint32_t>((n / C::kStages) & 1);
-      const long long t0 = clock64();
-      while (!sm100::mbar_try_wait(&full[s], ph) && clock64() - t0 < sm100::kWaitLimitCycles) {
+      while (!sm100::mbar_try_wait<PAIR>(&full[s], ph) && clock64() - t0 < sm100::kWaitLimitCycles) {
       }
     }
   }
 }
 
-template <int BN, int MODE>
+// MMA issuer (one thread; in pair mode only the even CTA's).
+template <int BN, int MODE, bool PAIR>
 __device__ __forceinline__ void role_mma(const FmmsParams &p, const Schedule &sch,
                                          uint8_t *stages, uint64_t *full, uint64_t *empty,
                                          uint64_t *acc_full, uint64_t *acc_empty,
                                          uint64_t *drain_bar, uint32_t tmem_base,
-                                         volatile int *abort_flag) {
-  using C = KCfg<BN, MODE>;
-  TileIter it(sch, blockIdx.x);
+                                         volatile int *abort_flag, int unit) {
+  using C = KCfg<BN, MODE, PAIR>;
+  TileIter it(sch, unit);
   Tile tile;
   int stage = 0;
   uint32_t phase = 0;
@@ -344,50 +415,80 @@ __device__ __forceinline__ void role_mma(const FmmsParams &p, const Schedule &sc
   uint32_t acc_phase = 0;
   bool ok = true;
   while (ok && it.next(tile)) {
-    if (!sm100::wait_bounded(&acc_empty[buf], acc_phase ^ 1u, abort_flag, p.err)) break;
+    if (!sm100::wait_bounded<PAIR>(&acc_empty[buf], acc_phase ^ 1u, abort_flag, p.err)) break;
     sm100::tc_fence_after();
     const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
-    for (int kb = 0; kb < p.nk; ++kb) {
-      if (!sm100::wait_bounded(&full[stage], phase, abort_flag, p.err)) {
+    const int nks = (p.nk + C::kSub - 1) / C::kSub;
+    for (int ks = 0; ks < nks; ++ks) {
+      if (!sm100::wait_bounded<PAIR>(&full[stage], phase, abort_flag, p.err)) {
         ok = false;
         break;
       }
       sm100::tc_fence_after();
+      const int nsub = imin(C::kSub, p.nk - ks * C::kSub);
       const uint32_t a_addr = sm100::smem_addr(stages + stage * C::kStageBytes);
       const uint32_t b_addr = a_addr + C::kStageW;
 #pragma unroll
-      for (int kk = 0; kk < kBlockK / 16; ++kk) {
-        sm100::mma_bf16_ss(d_tmem, sm100::smem_desc_sw128(a_addr + kk * 32),
-                           sm100::smem_desc_sw128(b_addr + kk * 32), C::kIdesc,
-                           (kb | kk) != 0 ? 1u : 0u);
+      for (int j = 0; j < C::kSub; ++j) {
+        if (j >= nsub) break;
+#pragma unroll
+        for (int kk = 0; kk < kBlockK / 16; ++kk) {
+          const uint64_t da = sm100::smem_desc_sw128(a_addr + j * C::kSubW + kk * 32);
+          const uint64_t db = sm100::smem_desc_sw128(b_addr + j * C::kSubH + kk * 32);
+          const uint32_t acc = (ks | j | kk) != 0 ? 1u : 0u;
+          if constexpr (PAIR) {
+            sm100::mma_bf16_ss_pair(d_tmem, da, db, C::kIdesc, acc);
+          } else {
+            sm100::mma_bf16_ss(d_tmem, da, db, C::kIdesc, acc);
+          }
+        }
       }
-      sm100::mma_commit(&empty[stage]);  // frees the stage once these MMAs finish
+      // Frees the stage once these MMAs finish.
+      if constexpr (PAIR) {
+        sm100::mma_commit_pair(&empty[stage]);
+      } else {
+        sm100::mma_commit(&empty[stage]);
+      }
       if (++stage == C::kStages) {
         stage = 0;
         phase ^= 1u;
       }
     }
     if (!ok) break;
-    sm100::mma_commit(&acc_full[buf]);   // accumulator ready for the epilogue
+    // Accumulator ready for the epilogue.
+    if constexpr (PAIR) {
+      sm100::mma_commit_pair(&acc_full[buf]);
+    } else {
+      sm100::mma_commit(&acc_full[buf]);
+    }
     if (++buf == C::kAccBufs) {
       buf = 0;
       acc_phase ^= 1u;
     }
   }
   // Drain: every MMA issued above has completed once this arrives.
-  sm100::mma_commit(drain_bar);
+  if constexpr (PAIR) {
+    sm100::mma_commit_pair(drain_bar);
+  } else {
+    sm100::mma_commit(drain_bar);
+  }
   const long long t0 = clock64();
-  while (!sm100::mbar_try_wait(drain_bar, 0) && clock64() - t0 < sm100::kWaitLimitCycles) {
+  while (!sm100::mbar_try_wait<PAIR>(drain_bar, 0) && clock64() - t0 < sm100::kWaitLimitCycles) {
   }
 }
 
-template <int BN, int MODE>
+// Epilogue warps.  In pair mode each CTA drains its own 128 accumulator rows
+// (its half of the pair tile); the even CTA hands every filled accumulator on
+// to the odd CTA, and the odd CTA's warps release it on the even CTA's
+// barrier, where the MMAs are issued.
+template <int BN, int MODE, bool PAIR>
 __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedule &sch,
                                               uint32_t tmem_base, uint64_t *acc_full,
                                               uint64_t *acc_empty, volatile int *abort_flag,
                                               int *last_flag, uint64_t *comb_key, float *comb_m,
-                                              float *comb_s, int warp, int lane) {
-  using C = KCfg<BN, MODE>;
+                                              float *comb_s, int warp, int lane, int unit,
+                                              int rank) {
+  using C = KCfg<BN, MODE, PAIR>;
   constexpr int CW = C::kCW;
   const int q = warp & 3;          // TMEM lane quarter this warp may access
   const int h = (warp - 2) >> 2;   // which of the quarter's warps: chunks h, h+4, ...
@@ -403,7 +504,7 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
     s_run[i] = 0.f;
   }
 
-  TileIter it(sch, blockIdx.x);
+  TileIter it(sch, unit);
   Tile tile;
   int buf = 0;
   uint32_t phase = 0;
@@ -413,12 +514,15 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
     // so that every epilogue warp reaches the same named barriers.  The
     // decision is made warp-uniform because the TMEM loads below are
     // warp-collective.
-    const bool got = aborted ? false : sm100::wait_bounded(&acc_full[buf], phase, abort_flag, p.err);
+    const bool got = aborted ? false : sm100::wait_bounded<PAIR>(&acc_full[buf], phase, abort_flag, p.err);
     aborted = __any_sync(0xffffffffu, !got);
     if (!aborted) {
+      if (PAIR && rank == 0 && warp == 2 && lane == 0)
+        sm100::mbar_arrive_cluster(sm100::cluster_addr(&acc_full[buf], 1));
       sm100::tc_fence_after();
-      const int v = tile.start + 32 * q + lane;           // row of W in this launch
-      const bool v_ok = v >= tile.lo && v < tile.hi;
+      const Tile mine = PAIR ? pair_half(tile, rank) : tile;
+      const int v = mine.start + 32 * q + lane;           // row of W in this launch
+      const bool v_ok = v >= mine.lo && v < mine.hi;
       const int vg = v + p.vocab_offset;                  // global token index
       const uint32_t tbase =
           tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(buf * BN);
@@ -489,7 +593,13 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
       }
       sm100::tc_fence_before();
       __syncwarp();
-      if (lane == 0) sm100::mbar_arrive(&acc_empty[buf]);
+      if (lane == 0) {
+        if (PAIR && rank == 1) {
+          sm100::mbar_arrive_cluster(sm100::cluster_addr(&acc_empty[buf], 0));
+        } else {
+          sm100::mbar_arrive(&acc_empty[buf]);
+        }
+      }
     }
     if (++buf == C::kAccBufs) {
       buf = 0;
@@ -568,12 +678,12 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
 // ---------------------------------------------------------------------------
 // Kernel
 // ---------------------------------------------------------------------------
-template <int BN, int MODE>
+template <int BN, int MODE, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     fmms_kernel(const __grid_constant__ CUtensorMap tmap_w,
                 const __grid_constant__ CUtensorMap tmap_w8,
                 const __grid_constant__ CUtensorMap tmap_h, const FmmsParams p) {
-  using C = KCfg<BN, MODE>;
+  using C = KCfg<BN, MODE, PAIR>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -594,11 +704,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // Pair mode: the two CTAs of a cluster form schedule unit blockIdx.x / 2.
+  const int rank = PAIR ? static_cast<int>(sm100::cluster_ctarank()) : 0;
+  const int unit = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
   Schedule sch;
   sch.V = p.V;
   sch.G = p.G;
-  sch.num_ctas = p.num_ctas;
+  sch.num_ctas = PAIR ? p.num_ctas / 2 : p.num_ctas;
   sch.ngran = p.ngran;
+  sch.tile_rows = PAIR ? 2 * kTileM : kTileM;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
@@ -607,7 +721,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < C::kAccBufs; ++b) {
       sm100::mbar_init(&acc_full[b], 1);
-      sm100::mbar_init(&acc_empty[b], kNumEpiWarps);
+      sm100::mbar_init(&acc_empty[b], C::kEpiArrivals);
     }
     sm100::mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -618,9 +732,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     sm100::prefetch_tensormap(&tmap_w8);
     sm100::prefetch_tensormap(&tmap_h);
   }
-  if (warp == 1) {
-    sm100::tmem_alloc(tmem_slot, C::kTmemCols);
-    sm100::tmem_relinquish();
+  if constexpr (PAIR) {
+    // Both CTAs' barriers are initialised before either CTA signals the
+    // other's; the pair then allocates tensor memory collectively.
+    __syncthreads();
+    sm100::cluster_sync();
+    if (warp == 1) {
+      sm100::tmem_alloc_pair(tmem_slot, C::kTmemCols);
+      sm100::tmem_relinquish_pair();
+    }
+  } else {
+    if (warp == 1) {
+      sm100::tmem_alloc(tmem_slot, C::kTmemCols);
+      sm100::tmem_relinquish();
+    }
   }
   sm100::tc_fence_before();
   __syncthreads();
@@ -629,22 +754,34 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     if (lane == 0)
-      role_producer<BN, MODE>(&tmap_w, &tmap_w8, &tmap_h, p, sch, stages, full, empty, abort_flag);
+      role_producer<BN, MODE, PAIR>(&tmap_w, &tmap_w8, &tmap_h, p, sch, stages, full, empty,
+                                    abort_flag, unit, rank);
     __syncwarp();
   } else if (warp == 1) {
-    if (lane == 0)
-      role_mma<BN, MODE>(p, sch, stages, full, empty, acc_full, acc_empty, drain_bar, tmem_base,
-                   abort_flag);
+    if (lane == 0 && rank == 0)
+      role_mma<BN, MODE, PAIR>(p, sch, stages, full, empty, acc_full, acc_empty, drain_bar,
+                               tmem_base, abort_flag, unit);
     __syncwarp();
   } else {
-    role_epilogue<BN, MODE>(p, sch, tmem_base, acc_full, acc_empty, abort_flag, last_flag,
-                            comb_key, comb_m, comb_s, warp, lane);
+    role_epilogue<BN, MODE, PAIR>(p, sch, tmem_base, acc_full, acc_empty, abort_flag, last_flag,
+                                  comb_key, comb_m, comb_s, warp, lane, unit, rank);
   }
 
   sm100::tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) {
+    // Neither CTA frees tensor memory while the other may still use it: the
+    // even CTA's MMAs write both, and each CTA's epilogue reads its own.
+    sm100::cluster_sync();
+  }
   sm100::tc_fence_after();
-  if (warp == 1) sm100::tmem_dealloc(tmem_base, C::kTmemCols);
+  if (warp == 1) {
+    if constexpr (PAIR) {
+      sm100::tmem_dealloc_pair(tmem_base, C::kTmemCols);
+    } else {
+      sm100::tmem_dealloc(tmem_base, C::kTmemCols);
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -654,7 +791,7 @@ template <int BN, int MODE>
 static cudaError_t launch_t(const CUtensorMap &tw, const CUtensorMap &tw8, const CUtensorMap &th,
                             const FmmsParams &p, cudaStream_t stream) {
   using C = KCfg<BN, MODE>;
-  auto kern = fmms_kernel<BN, MODE>;
+  auto kern = fmms_kernel<BN, MODE, false>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
@@ -681,6 +818,80 @@ cudaError_t launch_fmms(int mode, int BN, const CUtensorMap &tw, const CUtensorM
     case kModeFlat: return launch_mode<kModeFlat>(BN, tw, tw8, th, p, stream);
     case kModeGrouped: return launch_mode<kModeGrouped>(BN, tw, tw8, th, p, stream);
     case kModeLogits: return launch_mode<kModeLogits>(BN, tw, tw8, th, p, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+// Pair kernels: clusters of two CTAs, p.num_ctas = 2 x schedule units.
+template <int BN>
+static cudaLaunchConfig_t pair_config(int num_ctas, cudaStream_t stream,
+                                      cudaLaunchAttribute *attr) {
+  using C = KCfg<BN, kModeFlat, true>;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(num_ctas), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = stream;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cfg;
+}
+
+template <int BN>
+static cudaError_t pair_units_t(int *units) {
+  using C = KCfg<BN, kModeFlat, true>;
+  auto kern = fmms_kernel<BN, kModeFlat, true>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = pair_config<BN>(2, nullptr, attr);
+  int n = 0;
+  e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+  if (e != cudaSuccess) return e;
+  *units = n;
+  return cudaSuccess;
+}
+
+template <int BN>
+static cudaError_t launch_pair_t(const CUtensorMap &tw, const CUtensorMap &tw8,
+                                 const CUtensorMap &th, const FmmsParams &p,
+                                 cudaStream_t stream) {
+  using C = KCfg<BN, kModeFlat, true>;
+  auto kern = fmms_kernel<BN, kModeFlat, true>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = pair_config<BN>(p.num_ctas, stream, attr);
+  e = cudaLaunchKernelEx(&cfg, kern, tw, tw8, th, p);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+cudaError_t fmms_pair_units(int BN, int *units) {
+  switch (BN) {
+    case 16: return pair_units_t<16>(units);
+    case 32: return pair_units_t<32>(units);
+    case 64: return pair_units_t<64>(units);
+    case 128: return pair_units_t<128>(units);
+    case 256: return pair_units_t<256>(units);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_fmms_pair(int BN, const CUtensorMap &tw, const CUtensorMap &tw8,
+                             const CUtensorMap &th, const FmmsParams &p, cudaStream_t stream) {
+  switch (BN) {
+    case 16: return launch_pair_t<16>(tw, tw8, th, p, stream);
+    case 32: return launch_pair_t<32>(tw, tw8, th, p, stream);
+    case 64: return launch_pair_t<64>(tw, tw8, th, p, stream);
+    case 128: return launch_pair_t<128>(tw, tw8, th, p, stream);
+    case 256: return launch_pair_t<256>(tw, tw8, th, p, stream);
     default: return cudaErrorInvalidValue;
   }
 }

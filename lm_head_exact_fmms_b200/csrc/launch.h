@@ -13,9 +13,17 @@ namespace fmms {
 int fmms_batch_tile(int rows);
 
 // The fused kernel in mode kModeFlat / kModeGrouped / kModeLogits with batch
-// tile BN, grid p.num_ctas x 320 threads.
+// tile BN, grid p.num_ctas x kThreads threads.
 cudaError_t launch_fmms(int mode, int BN, const CUtensorMap &tw, const CUtensorMap &tw8,
                         const CUtensorMap &th, const FmmsParams &p, cudaStream_t stream);
+
+// The flat kernel on CTA pairs (clusters of two, tcgen05 cta_group::2):
+// p.num_ctas CTAs (even), th with boxes of BN/2 rows.
+cudaError_t launch_fmms_pair(int BN, const CUtensorMap &tw, const CUtensorMap &tw8,
+                             const CUtensorMap &th, const FmmsParams &p, cudaStream_t stream);
+
+// How many CTA pairs of the BN pair kernel can be resident at once.
+cudaError_t fmms_pair_units(int BN, int *units);
 
 // Group-Gumbel-Max merge of the grouped partials of one launch (B rows).
 struct MergeParams {

@@ -1,0 +1,167 @@
+"""The flat kernel on CTA pairs (two SMs sharing one M = 256 tcgen05 MMA),
+and pipeline stages of one or two 64-wide K sub-blocks.
+
+The pair kernel is a B200 design choice, not part of the method, so the
+sampled tokens must be those of the single-CTA kernel bit for bit, and both
+must match the oracle within the stated tie tolerance.  Every batch tile
+(16..256 rows), ragged batches and vocabularies (pair tiles of 256 rows
+whose odd half is partly or wholly empty), masks, per-row seeds, several
+samples per row, vocabulary shards and the bounded-wait failure path are
+covered with the pair kernel forced on.
+"""
+import time
+
+import numpy as np
+import pytest
+import torch
+
+from lm_head_exact_fmms_b200 import binding, synth
+
+pytestmark = pytest.mark.gpu
+
+TIE_REL = 2e-3
+
+
+@pytest.fixture(scope="module")
+def dev():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from lm_head_exact_fmms_b200 import build
+    build.build()
+    binding.load_library()
+    yield torch.device("cuda:0")
+    binding.fs_set_cta_pairs(-1)
+
+
+def with_policy(policy, fn):
+    binding.fs_set_cta_pairs(policy)
+    try:
+        out = fn()
+        torch.cuda.synchronize()
+        return out
+    finally:
+        binding.fs_set_cta_pairs(-1)
+
+
+def both(fn):
+    """(single-CTA result, pair result) of the same call."""
+    return with_policy(0, fn), with_policy(1, fn)
+
+
+def assert_parity(gpu, o_idx, o_best, o_second, what=""):
+    gpu = np.asarray(gpu)
+    bad = gpu != o_idx
+    if bad.any():
+        tie = (o_best - o_second) <= TIE_REL * (1.0 + np.abs(o_best))
+        hard = bad & ~tie
+        assert not hard.any(), "%s: rows %s gpu %s oracle %s" % (
+            what, np.flatnonzero(hard)[:8], gpu[hard][:8], o_idx[hard][:8])
+
+
+def rand_inputs(B, d, V, seed, w_std=None):
+    H = synth.make_hidden(B, d, device="cpu", seed=seed)
+    W = synth.make_weight(V, d, w_std if w_std is not None else 1.0 / np.sqrt(d), device="cpu",
+                          seed=seed + 1)
+    return H, W, H.cuda(), W.cuda()
+
+
+def test_policy_argument_checked(dev):
+    with pytest.raises(binding.FmmsError):
+        binding.fs_set_cta_pairs(2)
+    with pytest.raises(binding.FmmsError):
+        binding.fs_set_cta_pairs(-2)
+    binding.fs_set_cta_pairs(-1)
+
+
+@pytest.mark.parametrize("B,d,V", [
+    (1, 256, 4096), (8, 64, 300), (9, 128, 5000), (16, 64, 129), (17, 96, 4097),
+    (33, 128, 777), (64, 256, 12345), (65, 64, 2000), (100, 128, 256), (128, 64, 8),
+    (129, 192, 3001), (200, 64, 9000), (256, 256, 4096), (257, 64, 1500), (300, 40, 640),
+    # K not a multiple of the stage's two 64-wide sub-blocks (last stage half
+    # full), and a K tail shorter than one sub-block
+    (40, 192, 3000), (100, 200, 2500), (120, 72, 999), (50, 8, 100),
+])
+def test_pairs_equal_single_and_oracle(dev, oracle, B, d, V):
+    H, W, Hd, Wd = rand_inputs(B, d, V, seed=3 * B + V)
+    single, pair = both(lambda: binding.fs_sample(Hd, Wd, temperature=0.9, seed=21, step=2))
+    assert torch.equal(single, pair), (B, d, V)
+    assert_parity(pair.cpu().numpy(), *oracle.sample(H, W, T=0.9, seed=21, step=2),
+                  "B=%d d=%d V=%d" % (B, d, V))
+
+
+def test_pairs_masks_row_seeds_and_fully_masked_rows(dev, oracle):
+    B, d, V = 70, 128, 6001
+    H, W, Hd, Wd = rand_inputs(B, d, V, seed=17)
+    rs = synth.make_row_seeds(B)
+    allowed = torch.rand(B, V, generator=torch.Generator().manual_seed(8)) < 0.3
+    allowed[5] = False                        # no allowed token: -1
+    allowed[6] = False
+    allowed[6, V - 1] = True                  # one allowed token: always it
+    mask = synth.mask_from_bool(allowed)
+    for step in (0, 7):
+        single, pair = both(lambda: binding.fs_sample_ex(
+            Hd, Wd, temperature=0.7, seed=3, row_seeds=rs.cuda(), step=step,
+            mask_bits=mask.cuda()))
+        assert torch.equal(single, pair)
+        got = pair.cpu().numpy()
+        assert got[5] == -1 and got[6] == V - 1
+        assert_parity(got, *oracle.sample(H, W, T=0.7, seed=3, row_seeds=rs, step=step,
+                                          mask=mask), "masked step %d" % step)
+
+
+def test_pairs_multi_sample_and_shards(dev, oracle):
+    from lm_head_exact_fmms_b200.tp import shard_bounds
+    B, d, V, S = 96, 128, 7003, 3
+    H, W, Hd, Wd = rand_inputs(B, d, V, seed=29)
+    single, pair = both(lambda: binding.fs_sample_multi(Hd, Wd, S, temperature=1.1, seed=6,
+                                                        step=4))
+    assert torch.equal(single, pair)
+    idx, best, second = oracle.sample_multi(H, W, S, T=1.1, seed=6, step=4)
+    assert_parity(pair.cpu().numpy().ravel(), idx.ravel(), best.ravel(), second.ravel(), "multi")
+
+    def shards():
+        keys = [binding.fs_sample_shard_keys(Hd, Wd[lo:hi].contiguous(), lo, V, temperature=1.1,
+                                             seed=6, step=4)
+                for lo, hi in shard_bounds(V, 3)]
+        return binding.fs_keys_to_tokens(torch.stack(keys).max(dim=0).values.contiguous())
+    ref = with_policy(0, lambda: binding.fs_sample(Hd, Wd, temperature=1.1, seed=6, step=4))
+    assert torch.equal(with_policy(1, shards), ref)
+
+
+@pytest.mark.parametrize("B", [128, 256])
+def test_pairs_full_size_head(dev, oracle, B):
+    """The Qwen3-8B-shaped head the benchmark times: pair and single kernels
+    agree on every row; the oracle checks sampled rows."""
+    wl = synth.WORKLOADS["qwen3-8b"]
+    Wd = synth.make_weight(wl.V, wl.d, wl.w_std, device=dev)
+    Hd = synth.make_hidden(B, wl.d, device=dev)
+    rs = synth.make_row_seeds(B)
+    single, pair = both(lambda: binding.fs_sample_ex(Hd, Wd, temperature=wl.temperature, seed=0,
+                                                     row_seeds=rs.to(dev), step=0))
+    assert torch.equal(single, pair)
+    rows = np.array([0, B // 3, B - 1], dtype=np.int32)
+    idx, best, second = oracle.sample(Hd.cpu(), Wd.cpu(), T=wl.temperature, seed=0, row_seeds=rs,
+                                      step=0, rows=rows)
+    assert_parity(pair.cpu().numpy()[rows], idx, best, second, "qwen3-8b B=%d" % B)
+    del Wd, Hd
+    torch.cuda.empty_cache()
+
+
+def test_pairs_wait_timeout_is_reported_and_context_survives(dev, oracle):
+    """No loads are issued, so the even CTA's MMA wait and then every
+    epilogue wait of both CTAs of each pair run out; the kernel records
+    FS_ERR_DEVICE_TIMEOUT and exits, and the context samples correctly after."""
+    B, d, V = 160, 64, 4096
+    H = synth.make_hidden(B, d, seed=13)
+    W = synth.make_weight(V, d, 0.125, seed=14)
+    Hd, Wd = H.to(dev), W.to(dev)
+    ws = torch.zeros(binding.fs_workspace_bytes(B, V, 0), dtype=torch.uint8, device=dev)
+    t0 = time.time()
+    with_policy(1, lambda: binding.fs_test_stalled_sample(Hd, Wd, ws))
+    status = binding.fs_device_status(ws)
+    assert status == 5, binding.fs_status_string(status)
+    assert time.time() - t0 < 120
+    got = with_policy(1, lambda: binding.fs_sample_ex(Hd, Wd, temperature=1.0, seed=2, step=1,
+                                                      workspace=ws))
+    assert_parity(got.cpu().numpy(), *oracle.sample(H, W, T=1.0, seed=2, step=1), "after")
+    assert binding.fs_device_status(ws) == 0
