@@ -47,11 +47,11 @@
  *  workspace  entry points that take (workspace, workspace_bytes) use the
  *         caller's device buffer of at least fs_workspace_bytes(B, V, G) bytes,
  *         256-byte aligned, which must be zero-filled before its first use
- *         (cudaMemset).  Every call that completes leaves the parts that must
- *         start at zero (status, ticket, per-row keys, published maxima)
- *         zeroed again; the grouped calls' partials are per-call scratch.  One
- *         workspace may serve calls of any kind and size it is large enough
- *         for.  Calls that share a workspace must be ordered on one stream.  With
+ *         (cudaMemset).  Every call that completes leaves every byte it used
+ *         zeroed again (status, ticket, per-row keys, the grouped calls'
+ *         partials and published maxima), so one workspace may serve calls of
+ *         any kind and size it is large enough for, whatever part of it each
+ *         call lays out where.  Calls that share a workspace must be ordered on one stream.  With
  *         workspace == NULL the library uses its own per-device workspace,
  *         allocated on first use; such calls must not run concurrently on
  *         different streams.
@@ -309,15 +309,18 @@ fs_status fs_test_stalled_sample(const void *H, const void *W, int B, int d,
 /* ---- Kernel choice ---- */
 
 /* Whether flat-mode calls (fs_sample, fs_sample_ex, fs_sample_host,
- * fs_sample_noalloc, fs_sample_multi, fs_sample_shard_keys) run the fused
- * kernel on CTA pairs: clusters of two CTAs on two SMs that share one
- * M = 256 tensor-core MMA (tcgen05 cta_group::2), each SM staging 128 rows
- * of W and half of the batch rows of H per pipeline stage.  This is a B200
- * design choice, not part of the method: the sampled tokens are the same
- * either way.  policy: -1 automatic (the default: pairs for launches of more
- * than 64 batch rows), 0 never, 1 always.  Process-wide; applies to calls
- * made after it returns.  FS_ERR_INVALID_ARG for any other value.  When the
- * device cannot co-schedule a pair, the single-CTA kernel runs. */
+ * fs_sample_noalloc, fs_sample_multi, fs_sample_shard_keys) and grouped calls
+ * (fs_sample_grouped, fs_summarize_group) run the fused kernel on CTA pairs:
+ * clusters of two CTAs on two SMs that share one M = 256 tensor-core MMA
+ * (tcgen05 cta_group::2), each SM staging 128 rows of W and half of the batch
+ * rows of H per pipeline stage.  This is a B200 design choice, not part of
+ * the method: the results are the same either way (tokens bit for bit).
+ * policy: -1 automatic (the default: pairs for launches of more than 64
+ * batch rows), 0 never, 1 always.  Process-wide; applies to calls made after
+ * it returns.  FS_ERR_INVALID_ARG for any other value.  When the device
+ * cannot co-schedule a pair, the single-CTA kernel runs.  The unfused
+ * measurement path (fs_sample_unfused, fs_sample_topk) always runs on single
+ * CTAs. */
 fs_status fs_set_cta_pairs(int policy);
 
 /* ---- Host-only schedule query (no GPU needed) ---- */

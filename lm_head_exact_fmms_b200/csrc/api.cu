@@ -29,7 +29,7 @@ struct DeviceState {
   size_t h_stage_bytes = 0;
   void *o_stage = nullptr;  // fs_sample_host: device tokens
   size_t o_stage_bytes = 0;
-  int pair_units[5] = {-1, -1, -1, -1, -1};  // resident CTA pairs per batch tile (-1: unknown)
+  int pair_units[2][5] = {{-1, -1, -1, -1, -1}, {-1, -1, -1, -1, -1}};  // [flat, grouped][tile]
 };
 
 constexpr int kMaxDevices = 64;
@@ -197,12 +197,13 @@ int bn_index(int BN) {
   return BN <= 16 ? 0 : BN <= 32 ? 1 : BN <= 64 ? 2 : BN <= 128 ? 3 : 4;
 }
 
-// CTA pairs of the BN pair kernel that fit on the device at once (0: none).
-int pair_units(DeviceState *st, int BN) {
-  int &u = st->pair_units[bn_index(BN)];
+// CTA pairs of the BN pair kernel of `mode` that fit on the device at once
+// (0: none).
+int pair_units(DeviceState *st, int mode, int BN) {
+  int &u = st->pair_units[mode == fmms::kModeGrouped ? 1 : 0][bn_index(BN)];
   if (u < 0) {
     int n = 0;
-    if (fmms::fmms_pair_units(BN, &n) != cudaSuccess) {
+    if (fmms::fmms_pair_units(mode, BN, &n) != cudaSuccess) {
       cudaGetLastError();  // clear the error; the single-CTA kernel is used
       n = 0;
     }
@@ -211,11 +212,12 @@ int pair_units(DeviceState *st, int BN) {
   return u;
 }
 
-// Flat calls with a batch tile of 128 or more rows run on CTA pairs: each SM
-// then stages half of H per stage, which halves the batch operand's L2
-// traffic where it matters.
+// Flat and grouped calls with a batch tile of 128 or more rows run on CTA
+// pairs: each SM then stages half of H per stage, which halves the batch
+// operand's L2 traffic and the MMA issues per byte of W where the tensor
+// cores are busy.
 bool use_pairs(int mode, int BN) {
-  if (mode != fmms::kModeFlat || g_pair_policy == 0) return false;
+  if (mode == fmms::kModeLogits || g_pair_policy == 0) return false;
   return g_pair_policy == 1 || BN >= 128;
 }
 
@@ -267,7 +269,7 @@ fs_status run_locked(int mode, const void *H, const void *W, int B, int d, int V
   for (int b0 = 0; b0 < B; b0 += fmms::kMaxBN) {
     const int Bc = fmms::imin(fmms::kMaxBN, B - b0);
     const int BN = fmms::fmms_batch_tile(Bc);
-    const int units = use_pairs(mode, BN) ? pair_units(st, BN) : 0;
+    const int units = use_pairs(mode, BN) ? pair_units(st, mode, BN) : 0;
     const bool pair = units > 0;
     CUtensorMap th;
     if ((s = tensor_map(&th, H, d, B, pair ? BN / 2 : BN)) != FS_OK) return s;
@@ -298,9 +300,11 @@ fs_status run_locked(int mode, const void *H, const void *W, int B, int d, int V
     p.vocab_offset = shard.vocab_offset;
     p.out_keys = shard.out_keys ? shard.out_keys + static_cast<size_t>(b0) * S : nullptr;
     p.num_samples = S;
+    const int pair_units_used = pair ? fmms::make_schedule(V, sch.G, units).num_ctas : 0;
     if (pair) {
-      p.num_ctas = 2 * fmms::make_schedule(V, 1, units).num_ctas;
-      if (fmms::launch_fmms_pair(BN, tw, tw8, th, p, stream) != cudaSuccess) return FS_ERR_CUDA;
+      p.num_ctas = 2 * pair_units_used;
+      if (fmms::launch_fmms_pair(mode, BN, tw, tw8, th, p, stream) != cudaSuccess)
+        return FS_ERR_CUDA;
     } else {
       if (fmms::launch_fmms(mode, BN, tw, tw8, th, p, stream) != cudaSuccess) return FS_ERR_CUDA;
     }
@@ -313,7 +317,8 @@ fs_status run_locked(int mode, const void *H, const void *W, int B, int d, int V
       m.b_off = b0;
       m.V = V;
       m.G = sch.G;
-      m.num_ctas = sch.num_ctas;
+      m.num_ctas = pair ? pair_units_used : sch.num_ctas;
+      m.pair = pair ? 1 : 0;
       m.ngran = sch.ngran;
       m.seed = seed;
       m.row_seeds = row_seeds;

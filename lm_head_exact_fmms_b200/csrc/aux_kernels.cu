@@ -42,8 +42,12 @@ __global__ void __launch_bounds__(128) group_merge_kernel(const MergeParams m) {
     const int c_last = cta_of(hi - 1, sch);
     unsigned long long kmax = 0ull;
     float M = -INFINITY, S = 0.f;
-    for (int c = c_first; c <= c_last; ++c) {
-      const GroupPartial gp = m.partials[static_cast<size_t>(c + g) * m.B + b];
+    const int per_unit = m.pair ? 2 : 1;
+    for (int u = c_first * per_unit; u < (c_last + 1) * per_unit; ++u) {
+      const size_t slot = m.pair ? 2 * static_cast<size_t>(u / 2 + g) + (u & 1)
+                                 : static_cast<size_t>(u + g);
+      const GroupPartial gp = m.partials[slot * m.B + b];
+      m.partials[slot * m.B + b] = GroupPartial{0ull, 0.f, 0.f};  // leave the workspace zeroed
       kmax = gp.key > kmax ? gp.key : kmax;
       if (gp.m != -INFINITY) {
         if (M == -INFINITY) {

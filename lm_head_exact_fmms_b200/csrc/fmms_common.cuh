@@ -196,18 +196,23 @@ struct FmmsParams {
 // packed keys [sample][256 rows], of which a flat call uses (and needs) only
 // its samples' part; then, grouped only, the partials [slots][rows] and, for
 // G <= kMaxPublishedGroups, the published per-group maxima [G][rows] that
-// sharpen the exact-score filter (re-zeroed by the merge kernel).  Keys, the
-// ticket and the published maxima are left zeroed by every completed call;
-// partials are per-call scratch, each written before it is read.
+// sharpen the exact-score filter.  Where the partials and maxima lie depends
+// on (B, G), so one call's published maxima may sit where an earlier call
+// kept partials: every completed call therefore leaves all it used zeroed
+// (the merge kernel zeroes each partial it reads and each published maximum),
+// and every call finds its published maxima at zero.
 constexpr int kWsHeader = 256;
 constexpr int kWsKeys = 8 * kMaxBN;
 constexpr int kMaxPublishedGroups = 4096;
 constexpr int kMaxSamples = 64;
 constexpr int kWsKeysRegion = kMaxSamples * kWsKeys;
 
+// Partial slots: num_ctas + G - 1 for single CTAs; a CTA pair writes two
+// slots per (pair, group) segment, 2 (pairs + G - 1) in all, and a launch
+// never has more pairs than the single-CTA schedule has CTAs.
 FS_HD int64_t ws_partials_bytes(int B, int G, int num_ctas) {
   const int64_t rows = B < kMaxBN ? B : kMaxBN;
-  return (int64_t)(num_ctas + G - 1) * rows * (int64_t)sizeof(GroupPartial);
+  return 2 * (int64_t)(num_ctas + G - 1) * rows * (int64_t)sizeof(GroupPartial);
 }
 
 FS_HD int64_t ws_gkeys_bytes(int B, int G) {

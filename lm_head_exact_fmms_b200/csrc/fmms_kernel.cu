@@ -61,7 +61,7 @@ constexpr int ksub_for(int h_rows, int comb_bytes) {
 
 template <int BN, int MODE, bool PAIR = false>
 struct KCfg {
-  static_assert(!PAIR || MODE == kModeFlat, "CTA pairs run the flat mode only");
+  static_assert(!PAIR || MODE != kModeLogits, "the logits mode runs on single CTAs");
   static constexpr int kHRows = PAIR ? BN / 2 : BN;     // H rows this CTA stages
   static constexpr int kCombBytes = MODE == kModeGrouped ? 4 * BN * 16 : 0;  // grouped only
   static constexpr int kSub = ksub_for(kHRows, kCombBytes);  // 64-wide K blocks per stage
@@ -202,24 +202,43 @@ __device__ __forceinline__ void chunk_noise(const FmmsParams &p, int v, int col0
   }
 }
 
+// Transpose of the 32 x 32 bit matrix whose row r is lane r's x: afterwards
+// lane c holds the bits c of every lane's x, lane r's bit at position r.
+// Five rounds of swapping the off-diagonal blocks of size 16, 8, 4, 2, 1.
+__device__ __forceinline__ uint32_t bit_transpose32(uint32_t x, int lane) {
+  const uint32_t kMasks[5] = {0x0000FFFFu, 0x00FF00FFu, 0x0F0F0F0Fu, 0x33333333u, 0x55555555u};
+#pragma unroll
+  for (int i = 0, sft = 16; i < 5; ++i, sft >>= 1) {
+    const uint32_t m = kMasks[i];
+    const uint32_t y = __shfl_xor_sync(0xffffffffu, x, sft);
+    x = (lane & sft) ? ((x & ~m) | ((y >> sft) & m)) : ((x & m) | ((y & m) << sft));
+  }
+  return x;
+}
+
 // Bit j set when (row col0 + j, token v) is in range and, with a mask,
-// allowed for that row.
+// allowed for that row.  Warp-collective: the warp's lanes hold 32
+// consecutive tokens.  Lane j < CW gathers row col0 + j's 32 mask bits of
+// those tokens (two words at most); a bit-matrix transpose then hands every
+// lane its own token's bit of each row.
 template <int CW>
 __device__ __forceinline__ uint32_t chunk_allowed(const FmmsParams &p, int v, bool v_ok,
-                                                  int col0) {
-  uint32_t bits = 0;
-#pragma unroll
-  for (int j = 0; j < CW; ++j) {
-    const int col = col0 + j;
-    bool ok = v_ok && col < p.B;
-    if (ok && p.mask != nullptr) {
-      const uint32_t word =
-          __ldg(p.mask + static_cast<size_t>(p.b_off + col) * p.mask_words + (v >> 5));
-      ok = ((word >> (v & 31)) & 1u) != 0;
-    }
-    bits |= (ok ? 1u : 0u) << j;
+                                                  int col0, int lane) {
+  const int n = p.B - col0;
+  const uint32_t in_range = n >= CW ? ((1u << CW) - 1u) : ((1u << n) - 1u);
+  if (p.mask == nullptr) return v_ok ? in_range : 0u;
+  const int v0 = v - lane;  // token of lane 0 (a multiple of 8)
+  uint32_t rowbits = 0u;
+  if (lane < CW && lane < n) {
+    const uint32_t *row = p.mask + static_cast<size_t>(p.b_off + col0 + lane) * p.mask_words;
+    const int w0 = v0 >> 5;
+    const int sh = v0 & 31;
+    const uint32_t lo = w0 < p.mask_words ? __ldg(row + w0) : 0u;
+    const uint32_t hi = (sh != 0 && w0 + 1 < p.mask_words) ? __ldg(row + w0 + 1) : 0u;
+    rowbits = sh == 0 ? lo : ((lo >> sh) | (hi << (32 - sh)));
   }
-  return bits;
+  const uint32_t bits = bit_transpose32(rowbits, lane);
+  return v_ok ? (bits & in_range) : 0u;
 }
 
 // Bit j set when (row col0 + j, token v) is in range, mask not consulted.
@@ -495,13 +514,16 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
   const int etid = (warp - 2) * 32 + lane;
   const bool has_chunks = h < C::kChunks;
 
-  uint64_t best[C::kChunksPerWarp];
-  float m_run[C::kChunksPerWarp], s_run[C::kChunksPerWarp];
-#pragma unroll
-  for (int i = 0; i < C::kChunksPerWarp; ++i) {
-    best[i] = 0ull;
-    m_run[i] = -INFINITY;
-    s_run[i] = 0.f;
+  // Grouped mode: the running (best key, max, sum) of each (lane quarter,
+  // column) over the current segment live in shared memory, [4][BN] each,
+  // which keeps them out of the registers the chunk arithmetic needs.
+  if constexpr (MODE == kModeGrouped) {
+    for (int i = etid; i < 4 * BN; i += kEpiThreads) {
+      comb_key[i] = 0ull;
+      comb_m[i] = -INFINITY;
+      comb_s[i] = 0.f;
+    }
+    sm100::epi_sync(kEpiThreads);
   }
 
   TileIter it(sch, unit);
@@ -564,7 +586,7 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
               chunk_noise<CW>(p, vg, col0, lane, 2u * static_cast<uint32_t>(smp), words);
               if (chunk_any_candidate<CW>(acc, words, p, in_range, 0ull, pub, lane)) {
                 if (!have_allowed) {
-                  allowed = chunk_allowed<CW>(p, vg, v_ok, col0);
+                  allowed = chunk_allowed<CW>(p, vg, v_ok, col0, lane);
                   have_allowed = true;
                 }
                 uint64_t cbest = 0ull;
@@ -575,18 +597,24 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
             }
           } else {
             unsigned long long *gk =
-                p.gkeys ? p.gkeys + static_cast<size_t>(tile.slot - blockIdx.x) * p.B + c
-                        : nullptr;
+                p.gkeys ? p.gkeys + static_cast<size_t>(tile.slot - unit) * p.B + c : nullptr;
             const uint64_t pub = (gk != nullptr && c < p.B) ? ld_key(gk) : 0ull;
-            const uint32_t allowed = chunk_allowed<CW>(p, vg, v_ok, col0);
+            const uint32_t allowed = chunk_allowed<CW>(p, vg, v_ok, col0, lane);
             uint32_t words[CW];
             chunk_noise<CW>(p, vg, col0, lane, 0u, words);
-            chunk_lse<CW>(acc, p, allowed, lane, m_run[kk], s_run[kk]);
-            if (chunk_any_candidate<CW>(acc, words, p, allowed, best[kk], pub, lane)) {
-              chunk_keys<CW>(acc, words, p, vg, allowed, lane, best[kk]);
-              if (gk != nullptr && (lane & 1) == 0 && c < p.B && key_valid(best[kk]) &&
-                  best[kk] > pub)
-                atomicMax(gk, static_cast<unsigned long long>(best[kk]));
+            const int si = q * BN + c;  // this lane's (quarter, column) state
+            float m_run = comb_m[si], s_run = comb_s[si];
+            uint64_t best = comb_key[si];
+            chunk_lse<CW>(acc, p, allowed, lane, m_run, s_run);
+            if (chunk_any_candidate<CW>(acc, words, p, allowed, best, pub, lane)) {
+              chunk_keys<CW>(acc, words, p, vg, allowed, lane, best);
+              if (gk != nullptr && (lane & 1) == 0 && c < p.B && key_valid(best) && best > pub)
+                atomicMax(gk, static_cast<unsigned long long>(best));
+            }
+            if ((lane & 1) == 0) {  // the two lanes of a column hold the same values
+              comb_key[si] = best;
+              comb_m[si] = m_run;
+              comb_s[si] = s_run;
             }
           }
         }
@@ -608,37 +636,30 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
 
     if constexpr (MODE == kModeGrouped) {
       if (tile.last) {
-        // Segment done: combine the four lane quarters and write the partial.
-#pragma unroll
-        for (int kk = 0; kk < C::kChunksPerWarp; ++kk) {
-          if (!has_chunks) continue;
-          const int k = kk * C::kWarpsPerQuarter + h;
-          const int col = k * CW + column_of_lane<CW>(lane);
-          if (k * CW < p.B) {
-            comb_key[q * BN + col] = best[kk];
-            comb_m[q * BN + col] = m_run[kk];
-            comb_s[q * BN + col] = s_run[kk];
-          }
-          best[kk] = 0ull;
-          m_run[kk] = -INFINITY;
-          s_run[kk] = 0.f;
-        }
+        // Segment done: combine the four lane quarters, write the partial
+        // (slot per CTA: a pair's two CTAs write slots 2 s and 2 s + 1) and
+        // reset the state for the next segment.
         sm100::epi_sync(kEpiThreads);
-        if (!*abort_flag) {
-          for (int b = etid; b < p.B; b += kEpiThreads) {
-            uint64_t kb = 0ull;
-            float m = -INFINITY, s = 0.f;
+        const size_t slot = PAIR ? 2 * static_cast<size_t>(tile.slot) + rank
+                                 : static_cast<size_t>(tile.slot);
+        for (int b = etid; b < BN; b += kEpiThreads) {
+          uint64_t kb = 0ull;
+          float m = -INFINITY, s = 0.f;
 #pragma unroll
-            for (int qq = 0; qq < 4; ++qq) {
-              const uint64_t kq = comb_key[qq * BN + b];
-              kb = kq > kb ? kq : kb;
-              lse_merge(m, s, comb_m[qq * BN + b], comb_s[qq * BN + b]);
-            }
+          for (int qq = 0; qq < 4; ++qq) {
+            const uint64_t kq = comb_key[qq * BN + b];
+            kb = kq > kb ? kq : kb;
+            lse_merge(m, s, comb_m[qq * BN + b], comb_s[qq * BN + b]);
+            comb_key[qq * BN + b] = 0ull;
+            comb_m[qq * BN + b] = -INFINITY;
+            comb_s[qq * BN + b] = 0.f;
+          }
+          if (b < p.B && !*abort_flag) {
             GroupPartial gp;
             gp.key = kb;
             gp.m = m;
             gp.sum = s;
-            p.partials[static_cast<size_t>(tile.slot) * p.B + b] = gp;
+            p.partials[slot * p.B + b] = gp;
           }
         }
         sm100::epi_sync(kEpiThreads);
@@ -823,10 +844,10 @@ cudaError_t launch_fmms(int mode, int BN, const CUtensorMap &tw, const CUtensorM
 }
 
 // Pair kernels: clusters of two CTAs, p.num_ctas = 2 x schedule units.
-template <int BN>
+template <int BN, int MODE>
 static cudaLaunchConfig_t pair_config(int num_ctas, cudaStream_t stream,
                                       cudaLaunchAttribute *attr) {
-  using C = KCfg<BN, kModeFlat, true>;
+  using C = KCfg<BN, MODE, true>;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(num_ctas), 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
@@ -841,15 +862,15 @@ static cudaLaunchConfig_t pair_config(int num_ctas, cudaStream_t stream,
   return cfg;
 }
 
-template <int BN>
+template <int BN, int MODE>
 static cudaError_t pair_units_t(int *units) {
-  using C = KCfg<BN, kModeFlat, true>;
-  auto kern = fmms_kernel<BN, kModeFlat, true>;
+  using C = KCfg<BN, MODE, true>;
+  auto kern = fmms_kernel<BN, MODE, true>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   cudaLaunchAttribute attr[1];
-  cudaLaunchConfig_t cfg = pair_config<BN>(2, nullptr, attr);
+  cudaLaunchConfig_t cfg = pair_config<BN, MODE>(2, nullptr, attr);
   int n = 0;
   e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
   if (e != cudaSuccess) return e;
@@ -857,41 +878,61 @@ static cudaError_t pair_units_t(int *units) {
   return cudaSuccess;
 }
 
-template <int BN>
+template <int BN, int MODE>
 static cudaError_t launch_pair_t(const CUtensorMap &tw, const CUtensorMap &tw8,
                                  const CUtensorMap &th, const FmmsParams &p,
                                  cudaStream_t stream) {
-  using C = KCfg<BN, kModeFlat, true>;
-  auto kern = fmms_kernel<BN, kModeFlat, true>;
+  using C = KCfg<BN, MODE, true>;
+  auto kern = fmms_kernel<BN, MODE, true>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   cudaLaunchAttribute attr[1];
-  cudaLaunchConfig_t cfg = pair_config<BN>(p.num_ctas, stream, attr);
+  cudaLaunchConfig_t cfg = pair_config<BN, MODE>(p.num_ctas, stream, attr);
   e = cudaLaunchKernelEx(&cfg, kern, tw, tw8, th, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
-cudaError_t fmms_pair_units(int BN, int *units) {
+template <int MODE>
+static cudaError_t pair_units_mode(int BN, int *units) {
   switch (BN) {
-    case 16: return pair_units_t<16>(units);
-    case 32: return pair_units_t<32>(units);
-    case 64: return pair_units_t<64>(units);
-    case 128: return pair_units_t<128>(units);
-    case 256: return pair_units_t<256>(units);
+    case 16: return pair_units_t<16, MODE>(units);
+    case 32: return pair_units_t<32, MODE>(units);
+    case 64: return pair_units_t<64, MODE>(units);
+    case 128: return pair_units_t<128, MODE>(units);
+    case 256: return pair_units_t<256, MODE>(units);
     default: return cudaErrorInvalidValue;
   }
 }
 
-cudaError_t launch_fmms_pair(int BN, const CUtensorMap &tw, const CUtensorMap &tw8,
-                             const CUtensorMap &th, const FmmsParams &p, cudaStream_t stream) {
+template <int MODE>
+static cudaError_t launch_pair_mode(int BN, const CUtensorMap &tw, const CUtensorMap &tw8,
+                                    const CUtensorMap &th, const FmmsParams &p,
+                                    cudaStream_t stream) {
   switch (BN) {
-    case 16: return launch_pair_t<16>(tw, tw8, th, p, stream);
-    case 32: return launch_pair_t<32>(tw, tw8, th, p, stream);
-    case 64: return launch_pair_t<64>(tw, tw8, th, p, stream);
-    case 128: return launch_pair_t<128>(tw, tw8, th, p, stream);
-    case 256: return launch_pair_t<256>(tw, tw8, th, p, stream);
+    case 16: return launch_pair_t<16, MODE>(tw, tw8, th, p, stream);
+    case 32: return launch_pair_t<32, MODE>(tw, tw8, th, p, stream);
+    case 64: return launch_pair_t<64, MODE>(tw, tw8, th, p, stream);
+    case 128: return launch_pair_t<128, MODE>(tw, tw8, th, p, stream);
+    case 256: return launch_pair_t<256, MODE>(tw, tw8, th, p, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t fmms_pair_units(int mode, int BN, int *units) {
+  switch (mode) {
+    case kModeFlat: return pair_units_mode<kModeFlat>(BN, units);
+    case kModeGrouped: return pair_units_mode<kModeGrouped>(BN, units);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_fmms_pair(int mode, int BN, const CUtensorMap &tw, const CUtensorMap &tw8,
+                             const CUtensorMap &th, const FmmsParams &p, cudaStream_t stream) {
+  switch (mode) {
+    case kModeFlat: return launch_pair_mode<kModeFlat>(BN, tw, tw8, th, p, stream);
+    case kModeGrouped: return launch_pair_mode<kModeGrouped>(BN, tw, tw8, th, p, stream);
     default: return cudaErrorInvalidValue;
   }
 }

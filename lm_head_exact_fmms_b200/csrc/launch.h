@@ -17,19 +17,20 @@ int fmms_batch_tile(int rows);
 cudaError_t launch_fmms(int mode, int BN, const CUtensorMap &tw, const CUtensorMap &tw8,
                         const CUtensorMap &th, const FmmsParams &p, cudaStream_t stream);
 
-// The flat kernel on CTA pairs (clusters of two, tcgen05 cta_group::2):
-// p.num_ctas CTAs (even), th with boxes of BN/2 rows.
-cudaError_t launch_fmms_pair(int BN, const CUtensorMap &tw, const CUtensorMap &tw8,
+// The flat or grouped kernel on CTA pairs (clusters of two, tcgen05
+// cta_group::2): p.num_ctas CTAs (even), th with boxes of BN/2 rows.
+cudaError_t launch_fmms_pair(int mode, int BN, const CUtensorMap &tw, const CUtensorMap &tw8,
                              const CUtensorMap &th, const FmmsParams &p, cudaStream_t stream);
 
-// How many CTA pairs of the BN pair kernel can be resident at once.
-cudaError_t fmms_pair_units(int BN, int *units);
+// How many CTA pairs of the BN pair kernel of `mode` can be resident at once.
+cudaError_t fmms_pair_units(int mode, int BN, int *units);
 
 // Group-Gumbel-Max merge of the grouped partials of one launch (B rows).
 struct MergeParams {
-  const GroupPartial *partials;  // [num_ctas + G - 1][B]
+  GroupPartial *partials;        // [slots][B]; zeroed as they are read
   unsigned long long *gkeys;     // [G][B] published maxima to re-zero, or null
   int B, b_off, V, G, num_ctas, ngran;
+  int pair;                      // 1: partials of a CTA-pair launch (two slots per segment)
   uint64_t seed;
   const uint64_t *row_seeds;
   uint32_t step;

@@ -165,3 +165,65 @@ def test_pairs_wait_timeout_is_reported_and_context_survives(dev, oracle):
                                                       workspace=ws))
     assert_parity(got.cpu().numpy(), *oracle.sample(H, W, T=1.0, seed=2, step=1), "after")
     assert binding.fs_device_status(ws) == 0
+
+
+@pytest.mark.parametrize("B,d,V,G,masked", [
+    (20, 64, 6007, 3, True), (70, 128, 9001, 8, True), (130, 64, 5000, 1, False),
+    (160, 96, 12000, 64, False), (256, 128, 8192, 8, True), (300, 64, 3000, 1000, True),
+])
+def test_pairs_grouped(dev, oracle, B, d, V, G, masked):
+    """Group-Gumbel-Max on CTA pairs: per-group maxima and their tokens equal
+    the single-CTA kernel's bit for bit; the group log-sum-exps (merged in
+    another order) agree to float rounding; the tokens follow the oracle."""
+    H, W, Hd, Wd = rand_inputs(B, d, V, seed=B + G)
+    mask = synth.make_mask(B, V, 0.5, seed=G) if masked else None
+    md = mask.to(dev) if masked else None
+
+    def call():
+        summ = torch.empty(B, G, 3, dtype=torch.float32, device=dev)
+        tok = binding.fs_sample_grouped(Hd, Wd, G, temperature=0.8, seed=12, step=2,
+                                        mask_bits=md, out_summary=summ)
+        return tok, summ
+
+    (t0, s0), (t1, s1) = both(call)
+    a0, a1 = s0.cpu(), s1.cpu()
+    # max score and argmax, bitwise (argmax -1 of an all-masked group reads as NaN)
+    assert torch.equal(a0[:, :, :2].contiguous().view(torch.int32),
+                       a1[:, :, :2].contiguous().view(torch.int32))
+    l0, l1 = a0[:, :, 2].numpy(), a1[:, :, 2].numpy()
+    fin = np.isfinite(l0)
+    assert np.array_equal(fin, np.isfinite(l1))
+    assert np.allclose(l0[fin], l1[fin], rtol=1e-6, atol=1e-5)
+    idx, o_summ, margin = oracle.sample_grouped(H, W, G, T=0.8, seed=12, step=2, mask=mask)
+    got = t1.cpu().numpy()
+    for b in np.flatnonzero(got != idx):
+        scale = TIE_REL * (1 + abs(o_summ[b, :, 0].max()))
+        assert margin[b, 0] <= scale or margin[b, 1] <= scale, (b, got[b], idx[b])
+    assert (t0.cpu().numpy() == got).mean() > 0.99
+    if G == 1:
+        flat = with_policy(1, lambda: binding.fs_sample_ex(Hd, Wd, temperature=0.8, seed=12,
+                                                           step=2, mask_bits=md))
+        assert torch.equal(flat, t1)
+
+
+def test_pairs_grouped_full_size_head(dev, oracle):
+    """The grouped-masked workload at B = 512 (two pair launches): pair and
+    single kernels agree on every row; the oracle checks sampled rows."""
+    wl = synth.WORKLOADS["grouped-masked"]
+    B = 512
+    Wd = synth.make_weight(wl.V, wl.d, wl.w_std, device=dev)
+    Hd = synth.make_hidden(B, wl.d, device=dev)
+    mask = synth.make_mask(B, wl.V, wl.mask_allowed)
+    single, pair = both(lambda: binding.fs_sample_grouped(Hd, Wd, wl.groups,
+                                                          temperature=wl.temperature, seed=0,
+                                                          step=0, mask_bits=mask.to(dev)))
+    assert (single == pair).float().mean().item() > 0.99
+    rows = np.array([0, 255, 256, B - 1], dtype=np.int32)
+    idx, summ, margin = oracle.sample_grouped(Hd.cpu(), Wd.cpu(), wl.groups, T=wl.temperature,
+                                              seed=0, step=0, mask=mask, rows=rows)
+    got = pair.cpu().numpy()[rows]
+    for i in np.flatnonzero(got != idx):
+        scale = TIE_REL * (1 + abs(summ[i, :, 0].max()))
+        assert margin[i, 0] <= scale or margin[i, 1] <= scale, (rows[i], got[i], idx[i])
+    del Wd, Hd
+    torch.cuda.empty_cache()

@@ -446,6 +446,27 @@ def test_one_workspace_serves_every_kind_of_call(dev, oracle):
         assert g.shape == (B,)
 
 
+def test_grouped_calls_of_different_layouts_share_a_workspace(dev, oracle):
+    """Where the partials and the published per-group maxima lie depends on
+    (B, G), so a call's published maxima may sit where an earlier call kept
+    partials.  Every call must leave the whole workspace zero, and every
+    group maximum must stay exact (a stale published maximum would hide the
+    true one from the exact-score filter)."""
+    d, V = 64, 6007
+    H, W, Hd, Wd = rand_inputs(300, d, V, seed=5)
+    ws = torch.zeros(binding.fs_workspace_bytes(300, V, 1000), dtype=torch.uint8, device=dev)
+    for B, G in [(300, 1000), (20, 8), (256, 64), (20, 3), (150, 1000), (20, 8)]:
+        summ = torch.empty(B, G, 3, dtype=torch.float32, device=dev)
+        binding.fs_sample_grouped(Hd[:B], Wd, G, temperature=0.8, seed=12, step=2,
+                                  out_summary=summ, workspace=ws)
+        torch.cuda.synchronize()
+        assert int(ws.count_nonzero()) == 0, (B, G)
+        _, o_summ, _ = oracle.sample_grouped(H[:B], W, G, T=0.8, seed=12, step=2)
+        got = summ[:, :, 0].cpu().numpy().astype(np.float64)
+        want = o_summ[:, :, 0]
+        assert np.allclose(got, want, rtol=1e-5, atol=1e-4), (B, G, np.abs(got - want).max())
+
+
 # ------------------------------------------------ online grouped sampling
 @pytest.mark.parametrize("B,V,G,masked", [(16, 6000, 3, False), (64, 8192, 8, True),
                                           (300, 4000, 5, True)])
