@@ -77,7 +77,10 @@ def committed_traffic(workload_key):
     if t.get("kernel_source_sha") != kernel_source_hash():
         return None
     entry = t.get("workloads", {}).get(workload_key)
-    return None if entry is None else entry.get("dram_bytes_per_launch")
+    if entry is None:
+        return None
+    # per call, like the achieved figure: one fused launch per 256 rows
+    return entry.get("dram_bytes_per_launch") * entry.get("fused_launches_per_call", 1)
 
 
 class ClockSampler:
@@ -298,9 +301,12 @@ def run_gpu(args, world, rank, local):
     W = synth.make_weight(wl.V, wl.d, wl.w_std, device=dev)
     H = synth.make_hidden(B, wl.d, device=dev)
     rs = synth.make_row_seeds(B, device=dev) if wl.per_row_seeds else None
+    mask = synth.make_mask(B, wl.V, wl.mask_allowed).to(dev) if wl.mask_allowed else None
     out = torch.empty(B, dtype=torch.int32, device=dev)
-    ws = torch.zeros(binding.fs_workspace_bytes(B, wl.V, 0), dtype=torch.uint8, device=dev)
-    tp = args.tp and world > 1
+    ws = torch.zeros(binding.fs_workspace_bytes(B, wl.V, wl.groups or 0), dtype=torch.uint8,
+                     device=dev)
+    grouped = bool(wl.groups)
+    tp = args.tp and world > 1 and not grouped
     if tp:
         from lm_head_exact_fmms_b200 import tp as tpmod
         lo, hi = tpmod.shard_bounds(wl.V, world)[rank]
@@ -316,10 +322,15 @@ def run_gpu(args, world, rank, local):
                                          stream=stream)
             tpmod.reduce_keys(keys)
             binding.fs_keys_to_tokens(keys, out_idx=out, stream=stream)
+    elif grouped:
+        def step(i):
+            binding.fs_sample_grouped(H, W, wl.groups, temperature=wl.temperature, seed=0,
+                                      row_seeds=rs, step=i, mask_bits=mask, out_idx=out,
+                                      workspace=ws, stream=stream)
     else:
         def step(i):
             binding.fs_sample_ex(H, W, temperature=wl.temperature, seed=0, row_seeds=rs, step=i,
-                                 out_idx=out, workspace=ws, stream=stream)
+                                 mask_bits=mask, out_idx=out, workspace=ws, stream=stream)
 
     sampler = ClockSampler(local)
     region_ms, per_call = time_calls(step, args.steps, args.warmup, stream, world, sampler)
@@ -327,8 +338,9 @@ def run_gpu(args, world, rank, local):
     kernel_us = sum(per_call) / len(per_call)
     kernel_us = max_over_ranks(kernel_us, world)
     us_per_call = region_ms * 1e3 / args.steps
-    nbytes, flops = algorithmic(B, wl.d, wl.V, False)
-    launches_per_call = (B + 255) // 256 + (1 if tp else 0)
+    nbytes, flops = algorithmic(B, wl.d, wl.V, mask is not None)
+    # fused kernel per 256 rows, plus the group merge (grouped) or the decode (tp)
+    launches_per_call = (B + 255) // 256 * (2 if grouped else 1) + (1 if tp else 0)
     if tp:
         # each rank streams its shard; the roofline below is per rank
         nbytes = nbytes * W.shape[0] // wl.V
@@ -341,8 +353,8 @@ def run_gpu(args, world, rank, local):
         binding.fs_sample_host(Hh, W, temperature=wl.temperature, seed=0, row_seeds=rs, step=i,
                                out_idx_host=Oh, stream=stream)
 
-    if tp:
-        # the host-buffer entry point is single-GPU: time H2D + the sharded step + D2H here
+    if tp or grouped:
+        # the host-buffer entry point is flat and single-GPU: time H2D + the step + D2H here
         def step_host(i):
             H.copy_(Hh, non_blocking=True)
             step(i)
@@ -357,9 +369,12 @@ def run_gpu(args, world, rank, local):
         "dtype": "bf16",
         "data": "synthetic: seeded H ~ N(0,1), W ~ N(0, %g^2) bf16 (random-init %s head)"
                 % (wl.w_std, wl.name),
-        "config": {"workload": "%s LM head, d=%d V=%d B=%d T=%g%s, fused fs_sample_ex"
+        "config": {"workload": "%s LM head, d=%d V=%d B=%d T=%g%s%s, fused %s"
                                % (wl.name, wl.d, wl.V, B, wl.temperature,
-                                  ", per-row seeds" if wl.per_row_seeds else ""),
+                                  ", per-row seeds" if wl.per_row_seeds else "",
+                                  (", G=%d, %d%% mask" % (wl.groups, round(100 * wl.mask_allowed)))
+                                  if grouped else "",
+                                  "fs_sample_grouped" if grouped else "fs_sample_ex"),
                    "batch_per_gpu": B, "global_batch": B * world, "d": wl.d, "V": wl.V,
                    "parallelism": ("tensor-parallel vocabulary x%d" % world) if tp
                    else ("replicas x%d" % world),
@@ -367,7 +382,7 @@ def run_gpu(args, world, rank, local):
         "samples_per_s": round(B * world / (us_per_call * 1e-6), 1),
         "hbm_gbs_per_gpu": round(nbytes / (us_per_call * 1e-6) / 1e9, 1),
         "kernel_us": round(kernel_us, 3),
-        "roofline": roofline(B, wl.d, W.shape[0], False, kernel_us, peaks, peak_kind,
+        "roofline": roofline(B, wl.d, W.shape[0], mask is not None, kernel_us, peaks, peak_kind,
                              None if tp else committed_traffic("%s/B%d" % (wl.name, B))),
         "e2e": {"value": round(e2e_ms * 1e3 / args.steps, 3), "unit": UNIT,
                 "h2d_bytes_per_step": B * wl.d * 2, "d2h_bytes_per_step": B * 4,
@@ -384,7 +399,7 @@ def run_gpu(args, world, rank, local):
         result["multi_sample"] = multi_point(torch, binding, synth, W, wl, dev, stream, B)
         result["cuda_graph"] = graph_point(torch, binding, synth, W, wl, dev, B)
         result["top_k"] = topk_point(torch, binding, synth, W, wl, dev, stream, B)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not grouped:
         result["cpu_baseline"] = cpu_baseline(H, W, wl, B, rs)
     return result
 
@@ -404,10 +419,21 @@ def sweep(torch, binding, synth, W, wl, dev, stream, peaks, peak_kind, steps=200
         kus = sum(per) / len(per)
         rf = roofline(B, wl.d, wl.V, False, kus, peaks, peak_kind,
                       committed_traffic("%s/B%d" % (wl.name, B)))
-        rows.append({"B": B, "us_per_call": round(region_ms * 1e3 / steps, 3),
-                     "kernel_us": round(kus, 3), "bound": rf["bound"],
-                     "achieved": round(rf["achieved"], 1), "unit": rf["unit"],
-                     "frac": round(rf["frac"], 4)})
+        row = {"B": B, "us_per_call": round(region_ms * 1e3 / steps, 3),
+               "kernel_us": round(kus, 3), "bound": rf["bound"],
+               "achieved": round(rf["achieved"], 1), "unit": rf["unit"],
+               "frac": round(rf["frac"], 4),
+               # the library's automatic choice: CTA pairs above 64 rows per launch
+               "cta_pairs": B > 64}
+        if B > 64:
+            # the same call on the single-CTA kernel, for comparison
+            binding.fs_set_cta_pairs(0)
+            try:
+                _, per1 = time_calls(step, steps, warmup, stream)
+            finally:
+                binding.fs_set_cta_pairs(-1)
+            row["single_cta_kernel_us"] = round(sum(per1) / len(per1), 3)
+        rows.append(row)
     return rows
 
 

@@ -42,24 +42,38 @@ __global__ void __launch_bounds__(128) group_merge_kernel(const MergeParams m) {
     const int c_last = cta_of(hi - 1, sch);
     unsigned long long kmax = 0ull;
     float M = -INFINITY, S = 0.f;
+    // The group's partials: slots c + g for its CTAs c (2 (c + g) and
+    // 2 (c + g) + 1 for CTA pairs c).  Loads go out eight at a time, and the
+    // slots are zeroed only after all are read, so the loads overlap.
     const int per_unit = m.pair ? 2 : 1;
-    for (int u = c_first * per_unit; u < (c_last + 1) * per_unit; ++u) {
-      const size_t slot = m.pair ? 2 * static_cast<size_t>(u / 2 + g) + (u & 1)
-                                 : static_cast<size_t>(u + g);
-      const GroupPartial gp = m.partials[slot * m.B + b];
-      m.partials[slot * m.B + b] = GroupPartial{0ull, 0.f, 0.f};  // leave the workspace zeroed
-      kmax = gp.key > kmax ? gp.key : kmax;
-      if (gp.m != -INFINITY) {
-        if (M == -INFINITY) {
-          M = gp.m;
-          S = gp.sum;
-        } else {
-          const float mx = fmaxf(M, gp.m);
-          S = S * expf(M - mx) + gp.sum * expf(gp.m - mx);
-          M = mx;
+    const int nslots = (c_last - c_first + 1) * per_unit;
+    auto slot_of = [&](int i) -> size_t {
+      const int u = c_first * per_unit + i;
+      return m.pair ? 2 * static_cast<size_t>(u / 2 + g) + (u & 1) : static_cast<size_t>(u + g);
+    };
+    for (int i0 = 0; i0 < nslots; i0 += 8) {
+      GroupPartial gp[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (i0 + j < nslots) gp[j] = m.partials[slot_of(i0 + j) * m.B + b];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (i0 + j >= nslots) break;
+        kmax = gp[j].key > kmax ? gp[j].key : kmax;
+        if (gp[j].m != -INFINITY) {
+          if (M == -INFINITY) {
+            M = gp[j].m;
+            S = gp[j].sum;
+          } else {
+            const float mx = fmaxf(M, gp[j].m);
+            S = S * expf(M - mx) + gp[j].sum * expf(gp[j].m - mx);
+            M = mx;
+          }
         }
       }
     }
+    for (int i = 0; i < nslots; ++i)  // leave the workspace zeroed
+      m.partials[slot_of(i) * m.B + b] = GroupPartial{0ull, 0.f, 0.f};
     if (m.gkeys != nullptr) m.gkeys[static_cast<size_t>(g) * m.B + b] = 0ull;  // left zeroed
     const float lse = (M == -INFINITY) ? -INFINITY : M + logf(S);
     if (summary != nullptr) {
