@@ -45,18 +45,31 @@ namespace fmms {
 // barriers and (grouped mode) the combine area.
 constexpr int kSmemBudget = 232448 - 1024 - 256;
 
-// K sub-blocks of 64 elements per pipeline stage.  Two sub-blocks halve the
-// per-stage handshake (full wait, tcgen05 fence, commit, empty wait) per byte
-// of W and let W be fetched 256 bytes of a row at a time, but they halve the
-// number of stages.  Measured on the Qwen3-8B-shaped head: a ten-stage ring of
-// single sub-blocks is best while it fits (batch tiles up to 32 rows per
-// CTA); where H is large enough to shorten the ring below ten stages, two
-// sub-blocks win as long as four stages remain (64 rows; 128 rows per pair).
+// K sub-blocks of 64 elements per pipeline stage, and the number of stages.
+// Measured on the Qwen3-8B, Qwen3-1.7B and d=8192 heads: what sets the
+// streaming rate is the W bytes in flight per SM (stages x sub-blocks x
+// 16 KB), with at least three stages so that loads, MMAs and the stage
+// hand-back overlap, and at equal bytes the longer per-row bursts of more
+// sub-blocks per stage win (fewer handshakes per byte, 128 B more of each W
+// row per sub-block).  So: among 1..4 sub-blocks with at least three stages
+// (at most ten), the most W bytes in flight, ties to more sub-blocks.
+// E.g. single CTAs: 4 x 3 stages at 16 batch rows, 2 x 5 at 32, 3 x 3 at 64;
+// CTA pairs: 3 x 3 at 128 rows (64 H rows per CTA), 1 x 7 at 256.
+constexpr int kMaxStages = 10;
+constexpr int stages_for(int ksub, int h_rows, int comb_bytes) {
+  const int fit = (kSmemBudget - comb_bytes) / (ksub * (kTileM + h_rows) * kBlockK * 2);
+  return fit < kMaxStages ? fit : kMaxStages;
+}
 constexpr int ksub_for(int h_rows, int comb_bytes) {
-  const int stage1 = (kTileM + h_rows) * kBlockK * 2;
-  const int fit1 = (kSmemBudget - comb_bytes) / stage1;
-  const int fit2 = (kSmemBudget - comb_bytes) / (2 * stage1);
-  return (fit1 < 10 && fit2 >= 4) ? 2 : 1;
+  int best = 1, best_bytes = 0;
+  for (int k = 1; k <= 4; ++k) {
+    const int st = stages_for(k, h_rows, comb_bytes);
+    if (st >= 3 && st * k >= best_bytes) {
+      best = k;
+      best_bytes = st * k;
+    }
+  }
+  return best;
 }
 
 template <int BN, int MODE, bool PAIR = false>
@@ -70,8 +83,7 @@ struct KCfg {
   static constexpr int kStageW = kSub * kSubW;
   static constexpr int kStageH = kSub * kSubH;
   static constexpr int kStageBytes = kStageW + kStageH;
-  static constexpr int kStagesFit = (kSmemBudget - kCombBytes) / kStageBytes;
-  static constexpr int kStages = kStagesFit < 10 ? kStagesFit : 10;
+  static constexpr int kStages = stages_for(kSub, kHRows, kCombBytes);
   static constexpr int kCW = 16;                        // columns per epilogue chunk
   static constexpr int kChunks = BN / kCW;
   static constexpr int kWarpsPerQuarter = kNumEpiWarps / 4;

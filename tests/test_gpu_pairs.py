@@ -227,3 +227,42 @@ def test_pairs_grouped_full_size_head(dev, oracle):
         assert margin[i, 0] <= scale or margin[i, 1] <= scale, (rows[i], got[i], idx[i])
     del Wd, Hd
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("B,grouped", [(48, False), (200, False), (130, True)])
+def test_cuda_graph_replay(dev, B, grouped):
+    """Calls captured into a CUDA graph (single-CTA and CTA-pair launches,
+    the latter with a cluster launch attribute) replay to the eager tokens.
+    The first eager call sizes the library workspace, so capture allocates
+    nothing."""
+    d, V, G = 128, 9000, 4
+    _, _, Hd, Wd = rand_inputs(B, d, V, seed=B + 7)
+    rs = synth.make_row_seeds(B).to(dev)
+    outs = [torch.empty(B, dtype=torch.int32, device=dev) for _ in range(3)]
+
+    def call(i):
+        if grouped:
+            binding.fs_sample_grouped(Hd, Wd, G, temperature=0.9, seed=3, row_seeds=rs, step=i,
+                                      out_idx=outs[i], stream=torch.cuda.current_stream())
+        else:
+            binding.fs_sample_ex(Hd, Wd, temperature=0.9, seed=3, row_seeds=rs, step=i,
+                                 out_idx=outs[i], stream=torch.cuda.current_stream())
+
+    for i in range(3):
+        call(i)
+    torch.cuda.synchronize()
+    eager = [o.clone() for o in outs]
+    for o in outs:
+        o.fill_(-7)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for i in range(3):
+            call(i)
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    for i in range(3):
+        assert torch.equal(outs[i], eager[i]), i
+    del g
