@@ -266,3 +266,22 @@ def test_cuda_graph_replay(dev, B, grouped):
     for i in range(3):
         assert torch.equal(outs[i], eager[i]), i
     del g
+
+
+@pytest.mark.parametrize("B", [1, 16, 40, 64, 100, 200])
+@pytest.mark.parametrize("d", [320, 384, 448, 576])
+def test_partial_last_stage(dev, oracle, B, d):
+    """K lengths (d / 64 = 5, 6, 7, 9 sub-blocks) that leave the last stage
+    partly filled for every stage shape the kernel picks: four sub-blocks per
+    stage at 16 rows, two at 32, three at 64 and on pairs at 128, one on
+    pairs at 256; flat and grouped."""
+    V = 3001
+    H, W, Hd, Wd = rand_inputs(B, d, V, seed=B * 7 + d)
+    got = binding.fs_sample(Hd, Wd, temperature=0.9, seed=4, step=1).cpu().numpy()
+    assert_parity(got, *oracle.sample(H, W, T=0.9, seed=4, step=1), "B=%d d=%d" % (B, d))
+    G = 5
+    tok = binding.fs_sample_grouped(Hd, Wd, G, temperature=0.9, seed=4, step=1).cpu().numpy()
+    idx, summ, margin = oracle.sample_grouped(H, W, G, T=0.9, seed=4, step=1)
+    for b in np.flatnonzero(tok != idx):
+        scale = TIE_REL * (1 + abs(summ[b, :, 0].max()))
+        assert margin[b, 0] <= scale or margin[b, 1] <= scale, (b, tok[b], idx[b])
