@@ -27,7 +27,7 @@ METRIC = "FMMS µs/call & HBM GB/s (% roofline), d=4096 V=151936 bf16, B=1–256
 UNIT = "us/call"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
-KERNEL_SOURCES = ["lm_head_exact_fmms_b200/csrc/fmms_kernel.cu",
+KERNEL_SOURCES = ["lm_head_exact_fmms_b200/csrc/fmms_kernel.cuh",
                   "lm_head_exact_fmms_b200/csrc/noise.cuh",
                   "lm_head_exact_fmms_b200/csrc/sm100.cuh",
                   "lm_head_exact_fmms_b200/csrc/fmms_common.cuh"]

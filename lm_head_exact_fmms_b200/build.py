@@ -2,8 +2,9 @@
 
 Usage: python -m lm_head_exact_fmms_b200.build [--force]
 
-The library is built in-tree next to this file.  No fast-math: the Gumbel
-transform relies on the accurate logf/log1pf.
+The library is built in-tree next to this file.  The fused kernel's modes
+are instantiated in separate translation units (fmms_inst_*.cu), compiled in
+parallel.
 """
 import os
 import subprocess
@@ -15,8 +16,10 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libfmms.so")
 OBJDIR = os.path.join(HERE, "_build")
-SOURCES = ["fmms_kernel.cu", "aux_kernels.cu", "api.cu"]
-HEADERS = ["fmms_common.cuh", "sm100.cuh", "noise.cuh", "launch.h"]
+SOURCES = ["fmms_inst_flat.cu", "fmms_inst_flat_pair.cu", "fmms_inst_grouped.cu",
+           "fmms_inst_grouped_pair.cu", "fmms_inst_logits.cu", "fmms_kernel.cu", "aux_kernels.cu",
+           "api.cu"]
+HEADERS = ["fmms_kernel.cuh", "fmms_common.cuh", "sm100.cuh", "noise.cuh", "launch.h"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -29,7 +29,11 @@ struct DeviceState {
   size_t h_stage_bytes = 0;
   void *o_stage = nullptr;  // fs_sample_host: device tokens
   size_t o_stage_bytes = 0;
-  int pair_units[2][5] = {{-1, -1, -1, -1, -1}, {-1, -1, -1, -1, -1}};  // [flat, grouped][tile]
+  int pair_units[2][fmms::kMaxBN / 16];  // resident CTA pairs [flat, grouped][tile / 16 - 1]; -1: unknown
+  DeviceState() {
+    for (auto &row : pair_units)
+      for (int &u : row) u = -1;
+  }
 };
 
 constexpr int kMaxDevices = 64;
@@ -193,9 +197,7 @@ bool g_test_no_loads = false;
 // fs_set_cta_pairs: -1 automatic, 0 never, 1 whenever the call allows it.
 int g_pair_policy = -1;
 
-int bn_index(int BN) {
-  return BN <= 16 ? 0 : BN <= 32 ? 1 : BN <= 64 ? 2 : BN <= 128 ? 3 : 4;
-}
+int bn_index(int BN) { return BN / 16 - 1; }
 
 // CTA pairs of the BN pair kernel of `mode` that fit on the device at once
 // (0: none).

@@ -19,6 +19,12 @@ constexpr int kTileM = 128;   // vocabulary rows per tile (tcgen05 M)
 constexpr int kBlockK = 64;   // K elements per pipeline stage: one 128-byte swizzle row
 constexpr int kGranule = 8;   // vocabulary granule of the per-CTA split: one 8-row swizzle atom
 constexpr int kMaxBN = 256;   // batch rows per launch (tcgen05 N limit)
+
+// The batch tiles the kernels are built for: every multiple of 16 rows up to
+// 256 (tcgen05 N with M = 128 or, on CTA pairs, M = 256; 8-row halves).
+#define FMMS_FOR_EACH_BN(X) \
+  X(16) X(32) X(48) X(64) X(80) X(96) X(112) X(128) X(144) X(160) X(176) X(192) X(208) X(224) \
+  X(240) X(256)
 constexpr int kNumEpiWarps = 16;  // four per TMEM lane quarter
 constexpr int kThreads = 32 * (2 + kNumEpiWarps);  // TMA warp + MMA warp + epilogue
 constexpr int kEpiThreads = 32 * kNumEpiWarps;

@@ -1,0 +1,18 @@
+// fmms_inst_flat.cu -- the fused kernel in flat mode on single CTAs, built for every batch tile.
+#include "fmms_kernel.cuh"
+#include "launch.h"
+
+namespace fmms {
+
+cudaError_t launch_flat(int BN, const CUtensorMap &tw, const CUtensorMap &tw8,
+                        const CUtensorMap &th, const FmmsParams &p, cudaStream_t stream) {
+  switch (BN) {
+#define FMMS_CASE(n) \
+  case n: return launch_t<n, kModeFlat>(tw, tw8, th, p, stream);
+    FMMS_FOR_EACH_BN(FMMS_CASE)
+#undef FMMS_CASE
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace fmms

@@ -1,941 +1,17 @@
-// fmms_kernel.cu -- the fused matmul-sample (FMMS) kernel for sm_100a.
-//
-// What it computes (FlashSampling, arXiv:2603.15854, abstract): logits of a
-// vocabulary tile are formed on chip, scaled by 1/T, masked, perturbed with
-// Gumbel noise, and only one (score, token) maximiser per row and tile
-// survives; a reduction over tiles gives one token per row.  The B x V
-// logits never reach HBM (except in the logits mode kept for measurement).
-//
-// How (B200 design; the Triton kernel the pages describe is prior art only):
-//  * one persistent CTA per SM; each CTA owns a contiguous, 8-row-granular
-//    slice of the vocabulary (split-V), so small batches still keep all 148
-//    SMs streaming W and no W row is read twice;
-//  * swap-AB MMA: A = 128 vocabulary rows of W (M = 128), B = the batch of
-//    hidden states (N = 16..256), D = a 128-lane x N-column fp32 accumulator
-//    in tensor memory; the tile's vocabulary rows land on TMEM lanes, i.e. on
-//    epilogue threads;
-//  * warp roles: warp 0 issues TMA loads of W (evict-first) and H
-//    (evict-last) into a multi-stage 128-byte-swizzled shared-memory ring;
-//    warp 1 allocates TMEM and issues tcgen05.mma; warps 2-9 drain the
-//    double-buffered accumulator while the next tile is being multiplied;
-//  * epilogue per element: x = acc / T, Philox4x32-10 noise word for
-//    (seed, step, row, token) (one Philox call serves four consecutive
-//    tokens; four lanes exchange words with a 4x4 shuffle transpose), the
-//    Gumbel transform, s = x + g, then a 32-lane "transpose-reduce" leaves
-//    lane j with the packed max of column j;
-//  * flat mode: per CTA, one atomicMax of a packed (score, token) key per row
-//    into the workspace; the last CTA to finish (atomic ticket, no waiting)
-//    decodes the tokens and re-zeroes the workspace;
-//  * grouped mode: per (segment, row) partial (max key, lse pieces) for the
-//    Group-Gumbel-Max merge kernel;
-//  * logits mode: raw fp32 logits to HBM for the unfused measurement path.
-#include <cuda.h>
-#include <cuda_runtime.h>
-#include <math.h>
-#include <stdint.h>
-
-#include "fmms_common.cuh"
+// fmms_kernel.cu -- dispatch of the fused matmul-sample kernel by mode, batch
+// tile and CTA arrangement.  The kernel itself is in fmms_kernel.cuh; each
+// fmms_inst_*.cu builds one mode for every batch tile, so that the
+// instantiations compile in parallel.
 #include "launch.h"
-#include "noise.cuh"
-#include "sm100.cuh"
 
 namespace fmms {
-
-// Shared memory a kernel may use beyond the stages: alignment slack,
-// barriers and (grouped mode) the combine area.
-constexpr int kSmemBudget = 232448 - 1024 - 256;
-
-// K sub-blocks of 64 elements per pipeline stage, and the number of stages.
-// Measured on the Qwen3-8B, Qwen3-1.7B and d=8192 heads: what sets the
-// streaming rate is the W bytes in flight per SM (stages x sub-blocks x
-// 16 KB), with at least three stages so that loads, MMAs and the stage
-// hand-back overlap, and at equal bytes the longer per-row bursts of more
-// sub-blocks per stage win (fewer handshakes per byte, 128 B more of each W
-// row per sub-block).  So: among 1..4 sub-blocks with at least three stages
-// (at most ten), the most W bytes in flight, ties to more sub-blocks.
-// E.g. single CTAs: 4 x 3 stages at 16 batch rows, 2 x 5 at 32, 3 x 3 at 64;
-// CTA pairs: 3 x 3 at 128 rows (64 H rows per CTA), 1 x 7 at 256.
-constexpr int kMaxStages = 10;
-constexpr int stages_for(int ksub, int h_rows, int comb_bytes) {
-  const int fit = (kSmemBudget - comb_bytes) / (ksub * (kTileM + h_rows) * kBlockK * 2);
-  return fit < kMaxStages ? fit : kMaxStages;
-}
-constexpr int ksub_for(int h_rows, int comb_bytes) {
-  int best = 1, best_bytes = 0;
-  for (int k = 1; k <= 4; ++k) {
-    const int st = stages_for(k, h_rows, comb_bytes);
-    if (st >= 3 && st * k >= best_bytes) {
-      best = k;
-      best_bytes = st * k;
-    }
-  }
-  return best;
-}
-
-template <int BN, int MODE, bool PAIR = false>
-struct KCfg {
-  static_assert(!PAIR || MODE != kModeLogits, "the logits mode runs on single CTAs");
-  static constexpr int kHRows = PAIR ? BN / 2 : BN;     // H rows this CTA stages
-  static constexpr int kCombBytes = MODE == kModeGrouped ? 4 * BN * 16 : 0;  // grouped only
-  static constexpr int kSub = ksub_for(kHRows, kCombBytes);  // 64-wide K blocks per stage
-  static constexpr int kSubW = kTileM * kBlockK * 2;    // 16 KB of W per sub-block
-  static constexpr int kSubH = kHRows * kBlockK * 2;    // this CTA's H rows per sub-block
-  static constexpr int kStageW = kSub * kSubW;
-  static constexpr int kStageH = kSub * kSubH;
-  static constexpr int kStageBytes = kStageW + kStageH;
-  static constexpr int kStages = stages_for(kSub, kHRows, kCombBytes);
-  static constexpr int kCW = 16;                        // columns per epilogue chunk
-  static constexpr int kChunks = BN / kCW;
-  static constexpr int kWarpsPerQuarter = kNumEpiWarps / 4;
-  static constexpr int kChunksPerWarp = kChunks >= kWarpsPerQuarter ? kChunks / kWarpsPerQuarter : 1;
-  static constexpr int kAccBufs = BN <= 128 ? 4 : 2;     // accumulators in flight
-  static constexpr int kTmemCols = kAccBufs * BN < 32 ? 32 : kAccBufs * BN;
-  static constexpr uint32_t kIdesc = sm100::idesc_bf16_f32(PAIR ? 2 * kTileM : kTileM, BN);
-  static constexpr int kEpiArrivals = PAIR ? 2 * kNumEpiWarps : kNumEpiWarps;
-  static constexpr int kBarBytes = 256;
-  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBarBytes + kCombBytes;
-  static_assert(kSubH % 1024 == 0, "H sub-block must keep 1024-byte atom alignment");
-  static_assert((2 * kStages + 2 * kAccBufs + 1) * 8 + 16 <= kBarBytes, "barrier area too small");
-  static_assert(kTmemCols <= 512, "tensor memory holds 512 columns");
-  static_assert(kSmemBytes <= 232448, "shared memory budget");
-};
-
-// ---------------------------------------------------------------------------
-// Epilogue helpers
-// ---------------------------------------------------------------------------
-
-// Four lanes with the same token >> 2 each hold the four Philox words of one
-// column (lane i: column c + i, words for tokens 4q..4q+3).  Afterwards lane
-// i holds, in w[m], the word of token 4q + i for column c + m.
-__device__ __forceinline__ void quad_transpose(uint32_t (&w)[4], int lane) {
-  const bool b0 = (lane & 1) != 0;
-  const bool b1 = (lane & 2) != 0;
-  const uint32_t s01 = b0 ? w[0] : w[1];
-  const uint32_t s23 = b0 ? w[2] : w[3];
-  const uint32_t r01 = __shfl_xor_sync(0xffffffffu, s01, 1);
-  const uint32_t r23 = __shfl_xor_sync(0xffffffffu, s23, 1);
-  if (b0) {
-    w[0] = r01;
-    w[2] = r23;
-  } else {
-    w[1] = r01;
-    w[3] = r23;
-  }
-  const uint32_t s02 = b1 ? w[0] : w[2];
-  const uint32_t s13 = b1 ? w[1] : w[3];
-  const uint32_t r02 = __shfl_xor_sync(0xffffffffu, s02, 2);
-  const uint32_t r13 = __shfl_xor_sync(0xffffffffu, s13, 2);
-  if (b1) {
-    w[0] = r02;
-    w[1] = r13;
-  } else {
-    w[2] = r02;
-    w[3] = r13;
-  }
-}
-
-// Lane that ends up holding column j of a CW-column transpose-reduce.
-template <int CW>
-__device__ __forceinline__ int column_of_lane(int lane) {
-  return CW == 32 ? lane : (lane >> 1);
-}
-template <int CW>
-__device__ __forceinline__ int lane_of_column(int j) {
-  return CW == 32 ? j : 2 * j;
-}
-
-// Transpose-reduce: every lane holds CW values (one per column); afterwards
-// lane l holds the reduction over all 32 lanes of column column_of_lane(l).
-// Each halving round keeps one half of the columns and trades the other half
-// with the partner lane, so CW=32 costs 31 exchanges instead of 32 x 5.
-struct OpMaxU64 {
-  __device__ __forceinline__ static uint64_t apply(uint64_t a, uint64_t b) { return a > b ? a : b; }
-};
-struct OpMaxF {
-  __device__ __forceinline__ static float apply(float a, float b) { return fmaxf(a, b); }
-};
-struct OpAddF {
-  __device__ __forceinline__ static float apply(float a, float b) { return a + b; }
-};
-
-template <int CW, class Op, class T>
-__device__ __forceinline__ T transpose_reduce(T (&k)[CW], int lane) {
-#pragma unroll
-  for (int half = CW / 2, off = 16; half >= 1; half /= 2, off /= 2) {
-    const bool upper = (lane & off) != 0;
-#pragma unroll
-    for (int i = 0; i < half; ++i) {
-      const T send = upper ? k[i] : k[i + half];
-      const T keep = upper ? k[i + half] : k[i];
-      const T recv = __shfl_xor_sync(0xffffffffu, send, off);
-      k[i] = Op::apply(keep, recv);
-    }
-  }
-  if (CW == 16) k[0] = Op::apply(k[0], __shfl_xor_sync(0xffffffffu, k[0], 1));
-  return k[0];
-}
-
-// Folds (m2, s2) into the running log-sum-exp pieces (m, s): sum exp(x - m) = s.
-__device__ __forceinline__ void lse_merge(float &m, float &s, float m2, float s2) {
-  if (m2 == -INFINITY) return;
-  if (m == -INFINITY) {
-    m = m2;
-    s = s2;
-    return;
-  }
-  const float mx = fmaxf(m, m2);
-  s = s * __expf(m - mx) + s2 * __expf(m2 - mx);
-  m = mx;
-}
-
-// Reads a published key from global memory, bypassing L1 (other CTAs update it).
-__device__ __forceinline__ uint64_t ld_key(const unsigned long long *ptr) {
-  return __ldcg(ptr);
-}
-
-// Noise words of one chunk: afterwards words[j] is the word of (row col0 + j,
-// token v) for this lane's tile row v.  One Philox call per lane serves four
-// consecutive tokens of one row; the quad transpose hands each lane its word.
-template <int CW>
-__device__ __forceinline__ void chunk_noise(const FmmsParams &p, int v, int col0, int lane,
-                                            uint32_t tag, uint32_t (&words)[CW]) {
-#pragma unroll
-  for (int q4 = 0; q4 < CW / 4; ++q4) {
-    const int colp = col0 + 4 * q4 + (lane & 3);  // column of this lane's Philox call
-    const uint32_t bg = static_cast<uint32_t>(p.b_off + colp);
-    uint64_t k64 = p.seed;
-    if (p.row_seeds != nullptr && colp < p.B) k64 = __ldg(p.row_seeds + bg);
-    const Philox4 ph = philox4x32_10(static_cast<uint32_t>(v) >> 2, bg, p.step, tag,
-                                     static_cast<uint32_t>(k64), static_cast<uint32_t>(k64 >> 32));
-    uint32_t w[4] = {ph.w0, ph.w1, ph.w2, ph.w3};
-    quad_transpose(w, lane);
-#pragma unroll
-    for (int m = 0; m < 4; ++m) words[4 * q4 + m] = w[m];
-  }
-}
-
-// Transpose of the 32 x 32 bit matrix whose row r is lane r's x: afterwards
-// lane c holds the bits c of every lane's x, lane r's bit at position r.
-// Five rounds of swapping the off-diagonal blocks of size 16, 8, 4, 2, 1.
-__device__ __forceinline__ uint32_t bit_transpose32(uint32_t x, int lane) {
-  const uint32_t kMasks[5] = {0x0000FFFFu, 0x00FF00FFu, 0x0F0F0F0Fu, 0x33333333u, 0x55555555u};
-#pragma unroll
-  for (int i = 0, sft = 16; i < 5; ++i, sft >>= 1) {
-    const uint32_t m = kMasks[i];
-    const uint32_t y = __shfl_xor_sync(0xffffffffu, x, sft);
-    x = (lane & sft) ? ((x & ~m) | ((y >> sft) & m)) : ((x & m) | ((y & m) << sft));
-  }
-  return x;
-}
-
-// Bit j set when (row col0 + j, token v) is in range and, with a mask,
-// allowed for that row.  Warp-collective: the warp's lanes hold 32
-// consecutive tokens.  Lane j < CW gathers row col0 + j's 32 mask bits of
-// those tokens (two words at most); a bit-matrix transpose then hands every
-// lane its own token's bit of each row.
-template <int CW>
-__device__ __forceinline__ uint32_t chunk_allowed(const FmmsParams &p, int v, bool v_ok,
-                                                  int col0, int lane) {
-  const int n = p.B - col0;
-  const uint32_t in_range = n >= CW ? ((1u << CW) - 1u) : ((1u << n) - 1u);
-  if (p.mask == nullptr) return v_ok ? in_range : 0u;
-  const int v0 = v - lane;  // token of lane 0 (a multiple of 8)
-  uint32_t rowbits = 0u;
-  if (lane < CW && lane < n) {
-    const uint32_t *row = p.mask + static_cast<size_t>(p.b_off + col0 + lane) * p.mask_words;
-    const int w0 = v0 >> 5;
-    const int sh = v0 & 31;
-    const uint32_t lo = w0 < p.mask_words ? __ldg(row + w0) : 0u;
-    const uint32_t hi = (sh != 0 && w0 + 1 < p.mask_words) ? __ldg(row + w0 + 1) : 0u;
-    rowbits = sh == 0 ? lo : ((lo >> sh) | (hi << (32 - sh)));
-  }
-  const uint32_t bits = bit_transpose32(rowbits, lane);
-  return v_ok ? (bits & in_range) : 0u;
-}
-
-// Bit j set when (row col0 + j, token v) is in range, mask not consulted.
-template <int CW>
-__device__ __forceinline__ uint32_t chunk_in_range(const FmmsParams &p, bool v_ok, int col0) {
-  if (!v_ok) return 0u;
-  const int n = p.B - col0;
-  return n >= CW ? ((1u << CW) - 1u) : ((1u << n) - 1u);
-}
-
-// Exact scores s = x + g of the allowed elements as packed keys,
-// transpose-reduced into the lane's running best of its column.
-template <int CW>
-__device__ __forceinline__ void chunk_keys(const uint32_t (&acc)[CW], const uint32_t (&words)[CW],
-                                           const FmmsParams &p, int v, uint32_t allowed, int lane,
-                                           uint64_t &best) {
-  uint64_t key[CW];
-  const uint64_t low = 0xFFFFFFFFu - static_cast<uint32_t>(v);  // token part of the key
-#pragma unroll
-  for (int j = 0; j < CW; ++j) {
-    const float s = fmaf(__uint_as_float(acc[j]), p.inv_temp, gumbel_from_u32(words[j]));
-    const uint32_t hi = ((allowed >> j) & 1u) ? order_bits(__float_as_uint(s)) : 0u;
-    key[j] = (static_cast<uint64_t>(hi) << 32) | low;
-  }
-  const uint64_t cmax = transpose_reduce<CW, OpMaxU64>(key, lane);
-  best = cmax > best ? cmax : best;
-}
-
-// Log-sum-exp pieces of the allowed x = acc / T of one chunk, folded into the
-// lane's running (m, s) of its column.
-template <int CW>
-__device__ __forceinline__ void chunk_lse(const uint32_t (&acc)[CW], const FmmsParams &p,
-                                          uint32_t allowed, int lane, float &m_run, float &s_run) {
-  float xs[CW], t[CW];
-#pragma unroll
-  for (int j = 0; j < CW; ++j) {
-    xs[j] = ((allowed >> j) & 1u) ? __uint_as_float(acc[j]) * p.inv_temp : -INFINITY;
-    t[j] = xs[j];
-  }
-  const float colmax = transpose_reduce<CW, OpMaxF>(t, lane);
-  float e[CW];
-#pragma unroll
-  for (int j = 0; j < CW; ++j) {
-    const float cm = __shfl_sync(0xffffffffu, colmax, lane_of_column<CW>(j));
-    e[j] = (xs[j] == -INFINITY) ? 0.f : __expf(xs[j] - cm);
-  }
-  const float colsum = transpose_reduce<CW, OpAddF>(e, lane);
-  lse_merge(m_run, s_run, colmax, colsum);
-}
-
-// The filter: may any element of the chunk (bit set in `cand`) reach its
-// column's threshold?  The threshold of a column is the score of an element
-// already computed exactly (the lane's own best, or the best any CTA has
-// published for this row), so an element whose upper bound
-// x + gumbel_upper_bound(r) is below it can be neither the maximum nor tied
-// with it: skipping its exact score leaves the sampled token unchanged.
-template <int CW>
-__device__ __forceinline__ bool chunk_any_candidate(const uint32_t (&acc)[CW],
-                                                    const uint32_t (&words)[CW],
-                                                    const FmmsParams &p, uint32_t cand,
-                                                    uint64_t best, uint64_t published, int lane) {
-  const uint64_t k = published > best ? published : best;
-  const float t_col = key_valid(k) ? __uint_as_float(key_score_bits(k)) : -INFINITY;
-  bool any = false;
-#pragma unroll
-  for (int j = 0; j < CW; ++j) {
-    const float thr = __shfl_sync(0xffffffffu, t_col, lane_of_column<CW>(j));
-    const float ub = fmaf(__uint_as_float(acc[j]), p.inv_temp, gumbel_upper_bound(words[j]));
-    any = any || (((cand >> j) & 1u) && ub >= thr);
-  }
-  return __any_sync(0xffffffffu, any);
-}
-
-// ---------------------------------------------------------------------------
-// Roles
-// ---------------------------------------------------------------------------
-
-// Bytes of W a CTA loads per 64-wide K sub-block for `rows` rows from the
-// tile start (whole tile: one 128-row box; otherwise 8-row boxes).
-__device__ __forceinline__ uint32_t w_sub_bytes(int rows) {
-  if (rows <= 0) return 0u;
-  if (rows >= kTileM) return static_cast<uint32_t>(kTileM * kBlockK * 2);
-  return static_cast<uint32_t>((rows + kGranule - 1) / kGranule) * 1024u;
-}
-
-// TMA producer (one thread).  In pair mode both CTAs load their own half of
-// every stage (128 W rows, BN/2 H rows) and count the bytes on the even
-// CTA's full barrier; the even CTA also hands each freed stage on to the odd
-// CTA, whose MMA reads happen in the even CTA's tcgen05 pipeline.
-template <int BN, int MODE, bool PAIR>
-__device__ __forceinline__ void role_producer(const CUtensorMap *tw, const CUtensorMap *tw8,
-                                              const CUtensorMap *th, const FmmsParams &p,
-                                              const Schedule &sch, uint8_t *stages,
-                                              uint64_t *full, uint64_t *empty,
-                                              volatile int *abort_flag, int unit, int rank) {
-  using C = KCfg<BN, MODE, PAIR>;
-  const uint64_t pol_w = sm100::l2_policy_evict_first();
-  const uint64_t pol_h = sm100::l2_policy_evict_last();
-  TileIter it(sch, unit);
-  Tile tile;
-  int stage = 0;
-  uint32_t phase = 0;
-  long long issued = 0;
-  bool ok = p.test_no_loads == 0;
-  while (ok && it.next(tile)) {
-    const Tile mine = PAIR ? pair_half(tile, rank) : tile;
-    const int rows = mine.hi - mine.start;
-    const bool whole = rows >= kTileM;
-    const int nbox8 = rows > 0 ? (rows + kGranule - 1) / kGranule : 0;
-    uint32_t sub_bytes = w_sub_bytes(rows) + C::kSubH;  // counted on this CTA's barrier
-    if (PAIR) {
-      const Tile other = pair_half(tile, 1 - rank);
-      sub_bytes += w_sub_bytes(other.hi - other.start) + C::kSubH;
-    }
-    const int nks = (p.nk + C::kSub - 1) / C::kSub;
-    for (int ks = 0; ks < nks; ++ks) {
-      const int sub0 = ks * C::kSub;
-      const int nsub = imin(C::kSub, p.nk - sub0);
-      const uint32_t bytes = sub_bytes * static_cast<uint32_t>(nsub);
-      if (!sm100::wait_bounded<PAIR>(&empty[stage], phase ^ 1u, abort_flag, p.err)) {
-        ok = false;
-        break;
-      }
-      if (PAIR && rank == 0 && issued >= C::kStages)
-        sm100::mbar_arrive_cluster(sm100::cluster_addr(&empty[stage], 1));
-      uint8_t *sw0 = stages + stage * C::kStageBytes;
-      uint8_t *sh0 = sw0 + C::kStageW;
-      if (!PAIR || rank == 0) sm100::mbar_arrive_expect_tx(&full[stage], bytes);
-      const uint32_t bar = PAIR ? sm100::cluster_addr(&full[stage], 0) : 0u;
-#pragma unroll
-      for (int j = 0; j < C::kSub; ++j) {
-        if (j >= nsub) break;
-        uint8_t *sw = sw0 + j * C::kSubW;
-        uint8_t *sh = sh0 + j * C::kSubH;
-        const int x = (sub0 + j) * kBlockK;
-        if constexpr (PAIR) {
-          if (whole) {
-            sm100::tma_load_2d_pair(sw, tw, bar, x, mine.start, pol_w);
-          } else {
-            for (int i = 0; i < nbox8; ++i)
-              sm100::tma_load_2d_pair(sw + i * 1024, tw8, bar, x, mine.start + kGranule * i,
-                                      pol_w);
-          }
-          sm100::tma_load_2d_pair(sh, th, bar, x, p.b_off + rank * C::kHRows, pol_h);
-        } else {
-          if (whole) {
-            sm100::tma_load_2d(sw, tw, &full[stage], x, mine.start, pol_w);
-          } else {
-            for (int i = 0; i < nbox8; ++i)
-              sm100::tma_load_2d(sw + i * 1024, tw8, &full[stage], x, mine.start + kGranule * i,
-                                 pol_w);
-          }
-          sm100::tma_load_2d(sh, th, &full[stage], x, p.b_off, pol_h);
-        }
-      }
-      ++issued;
-      if (++stage == C::kStages) {
-        stage = 0;
-        phase ^= 1u;
-      }
-    }
-  }
-  if (!ok && issued > 0 && (!PAIR || rank == 0)) {
-    // Gave up: let the copies already in flight land before the CTA exits.
-    // (The odd CTA of a pair cannot observe its copies, which complete on the
-    // even CTA's barriers; it exits only after the cluster barrier at the end
-    // of the kernel, which the even CTA reaches after this drain.)
-    // One time limit covers the whole drain.
-    const long long first = issued > C::kStages ? issued - C::kStages : 0;
-    const long long t0 = clock64();
-    for (long long n = first; n < issued; ++n) {
-      const int s = static_cast<int>(n % C::kStages);
-      const uint32_t ph = static_cast<uint32_t>((n / C::kStages) & 1);
-      while (!sm100::mbar_try_wait<PAIR>(&full[s], ph) && clock64() - t0 < sm100::kWaitLimitCycles) {
-      }
-    }
-  }
-}
-
-// MMA issuer (one thread; in pair mode only the even CTA's).
-template <int BN, int MODE, bool PAIR>
-__device__ __forceinline__ void role_mma(const FmmsParams &p, const Schedule &sch,
-                                         uint8_t *stages, uint64_t *full, uint64_t *empty,
-                                         uint64_t *acc_full, uint64_t *acc_empty,
-                                         uint64_t *drain_bar, uint32_t tmem_base,
-                                         volatile int *abort_flag, int unit) {
-  using C = KCfg<BN, MODE, PAIR>;
-  TileIter it(sch, unit);
-  Tile tile;
-  int stage = 0;
-  uint32_t phase = 0;
-  int buf = 0;
-  uint32_t acc_phase = 0;
-  bool ok = true;
-  while (ok && it.next(tile)) {
-    if (!sm100::wait_bounded<PAIR>(&acc_empty[buf], acc_phase ^ 1u, abort_flag, p.err)) break;
-    sm100::tc_fence_after();
-    const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
-    const int nks = (p.nk + C::kSub - 1) / C::kSub;
-    for (int ks = 0; ks < nks; ++ks) {
-      if (!sm100::wait_bounded<PAIR>(&full[stage], phase, abort_flag, p.err)) {
-        ok = false;
-        break;
-      }
-      sm100::tc_fence_after();
-      const int nsub = imin(C::kSub, p.nk - ks * C::kSub);
-      const uint32_t a_addr = sm100::smem_addr(stages + stage * C::kStageBytes);
-      const uint32_t b_addr = a_addr + C::kStageW;
-#pragma unroll
-      for (int j = 0; j < C::kSub; ++j) {
-        if (j >= nsub) break;
-#pragma unroll
-        for (int kk = 0; kk < kBlockK / 16; ++kk) {
-          const uint64_t da = sm100::smem_desc_sw128(a_addr + j * C::kSubW + kk * 32);
-          const uint64_t db = sm100::smem_desc_sw128(b_addr + j * C::kSubH + kk * 32);
-          const uint32_t acc = (ks | j | kk) != 0 ? 1u : 0u;
-          if constexpr (PAIR) {
-            sm100::mma_bf16_ss_pair(d_tmem, da, db, C::kIdesc, acc);
-          } else {
-            sm100::mma_bf16_ss(d_tmem, da, db, C::kIdesc, acc);
-          }
-        }
-      }
-      // Frees the stage once these MMAs finish.
-      if constexpr (PAIR) {
-        sm100::mma_commit_pair(&empty[stage]);
-      } else {
-        sm100::mma_commit(&empty[stage]);
-      }
-      if (++stage == C::kStages) {
-        stage = 0;
-        phase ^= 1u;
-      }
-    }
-    if (!ok) break;
-    // Accumulator ready for the epilogue.
-    if constexpr (PAIR) {
-      sm100::mma_commit_pair(&acc_full[buf]);
-    } else {
-      sm100::mma_commit(&acc_full[buf]);
-    }
-    if (++buf == C::kAccBufs) {
-      buf = 0;
-      acc_phase ^= 1u;
-    }
-  }
-  // Drain: every MMA issued above has completed once this arrives.
-  if constexpr (PAIR) {
-    sm100::mma_commit_pair(drain_bar);
-  } else {
-    sm100::mma_commit(drain_bar);
-  }
-  const long long t0 = clock64();
-  while (!sm100::mbar_try_wait<PAIR>(drain_bar, 0) && clock64() - t0 < sm100::kWaitLimitCycles) {
-  }
-}
-
-// Epilogue warps.  In pair mode each CTA drains its own 128 accumulator rows
-// (its half of the pair tile); the even CTA hands every filled accumulator on
-// to the odd CTA, and the odd CTA's warps release it on the even CTA's
-// barrier, where the MMAs are issued.
-template <int BN, int MODE, bool PAIR>
-__device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedule &sch,
-                                              uint32_t tmem_base, uint64_t *acc_full,
-                                              uint64_t *acc_empty, volatile int *abort_flag,
-                                              int *last_flag, uint64_t *comb_key, float *comb_m,
-                                              float *comb_s, int warp, int lane, int unit,
-                                              int rank) {
-  using C = KCfg<BN, MODE, PAIR>;
-  constexpr int CW = C::kCW;
-  const int q = warp & 3;          // TMEM lane quarter this warp may access
-  const int h = (warp - 2) >> 2;   // which of the quarter's warps: chunks h, h+4, ...
-  const int etid = (warp - 2) * 32 + lane;
-  const bool has_chunks = h < C::kChunks;
-
-  // Grouped mode: the running (best key, max, sum) of each (lane quarter,
-  // column) over the current segment live in shared memory, [4][BN] each,
-  // which keeps them out of the registers the chunk arithmetic needs.
-  if constexpr (MODE == kModeGrouped) {
-    for (int i = etid; i < 4 * BN; i += kEpiThreads) {
-      comb_key[i] = 0ull;
-      comb_m[i] = -INFINITY;
-      comb_s[i] = 0.f;
-    }
-    sm100::epi_sync(kEpiThreads);
-  }
-
-  TileIter it(sch, unit);
-  Tile tile;
-  int buf = 0;
-  uint32_t phase = 0;
-  bool aborted = false;
-  while (it.next(tile)) {
-    // After an abort the loop keeps walking the tiles without touching TMEM,
-    // so that every epilogue warp reaches the same named barriers.  The
-    // decision is made warp-uniform because the TMEM loads below are
-    // warp-collective.
-    const bool got = aborted ? false : sm100::wait_bounded<PAIR>(&acc_full[buf], phase, abort_flag, p.err);
-    aborted = __any_sync(0xffffffffu, !got);
-    if (!aborted) {
-      if (PAIR && rank == 0 && warp == 2 && lane == 0)
-        sm100::mbar_arrive_cluster(sm100::cluster_addr(&acc_full[buf], 1));
-      sm100::tc_fence_after();
-      const Tile mine = PAIR ? pair_half(tile, rank) : tile;
-      const int v = mine.start + 32 * q + lane;           // row of W in this launch
-      const bool v_ok = v >= mine.lo && v < mine.hi;
-      const int vg = v + p.vocab_offset;                  // global token index
-      const uint32_t tbase =
-          tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(buf * BN);
-#pragma unroll
-      for (int kk = 0; kk < C::kChunksPerWarp; ++kk) {
-        if (!has_chunks) continue;
-        const int k = kk * C::kWarpsPerQuarter + h;
-        const int col0 = k * CW;
-        if (col0 >= p.B) continue;  // warp-uniform
-        uint32_t acc[CW];
-        if constexpr (CW == 32) {
-          sm100::tmem_ld_32(tbase + col0, acc);
-        } else {
-          sm100::tmem_ld_16(tbase + col0, acc);
-        }
-        sm100::tmem_wait_ld();
-        if constexpr (MODE == kModeLogits) {
-          if (v_ok) {
-#pragma unroll
-            for (int j = 0; j < CW; ++j)
-              if (col0 + j < p.B)
-                p.logits[static_cast<size_t>(col0 + j) * p.V + v] = __uint_as_float(acc[j]);
-          }
-        } else {
-          const int c = col0 + column_of_lane<CW>(lane);  // this lane's column
-          if constexpr (MODE == kModeFlat) {
-            // Sample smp draws with token-noise tag 2 smp and keeps its running
-            // per-row maximum in the published keys [smp][row]: every exact
-            // chunk raises it at once, which also sharpens every CTA's filter.
-            // The mask is consulted only on the exact path.
-            const uint32_t in_range = chunk_in_range<CW>(p, v_ok, col0);
-            uint32_t allowed = 0u;
-            bool have_allowed = false;
-#pragma unroll 1
-            for (int smp = 0; smp < p.num_samples; ++smp) {
-              unsigned long long *kp = p.keys + smp * kMaxBN + c;
-              const uint64_t pub = c < p.B ? ld_key(kp) : 0ull;  // in flight during Philox
-              uint32_t words[CW];
-              chunk_noise<CW>(p, vg, col0, lane, 2u * static_cast<uint32_t>(smp), words);
-              if (chunk_any_candidate<CW>(acc, words, p, in_range, 0ull, pub, lane)) {
-                if (!have_allowed) {
-                  allowed = chunk_allowed<CW>(p, vg, v_ok, col0, lane);
-                  have_allowed = true;
-                }
-                uint64_t cbest = 0ull;
-                chunk_keys<CW>(acc, words, p, vg, allowed, lane, cbest);
-                if ((lane & 1) == 0 && c < p.B && key_valid(cbest) && cbest > pub)
-                  atomicMax(kp, static_cast<unsigned long long>(cbest));
-              }
-            }
-          } else {
-            unsigned long long *gk =
-                p.gkeys ? p.gkeys + static_cast<size_t>(tile.slot - unit) * p.B + c : nullptr;
-            const uint64_t pub = (gk != nullptr && c < p.B) ? ld_key(gk) : 0ull;
-            const uint32_t allowed = chunk_allowed<CW>(p, vg, v_ok, col0, lane);
-            uint32_t words[CW];
-            chunk_noise<CW>(p, vg, col0, lane, 0u, words);
-            const int si = q * BN + c;  // this lane's (quarter, column) state
-            float m_run = comb_m[si], s_run = comb_s[si];
-            uint64_t best = comb_key[si];
-            chunk_lse<CW>(acc, p, allowed, lane, m_run, s_run);
-            if (chunk_any_candidate<CW>(acc, words, p, allowed, best, pub, lane)) {
-              chunk_keys<CW>(acc, words, p, vg, allowed, lane, best);
-              if (gk != nullptr && (lane & 1) == 0 && c < p.B && key_valid(best) && best > pub)
-                atomicMax(gk, static_cast<unsigned long long>(best));
-            }
-            if ((lane & 1) == 0) {  // the two lanes of a column hold the same values
-              comb_key[si] = best;
-              comb_m[si] = m_run;
-              comb_s[si] = s_run;
-            }
-          }
-        }
-      }
-      sm100::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        if (PAIR && rank == 1) {
-          sm100::mbar_arrive_cluster(sm100::cluster_addr(&acc_empty[buf], 0));
-        } else {
-          sm100::mbar_arrive(&acc_empty[buf]);
-        }
-      }
-    }
-    if (++buf == C::kAccBufs) {
-      buf = 0;
-      phase ^= 1u;
-    }
-
-    if constexpr (MODE == kModeGrouped) {
-      if (tile.last) {
-        // Segment done: combine the four lane quarters, write the partial
-        // (slot per CTA: a pair's two CTAs write slots 2 s and 2 s + 1) and
-        // reset the state for the next segment.
-        sm100::epi_sync(kEpiThreads);
-        const size_t slot = PAIR ? 2 * static_cast<size_t>(tile.slot) + rank
-                                 : static_cast<size_t>(tile.slot);
-        for (int b = etid; b < BN; b += kEpiThreads) {
-          uint64_t kb = 0ull;
-          float m = -INFINITY, s = 0.f;
-#pragma unroll
-          for (int qq = 0; qq < 4; ++qq) {
-            const uint64_t kq = comb_key[qq * BN + b];
-            kb = kq > kb ? kq : kb;
-            lse_merge(m, s, comb_m[qq * BN + b], comb_s[qq * BN + b]);
-            comb_key[qq * BN + b] = 0ull;
-            comb_m[qq * BN + b] = -INFINITY;
-            comb_s[qq * BN + b] = 0.f;
-          }
-          if (b < p.B && !*abort_flag) {
-            GroupPartial gp;
-            gp.key = kb;
-            gp.m = m;
-            gp.sum = s;
-            p.partials[slot * p.B + b] = gp;
-          }
-        }
-        sm100::epi_sync(kEpiThreads);
-      }
-    }
-  }
-
-  if constexpr (MODE == kModeFlat) {
-    // Every maximum is already published; take a ticket, and the last CTA
-    // decodes the keys and re-zeroes them for the next call.
-    __threadfence();
-    sm100::epi_sync(kEpiThreads);
-    if (etid == 0) {
-      int last = 0;
-      if (!*abort_flag)
-        last = (atomicAdd(p.ticket, 1u) == static_cast<unsigned>(p.num_ctas - 1)) ? 1 : 0;
-      *last_flag = last;
-    }
-    sm100::epi_sync(kEpiThreads);
-    if (*last_flag) {
-      __threadfence();
-      const int total = p.B * p.num_samples;
-      for (int i = etid; i < total; i += kEpiThreads) {
-        const int b = i / p.num_samples;
-        const int smp = i - b * p.num_samples;
-        const unsigned long long kb = atomicExch(p.keys + smp * kMaxBN + b, 0ull);
-        if (p.out_keys != nullptr)
-          p.out_keys[i] = static_cast<long long>(kb ^ 0x8000000000000000ull);  // signed order
-        else
-          p.out_idx[i] = key_token(kb);
-      }
-      if (etid == 0) atomicExch(p.ticket, 0u);
-    }
-  }
-}
-
-// ---------------------------------------------------------------------------
-// Kernel
-// ---------------------------------------------------------------------------
-template <int BN, int MODE, bool PAIR>
-__global__ void __launch_bounds__(kThreads, 1)
-    fmms_kernel(const __grid_constant__ CUtensorMap tmap_w,
-                const __grid_constant__ CUtensorMap tmap_w8,
-                const __grid_constant__ CUtensorMap tmap_h, const FmmsParams p) {
-  using C = KCfg<BN, MODE, PAIR>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t *stages = smem;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kStages * C::kStageBytes);
-  uint64_t *full = bars;
-  uint64_t *empty = full + C::kStages;
-  uint64_t *acc_full = empty + C::kStages;
-  uint64_t *acc_empty = acc_full + C::kAccBufs;
-  uint64_t *drain_bar = acc_empty + C::kAccBufs;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain_bar + 1);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-  int *last_flag = reinterpret_cast<int *>(tmem_slot + 2);
-  uint8_t *comb = reinterpret_cast<uint8_t *>(bars) + C::kBarBytes;
-  uint64_t *comb_key = reinterpret_cast<uint64_t *>(comb);
-  float *comb_m = reinterpret_cast<float *>(comb_key + 4 * BN);
-  float *comb_s = comb_m + 4 * BN;
-
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  // Pair mode: the two CTAs of a cluster form schedule unit blockIdx.x / 2.
-  const int rank = PAIR ? static_cast<int>(sm100::cluster_ctarank()) : 0;
-  const int unit = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
-  Schedule sch;
-  sch.V = p.V;
-  sch.G = p.G;
-  sch.num_ctas = PAIR ? p.num_ctas / 2 : p.num_ctas;
-  sch.ngran = p.ngran;
-  sch.tile_rows = PAIR ? 2 * kTileM : kTileM;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < C::kStages; ++s) {
-      sm100::mbar_init(&full[s], 1);
-      sm100::mbar_init(&empty[s], 1);
-    }
-    for (int b = 0; b < C::kAccBufs; ++b) {
-      sm100::mbar_init(&acc_full[b], 1);
-      sm100::mbar_init(&acc_empty[b], C::kEpiArrivals);
-    }
-    sm100::mbar_init(drain_bar, 1);
-    *abort_flag = 0;
-    *last_flag = 0;
-    sm100::fence_mbar_init();
-    sm100::fence_async_smem();
-    sm100::prefetch_tensormap(&tmap_w);
-    sm100::prefetch_tensormap(&tmap_w8);
-    sm100::prefetch_tensormap(&tmap_h);
-  }
-  if constexpr (PAIR) {
-    // Both CTAs' barriers are initialised before either CTA signals the
-    // other's; the pair then allocates tensor memory collectively.
-    __syncthreads();
-    sm100::cluster_sync();
-    if (warp == 1) {
-      sm100::tmem_alloc_pair(tmem_slot, C::kTmemCols);
-      sm100::tmem_relinquish_pair();
-    }
-  } else {
-    if (warp == 1) {
-      sm100::tmem_alloc(tmem_slot, C::kTmemCols);
-      sm100::tmem_relinquish();
-    }
-  }
-  sm100::tc_fence_before();
-  __syncthreads();
-  sm100::tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
-
-  if (warp == 0) {
-    if (lane == 0)
-      role_producer<BN, MODE, PAIR>(&tmap_w, &tmap_w8, &tmap_h, p, sch, stages, full, empty,
-                                    abort_flag, unit, rank);
-    __syncwarp();
-  } else if (warp == 1) {
-    if (lane == 0 && rank == 0)
-      role_mma<BN, MODE, PAIR>(p, sch, stages, full, empty, acc_full, acc_empty, drain_bar,
-                               tmem_base, abort_flag, unit);
-    __syncwarp();
-  } else {
-    role_epilogue<BN, MODE, PAIR>(p, sch, tmem_base, acc_full, acc_empty, abort_flag, last_flag,
-                                  comb_key, comb_m, comb_s, warp, lane, unit, rank);
-  }
-
-  sm100::tc_fence_before();
-  __syncthreads();
-  if constexpr (PAIR) {
-    // Neither CTA frees tensor memory while the other may still use it: the
-    // even CTA's MMAs write both, and each CTA's epilogue reads its own.
-    sm100::cluster_sync();
-  }
-  sm100::tc_fence_after();
-  if (warp == 1) {
-    if constexpr (PAIR) {
-      sm100::tmem_dealloc_pair(tmem_base, C::kTmemCols);
-    } else {
-      sm100::tmem_dealloc(tmem_base, C::kTmemCols);
-    }
-  }
-}
-
-// ---------------------------------------------------------------------------
-// Host launchers
-// ---------------------------------------------------------------------------
-template <int BN, int MODE>
-static cudaError_t launch_t(const CUtensorMap &tw, const CUtensorMap &tw8, const CUtensorMap &th,
-                            const FmmsParams &p, cudaStream_t stream) {
-  using C = KCfg<BN, MODE>;
-  auto kern = fmms_kernel<BN, MODE, false>;
-  cudaError_t e =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
-  if (e != cudaSuccess) return e;
-  kern<<<p.num_ctas, kThreads, C::kSmemBytes, stream>>>(tw, tw8, th, p);
-  return cudaGetLastError();
-}
-
-template <int MODE>
-static cudaError_t launch_mode(int BN, const CUtensorMap &tw, const CUtensorMap &tw8,
-                               const CUtensorMap &th, const FmmsParams &p, cudaStream_t stream) {
-  switch (BN) {
-    case 16: return launch_t<16, MODE>(tw, tw8, th, p, stream);
-    case 32: return launch_t<32, MODE>(tw, tw8, th, p, stream);
-    case 64: return launch_t<64, MODE>(tw, tw8, th, p, stream);
-    case 128: return launch_t<128, MODE>(tw, tw8, th, p, stream);
-    case 256: return launch_t<256, MODE>(tw, tw8, th, p, stream);
-    default: return cudaErrorInvalidValue;
-  }
-}
 
 cudaError_t launch_fmms(int mode, int BN, const CUtensorMap &tw, const CUtensorMap &tw8,
                         const CUtensorMap &th, const FmmsParams &p, cudaStream_t stream) {
   switch (mode) {
-    case kModeFlat: return launch_mode<kModeFlat>(BN, tw, tw8, th, p, stream);
-    case kModeGrouped: return launch_mode<kModeGrouped>(BN, tw, tw8, th, p, stream);
-    case kModeLogits: return launch_mode<kModeLogits>(BN, tw, tw8, th, p, stream);
-    default: return cudaErrorInvalidValue;
-  }
-}
-
-// Pair kernels: clusters of two CTAs, p.num_ctas = 2 x schedule units.
-template <int BN, int MODE>
-static cudaLaunchConfig_t pair_config(int num_ctas, cudaStream_t stream,
-                                      cudaLaunchAttribute *attr) {
-  using C = KCfg<BN, MODE, true>;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(num_ctas), 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = C::kSmemBytes;
-  cfg.stream = stream;
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cfg;
-}
-
-template <int BN, int MODE>
-static cudaError_t pair_units_t(int *units) {
-  using C = KCfg<BN, MODE, true>;
-  auto kern = fmms_kernel<BN, MODE, true>;
-  cudaError_t e =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
-  if (e != cudaSuccess) return e;
-  cudaLaunchAttribute attr[1];
-  cudaLaunchConfig_t cfg = pair_config<BN, MODE>(2, nullptr, attr);
-  int n = 0;
-  e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
-  if (e != cudaSuccess) return e;
-  *units = n;
-  return cudaSuccess;
-}
-
-template <int BN, int MODE>
-static cudaError_t launch_pair_t(const CUtensorMap &tw, const CUtensorMap &tw8,
-                                 const CUtensorMap &th, const FmmsParams &p,
-                                 cudaStream_t stream) {
-  using C = KCfg<BN, MODE, true>;
-  auto kern = fmms_kernel<BN, MODE, true>;
-  cudaError_t e =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
-  if (e != cudaSuccess) return e;
-  cudaLaunchAttribute attr[1];
-  cudaLaunchConfig_t cfg = pair_config<BN, MODE>(p.num_ctas, stream, attr);
-  e = cudaLaunchKernelEx(&cfg, kern, tw, tw8, th, p);
-  if (e != cudaSuccess) return e;
-  return cudaGetLastError();
-}
-
-template <int MODE>
-static cudaError_t pair_units_mode(int BN, int *units) {
-  switch (BN) {
-    case 16: return pair_units_t<16, MODE>(units);
-    case 32: return pair_units_t<32, MODE>(units);
-    case 64: return pair_units_t<64, MODE>(units);
-    case 128: return pair_units_t<128, MODE>(units);
-    case 256: return pair_units_t<256, MODE>(units);
-    default: return cudaErrorInvalidValue;
-  }
-}
-
-template <int MODE>
-static cudaError_t launch_pair_mode(int BN, const CUtensorMap &tw, const CUtensorMap &tw8,
-                                    const CUtensorMap &th, const FmmsParams &p,
-                                    cudaStream_t stream) {
-  switch (BN) {
-    case 16: return launch_pair_t<16, MODE>(tw, tw8, th, p, stream);
-    case 32: return launch_pair_t<32, MODE>(tw, tw8, th, p, stream);
-    case 64: return launch_pair_t<64, MODE>(tw, tw8, th, p, stream);
-    case 128: return launch_pair_t<128, MODE>(tw, tw8, th, p, stream);
-    case 256: return launch_pair_t<256, MODE>(tw, tw8, th, p, stream);
-    default: return cudaErrorInvalidValue;
-  }
-}
-
-cudaError_t fmms_pair_units(int mode, int BN, int *units) {
-  switch (mode) {
-    case kModeFlat: return pair_units_mode<kModeFlat>(BN, units);
-    case kModeGrouped: return pair_units_mode<kModeGrouped>(BN, units);
+    case kModeFlat: return launch_flat(BN, tw, tw8, th, p, stream);
+    case kModeGrouped: return launch_grouped(BN, tw, tw8, th, p, stream);
+    case kModeLogits: return launch_logits(BN, tw, tw8, th, p, stream);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -943,18 +19,23 @@ cudaError_t fmms_pair_units(int mode, int BN, int *units) {
 cudaError_t launch_fmms_pair(int mode, int BN, const CUtensorMap &tw, const CUtensorMap &tw8,
                              const CUtensorMap &th, const FmmsParams &p, cudaStream_t stream) {
   switch (mode) {
-    case kModeFlat: return launch_pair_mode<kModeFlat>(BN, tw, tw8, th, p, stream);
-    case kModeGrouped: return launch_pair_mode<kModeGrouped>(BN, tw, tw8, th, p, stream);
+    case kModeFlat: return launch_flat_pair(BN, tw, tw8, th, p, stream);
+    case kModeGrouped: return launch_grouped_pair(BN, tw, tw8, th, p, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t fmms_pair_units(int mode, int BN, int *units) {
+  switch (mode) {
+    case kModeFlat: return pair_units_flat(BN, units);
+    case kModeGrouped: return pair_units_grouped(BN, units);
     default: return cudaErrorInvalidValue;
   }
 }
 
 int fmms_batch_tile(int rows) {
-  if (rows <= 16) return 16;
-  if (rows <= 32) return 32;
-  if (rows <= 64) return 64;
-  if (rows <= 128) return 128;
-  return 256;
+  const int bn = (rows + 15) / 16 * 16;
+  return bn < 16 ? 16 : (bn > kMaxBN ? kMaxBN : bn);
 }
 
 }  // namespace fmms

@@ -9,8 +9,23 @@
 
 namespace fmms {
 
-// Smallest supported MMA N (16, 32, 64, 128, 256) holding `rows` batch rows.
+// Batch tile (MMA N) of a launch of `rows` rows: the next multiple of 16,
+// at most 256.
 int fmms_batch_tile(int rows);
+
+// Per-mode launchers for every batch tile (fmms_inst_*.cu).
+cudaError_t launch_flat(int BN, const CUtensorMap &tw, const CUtensorMap &tw8,
+                        const CUtensorMap &th, const FmmsParams &p, cudaStream_t stream);
+cudaError_t launch_grouped(int BN, const CUtensorMap &tw, const CUtensorMap &tw8,
+                           const CUtensorMap &th, const FmmsParams &p, cudaStream_t stream);
+cudaError_t launch_logits(int BN, const CUtensorMap &tw, const CUtensorMap &tw8,
+                          const CUtensorMap &th, const FmmsParams &p, cudaStream_t stream);
+cudaError_t launch_flat_pair(int BN, const CUtensorMap &tw, const CUtensorMap &tw8,
+                             const CUtensorMap &th, const FmmsParams &p, cudaStream_t stream);
+cudaError_t launch_grouped_pair(int BN, const CUtensorMap &tw, const CUtensorMap &tw8,
+                                const CUtensorMap &th, const FmmsParams &p, cudaStream_t stream);
+cudaError_t pair_units_flat(int BN, int *units);
+cudaError_t pair_units_grouped(int BN, int *units);
 
 // The fused kernel in mode kModeFlat / kModeGrouped / kModeLogits with batch
 // tile BN, grid p.num_ctas x kThreads threads.
