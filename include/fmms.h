@@ -229,9 +229,14 @@ fs_status fs_sample_topk(const void *H, const void *W, int B, int d, int V,
 /* End-to-end call with HOST buffers: H_host (bf16 [B, d]) and out_idx_host
  * (int32 [B]) are host pointers (page-locked for the copies to be
  * asynchronous); W and row_seeds/mask_bits stay device pointers.  Enqueues
- * the host-to-device copy of H into a library-owned device buffer, the
- * fused sample, and the device-to-host copy of the tokens on `stream`; the
- * tokens are valid once the stream is synchronised. */
+ * the host-to-device copy of H into a library-owned device buffer on a
+ * library stream (after the previous fs_sample_host call's kernel, which
+ * reads that buffer), the fused sample on `stream` (it starts streaming W at
+ * once and waits on the device, with the usual one-second limit, for the
+ * copy of H to land), and the device-to-host copy of the tokens on
+ * `stream`; the tokens are valid once `stream` is synchronised.  H_host must
+ * stay unchanged until then.  Without stream memory operations on the
+ * device, the copy of H runs on `stream` before the sample. */
 fs_status fs_sample_host(const void *H_host, const void *W, int B, int d,
                          int V, float temperature, uint64_t seed,
                          const uint64_t *row_seeds, uint32_t step,

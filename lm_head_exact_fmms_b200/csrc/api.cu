@@ -29,6 +29,16 @@ struct DeviceState {
   size_t h_stage_bytes = 0;
   void *o_stage = nullptr;  // fs_sample_host: device tokens
   size_t o_stage_bytes = 0;
+  // fs_sample_host: H is copied on copy_stream while the kernel already
+  // streams W; h_flags takes the call's epoch once the copy has landed.
+  // kernel_done keeps the next call's copy off h_stage until this call's
+  // kernel has finished with it.
+  bool host_overlap_init = false;
+  bool host_overlap = false;
+  cudaStream_t copy_stream = nullptr;
+  cudaEvent_t kernel_done = nullptr;
+  uint32_t *h_flags = nullptr;  // device word: epoch of the H copy that has landed
+  uint32_t h_epoch = 0;
   int pair_units[2][fmms::kMaxBN / 16];  // resident CTA pairs [flat, grouped][tile / 16 - 1]; -1: unknown
   DeviceState() {
     for (auto &row : pair_units)
@@ -76,6 +86,24 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_
                                    const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
                                    const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// cuStreamWriteValue32: a 32-bit store done by the copy engine in stream
+// order, so it needs no SM while the persistent kernel holds all of them.
+using StreamWriteValue32Fn = CUresult (*)(CUstream, CUdeviceptr, cuuint32_t, unsigned int);
+
+StreamWriteValue32Fn write_value_fn() {
+  static StreamWriteValue32Fn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuStreamWriteValue32", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<StreamWriteValue32Fn>(p);
+  });
+  return fn;
+}
 
 EncodeTiledFn encode_fn() {
   static EncodeTiledFn fn = nullptr;
@@ -230,6 +258,9 @@ struct ShardOpts {
   long long *out_keys = nullptr;  // write packed keys instead of tokens
   int num_samples = 1;          // samples per row (flat mode)
   int top_k = 0;                // logits mode: top-k selection instead of full sampling
+  const uint32_t *h_ready = nullptr;  // H arriving in chunks (fs_sample_host), else null
+  uint32_t h_epoch = 0;
+  int h_chunk_subs = 0;
 };
 
 // The fused path in all three modes, chunked over 256 batch rows.
@@ -302,6 +333,9 @@ fs_status run_locked(int mode, const void *H, const void *W, int B, int d, int V
     p.vocab_offset = shard.vocab_offset;
     p.out_keys = shard.out_keys ? shard.out_keys + static_cast<size_t>(b0) * S : nullptr;
     p.num_samples = S;
+    p.h_ready = shard.h_ready;
+    p.h_epoch = shard.h_epoch;
+    p.h_chunk_subs = shard.h_chunk_subs;
     const int pair_units_used = pair ? fmms::make_schedule(V, sch.G, units).num_ctas : 0;
     if (pair) {
       p.num_ctas = 2 * pair_units_used;
@@ -410,23 +444,56 @@ fs_status fs_sample_host(const void *H_host, const void *W, int B, int d, int V,
   if (!(temperature > 0.f) || !isfinite(temperature) || !W || !aligned16(W))
     return FS_ERR_INVALID_ARG;
   cudaStream_t st_ = static_cast<cudaStream_t>(stream);
-  void *hdev = nullptr, *odev = nullptr;
-  {
-    std::lock_guard<std::mutex> lock(g_mu);
-    DeviceState *st = nullptr;
-    fs_status s = get_device(&st);
-    if (s != FS_OK) return s;
-    const size_t hbytes = static_cast<size_t>(B) * d * 2;
-    if ((s = grow(&st->h_stage, &st->h_stage_bytes, hbytes)) != FS_OK) return s;
-    if ((s = grow(&st->o_stage, &st->o_stage_bytes, static_cast<size_t>(B) * 4)) != FS_OK) return s;
-    hdev = st->h_stage;
-    odev = st->o_stage;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState *st = nullptr;
+  fs_status s = get_device(&st);
+  if (s != FS_OK) return s;
+  const size_t hbytes = static_cast<size_t>(B) * d * 2;
+  if ((s = grow(&st->h_stage, &st->h_stage_bytes, hbytes)) != FS_OK) return s;
+  if ((s = grow(&st->o_stage, &st->o_stage_bytes, static_cast<size_t>(B) * 4)) != FS_OK) return s;
+  char *hdev = static_cast<char *>(st->h_stage);
+  int32_t *odev = static_cast<int32_t *>(st->o_stage);
+
+  if (!st->host_overlap_init) {
+    st->host_overlap_init = true;
+    st->host_overlap =
+        write_value_fn() != nullptr &&
+        cudaStreamCreateWithFlags(&st->copy_stream, cudaStreamNonBlocking) == cudaSuccess &&
+        cudaEventCreateWithFlags(&st->kernel_done, cudaEventDisableTiming) == cudaSuccess &&
+        cudaMalloc(&st->h_flags, sizeof(uint32_t)) == cudaSuccess &&
+        cudaMemset(st->h_flags, 0, sizeof(uint32_t)) == cudaSuccess &&
+        cudaDeviceSynchronize() == cudaSuccess;
+  }
+
+  ShardOpts opts;
+  if (st->host_overlap) {
+    // H is copied on the library's copy stream once the previous call's
+    // kernel is done with the staging buffer, and a copy-engine write then
+    // sets the flag to this call's epoch.  The kernel, launched at once,
+    // streams W from its start and loads H once the flag holds the epoch, so
+    // the launch and the first W loads overlap the copy.  (Copying H in
+    // several K-column chunks, each with its own flag, measured slower: 2-D
+    // copies of 64-row strips and the extra waits cost more than they hid.)
+    const int nk = (d + fmms::kBlockK - 1) / fmms::kBlockK;
+    const uint32_t epoch = ++st->h_epoch == 0 ? ++st->h_epoch : st->h_epoch;
+    if (cudaStreamWaitEvent(st->copy_stream, st->kernel_done, 0) != cudaSuccess) return FS_ERR_CUDA;
+    if (cudaMemcpyAsync(hdev, H_host, hbytes, cudaMemcpyHostToDevice, st->copy_stream) !=
+        cudaSuccess)
+      return FS_ERR_CUDA;
+    if (write_value_fn()(reinterpret_cast<CUstream>(st->copy_stream),
+                         reinterpret_cast<CUdeviceptr>(st->h_flags), epoch, 0) != CUDA_SUCCESS)
+      return FS_ERR_CUDA;
+    opts.h_ready = st->h_flags;
+    opts.h_epoch = epoch;
+    opts.h_chunk_subs = nk;
+  } else {
     if (cudaMemcpyAsync(hdev, H_host, hbytes, cudaMemcpyHostToDevice, st_) != cudaSuccess)
       return FS_ERR_CUDA;
   }
-  fs_status s = run(fmms::kModeFlat, hdev, W, B, d, V, 1, temperature, seed, row_seeds, step,
-                    mask_bits, static_cast<int32_t *>(odev), nullptr, nullptr, nullptr, 0, st_);
+  s = run_locked(fmms::kModeFlat, hdev, W, B, d, V, 1, temperature, seed, row_seeds, step,
+                 mask_bits, odev, nullptr, nullptr, nullptr, 0, st_, opts);
   if (s != FS_OK) return s;
+  if (st->host_overlap && cudaEventRecord(st->kernel_done, st_) != cudaSuccess) return FS_ERR_CUDA;
   if (cudaMemcpyAsync(out_idx_host, odev, static_cast<size_t>(B) * 4, cudaMemcpyDeviceToHost,
                       st_) != cudaSuccess)
     return FS_ERR_CUDA;

@@ -195,6 +195,12 @@ struct FmmsParams {
   int vocab_offset;            // global token index of W row 0 (a vocabulary shard), % 8 == 0
   long long *out_keys;         // if set: per-row packed keys XOR 2^63 instead of tokens
   int num_samples;             // samples per row (flat mode), 1..kMaxSamples
+  // H arriving while the kernel runs (fs_sample_host): 64-wide K sub-block s
+  // of H may be loaded once h_ready[s / h_chunk_subs] == h_epoch.  Null: H is
+  // complete when the kernel starts.
+  const uint32_t *h_ready;
+  uint32_t h_epoch;
+  int h_chunk_subs;
 };
 
 // Workspace layout (bytes), fixed so that calls of different kinds can share

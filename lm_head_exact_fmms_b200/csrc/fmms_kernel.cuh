@@ -365,6 +365,7 @@ __device__ __forceinline__ void role_producer(const CUtensorMap *tw, const CUten
   int stage = 0;
   uint32_t phase = 0;
   long long issued = 0;
+  int h_chunks_ready = -1;  // chunks of H known to have arrived (h_ready mode)
   bool ok = p.test_no_loads == 0;
   while (ok && it.next(tile)) {
     const Tile mine = PAIR ? pair_half(tile, rank) : tile;
@@ -391,29 +392,49 @@ __device__ __forceinline__ void role_producer(const CUtensorMap *tw, const CUten
       uint8_t *sh0 = sw0 + C::kStageW;
       if (!PAIR || rank == 0) sm100::mbar_arrive_expect_tx(&full[stage], bytes);
       const uint32_t bar = PAIR ? sm100::cluster_addr(&full[stage], 0) : 0u;
+      // W first: it never waits for H.
 #pragma unroll
       for (int j = 0; j < C::kSub; ++j) {
         if (j >= nsub) break;
         uint8_t *sw = sw0 + j * C::kSubW;
+        const int x = (sub0 + j) * kBlockK;
+        if (whole) {
+          if constexpr (PAIR) {
+            sm100::tma_load_2d_pair(sw, tw, bar, x, mine.start, pol_w);
+          } else {
+            sm100::tma_load_2d(sw, tw, &full[stage], x, mine.start, pol_w);
+          }
+        } else {
+          for (int i = 0; i < nbox8; ++i) {
+            if constexpr (PAIR) {
+              sm100::tma_load_2d_pair(sw + i * 1024, tw8, bar, x, mine.start + kGranule * i,
+                                      pol_w);
+            } else {
+              sm100::tma_load_2d(sw + i * 1024, tw8, &full[stage], x, mine.start + kGranule * i,
+                                 pol_w);
+            }
+          }
+        }
+      }
+      // H still arriving from the host: wait for the chunk this stage ends in.
+      if (p.h_ready != nullptr) {
+        const int need = (sub0 + nsub - 1) / p.h_chunk_subs;
+        if (need > h_chunks_ready) {
+          if (!sm100::wait_flag_bounded(p.h_ready + need, p.h_epoch, abort_flag, p.err)) {
+            ok = false;
+            break;
+          }
+          h_chunks_ready = need;
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < C::kSub; ++j) {
+        if (j >= nsub) break;
         uint8_t *sh = sh0 + j * C::kSubH;
         const int x = (sub0 + j) * kBlockK;
         if constexpr (PAIR) {
-          if (whole) {
-            sm100::tma_load_2d_pair(sw, tw, bar, x, mine.start, pol_w);
-          } else {
-            for (int i = 0; i < nbox8; ++i)
-              sm100::tma_load_2d_pair(sw + i * 1024, tw8, bar, x, mine.start + kGranule * i,
-                                      pol_w);
-          }
           sm100::tma_load_2d_pair(sh, th, bar, x, p.b_off + rank * C::kHRows, pol_h);
         } else {
-          if (whole) {
-            sm100::tma_load_2d(sw, tw, &full[stage], x, mine.start, pol_w);
-          } else {
-            for (int i = 0; i < nbox8; ++i)
-              sm100::tma_load_2d(sw + i * 1024, tw8, &full[stage], x, mine.start + kGranule * i,
-                                 pol_w);
-          }
           sm100::tma_load_2d(sh, th, &full[stage], x, p.b_off, pol_h);
         }
       }

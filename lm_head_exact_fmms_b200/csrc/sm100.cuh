@@ -87,6 +87,27 @@ __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity,
   }
 }
 
+// Waits until *flag == value (written by a copy engine after a host-to-device
+// copy), with the same time limit as wait_bounded; then orders the TMA loads
+// that follow (async proxy) after the observation.
+__device__ __forceinline__ bool wait_flag_bounded(const uint32_t *flag, uint32_t value,
+                                                  volatile int *abort_flag, int *err) {
+  const long long t0 = clock64();
+  while (true) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+    if (v == value) break;
+    if (*abort_flag) return false;
+    if (clock64() - t0 > kWaitLimitCycles) {
+      *abort_flag = 1;
+      atomicCAS(err, 0, kErrTimeout);
+      return false;
+    }
+  }
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  return true;
+}
+
 // --------------------------------------------------------------------- TMA
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   uint64_t p;

@@ -214,6 +214,26 @@ def test_host_entry_point(dev):
     assert torch.equal(out, ref)
 
 
+def test_host_entry_point_back_to_back(dev):
+    """fs_sample_host copies H in K-column chunks on a copy stream while the
+    kernel already streams W.  Calls issued back to back with different host
+    H (no synchronisation in between), including a 300-row call (two
+    launches) and d not a multiple of the chunk size, must each give the
+    tokens of the device entry point on the same H."""
+    d, V = 200, 7001
+    W = synth.make_weight(V, d, 1.0 / np.sqrt(d), device="cpu", seed=71).to(dev)
+    calls = []
+    for i, B in enumerate([24, 300, 7, 24, 129]):
+        H = synth.make_hidden(B, d, device="cpu", seed=100 + i).pin_memory()
+        out = torch.empty(B, dtype=torch.int32).pin_memory()
+        binding.fs_sample_host(H, W, temperature=0.8, seed=5, step=i, out_idx_host=out)
+        calls.append((H, out, i))
+    torch.cuda.synchronize()
+    for H, out, i in calls:
+        ref = binding.fs_sample_ex(H.to(dev), W, temperature=0.8, seed=5, step=i).cpu()
+        assert torch.equal(out, ref), i
+
+
 def test_gumbel_max_is_softmax_on_gpu(dev, oracle):
     """Draws of identical rows (noise differs per row index) follow the exact
     softmax of l / T (chi-square)."""
