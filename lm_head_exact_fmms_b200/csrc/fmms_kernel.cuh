@@ -12,24 +12,31 @@
 //    slice of the vocabulary (split-V), so small batches still keep all 148
 //    SMs streaming W and no W row is read twice;
 //  * swap-AB MMA: A = 128 vocabulary rows of W (M = 128), B = the batch of
-//    hidden states (N = 16..256), D = a 128-lane x N-column fp32 accumulator
-//    in tensor memory; the tile's vocabulary rows land on TMEM lanes, i.e. on
-//    epilogue threads;
+//    hidden states (N = the batch tile, a multiple of 16 up to 256), D = a
+//    128-lane x N-column fp32 accumulator in tensor memory; the tile's
+//    vocabulary rows land on TMEM lanes, i.e. on epilogue threads;
+//  * CTA pairs (PAIR): two CTAs of a cluster share one M = 256 MMA
+//    (tcgen05 cta_group::2); each stages its own 128 W rows and half of the
+//    H rows and drains its own 128 accumulator rows;
 //  * warp roles: warp 0 issues TMA loads of W (evict-first) and H
-//    (evict-last) into a multi-stage 128-byte-swizzled shared-memory ring;
-//    warp 1 allocates TMEM and issues tcgen05.mma; warps 2-9 drain the
-//    double-buffered accumulator while the next tile is being multiplied;
-//  * epilogue per element: x = acc / T, Philox4x32-10 noise word for
+//    (evict-last) into a ring of 3-10 stages of 1-4 64-wide K sub-blocks
+//    (128-byte swizzle); warp 1 allocates TMEM and issues tcgen05.mma;
+//    warps 2-17 (four per TMEM lane quarter) drain up to four accumulators
+//    while the next tiles are being multiplied;
+//  * epilogue per 16-column chunk: x = acc / T, Philox4x32-10 noise words for
 //    (seed, step, row, token) (one Philox call serves four consecutive
-//    tokens; four lanes exchange words with a 4x4 shuffle transpose), the
-//    Gumbel transform, s = x + g, then a 32-lane "transpose-reduce" leaves
-//    lane j with the packed max of column j;
-//  * flat mode: per CTA, one atomicMax of a packed (score, token) key per row
-//    into the workspace; the last CTA to finish (atomic ticket, no waiting)
-//    decodes the tokens and re-zeroes the workspace;
+//    tokens; four lanes exchange words with a 4x4 shuffle transpose), a
+//    log-free upper bound of each Gumbel value, and only where a bound
+//    reaches the row's best published score the exact transform, s = x + g
+//    and a 32-lane "transpose-reduce" that leaves each lane pair with the
+//    packed max of one column;
+//  * flat mode: every improvement of a row's maximum is published with one
+//    atomicMax of a packed (score, token) key; the last CTA to finish (atomic
+//    ticket, no waiting) decodes the tokens and re-zeroes the keys;
 //  * grouped mode: per (segment, row) partial (max key, lse pieces) for the
 //    Group-Gumbel-Max merge kernel;
 //  * logits mode: raw fp32 logits to HBM for the unfused measurement path.
+// Every wait is bounded; a CTA that gives up records FS_ERR_DEVICE_TIMEOUT.
 #pragma once
 
 #include <cuda.h>
