@@ -37,10 +37,11 @@ FS_HD int imax(int a, int b) { return a > b ? a : b; }
 // num_ctas owns granules [floor(c n / C), floor((c+1) n / C)), so every CTA
 // streams the same number of W rows to within one granule.  Group g of G
 // covers [floor(g V / G), floor((g+1) V / G)).  A CTA's range is cut at group
-// boundaries into segments; each segment is walked in 128-row tiles whose
-// start is rounded down to a multiple of 8 (rows before the segment are
-// loaded but ignored).  Segment (c, g) owns partial slot c + g, which is
-// unique because c and g never both stay put from one segment to the next.
+// boundaries into segments; each segment is walked in 128-row tiles (256 on
+// CTA pairs) starting at its first token rounded down to a multiple of 8 (rows
+// before the segment are loaded but ignored), its partial tile first.
+// Segment (c, g) owns partial slot c + g, which is unique because c and g
+// never both stay put from one segment to the next.
 // ---------------------------------------------------------------------------
 struct Schedule {
   int V;
@@ -104,6 +105,7 @@ struct TileIter {
   int v;       // first token of the current segment
   int seg_hi;  // end of the current segment
   int t;       // start of the next tile
+  int len;     // rows of the next tile
   int slot;
 
   FS_HD TileIter(const Schedule &s, int c) {
@@ -115,9 +117,15 @@ struct TileIter {
     cta_hi = cta_begin(c + 1, s);
     seg_hi = v;
     t = v;
+    len = rows;
     slot = c;
   }
 
+  // A segment's partial tile comes first: its remainder rows, rounded up to a
+  // multiple of 8, then whole tiles (the last may lack up to 7 rows).  The MMA
+  // loop of a partial tile costs as much as a whole tile's; run first it
+  // overlaps the other CTAs' streaming, run last it would be a tail with HBM
+  // idle.
   FS_HD bool next(Tile &tile) {
     if (t >= seg_hi) {
       v = seg_hi;
@@ -127,12 +135,15 @@ struct TileIter {
       seg_hi = imin(cta_hi, gend);
       slot = cta + g;
       t = v & ~(kGranule - 1);
+      const int rem = (seg_hi - t) % rows;
+      len = rem == 0 ? rows : (rem + kGranule - 1) & ~(kGranule - 1);
     }
     tile.start = t;
     tile.lo = imax(t, v);
-    tile.hi = imin(t + rows, seg_hi);
+    tile.hi = imin(t + len, seg_hi);
     tile.slot = slot;
-    t += rows;
+    t += len;
+    len = rows;
     tile.last = (t >= seg_hi) ? 1 : 0;
     return true;
   }

@@ -614,10 +614,13 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
         sm100::tmem_wait_ld();
         if constexpr (MODE == kModeLogits) {
           if (v_ok) {
+            float *dst = p.logits + static_cast<size_t>(col0) * p.V + v;
+            const int ncol = imin(CW, p.B - col0);
 #pragma unroll
-            for (int j = 0; j < CW; ++j)
-              if (col0 + j < p.B)
-                p.logits[static_cast<size_t>(col0 + j) * p.V + v] = __uint_as_float(acc[j]);
+            for (int j = 0; j < CW; ++j) {
+              if (j < ncol) *dst = __uint_as_float(acc[j]);
+              dst += p.V;
+            }
           }
         } else {
           const int c = col0 + column_of_lane<CW>(lane);  // this lane's column
