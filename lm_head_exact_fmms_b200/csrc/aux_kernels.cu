@@ -12,13 +12,34 @@
 #include "fmms_common.cuh"
 #include "launch.h"
 #include "noise.cuh"
+#include "sm100.cuh"
 
 namespace fmms {
+
+// Launches `kern` with programmatic stream serialization: it may be scheduled
+// while the kernel ahead of it is finishing, and waits for that kernel with
+// grid_dependency_wait() before touching its results.
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_dependent(void (*kern)(KArgs...), dim3 grid, dim3 block,
+                                    cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
 
 // ---------------------------------------------------------------------------
 // Group merge: one warp per row; lanes stride over the groups.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(128) group_merge_kernel(const MergeParams m) {
+  sm100::grid_dependency_wait();  // the fused kernel's partials
   const int b = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
   const int lane = threadIdx.x & 31;
   if (b >= m.B) return;
@@ -113,6 +134,7 @@ __global__ void __launch_bounds__(128) group_merge_kernel(const MergeParams m) {
 __global__ void __launch_bounds__(128)
     merge_summaries_kernel(const fs_group_summary *summaries, int G, int B, uint64_t seed,
                            const uint64_t *row_seeds, uint32_t step, int32_t *out_idx) {
+  sm100::grid_dependency_wait();
   const int b = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
   const int lane = threadIdx.x & 31;
   if (b >= B) return;
@@ -150,16 +172,15 @@ cudaError_t launch_merge_summaries(const void *summaries, int G, int B, uint64_t
                                    cudaStream_t stream) {
   const int threads = 128;
   const int blocks = (B * 32 + threads - 1) / threads;
-  merge_summaries_kernel<<<blocks, threads, 0, stream>>>(
-      static_cast<const fs_group_summary *>(summaries), G, B, seed, row_seeds, step, out_idx);
-  return cudaGetLastError();
+  return launch_dependent(merge_summaries_kernel, dim3(blocks), dim3(threads), stream,
+                          static_cast<const fs_group_summary *>(summaries), G, B, seed, row_seeds,
+                          step, out_idx);
 }
 
 cudaError_t launch_group_merge(const MergeParams &m, cudaStream_t stream) {
   const int threads = 128;
   const int blocks = (m.B * 32 + threads - 1) / threads;
-  group_merge_kernel<<<blocks, threads, 0, stream>>>(m);
-  return cudaGetLastError();
+  return launch_dependent(group_merge_kernel, dim3(blocks), dim3(threads), stream, m);
 }
 
 // ---------------------------------------------------------------------------
@@ -169,6 +190,7 @@ cudaError_t launch_group_merge(const MergeParams &m, cudaStream_t stream) {
 // block decodes.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) sample_logits_kernel(const SampleLogitsParams s) {
+  sm100::grid_dependency_wait();  // the logits
   const int b = blockIdx.y;
   const uint32_t bg = static_cast<uint32_t>(s.b_off + b);
   const uint64_t k64 = s.row_seeds ? s.row_seeds[bg] : s.seed;
@@ -236,9 +258,7 @@ cudaError_t launch_sample_logits(const SampleLogitsParams &s, cudaStream_t strea
   const int target = (4 * s.num_sms + s.B - 1) / s.B;  // about four blocks per SM in total
   if (per_row > target) per_row = target;
   if (per_row < 1) per_row = 1;
-  dim3 grid(per_row, s.B);
-  sample_logits_kernel<<<grid, threads, 0, stream>>>(s);
-  return cudaGetLastError();
+  return launch_dependent(sample_logits_kernel, dim3(per_row, s.B), dim3(threads), stream, s);
 }
 
 // ---------------------------------------------------------------------------
@@ -323,6 +343,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_sample_kernel(const SampleL
   __shared__ int warp_sums[32];
   __shared__ int sh_digit, sh_above, sh_total;
   __shared__ uint64_t warp_best[32];
+  sm100::grid_dependency_wait();  // the logits
   const int b = blockIdx.x;
   const uint32_t bg = static_cast<uint32_t>(s.b_off + b);
   const float *row = s.logits + static_cast<size_t>(b) * s.V;
@@ -444,22 +465,22 @@ __global__ void __launch_bounds__(kTopkThreads) topk_sample_kernel(const SampleL
 }
 
 cudaError_t launch_topk_sample(const SampleLogitsParams &s, int K, cudaStream_t stream) {
-  topk_sample_kernel<<<s.B, kTopkThreads, 0, stream>>>(s, K);
-  return cudaGetLastError();
+  return launch_dependent(topk_sample_kernel, dim3(s.B), dim3(kTopkThreads), stream, s, K);
 }
 
 // ---------------------------------------------------------------------------
 // Vocabulary shards: tokens from the reduced keys.
 // ---------------------------------------------------------------------------
 __global__ void keys_to_tokens_kernel(const long long *keys, int B, int32_t *out_idx) {
+  sm100::grid_dependency_wait();  // the reduced keys
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b < B) out_idx[b] = key_token(static_cast<uint64_t>(keys[b]) ^ 0x8000000000000000ull);
 }
 
 cudaError_t launch_keys_to_tokens(const long long *keys, int B, int32_t *out_idx,
                                   cudaStream_t stream) {
-  keys_to_tokens_kernel<<<(B + 255) / 256, 256, 0, stream>>>(keys, B, out_idx);
-  return cudaGetLastError();
+  return launch_dependent(keys_to_tokens_kernel, dim3((B + 255) / 256), dim3(256), stream, keys, B,
+                          out_idx);
 }
 
 // ---------------------------------------------------------------------------

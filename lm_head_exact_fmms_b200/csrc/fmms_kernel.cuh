@@ -842,6 +842,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                   comb_key, comb_m, comb_s, warp, lane, unit, rank);
   }
 
+  // The group merge or the logits sampler that follows may start launching.
+  sm100::launch_dependents();
   sm100::tc_fence_before();
   __syncthreads();
   if constexpr (PAIR) {

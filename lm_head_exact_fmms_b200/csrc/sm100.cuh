@@ -327,6 +327,20 @@ __device__ __forceinline__ void mma_commit_pair(uint64_t *bar) {
                : "memory");
 }
 
+// Programmatic dependent launch: a kernel launched with the
+// programmatic-stream-serialization attribute may start before the kernel
+// ahead of it in the stream ends; grid_dependency_wait() returns once that
+// kernel has completed and its memory is visible.  launch_dependents() lets
+// such a dependent be scheduled once every CTA of this grid has issued it or
+// exited, so the dependent's launch overlaps this grid's last work.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Named barrier among the epilogue warps only.
 __device__ __forceinline__ void epi_sync(int nthreads) {
   asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
