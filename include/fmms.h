@@ -214,11 +214,15 @@ fs_status fs_keys_to_tokens(const int64_t *keys, int B, int32_t *out_idx,
  * candidates of row b are its K allowed tokens with the largest logits l
  * (ties toward the smaller index; every allowed token if there are fewer),
  * and the token is the argmax over them of x + g with the same noise as
- * fs_sample_ex, so K >= V gives the fs_sample_ex token.  Two kernels: the
- * matmul writes fp32 logits to `logits` (device [B][V], caller-owned, as in
- * fs_sample_unfused), then one block per row selects the K-th largest logit
- * exactly (radix select over the order-preserving bits) and samples.  K >= 1;
- * other arguments as fs_sample_ex. */
+ * fs_sample_ex, so K >= V gives the fs_sample_ex token.  The matmul writes
+ * fp32 logits to `logits` (device [B][V], caller-owned, as in
+ * fs_sample_unfused); then an exact radix select of the K-th largest logit
+ * (three histogram passes over the order-preserving bits, each row split over
+ * several blocks) and a candidate pass that samples.  The select's per-row
+ * histograms live in a library-owned device buffer (allocated on first use,
+ * a few MB, left zeroed by every call), so top-k calls on one device must not
+ * overlap on the GPU (order them on one stream).  K >= 1; other arguments as
+ * fs_sample_ex. */
 fs_status fs_sample_topk(const void *H, const void *W, int B, int d, int V,
                          int K, float temperature, uint64_t seed,
                          const uint64_t *row_seeds, uint32_t step,

@@ -29,6 +29,8 @@ struct DeviceState {
   size_t h_stage_bytes = 0;
   void *o_stage = nullptr;  // fs_sample_host: device tokens
   size_t o_stage_bytes = 0;
+  void *topk_scratch = nullptr;  // fs_sample_topk: per-row select histograms (left zeroed)
+  size_t topk_scratch_bytes = 0;
   // fs_sample_host: H is copied on copy_stream while the kernel already
   // streams W; h_flags takes the call's epoch once the copy has landed.
   // kernel_done keeps the next call's copy off h_stage until this call's
@@ -378,8 +380,15 @@ fs_status run_locked(int mode, const void *H, const void *W, int B, int d, int V
       sp.ticket = w.ticket;
       sp.out_idx = out_idx + b0;
       sp.num_sms = st->sms;
-      const cudaError_t e = shard.top_k > 0 ? fmms::launch_topk_sample(sp, shard.top_k, stream)
-                                            : fmms::launch_sample_logits(sp, stream);
+      cudaError_t e;
+      if (shard.top_k > 0) {
+        s = grow(&st->topk_scratch, &st->topk_scratch_bytes,
+                 fmms::topk_scratch_bytes(Bc, V, st->sms));
+        if (s != FS_OK) return s;
+        e = fmms::launch_topk_sample(sp, shard.top_k, st->topk_scratch, stream);
+      } else {
+        e = fmms::launch_sample_logits(sp, stream);
+      }
       if (e != cudaSuccess) return FS_ERR_CUDA;
     }
   }

@@ -264,20 +264,55 @@ cudaError_t launch_sample_logits(const SampleLogitsParams &s, cudaStream_t strea
 // ---------------------------------------------------------------------------
 // Top-k sampling over fp32 logits [B][V] (readus.org page, "Top-K and
 // masking": a prefilter isolates the candidates, exact Gumbel-max runs on
-// them).  One block per row: an exact radix select finds the k-th largest
-// order-preserving key of the allowed logits (passes over bits 31-21, 20-10,
-// 9-0), then the candidates -- keys above it, and as many keys equal to it as
-// k allows, in index order -- get their noise and the Gumbel-max.
+// them).  An exact radix select finds each row's k-th largest
+// order-preserving key among the allowed logits, over bits 31-21, 20-10 and
+// 9-0; the candidates -- keys above it, and as many keys equal to it as k
+// allows, in index order -- then get their noise and the Gumbel-max.  Each
+// row is split over P blocks (P x rows ~ two blocks per SM), one launch per
+// pass: three histogram passes into per-row global histograms, then the
+// candidate pass, whose last block per row writes the token and re-zeroes
+// the row's scratch.
 // ---------------------------------------------------------------------------
 constexpr int kTopkThreads = 1024;
+constexpr int kTopkItems = 8;      // consecutive elements per thread per iteration
 constexpr int kTopkBins = 2048;
-constexpr int kTopkItems = 8;     // consecutive elements per thread per iteration
-constexpr int kTopkSubHists = 4;  // warp-interleaved copies of the histogram
+constexpr int kTopkSubHists = 4;   // warp-interleaved copies of the shared histogram
+constexpr int kTopkMinSlice = kTopkThreads * kTopkItems;
 
-__device__ __forceinline__ bool topk_allowed(const SampleLogitsParams &s, uint32_t bg, int v) {
-  if (s.mask == nullptr) return true;
-  return ((s.mask[static_cast<size_t>(bg) * s.mask_words + (v >> 5)] >> (v & 31)) & 1u) != 0;
+// Per-launch scratch offsets for `rows` rows split over P blocks each.
+struct TopkLayout {
+  size_t hist0, hist1, hist2, hist2blk, rowkey, ticket, bytes;
+};
+static TopkLayout topk_layout(int rows, int P) {
+  TopkLayout l;
+  size_t o = 0;
+  l.hist0 = o;    o += static_cast<size_t>(rows) * kTopkBins * 4;
+  l.hist1 = o;    o += static_cast<size_t>(rows) * kTopkBins * 4;
+  l.hist2 = o;    o += static_cast<size_t>(rows) * 1024 * 4;
+  l.hist2blk = o; o += static_cast<size_t>(rows) * P * 1024 * 4;
+  l.rowkey = o;   o += static_cast<size_t>(rows) * 8;
+  l.ticket = o;   o += static_cast<size_t>(rows) * 4;
+  l.bytes = (o + 255) / 256 * 256;
+  return l;
 }
+
+static int topk_blocks_per_row(int rows, int V, int num_sms) {
+  const int want = (2 * num_sms + rows - 1) / rows;
+  const int most = (V + kTopkMinSlice - 1) / kTopkMinSlice;
+  return want < 1 ? 1 : (want > most ? most : want);
+}
+
+size_t topk_scratch_bytes(int rows, int V, int num_sms) {
+  return topk_layout(rows, topk_blocks_per_row(rows, V, num_sms)).bytes;
+}
+
+struct TopkArgs {
+  SampleLogitsParams s;
+  int K, P, slice;
+  int *hist0, *hist1, *hist2, *hist2blk;
+  unsigned long long *rowkey;
+  unsigned int *ticket;
+};
 
 // Block-wide exclusive scan of one int per thread (1024 threads); returns the
 // thread's prefix and writes the total to *total.
@@ -308,12 +343,50 @@ __device__ __forceinline__ int block_exclusive_scan(int x, int *warp_sums, int *
   return r;
 }
 
-// Loads this thread's kTopkItems consecutive logits starting at v0 and their
-// order-preserving keys; ok[i] is false past V or for a masked token.
+struct TopkShared {
+  int hist[kTopkSubHists * kTopkBins];
+  int warp_sums[32];
+  int digit, above, total;
+  unsigned long long warp_best[32];
+};
+
+// The digit of a global histogram row (nb = 2048 or 1024 bins) that holds the
+// k-th largest key (1-based): sets sh.digit and sh.above (keys in higher
+// bins).  With total_out, also the histogram's total.
+__device__ void topk_select_digit(const int *h, int nb, int k, TopkShared &sh, int *total_out) {
+  int c_hi, c_lo, hi_bin, lo_bin;
+  if (nb == kTopkBins) {
+    const int t = kTopkThreads - 1 - threadIdx.x;  // thread 0 holds the two top bins
+    hi_bin = 2 * t + 1;
+    lo_bin = 2 * t;
+    c_hi = __ldcg(h + hi_bin);
+    c_lo = __ldcg(h + lo_bin);
+  } else {
+    hi_bin = nb - 1 - threadIdx.x;
+    lo_bin = -1;
+    c_hi = __ldcg(h + hi_bin);
+    c_lo = 0;
+  }
+  const int above = block_exclusive_scan(c_hi + c_lo, sh.warp_sums, &sh.total);
+  if (total_out) *total_out = sh.total;
+  if (above < k && above + c_hi >= k) {
+    sh.digit = hi_bin;
+    sh.above = above;
+  } else if (lo_bin >= 0 && above + c_hi < k && above + c_hi + c_lo >= k) {
+    sh.digit = lo_bin;
+    sh.above = above + c_hi;
+  }
+  __syncthreads();
+}
+
+// Loads this thread's kTopkItems consecutive logits starting at v0 (below
+// hi) and their order-preserving keys; ok[i] is false past hi or for a
+// masked token.
 __device__ __forceinline__ void topk_load(const SampleLogitsParams &s, const float *row,
-                                          uint32_t bg, int v0, bool vec, float (&l)[kTopkItems],
-                                          uint32_t (&key)[kTopkItems], bool (&ok)[kTopkItems]) {
-  if (vec && v0 + kTopkItems <= s.V) {
+                                          uint32_t bg, int v0, int hi, bool vec,
+                                          float (&l)[kTopkItems], uint32_t (&key)[kTopkItems],
+                                          bool (&ok)[kTopkItems]) {
+  if (vec && v0 + kTopkItems <= hi) {
     const float4 a = *reinterpret_cast<const float4 *>(row + v0);
     const float4 c = *reinterpret_cast<const float4 *>(row + v0 + 4);
     l[0] = a.x; l[1] = a.y; l[2] = a.z; l[3] = a.w;
@@ -323,12 +396,12 @@ __device__ __forceinline__ void topk_load(const SampleLogitsParams &s, const flo
   } else {
 #pragma unroll
     for (int i = 0; i < kTopkItems; ++i) {
-      ok[i] = v0 + i < s.V;
+      ok[i] = v0 + i < hi;
       l[i] = ok[i] ? row[v0 + i] : 0.f;
     }
   }
   uint32_t mword = 0xFFFFFFFFu;
-  if (s.mask != nullptr && v0 < s.V)   // 8 consecutive tokens share one mask word
+  if (s.mask != nullptr && v0 < hi)   // 8 consecutive tokens from a multiple of 8 share one word
     mword = s.mask[static_cast<size_t>(bg) * s.mask_words + (v0 >> 5)];
 #pragma unroll
   for (int i = 0; i < kTopkItems; ++i) {
@@ -337,104 +410,124 @@ __device__ __forceinline__ void topk_load(const SampleLogitsParams &s, const flo
   }
 }
 
-__global__ void __launch_bounds__(kTopkThreads) topk_sample_kernel(const SampleLogitsParams s,
-                                                                   int K) {
-  __shared__ int hist[kTopkSubHists * kTopkBins];
-  __shared__ int warp_sums[32];
-  __shared__ int sh_digit, sh_above, sh_total;
-  __shared__ uint64_t warp_best[32];
-  sm100::grid_dependency_wait();  // the logits
-  const int b = blockIdx.x;
-  const uint32_t bg = static_cast<uint32_t>(s.b_off + b);
-  const float *row = s.logits + static_cast<size_t>(b) * s.V;
-  const int lane = threadIdx.x & 31;
-  const bool vec = (s.V & 3) == 0;
-  const int span = kTopkThreads * kTopkItems;
-  int *my_hist = hist + ((threadIdx.x >> 5) & (kTopkSubHists - 1)) * kTopkBins;
+// The selection state before pass `pass`: the key prefix found so far, its
+// mask, the rank still to find among keys matching it, and whether every
+// allowed token is a candidate (k >= allowed tokens).
+struct TopkState {
+  uint32_t prefix, pmask;
+  int k_rem;
+  bool all_allowed;
+};
 
-  // ---- radix select of the K-th largest key among allowed logits
-  uint32_t prefix = 0, pmask = 0;
-  int k_rem = K;   // rank still to find among keys matching the prefix
-  int n_allowed = 0;
+__device__ TopkState topk_state(const TopkArgs &a, int b, int passes, TopkShared &sh) {
+  TopkState st{0u, 0u, a.K, false};
   const int shifts[3] = {21, 10, 0};
   const int widths[3] = {11, 11, 10};
-  for (int pass = 0; pass < 3; ++pass) {
-    const int shift = shifts[pass];
-    const uint32_t dmask = (1u << widths[pass]) - 1u;
-    for (int i = threadIdx.x; i < kTopkSubHists * kTopkBins; i += kTopkThreads) hist[i] = 0;
-    __syncthreads();
-    for (int base = 0; base < s.V; base += span) {
-      float l[kTopkItems];
-      uint32_t key[kTopkItems];
-      bool ok[kTopkItems];
-      topk_load(s, row, bg, base + threadIdx.x * kTopkItems, vec, l, key, ok);
-#pragma unroll
-      for (int i = 0; i < kTopkItems; ++i)
-        if (ok[i] && (key[i] & pmask) == prefix) atomicAdd(&my_hist[(key[i] >> shift) & dmask], 1);
+  const int *hists[3] = {a.hist0, a.hist1, a.hist2};
+  for (int pass = 0; pass < passes; ++pass) {
+    const int nb = 1 << widths[pass];
+    int total = 0;
+    topk_select_digit(hists[pass] + static_cast<size_t>(b) * (pass < 2 ? kTopkBins : 1024), nb,
+                      st.k_rem, sh, pass == 0 ? &total : nullptr);
+    if (pass == 0 && total <= a.K) {
+      st.all_allowed = true;
+      return st;
     }
-    __syncthreads();
-    for (int i = threadIdx.x; i < kTopkBins; i += kTopkThreads) {   // fold the copies
-      int c = 0;
-#pragma unroll
-      for (int h = 0; h < kTopkSubHists; ++h) c += hist[h * kTopkBins + i];
-      hist[i] = c;
-    }
-    __syncthreads();
-    if (pass == 0) {
-      int c = 0;
-      for (int i = threadIdx.x; i < kTopkBins; i += kTopkThreads) c += hist[i];
-      block_exclusive_scan(c, warp_sums, &sh_total);
-      n_allowed = sh_total;
-      if (n_allowed <= K) break;   // every allowed token is a candidate
-    }
-    {
-      // suffix sums from the top bin: thread 0 holds bins 2047 and 2046
-      const int t = kTopkThreads - 1 - threadIdx.x;
-      const int hi_bin = 2 * t + 1, lo_bin = 2 * t;
-      const int c_hi = hist[hi_bin], c_lo = hist[lo_bin];
-      int total;
-      const int above = block_exclusive_scan(c_hi + c_lo, warp_sums, &total);
-      if (above < k_rem && above + c_hi >= k_rem) {
-        sh_digit = hi_bin;
-        sh_above = above;
-      } else if (above + c_hi < k_rem && above + c_hi + c_lo >= k_rem) {
-        sh_digit = lo_bin;
-        sh_above = above + c_hi;
-      }
-      __syncthreads();
-    }
-    prefix |= static_cast<uint32_t>(sh_digit) << shift;
-    pmask |= dmask << shift;
-    k_rem -= sh_above;
+    st.prefix |= static_cast<uint32_t>(sh.digit) << shifts[pass];
+    st.pmask |= static_cast<uint32_t>(nb - 1) << shifts[pass];
+    st.k_rem -= sh.above;
     __syncthreads();
   }
-  const bool all_allowed = n_allowed <= K;
-  // prefix is the K-th largest key; the first k_rem keys equal to it (in
-  // index order) are candidates, as is every larger key.
+  return st;
+}
 
-  // ---- candidates and Gumbel-max
+// Histogram pass `PASS` (0, 1, 2) of block (p, b) over its slice.
+template <int PASS>
+__global__ void __launch_bounds__(kTopkThreads) topk_hist_kernel(const TopkArgs a) {
+  __shared__ TopkShared sh;
+  sm100::grid_dependency_wait();  // the logits, or the previous pass's histograms
+  const int p = blockIdx.x, b = blockIdx.y;
+  const SampleLogitsParams &s = a.s;
+  const uint32_t bg = static_cast<uint32_t>(s.b_off + b);
+  const float *row = s.logits + static_cast<size_t>(b) * s.V;
+  const int lo = p * a.slice, hi = imin(s.V, lo + a.slice);
+  const bool vec = (s.V & 3) == 0;
+  const TopkState st = topk_state(a, b, PASS, sh);
+  if (st.all_allowed) return;
+  constexpr int kShift = PASS == 0 ? 21 : (PASS == 1 ? 10 : 0);
+  constexpr uint32_t kDMask = PASS == 2 ? 1023u : 2047u;
+  constexpr int kBins = PASS == 2 ? 1024 : kTopkBins;
+  for (int i = threadIdx.x; i < kTopkSubHists * kBins; i += kTopkThreads) sh.hist[i] = 0;
+  __syncthreads();
+  int *my_hist = sh.hist + ((threadIdx.x >> 5) & (kTopkSubHists - 1)) * kBins;
+  for (int base = lo; base < hi; base += kTopkThreads * kTopkItems) {
+    float l[kTopkItems];
+    uint32_t key[kTopkItems];
+    bool ok[kTopkItems];
+    topk_load(s, row, bg, base + threadIdx.x * kTopkItems, hi, vec, l, key, ok);
+#pragma unroll
+    for (int i = 0; i < kTopkItems; ++i)
+      if (ok[i] && (key[i] & st.pmask) == st.prefix)
+        atomicAdd(&my_hist[(key[i] >> kShift) & kDMask], 1);
+  }
+  __syncthreads();
+  int *gh = (PASS == 0 ? a.hist0 : PASS == 1 ? a.hist1 : a.hist2) +
+            static_cast<size_t>(b) * kBins;
+  for (int i = threadIdx.x; i < kBins; i += kTopkThreads) {
+    int c = 0;
+#pragma unroll
+    for (int h = 0; h < kTopkSubHists; ++h) c += sh.hist[h * kBins + i];
+    if (c) atomicAdd(gh + i, c);
+    if (PASS == 2) a.hist2blk[(static_cast<size_t>(b) * a.P + p) * 1024 + i] = c;
+  }
+}
+
+// Candidate pass of block (p, b): Gumbel-max over the slice's candidates; the
+// last block of the row writes its token and re-zeroes the row's scratch.
+__global__ void __launch_bounds__(kTopkThreads) topk_final_kernel(const TopkArgs a) {
+  __shared__ TopkShared sh;
+  __shared__ int last_block;
+  sm100::grid_dependency_wait();  // the histograms
+  const int p = blockIdx.x, b = blockIdx.y;
+  const SampleLogitsParams &s = a.s;
+  const uint32_t bg = static_cast<uint32_t>(s.b_off + b);
+  const float *row = s.logits + static_cast<size_t>(b) * s.V;
+  const int lo = p * a.slice, hi = imin(s.V, lo + a.slice);
+  const bool vec = (s.V & 3) == 0;
+  const int lane = threadIdx.x & 31;
+  const TopkState st = topk_state(a, b, 3, sh);
+  // Keys equal to the k-th largest: the first k_rem of them, in index order,
+  // are candidates; blocks before this one hold `before` of them.
+  int take = 0;
+  if (!st.all_allowed) {
+    const int digit = static_cast<int>(st.prefix & 1023u);
+    const int *hb = a.hist2blk + static_cast<size_t>(b) * a.P * 1024 + digit;
+    int before = 0;
+    for (int q = 0; q < p; ++q) before += __ldcg(hb + static_cast<size_t>(q) * 1024);
+    take = imin(imax(st.k_rem - before, 0), __ldcg(hb + static_cast<size_t>(p) * 1024));
+  }
   const uint64_t k64 = s.row_seeds ? s.row_seeds[bg] : s.seed;
   uint64_t best = 0ull;
   int eq_seen = 0;
-  for (int base = 0; base < s.V; base += span) {
+  for (int base = lo; base < hi; base += kTopkThreads * kTopkItems) {
     const int v0 = base + threadIdx.x * kTopkItems;
     float l[kTopkItems];
     uint32_t key[kTopkItems];
     bool ok[kTopkItems];
-    topk_load(s, row, bg, v0, vec, l, key, ok);
+    topk_load(s, row, bg, v0, hi, vec, l, key, ok);
     int n_eq_mine = 0;
 #pragma unroll
     for (int i = 0; i < kTopkItems; ++i)
-      n_eq_mine += (ok[i] && !all_allowed && key[i] == prefix) ? 1 : 0;
-    const int rank0 = eq_seen + block_exclusive_scan(n_eq_mine, warp_sums, &sh_total);
-    eq_seen += sh_total;
+      n_eq_mine += (ok[i] && !st.all_allowed && key[i] == st.prefix) ? 1 : 0;
+    const int rank0 = eq_seen + block_exclusive_scan(n_eq_mine, sh.warp_sums, &sh.total);
+    eq_seen += sh.total;
     int r = rank0;
 #pragma unroll
     for (int i = 0; i < kTopkItems; ++i) {
       if (!ok[i]) continue;
-      bool cand = all_allowed || key[i] > prefix;
-      if (!all_allowed && key[i] == prefix) {
-        cand = r < k_rem;
+      bool cand = st.all_allowed || key[i] > st.prefix;
+      if (!st.all_allowed && key[i] == st.prefix) {
+        cand = r < take;
         ++r;
       }
       if (cand) {
@@ -455,17 +548,56 @@ __global__ void __launch_bounds__(kTopkThreads) topk_sample_kernel(const SampleL
     const uint64_t o = __shfl_xor_sync(0xffffffffu, best, off);
     best = o > best ? o : best;
   }
-  if (lane == 0) warp_best[threadIdx.x >> 5] = best;
+  if (lane == 0) sh.warp_best[threadIdx.x >> 5] = best;
   __syncthreads();
   if (threadIdx.x == 0) {
     uint64_t r = 0ull;
-    for (int i = 0; i < kTopkThreads / 32; ++i) r = warp_best[i] > r ? warp_best[i] : r;
-    s.out_idx[b] = key_token(r);
+    for (int i = 0; i < kTopkThreads / 32; ++i) r = sh.warp_best[i] > r ? sh.warp_best[i] : r;
+    if (r) atomicMax(a.rowkey + b, static_cast<unsigned long long>(r));
+    __threadfence();
+    last_block = atomicAdd(a.ticket + b, 1u) == static_cast<unsigned>(a.P - 1);
+  }
+  __syncthreads();
+  if (last_block) {
+    __threadfence();
+    if (threadIdx.x == 0) {
+      const unsigned long long kb = atomicExch(a.rowkey + b, 0ull);
+      s.out_idx[b] = key_token(kb);
+      a.ticket[b] = 0u;
+    }
+    // every block of the row has read the histograms before taking its ticket
+    for (int i = threadIdx.x; i < kTopkBins; i += kTopkThreads) {
+      a.hist0[static_cast<size_t>(b) * kTopkBins + i] = 0;
+      a.hist1[static_cast<size_t>(b) * kTopkBins + i] = 0;
+    }
+    for (int i = threadIdx.x; i < 1024; i += kTopkThreads) a.hist2[static_cast<size_t>(b) * 1024 + i] = 0;
+    for (int i = threadIdx.x; i < a.P * 1024; i += kTopkThreads)
+      a.hist2blk[static_cast<size_t>(b) * a.P * 1024 + i] = 0;
   }
 }
 
-cudaError_t launch_topk_sample(const SampleLogitsParams &s, int K, cudaStream_t stream) {
-  return launch_dependent(topk_sample_kernel, dim3(s.B), dim3(kTopkThreads), stream, s, K);
+cudaError_t launch_topk_sample(const SampleLogitsParams &s, int K, void *scratch,
+                               cudaStream_t stream) {
+  const int P = topk_blocks_per_row(s.B, s.V, s.num_sms);
+  const TopkLayout lay = topk_layout(s.B, P);
+  char *base = static_cast<char *>(scratch);
+  TopkArgs a;
+  a.s = s;
+  a.K = K;
+  a.P = P;
+  a.slice = ((s.V + P - 1) / P + kTopkItems - 1) / kTopkItems * kTopkItems;
+  a.hist0 = reinterpret_cast<int *>(base + lay.hist0);
+  a.hist1 = reinterpret_cast<int *>(base + lay.hist1);
+  a.hist2 = reinterpret_cast<int *>(base + lay.hist2);
+  a.hist2blk = reinterpret_cast<int *>(base + lay.hist2blk);
+  a.rowkey = reinterpret_cast<unsigned long long *>(base + lay.rowkey);
+  a.ticket = reinterpret_cast<unsigned int *>(base + lay.ticket);
+  const dim3 grid(P, s.B), block(kTopkThreads);
+  cudaError_t e;
+  if ((e = launch_dependent(topk_hist_kernel<0>, grid, block, stream, a)) != cudaSuccess) return e;
+  if ((e = launch_dependent(topk_hist_kernel<1>, grid, block, stream, a)) != cudaSuccess) return e;
+  if ((e = launch_dependent(topk_hist_kernel<2>, grid, block, stream, a)) != cudaSuccess) return e;
+  return launch_dependent(topk_final_kernel, grid, block, stream, a);
 }
 
 // ---------------------------------------------------------------------------

@@ -71,8 +71,13 @@ struct SampleLogitsParams {
 };
 cudaError_t launch_sample_logits(const SampleLogitsParams &s, cudaStream_t stream);
 
-// Top-k sampling over the fp32 logits: one block per row.
-cudaError_t launch_topk_sample(const SampleLogitsParams &s, int K, cudaStream_t stream);
+// Top-k sampling over the fp32 logits: each row split over several blocks,
+// four launches (three radix-histogram passes, then the candidates).
+// `scratch` holds topk_scratch_bytes(s.B, s.V, s.num_sms) bytes, zero on
+// entry and left zero.
+size_t topk_scratch_bytes(int rows, int V, int num_sms);
+cudaError_t launch_topk_sample(const SampleLogitsParams &s, int K, void *scratch,
+                               cudaStream_t stream);
 
 // Group-Gumbel-Max over per-group summaries [G][B] (fs_group_summary records).
 cudaError_t launch_merge_summaries(const void *summaries, int G, int B, uint64_t seed,

@@ -525,7 +525,9 @@ def test_online_groups_match_fused_grouped(dev, oracle, B, V, G, masked):
 # --------------------------------------------------------------- top-k
 @pytest.mark.parametrize("B,d,V,K,masked", [(1, 64, 4096, 1, False), (7, 64, 3001, 5, True),
                                             (64, 128, 9000, 50, False), (33, 64, 1000, 1000, True),
-                                            (300, 32, 2048, 20, True), (4, 64, 700, 9999, False)])
+                                            (300, 32, 2048, 20, True), (4, 64, 700, 9999, False),
+                                            (1, 64, 100003, 50, True), (2, 64, 65536, 7, False),
+                                            (5, 32, 40000, 3000, True)])
 def test_topk_parity(dev, oracle, B, d, V, K, masked):
     H, W, Hd, Wd = rand_inputs(B, d, V, seed=K + V)
     mask = synth.make_mask(B, V, 0.6, seed=K) if masked else None
@@ -559,6 +561,30 @@ def test_topk_ties_at_the_boundary(dev, oracle):
         idx, best, second = oracle.sample_topk(H, W, K, T=1.0, seed=1, step=step)
         assert set(idx.tolist()) <= keep and set(got.tolist()) <= keep
         assert_parity(got, idx, best, second, "topk ties")
+
+
+def test_topk_ties_across_blocks(dev, oracle):
+    """Rows split over several select blocks (V = 65536, one block per 8192
+    tokens here): seven copies of the dominant W row sit in different
+    blocks, so the k-th place falls inside a tie that spans blocks and the
+    four smallest indices must be kept."""
+    B, d, V, K = 3, 64, 65536, 4
+    _, W, _, _ = rand_inputs(B, d, V, seed=15)
+    h = synth.make_hidden(1, d, seed=16)
+    H = h.repeat(B, 1).contiguous()
+    W = W.clone()
+    hf = h[0].float()
+    dom = (hf * 8.0 / (hf * hf).sum()).to(torch.bfloat16)
+    copies = [5, 9000, 9001, 20000, 40000, 50000, 65000]
+    for r in copies:
+        W[r] = dom
+    keep = set(copies[:K])
+    Hd, Wd = H.to(dev), W.to(dev)
+    for step in range(6):
+        got = binding.fs_sample_topk(Hd, Wd, K, temperature=1.0, seed=3, step=step).cpu().numpy()
+        idx, best, second = oracle.sample_topk(H, W, K, T=1.0, seed=3, step=step)
+        assert set(idx.tolist()) <= keep and set(got.tolist()) <= keep, (got, idx)
+        assert_parity(got, idx, best, second, "topk ties across blocks")
 
 
 def test_topk_full_vocab(dev, oracle):
