@@ -296,8 +296,10 @@ static TopkLayout topk_layout(int rows, int P) {
   return l;
 }
 
+// Blocks per row: as many as keep the grid within one wave of two
+// 1024-thread blocks per SM, each with at least kTopkMinSlice tokens.
 static int topk_blocks_per_row(int rows, int V, int num_sms) {
-  const int want = (2 * num_sms + rows - 1) / rows;
+  const int want = 2 * num_sms / rows;
   const int most = (V + kTopkMinSlice - 1) / kTopkMinSlice;
   return want < 1 ? 1 : (want > most ? most : want);
 }
@@ -498,14 +500,18 @@ __global__ void __launch_bounds__(kTopkThreads) topk_final_kernel(const TopkArgs
   const TopkState st = topk_state(a, b, 3, sh);
   // Keys equal to the k-th largest: the first k_rem of them, in index order,
   // are candidates; blocks before this one hold `before` of them.
-  int take = 0;
+  int take = 0, n_eq = 0;
   if (!st.all_allowed) {
     const int digit = static_cast<int>(st.prefix & 1023u);
     const int *hb = a.hist2blk + static_cast<size_t>(b) * a.P * 1024 + digit;
     int before = 0;
     for (int q = 0; q < p; ++q) before += __ldcg(hb + static_cast<size_t>(q) * 1024);
-    take = imin(imax(st.k_rem - before, 0), __ldcg(hb + static_cast<size_t>(p) * 1024));
+    n_eq = __ldcg(hb + static_cast<size_t>(p) * 1024);
+    take = imin(imax(st.k_rem - before, 0), n_eq);
   }
+  // Ranking the equal keys in index order is needed only when some but not
+  // all of this slice's equal keys are candidates (block-uniform).
+  const bool rank_ties = take > 0 && take < n_eq;
   const uint64_t k64 = s.row_seeds ? s.row_seeds[bg] : s.seed;
   uint64_t best = 0ull;
   int eq_seen = 0;
@@ -515,19 +521,20 @@ __global__ void __launch_bounds__(kTopkThreads) topk_final_kernel(const TopkArgs
     uint32_t key[kTopkItems];
     bool ok[kTopkItems];
     topk_load(s, row, bg, v0, hi, vec, l, key, ok);
-    int n_eq_mine = 0;
+    int r = 0;
+    if (rank_ties) {
+      int n_eq_mine = 0;
 #pragma unroll
-    for (int i = 0; i < kTopkItems; ++i)
-      n_eq_mine += (ok[i] && !st.all_allowed && key[i] == st.prefix) ? 1 : 0;
-    const int rank0 = eq_seen + block_exclusive_scan(n_eq_mine, sh.warp_sums, &sh.total);
-    eq_seen += sh.total;
-    int r = rank0;
+      for (int i = 0; i < kTopkItems; ++i) n_eq_mine += (ok[i] && key[i] == st.prefix) ? 1 : 0;
+      r = eq_seen + block_exclusive_scan(n_eq_mine, sh.warp_sums, &sh.total);
+      eq_seen += sh.total;
+    }
 #pragma unroll
     for (int i = 0; i < kTopkItems; ++i) {
       if (!ok[i]) continue;
       bool cand = st.all_allowed || key[i] > st.prefix;
       if (!st.all_allowed && key[i] == st.prefix) {
-        cand = r < take;
+        cand = rank_ties ? r < take : take > 0;
         ++r;
       }
       if (cand) {
