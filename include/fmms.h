@@ -237,7 +237,8 @@ fs_status fs_sample_topk(const void *H, const void *W, int B, int d, int V,
  * library stream (after the previous fs_sample_host call's kernel, which
  * reads that buffer), the fused sample on `stream` (it starts streaming W at
  * once and waits on the device, with the usual one-second limit, for the
- * copy of H to land), and the device-to-host copy of the tokens on
+ * copy of H to land), and the tokens: written by the kernel straight into
+ * out_idx_host when it is page-locked, else copied from a device buffer on
  * `stream`; the tokens are valid once `stream` is synchronised.  H_host must
  * stay unchanged until then.  Without stream memory operations on the
  * device, the copy of H runs on `stream` before the sample. */

@@ -499,12 +499,20 @@ fs_status fs_sample_host(const void *H_host, const void *W, int B, int d, int V,
     if (cudaMemcpyAsync(hdev, H_host, hbytes, cudaMemcpyHostToDevice, st_) != cudaSuccess)
       return FS_ERR_CUDA;
   }
+  // Page-locked token buffer: the kernel's last CTA stores the tokens into it
+  // directly over PCIe (no separate device-to-host copy); otherwise they go
+  // through the device staging buffer and a copy.
+  cudaPointerAttributes pa;
+  const bool direct = cudaPointerGetAttributes(&pa, out_idx_host) == cudaSuccess &&
+                      pa.type == cudaMemoryTypeHost && pa.devicePointer != nullptr;
+  if (!direct) cudaGetLastError();  // clear a lookup error on pageable memory
+  int32_t *out_dev = direct ? static_cast<int32_t *>(pa.devicePointer) : odev;
   s = run_locked(fmms::kModeFlat, hdev, W, B, d, V, 1, temperature, seed, row_seeds, step,
-                 mask_bits, odev, nullptr, nullptr, nullptr, 0, st_, opts);
+                 mask_bits, out_dev, nullptr, nullptr, nullptr, 0, st_, opts);
   if (s != FS_OK) return s;
   if (st->host_overlap && cudaEventRecord(st->kernel_done, st_) != cudaSuccess) return FS_ERR_CUDA;
-  if (cudaMemcpyAsync(out_idx_host, odev, static_cast<size_t>(B) * 4, cudaMemcpyDeviceToHost,
-                      st_) != cudaSuccess)
+  if (!direct && cudaMemcpyAsync(out_idx_host, odev, static_cast<size_t>(B) * 4,
+                                 cudaMemcpyDeviceToHost, st_) != cudaSuccess)
     return FS_ERR_CUDA;
   return FS_OK;
 }

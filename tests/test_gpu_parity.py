@@ -215,11 +215,12 @@ def test_host_entry_point(dev):
 
 
 def test_host_entry_point_back_to_back(dev):
-    """fs_sample_host copies H in K-column chunks on a copy stream while the
-    kernel already streams W.  Calls issued back to back with different host
-    H (no synchronisation in between), including a 300-row call (two
-    launches) and d not a multiple of the chunk size, must each give the
-    tokens of the device entry point on the same H."""
+    """fs_sample_host copies H on a copy stream while the kernel already
+    streams W, and the kernel writes the tokens straight into a page-locked
+    out buffer.  Calls issued back to back with different host H (no
+    synchronisation in between), including a 300-row call (two launches),
+    must each give the tokens of the device entry point on the same H; so
+    must a call with pageable buffers, which takes the copy path."""
     d, V = 200, 7001
     W = synth.make_weight(V, d, 1.0 / np.sqrt(d), device="cpu", seed=71).to(dev)
     calls = []
@@ -232,6 +233,13 @@ def test_host_entry_point_back_to_back(dev):
     for H, out, i in calls:
         ref = binding.fs_sample_ex(H.to(dev), W, temperature=0.8, seed=5, step=i).cpu()
         assert torch.equal(out, ref), i
+    # pageable (not page-locked) host buffers take the copy path
+    H = synth.make_hidden(24, d, device="cpu", seed=99)
+    out = torch.empty(24, dtype=torch.int32)
+    binding.fs_sample_host(H, W, temperature=0.8, seed=5, step=9, out_idx_host=out)
+    torch.cuda.synchronize()
+    ref = binding.fs_sample_ex(H.to(dev), W, temperature=0.8, seed=5, step=9).cpu()
+    assert torch.equal(out, ref)
 
 
 def test_gumbel_max_is_softmax_on_gpu(dev, oracle):
