@@ -261,6 +261,12 @@ def median(xs):
     return s[len(s) // 2]
 
 
+def percentiles(xs, qs=(10, 50, 90)):
+    """Nearest-rank percentiles of the per-call kernel times."""
+    s = sorted(xs)
+    return [s[min(len(s) - 1, max(0, (q * len(s) + 99) // 100 - 1))] for q in qs]
+
+
 def cpu_baseline(H, W, wl, B, rs, budget_s=12.0, max_rows=64):
     """The oracle as it stands, on this host's cores, over a bounded sample of
     the workload's rows; scaled to us per B-row call."""
@@ -420,7 +426,9 @@ def sweep(torch, binding, synth, W, wl, dev, stream, peaks, peak_kind, steps=200
         rf = roofline(B, wl.d, wl.V, False, kus, peaks, peak_kind,
                       committed_traffic("%s/B%d" % (wl.name, B)))
         row = {"B": B, "us_per_call": round(region_ms * 1e3 / steps, 3),
-               "kernel_us": round(kus, 3), "bound": rf["bound"],
+               "kernel_us": round(kus, 3),
+               "kernel_us_p10_p50_p90": [round(x, 3) for x in percentiles(per)],
+               "bound": rf["bound"],
                "achieved": round(rf["achieved"], 1), "unit": rf["unit"],
                "frac": round(rf["frac"], 4),
                # the library's automatic choice: CTA pairs above 64 rows per launch
