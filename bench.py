@@ -527,8 +527,8 @@ def graph_point(torch, binding, synth, W, wl, dev, B, calls=10, replays=30):
 
 
 def topk_point(torch, binding, synth, W, wl, dev, stream, B, K=50, steps=100):
-    """Top-k sampling: the fused kernel writes fp32 logits to HBM, then three
-    radix-histogram launches and a final select launch sample each row."""
+    """Top-k sampling: the fused kernel writes fp32 logits to HBM, then a
+    per-block candidate launch and a per-row select launch sample each row."""
     H = synth.make_hidden(B, wl.d, device=dev)
     rs = synth.make_row_seeds(B, device=dev) if wl.per_row_seeds else None
     out = torch.empty(B, dtype=torch.int32, device=dev)
@@ -540,7 +540,7 @@ def topk_point(torch, binding, synth, W, wl, dev, stream, B, K=50, steps=100):
 
     region_ms, _ = time_calls(step, steps, 10, stream)
     return {"B": B, "K": K, "us_per_call": round(region_ms * 1e3 / steps, 3),
-            "launches_per_call": (B + 255) // 256 + 4}
+            "launches_per_call": 3 * ((B + 255) // 256)}
 
 
 def unfused_point(torch, binding, synth, W, wl, dev, stream, B, steps=100):

@@ -216,13 +216,16 @@ fs_status fs_keys_to_tokens(const int64_t *keys, int B, int32_t *out_idx,
  * and the token is the argmax over them of x + g with the same noise as
  * fs_sample_ex, so K >= V gives the fs_sample_ex token.  The matmul writes
  * fp32 logits to `logits` (device [B][V], caller-owned, as in
- * fs_sample_unfused); then an exact radix select of the K-th largest logit
- * (three histogram passes over the order-preserving bits, each row split over
- * several blocks) and a candidate pass that samples.  The select's per-row
- * histograms live in a library-owned device buffer (allocated on first use,
- * a few MB, left zeroed by every call), so top-k calls on one device must not
- * overlap on the GPU (order them on one stream).  K >= 1; other arguments as
- * fs_sample_ex. */
+ * fs_sample_unfused); then two launches: every row is split over several
+ * blocks, each of which narrows its slice to a candidate list by radix
+ * histograms over the order-preserving bits (the lists together hold the
+ * row's top K), and one block per row selects the exact top K from the
+ * lists and samples.  The lists live in a library-owned device buffer
+ * (allocated on first use and grown as needed: 8 x rows x P x
+ * min(max(K, 2048), V / P) bytes for P blocks per row, 4 MB at 64 rows and
+ * K <= 2048, at most about 8 x rows x V bytes), so top-k
+ * calls on one device must not overlap on the GPU (order them on one
+ * stream).  K >= 1; other arguments as fs_sample_ex. */
 fs_status fs_sample_topk(const void *H, const void *W, int B, int d, int V,
                          int K, float temperature, uint64_t seed,
                          const uint64_t *row_seeds, uint32_t step,

@@ -29,7 +29,7 @@ struct DeviceState {
   size_t h_stage_bytes = 0;
   void *o_stage = nullptr;  // fs_sample_host: device tokens
   size_t o_stage_bytes = 0;
-  void *topk_scratch = nullptr;  // fs_sample_topk: per-row select histograms (left zeroed)
+  void *topk_scratch = nullptr;  // fs_sample_topk: per-block candidate lists and counts
   size_t topk_scratch_bytes = 0;
   // fs_sample_host: H is copied on copy_stream while the kernel already
   // streams W; h_flags takes the call's epoch once the copy has landed.
@@ -383,7 +383,7 @@ fs_status run_locked(int mode, const void *H, const void *W, int B, int d, int V
       cudaError_t e;
       if (shard.top_k > 0) {
         s = grow(&st->topk_scratch, &st->topk_scratch_bytes,
-                 fmms::topk_scratch_bytes(Bc, V, st->sms));
+                 fmms::topk_scratch_bytes(Bc, V, shard.top_k, st->sms));
         if (s != FS_OK) return s;
         e = fmms::launch_topk_sample(sp, shard.top_k, st->topk_scratch, stream);
       } else {

@@ -20,12 +20,12 @@ namespace fmms {
 // while the kernel ahead of it is finishing, and waits for that kernel with
 // grid_dependency_wait() before touching its results.
 template <typename... KArgs, typename... Args>
-static cudaError_t launch_dependent(void (*kern)(KArgs...), dim3 grid, dim3 block,
-                                    cudaStream_t stream, Args... args) {
+static cudaError_t launch_dependent_smem(void (*kern)(KArgs...), dim3 grid, dim3 block,
+                                         size_t smem, cudaStream_t stream, Args... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -33,6 +33,12 @@ static cudaError_t launch_dependent(void (*kern)(KArgs...), dim3 grid, dim3 bloc
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_dependent(void (*kern)(KArgs...), dim3 grid, dim3 block,
+                                    cudaStream_t stream, Args... args) {
+  return launch_dependent_smem(kern, grid, block, 0, stream, args...);
 }
 
 // ---------------------------------------------------------------------------
@@ -264,60 +270,66 @@ cudaError_t launch_sample_logits(const SampleLogitsParams &s, cudaStream_t strea
 // ---------------------------------------------------------------------------
 // Top-k sampling over fp32 logits [B][V] (readus.org page, "Top-K and
 // masking": a prefilter isolates the candidates, exact Gumbel-max runs on
-// them).  An exact radix select finds each row's k-th largest
-// order-preserving key among the allowed logits, over bits 31-21, 20-10 and
-// 9-0; the candidates -- keys above it, and as many keys equal to it as k
-// allows, in index order -- then get their noise and the Gumbel-max.  Each
-// row is split over P blocks (P x rows ~ two blocks per SM), one launch per
-// pass: three histogram passes into per-row global histograms, then the
-// candidate pass, whose last block per row writes the token and re-zeroes
-// the row's scratch.
+// them).  The candidates of a row are its K allowed tokens with the largest
+// logits, ties toward the smaller index.  Two launches:
+//   1. topk_local_kernel: each row is split over P blocks (P x rows at most
+//      one block per SM, so the grid is one wave).  A block finds, with shared-memory radix histograms
+//      over the order-preserving bits of its slice's keys (bits 31-21, then
+//      20-10 and 9-0 only while the candidate set exceeds its capacity), a
+//      key threshold with at least min(K, allowed) of its keys at or above
+//      it, and writes those (key, token) pairs in token order to its
+//      candidate list.  The row's K-th largest key is at least every block's
+//      local K-th largest, so the union of the lists holds the row's top K,
+//      and every token tied with the row's K-th key.
+//   2. topk_row_kernel: one block per row selects the exact K-th largest key
+//      among the row's candidates (the same radix passes), keeps the tied
+//      keys in token order as K allows, draws the noise of the selected
+//      tokens and writes the Gumbel-max token.
+// Nothing carries over between calls: the candidate counts are written, not
+// accumulated.
 // ---------------------------------------------------------------------------
 constexpr int kTopkThreads = 1024;
 constexpr int kTopkItems = 8;      // consecutive elements per thread per iteration
 constexpr int kTopkBins = 2048;
 constexpr int kTopkSubHists = 4;   // warp-interleaved copies of the shared histogram
 constexpr int kTopkMinSlice = kTopkThreads * kTopkItems;
+constexpr int kTopkMinCap = 2048;  // candidate capacity per block, at least K
+constexpr int kTopkMaxP = 512;
+constexpr int kTopkRowCap = 8192;  // candidates a row's select block keeps in shared memory
 
-// Per-launch scratch offsets for `rows` rows split over P blocks each.
-struct TopkLayout {
-  size_t hist0, hist1, hist2, hist2blk, rowkey, ticket, bytes;
+struct TopkGeom {
+  int P, slice, cap;
 };
-static TopkLayout topk_layout(int rows, int P) {
-  TopkLayout l;
-  size_t o = 0;
-  l.hist0 = o;    o += static_cast<size_t>(rows) * kTopkBins * 4;
-  l.hist1 = o;    o += static_cast<size_t>(rows) * kTopkBins * 4;
-  l.hist2 = o;    o += static_cast<size_t>(rows) * 1024 * 4;
-  l.hist2blk = o; o += static_cast<size_t>(rows) * P * 1024 * 4;
-  l.rowkey = o;   o += static_cast<size_t>(rows) * 8;
-  l.ticket = o;   o += static_cast<size_t>(rows) * 4;
-  l.bytes = (o + 255) / 256 * 256;
-  return l;
-}
-
-// Blocks per row: as many as keep the grid within one wave of two
-// 1024-thread blocks per SM, each with at least kTopkMinSlice tokens.
-static int topk_blocks_per_row(int rows, int V, int num_sms) {
-  const int want = 2 * num_sms / rows;
+static TopkGeom topk_geom(int rows, int V, int K, int num_sms) {
+  TopkGeom g;
+  const int want = num_sms / rows;  // one wave: a 1024-thread block fills an SM's registers
   const int most = (V + kTopkMinSlice - 1) / kTopkMinSlice;
-  return want < 1 ? 1 : (want > most ? most : want);
+  g.P = want < 1 ? 1 : (want > most ? most : want);
+  if (g.P > kTopkMaxP) g.P = kTopkMaxP;
+  g.slice = ((V + g.P - 1) / g.P + kTopkItems - 1) / kTopkItems * kTopkItems;
+  g.cap = K > kTopkMinCap ? K : kTopkMinCap;
+  if (g.cap > g.slice) g.cap = g.slice;
+  return g;
 }
 
-size_t topk_scratch_bytes(int rows, int V, int num_sms) {
-  return topk_layout(rows, topk_blocks_per_row(rows, V, num_sms)).bytes;
+size_t topk_scratch_bytes(int rows, int V, int K, int num_sms) {
+  const TopkGeom g = topk_geom(rows, V, K, num_sms);
+  const size_t lists = static_cast<size_t>(rows) * g.P * g.cap * 8;
+  const size_t counts = static_cast<size_t>(rows) * g.P * 8;  // lengths and thresholds
+  return (lists + counts + 255) / 256 * 256;
 }
 
 struct TopkArgs {
   SampleLogitsParams s;
-  int K, P, slice;
-  int *hist0, *hist1, *hist2, *hist2blk;
-  unsigned long long *rowkey;
-  unsigned int *ticket;
+  int K, P, slice, cap;
+  unsigned long long *cand;  // [rows][P][cap]: (key << 32) | token
+  int *cnt;                  // [rows][P]: list lengths
+  unsigned int *thr;         // [rows][P]: each block's key threshold (0: every allowed key)
 };
 
 // Block-wide exclusive scan of one int per thread (1024 threads); returns the
-// thread's prefix and writes the total to *total.
+// thread's prefix and writes the total to *total, which must be in shared
+// memory (one thread writes it, every thread may read it after the call).
 __device__ __forceinline__ int block_exclusive_scan(int x, int *warp_sums, int *total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int incl = x;
@@ -352,33 +364,44 @@ struct TopkShared {
   unsigned long long warp_best[32];
 };
 
-// The digit of a global histogram row (nb = 2048 or 1024 bins) that holds the
-// k-th largest key (1-based): sets sh.digit and sh.above (keys in higher
-// bins).  With total_out, also the histogram's total.
-__device__ void topk_select_digit(const int *h, int nb, int k, TopkShared &sh, int *total_out) {
+// The digit of a shared histogram (nb = 2048 or 1024 bins, in sh.hist) that
+// holds the k-th largest key (1-based): returns it and its count, and sets
+// *above to the keys in higher bins.  *total gets the histogram's total; when
+// it is below k the digit is 0 and the other results are meaningless.
+__device__ int topk_select_digit(int nb, int k, TopkShared &sh, int *above, int *count,
+                                 int *total) {
+  if (threadIdx.x == 0) {  // ordered before the writes below by the scan's barriers
+    sh.digit = 0;
+    sh.above = 0;
+  }
   int c_hi, c_lo, hi_bin, lo_bin;
   if (nb == kTopkBins) {
     const int t = kTopkThreads - 1 - threadIdx.x;  // thread 0 holds the two top bins
     hi_bin = 2 * t + 1;
     lo_bin = 2 * t;
-    c_hi = __ldcg(h + hi_bin);
-    c_lo = __ldcg(h + lo_bin);
+    c_hi = sh.hist[hi_bin];
+    c_lo = sh.hist[lo_bin];
   } else {
     hi_bin = nb - 1 - threadIdx.x;
     lo_bin = -1;
-    c_hi = __ldcg(h + hi_bin);
+    c_hi = sh.hist[hi_bin];
     c_lo = 0;
   }
-  const int above = block_exclusive_scan(c_hi + c_lo, sh.warp_sums, &sh.total);
-  if (total_out) *total_out = sh.total;
-  if (above < k && above + c_hi >= k) {
+  const int ab = block_exclusive_scan(c_hi + c_lo, sh.warp_sums, &sh.total);
+  if (ab < k && ab + c_hi >= k) {
     sh.digit = hi_bin;
-    sh.above = above;
-  } else if (lo_bin >= 0 && above + c_hi < k && above + c_hi + c_lo >= k) {
+    sh.above = ab;
+  } else if (lo_bin >= 0 && ab + c_hi < k && ab + c_hi + c_lo >= k) {
     sh.digit = lo_bin;
-    sh.above = above + c_hi;
+    sh.above = ab + c_hi;
   }
   __syncthreads();
+  const int d = sh.digit;
+  *above = sh.above;
+  *count = sh.hist[d];
+  *total = sh.total;
+  __syncthreads();  // the caller may rebuild sh.hist next
+  return d;
 }
 
 // Loads this thread's kTopkItems consecutive logits starting at v0 (below
@@ -386,8 +409,8 @@ __device__ void topk_select_digit(const int *h, int nb, int k, TopkShared &sh, i
 // masked token.
 __device__ __forceinline__ void topk_load(const SampleLogitsParams &s, const float *row,
                                           uint32_t bg, int v0, int hi, bool vec,
-                                          float (&l)[kTopkItems], uint32_t (&key)[kTopkItems],
-                                          bool (&ok)[kTopkItems]) {
+                                          uint32_t (&key)[kTopkItems], bool (&ok)[kTopkItems]) {
+  float l[kTopkItems];
   if (vec && v0 + kTopkItems <= hi) {
     const float4 a = *reinterpret_cast<const float4 *>(row + v0);
     const float4 c = *reinterpret_cast<const float4 *>(row + v0 + 4);
@@ -412,201 +435,384 @@ __device__ __forceinline__ void topk_load(const SampleLogitsParams &s, const flo
   }
 }
 
-// The selection state before pass `pass`: the key prefix found so far, its
-// mask, the rank still to find among keys matching it, and whether every
-// allowed token is a candidate (k >= allowed tokens).
-struct TopkState {
-  uint32_t prefix, pmask;
-  int k_rem;
-  bool all_allowed;
-};
-
-__device__ TopkState topk_state(const TopkArgs &a, int b, int passes, TopkShared &sh) {
-  TopkState st{0u, 0u, a.K, false};
-  const int shifts[3] = {21, 10, 0};
-  const int widths[3] = {11, 11, 10};
-  const int *hists[3] = {a.hist0, a.hist1, a.hist2};
-  for (int pass = 0; pass < passes; ++pass) {
-    const int nb = 1 << widths[pass];
-    int total = 0;
-    topk_select_digit(hists[pass] + static_cast<size_t>(b) * (pass < 2 ? kTopkBins : 1024), nb,
-                      st.k_rem, sh, pass == 0 ? &total : nullptr);
-    if (pass == 0 && total <= a.K) {
-      st.all_allowed = true;
-      return st;
-    }
-    st.prefix |= static_cast<uint32_t>(sh.digit) << shifts[pass];
-    st.pmask |= static_cast<uint32_t>(nb - 1) << shifts[pass];
-    st.k_rem -= sh.above;
-    __syncthreads();
-  }
-  return st;
-}
-
-// Histogram pass `PASS` (0, 1, 2) of block (p, b) over its slice.
-template <int PASS>
-__global__ void __launch_bounds__(kTopkThreads) topk_hist_kernel(const TopkArgs a) {
-  __shared__ TopkShared sh;
-  sm100::grid_dependency_wait();  // the logits, or the previous pass's histograms
-  const int p = blockIdx.x, b = blockIdx.y;
-  const SampleLogitsParams &s = a.s;
-  const uint32_t bg = static_cast<uint32_t>(s.b_off + b);
-  const float *row = s.logits + static_cast<size_t>(b) * s.V;
-  const int lo = p * a.slice, hi = imin(s.V, lo + a.slice);
-  const bool vec = (s.V & 3) == 0;
-  const TopkState st = topk_state(a, b, PASS, sh);
-  if (st.all_allowed) return;
-  constexpr int kShift = PASS == 0 ? 21 : (PASS == 1 ? 10 : 0);
-  constexpr uint32_t kDMask = PASS == 2 ? 1023u : 2047u;
-  constexpr int kBins = PASS == 2 ? 1024 : kTopkBins;
-  for (int i = threadIdx.x; i < kTopkSubHists * kBins; i += kTopkThreads) sh.hist[i] = 0;
+// Histogram, in sh.hist[0, nb), of digit (key >> shift) & (nb - 1) over the
+// allowed keys of [lo, hi) with (key & pmask) == prefix.
+__device__ void topk_slice_hist(const SampleLogitsParams &s, const float *row, uint32_t bg,
+                                int lo, int hi, bool vec, uint32_t prefix, uint32_t pmask,
+                                int shift, int nb, TopkShared &sh) {
+  for (int i = threadIdx.x; i < kTopkSubHists * nb; i += kTopkThreads) sh.hist[i] = 0;
   __syncthreads();
-  int *my_hist = sh.hist + ((threadIdx.x >> 5) & (kTopkSubHists - 1)) * kBins;
+  int *my_hist = sh.hist + ((threadIdx.x >> 5) & (kTopkSubHists - 1)) * nb;
+  const uint32_t dmask = static_cast<uint32_t>(nb - 1);
   for (int base = lo; base < hi; base += kTopkThreads * kTopkItems) {
-    float l[kTopkItems];
     uint32_t key[kTopkItems];
     bool ok[kTopkItems];
-    topk_load(s, row, bg, base + threadIdx.x * kTopkItems, hi, vec, l, key, ok);
+    topk_load(s, row, bg, base + threadIdx.x * kTopkItems, hi, vec, key, ok);
 #pragma unroll
     for (int i = 0; i < kTopkItems; ++i)
-      if (ok[i] && (key[i] & st.pmask) == st.prefix)
-        atomicAdd(&my_hist[(key[i] >> kShift) & kDMask], 1);
+      if (ok[i] && (key[i] & pmask) == prefix) atomicAdd(&my_hist[(key[i] >> shift) & dmask], 1);
   }
   __syncthreads();
-  int *gh = (PASS == 0 ? a.hist0 : PASS == 1 ? a.hist1 : a.hist2) +
-            static_cast<size_t>(b) * kBins;
-  for (int i = threadIdx.x; i < kBins; i += kTopkThreads) {
+  for (int i = threadIdx.x; i < nb; i += kTopkThreads) {
     int c = 0;
 #pragma unroll
-    for (int h = 0; h < kTopkSubHists; ++h) c += sh.hist[h * kBins + i];
-    if (c) atomicAdd(gh + i, c);
-    if (PASS == 2) a.hist2blk[(static_cast<size_t>(b) * a.P + p) * 1024 + i] = c;
+    for (int h = 0; h < kTopkSubHists; ++h) c += sh.hist[h * nb + i];
+    sh.hist[i] = c;  // thread i alone reads and writes bin i of every copy
   }
+  __syncthreads();
 }
 
-// Candidate pass of block (p, b): Gumbel-max over the slice's candidates; the
-// last block of the row writes its token and re-zeroes the row's scratch.
-__global__ void __launch_bounds__(kTopkThreads) topk_final_kernel(const TopkArgs a) {
-  __shared__ TopkShared sh;
-  __shared__ int last_block;
-  sm100::grid_dependency_wait();  // the histograms
-  const int p = blockIdx.x, b = blockIdx.y;
-  const SampleLogitsParams &s = a.s;
-  const uint32_t bg = static_cast<uint32_t>(s.b_off + b);
-  const float *row = s.logits + static_cast<size_t>(b) * s.V;
-  const int lo = p * a.slice, hi = imin(s.V, lo + a.slice);
-  const bool vec = (s.V & 3) == 0;
+// Appends the allowed keys of [lo, hi) that pass the threshold -- keys >=
+// lo_key, or in exact mode keys > lo_key and the first `take` keys equal to
+// it in token order -- to `out` (capacity cap; *n_out counts every passing
+// key, stored or not) and counts the allowed keys into *n_ok.
+__device__ void topk_extract(const SampleLogitsParams &s, const float *row, uint32_t bg, int lo,
+                             int hi, bool vec, uint32_t lo_key, bool exact, int take,
+                             unsigned long long *out, int cap, int *n_out, int *n_ok,
+                             TopkShared &sh) {
   const int lane = threadIdx.x & 31;
-  const TopkState st = topk_state(a, b, 3, sh);
-  // Keys equal to the k-th largest: the first k_rem of them, in index order,
-  // are candidates; blocks before this one hold `before` of them.
-  int take = 0, n_eq = 0;
-  if (!st.all_allowed) {
-    const int digit = static_cast<int>(st.prefix & 1023u);
-    const int *hb = a.hist2blk + static_cast<size_t>(b) * a.P * 1024 + digit;
-    int before = 0;
-    for (int q = 0; q < p; ++q) before += __ldcg(hb + static_cast<size_t>(q) * 1024);
-    n_eq = __ldcg(hb + static_cast<size_t>(p) * 1024);
-    take = imin(imax(st.k_rem - before, 0), n_eq);
-  }
-  // Ranking the equal keys in index order is needed only when some but not
-  // all of this slice's equal keys are candidates (block-uniform).
-  const bool rank_ties = take > 0 && take < n_eq;
-  const uint64_t k64 = s.row_seeds ? s.row_seeds[bg] : s.seed;
-  uint64_t best = 0ull;
-  int eq_seen = 0;
+  int eq_seen = 0, ok_mine = 0;
   for (int base = lo; base < hi; base += kTopkThreads * kTopkItems) {
     const int v0 = base + threadIdx.x * kTopkItems;
-    float l[kTopkItems];
     uint32_t key[kTopkItems];
     bool ok[kTopkItems];
-    topk_load(s, row, bg, v0, hi, vec, l, key, ok);
+    topk_load(s, row, bg, v0, hi, vec, key, ok);
     int r = 0;
-    if (rank_ties) {
-      int n_eq_mine = 0;
+    if (exact) {  // block-uniform: rank the tied keys in token order
+      int n_eq = 0;
 #pragma unroll
-      for (int i = 0; i < kTopkItems; ++i) n_eq_mine += (ok[i] && key[i] == st.prefix) ? 1 : 0;
-      r = eq_seen + block_exclusive_scan(n_eq_mine, sh.warp_sums, &sh.total);
+      for (int i = 0; i < kTopkItems; ++i) n_eq += (ok[i] && key[i] == lo_key) ? 1 : 0;
+      r = eq_seen + block_exclusive_scan(n_eq, sh.warp_sums, &sh.total);
       eq_seen += sh.total;
     }
+    uint32_t sel = 0u;
 #pragma unroll
     for (int i = 0; i < kTopkItems; ++i) {
       if (!ok[i]) continue;
-      bool cand = st.all_allowed || key[i] > st.prefix;
-      if (!st.all_allowed && key[i] == st.prefix) {
-        cand = rank_ties ? r < take : take > 0;
-        ++r;
+      ++ok_mine;
+      bool c;
+      if (exact) {
+        c = key[i] > lo_key;
+        if (key[i] == lo_key) c = r++ < take;
+      } else {
+        c = key[i] >= lo_key;
       }
-      if (cand) {
-        const int v = v0 + i;
-        const Philox4 ph = philox4x32_10(static_cast<uint32_t>(v) >> 2, bg, s.step, 0u,
-                                         static_cast<uint32_t>(k64),
-                                         static_cast<uint32_t>(k64 >> 32));
-        const uint32_t w =
-            (v & 3) == 0 ? ph.w0 : (v & 3) == 1 ? ph.w1 : (v & 3) == 2 ? ph.w2 : ph.w3;
-        const float sc = fmaf(l[i], s.inv_temp, gumbel_from_u32(w));
-        const uint64_t k = pack_key(__float_as_uint(sc), v);
-        best = k > best ? k : best;
-      }
+      if (c) sel |= 1u << i;
+    }
+    // Warp-aggregated append: one shared-memory atomic per warp.
+    const int n = __popc(sel);
+    int incl = n;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += y;
+    }
+    int wbase = 0;
+    if (lane == 31 && incl > 0) wbase = atomicAdd(n_out, incl);
+    wbase = __shfl_sync(0xffffffffu, wbase, 31);
+    int pos = wbase + incl - n;
+#pragma unroll
+    for (int i = 0; i < kTopkItems; ++i) {
+      if (((sel >> i) & 1u) && pos < cap)
+        out[pos] = (static_cast<unsigned long long>(key[i]) << 32) |
+                   static_cast<uint32_t>(v0 + i);
+      pos += (sel >> i) & 1u;
     }
   }
 #pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) {
-    const uint64_t o = __shfl_xor_sync(0xffffffffu, best, off);
-    best = o > best ? o : best;
+  for (int off = 16; off >= 1; off >>= 1) ok_mine += __shfl_xor_sync(0xffffffffu, ok_mine, off);
+  if (lane == 0 && ok_mine) atomicAdd(n_ok, ok_mine);
+  __syncthreads();
+}
+
+// Candidate list of block (p, b): the allowed keys of its slice at or above a
+// threshold (in no particular order), its count and the threshold.  A slice
+// of more than two sample widths first tries a threshold read off a
+// histogram of its first kTopkMinSlice tokens, with room for half as many
+// again as the sample predicts; the extraction pass verifies it (at least
+// min(K, allowed) keys pass, at most cap).  Otherwise, or when that check
+// fails, exact radix histograms of the whole slice set the threshold.
+__global__ void __launch_bounds__(kTopkThreads) topk_local_kernel(const TopkArgs a) {
+  __shared__ TopkShared sh;
+  __shared__ int n_out, n_ok;
+  sm100::grid_dependency_wait();  // the logits
+  const int p = blockIdx.x, b = blockIdx.y;
+  const SampleLogitsParams &s = a.s;
+  const uint32_t bg = static_cast<uint32_t>(s.b_off + b);
+  const float *row = s.logits + static_cast<size_t>(b) * s.V;
+  const int lo = p * a.slice, hi = imin(s.V, lo + a.slice);
+  const bool vec = (s.V & 3) == 0;
+  unsigned long long *out = a.cand + (static_cast<size_t>(b) * a.P + p) * a.cap;
+  if (threadIdx.x == 0) {
+    n_out = 0;
+    n_ok = 0;
+  }
+  __syncthreads();
+
+  uint32_t thr = 0u;
+  bool done = false;
+  const int len = hi - lo;
+  if (len > 2 * kTopkMinSlice) {
+    topk_slice_hist(s, row, bg, lo, lo + kTopkMinSlice, vec, 0u, 0u, 21, kTopkBins, sh);
+    const long long want = static_cast<long long>(a.K) * kTopkMinSlice / len;
+    const int target = static_cast<int>(want + want / 2 + 16);
+    int above, count, ok_sample;
+    const int d = topk_select_digit(kTopkBins, target, sh, &above, &count, &ok_sample);
+    if (ok_sample > target) {
+      const uint32_t lo_key = static_cast<uint32_t>(d) << 21;
+      topk_extract(s, row, bg, lo, hi, vec, lo_key, false, 0, out, a.cap, &n_out, &n_ok, sh);
+      const int got = n_out, allowed = n_ok;
+      done = got >= imin(a.K, allowed) && got <= a.cap;
+      if (done) {
+        thr = got >= a.K ? lo_key : 0u;
+      } else {
+        __syncthreads();  // every thread has read the counts
+        if (threadIdx.x == 0) {
+          n_out = 0;
+          n_ok = 0;
+        }
+        __syncthreads();
+      }
+    }
+  }
+
+  if (!done) {
+    // Exact threshold: keys >= lo_key, or in exact mode keys > kb and the
+    // first `take` keys equal to kb (lo_key = kb).
+    uint32_t lo_key = 0u;
+    bool exact = false;
+    int take = 0;
+    topk_slice_hist(s, row, bg, lo, hi, vec, 0u, 0u, 21, kTopkBins, sh);
+    int above, count, allowed;
+    const int d1 = topk_select_digit(kTopkBins, a.K, sh, &above, &count, &allowed);
+    if (allowed > a.K) {
+      uint32_t pre = static_cast<uint32_t>(d1) << 21;
+      int k_rem = a.K - above;
+      if (above + count <= a.cap) {
+        lo_key = pre;
+      } else {
+        topk_slice_hist(s, row, bg, lo, hi, vec, pre, 0xFFE00000u, 10, kTopkBins, sh);
+        int above2, count2, tot2;
+        const int d2 = topk_select_digit(kTopkBins, k_rem, sh, &above2, &count2, &tot2);
+        pre |= static_cast<uint32_t>(d2) << 10;
+        above += above2;
+        k_rem -= above2;
+        if (above + count2 <= a.cap) {
+          lo_key = pre;
+        } else {
+          topk_slice_hist(s, row, bg, lo, hi, vec, pre, 0xFFFFFC00u, 0, 1024, sh);
+          int above3, count3, tot3;
+          const int d3 = topk_select_digit(1024, k_rem, sh, &above3, &count3, &tot3);
+          lo_key = pre | static_cast<uint32_t>(d3);
+          exact = true;
+          take = k_rem - above3;  // 1 <= take <= count3
+        }
+      }
+      thr = lo_key;
+    }
+    topk_extract(s, row, bg, lo, hi, vec, lo_key, exact, take, out, a.cap, &n_out, &n_ok, sh);
+  }
+  if (threadIdx.x == 0) {
+    const size_t at = static_cast<size_t>(b) * a.P + p;
+    a.cnt[at] = imin(n_out, a.cap);
+    a.thr[at] = thr;
+  }
+}
+
+// A row's candidates for topk_row_kernel: kept in shared memory when they
+// fit, else read from the blocks' lists (flat index i over the lists, whose
+// offsets are in shared memory), keys below t0 excluded.
+struct TopkRowCands {
+  const unsigned long long *sm;     // kept entries, or nullptr
+  const unsigned long long *lists;  // [P][cap]
+  const int *offs;                  // P + 1 list offsets
+  int P, cap;
+  uint32_t t0;
+  __device__ __forceinline__ bool entry(int i, unsigned long long &e) const {
+    if (sm != nullptr) {
+      e = sm[i];
+      return true;
+    }
+    int q = 0, qe = P;  // the list holding flat index i: offs[q] <= i < offs[q + 1]
+    while (qe - q > 1) {
+      const int mid = (q + qe) >> 1;
+      if (offs[mid] <= i) q = mid; else qe = mid;
+    }
+    e = __ldcg(lists + static_cast<size_t>(q) * cap + (i - offs[q]));
+    return static_cast<uint32_t>(e >> 32) >= t0;
+  }
+};
+
+// The k-th largest (1-based, k <= the participating count) of the 32-bit
+// values of entries [0, n): MODE 0 the key of every entry; MODE 1 ~token of
+// the entries whose key is kb (so the k-th largest is the k-th smallest
+// token).  Three radix passes over bits 31-21, 20-10, 9-0; *n_above gets the
+// count of larger values, *n_eq the count equal to the result.
+template <int MODE>
+__device__ uint32_t topk_row_kth(const TopkRowCands &c, int n, int k, uint32_t kb,
+                                 TopkShared &sh, int *n_above, int *n_eq) {
+  uint32_t pre = 0u, pmask = 0u;
+  int above_total = 0, count = 0;
+#pragma unroll 1
+  for (int level = 0; level < 3; ++level) {
+    const int shift = level == 0 ? 21 : (level == 1 ? 10 : 0);
+    const int nb = level == 2 ? 1024 : kTopkBins;
+    for (int i = threadIdx.x; i < kTopkSubHists * nb; i += kTopkThreads) sh.hist[i] = 0;
+    __syncthreads();
+    int *my_hist = sh.hist + ((threadIdx.x >> 5) & (kTopkSubHists - 1)) * nb;
+    for (int i = threadIdx.x; i < n; i += kTopkThreads) {
+      unsigned long long e;
+      if (!c.entry(i, e)) continue;
+      const uint32_t key = static_cast<uint32_t>(e >> 32);
+      if (MODE == 1 && key != kb) continue;
+      const uint32_t v = MODE == 0 ? key : ~static_cast<uint32_t>(e);
+      if ((v & pmask) == pre) atomicAdd(&my_hist[(v >> shift) & static_cast<uint32_t>(nb - 1)], 1);
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < nb; i += kTopkThreads) {
+      int t = 0;
+#pragma unroll
+      for (int h = 0; h < kTopkSubHists; ++h) t += sh.hist[h * nb + i];
+      sh.hist[i] = t;
+    }
+    __syncthreads();
+    int above, tot;
+    const int d = topk_select_digit(nb, k, sh, &above, &count, &tot);
+    pre |= static_cast<uint32_t>(d) << shift;
+    pmask |= static_cast<uint32_t>(nb - 1) << shift;
+    k -= above;
+    above_total += above;
+  }
+  *n_above = above_total;
+  *n_eq = count;
+  return pre;
+}
+
+// Row b: keeps the candidates at or above the largest block threshold (the
+// row's k-th largest key is at least every block's), selects the exact top
+// K (ties toward the smaller token), draws their noise and writes the
+// Gumbel-max token.
+__global__ void __launch_bounds__(kTopkThreads) topk_row_kernel(const TopkArgs a) {
+  __shared__ TopkShared sh;
+  __shared__ int offs[kTopkMaxP + 1];
+  __shared__ int n_kept;
+  __shared__ unsigned int t0;
+  extern __shared__ unsigned long long kept[];  // kTopkRowCap entries
+  sm100::grid_dependency_wait();  // the candidate lists
+  const int b = blockIdx.x;
+  const int lane = threadIdx.x & 31;
+  const SampleLogitsParams &s = a.s;
+  const uint32_t bg = static_cast<uint32_t>(s.b_off + b);
+  const unsigned long long *lists = a.cand + static_cast<size_t>(b) * a.P * a.cap;
+
+  if (threadIdx.x == 0) {
+    n_kept = 0;
+    t0 = 0u;
+  }
+  __syncthreads();
+  int cq = 0;
+  if (threadIdx.x < a.P) {
+    cq = __ldcg(a.cnt + static_cast<size_t>(b) * a.P + threadIdx.x);
+    atomicMax(&t0, __ldcg(a.thr + static_cast<size_t>(b) * a.P + threadIdx.x));
+  }
+  const int off = block_exclusive_scan(cq, sh.warp_sums, &sh.total);  // orders the writes above
+  const int total = sh.total;
+  if (threadIdx.x < a.P) offs[threadIdx.x] = off;
+  if (threadIdx.x == 0) offs[a.P] = total;
+  __syncthreads();
+
+  // Keep the entries with key >= t0 in shared memory while they fit.
+  TopkRowCands c{nullptr, lists, offs, a.P, a.cap, t0};
+  for (int i0 = 0; i0 < total; i0 += kTopkThreads) {
+    const int i = i0 + threadIdx.x;
+    unsigned long long e = 0ull;
+    const bool keep = i < total && c.entry(i, e);
+    const unsigned m = __ballot_sync(0xffffffffu, keep);
+    int wbase = 0;
+    if (lane == 0 && m) wbase = atomicAdd(&n_kept, __popc(m));
+    wbase = __shfl_sync(0xffffffffu, wbase, 0);
+    const int pos = wbase + __popc(m & ((1u << lane) - 1u));
+    if (keep && pos < kTopkRowCap) kept[pos] = e;
+  }
+  __syncthreads();
+  const int n_all = n_kept;
+  int n = total;
+  if (n_all <= kTopkRowCap) {
+    c.sm = kept;
+    n = n_all;
+  }
+
+  bool all = n_all <= a.K;
+  uint32_t kb = 0u, ti = 0u;
+  int take = 0, n_eq = 0;
+  bool rank_ties = false;
+  if (!all) {
+    int n_above;
+    kb = topk_row_kth<0>(c, n, a.K, 0u, sh, &n_above, &n_eq);
+    take = a.K - n_above;  // 1 <= take <= n_eq
+    if (take < n_eq) {
+      rank_ties = true;
+      int a2, e2;
+      ti = topk_row_kth<1>(c, n, take, kb, sh, &a2, &e2);
+    }
+  }
+
+  const uint64_t k64 = s.row_seeds ? s.row_seeds[bg] : s.seed;
+  uint64_t best = 0ull;
+  for (int i = threadIdx.x; i < n; i += kTopkThreads) {
+    unsigned long long e;
+    if (!c.entry(i, e)) continue;
+    const uint32_t key = static_cast<uint32_t>(e >> 32);
+    const bool sel = all || key > kb ||
+                     (key == kb && (!rank_ties || ~static_cast<uint32_t>(e) >= ti));
+    if (!sel) continue;
+    const int v = static_cast<int>(static_cast<uint32_t>(e));
+    const float l = __uint_as_float(order_bits_inv(key));
+    const Philox4 ph = philox4x32_10(static_cast<uint32_t>(v) >> 2, bg, s.step, 0u,
+                                     static_cast<uint32_t>(k64), static_cast<uint32_t>(k64 >> 32));
+    const uint32_t w = (v & 3) == 0 ? ph.w0 : (v & 3) == 1 ? ph.w1 : (v & 3) == 2 ? ph.w2 : ph.w3;
+    const float sc = fmaf(l, s.inv_temp, gumbel_from_u32(w));
+    const uint64_t k = pack_key(__float_as_uint(sc), v);
+    best = k > best ? k : best;
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    const uint64_t x = __shfl_xor_sync(0xffffffffu, best, o);
+    best = x > best ? x : best;
   }
   if (lane == 0) sh.warp_best[threadIdx.x >> 5] = best;
   __syncthreads();
   if (threadIdx.x == 0) {
     uint64_t r = 0ull;
     for (int i = 0; i < kTopkThreads / 32; ++i) r = sh.warp_best[i] > r ? sh.warp_best[i] : r;
-    if (r) atomicMax(a.rowkey + b, static_cast<unsigned long long>(r));
-    __threadfence();
-    last_block = atomicAdd(a.ticket + b, 1u) == static_cast<unsigned>(a.P - 1);
-  }
-  __syncthreads();
-  if (last_block) {
-    __threadfence();
-    if (threadIdx.x == 0) {
-      const unsigned long long kb = atomicExch(a.rowkey + b, 0ull);
-      s.out_idx[b] = key_token(kb);
-      a.ticket[b] = 0u;
-    }
-    // every block of the row has read the histograms before taking its ticket
-    for (int i = threadIdx.x; i < kTopkBins; i += kTopkThreads) {
-      a.hist0[static_cast<size_t>(b) * kTopkBins + i] = 0;
-      a.hist1[static_cast<size_t>(b) * kTopkBins + i] = 0;
-    }
-    for (int i = threadIdx.x; i < 1024; i += kTopkThreads) a.hist2[static_cast<size_t>(b) * 1024 + i] = 0;
-    for (int i = threadIdx.x; i < a.P * 1024; i += kTopkThreads)
-      a.hist2blk[static_cast<size_t>(b) * a.P * 1024 + i] = 0;
+    s.out_idx[b] = key_token(r);
   }
 }
 
 cudaError_t launch_topk_sample(const SampleLogitsParams &s, int K, void *scratch,
                                cudaStream_t stream) {
-  const int P = topk_blocks_per_row(s.B, s.V, s.num_sms);
-  const TopkLayout lay = topk_layout(s.B, P);
-  char *base = static_cast<char *>(scratch);
+  const TopkGeom g = topk_geom(s.B, s.V, K, s.num_sms);
   TopkArgs a;
   a.s = s;
   a.K = K;
-  a.P = P;
-  a.slice = ((s.V + P - 1) / P + kTopkItems - 1) / kTopkItems * kTopkItems;
-  a.hist0 = reinterpret_cast<int *>(base + lay.hist0);
-  a.hist1 = reinterpret_cast<int *>(base + lay.hist1);
-  a.hist2 = reinterpret_cast<int *>(base + lay.hist2);
-  a.hist2blk = reinterpret_cast<int *>(base + lay.hist2blk);
-  a.rowkey = reinterpret_cast<unsigned long long *>(base + lay.rowkey);
-  a.ticket = reinterpret_cast<unsigned int *>(base + lay.ticket);
-  const dim3 grid(P, s.B), block(kTopkThreads);
-  cudaError_t e;
-  if ((e = launch_dependent(topk_hist_kernel<0>, grid, block, stream, a)) != cudaSuccess) return e;
-  if ((e = launch_dependent(topk_hist_kernel<1>, grid, block, stream, a)) != cudaSuccess) return e;
-  if ((e = launch_dependent(topk_hist_kernel<2>, grid, block, stream, a)) != cudaSuccess) return e;
-  return launch_dependent(topk_final_kernel, grid, block, stream, a);
+  a.P = g.P;
+  a.slice = g.slice;
+  a.cap = g.cap;
+  char *base = static_cast<char *>(scratch);
+  const size_t lists = static_cast<size_t>(s.B) * g.P * g.cap * 8;
+  a.cand = reinterpret_cast<unsigned long long *>(base);
+  a.cnt = reinterpret_cast<int *>(base + lists);
+  a.thr = reinterpret_cast<unsigned int *>(base + lists + static_cast<size_t>(s.B) * g.P * 4);
+  const size_t row_smem = static_cast<size_t>(kTopkRowCap) * 8;  // above the default limit
+  cudaError_t e = cudaFuncSetAttribute(topk_row_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(row_smem));
+  if (e != cudaSuccess) return e;
+  e = launch_dependent(topk_local_kernel, dim3(g.P, s.B), dim3(kTopkThreads), stream, a);
+  if (e != cudaSuccess) return e;
+  return launch_dependent_smem(topk_row_kernel, dim3(s.B), dim3(kTopkThreads), row_smem, stream,
+                               a);
 }
-
 // ---------------------------------------------------------------------------
 // Vocabulary shards: tokens from the reduced keys.
 // ---------------------------------------------------------------------------

@@ -71,11 +71,11 @@ struct SampleLogitsParams {
 };
 cudaError_t launch_sample_logits(const SampleLogitsParams &s, cudaStream_t stream);
 
-// Top-k sampling over the fp32 logits: each row split over several blocks,
-// four launches (three radix-histogram passes, then the candidates).
-// `scratch` holds topk_scratch_bytes(s.B, s.V, s.num_sms) bytes, zero on
-// entry and left zero.
-size_t topk_scratch_bytes(int rows, int V, int num_sms);
+// Top-k sampling over the fp32 logits: two launches (per-block candidate
+// lists by radix histograms, then one block per row selects and samples).
+// `scratch` holds topk_scratch_bytes(s.B, s.V, K, s.num_sms) bytes; no
+// contents carry over between calls.
+size_t topk_scratch_bytes(int rows, int V, int K, int num_sms);
 cudaError_t launch_topk_sample(const SampleLogitsParams &s, int K, void *scratch,
                                cudaStream_t stream);
 

@@ -595,6 +595,78 @@ def test_topk_ties_across_blocks(dev, oracle):
         assert_parity(got, idx, best, second, "topk ties across blocks")
 
 
+@pytest.mark.parametrize("masked", [False, True])
+def test_topk_dense_boundary_bins(dev, oracle, masked):
+    """K = 1900 of 8192-token select slices: the k-th place falls in a
+    top-level histogram bin so full that a slice's candidates overflow their
+    capacity, so each slice narrows its threshold with a second radix pass."""
+    B, d, V, K = 3, 64, 65536, 1900
+    H, W, Hd, Wd = rand_inputs(B, d, V, seed=23)
+    mask = synth.make_mask(B, V, 0.6, seed=24) if masked else None
+    md = mask.to(dev) if masked else None
+    for step in range(3):
+        got = binding.fs_sample_topk(Hd, Wd, K, temperature=0.9, seed=4, step=step,
+                                     mask_bits=md).cpu().numpy()
+        idx, best, second = oracle.sample_topk(H, W, K, T=0.9, seed=4, step=step, mask=mask)
+        assert_parity(got, idx, best, second, "topk dense bins")
+
+
+@pytest.mark.parametrize("K,allowed", [(50, None), (1900, None), (50, 0.6), (400, 0.02)])
+def test_topk_sampled_threshold(dev, oracle, K, allowed):
+    """40 rows of V = 100000: three select blocks per row on 148 SMs, slices
+    of 33336 tokens, so each block first tries a threshold from a histogram
+    of its first 8192 tokens.  K = 50 keeps it; K = 1900 overflows the
+    candidate capacity and a 2 % mask leaves too few allowed keys above it,
+    so those blocks fall back to exact histograms of the whole slice."""
+    B, d, V = 40, 32, 100000
+    H, W, Hd, Wd = rand_inputs(B, d, V, seed=51)
+    mask = synth.make_mask(B, V, allowed, seed=52) if allowed else None
+    md = mask.to(dev) if allowed else None
+    rs = synth.make_row_seeds(B)
+    got = binding.fs_sample_topk(Hd, Wd, K, temperature=0.8, seed=5, row_seeds=rs.to(dev), step=1,
+                                 mask_bits=md).cpu().numpy()
+    idx, best, second = oracle.sample_topk(H, W, K, T=0.8, seed=5, row_seeds=rs, step=1, mask=mask)
+    assert_parity(got, idx, best, second, "topk sampled threshold K=%d" % K)
+
+
+@pytest.mark.parametrize("K,masked", [(1, False), (1, True), (5000, False), (5000, True)])
+def test_topk_all_logits_tied(dev, oracle, K, masked):
+    """W = 0: every logit is exactly 0, so every slice resolves its threshold
+    to the exact key and keeps its tied tokens in index order; the sampled
+    token is the Gumbel-max over the K smallest allowed indices."""
+    B, d, V = 4, 64, 20000
+    H, _, Hd, _ = rand_inputs(B, d, V, seed=31)
+    W = torch.zeros(V, d, dtype=torch.bfloat16)
+    Wd = W.to(dev)
+    mask = synth.make_mask(B, V, 0.5, seed=32) if masked else None
+    md = mask.to(dev) if masked else None
+    got = binding.fs_sample_topk(Hd, Wd, K, temperature=1.0, seed=7, step=2,
+                                 mask_bits=md).cpu().numpy()
+    idx, best, second = oracle.sample_topk(H, W, K, T=1.0, seed=7, step=2, mask=mask)
+    assert np.array_equal(got, idx), (got, idx)
+    if K == 1 and not masked:
+        assert (got == 0).all()
+
+
+def test_topk_large_tie_inside_one_slice(dev, oracle):
+    """3000 copies of the dominant W row inside the first select slice and
+    K = 2500: the slice's candidates exceed its capacity down to the exact
+    key, so it keeps the 2500 smallest tied indices, and so must the row."""
+    B, d, V, K = 2, 64, 20000, 2500
+    _, W, _, _ = rand_inputs(B, d, V, seed=41)
+    h = synth.make_hidden(1, d, seed=42)
+    H = h.repeat(B, 1).contiguous()
+    W = W.clone()
+    hf = h[0].float()
+    W[100:3100] = (hf * 8.0 / (hf * hf).sum()).to(torch.bfloat16)
+    Hd, Wd = H.to(dev), W.to(dev)
+    for step in range(4):
+        got = binding.fs_sample_topk(Hd, Wd, K, temperature=1.0, seed=9, step=step).cpu().numpy()
+        idx, best, second = oracle.sample_topk(H, W, K, T=1.0, seed=9, step=step)
+        assert ((got >= 100) & (got < 100 + K)).all(), got
+        assert_parity(got, idx, best, second, "topk large tie")
+
+
 def test_topk_full_vocab(dev, oracle):
     wl = synth.WORKLOADS["qwen3-8b"]
     B, K = 64, 40
