@@ -289,13 +289,14 @@ cudaError_t launch_sample_logits(const SampleLogitsParams &s, cudaStream_t strea
 // accumulated.
 // ---------------------------------------------------------------------------
 constexpr int kTopkThreads = 1024;
-constexpr int kTopkItems = 8;      // consecutive elements per thread per iteration
+constexpr int kTopkItems = 16;     // consecutive elements per thread per iteration (4 x 16 B)
 constexpr int kTopkBins = 2048;
 constexpr int kTopkSubHists = 4;   // warp-interleaved copies of the shared histogram
 constexpr int kTopkMinSlice = kTopkThreads * kTopkItems;
 constexpr int kTopkMinCap = 2048;  // candidate capacity per block, at least K
 constexpr int kTopkMaxP = 512;
 constexpr int kTopkRowCap = 8192;  // candidates a row's select block keeps in shared memory
+constexpr int kTopkRowSmall = 256; // at most this many left after one radix level: rank them
 
 struct TopkGeom {
   int P, slice, cap;
@@ -405,34 +406,39 @@ __device__ int topk_select_digit(int nb, int k, TopkShared &sh, int *above, int 
 }
 
 // Loads this thread's kTopkItems consecutive logits starting at v0 (below
-// hi) and their order-preserving keys; ok[i] is false past hi or for a
-// masked token.
-__device__ __forceinline__ void topk_load(const SampleLogitsParams &s, const float *row,
-                                          uint32_t bg, int v0, int hi, bool vec,
-                                          uint32_t (&key)[kTopkItems], bool (&ok)[kTopkItems]) {
-  float l[kTopkItems];
+// hi; four 16-byte loads in flight when the row allows) as order-preserving
+// keys; bit i of the result is set for an in-range, allowed token v0 + i.
+__device__ __forceinline__ uint32_t topk_load(const SampleLogitsParams &s, const float *row,
+                                              uint32_t bg, int v0, int hi, bool vec,
+                                              uint32_t (&key)[kTopkItems]) {
+  uint32_t okm;
   if (vec && v0 + kTopkItems <= hi) {
-    const float4 a = *reinterpret_cast<const float4 *>(row + v0);
-    const float4 c = *reinterpret_cast<const float4 *>(row + v0 + 4);
-    l[0] = a.x; l[1] = a.y; l[2] = a.z; l[3] = a.w;
-    l[4] = c.x; l[5] = c.y; l[6] = c.z; l[7] = c.w;
+    const float4 *src = reinterpret_cast<const float4 *>(row + v0);
+    float4 q[kTopkItems / 4];
 #pragma unroll
-    for (int i = 0; i < kTopkItems; ++i) ok[i] = true;
+    for (int j = 0; j < kTopkItems / 4; ++j) q[j] = src[j];
+#pragma unroll
+    for (int j = 0; j < kTopkItems / 4; ++j) {
+      key[4 * j + 0] = __float_as_uint(q[j].x);
+      key[4 * j + 1] = __float_as_uint(q[j].y);
+      key[4 * j + 2] = __float_as_uint(q[j].z);
+      key[4 * j + 3] = __float_as_uint(q[j].w);
+    }
+    okm = (1u << kTopkItems) - 1u;
   } else {
+    okm = 0u;
 #pragma unroll
     for (int i = 0; i < kTopkItems; ++i) {
-      ok[i] = v0 + i < hi;
-      l[i] = ok[i] ? row[v0 + i] : 0.f;
+      const bool in = v0 + i < hi;
+      key[i] = in ? __float_as_uint(row[v0 + i]) : 0u;
+      okm |= in ? (1u << i) : 0u;
     }
   }
-  uint32_t mword = 0xFFFFFFFFu;
-  if (s.mask != nullptr && v0 < hi)   // 8 consecutive tokens from a multiple of 8 share one word
-    mword = s.mask[static_cast<size_t>(bg) * s.mask_words + (v0 >> 5)];
+  if (s.mask != nullptr && v0 < hi)  // 16 tokens from a multiple of 16 lie in one mask word
+    okm &= s.mask[static_cast<size_t>(bg) * s.mask_words + (v0 >> 5)] >> (v0 & 31);
 #pragma unroll
-  for (int i = 0; i < kTopkItems; ++i) {
-    ok[i] = ok[i] && ((mword >> ((v0 + i) & 31)) & 1u);
-    key[i] = order_bits(__float_as_uint(l[i]));
-  }
+  for (int i = 0; i < kTopkItems; ++i) key[i] = order_bits(key[i]);
+  return okm;
 }
 
 // Histogram, in sh.hist[0, nb), of digit (key >> shift) & (nb - 1) over the
@@ -446,11 +452,11 @@ __device__ void topk_slice_hist(const SampleLogitsParams &s, const float *row, u
   const uint32_t dmask = static_cast<uint32_t>(nb - 1);
   for (int base = lo; base < hi; base += kTopkThreads * kTopkItems) {
     uint32_t key[kTopkItems];
-    bool ok[kTopkItems];
-    topk_load(s, row, bg, base + threadIdx.x * kTopkItems, hi, vec, key, ok);
+    const uint32_t okm = topk_load(s, row, bg, base + threadIdx.x * kTopkItems, hi, vec, key);
 #pragma unroll
     for (int i = 0; i < kTopkItems; ++i)
-      if (ok[i] && (key[i] & pmask) == prefix) atomicAdd(&my_hist[(key[i] >> shift) & dmask], 1);
+      if (((okm >> i) & 1u) && (key[i] & pmask) == prefix)
+        atomicAdd(&my_hist[(key[i] >> shift) & dmask], 1);
   }
   __syncthreads();
   for (int i = threadIdx.x; i < nb; i += kTopkThreads) {
@@ -475,21 +481,20 @@ __device__ void topk_extract(const SampleLogitsParams &s, const float *row, uint
   for (int base = lo; base < hi; base += kTopkThreads * kTopkItems) {
     const int v0 = base + threadIdx.x * kTopkItems;
     uint32_t key[kTopkItems];
-    bool ok[kTopkItems];
-    topk_load(s, row, bg, v0, hi, vec, key, ok);
+    const uint32_t okm = topk_load(s, row, bg, v0, hi, vec, key);
     int r = 0;
     if (exact) {  // block-uniform: rank the tied keys in token order
       int n_eq = 0;
 #pragma unroll
-      for (int i = 0; i < kTopkItems; ++i) n_eq += (ok[i] && key[i] == lo_key) ? 1 : 0;
+      for (int i = 0; i < kTopkItems; ++i) n_eq += (((okm >> i) & 1u) && key[i] == lo_key) ? 1 : 0;
       r = eq_seen + block_exclusive_scan(n_eq, sh.warp_sums, &sh.total);
       eq_seen += sh.total;
     }
     uint32_t sel = 0u;
+    ok_mine += __popc(okm);
 #pragma unroll
     for (int i = 0; i < kTopkItems; ++i) {
-      if (!ok[i]) continue;
-      ++ok_mine;
+      if (!((okm >> i) & 1u)) continue;
       bool c;
       if (exact) {
         c = key[i] > lo_key;
@@ -695,8 +700,9 @@ __device__ uint32_t topk_row_kth(const TopkRowCands &c, int n, int k, uint32_t k
 __global__ void __launch_bounds__(kTopkThreads) topk_row_kernel(const TopkArgs a) {
   __shared__ TopkShared sh;
   __shared__ int offs[kTopkMaxP + 1];
-  __shared__ int n_kept;
+  __shared__ int n_kept, n_small;
   __shared__ unsigned int t0;
+  __shared__ unsigned long long small[kTopkRowSmall];
   extern __shared__ unsigned long long kept[];  // kTopkRowCap entries
   sm100::grid_dependency_wait();  // the candidate lists
   const int b = blockIdx.x;
@@ -707,6 +713,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_row_kernel(const TopkArgs a
 
   if (threadIdx.x == 0) {
     n_kept = 0;
+    n_small = 0;
     t0 = 0u;
   }
   __syncthreads();
@@ -742,11 +749,49 @@ __global__ void __launch_bounds__(kTopkThreads) topk_row_kernel(const TopkArgs a
     n = n_all;
   }
 
-  bool all = n_all <= a.K;
+  const bool all = n_all <= a.K;
+  // One radix level over the kept keys (bits 31-21); when the keys at or
+  // above the k-th largest key's digit are few, they are ranked directly:
+  // rank = entries with a larger key, or the same key and a smaller token.
+  bool by_rank = false;
+  if (!all && c.sm != nullptr) {
+    for (int i = threadIdx.x; i < kTopkSubHists * kTopkBins; i += kTopkThreads) sh.hist[i] = 0;
+    __syncthreads();
+    int *my_hist = sh.hist + ((threadIdx.x >> 5) & (kTopkSubHists - 1)) * kTopkBins;
+    for (int i = threadIdx.x; i < n; i += kTopkThreads)
+      atomicAdd(&my_hist[static_cast<uint32_t>(kept[i] >> 53)], 1);
+    __syncthreads();
+    for (int i = threadIdx.x; i < kTopkBins; i += kTopkThreads) {
+      int t = 0;
+#pragma unroll
+      for (int h = 0; h < kTopkSubHists; ++h) t += sh.hist[h * kTopkBins + i];
+      sh.hist[i] = t;
+    }
+    __syncthreads();
+    int above, count, tot;
+    const uint32_t d1 = static_cast<uint32_t>(topk_select_digit(kTopkBins, a.K, sh, &above, &count, &tot));
+    if (above + count <= kTopkRowSmall) {
+      by_rank = true;
+      for (int i0 = 0; i0 < n; i0 += kTopkThreads) {
+        const int i = i0 + threadIdx.x;
+        const unsigned long long e = i < n ? kept[i] : 0ull;
+        const bool keep = i < n && static_cast<uint32_t>(e >> 53) >= d1;
+        const unsigned m = __ballot_sync(0xffffffffu, keep);
+        int wbase = 0;
+        if (lane == 0 && m) wbase = atomicAdd(&n_small, __popc(m));
+        wbase = __shfl_sync(0xffffffffu, wbase, 0);
+        const int pos = wbase + __popc(m & ((1u << lane) - 1u));
+        if (keep && pos < kTopkRowSmall) small[pos] = e;
+      }
+      __syncthreads();
+      c.sm = small;
+      n = n_small;  // == above + count
+    }
+  }
   uint32_t kb = 0u, ti = 0u;
   int take = 0, n_eq = 0;
   bool rank_ties = false;
-  if (!all) {
+  if (!all && !by_rank) {
     int n_above;
     kb = topk_row_kth<0>(c, n, a.K, 0u, sh, &n_above, &n_eq);
     take = a.K - n_above;  // 1 <= take <= n_eq
@@ -759,12 +804,36 @@ __global__ void __launch_bounds__(kTopkThreads) topk_row_kernel(const TopkArgs a
 
   const uint64_t k64 = s.row_seeds ? s.row_seeds[bg] : s.seed;
   uint64_t best = 0ull;
-  for (int i = threadIdx.x; i < n; i += kTopkThreads) {
-    unsigned long long e;
-    if (!c.entry(i, e)) continue;
+  // Ranking: G consecutive lanes share an entry (G = 1024 / n rounded down to
+  // a power of two, at most 32), each counting over every G-th entry.
+  int gsh = 0;
+  if (by_rank)
+    while (gsh < 5 && (n << (gsh + 1)) <= kTopkThreads) ++gsh;
+  const int G = 1 << gsh;
+  const int per_pass = kTopkThreads >> gsh;
+  for (int i0 = 0; i0 < n; i0 += per_pass) {  // block-uniform trip count
+    const int i = i0 + (threadIdx.x >> gsh);
+    const int sub = threadIdx.x & (G - 1);
+    unsigned long long e = 0ull;
+    const bool have = i < n && c.entry(i, e);
     const uint32_t key = static_cast<uint32_t>(e >> 32);
-    const bool sel = all || key > kb ||
-                     (key == kb && (!rank_ties || ~static_cast<uint32_t>(e) >= ti));
+    bool sel;
+    if (by_rank) {
+      const uint32_t tok = static_cast<uint32_t>(e);
+      int rank = 0;
+      if (have) {
+        for (int j = sub; j < n && rank < a.K; j += G) {
+          const unsigned long long f = small[j];
+          const uint32_t kf = static_cast<uint32_t>(f >> 32);
+          rank += (kf > key || (kf == key && static_cast<uint32_t>(f) < tok)) ? 1 : 0;
+        }
+      }
+      for (int o = G >> 1; o >= 1; o >>= 1) rank += __shfl_xor_sync(0xffffffffu, rank, o);
+      sel = have && sub == 0 && rank < a.K;
+    } else {
+      sel = have && (all || key > kb ||
+                     (key == kb && (!rank_ties || ~static_cast<uint32_t>(e) >= ti)));
+    }
     if (!sel) continue;
     const int v = static_cast<int>(static_cast<uint32_t>(e));
     const float l = __uint_as_float(order_bits_inv(key));

@@ -572,7 +572,7 @@ def test_topk_ties_at_the_boundary(dev, oracle):
 
 
 def test_topk_ties_across_blocks(dev, oracle):
-    """Rows split over several select blocks (V = 65536, one block per 8192
+    """Rows split over several select blocks (V = 65536, one block per 16384
     tokens here): seven copies of the dominant W row sit in different
     blocks, so the k-th place falls inside a tie that spans blocks and the
     four smallest indices must be kept."""
@@ -597,7 +597,7 @@ def test_topk_ties_across_blocks(dev, oracle):
 
 @pytest.mark.parametrize("masked", [False, True])
 def test_topk_dense_boundary_bins(dev, oracle, masked):
-    """K = 1900 of 8192-token select slices: the k-th place falls in a
+    """K = 1900 of 16384-token select slices: the k-th place falls in a
     top-level histogram bin so full that a slice's candidates overflow their
     capacity, so each slice narrows its threshold with a second radix pass."""
     B, d, V, K = 3, 64, 65536, 1900
@@ -614,8 +614,8 @@ def test_topk_dense_boundary_bins(dev, oracle, masked):
 @pytest.mark.parametrize("K,allowed", [(50, None), (1900, None), (50, 0.6), (400, 0.02)])
 def test_topk_sampled_threshold(dev, oracle, K, allowed):
     """40 rows of V = 100000: three select blocks per row on 148 SMs, slices
-    of 33336 tokens, so each block first tries a threshold from a histogram
-    of its first 8192 tokens.  K = 50 keeps it; K = 1900 overflows the
+    of 33344 tokens, so each block first tries a threshold from a histogram
+    of its first 16384 tokens.  K = 50 keeps it; K = 1900 overflows the
     candidate capacity and a 2 % mask leaves too few allowed keys above it,
     so those blocks fall back to exact histograms of the whole slice."""
     B, d, V = 40, 32, 100000
