@@ -209,6 +209,73 @@ fs_status fs_sample_shard_keys(const void *H, const void *W_shard, int B, int d,
 fs_status fs_keys_to_tokens(const int64_t *keys, int B, int32_t *out_idx,
                             fs_stream_t stream);
 
+/* ---- Tensor-parallel vocabulary sampling with the exchange fused into the
+ * kernel (readus.org page, "distributed FlashSampling": every GPU is one
+ * group and sends only its winner's index and score; abstract: the argmax
+ * decomposes over any partition).  Instead of an all-reduce after the
+ * kernel, the last CTA of each rank's kernel writes its rows' packed
+ * (score, token) maxima straight into every rank's exchange area over
+ * NVLink (atomic max on peer memory), counts itself in every area, and the
+ * arrival that completes an area decodes it; no kernel waits for another.
+ * The stream that needs the tokens then waits on the area's flag.
+ *
+ * Protocol for a group of `world` ranks (one process per GPU):
+ *   1. each rank: fs_tp_area_create(&mine); fs_ipc_handle(mine, h) and
+ *      exchange the handles (e.g. an all-gather); fs_ipc_open on every
+ *      peer's handle; areas[r] = rank r's area as mapped in this process
+ *      (areas[own rank] = mine).  Every rank uses the same order.
+ *   2. call number seq = 0, 1, 2, ... (the same on every rank):
+ *      fs_sample_tp(..., areas, world, seq, ...) then
+ *      fs_tp_wait(mine, B, seq, out_idx, stream) on the same stream; out_idx
+ *      holds the tokens once the stream gets there.
+ *   3. at the end: fs_ipc_close on the peers' areas, fs_tp_area_destroy.
+ * A rank must not issue call seq + 1 on a stream that has not passed its
+ * fs_tp_wait of call seq (the alternate halves of the area rely on it).
+ * If any rank's kernel records a device error, it still completes the
+ * exchange; every rank then gets -1 for every row of that call and
+ * fs_tp_failed reports the call.  Sequence numbers wrap after 2^32 calls. */
+#define FS_IPC_HANDLE_BYTES 64
+
+/* Bytes of one exchange area (fixed; up to 256 rows per call). */
+size_t fs_tp_area_bytes(void);
+
+/* Allocates a zeroed exchange area on the current device (cudaMalloc, so
+ * that it can be shared by IPC), or frees one. */
+fs_status fs_tp_area_create(void **area);
+fs_status fs_tp_area_destroy(void *area);
+
+/* CUDA IPC for exchange areas: the FS_IPC_HANDLE_BYTES-byte handle of an
+ * area created here, and opening (with peer access enabled) or closing a
+ * peer's area in this process. */
+fs_status fs_ipc_handle(const void *area, void *handle);
+fs_status fs_ipc_open(const void *handle, void **area);
+fs_status fs_ipc_close(void *area);
+
+/* One rank's part of tensor-parallel sampling: samples the shard as
+ * fs_sample_shard_keys does (same arguments; B <= 256, else
+ * FS_ERR_UNSUPPORTED) and exchanges the result through `areas` (host array of
+ * `world` <= 16 device pointers, each 256-byte aligned).  Asynchronous on
+ * `stream`; follow it with fs_tp_wait.  The tokens equal single-GPU
+ * fs_sample_ex on the full head bit for bit. */
+fs_status fs_sample_tp(const void *H, const void *W_shard, int B, int d,
+                       int V_shard, int vocab_offset, int V_total,
+                       float temperature, uint64_t seed,
+                       const uint64_t *row_seeds, uint32_t step,
+                       const uint32_t *mask_bits, void *const *areas, int world,
+                       uint32_t seq, void *workspace, size_t workspace_bytes,
+                       fs_stream_t stream);
+
+/* Makes `stream` wait (a stream memory operation, no kernel) until call
+ * `seq` has been decoded into this rank's area `area`, then copies its B
+ * tokens to out_idx (device int32 [B]).  FS_ERR_UNSUPPORTED when the device
+ * has no stream memory operations. */
+fs_status fs_tp_wait(const void *area, int B, uint32_t seq, int32_t *out_idx,
+                     fs_stream_t stream);
+
+/* Synchronous: seq + 1 of the last call decoded with a device error in
+ * `area` (0: none). */
+fs_status fs_tp_failed(const void *area, uint32_t *failed);
+
 /* Top-k sampling (readus.org page, "Top-K and masking": a fast prefilter
  * isolates the candidates, then exact Gumbel-max runs on that subset).  The
  * candidates of row b are its K allowed tokens with the largest logits l
@@ -307,6 +374,14 @@ fs_status fs_philox4x32_10(const uint32_t *ctr, const uint32_t *key,
  * function the sampling kernels use); device arrays of n elements. */
 fs_status fs_gumbel(const uint32_t *r, float *g, int64_t n,
                     fs_stream_t stream);
+
+/* Failure-detection test switch: while on (1), every fused-kernel launch's
+ * load-issuing warp issues nothing, so the kernel's bounded waits run out
+ * after about one second and it records FS_ERR_DEVICE_TIMEOUT, as in
+ * fs_test_stalled_sample; for exercising error paths of other entry points
+ * (fs_sample_tp marks the exchanged call as failed).  Off (0) by default;
+ * process-wide. */
+fs_status fs_test_stall_loads(int on);
 
 /* Failure-detection test: launches the flat kernel on these arguments with
  * its load-issuing warp told to issue nothing, so the MMA warp's wait for

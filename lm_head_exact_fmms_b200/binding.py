@@ -24,7 +24,11 @@ EXPORTED = ("fs_sample", "fs_sample_ex", "fs_sample_grouped", "fs_sample_unfused
             "fs_sample_noalloc", "fs_test_stalled_sample", "fs_sample_shard_keys",
             "fs_keys_to_tokens", "fs_sample_multi", "fs_workspace_bytes_multi",
             "fs_summarize_group", "fs_merge_groups", "fs_workspace_bytes_summary",
-            "fs_sample_topk", "fs_set_cta_pairs")
+            "fs_sample_topk", "fs_set_cta_pairs", "fs_tp_area_bytes", "fs_tp_area_create",
+            "fs_tp_area_destroy", "fs_ipc_handle", "fs_ipc_open", "fs_ipc_close", "fs_sample_tp",
+            "fs_tp_wait", "fs_tp_failed", "fs_test_stall_loads")
+
+FS_IPC_HANDLE_BYTES = 64
 
 
 class FmmsError(RuntimeError):
@@ -73,6 +77,18 @@ def load_library():
     lib.fs_workspace_bytes_summary.argtypes = [i32, i32]
     lib.fs_workspace_bytes_summary.restype = sz
     lib.fs_sample_topk.argtypes = common + [i32, f32, u64, vp, u32, vp, vp, vp, vp, sz, vp]
+    lib.fs_tp_area_bytes.argtypes = []
+    lib.fs_tp_area_bytes.restype = sz
+    lib.fs_tp_area_create.argtypes = [ctypes.POINTER(ctypes.c_void_p)]
+    lib.fs_tp_area_destroy.argtypes = [vp]
+    lib.fs_ipc_handle.argtypes = [vp, vp]
+    lib.fs_ipc_open.argtypes = [vp, ctypes.POINTER(ctypes.c_void_p)]
+    lib.fs_ipc_close.argtypes = [vp]
+    lib.fs_sample_tp.argtypes = common + [i32, i32, f32, u64, vp, u32, vp, vp, i32, u32, vp, sz,
+                                          vp]
+    lib.fs_tp_wait.argtypes = [vp, i32, u32, vp, vp]
+    lib.fs_tp_failed.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
+    lib.fs_test_stall_loads.argtypes = [i32]
     lib.fs_workspace_bytes.argtypes = [i32, i32, i32]
     lib.fs_workspace_bytes.restype = sz
     lib.fs_device_status.argtypes = [vp, sz, vp]
@@ -86,7 +102,7 @@ def load_library():
                                        ctypes.POINTER(ctypes.c_int)]
     for name in EXPORTED:
         if name not in ("fs_workspace_bytes", "fs_workspace_bytes_multi",
-                        "fs_workspace_bytes_summary", "fs_status_string"):
+                        "fs_workspace_bytes_summary", "fs_status_string", "fs_tp_area_bytes"):
             getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -344,6 +360,82 @@ def fs_sample_shard_keys(H, W_shard, vocab_offset, V_total, temperature=1.0, see
                                     int(step), _ptr(mask_bits), _ptr(out_keys), _ptr(workspace),
                                     ws_bytes, _stream(stream)), "fs_sample_shard_keys")
     return out_keys
+
+
+def fs_tp_area_bytes():
+    return int(load_library().fs_tp_area_bytes())
+
+
+def fs_tp_area_create():
+    """A zeroed exchange area on the current device; returns its address (int)."""
+    lib = load_library()
+    p = ctypes.c_void_p()
+    _check(lib.fs_tp_area_create(ctypes.byref(p)), "fs_tp_area_create")
+    return int(p.value)
+
+
+def fs_tp_area_destroy(area):
+    _check(load_library().fs_tp_area_destroy(ctypes.c_void_p(area)), "fs_tp_area_destroy")
+
+
+def fs_ipc_handle(area):
+    """The IPC handle (bytes) of an area made by fs_tp_area_create."""
+    buf = ctypes.create_string_buffer(FS_IPC_HANDLE_BYTES)
+    _check(load_library().fs_ipc_handle(ctypes.c_void_p(area), buf), "fs_ipc_handle")
+    return buf.raw
+
+
+def fs_ipc_open(handle):
+    """Maps a peer's area from its handle; returns the address here (int)."""
+    if len(handle) != FS_IPC_HANDLE_BYTES:
+        raise ValueError("an IPC handle has %d bytes" % FS_IPC_HANDLE_BYTES)
+    p = ctypes.c_void_p()
+    _check(load_library().fs_ipc_open(ctypes.create_string_buffer(bytes(handle),
+                                                                  FS_IPC_HANDLE_BYTES),
+                                      ctypes.byref(p)), "fs_ipc_open")
+    return int(p.value)
+
+
+def fs_ipc_close(area):
+    _check(load_library().fs_ipc_close(ctypes.c_void_p(area)), "fs_ipc_close")
+
+
+def fs_sample_tp(H, W_shard, vocab_offset, V_total, areas, seq, temperature=1.0, seed=0,
+                 row_seeds=None, step=0, mask_bits=None, workspace=None, stream=None):
+    """One rank's shard with the exchange fused into the kernel; `areas` are
+    the addresses of every rank's exchange area as mapped here."""
+    lib = load_library()
+    B, d, Vs = _check_operands(H, W_shard)
+    row_seeds = _opt_dev(row_seeds, torch.int64, B, "row_seeds", H.device)
+    mask_bits = _opt_dev(mask_bits, torch.int32, B * ((V_total + 31) // 32), "mask_bits",
+                         H.device)
+    table = (ctypes.c_void_p * len(areas))(*[ctypes.c_void_p(a) for a in areas])
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.fs_sample_tp(_ptr(H), _ptr(W_shard), B, d, Vs, int(vocab_offset), int(V_total),
+                            float(temperature), _seed(seed), _ptr(row_seeds), int(step),
+                            _ptr(mask_bits), table, len(areas), int(seq) & 0xFFFFFFFF,
+                            _ptr(workspace), ws_bytes, _stream(stream)), "fs_sample_tp")
+
+
+def fs_tp_wait(area, B, seq, out_idx=None, device=None, stream=None):
+    """Orders the stream after call `seq`'s tokens reached `area`; returns them."""
+    lib = load_library()
+    dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
+    out_idx = _out(out_idx, B, dev)
+    _check(lib.fs_tp_wait(ctypes.c_void_p(area), int(B), int(seq) & 0xFFFFFFFF, _ptr(out_idx),
+                          _stream(stream)), "fs_tp_wait")
+    return out_idx
+
+
+def fs_tp_failed(area):
+    v = ctypes.c_uint32()
+    _check(load_library().fs_tp_failed(ctypes.c_void_p(area), ctypes.byref(v)), "fs_tp_failed")
+    return int(v.value)
+
+
+def fs_test_stall_loads(on):
+    """Test switch: fused kernels issue no loads, so their waits time out."""
+    _check(load_library().fs_test_stall_loads(1 if on else 0), "fs_test_stall_loads")
 
 
 def fs_keys_to_tokens(keys, out_idx=None, stream=None):

@@ -107,6 +107,22 @@ StreamWriteValue32Fn write_value_fn() {
   return fn;
 }
 
+using StreamWaitValue32Fn = CUresult (*)(CUstream, CUdeviceptr, cuuint32_t, unsigned int);
+
+StreamWaitValue32Fn wait_value_fn() {
+  static StreamWaitValue32Fn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuStreamWaitValue32", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<StreamWaitValue32Fn>(p);
+  });
+  return fn;
+}
+
 EncodeTiledFn encode_fn() {
   static EncodeTiledFn fn = nullptr;
   static std::once_flag once;
@@ -221,8 +237,10 @@ fs_status resolve_workspace(DeviceState *st, const Schedule &sch, int B, int sam
   return FS_OK;
 }
 
-// Set only for the duration of fs_test_stalled_sample (under g_mu).
+// Set for the duration of fs_test_stalled_sample, or between
+// fs_test_stall_loads(1) and fs_test_stall_loads(0) (under g_mu).
 bool g_test_no_loads = false;
+bool g_test_stall = false;
 
 // fs_set_cta_pairs: -1 automatic, 0 never, 1 whenever the call allows it.
 int g_pair_policy = -1;
@@ -263,6 +281,9 @@ struct ShardOpts {
   const uint32_t *h_ready = nullptr;  // H arriving in chunks (fs_sample_host), else null
   uint32_t h_epoch = 0;
   int h_chunk_subs = 0;
+  int tp_world = 0;             // fused vocabulary-parallel exchange (flat mode)
+  uint32_t tp_seq = 0;
+  void *const *tp_areas = nullptr;
 };
 
 // The fused path in all three modes, chunked over 256 batch rows.
@@ -331,13 +352,17 @@ fs_status run_locked(int mode, const void *H, const void *W, int B, int d, int V
     p.partials = w.partials;
     p.gkeys = mode == fmms::kModeGrouped ? w.gkeys : nullptr;
     p.logits = logits ? logits + static_cast<size_t>(b0) * V : nullptr;
-    p.test_no_loads = g_test_no_loads ? 1 : 0;
+    p.test_no_loads = (g_test_no_loads || g_test_stall) ? 1 : 0;
     p.vocab_offset = shard.vocab_offset;
     p.out_keys = shard.out_keys ? shard.out_keys + static_cast<size_t>(b0) * S : nullptr;
     p.num_samples = S;
     p.h_ready = shard.h_ready;
     p.h_epoch = shard.h_epoch;
     p.h_chunk_subs = shard.h_chunk_subs;
+    p.tp_world = shard.tp_world;
+    p.tp_seq = shard.tp_seq;
+    for (int r = 0; r < shard.tp_world; ++r)
+      p.tp_area[r] = static_cast<fmms::TpArea *>(shard.tp_areas[r]);
     const int pair_units_used = pair ? fmms::make_schedule(V, sch.G, units).num_ctas : 0;
     if (pair) {
       p.num_ctas = 2 * pair_units_used;
@@ -517,6 +542,12 @@ fs_status fs_sample_host(const void *H_host, const void *W, int B, int d, int V,
   return FS_OK;
 }
 
+fs_status fs_test_stall_loads(int on) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  g_test_stall = on != 0;
+  return FS_OK;
+}
+
 fs_status fs_test_stalled_sample(const void *H, const void *W, int B, int d, int V,
                                  int32_t *out_idx, void *workspace, size_t workspace_bytes,
                                  fs_stream_t stream) {
@@ -548,6 +579,106 @@ fs_status fs_sample_shard_keys(const void *H, const void *W_shard, int B, int d,
   return run_locked(fmms::kModeFlat, H, W_shard, B, d, V_shard, 1, temperature, seed, row_seeds,
                     step, mask_bits, reinterpret_cast<int32_t *>(out_keys), nullptr, nullptr,
                     workspace, workspace_bytes, static_cast<cudaStream_t>(stream), opts);
+}
+
+// ------------------------------------------- fused vocabulary-parallel exchange
+size_t fs_tp_area_bytes(void) { return fmms::kTpAreaBytes; }
+
+fs_status fs_tp_area_create(void **area) {
+  if (area == nullptr) return FS_ERR_INVALID_ARG;
+  DeviceState *st = nullptr;
+  fs_status s = get_device(&st);
+  if (s != FS_OK) return s;
+  *area = nullptr;
+  if (cudaMalloc(area, fmms::kTpAreaBytes) != cudaSuccess) return FS_ERR_CUDA;
+  if (cudaMemset(*area, 0, fmms::kTpAreaBytes) != cudaSuccess ||
+      cudaDeviceSynchronize() != cudaSuccess) {
+    cudaFree(*area);
+    *area = nullptr;
+    return FS_ERR_CUDA;
+  }
+  return FS_OK;
+}
+
+fs_status fs_tp_area_destroy(void *area) {
+  if (area == nullptr) return FS_OK;
+  return cudaFree(area) == cudaSuccess ? FS_OK : FS_ERR_CUDA;
+}
+
+fs_status fs_ipc_handle(const void *area, void *handle) {
+  if (area == nullptr || handle == nullptr) return FS_ERR_INVALID_ARG;
+  cudaIpcMemHandle_t h;
+  if (cudaIpcGetMemHandle(&h, const_cast<void *>(area)) != cudaSuccess) return FS_ERR_CUDA;
+  static_assert(sizeof(h) == FS_IPC_HANDLE_BYTES, "IPC handle size");
+  memcpy(handle, &h, sizeof h);
+  return FS_OK;
+}
+
+fs_status fs_ipc_open(const void *handle, void **area) {
+  if (handle == nullptr || area == nullptr) return FS_ERR_INVALID_ARG;
+  cudaIpcMemHandle_t h;
+  memcpy(&h, handle, sizeof h);
+  *area = nullptr;
+  return cudaIpcOpenMemHandle(area, h, cudaIpcMemLazyEnablePeerAccess) == cudaSuccess
+             ? FS_OK
+             : FS_ERR_CUDA;
+}
+
+fs_status fs_ipc_close(void *area) {
+  if (area == nullptr) return FS_OK;
+  return cudaIpcCloseMemHandle(area) == cudaSuccess ? FS_OK : FS_ERR_CUDA;
+}
+
+fs_status fs_sample_tp(const void *H, const void *W_shard, int B, int d, int V_shard,
+                       int vocab_offset, int V_total, float temperature, uint64_t seed,
+                       const uint64_t *row_seeds, uint32_t step, const uint32_t *mask_bits,
+                       void *const *areas, int world, uint32_t seq, void *workspace,
+                       size_t workspace_bytes, fs_stream_t stream) {
+  static int32_t unused;  // the tokens go to the exchange areas
+  fs_status s = validate(H, W_shard, B, d, V_shard, temperature, &unused);
+  if (s != FS_OK) return s;
+  if (B > fmms::kMaxBN) return FS_ERR_UNSUPPORTED;
+  if (vocab_offset < 0 || (vocab_offset % fmms::kGranule) != 0 || V_total < 1 ||
+      static_cast<int64_t>(vocab_offset) + V_shard > V_total)
+    return FS_ERR_INVALID_ARG;
+  if (areas == nullptr || world < 1 || world > fmms::kMaxTpWorld) return FS_ERR_INVALID_ARG;
+  for (int r = 0; r < world; ++r)
+    if (areas[r] == nullptr || (reinterpret_cast<uintptr_t>(areas[r]) & 255) != 0)
+      return FS_ERR_INVALID_ARG;
+  ShardOpts opts;
+  opts.vocab_offset = vocab_offset;
+  opts.V_total = V_total;
+  opts.tp_world = world;
+  opts.tp_seq = seq;
+  opts.tp_areas = areas;
+  std::lock_guard<std::mutex> lock(g_mu);
+  return run_locked(fmms::kModeFlat, H, W_shard, B, d, V_shard, 1, temperature, seed, row_seeds,
+                    step, mask_bits, &unused, nullptr, nullptr, workspace, workspace_bytes,
+                    static_cast<cudaStream_t>(stream), opts);
+}
+
+fs_status fs_tp_wait(const void *area, int B, uint32_t seq, int32_t *out_idx,
+                     fs_stream_t stream) {
+  if (area == nullptr || out_idx == nullptr || B < 1 || B > fmms::kMaxBN)
+    return FS_ERR_INVALID_ARG;
+  const StreamWaitValue32Fn wait = wait_value_fn();
+  if (wait == nullptr) return FS_ERR_UNSUPPORTED;
+  const fmms::TpArea *a = static_cast<const fmms::TpArea *>(area);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (wait(reinterpret_cast<CUstream>(st), reinterpret_cast<CUdeviceptr>(&a->flag), seq + 1u,
+           CU_STREAM_WAIT_VALUE_GEQ) != CUDA_SUCCESS)
+    return FS_ERR_CUDA;
+  if (cudaMemcpyAsync(out_idx, a->tokens[seq & 1u], static_cast<size_t>(B) * 4,
+                      cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return FS_ERR_CUDA;
+  return FS_OK;
+}
+
+fs_status fs_tp_failed(const void *area, uint32_t *failed) {
+  if (area == nullptr || failed == nullptr) return FS_ERR_INVALID_ARG;
+  const fmms::TpArea *a = static_cast<const fmms::TpArea *>(area);
+  return cudaMemcpy(failed, &a->failed, 4, cudaMemcpyDeviceToHost) == cudaSuccess ? FS_OK
+                                                                                 : FS_ERR_CUDA;
 }
 
 fs_status fs_sample_multi(const void *H, const void *W, int B, int d, int V, int num_samples,

@@ -180,6 +180,29 @@ struct __align__(16) GroupPartial {
 
 enum Mode { kModeFlat = 0, kModeGrouped = 1, kModeLogits = 2 };
 
+// Fused vocabulary-parallel exchange.  Each rank of a tensor-parallel group
+// owns one exchange area in its own device memory; every rank's kernel maps
+// all of them (its own and its peers', over NVLink).  Calls are numbered by a
+// sequence number seq, the same on every rank; seq & 1 selects the half of
+// the area a call uses, so a rank one call ahead never touches the half
+// still being decoded.  Per call, the last CTA of each rank's kernel raises
+// every area's keys to its rows' packed maxima, then counts itself in every
+// area's arrivals; the arrival that completes an area decodes its keys into
+// its tokens, clears the keys and the count, and sets its flag to seq + 1.
+// No kernel waits for another: the stream that needs the tokens waits on the
+// flag (a stream memory operation).
+constexpr int kMaxTpWorld = 16;
+struct TpArea {
+  unsigned int arrivals[2];  // ranks counted in, per parity
+  unsigned int err[2];       // set by a rank whose kernel recorded a device error
+  unsigned int flag;         // seq + 1 of the last call decoded into tokens
+  unsigned int failed;       // seq + 1 of the last call decoded with an error
+  unsigned int pad[2];
+  unsigned long long keys[2][kMaxBN];
+  int tokens[2][kMaxBN];     // -1 for every row of a call with an error
+};
+constexpr size_t kTpAreaBytes = (sizeof(TpArea) + 255) / 256 * 256;
+
 struct FmmsParams {
   int B;            // rows in this launch (<= BN)
   int b_off;        // global index of this launch's row 0 (noise, mask, seeds)
@@ -212,6 +235,11 @@ struct FmmsParams {
   const uint32_t *h_ready;
   uint32_t h_epoch;
   int h_chunk_subs;
+  // Fused vocabulary-parallel exchange (flat mode): tp_world > 0 replaces the
+  // token output; tp_area[r] is rank r's exchange area, mapped here.
+  int tp_world;
+  uint32_t tp_seq;
+  TpArea *tp_area[kMaxTpWorld];
 };
 
 // Workspace layout (bytes), fixed so that calls of different kinds can share

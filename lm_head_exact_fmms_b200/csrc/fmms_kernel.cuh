@@ -342,6 +342,57 @@ __device__ __forceinline__ bool chunk_any_candidate(const uint32_t (&acc)[CW],
   return __any_sync(0xffffffffu, any);
 }
 
+// Fused vocabulary-parallel exchange, run by the epilogue threads of the
+// last CTA of a rank's kernel (see TpArea): raise every rank's area to this
+// rank's per-row maxima, count this rank in every area, and decode each area
+// whose count this arrival completed.  `dec` is a shared-memory word;
+// `failed`: some CTA of this call gave up on a bounded wait.
+__device__ __forceinline__ void tp_exchange(const FmmsParams &p, int etid, int *dec, bool failed) {
+  const int world = p.tp_world;
+  const uint32_t par = p.tp_seq & 1u;
+  if (etid == 0) *dec = 0;
+  for (int i = etid; i < world * p.B; i += kEpiThreads) {
+    const int q = i / p.B;
+    const int b = i - q * p.B;
+    const unsigned long long kb = __ldcg(p.keys + b);
+    if (key_valid(kb)) atomicMax(&p.tp_area[q]->keys[par][b], kb);
+  }
+  if (failed)
+    for (int q = etid; q < world; q += kEpiThreads) atomicOr(&p.tp_area[q]->err[par], 1u);
+  __threadfence_system();
+  sm100::epi_sync(kEpiThreads);
+  for (int b = etid; b < p.B; b += kEpiThreads) p.keys[b] = 0ull;  // for this rank's next call
+  if (etid < world) {
+    __threadfence_system();
+    const unsigned old = atomicAdd(&p.tp_area[etid]->arrivals[par], 1u);
+    if (old == static_cast<unsigned>(world - 1)) atomicOr(dec, 1 << etid);
+  }
+  if (etid == 0) atomicExch(p.ticket, 0u);
+  sm100::epi_sync(kEpiThreads);
+  const int mine = *dec;
+  for (int q = 0; q < world; ++q) {
+    if (!((mine >> q) & 1)) continue;  // uniform across the CTA
+    TpArea *a = p.tp_area[q];
+    __threadfence_system();
+    const bool bad = atomicAdd(&a->err[par], 0u) != 0u;
+    for (int b = etid; b < p.B; b += kEpiThreads) {
+      const unsigned long long kb = atomicExch(&a->keys[par][b], 0ull);
+      a->tokens[par][b] = bad ? -1 : key_token(kb);
+    }
+    __threadfence_system();
+    sm100::epi_sync(kEpiThreads);
+    if (etid == 0) {
+      atomicExch(&a->arrivals[par], 0u);
+      if (bad) {
+        atomicExch(&a->err[par], 0u);
+        atomicExch(&a->failed, p.tp_seq + 1u);
+      }
+      __threadfence_system();
+      sm100::st_release_sys(&a->flag, p.tp_seq + 1u);
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Roles
 // ---------------------------------------------------------------------------
@@ -723,17 +774,30 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
 
   if constexpr (MODE == kModeFlat) {
     // Every maximum is already published; take a ticket, and the last CTA
-    // decodes the keys and re-zeroes them for the next call.
+    // decodes the keys and re-zeroes them for the next call.  With the fused
+    // exchange an aborted CTA counts itself too (in the ticket's high half),
+    // so that the exchange still completes, marked as failed, and no peer's
+    // stream waits forever.
     __threadfence();
     sm100::epi_sync(kEpiThreads);
     if (etid == 0) {
       int last = 0;
-      if (!*abort_flag)
+      if (p.tp_world > 0) {
+        const unsigned inc = *abort_flag ? 0x10000u : 1u;
+        const unsigned old = atomicAdd(p.ticket, inc);
+        const unsigned failed = (old >> 16) + (inc >> 16);
+        if ((old & 0xFFFFu) + (old >> 16) + 1u == static_cast<unsigned>(p.num_ctas))
+          last = failed ? 2 : 1;
+      } else if (!*abort_flag) {
         last = (atomicAdd(p.ticket, 1u) == static_cast<unsigned>(p.num_ctas - 1)) ? 1 : 0;
+      }
       *last_flag = last;
     }
     sm100::epi_sync(kEpiThreads);
-    if (*last_flag) {
+    if (*last_flag && p.tp_world > 0) {
+      __threadfence();
+      tp_exchange(p, etid, last_flag + 1, *last_flag == 2);
+    } else if (*last_flag) {
       __threadfence();
       const int total = p.B * p.num_samples;
       for (int i = etid; i < total; i += kEpiThreads) {
@@ -771,7 +835,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *drain_bar = acc_empty + C::kAccBufs;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain_bar + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-  int *last_flag = reinterpret_cast<int *>(tmem_slot + 2);
+  int *last_flag = reinterpret_cast<int *>(tmem_slot + 2);  // tmem_slot + 3: exchange word
   uint8_t *comb = reinterpret_cast<uint8_t *>(bars) + C::kBarBytes;
   uint64_t *comb_key = reinterpret_cast<uint64_t *>(comb);
   float *comb_m = reinterpret_cast<float *>(comb_key + 4 * BN);

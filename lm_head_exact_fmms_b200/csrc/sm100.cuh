@@ -96,6 +96,12 @@ __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity,
   }
 }
 
+// Store with release semantics at system scope (a flag that another GPU's
+// stream, or the host, waits on after the data it guards).
+__device__ __forceinline__ void st_release_sys(unsigned int *addr, unsigned int v) {
+  asm volatile("st.release.sys.u32 [%0], %1;" ::"l"(addr), "r"(v) : "memory");
+}
+
 // Waits until *flag == value (written by a copy engine after a host-to-device
 // copy), with the same time limit as wait_bounded; then orders the TMA loads
 // that follow (async proxy) after the observation.

@@ -3,12 +3,18 @@
 The LM head's vocabulary rows are split over the ranks of a process group;
 each rank samples its shard with global token indices (so noise, mask and
 tie-breaking are those of the full head), producing one packed
-(score, token) key per row, and a single int64 MAX all-reduce of 8 bytes per
-row picks the winner (readus.org page, "distributed FlashSampling": each GPU
-is one group and sends only its winning index and score; abstract: argmax
-decomposes over a partition).  The tokens equal single-GPU sampling bit for
-bit.  torch.distributed (NCCL) carries the exchange; the sampling itself runs
-in the library's kernels.
+(score, token) key per row, and the maximum over ranks picks the winner
+(readus.org page, "distributed FlashSampling": each GPU is one group and
+sends only its winning index and score; abstract: argmax decomposes over a
+partition).  The tokens equal single-GPU sampling bit for bit.
+
+Two ways to exchange the keys:
+  * FusedExchange: the kernel's last CTA writes the keys straight into every
+    rank's exchange area over NVLink and the rank completing an area decodes
+    it (fs_sample_tp); the stream then waits on the area's flag.  Only the
+    IPC handles of the areas go through torch.distributed, once.
+  * tp_sample: an int64 MAX all-reduce of 8 bytes per row through
+    torch.distributed (NCCL) after the kernel, then a decode kernel.
 """
 import torch
 import torch.distributed as dist
@@ -43,3 +49,86 @@ def tp_sample(H, W_shard, vocab_offset, V_total, temperature=1.0, seed=0, row_se
                                         stream=stream)
     reduce_keys(keys, group)
     return binding.fs_keys_to_tokens(keys, stream=stream)
+
+
+def exchange_handles(handle, group=None):
+    """All ranks' IPC handles (bytes), in rank order, via an all-gather."""
+    world = dist.get_world_size(group)
+    out = [None] * world
+    dist.all_gather_object(out, bytes(handle), group=group)
+    return out
+
+
+class FusedExchange:
+    """The exchange areas of a process group for fs_sample_tp: this rank's
+    own area and its peers', mapped here by CUDA IPC.  Every rank calls
+    sample() in the same order (the call sequence number is kept here)."""
+
+    def __init__(self, group=None):
+        self.group = group
+        self.rank = dist.get_rank(group)
+        self.world = dist.get_world_size(group)
+        self.mine = binding.fs_tp_area_create()
+        handles = exchange_handles(binding.fs_ipc_handle(self.mine), group)
+        self._opened = []
+        self.areas = []
+        for r, h in enumerate(handles):
+            if r == self.rank:
+                self.areas.append(self.mine)
+            else:
+                a = binding.fs_ipc_open(h)
+                self._opened.append(a)
+                self.areas.append(a)
+        self.seq = 0
+
+    def sample(self, H, W_shard, vocab_offset, V_total, temperature=1.0, seed=0, row_seeds=None,
+               step=0, mask_bits=None, out_idx=None, workspace=None, stream=None):
+        """Samples B <= 256 rows of the sharded head; every rank gets all tokens."""
+        binding.fs_sample_tp(H, W_shard, vocab_offset, V_total, self.areas, self.seq, temperature,
+                             seed, row_seeds, step, mask_bits, workspace=workspace, stream=stream)
+        out = binding.fs_tp_wait(self.mine, H.shape[0], self.seq, out_idx, device=H.device,
+                                 stream=stream)
+        self.seq += 1
+        return out
+
+    def close(self):
+        """Unmaps the peers' areas and frees this rank's, once every rank is
+        done with the exchange."""
+        torch.cuda.synchronize()
+        dist.barrier(group=self.group)
+        for a in self._opened:
+            binding.fs_ipc_close(a)
+        self._opened = []
+        dist.barrier(group=self.group)
+        binding.fs_tp_area_destroy(self.mine)
+        self.mine = None
+
+
+class LocalExchange:
+    """`world` shards on one GPU, each with its own exchange area in this
+    process: the same kernels and protocol as FusedExchange, with the ranks'
+    calls issued one after another on one stream (no call waits for a later
+    one, so nothing waits for a kernel that has not run)."""
+
+    def __init__(self, world):
+        self.world = world
+        self.areas = [binding.fs_tp_area_create() for _ in range(world)]
+        self.seq = 0
+
+    def sample(self, H, shards, V_total, temperature=1.0, seed=0, row_seeds=None, step=0,
+               mask_bits=None, workspaces=None, stream=None):
+        """shards: [(W_shard, vocab_offset)] per rank.  Returns each rank's tokens."""
+        for r, (Ws, off) in enumerate(shards):
+            ws = workspaces[r] if workspaces is not None else None
+            binding.fs_sample_tp(H, Ws, off, V_total, self.areas, self.seq, temperature, seed,
+                                 row_seeds, step, mask_bits, workspace=ws, stream=stream)
+        outs = [binding.fs_tp_wait(a, H.shape[0], self.seq, device=H.device, stream=stream)
+                for a in self.areas]
+        self.seq += 1
+        return outs
+
+    def close(self):
+        torch.cuda.synchronize()
+        for a in self.areas:
+            binding.fs_tp_area_destroy(a)
+        self.areas = []

@@ -424,6 +424,76 @@ def test_vocab_shards_equal_single_gpu(dev, world, B):
         assert torch.equal(got, ref)
 
 
+@pytest.mark.parametrize("world,B", [(1, 5), (2, 8), (3, 64), (5, 200), (8, 256)])
+def test_fused_exchange_equals_single_gpu(dev, world, B):
+    """fs_sample_tp on `world` shards of the head, each with its own exchange
+    area (all on this GPU, the ranks' calls one after another on one stream):
+    every rank's tokens equal single-GPU sampling bit for bit, over five calls
+    so that both halves of the areas are used and cleared more than once."""
+    from lm_head_exact_fmms_b200.tp import LocalExchange, shard_bounds
+    d, V = 256, 30011
+    H, W, Hd, Wd = rand_inputs(B, d, V, seed=world * 11 + B)
+    rs = synth.make_row_seeds(B).to(dev)
+    mask = synth.make_mask(B, V, 0.5, seed=world + 1).to(dev)
+    shards = [(Wd[lo:hi].contiguous(), lo) for lo, hi in shard_bounds(V, world)]
+    ex = LocalExchange(world)
+    try:
+        for step in range(5):
+            ref = binding.fs_sample_ex(Hd, Wd, temperature=0.9, seed=4, row_seeds=rs, step=step,
+                                       mask_bits=mask)
+            outs = ex.sample(Hd, shards, V, temperature=0.9, seed=4, row_seeds=rs, step=step,
+                             mask_bits=mask)
+            for r, o in enumerate(outs):
+                assert torch.equal(o, ref), (step, r)
+        assert all(binding.fs_tp_failed(a) == 0 for a in ex.areas)
+    finally:
+        ex.close()
+
+
+def test_fused_exchange_marks_a_failed_call(dev):
+    """One rank's kernel gives up on its bounded waits (test switch: no loads
+    issued): it still completes the exchange, marked as failed, so no rank's
+    wait hangs; every rank gets -1 for every row of that call, the areas
+    report it, the failing rank's workspace reports the timeout, and the next
+    call is correct again."""
+    from lm_head_exact_fmms_b200.tp import LocalExchange, shard_bounds
+    world, B, d, V = 3, 16, 128, 9001
+    H, W, Hd, Wd = rand_inputs(B, d, V, seed=91)
+    bounds = shard_bounds(V, world)
+    shards = [(Wd[lo:hi].contiguous(), lo) for lo, hi in bounds]
+    wss = [torch.zeros(binding.fs_workspace_bytes(B, hi - lo, 0), dtype=torch.uint8, device=dev)
+           for lo, hi in bounds]
+    ex = LocalExchange(world)
+    try:
+        for call in range(3):
+            for r, (Ws, off) in enumerate(shards):
+                stall = call == 1 and r == 1
+                if stall:
+                    binding.fs_test_stall_loads(True)
+                try:
+                    binding.fs_sample_tp(Hd, Ws, off, V, ex.areas, ex.seq, temperature=1.0, seed=2,
+                                         step=call, workspace=wss[r])
+                finally:
+                    if stall:
+                        binding.fs_test_stall_loads(False)
+            outs = [binding.fs_tp_wait(a, B, ex.seq, device=dev) for a in ex.areas]
+            ex.seq += 1
+            torch.cuda.synchronize()
+            if call == 1:
+                for o in outs:
+                    assert (o == -1).all()
+                assert [binding.fs_tp_failed(a) for a in ex.areas] == [2] * world
+                assert binding.fs_device_status(wss[1]) == 5  # FS_ERR_DEVICE_TIMEOUT
+                assert binding.fs_device_status(wss[0]) == 0
+            else:
+                ref = binding.fs_sample_ex(Hd, Wd, temperature=1.0, seed=2, step=call)
+                for o in outs:
+                    assert torch.equal(o, ref)
+    finally:
+        binding.fs_test_stall_loads(False)
+        ex.close()
+
+
 # ----------------------------------------------------- several samples per row
 @pytest.mark.parametrize("B,d,V,S", [(1, 64, 4096, 8), (17, 96, 3001, 3), (64, 128, 9000, 4),
                                      (300, 64, 2048, 2)])

@@ -104,3 +104,34 @@ def test_two_rank_exchange_matches_flat_oracle(oracle, world):
     for r in range(world):
         assert results[r] == flat.tolist()
     assert flat[1] == -1 and flat[2] == V - 1
+
+
+def _handles_rank(rank, world, port, results):
+    import torch.distributed as dist
+    from lm_head_exact_fmms_b200.tp import exchange_handles
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    mine = bytes([rank + 1]) * 64
+    results[rank] = exchange_handles(mine)
+    dist.destroy_process_group()
+
+
+def test_exchange_handles_in_rank_order():
+    """The fused exchange's only host collective: every rank receives every
+    rank's 64-byte IPC handle, in rank order (gloo, three ranks)."""
+    world = 3
+    ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    results = mgr.dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_handles_rank, args=(r, world, port, results))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    want = [bytes([r + 1]) * 64 for r in range(world)]
+    for r in range(world):
+        assert list(results[r]) == want
