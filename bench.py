@@ -44,8 +44,12 @@ def parse_args():
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--tp", action="store_true",
-                    help="split the vocabulary across the ranks (one int64 MAX all-reduce of "
-                         "8 bytes per row per step) instead of running independent replicas")
+                    help="split the vocabulary across the ranks instead of running independent "
+                         "replicas; the kernels exchange the per-row keys through each other's "
+                         "memory (fs_sample_tp)")
+    ap.add_argument("--tp-nccl", action="store_true",
+                    help="with --tp: exchange the keys with an int64 MAX all-reduce (NCCL) after "
+                         "the kernel instead")
     return ap.parse_args()
 
 
@@ -320,14 +324,21 @@ def run_gpu(args, world, rank, local):
         W = W_full[lo:hi].contiguous()
         del W_full
         torch.cuda.empty_cache()
-        keys = torch.empty(B, dtype=torch.int64, device=dev)
+        if args.tp_nccl or B > 256:
+            keys = torch.empty(B, dtype=torch.int64, device=dev)
 
-        def step(i):
-            binding.fs_sample_shard_keys(H, W, lo, wl.V, temperature=wl.temperature, seed=0,
-                                         row_seeds=rs, step=i, out_keys=keys, workspace=ws,
-                                         stream=stream)
-            tpmod.reduce_keys(keys)
-            binding.fs_keys_to_tokens(keys, out_idx=out, stream=stream)
+            def step(i):
+                binding.fs_sample_shard_keys(H, W, lo, wl.V, temperature=wl.temperature, seed=0,
+                                             row_seeds=rs, step=i, out_keys=keys, workspace=ws,
+                                             stream=stream)
+                tpmod.reduce_keys(keys)
+                binding.fs_keys_to_tokens(keys, out_idx=out, stream=stream)
+        else:
+            exchange = tpmod.FusedExchange()
+
+            def step(i):
+                exchange.sample(H, W, lo, wl.V, temperature=wl.temperature, seed=0, row_seeds=rs,
+                                step=i, out_idx=out, workspace=ws, stream=stream)
     elif grouped:
         def step(i):
             binding.fs_sample_grouped(H, W, wl.groups, temperature=wl.temperature, seed=0,
@@ -346,7 +357,8 @@ def run_gpu(args, world, rank, local):
     us_per_call = region_ms * 1e3 / args.steps
     nbytes, flops = algorithmic(B, wl.d, wl.V, mask is not None)
     # fused kernel per 256 rows, plus the group merge (grouped) or the decode (tp)
-    launches_per_call = (B + 255) // 256 * (2 if grouped else 1) + (1 if tp else 0)
+    fused_tp = tp and not (args.tp_nccl or B > 256)
+    launches_per_call = (B + 255) // 256 * (2 if grouped else 1) + (1 if tp and not fused_tp else 0)
     if tp:
         # each rank streams its shard; the roofline below is per rank
         nbytes = nbytes * W.shape[0] // wl.V
@@ -382,7 +394,9 @@ def run_gpu(args, world, rank, local):
                                   if grouped else "",
                                   "fs_sample_grouped" if grouped else "fs_sample_ex"),
                    "batch_per_gpu": B, "global_batch": B * world, "d": wl.d, "V": wl.V,
-                   "parallelism": ("tensor-parallel vocabulary x%d" % world) if tp
+                   "parallelism": ("tensor-parallel vocabulary x%d (%s)" % (
+                       world, "fused peer-memory exchange" if fused_tp else "NCCL all-reduce"))
+                   if tp
                    else ("replicas x%d" % world),
                    "l2": "no flush: W (%.2f GB) exceeds the 126 MB L2" % (wl.V * wl.d * 2 / 1e9)},
         "samples_per_s": round(B * world / (us_per_call * 1e-6), 1),
@@ -407,6 +421,8 @@ def run_gpu(args, world, rank, local):
         result["top_k"] = topk_point(torch, binding, synth, W, wl, dev, stream, B)
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not grouped:
         result["cpu_baseline"] = cpu_baseline(H, W, wl, B, rs)
+    if fused_tp:
+        exchange.close()  # every rank, after its last call
     return result
 
 
