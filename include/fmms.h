@@ -303,9 +303,10 @@ fs_status fs_sample_topk(const void *H, const void *W, int B, int d, int V,
 /* End-to-end call with HOST buffers: H_host (bf16 [B, d]) and out_idx_host
  * (int32 [B]) are host pointers (page-locked for the copies to be
  * asynchronous); W and row_seeds/mask_bits stay device pointers.  Enqueues
- * the host-to-device copy of H into a library-owned device buffer on a
- * library stream (after the previous fs_sample_host call's kernel, which
- * reads that buffer), the fused sample on `stream` (it starts streaming W at
+ * the host-to-device copy of H into one of two library-owned device buffers,
+ * used by alternate calls, on a library stream (after the kernel of the call
+ * two back, which read that buffer; so the copy overlaps the previous
+ * call's kernel), the fused sample on `stream` (it starts streaming W at
  * once and waits on the device, with the usual one-second limit, for the
  * copy of H to land), and the tokens: written by the kernel straight into
  * out_idx_host when it is page-locked, else copied from a device buffer on

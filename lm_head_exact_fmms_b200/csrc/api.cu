@@ -25,22 +25,25 @@ struct DeviceState {
   int cc_major = 0;
   void *ws = nullptr;       // library-owned workspace
   size_t ws_bytes = 0;
-  void *h_stage = nullptr;  // fs_sample_host: device copy of H
-  size_t h_stage_bytes = 0;
+  void *h_stage[2] = {nullptr, nullptr};  // fs_sample_host: device copies of H, by call parity
+  size_t h_stage_bytes[2] = {0, 0};
   void *o_stage = nullptr;  // fs_sample_host: device tokens
   size_t o_stage_bytes = 0;
   void *topk_scratch = nullptr;  // fs_sample_topk: per-block candidate lists and counts
   size_t topk_scratch_bytes = 0;
   // fs_sample_host: H is copied on copy_stream while the kernel already
-  // streams W; h_flags takes the call's epoch once the copy has landed.
-  // kernel_done keeps the next call's copy off h_stage until this call's
-  // kernel has finished with it.
+  // streams W; h_flags[k] takes the call's epoch once the copy into
+  // h_stage[k] has landed.  Calls alternate between the two buffers, and
+  // kernel_done[k] keeps a copy off h_stage[k] until the kernel that last
+  // read it (two calls back) has finished, so a call's copy runs during the
+  // previous call's kernel.
   bool host_overlap_init = false;
   bool host_overlap = false;
   cudaStream_t copy_stream = nullptr;
-  cudaEvent_t kernel_done = nullptr;
-  uint32_t *h_flags = nullptr;  // device word: epoch of the H copy that has landed
+  cudaEvent_t kernel_done[2] = {nullptr, nullptr};
+  uint32_t *h_flags = nullptr;  // device words [2]: epoch of the H copy that has landed
   uint32_t h_epoch = 0;
+  uint32_t h_calls = 0;
   int pair_units[2][fmms::kMaxBN / 16];  // resident CTA pairs [flat, grouped][tile / 16 - 1]; -1: unknown
   DeviceState() {
     for (auto &row : pair_units)
@@ -483,9 +486,10 @@ fs_status fs_sample_host(const void *H_host, const void *W, int B, int d, int V,
   fs_status s = get_device(&st);
   if (s != FS_OK) return s;
   const size_t hbytes = static_cast<size_t>(B) * d * 2;
-  if ((s = grow(&st->h_stage, &st->h_stage_bytes, hbytes)) != FS_OK) return s;
+  const int hb = static_cast<int>(st->h_calls++ & 1u);
+  if ((s = grow(&st->h_stage[hb], &st->h_stage_bytes[hb], hbytes)) != FS_OK) return s;
   if ((s = grow(&st->o_stage, &st->o_stage_bytes, static_cast<size_t>(B) * 4)) != FS_OK) return s;
-  char *hdev = static_cast<char *>(st->h_stage);
+  char *hdev = static_cast<char *>(st->h_stage[hb]);
   int32_t *odev = static_cast<int32_t *>(st->o_stage);
 
   if (!st->host_overlap_init) {
@@ -493,31 +497,35 @@ fs_status fs_sample_host(const void *H_host, const void *W, int B, int d, int V,
     st->host_overlap =
         write_value_fn() != nullptr &&
         cudaStreamCreateWithFlags(&st->copy_stream, cudaStreamNonBlocking) == cudaSuccess &&
-        cudaEventCreateWithFlags(&st->kernel_done, cudaEventDisableTiming) == cudaSuccess &&
-        cudaMalloc(&st->h_flags, sizeof(uint32_t)) == cudaSuccess &&
-        cudaMemset(st->h_flags, 0, sizeof(uint32_t)) == cudaSuccess &&
+        cudaEventCreateWithFlags(&st->kernel_done[0], cudaEventDisableTiming) == cudaSuccess &&
+        cudaEventCreateWithFlags(&st->kernel_done[1], cudaEventDisableTiming) == cudaSuccess &&
+        cudaMalloc(&st->h_flags, 2 * sizeof(uint32_t)) == cudaSuccess &&
+        cudaMemset(st->h_flags, 0, 2 * sizeof(uint32_t)) == cudaSuccess &&
         cudaDeviceSynchronize() == cudaSuccess;
   }
 
   ShardOpts opts;
   if (st->host_overlap) {
-    // H is copied on the library's copy stream once the previous call's
-    // kernel is done with the staging buffer, and a copy-engine write then
-    // sets the flag to this call's epoch.  The kernel, launched at once,
-    // streams W from its start and loads H once the flag holds the epoch, so
-    // the launch and the first W loads overlap the copy.  (Copying H in
+    // H is copied on the library's copy stream into this call's staging
+    // buffer once the kernel two calls back is done with it, and a
+    // copy-engine write then sets the buffer's flag to this call's epoch.
+    // The kernel, launched at once, streams W from its start and loads H
+    // once the flag holds the epoch, so the copy overlaps the previous
+    // call's kernel and this one's first W loads.  (Copying H in
     // several K-column chunks, each with its own flag, measured slower: 2-D
     // copies of 64-row strips and the extra waits cost more than they hid.)
     const int nk = (d + fmms::kBlockK - 1) / fmms::kBlockK;
     const uint32_t epoch = ++st->h_epoch == 0 ? ++st->h_epoch : st->h_epoch;
-    if (cudaStreamWaitEvent(st->copy_stream, st->kernel_done, 0) != cudaSuccess) return FS_ERR_CUDA;
+    if (cudaStreamWaitEvent(st->copy_stream, st->kernel_done[hb], 0) != cudaSuccess)
+      return FS_ERR_CUDA;
     if (cudaMemcpyAsync(hdev, H_host, hbytes, cudaMemcpyHostToDevice, st->copy_stream) !=
         cudaSuccess)
       return FS_ERR_CUDA;
     if (write_value_fn()(reinterpret_cast<CUstream>(st->copy_stream),
-                         reinterpret_cast<CUdeviceptr>(st->h_flags), epoch, 0) != CUDA_SUCCESS)
+                         reinterpret_cast<CUdeviceptr>(st->h_flags + hb), epoch, 0) !=
+        CUDA_SUCCESS)
       return FS_ERR_CUDA;
-    opts.h_ready = st->h_flags;
+    opts.h_ready = st->h_flags + hb;
     opts.h_epoch = epoch;
     opts.h_chunk_subs = nk;
   } else {
@@ -535,7 +543,8 @@ fs_status fs_sample_host(const void *H_host, const void *W, int B, int d, int V,
   s = run_locked(fmms::kModeFlat, hdev, W, B, d, V, 1, temperature, seed, row_seeds, step,
                  mask_bits, out_dev, nullptr, nullptr, nullptr, 0, st_, opts);
   if (s != FS_OK) return s;
-  if (st->host_overlap && cudaEventRecord(st->kernel_done, st_) != cudaSuccess) return FS_ERR_CUDA;
+  if (st->host_overlap && cudaEventRecord(st->kernel_done[hb], st_) != cudaSuccess)
+    return FS_ERR_CUDA;
   if (!direct && cudaMemcpyAsync(out_idx_host, odev, static_cast<size_t>(B) * 4,
                                  cudaMemcpyDeviceToHost, st_) != cudaSuccess)
     return FS_ERR_CUDA;

@@ -405,6 +405,27 @@ __device__ __forceinline__ uint32_t w_sub_bytes(int rows) {
   return static_cast<uint32_t>((rows + kGranule - 1) / kGranule) * 1024u;
 }
 
+// The H loads of one stage (this CTA's rows of the batch operand).
+template <int BN, int MODE, bool PAIR>
+__device__ __forceinline__ void issue_h(const CUtensorMap *th, const FmmsParams &p,
+                                        uint8_t *stages, uint64_t *full, int stage, int sub0,
+                                        int nsub, int rank, uint64_t pol_h) {
+  using C = KCfg<BN, MODE, PAIR>;
+  uint8_t *sh0 = stages + stage * C::kStageBytes + C::kStageW;
+  const uint32_t bar = PAIR ? sm100::cluster_addr(&full[stage], 0) : 0u;
+#pragma unroll
+  for (int j = 0; j < C::kSub; ++j) {
+    if (j >= nsub) break;
+    uint8_t *sh = sh0 + j * C::kSubH;
+    const int x = (sub0 + j) * kBlockK;
+    if constexpr (PAIR) {
+      sm100::tma_load_2d_pair(sh, th, bar, x, p.b_off + rank * C::kHRows, pol_h);
+    } else {
+      sm100::tma_load_2d(sh, th, &full[stage], x, p.b_off, pol_h);
+    }
+  }
+}
+
 // TMA producer (one thread).  In pair mode both CTAs load their own half of
 // every stage (128 W rows, BN/2 H rows) and count the bytes on the even
 // CTA's full barrier; the even CTA also hands each freed stage on to the odd
@@ -424,6 +445,11 @@ __device__ __forceinline__ void role_producer(const CUtensorMap *tw, const CUten
   uint32_t phase = 0;
   long long issued = 0;
   int h_chunks_ready = -1;  // chunks of H known to have arrived (h_ready mode)
+  // h_ready mode: stages whose W loads went out while the copy of H was still
+  // in flight; their H loads follow once it has landed, so the ring fills
+  // with W during the copy instead of stopping at the first stage.
+  int pend_stage[C::kStages], pend_sub0[C::kStages], pend_nsub[C::kStages];
+  int npend = 0, pend_need = 0;
   bool ok = p.test_no_loads == 0;
   while (ok && it.next(tile)) {
     const Tile mine = PAIR ? pair_half(tile, rank) : tile;
@@ -447,7 +473,6 @@ __device__ __forceinline__ void role_producer(const CUtensorMap *tw, const CUten
       if (PAIR && rank == 0 && issued >= C::kStages)
         sm100::mbar_arrive_cluster(sm100::cluster_addr(&empty[stage], 1));
       uint8_t *sw0 = stages + stage * C::kStageBytes;
-      uint8_t *sh0 = sw0 + C::kStageW;
       if (!PAIR || rank == 0) sm100::mbar_arrive_expect_tx(&full[stage], bytes);
       const uint32_t bar = PAIR ? sm100::cluster_addr(&full[stage], 0) : 0u;
       // W first: it never waits for H.
@@ -474,34 +499,53 @@ __device__ __forceinline__ void role_producer(const CUtensorMap *tw, const CUten
           }
         }
       }
-      // H still arriving from the host: wait for the chunk this stage ends in.
+      // H still arriving from the host: until the chunk this stage ends in
+      // is known to have landed, defer the stage's H loads while free stages
+      // remain; then wait for it and issue every deferred H load.
+      bool h_now = true;
       if (p.h_ready != nullptr) {
         const int need = (sub0 + nsub - 1) / p.h_chunk_subs;
         if (need > h_chunks_ready) {
-          if (!sm100::wait_flag_bounded(p.h_ready + need, p.h_epoch, abort_flag, p.err)) {
-            ok = false;
-            break;
+          pend_stage[npend] = stage;
+          pend_sub0[npend] = sub0;
+          pend_nsub[npend] = nsub;
+          pend_need = need;
+          ++npend;
+          h_now = false;
+          if (npend == C::kStages || sm100::flag_is(p.h_ready + need, p.h_epoch)) {
+            const bool landed =
+                sm100::wait_flag_bounded(p.h_ready + need, p.h_epoch, abort_flag, p.err);
+            h_chunks_ready = need;
+            // After a timeout too: the loads stay in bounds, and completing
+            // the stages lets the drain below account for every copy.
+            for (int q = 0; q < npend; ++q)
+              issue_h<BN, MODE, PAIR>(th, p, stages, full, pend_stage[q], pend_sub0[q],
+                                      pend_nsub[q], rank, pol_h);
+            npend = 0;
+            if (!landed) {
+              ok = false;
+              ++issued;
+              break;
+            }
           }
-          h_chunks_ready = need;
         }
       }
-#pragma unroll
-      for (int j = 0; j < C::kSub; ++j) {
-        if (j >= nsub) break;
-        uint8_t *sh = sh0 + j * C::kSubH;
-        const int x = (sub0 + j) * kBlockK;
-        if constexpr (PAIR) {
-          sm100::tma_load_2d_pair(sh, th, bar, x, p.b_off + rank * C::kHRows, pol_h);
-        } else {
-          sm100::tma_load_2d(sh, th, &full[stage], x, p.b_off, pol_h);
-        }
-      }
+      if (h_now) issue_h<BN, MODE, PAIR>(th, p, stages, full, stage, sub0, nsub, rank, pol_h);
       ++issued;
       if (++stage == C::kStages) {
         stage = 0;
         phase ^= 1u;
       }
     }
+  }
+  if (ok && npend > 0) {
+    // The CTA's last stages are still waiting for H (a range shorter than the ring).
+    const bool landed = sm100::wait_flag_bounded(p.h_ready + pend_need, p.h_epoch, abort_flag, p.err);
+    for (int q = 0; q < npend; ++q)
+      issue_h<BN, MODE, PAIR>(th, p, stages, full, pend_stage[q], pend_sub0[q], pend_nsub[q], rank,
+                              pol_h);
+    npend = 0;
+    ok = landed;
   }
   if (!ok && issued > 0 && (!PAIR || rank == 0)) {
     // Gave up: let the copies already in flight land before the CTA exits.

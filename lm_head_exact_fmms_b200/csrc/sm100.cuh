@@ -102,6 +102,13 @@ __device__ __forceinline__ void st_release_sys(unsigned int *addr, unsigned int 
   asm volatile("st.release.sys.u32 [%0], %1;" ::"l"(addr), "r"(v) : "memory");
 }
 
+// One acquire load: whether *flag == value already.
+__device__ __forceinline__ bool flag_is(const uint32_t *flag, uint32_t value) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+  return v == value;
+}
+
 // Waits until *flag == value (written by a copy engine after a host-to-device
 // copy), with the same time limit as wait_bounded; then orders the TMA loads
 // that follow (async proxy) after the observation.

@@ -242,6 +242,29 @@ def test_host_entry_point_back_to_back(dev):
     assert torch.equal(out, ref)
 
 
+def test_host_entry_point_full_size(dev):
+    """fs_sample_host on the Qwen3-8B-shaped head (many stages per CTA, so the
+    ring fills with W while H is still being copied): the tokens of
+    fs_sample_ex on the same H, over consecutive calls."""
+    wl = synth.WORKLOADS["qwen3-8b"]
+    Wd = synth.make_weight(wl.V, wl.d, wl.w_std, device=dev)
+    rs = synth.make_row_seeds(64).to(dev)
+    try:
+        for i, B in enumerate([64, 1, 200]):
+            H = synth.make_hidden(B, wl.d, device="cpu", seed=300 + i).pin_memory()
+            out = torch.empty(B, dtype=torch.int32).pin_memory()
+            rsb = synth.make_row_seeds(B).to(dev)
+            binding.fs_sample_host(H, Wd, temperature=0.7, seed=0, row_seeds=rsb, step=i,
+                                   out_idx_host=out)
+            torch.cuda.synchronize()
+            ref = binding.fs_sample_ex(H.to(dev), Wd, temperature=0.7, seed=0, row_seeds=rsb,
+                                       step=i).cpu()
+            assert torch.equal(out, ref), B
+    finally:
+        del Wd
+        torch.cuda.empty_cache()
+
+
 def test_gumbel_max_is_softmax_on_gpu(dev, oracle):
     """Draws of identical rows (noise differs per row index) follow the exact
     softmax of l / T (chi-square)."""
