@@ -193,8 +193,15 @@ __device__ __forceinline__ T transpose_reduce(T (&k)[CW], int lane) {
   return k[0];
 }
 
-// Folds (m2, s2) into the running log-sum-exp pieces (m, s): sum exp(x - m) = s.
-__device__ __forceinline__ void lse_merge(float &m, float &s, float m2, float s2) {
+// 2^x with the hardware's approximate base-2 exponential (2^-inf = 0).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// lse_merge in base 2: sum 2^(x2 - m) = s, for x2 = x log2(e).
+__device__ __forceinline__ void lse2_merge(float &m, float &s, float m2, float s2) {
   if (m2 == -INFINITY) return;
   if (m == -INFINITY) {
     m = m2;
@@ -202,7 +209,7 @@ __device__ __forceinline__ void lse_merge(float &m, float &s, float m2, float s2
     return;
   }
   const float mx = fmaxf(m, m2);
-  s = s * __expf(m - mx) + s2 * __expf(m2 - mx);
+  s = s * ex2_approx(m - mx) + s2 * ex2_approx(m2 - mx);
   m = mx;
 }
 
@@ -297,26 +304,54 @@ __device__ __forceinline__ void chunk_keys(const uint32_t (&acc)[CW], const uint
   best = cmax > best ? cmax : best;
 }
 
-// Log-sum-exp pieces of the allowed x = acc / T of one chunk, folded into the
-// lane's running (m, s) of its column.
+// Log-sum-exp pieces, in base 2, of the allowed x2 = acc / T * log2(e) of one
+// chunk (c1 = log2(e) / T), folded into the lane's running (m_run, s_run) of
+// its column.  `ref` holds the running maxima of the chunk's CW columns
+// (shared memory).  When every allowed element lies at most 60 above its
+// column's running maximum, the chunk's terms are summed against those maxima
+// as they stand: no maximum reduction, no broadcast, no rescaling (the sums
+// stay below 2^75).  Otherwise (a segment's first chunk among them) the
+// chunk's column maxima are reduced and merged.
 template <int CW>
-__device__ __forceinline__ void chunk_lse(const uint32_t (&acc)[CW], const FmmsParams &p,
-                                          uint32_t allowed, int lane, float &m_run, float &s_run) {
+__device__ __forceinline__ void chunk_lse2(const uint32_t (&acc)[CW], float c1, uint32_t allowed,
+                                           const float *ref, int lane, float &m_run,
+                                           float &s_run) {
+  float r[CW];
+#pragma unroll
+  for (int j4 = 0; j4 < CW / 4; ++j4) {
+    const float4 v = reinterpret_cast<const float4 *>(ref)[j4];
+    r[4 * j4 + 0] = v.x;
+    r[4 * j4 + 1] = v.y;
+    r[4 * j4 + 2] = v.z;
+    r[4 * j4 + 3] = v.w;
+  }
+  float e[CW];
+  bool over = false;
+#pragma unroll
+  for (int j = 0; j < CW; ++j) {
+    const bool a = (allowed >> j) & 1u;
+    const float dlt = fmaf(__uint_as_float(acc[j]), c1, -r[j]);
+    over = over || (a && !(dlt <= 60.f));  // also a column with no maximum yet (+inf)
+    e[j] = a ? ex2_approx(dlt) : 0.f;
+  }
+  if (!__any_sync(0xffffffffu, over)) {
+    s_run += transpose_reduce<CW, OpAddF>(e, lane);
+    return;
+  }
   float xs[CW], t[CW];
 #pragma unroll
   for (int j = 0; j < CW; ++j) {
-    xs[j] = ((allowed >> j) & 1u) ? __uint_as_float(acc[j]) * p.inv_temp : -INFINITY;
+    xs[j] = ((allowed >> j) & 1u) ? __uint_as_float(acc[j]) * c1 : -INFINITY;
     t[j] = xs[j];
   }
   const float colmax = transpose_reduce<CW, OpMaxF>(t, lane);
-  float e[CW];
 #pragma unroll
   for (int j = 0; j < CW; ++j) {
     const float cm = __shfl_sync(0xffffffffu, colmax, lane_of_column<CW>(j));
-    e[j] = (xs[j] == -INFINITY) ? 0.f : __expf(xs[j] - cm);
+    e[j] = (xs[j] == -INFINITY) ? 0.f : ex2_approx(xs[j] - cm);
   }
   const float colsum = transpose_reduce<CW, OpAddF>(e, lane);
-  lse_merge(m_run, s_run, colmax, colsum);
+  lse2_merge(m_run, s_run, colmax, colsum);
 }
 
 // The filter: may any element of the chunk (bit set in `cand`) reach its
@@ -657,6 +692,7 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
   constexpr int CW = C::kCW;
   const int q = warp & 3;          // TMEM lane quarter this warp may access
   const int h = (warp - 2) >> 2;   // which of the quarter's warps: chunks h, h+4, ...
+  const float c1 = p.inv_temp * 1.4426950408889634f;  // log2(e) / T: base-2 log-sum-exp
   const int etid = (warp - 2) * 32 + lane;
   const bool has_chunks = h < C::kChunks;
 
@@ -754,7 +790,7 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
             const int si = q * BN + c;  // this lane's (quarter, column) state
             float m_run = comb_m[si], s_run = comb_s[si];
             uint64_t best = comb_key[si];
-            chunk_lse<CW>(acc, p, allowed, lane, m_run, s_run);
+            chunk_lse2<CW>(acc, c1, allowed, comb_m + q * BN + col0, lane, m_run, s_run);
             if (chunk_any_candidate<CW>(acc, words, p, allowed, best, pub, lane)) {
               chunk_keys<CW>(acc, words, p, vg, allowed, lane, best);
               if (gk != nullptr && (lane & 1) == 0 && c < p.B && key_valid(best) && best > pub)
@@ -798,7 +834,7 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
           for (int qq = 0; qq < 4; ++qq) {
             const uint64_t kq = comb_key[qq * BN + b];
             kb = kq > kb ? kq : kb;
-            lse_merge(m, s, comb_m[qq * BN + b], comb_s[qq * BN + b]);
+            lse2_merge(m, s, comb_m[qq * BN + b], comb_s[qq * BN + b]);
             comb_key[qq * BN + b] = 0ull;
             comb_m[qq * BN + b] = -INFINITY;
             comb_s[qq * BN + b] = 0.f;
@@ -806,7 +842,7 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
           if (b < p.B && !*abort_flag) {
             GroupPartial gp;
             gp.key = kb;
-            gp.m = m;
+            gp.m = m * 0.69314718055994531f;  // base-2 maximum back to natural units
             gp.sum = s;
             p.partials[slot * p.B + b] = gp;
           }
