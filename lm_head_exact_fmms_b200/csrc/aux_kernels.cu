@@ -273,20 +273,22 @@ cudaError_t launch_sample_logits(const SampleLogitsParams &s, cudaStream_t strea
 // them).  The candidates of a row are its K allowed tokens with the largest
 // logits, ties toward the smaller index.  Two launches:
 //   1. topk_local_kernel: each row is split over P blocks (P x rows at most
-//      one block per SM, so the grid is one wave).  A block finds, with shared-memory radix histograms
-//      over the order-preserving bits of its slice's keys (bits 31-21, then
-//      20-10 and 9-0 only while the candidate set exceeds its capacity), a
-//      key threshold with at least min(K, allowed) of its keys at or above
-//      it, and writes those (key, token) pairs in token order to its
-//      candidate list.  The row's K-th largest key is at least every block's
-//      local K-th largest, so the union of the lists holds the row's top K,
-//      and every token tied with the row's K-th key.
-//   2. topk_row_kernel: one block per row selects the exact K-th largest key
-//      among the row's candidates (the same radix passes), keeps the tied
-//      keys in token order as K allows, draws the noise of the selected
-//      tokens and writes the Gumbel-max token.
-// Nothing carries over between calls: the candidate counts are written, not
-// accumulated.
+//      one block per SM, so the grid is one wave).  A block finds a key
+//      threshold at or below its slice's K-th largest allowed key (or 0 when
+//      the slice has at most K) whose passing keys fit its capacity -- read
+//      off a histogram of a sample and verified by the extraction pass, else
+//      set by exact shared-memory radix histograms of the slice, down to the
+//      exact key with its tied tokens ranked in token order -- and writes the
+//      passing (key, token) pairs and the threshold.  The row's K-th largest
+//      key is at least every block's threshold, so the union of the lists
+//      holds the row's top K and every token tied with the row's K-th key.
+//   2. topk_row_kernel: one block per row keeps the candidates at or above
+//      the largest block threshold, selects the exact top K among them (one
+//      radix level, then direct ranks; larger sets take three radix levels
+//      and a radix select on the token for a split tie), draws the noise of
+//      the selected tokens and writes the Gumbel-max token.
+// Nothing carries over between calls: the list lengths and thresholds are
+// written, not accumulated.
 // ---------------------------------------------------------------------------
 constexpr int kTopkThreads = 1024;
 constexpr int kTopkItems = 16;     // consecutive elements per thread per iteration (4 x 16 B)
