@@ -124,3 +124,30 @@ def test_flagship_schedule_balance(lib):
     nc, per_cta = _all_tiles(151936, 0, 148)
     rows = [int(sum(t[2] - t[1] for t in tiles)) for tiles in per_cta]
     assert nc == 148 and min(rows) >= 1024 and max(rows) <= 1032
+
+
+def test_fused_exchange_validation(lib):
+    """fs_sample_tp and its helpers reject bad arguments before any CUDA call."""
+    areas = (ctypes.c_void_p * 2)(0x100000, 0x200000)          # 256-byte aligned, never touched
+    odd = (ctypes.c_void_p * 2)(0x100000, 0x200008)
+
+    def tp(H=FAKE, B=4, V_shard=100, off=0, V_total=200, table=areas, world=2):
+        return lib.fs_sample_tp(H, FAKE, B, 64, V_shard, off, V_total, 1.0, 0, None, 0, None,
+                                table, world, 0, None, 0, None)
+    assert tp(H=None) == 1
+    assert tp(B=257) == 2                     # more than one launch's rows
+    assert tp(off=4) == 1                     # shard offsets are multiples of 8
+    assert tp(off=104) == 1                   # shard beyond V_total
+    assert tp(table=None) == 1
+    assert tp(world=0) == 1 and tp(world=17) == 1
+    assert tp(table=odd) == 1                 # areas are 256-byte aligned
+    assert lib.fs_tp_wait(None, 4, 0, FAKE, None) == 1
+    assert lib.fs_tp_wait(FAKE, 0, 0, FAKE, None) == 1
+    assert lib.fs_tp_wait(FAKE, 257, 0, FAKE, None) == 1
+    assert lib.fs_ipc_handle(None, None) == 1
+    assert lib.fs_ipc_open(None, None) == 1
+    assert lib.fs_tp_area_create(None) == 1
+    assert lib.fs_tp_area_destroy(None) == 0 and lib.fs_ipc_close(None) == 0
+    # the area holds two halves of 256 keys and 256 tokens plus its header
+    assert binding.fs_tp_area_bytes() >= 2 * 256 * (8 + 4) + 32
+    assert binding.fs_tp_area_bytes() % 256 == 0
