@@ -387,18 +387,7 @@ def run_gpu(args, world, rank, local):
         "dtype": "bf16",
         "data": "synthetic: seeded H ~ N(0,1), W ~ N(0, %g^2) bf16 (random-init %s head)"
                 % (wl.w_std, wl.name),
-        "config": {"workload": "%s LM head, d=%d V=%d B=%d T=%g%s%s, fused %s"
-                               % (wl.name, wl.d, wl.V, B, wl.temperature,
-                                  ", per-row seeds" if wl.per_row_seeds else "",
-                                  (", G=%d, %d%% mask" % (wl.groups, round(100 * wl.mask_allowed)))
-                                  if grouped else "",
-                                  "fs_sample_grouped" if grouped else "fs_sample_ex"),
-                   "batch_per_gpu": B, "global_batch": B * world, "d": wl.d, "V": wl.V,
-                   "parallelism": ("tensor-parallel vocabulary x%d (%s)" % (
-                       world, "fused peer-memory exchange" if fused_tp else "NCCL all-reduce"))
-                   if tp
-                   else ("replicas x%d" % world),
-                   "l2": "no flush: W (%.2f GB) exceeds the 126 MB L2" % (wl.V * wl.d * 2 / 1e9)},
+        "config": workload_config(wl, B, world, tp, fused_tp),
         "samples_per_s": round(B * world / (us_per_call * 1e-6), 1),
         "hbm_gbs_per_gpu": round(nbytes / (us_per_call * 1e-6) / 1e9, 1),
         "kernel_us": round(kernel_us, 3),
@@ -576,6 +565,22 @@ def unfused_point(torch, binding, synth, W, wl, dev, stream, B, steps=100):
 
 
 # ------------------------------------------------------ the reference arm
+def workload_config(wl, B, world, tp=False, fused_tp=False):
+    """The `config` object of the JSON line (both arms print the same one)."""
+    grouped = bool(wl.groups)
+    return {"workload": "%s LM head, d=%d V=%d B=%d T=%g%s%s, fused %s"
+                        % (wl.name, wl.d, wl.V, B, wl.temperature,
+                           ", per-row seeds" if wl.per_row_seeds else "",
+                           (", G=%d, %d%% mask" % (wl.groups, round(100 * wl.mask_allowed)))
+                           if grouped else "",
+                           "fs_sample_grouped" if grouped else "fs_sample_ex"),
+            "batch_per_gpu": B, "global_batch": B * world, "d": wl.d, "V": wl.V,
+            "parallelism": ("tensor-parallel vocabulary x%d (%s)" % (
+                world, "fused peer-memory exchange" if fused_tp else "NCCL all-reduce"))
+            if tp else ("replicas x%d" % world),
+            "l2": "no flush: W (%.2f GB) exceeds the 126 MB L2" % (wl.V * wl.d * 2 / 1e9)}
+
+
 def run_reference(args, world, rank):
     """The CPU oracle timed on this host's cores, on the same workload, metric
     and unit; each step is a bounded sample (one row over a vocabulary slice)."""
@@ -616,9 +621,9 @@ def run_reference(args, world, rank):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(sum(times) / len(times) * 1e3, 3), "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "%s LM head, d=%d V=%d B=%d T=%g" % (wl.name, wl.d, wl.V, B,
-                                                                   wl.temperature),
-                   "global_batch": B, "parallelism": "CPU oracle, %d threads" % cores},
+        "config": workload_config(wl, B, world, args.tp and world > 1 and not wl.groups,
+                                  args.tp and world > 1 and not wl.groups
+                                  and not (args.tp_nccl or B > 256)),
         "cpu_baseline": {"value": round(value, 1), "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": "each step: 1 row x %d-token vocabulary slice; value scaled "
                                    "by (V/%d) x B" % (Vs, Vs)},
