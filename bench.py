@@ -271,6 +271,17 @@ def percentiles(xs, qs=(10, 50, 90)):
     return [s[min(len(s) - 1, max(0, (q * len(s) + 99) // 100 - 1))] for q in qs]
 
 
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def cpu_baseline(H, W, wl, B, rs, budget_s=12.0, max_rows=64):
     """The oracle as it stands, on this host's cores, over a bounded sample of
     the workload's rows; scaled to us per B-row call."""
@@ -289,7 +300,7 @@ def cpu_baseline(H, W, wl, B, rs, budget_s=12.0, max_rows=64):
             break
     per_row = sum(times) / len(times)
     return {"value": per_row * B * 1e6, "unit": UNIT, "cores": oracle.num_threads(),
-            "kind": "oracle",
+            "cpu": cpu_model(), "kind": "oracle",
             "sample": "%d of the %d rows of one B=%d call (full vocabulary each), fp64 oracle; "
                       "value = mean row time x %d rows" % (len(times), B, B, B),
             "seconds": round(sum(times), 2)}
@@ -624,7 +635,8 @@ def run_reference(args, world, rank):
         "config": workload_config(wl, B, world, args.tp and world > 1 and not wl.groups,
                                   args.tp and world > 1 and not wl.groups
                                   and not (args.tp_nccl or B > 256)),
-        "cpu_baseline": {"value": round(value, 1), "unit": UNIT, "cores": cores, "kind": "oracle",
+        "cpu_baseline": {"value": round(value, 1), "unit": UNIT, "cores": cores, "cpu": cpu_model(),
+                         "kind": "oracle",
                          "sample": "each step: 1 row x %d-token vocabulary slice; value scaled "
                                    "by (V/%d) x B" % (Vs, Vs)},
         "e2e": {"value": round(value, 1), "unit": UNIT, "h2d_bytes_per_step": 0,
