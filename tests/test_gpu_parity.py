@@ -64,6 +64,28 @@ def test_philox_bitwise(dev, oracle):
     assert np.array_equal(got, ref)
 
 
+def test_philox_bitwise_sequential_counters(dev, oracle):
+    """2^26 counters laid out as the samplers use them -- word 0 the token
+    index / 4 running through 2^24 values, words 1-3 (row, step, tag) and the
+    key varied -- bit for bit between the device Philox and the oracle's."""
+    n = 1 << 24
+    c0 = np.arange(n, dtype=np.uint32)
+    for row, step, tag, seed in [(0, 0, 0, 0), (255, 7, 1, 0x0123456789ABCDEF),
+                                 (1 << 20, 0xFFFFFFFF, 2, 1000), (3, 1 << 31, 0, 2 ** 64 - 1)]:
+        ctr = np.empty((n, 4), dtype=np.uint32)
+        ctr[:, 0] = c0
+        ctr[:, 1] = row
+        ctr[:, 2] = step
+        ctr[:, 3] = tag
+        key = np.array([seed & 0xFFFFFFFF, seed >> 32], dtype=np.uint32)
+        ref = oracle.philox4x32_10(ctr, key)
+        t_ctr = torch.from_numpy(ctr.view(np.int32)).to(dev)
+        t_key = torch.from_numpy(np.broadcast_to(key, (n, 2)).copy().view(np.int32)).to(dev)
+        got = binding.fs_philox4x32_10(t_ctr, t_key).cpu().numpy().view(np.uint32)
+        assert np.array_equal(got, ref), (row, step, tag, seed)
+        del t_ctr, t_key
+
+
 def gumbel_rs():
     lo = np.arange(0, 1 << 20, dtype=np.uint64)
     hi = np.arange((1 << 32) - (1 << 20), 1 << 32, dtype=np.uint64)
