@@ -321,9 +321,11 @@ fs_status run_locked(int mode, const void *H, const void *W, int B, int d, int V
   if (s != FS_OK) return s;
   const Workspace w = carve(wsp, B, sch.G, sch.num_ctas, S, grouped);
 
-  CUtensorMap tw, tw8;
+  CUtensorMap tw;
+  fmms::PartMaps twp;
   if ((s = tensor_map(&tw, W, d, V, fmms::kTileM)) != FS_OK) return s;
-  if ((s = tensor_map(&tw8, W, d, V, fmms::kGranule)) != FS_OK) return s;
+  for (int b = 0; b < 4; ++b)
+    if ((s = tensor_map(&twp.box[b], W, d, V, fmms::kGranule << b)) != FS_OK) return s;
 
   for (int b0 = 0; b0 < B; b0 += fmms::kMaxBN) {
     const int Bc = fmms::imin(fmms::kMaxBN, B - b0);
@@ -369,10 +371,10 @@ fs_status run_locked(int mode, const void *H, const void *W, int B, int d, int V
     const int pair_units_used = pair ? fmms::make_schedule(V, sch.G, units).num_ctas : 0;
     if (pair) {
       p.num_ctas = 2 * pair_units_used;
-      if (fmms::launch_fmms_pair(mode, BN, tw, tw8, th, p, stream) != cudaSuccess)
+      if (fmms::launch_fmms_pair(mode, BN, tw, twp, th, p, stream) != cudaSuccess)
         return FS_ERR_CUDA;
     } else {
-      if (fmms::launch_fmms(mode, BN, tw, tw8, th, p, stream) != cudaSuccess) return FS_ERR_CUDA;
+      if (fmms::launch_fmms(mode, BN, tw, twp, th, p, stream) != cudaSuccess) return FS_ERR_CUDA;
     }
 
     if (mode == fmms::kModeGrouped) {

@@ -4,11 +4,11 @@
 
 namespace fmms {
 
-cudaError_t launch_logits(int BN, const CUtensorMap &tw, const CUtensorMap &tw8,
+cudaError_t launch_logits(int BN, const CUtensorMap &tw, const PartMaps &twp,
                           const CUtensorMap &th, const FmmsParams &p, cudaStream_t stream) {
   switch (BN) {
 #define FMMS_CASE(n) \
-  case n: return launch_t<n, kModeLogits>(tw, tw8, th, p, stream);
+  case n: return launch_t<n, kModeLogits>(tw, twp, th, p, stream);
     FMMS_FOR_EACH_BN(FMMS_CASE)
 #undef FMMS_CASE
     default: return cudaErrorInvalidValue;

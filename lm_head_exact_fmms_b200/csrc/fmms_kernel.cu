@@ -6,21 +6,21 @@
 
 namespace fmms {
 
-cudaError_t launch_fmms(int mode, int BN, const CUtensorMap &tw, const CUtensorMap &tw8,
+cudaError_t launch_fmms(int mode, int BN, const CUtensorMap &tw, const PartMaps &twp,
                         const CUtensorMap &th, const FmmsParams &p, cudaStream_t stream) {
   switch (mode) {
-    case kModeFlat: return launch_flat(BN, tw, tw8, th, p, stream);
-    case kModeGrouped: return launch_grouped(BN, tw, tw8, th, p, stream);
-    case kModeLogits: return launch_logits(BN, tw, tw8, th, p, stream);
+    case kModeFlat: return launch_flat(BN, tw, twp, th, p, stream);
+    case kModeGrouped: return launch_grouped(BN, tw, twp, th, p, stream);
+    case kModeLogits: return launch_logits(BN, tw, twp, th, p, stream);
     default: return cudaErrorInvalidValue;
   }
 }
 
-cudaError_t launch_fmms_pair(int mode, int BN, const CUtensorMap &tw, const CUtensorMap &tw8,
+cudaError_t launch_fmms_pair(int mode, int BN, const CUtensorMap &tw, const PartMaps &twp,
                              const CUtensorMap &th, const FmmsParams &p, cudaStream_t stream) {
   switch (mode) {
-    case kModeFlat: return launch_flat_pair(BN, tw, tw8, th, p, stream);
-    case kModeGrouped: return launch_grouped_pair(BN, tw, tw8, th, p, stream);
+    case kModeFlat: return launch_flat_pair(BN, tw, twp, th, p, stream);
+    case kModeGrouped: return launch_grouped_pair(BN, tw, twp, th, p, stream);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -466,7 +466,7 @@ __device__ __forceinline__ void issue_h(const CUtensorMap *th, const FmmsParams 
 // CTA's full barrier; the even CTA also hands each freed stage on to the odd
 // CTA, whose MMA reads happen in the even CTA's tcgen05 pipeline.
 template <int BN, int MODE, bool PAIR>
-__device__ __forceinline__ void role_producer(const CUtensorMap *tw, const CUtensorMap *tw8,
+__device__ __forceinline__ void role_producer(const CUtensorMap *tw, const PartMaps *twp,
                                               const CUtensorMap *th, const FmmsParams &p,
                                               const Schedule &sch, uint8_t *stages,
                                               uint64_t *full, uint64_t *empty,
@@ -489,8 +489,11 @@ __device__ __forceinline__ void role_producer(const CUtensorMap *tw, const CUten
   while (ok && it.next(tile)) {
     const Tile mine = PAIR ? pair_half(tile, rank) : tile;
     const int rows = mine.hi - mine.start;
-    const bool whole = rows >= kTileM;
     const int nbox8 = rows > 0 ? (rows + kGranule - 1) / kGranule : 0;
+    // 16 granules (a tile cut short by fewer than 8 rows at the end of a
+    // segment) load as one 128-row box: the rows past the tile's end are in
+    // bounds (the next segment's) or zero-filled past V, and masked anyway.
+    const bool whole = nbox8 >= kTileM / kGranule;
     uint32_t sub_bytes = w_sub_bytes(rows) + C::kSubH;  // counted on this CTA's barrier
     if (PAIR) {
       const Tile other = pair_half(tile, 1 - rank);
@@ -523,14 +526,20 @@ __device__ __forceinline__ void role_producer(const CUtensorMap *tw, const CUten
             sm100::tma_load_2d(sw, tw, &full[stage], x, mine.start, pol_w);
           }
         } else {
-          for (int i = 0; i < nbox8; ++i) {
+          // Boxes of 64, 32, 16 and 8 rows: the binary digits of the tile's
+          // 8-row count, each at its 1024-byte-aligned place in the stage.
+          int row = 0;
+#pragma unroll
+          for (int b = 3; b >= 0; --b) {
+            if (!((nbox8 >> b) & 1)) continue;
             if constexpr (PAIR) {
-              sm100::tma_load_2d_pair(sw + i * 1024, tw8, bar, x, mine.start + kGranule * i,
+              sm100::tma_load_2d_pair(sw + row * 128, &twp->box[b], bar, x, mine.start + row,
                                       pol_w);
             } else {
-              sm100::tma_load_2d(sw + i * 1024, tw8, &full[stage], x, mine.start + kGranule * i,
+              sm100::tma_load_2d(sw + row * 128, &twp->box[b], &full[stage], x, mine.start + row,
                                  pol_w);
             }
+            row += kGranule << b;
           }
         }
       }
@@ -900,7 +909,7 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
 template <int BN, int MODE, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     fmms_kernel(const __grid_constant__ CUtensorMap tmap_w,
-                const __grid_constant__ CUtensorMap tmap_w8,
+                const __grid_constant__ PartMaps tmap_wp,
                 const __grid_constant__ CUtensorMap tmap_h, const FmmsParams p) {
   using C = KCfg<BN, MODE, PAIR>;
   extern __shared__ uint8_t smem_raw[];
@@ -948,7 +957,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     sm100::fence_mbar_init();
     sm100::fence_async_smem();
     sm100::prefetch_tensormap(&tmap_w);
-    sm100::prefetch_tensormap(&tmap_w8);
+#pragma unroll
+    for (int b = 0; b < 4; ++b) sm100::prefetch_tensormap(&tmap_wp.box[b]);
     sm100::prefetch_tensormap(&tmap_h);
   }
   if constexpr (PAIR) {
@@ -973,7 +983,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     if (lane == 0)
-      role_producer<BN, MODE, PAIR>(&tmap_w, &tmap_w8, &tmap_h, p, sch, stages, full, empty,
+      role_producer<BN, MODE, PAIR>(&tmap_w, &tmap_wp, &tmap_h, p, sch, stages, full, empty,
                                     abort_flag, unit, rank);
     __syncwarp();
   } else if (warp == 1) {
@@ -1009,14 +1019,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 // Host launchers
 // ---------------------------------------------------------------------------
 template <int BN, int MODE>
-cudaError_t launch_t(const CUtensorMap &tw, const CUtensorMap &tw8, const CUtensorMap &th,
+cudaError_t launch_t(const CUtensorMap &tw, const PartMaps &twp, const CUtensorMap &th,
                             const FmmsParams &p, cudaStream_t stream) {
   using C = KCfg<BN, MODE>;
   auto kern = fmms_kernel<BN, MODE, false>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  kern<<<p.num_ctas, kThreads, C::kSmemBytes, stream>>>(tw, tw8, th, p);
+  kern<<<p.num_ctas, kThreads, C::kSmemBytes, stream>>>(tw, twp, th, p);
   return cudaGetLastError();
 }
 
@@ -1056,7 +1066,7 @@ cudaError_t pair_units_t(int *units) {
 }
 
 template <int BN, int MODE>
-cudaError_t launch_pair_t(const CUtensorMap &tw, const CUtensorMap &tw8,
+cudaError_t launch_pair_t(const CUtensorMap &tw, const PartMaps &twp,
                                  const CUtensorMap &th, const FmmsParams &p,
                                  cudaStream_t stream) {
   using C = KCfg<BN, MODE, true>;
@@ -1066,7 +1076,7 @@ cudaError_t launch_pair_t(const CUtensorMap &tw, const CUtensorMap &tw8,
   if (e != cudaSuccess) return e;
   cudaLaunchAttribute attr[1];
   cudaLaunchConfig_t cfg = pair_config<BN, MODE>(p.num_ctas, stream, attr);
-  e = cudaLaunchKernelEx(&cfg, kern, tw, tw8, th, p);
+  e = cudaLaunchKernelEx(&cfg, kern, tw, twp, th, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -9,32 +9,39 @@
 
 namespace fmms {
 
+// Tensor maps of W for partial tiles: boxes of 8, 16, 32 and 64 rows.  A
+// partial tile of 8k rows is loaded as at most four boxes, one for each
+// binary digit of k, instead of k boxes of 8 rows.
+struct PartMaps {
+  CUtensorMap box[4];
+};
+
 // Batch tile (MMA N) of a launch of `rows` rows: the next multiple of 16,
 // at most 256.
 int fmms_batch_tile(int rows);
 
 // Per-mode launchers for every batch tile (fmms_inst_*.cu).
-cudaError_t launch_flat(int BN, const CUtensorMap &tw, const CUtensorMap &tw8,
+cudaError_t launch_flat(int BN, const CUtensorMap &tw, const PartMaps &twp,
                         const CUtensorMap &th, const FmmsParams &p, cudaStream_t stream);
-cudaError_t launch_grouped(int BN, const CUtensorMap &tw, const CUtensorMap &tw8,
+cudaError_t launch_grouped(int BN, const CUtensorMap &tw, const PartMaps &twp,
                            const CUtensorMap &th, const FmmsParams &p, cudaStream_t stream);
-cudaError_t launch_logits(int BN, const CUtensorMap &tw, const CUtensorMap &tw8,
+cudaError_t launch_logits(int BN, const CUtensorMap &tw, const PartMaps &twp,
                           const CUtensorMap &th, const FmmsParams &p, cudaStream_t stream);
-cudaError_t launch_flat_pair(int BN, const CUtensorMap &tw, const CUtensorMap &tw8,
+cudaError_t launch_flat_pair(int BN, const CUtensorMap &tw, const PartMaps &twp,
                              const CUtensorMap &th, const FmmsParams &p, cudaStream_t stream);
-cudaError_t launch_grouped_pair(int BN, const CUtensorMap &tw, const CUtensorMap &tw8,
+cudaError_t launch_grouped_pair(int BN, const CUtensorMap &tw, const PartMaps &twp,
                                 const CUtensorMap &th, const FmmsParams &p, cudaStream_t stream);
 cudaError_t pair_units_flat(int BN, int *units);
 cudaError_t pair_units_grouped(int BN, int *units);
 
 // The fused kernel in mode kModeFlat / kModeGrouped / kModeLogits with batch
 // tile BN, grid p.num_ctas x kThreads threads.
-cudaError_t launch_fmms(int mode, int BN, const CUtensorMap &tw, const CUtensorMap &tw8,
+cudaError_t launch_fmms(int mode, int BN, const CUtensorMap &tw, const PartMaps &twp,
                         const CUtensorMap &th, const FmmsParams &p, cudaStream_t stream);
 
 // The flat or grouped kernel on CTA pairs (clusters of two, tcgen05
 // cta_group::2): p.num_ctas CTAs (even), th with boxes of BN/2 rows.
-cudaError_t launch_fmms_pair(int mode, int BN, const CUtensorMap &tw, const CUtensorMap &tw8,
+cudaError_t launch_fmms_pair(int mode, int BN, const CUtensorMap &tw, const PartMaps &twp,
                              const CUtensorMap &th, const FmmsParams &p, cudaStream_t stream);
 
 // How many CTA pairs of the BN pair kernel of `mode` can be resident at once.

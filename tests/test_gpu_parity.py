@@ -355,6 +355,20 @@ def test_grouped_parity(dev, oracle, G, masked):
 
 
 # ------------------------------------------------------------ unfused mode
+@pytest.mark.parametrize("V", [4097, 9001, 30011, 30013, 151933, 18944 * 8 + 5])
+def test_logits_of_every_tile_shape(dev, V):
+    """The logits the fused kernel computes (logits mode) equal an fp32 matmul
+    on every vocabulary row, for vocabularies whose CTA ranges give partial
+    tiles of every size class (loaded as 64/32/16/8-row boxes) and tiles cut
+    short by 1-7 rows at the end (loaded as one 128-row box)."""
+    B, d = 16, 128
+    H, W, Hd, Wd = rand_inputs(B, d, V, seed=V % 1000)
+    logits = torch.empty(B, V, dtype=torch.float32, device=dev)
+    binding.fs_sample_unfused(Hd, Wd, temperature=1.0, logits=logits)
+    ref = Hd.float() @ Wd.float().t()
+    assert (logits - ref).abs().max().item() < 1e-3
+
+
 @pytest.mark.parametrize("B,V", [(1, 4096), (37, 5001), (256, 3000)])
 def test_unfused_parity(dev, oracle, B, V):
     d = 128
