@@ -494,6 +494,13 @@ __device__ __forceinline__ void role_producer(const CUtensorMap *tw, const PartM
     // segment) load as one 128-row box: the rows past the tile's end are in
     // bounds (the next segment's) or zero-filled past V, and masked anyway.
     const bool whole = nbox8 >= kTileM / kGranule;
+    // A small partial tile (at most 32 rows) costs a whole tile's MMA loop
+    // while streaming few W bytes: meanwhile prefetch the segment's next tile
+    // into L2, so that its loads catch up.  (Larger partial tiles stream
+    // enough themselves; prefetching for them overflowed L2 on heads where
+    // every CTA starts with one.)
+    const int next_start = it.t < it.seg_hi ? it.t + (PAIR ? rank * kTileM : 0) : -1;
+    const bool prefetch_next = nbox8 <= 4 && next_start >= 0 && next_start < p.V;
     uint32_t sub_bytes = w_sub_bytes(rows) + C::kSubH;  // counted on this CTA's barrier
     if (PAIR) {
       const Tile other = pair_half(tile, 1 - rank);
@@ -526,6 +533,7 @@ __device__ __forceinline__ void role_producer(const CUtensorMap *tw, const PartM
             sm100::tma_load_2d(sw, tw, &full[stage], x, mine.start, pol_w);
           }
         } else {
+          if (prefetch_next) sm100::tma_prefetch_2d(tw, x, next_start);
           // Boxes of 64, 32, 16 and 8 rows: the binary digits of the tile's
           // 8-row count, each at its 1024-byte-aligned place in the stage.
           int row = 0;
