@@ -495,12 +495,13 @@ __device__ __forceinline__ void role_producer(const CUtensorMap *tw, const PartM
     // bounds (the next segment's) or zero-filled past V, and masked anyway.
     const bool whole = nbox8 >= kTileM / kGranule;
     // A small partial tile (at most 32 rows) costs a whole tile's MMA loop
-    // while streaming few W bytes: meanwhile prefetch the segment's next tile
-    // into L2, so that its loads catch up.  (Larger partial tiles stream
-    // enough themselves; prefetching for them overflowed L2 on heads where
-    // every CTA starts with one.)
-    const int next_start = it.t < it.seg_hi ? it.t + (PAIR ? rank * kTileM : 0) : -1;
-    const bool prefetch_next = nbox8 <= 4 && next_start >= 0 && next_start < p.V;
+    // while streaming few W bytes: meanwhile the single-CTA kernel (the
+    // bandwidth-bound batch sizes) prefetches the segment's next tile into
+    // L2, so that its loads catch up.  (Larger partial tiles stream enough
+    // themselves, and prefetching for them overflowed L2 on heads where every
+    // CTA starts with one; on CTA pairs, tensor-bound, it only added traffic.)
+    const int next_start = it.t < it.seg_hi ? it.t : -1;
+    const bool prefetch_next = !PAIR && nbox8 <= 4 && next_start >= 0 && next_start < p.V;
     uint32_t sub_bytes = w_sub_bytes(rows) + C::kSubH;  // counted on this CTA's barrier
     if (PAIR) {
       const Tile other = pair_half(tile, 1 - rank);
