@@ -86,7 +86,21 @@ struct Tile {
   int hi;     // one past the last valid row (hi - start <= tile rows)
   int slot;   // partial slot of the segment
   int last;   // 1 on the last tile of a segment
+  // Merged partial: an 8-row partial tile [pstart, pstart + 8) (valid rows
+  // [plo, phi)) multiplied in the same stages as this whole tile, sharing
+  // its H loads, into an accumulator of its own.  pstart < 0: none.
+  int pstart, plo, phi;
 };
+
+// The merged partial of a tile as a tile of its own.
+FS_HD Tile partial_of(const Tile &t) {
+  Tile p = t;
+  p.start = t.pstart;
+  p.lo = t.plo;
+  p.hi = t.phi;
+  p.pstart = -1;
+  return p;
+}
 
 // The 128-row half of a 256-row pair tile that CTA `rank` of the pair
 // multiplies; hi <= lo when the half holds no valid row.
@@ -107,8 +121,10 @@ struct TileIter {
   int t;       // start of the next tile
   int len;     // rows of the next tile
   int slot;
+  int merge;   // merge a segment's 8-row partial tile into its first whole tile
 
-  FS_HD TileIter(const Schedule &s, int c) {
+  FS_HD TileIter(const Schedule &s, int c, int merge_partial = 0) {
+    merge = merge_partial;
     V = s.V;
     G = s.G;
     rows = s.tile_rows;
@@ -125,8 +141,11 @@ struct TileIter {
   // multiple of 8, then whole tiles (the last may lack up to 7 rows).  The MMA
   // loop of a partial tile costs as much as a whole tile's; run first it
   // overlaps the other CTAs' streaming, run last it would be a tail with HBM
-  // idle.
+  // idle.  With `merge`, an 8-row partial tile followed by a whole tile is
+  // returned with it (pstart), so that both share one pass over H.
   FS_HD bool next(Tile &tile) {
+    tile.pstart = -1;
+    tile.plo = tile.phi = 0;
     if (t >= seg_hi) {
       v = seg_hi;
       if (v >= cta_hi) return false;
@@ -137,6 +156,13 @@ struct TileIter {
       t = v & ~(kGranule - 1);
       const int rem = (seg_hi - t) % rows;
       len = rem == 0 ? rows : (rem + kGranule - 1) & ~(kGranule - 1);
+    }
+    if (merge && len == kGranule && t + len < seg_hi) {
+      tile.pstart = t;
+      tile.plo = imax(t, v);
+      tile.phi = imin(t + len, seg_hi);
+      t += len;
+      len = rows;
     }
     tile.start = t;
     tile.lo = imax(t, v);

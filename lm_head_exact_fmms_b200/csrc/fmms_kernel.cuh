@@ -66,14 +66,14 @@ constexpr int kSmemBudget = 232448 - 1024 - 256;
 // E.g. single CTAs: 4 x 3 stages at 16 batch rows, 2 x 5 at 32, 3 x 3 at 64;
 // CTA pairs: 3 x 3 at 128 rows (64 H rows per CTA), 1 x 7 at 256.
 constexpr int kMaxStages = 10;
-constexpr int stages_for(int ksub, int h_rows, int comb_bytes) {
-  const int fit = (kSmemBudget - comb_bytes) / (ksub * (kTileM + h_rows) * kBlockK * 2);
+constexpr int stages_for(int ksub, int h_rows, int comb_bytes, int p_bytes) {
+  const int fit = (kSmemBudget - comb_bytes) / (ksub * ((kTileM + h_rows) * kBlockK * 2 + p_bytes));
   return fit < kMaxStages ? fit : kMaxStages;
 }
-constexpr int ksub_for(int h_rows, int comb_bytes) {
+constexpr int ksub_for(int h_rows, int comb_bytes, int p_bytes) {
   int best = 1, best_bytes = 0;
   for (int k = 1; k <= 4; ++k) {
-    const int st = stages_for(k, h_rows, comb_bytes);
+    const int st = stages_for(k, h_rows, comb_bytes, p_bytes);
     if (st >= 3 && st * k >= best_bytes) {
       best = k;
       best_bytes = st * k;
@@ -95,13 +95,22 @@ struct KCfg {
   static_assert(!PAIR || MODE != kModeLogits, "the logits mode runs on single CTAs");
   static constexpr int kHRows = PAIR ? BN / 2 : BN;     // H rows this CTA stages
   static constexpr int kCombBytes = MODE == kModeGrouped ? 4 * BN * 16 : 0;  // grouped only
-  static constexpr int kSub = ksub_for(kHRows, kCombBytes);  // 64-wide K blocks per stage
+  // Merged 8-row partial tiles (single CTAs of 32 to 64 batch rows; at 16
+  // the extra kilobyte per sub-block would shorten the ring, and above 64
+  // rows CTA pairs run): each stage starts with one 8-row W slot per
+  // sub-block.
+  static constexpr bool kMerge = !PAIR && BN >= 32 && BN <= 64;
+  static constexpr int kSubP = kMerge ? kGranule * kBlockK * 2 : 0;  // 1 KB per sub-block
+  static constexpr int kSub = ksub_for(kHRows, kCombBytes, kSubP);  // 64-wide K blocks per stage
   static constexpr int kSubW = kTileM * kBlockK * 2;    // 16 KB of W per sub-block
   static constexpr int kSubH = kHRows * kBlockK * 2;    // this CTA's H rows per sub-block
+  static constexpr int kStageP = kSub * kSubP;
   static constexpr int kStageW = kSub * kSubW;
   static constexpr int kStageH = kSub * kSubH;
-  static constexpr int kStageBytes = kStageW + kStageH;
-  static constexpr int kStages = stages_for(kSub, kHRows, kCombBytes);
+  static constexpr int kOffW = kStageP;                 // stage layout: [P][W][H]
+  static constexpr int kOffH = kStageP + kStageW;
+  static constexpr int kStageBytes = kStageP + kStageW + kStageH;
+  static constexpr int kStages = stages_for(kSub, kHRows, kCombBytes, kSubP);
   static constexpr int kCW = 16;                        // columns per epilogue chunk
   static constexpr int kChunks = BN / kCW;
   static constexpr int kWarpsPerQuarter = kNumEpiWarps / 4;
@@ -446,7 +455,7 @@ __device__ __forceinline__ void issue_h(const CUtensorMap *th, const FmmsParams 
                                         uint8_t *stages, uint64_t *full, int stage, int sub0,
                                         int nsub, int rank, uint64_t pol_h) {
   using C = KCfg<BN, MODE, PAIR>;
-  uint8_t *sh0 = stages + stage * C::kStageBytes + C::kStageW;
+  uint8_t *sh0 = stages + stage * C::kStageBytes + C::kOffH;
   const uint32_t bar = PAIR ? sm100::cluster_addr(&full[stage], 0) : 0u;
 #pragma unroll
   for (int j = 0; j < C::kSub; ++j) {
@@ -474,7 +483,7 @@ __device__ __forceinline__ void role_producer(const CUtensorMap *tw, const PartM
   using C = KCfg<BN, MODE, PAIR>;
   const uint64_t pol_w = sm100::l2_policy_evict_first();
   const uint64_t pol_h = sm100::l2_policy_evict_last();
-  TileIter it(sch, unit);
+  TileIter it(sch, unit, C::kMerge ? 1 : 0);
   Tile tile;
   int stage = 0;
   uint32_t phase = 0;
@@ -487,6 +496,7 @@ __device__ __forceinline__ void role_producer(const CUtensorMap *tw, const PartM
   int npend = 0, pend_need = 0;
   bool ok = p.test_no_loads == 0;
   while (ok && it.next(tile)) {
+    const bool merged = C::kMerge && tile.pstart >= 0;
     const Tile mine = PAIR ? pair_half(tile, rank) : tile;
     const int rows = mine.hi - mine.start;
     const int nbox8 = rows > 0 ? (rows + kGranule - 1) / kGranule : 0;
@@ -502,7 +512,7 @@ __device__ __forceinline__ void role_producer(const CUtensorMap *tw, const PartM
     // CTA starts with one; on CTA pairs, tensor-bound, it only added traffic.)
     const int next_start = it.t < it.seg_hi ? it.t : -1;
     const bool prefetch_next = !PAIR && nbox8 <= 4 && next_start >= 0 && next_start < p.V;
-    uint32_t sub_bytes = w_sub_bytes(rows) + C::kSubH;  // counted on this CTA's barrier
+    uint32_t sub_bytes = w_sub_bytes(rows) + C::kSubH + (merged ? C::kSubP : 0u);  // this CTA's
     if (PAIR) {
       const Tile other = pair_half(tile, 1 - rank);
       sub_bytes += w_sub_bytes(other.hi - other.start) + C::kSubH;
@@ -518,7 +528,8 @@ __device__ __forceinline__ void role_producer(const CUtensorMap *tw, const PartM
       }
       if (PAIR && rank == 0 && issued >= C::kStages)
         sm100::mbar_arrive_cluster(sm100::cluster_addr(&empty[stage], 1));
-      uint8_t *sw0 = stages + stage * C::kStageBytes;
+      uint8_t *sp0 = stages + stage * C::kStageBytes;
+      uint8_t *sw0 = sp0 + C::kOffW;
       if (!PAIR || rank == 0) sm100::mbar_arrive_expect_tx(&full[stage], bytes);
       const uint32_t bar = PAIR ? sm100::cluster_addr(&full[stage], 0) : 0u;
       // W first: it never waits for H.
@@ -527,6 +538,12 @@ __device__ __forceinline__ void role_producer(const CUtensorMap *tw, const PartM
         if (j >= nsub) break;
         uint8_t *sw = sw0 + j * C::kSubW;
         const int x = (sub0 + j) * kBlockK;
+        if constexpr (C::kMerge) {
+          // the merged partial's 8 rows, into this sub-block's P slot
+          if (merged)
+            sm100::tma_load_2d(sp0 + j * C::kSubP, &twp->box[0], &full[stage], x, tile.pstart,
+                               pol_w);
+        }
         if (whole) {
           if constexpr (PAIR) {
             sm100::tma_load_2d_pair(sw, tw, bar, x, mine.start, pol_w);
@@ -625,7 +642,7 @@ __device__ __forceinline__ void role_mma(const FmmsParams &p, const Schedule &sc
                                          uint64_t *drain_bar, uint32_t tmem_base,
                                          volatile int *abort_flag, int unit) {
   using C = KCfg<BN, MODE, PAIR>;
-  TileIter it(sch, unit);
+  TileIter it(sch, unit, C::kMerge ? 1 : 0);
   Tile tile;
   int stage = 0;
   uint32_t phase = 0;
@@ -633,9 +650,16 @@ __device__ __forceinline__ void role_mma(const FmmsParams &p, const Schedule &sc
   uint32_t acc_phase = 0;
   bool ok = true;
   while (ok && it.next(tile)) {
+    // A merged partial takes the next accumulator too.
+    const bool merged = C::kMerge && tile.pstart >= 0;
+    const int buf2 = buf + 1 == C::kAccBufs ? 0 : buf + 1;
+    const uint32_t phase2 = buf + 1 == C::kAccBufs ? acc_phase ^ 1u : acc_phase;
     if (!sm100::wait_bounded<PAIR>(&acc_empty[buf], acc_phase ^ 1u, abort_flag, p.err)) break;
+    if (merged && !sm100::wait_bounded<PAIR>(&acc_empty[buf2], phase2 ^ 1u, abort_flag, p.err))
+      break;
     sm100::tc_fence_after();
     const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
+    const uint32_t d_tmem2 = tmem_base + static_cast<uint32_t>(buf2 * BN);
     const int nks = (p.nk + C::kSub - 1) / C::kSub;
     for (int ks = 0; ks < nks; ++ks) {
       if (!sm100::wait_bounded<PAIR>(&full[stage], phase, abort_flag, p.err)) {
@@ -644,8 +668,9 @@ __device__ __forceinline__ void role_mma(const FmmsParams &p, const Schedule &sc
       }
       sm100::tc_fence_after();
       const int nsub = imin(C::kSub, p.nk - ks * C::kSub);
-      const uint32_t a_addr = sm100::smem_addr(stages + stage * C::kStageBytes);
-      const uint32_t b_addr = a_addr + C::kStageW;
+      const uint32_t p_addr = sm100::smem_addr(stages + stage * C::kStageBytes);
+      const uint32_t a_addr = p_addr + C::kOffW;
+      const uint32_t b_addr = p_addr + C::kOffH;
 #pragma unroll
       for (int j = 0; j < C::kSub; ++j) {
         if (j >= nsub) break;
@@ -658,6 +683,23 @@ __device__ __forceinline__ void role_mma(const FmmsParams &p, const Schedule &sc
             sm100::mma_bf16_ss_pair(d_tmem, da, db, C::kIdesc, acc);
           } else {
             sm100::mma_bf16_ss(d_tmem, da, db, C::kIdesc, acc);
+          }
+        }
+      }
+      if constexpr (C::kMerge) {
+        // The merged partial: rows 0-7 from its P slot; rows 8-127 of the
+        // operand run on into the rest of the stage and land in accumulator
+        // rows the epilogue never reads.
+        if (merged) {
+#pragma unroll
+          for (int j = 0; j < C::kSub; ++j) {
+            if (j >= nsub) break;
+#pragma unroll
+            for (int kk = 0; kk < kBlockK / 16; ++kk) {
+              const uint64_t dp = sm100::smem_desc_sw128(p_addr + j * C::kSubP + kk * 32);
+              const uint64_t db = sm100::smem_desc_sw128(b_addr + j * C::kSubH + kk * 32);
+              sm100::mma_bf16_ss(d_tmem2, dp, db, C::kIdesc, (ks | j | kk) != 0 ? 1u : 0u);
+            }
           }
         }
       }
@@ -678,10 +720,13 @@ __device__ __forceinline__ void role_mma(const FmmsParams &p, const Schedule &sc
       sm100::mma_commit_pair(&acc_full[buf]);
     } else {
       sm100::mma_commit(&acc_full[buf]);
+      if (merged) sm100::mma_commit(&acc_full[buf2]);
     }
-    if (++buf == C::kAccBufs) {
-      buf = 0;
-      acc_phase ^= 1u;
+    for (int n = merged ? 2 : 1; n > 0; --n) {
+      if (++buf == C::kAccBufs) {
+        buf = 0;
+        acc_phase ^= 1u;
+      }
     }
   }
   // Drain: every MMA issued above has completed once this arrives.
@@ -726,12 +771,13 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
     sm100::epi_sync(kEpiThreads);
   }
 
-  TileIter it(sch, unit);
+  TileIter it(sch, unit, C::kMerge ? 1 : 0);
   Tile tile;
   int buf = 0;
   uint32_t phase = 0;
   bool aborted = false;
-  while (it.next(tile)) {
+  // One accumulator: wait for it, run the chunk pipeline over it, hand it back.
+  auto run_acc = [&](const Tile &cur) {
     // After an abort the loop keeps walking the tiles without touching TMEM,
     // so that every epilogue warp reaches the same named barriers.  The
     // decision is made warp-uniform because the TMEM loads below are
@@ -742,7 +788,7 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
       if (PAIR && rank == 0 && warp == 2 && lane == 0)
         sm100::mbar_arrive_cluster(sm100::cluster_addr(&acc_full[buf], 1));
       sm100::tc_fence_after();
-      const Tile mine = PAIR ? pair_half(tile, rank) : tile;
+      const Tile mine = PAIR ? pair_half(cur, rank) : cur;
       const int v = mine.start + 32 * q + lane;           // row of W in this launch
       const bool v_ok = v >= mine.lo && v < mine.hi;
       const int vg = v + p.vocab_offset;                  // global token index
@@ -836,6 +882,11 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
       buf = 0;
       phase ^= 1u;
     }
+  };
+  while (it.next(tile)) {
+    run_acc(tile);
+    // A merged partial comes as a second accumulator after its whole tile.
+    if (C::kMerge && tile.pstart >= 0) run_acc(partial_of(tile));
 
     if constexpr (MODE == kModeGrouped) {
       if (tile.last) {
