@@ -95,11 +95,12 @@ struct KCfg {
   static_assert(!PAIR || MODE != kModeLogits, "the logits mode runs on single CTAs");
   static constexpr int kHRows = PAIR ? BN / 2 : BN;     // H rows this CTA stages
   static constexpr int kCombBytes = MODE == kModeGrouped ? 4 * BN * 16 : 0;  // grouped only
-  // Merged 8-row partial tiles (single CTAs of 32 to 64 batch rows; at 16
-  // the extra kilobyte per sub-block would shorten the ring, and above 64
-  // rows CTA pairs run): each stage starts with one 8-row W slot per
-  // sub-block.
-  static constexpr bool kMerge = !PAIR && BN >= 32 && BN <= 64;
+  // Merged 8-row partial tiles (single CTAs of up to 64 batch rows; above
+  // that CTA pairs run): each stage starts with one 8-row W slot per
+  // sub-block.  (At 16 rows the extra kilobyte turns the ring from 4 x 3
+  // into 2 x 5 sub-blocks, 160 instead of 192 KB of W in flight; merging
+  // still wins: Qwen3-8B head B=1 191.5 -> 186.5 us.)
+  static constexpr bool kMerge = !PAIR && BN <= 64;
   static constexpr int kSubP = kMerge ? kGranule * kBlockK * 2 : 0;  // 1 KB per sub-block
   static constexpr int kSub = ksub_for(kHRows, kCombBytes, kSubP);  // 64-wide K blocks per stage
   static constexpr int kSubW = kTileM * kBlockK * 2;    // 16 KB of W per sub-block
