@@ -412,6 +412,19 @@ fs_status fs_test_stalled_sample(const void *H, const void *W, int B, int d,
  * CTAs. */
 fs_status fs_set_cta_pairs(int policy);
 
+/* Kernel choice for single-CTA launches of up to 64 batch rows: a CTA whose
+ * vocabulary range starts with an 8-row partial tile can either run it as a
+ * tile of its own (which streams all of H again for 8 rows of W) or multiply
+ * it in the same pipeline stages as its first whole tile, sharing the H
+ * loads (a 1 KB slot per stage for its rows, a second MMA into its own
+ * accumulator).  The results are the same either way (tokens bit for bit);
+ * the merged variant pays where many CTAs have such a tile (the Qwen3 heads,
+ * 48 of 148) and costs a little ring space elsewhere.  policy: -1 automatic
+ * (the default: merge when at least one CTA in ten has one), 0 never,
+ * 1 always.  Process-wide; applies to calls made after it returns.
+ * FS_ERR_INVALID_ARG for any other value. */
+fs_status fs_set_partial_merge(int policy);
+
 /* ---- Host-only schedule query (no GPU needed) ---- */
 
 /* The vocabulary schedule of the fused kernel for V tokens, G groups

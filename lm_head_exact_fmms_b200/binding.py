@@ -26,7 +26,7 @@ EXPORTED = ("fs_sample", "fs_sample_ex", "fs_sample_grouped", "fs_sample_unfused
             "fs_summarize_group", "fs_merge_groups", "fs_workspace_bytes_summary",
             "fs_sample_topk", "fs_set_cta_pairs", "fs_tp_area_bytes", "fs_tp_area_create",
             "fs_tp_area_destroy", "fs_ipc_handle", "fs_ipc_open", "fs_ipc_close", "fs_sample_tp",
-            "fs_tp_wait", "fs_tp_failed", "fs_test_stall_loads")
+            "fs_tp_wait", "fs_tp_failed", "fs_test_stall_loads", "fs_set_partial_merge")
 
 FS_IPC_HANDLE_BYTES = 64
 
@@ -89,6 +89,7 @@ def load_library():
     lib.fs_tp_wait.argtypes = [vp, i32, u32, vp, vp]
     lib.fs_tp_failed.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
     lib.fs_test_stall_loads.argtypes = [i32]
+    lib.fs_set_partial_merge.argtypes = [i32]
     lib.fs_workspace_bytes.argtypes = [i32, i32, i32]
     lib.fs_workspace_bytes.restype = sz
     lib.fs_device_status.argtypes = [vp, sz, vp]
@@ -431,6 +432,11 @@ def fs_tp_failed(area):
     v = ctypes.c_uint32()
     _check(load_library().fs_tp_failed(ctypes.c_void_p(area), ctypes.byref(v)), "fs_tp_failed")
     return int(v.value)
+
+
+def fs_set_partial_merge(policy):
+    """-1 automatic, 0 never, 1 always: merged 8-row partial tiles (single CTAs)."""
+    _check(load_library().fs_set_partial_merge(int(policy)), "fs_set_partial_merge")
 
 
 def fs_test_stall_loads(on):

@@ -247,6 +247,8 @@ bool g_test_stall = false;
 
 // fs_set_cta_pairs: -1 automatic, 0 never, 1 whenever the call allows it.
 int g_pair_policy = -1;
+// fs_set_partial_merge: -1 automatic, 0 never, 1 always (single CTAs, <= 64 rows).
+int g_merge_policy = -1;
 
 int bn_index(int BN) { return BN / 16 - 1; }
 
@@ -288,6 +290,39 @@ struct ShardOpts {
   uint32_t tp_seq = 0;
   void *const *tp_areas = nullptr;
 };
+
+// Whether the kernel variant with merged 8-row partial tiles pays for this
+// vocabulary split: at least one CTA in ten starts a segment with an 8-row
+// partial tile (the Qwen3 heads: 48 of 148).  Elsewhere its extra slot per
+// stage only costs ring space.  Remembers the last few answers.
+bool merge_partials(const Schedule &sch) {
+  if (g_merge_policy >= 0) return g_merge_policy == 1;
+  struct Entry {
+    int V, G, num_ctas;
+    bool merge;
+  };
+  static Entry memo[8];
+  static int memo_next = 0, memo_used = 0;
+  for (int i = 0; i < memo_used; ++i)
+    if (memo[i].V == sch.V && memo[i].G == sch.G && memo[i].num_ctas == sch.num_ctas)
+      return memo[i].merge;
+  int with = 0;
+  for (int c = 0; c < sch.num_ctas; ++c) {
+    fmms::TileIter it(sch, c, 1);
+    fmms::Tile t;
+    while (it.next(t)) {
+      if (t.pstart >= 0) {
+        ++with;
+        break;
+      }
+    }
+  }
+  const bool merge = with * 10 >= sch.num_ctas;
+  memo[memo_next] = Entry{sch.V, sch.G, sch.num_ctas, merge};
+  memo_next = (memo_next + 1) % 8;
+  if (memo_used < 8) ++memo_used;
+  return merge;
+}
 
 // The fused path in all three modes, chunked over 256 batch rows.
 fs_status run_locked(int mode, const void *H, const void *W, int B, int d, int V, int G,
@@ -374,7 +409,8 @@ fs_status run_locked(int mode, const void *H, const void *W, int B, int d, int V
       if (fmms::launch_fmms_pair(mode, BN, tw, twp, th, p, stream) != cudaSuccess)
         return FS_ERR_CUDA;
     } else {
-      if (fmms::launch_fmms(mode, BN, tw, twp, th, p, stream) != cudaSuccess) return FS_ERR_CUDA;
+      if (fmms::launch_fmms(mode, BN, merge_partials(sch), tw, twp, th, p, stream) != cudaSuccess)
+        return FS_ERR_CUDA;
     }
 
     if (mode == fmms::kModeGrouped) {
@@ -849,6 +885,13 @@ fs_status fs_gumbel(const uint32_t *r, float *g, int64_t n, fs_stream_t stream) 
   return fmms::launch_gumbel_test(r, g, n, static_cast<cudaStream_t>(stream)) == cudaSuccess
              ? FS_OK
              : FS_ERR_CUDA;
+}
+
+fs_status fs_set_partial_merge(int policy) {
+  if (policy < -1 || policy > 1) return FS_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(g_mu);
+  g_merge_policy = policy;
+  return FS_OK;
 }
 
 fs_status fs_set_cta_pairs(int policy) {

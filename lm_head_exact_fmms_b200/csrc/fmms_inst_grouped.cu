@@ -1,14 +1,17 @@
-// fmms_inst_grouped.cu -- the fused kernel in grouped mode on single CTAs, built for every batch tile.
+// fmms_inst_grouped.cu -- the fused kernel in grouped mode on single CTAs, built for every batch tile
+// (up to 64 rows also with merged 8-row partial tiles).
 #include "fmms_kernel.cuh"
 #include "launch.h"
 
 namespace fmms {
 
-cudaError_t launch_grouped(int BN, const CUtensorMap &tw, const PartMaps &twp,
+cudaError_t launch_grouped(int BN, bool merge, const CUtensorMap &tw, const PartMaps &twp,
                            const CUtensorMap &th, const FmmsParams &p, cudaStream_t stream) {
   switch (BN) {
 #define FMMS_CASE(n) \
-  case n: return launch_t<n, kModeGrouped>(tw, twp, th, p, stream);
+  case n:                                                                 \
+    return merge ? launch_t<n, kModeGrouped, (n <= 64)>(tw, twp, th, p, stream)     \
+                 : launch_t<n, kModeGrouped, false>(tw, twp, th, p, stream);
     FMMS_FOR_EACH_BN(FMMS_CASE)
 #undef FMMS_CASE
     default: return cudaErrorInvalidValue;

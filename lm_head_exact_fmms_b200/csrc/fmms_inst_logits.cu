@@ -4,11 +4,13 @@
 
 namespace fmms {
 
-cudaError_t launch_logits(int BN, const CUtensorMap &tw, const PartMaps &twp,
+cudaError_t launch_logits(int BN, bool merge, const CUtensorMap &tw, const PartMaps &twp,
                           const CUtensorMap &th, const FmmsParams &p, cudaStream_t stream) {
   switch (BN) {
 #define FMMS_CASE(n) \
-  case n: return launch_t<n, kModeLogits>(tw, twp, th, p, stream);
+  case n:                                                                 \
+    return merge ? launch_t<n, kModeLogits, (n <= 64)>(tw, twp, th, p, stream)     \
+                 : launch_t<n, kModeLogits, false>(tw, twp, th, p, stream);
     FMMS_FOR_EACH_BN(FMMS_CASE)
 #undef FMMS_CASE
     default: return cudaErrorInvalidValue;

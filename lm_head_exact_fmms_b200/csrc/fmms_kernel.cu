@@ -6,12 +6,12 @@
 
 namespace fmms {
 
-cudaError_t launch_fmms(int mode, int BN, const CUtensorMap &tw, const PartMaps &twp,
+cudaError_t launch_fmms(int mode, int BN, bool merge, const CUtensorMap &tw, const PartMaps &twp,
                         const CUtensorMap &th, const FmmsParams &p, cudaStream_t stream) {
   switch (mode) {
-    case kModeFlat: return launch_flat(BN, tw, twp, th, p, stream);
-    case kModeGrouped: return launch_grouped(BN, tw, twp, th, p, stream);
-    case kModeLogits: return launch_logits(BN, tw, twp, th, p, stream);
+    case kModeFlat: return launch_flat(BN, merge, tw, twp, th, p, stream);
+    case kModeGrouped: return launch_grouped(BN, merge, tw, twp, th, p, stream);
+    case kModeLogits: return launch_logits(BN, merge, tw, twp, th, p, stream);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -89,18 +89,20 @@ constexpr int tmem_cols_for(int cols) {
   return n;
 }
 
-template <int BN, int MODE, bool PAIR = false>
+template <int BN, int MODE, bool PAIR = false, bool MERGE = false>
 struct KCfg {
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= kMaxBN, "batch tile: a multiple of 16 rows");
   static_assert(!PAIR || MODE != kModeLogits, "the logits mode runs on single CTAs");
   static constexpr int kHRows = PAIR ? BN / 2 : BN;     // H rows this CTA stages
   static constexpr int kCombBytes = MODE == kModeGrouped ? 4 * BN * 16 : 0;  // grouped only
-  // Merged 8-row partial tiles (single CTAs of up to 64 batch rows; above
-  // that CTA pairs run): each stage starts with one 8-row W slot per
-  // sub-block.  (At 16 rows the extra kilobyte turns the ring from 4 x 3
-  // into 2 x 5 sub-blocks, 160 instead of 192 KB of W in flight; merging
-  // still wins: Qwen3-8B head B=1 191.5 -> 186.5 us.)
-  static constexpr bool kMerge = !PAIR && BN <= 64;
+  // Merged 8-row partial tiles (MERGE; single CTAs of up to 64 batch rows,
+  // above that CTA pairs run): each stage starts with one 8-row W slot per
+  // sub-block.  The host picks this variant for vocabularies whose split
+  // gives many CTAs an 8-row partial tile (the Qwen3 heads: B=1 191.5 ->
+  // 186.5 us, B=64 198 -> 192 us); elsewhere the slot only costs ring space
+  // (at 16 rows the ring goes from 4 x 3 to 2 x 5 sub-blocks) and the
+  // d=8192 head ran 3-4 % slower with it.
+  static constexpr bool kMerge = MERGE && !PAIR && BN <= 64;
   static constexpr int kSubP = kMerge ? kGranule * kBlockK * 2 : 0;  // 1 KB per sub-block
   static constexpr int kSub = ksub_for(kHRows, kCombBytes, kSubP);  // 64-wide K blocks per stage
   static constexpr int kSubW = kTileM * kBlockK * 2;    // 16 KB of W per sub-block
@@ -451,11 +453,11 @@ __device__ __forceinline__ uint32_t w_sub_bytes(int rows) {
 }
 
 // The H loads of one stage (this CTA's rows of the batch operand).
-template <int BN, int MODE, bool PAIR>
+template <int BN, int MODE, bool PAIR, bool MERGE = false>
 __device__ __forceinline__ void issue_h(const CUtensorMap *th, const FmmsParams &p,
                                         uint8_t *stages, uint64_t *full, int stage, int sub0,
                                         int nsub, int rank, uint64_t pol_h) {
-  using C = KCfg<BN, MODE, PAIR>;
+  using C = KCfg<BN, MODE, PAIR, MERGE>;
   uint8_t *sh0 = stages + stage * C::kStageBytes + C::kOffH;
   const uint32_t bar = PAIR ? sm100::cluster_addr(&full[stage], 0) : 0u;
 #pragma unroll
@@ -475,13 +477,13 @@ __device__ __forceinline__ void issue_h(const CUtensorMap *th, const FmmsParams 
 // every stage (128 W rows, BN/2 H rows) and count the bytes on the even
 // CTA's full barrier; the even CTA also hands each freed stage on to the odd
 // CTA, whose MMA reads happen in the even CTA's tcgen05 pipeline.
-template <int BN, int MODE, bool PAIR>
+template <int BN, int MODE, bool PAIR, bool MERGE = false>
 __device__ __forceinline__ void role_producer(const CUtensorMap *tw, const PartMaps *twp,
                                               const CUtensorMap *th, const FmmsParams &p,
                                               const Schedule &sch, uint8_t *stages,
                                               uint64_t *full, uint64_t *empty,
                                               volatile int *abort_flag, int unit, int rank) {
-  using C = KCfg<BN, MODE, PAIR>;
+  using C = KCfg<BN, MODE, PAIR, MERGE>;
   const uint64_t pol_w = sm100::l2_policy_evict_first();
   const uint64_t pol_h = sm100::l2_policy_evict_last();
   TileIter it(sch, unit, C::kMerge ? 1 : 0);
@@ -590,7 +592,7 @@ __device__ __forceinline__ void role_producer(const CUtensorMap *tw, const PartM
             // After a timeout too: the loads stay in bounds, and completing
             // the stages lets the drain below account for every copy.
             for (int q = 0; q < npend; ++q)
-              issue_h<BN, MODE, PAIR>(th, p, stages, full, pend_stage[q], pend_sub0[q],
+              issue_h<BN, MODE, PAIR, MERGE>(th, p, stages, full, pend_stage[q], pend_sub0[q],
                                       pend_nsub[q], rank, pol_h);
             npend = 0;
             if (!landed) {
@@ -601,7 +603,7 @@ __device__ __forceinline__ void role_producer(const CUtensorMap *tw, const PartM
           }
         }
       }
-      if (h_now) issue_h<BN, MODE, PAIR>(th, p, stages, full, stage, sub0, nsub, rank, pol_h);
+      if (h_now) issue_h<BN, MODE, PAIR, MERGE>(th, p, stages, full, stage, sub0, nsub, rank, pol_h);
       ++issued;
       if (++stage == C::kStages) {
         stage = 0;
@@ -613,7 +615,7 @@ __device__ __forceinline__ void role_producer(const CUtensorMap *tw, const PartM
     // The CTA's last stages are still waiting for H (a range shorter than the ring).
     const bool landed = sm100::wait_flag_bounded(p.h_ready + pend_need, p.h_epoch, abort_flag, p.err);
     for (int q = 0; q < npend; ++q)
-      issue_h<BN, MODE, PAIR>(th, p, stages, full, pend_stage[q], pend_sub0[q], pend_nsub[q], rank,
+      issue_h<BN, MODE, PAIR, MERGE>(th, p, stages, full, pend_stage[q], pend_sub0[q], pend_nsub[q], rank,
                               pol_h);
     npend = 0;
     ok = landed;
@@ -636,13 +638,13 @@ __device__ __forceinline__ void role_producer(const CUtensorMap *tw, const PartM
 }
 
 // MMA issuer (one thread; in pair mode only the even CTA's).
-template <int BN, int MODE, bool PAIR>
+template <int BN, int MODE, bool PAIR, bool MERGE = false>
 __device__ __forceinline__ void role_mma(const FmmsParams &p, const Schedule &sch,
                                          uint8_t *stages, uint64_t *full, uint64_t *empty,
                                          uint64_t *acc_full, uint64_t *acc_empty,
                                          uint64_t *drain_bar, uint32_t tmem_base,
                                          volatile int *abort_flag, int unit) {
-  using C = KCfg<BN, MODE, PAIR>;
+  using C = KCfg<BN, MODE, PAIR, MERGE>;
   TileIter it(sch, unit, C::kMerge ? 1 : 0);
   Tile tile;
   int stage = 0;
@@ -745,14 +747,14 @@ __device__ __forceinline__ void role_mma(const FmmsParams &p, const Schedule &sc
 // (its half of the pair tile); the even CTA hands every filled accumulator on
 // to the odd CTA, and the odd CTA's warps release it on the even CTA's
 // barrier, where the MMAs are issued.
-template <int BN, int MODE, bool PAIR>
+template <int BN, int MODE, bool PAIR, bool MERGE = false>
 __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedule &sch,
                                               uint32_t tmem_base, uint64_t *acc_full,
                                               uint64_t *acc_empty, volatile int *abort_flag,
                                               int *last_flag, uint64_t *comb_key, float *comb_m,
                                               float *comb_s, int warp, int lane, int unit,
                                               int rank) {
-  using C = KCfg<BN, MODE, PAIR>;
+  using C = KCfg<BN, MODE, PAIR, MERGE>;
   constexpr int CW = C::kCW;
   const int q = warp & 3;          // TMEM lane quarter this warp may access
   const int h = (warp - 2) >> 2;   // which of the quarter's warps: chunks h, h+4, ...
@@ -967,12 +969,12 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
 // ---------------------------------------------------------------------------
 // Kernel
 // ---------------------------------------------------------------------------
-template <int BN, int MODE, bool PAIR>
+template <int BN, int MODE, bool PAIR, bool MERGE = false>
 __global__ void __launch_bounds__(kThreads, 1)
     fmms_kernel(const __grid_constant__ CUtensorMap tmap_w,
                 const __grid_constant__ PartMaps tmap_wp,
                 const __grid_constant__ CUtensorMap tmap_h, const FmmsParams p) {
-  using C = KCfg<BN, MODE, PAIR>;
+  using C = KCfg<BN, MODE, PAIR, MERGE>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -1044,16 +1046,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     if (lane == 0)
-      role_producer<BN, MODE, PAIR>(&tmap_w, &tmap_wp, &tmap_h, p, sch, stages, full, empty,
+      role_producer<BN, MODE, PAIR, MERGE>(&tmap_w, &tmap_wp, &tmap_h, p, sch, stages, full, empty,
                                     abort_flag, unit, rank);
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0 && rank == 0)
-      role_mma<BN, MODE, PAIR>(p, sch, stages, full, empty, acc_full, acc_empty, drain_bar,
+      role_mma<BN, MODE, PAIR, MERGE>(p, sch, stages, full, empty, acc_full, acc_empty, drain_bar,
                                tmem_base, abort_flag, unit);
     __syncwarp();
   } else {
-    role_epilogue<BN, MODE, PAIR>(p, sch, tmem_base, acc_full, acc_empty, abort_flag, last_flag,
+    role_epilogue<BN, MODE, PAIR, MERGE>(p, sch, tmem_base, acc_full, acc_empty, abort_flag, last_flag,
                                   comb_key, comb_m, comb_s, warp, lane, unit, rank);
   }
 
@@ -1079,11 +1081,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------------------
 // Host launchers
 // ---------------------------------------------------------------------------
-template <int BN, int MODE>
+template <int BN, int MODE, bool MERGE = false>
 cudaError_t launch_t(const CUtensorMap &tw, const PartMaps &twp, const CUtensorMap &th,
                             const FmmsParams &p, cudaStream_t stream) {
-  using C = KCfg<BN, MODE>;
-  auto kern = fmms_kernel<BN, MODE, false>;
+  using C = KCfg<BN, MODE, false, MERGE>;
+  auto kern = fmms_kernel<BN, MODE, false, MERGE>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;

@@ -21,11 +21,11 @@ struct PartMaps {
 int fmms_batch_tile(int rows);
 
 // Per-mode launchers for every batch tile (fmms_inst_*.cu).
-cudaError_t launch_flat(int BN, const CUtensorMap &tw, const PartMaps &twp,
+cudaError_t launch_flat(int BN, bool merge, const CUtensorMap &tw, const PartMaps &twp,
                         const CUtensorMap &th, const FmmsParams &p, cudaStream_t stream);
-cudaError_t launch_grouped(int BN, const CUtensorMap &tw, const PartMaps &twp,
+cudaError_t launch_grouped(int BN, bool merge, const CUtensorMap &tw, const PartMaps &twp,
                            const CUtensorMap &th, const FmmsParams &p, cudaStream_t stream);
-cudaError_t launch_logits(int BN, const CUtensorMap &tw, const PartMaps &twp,
+cudaError_t launch_logits(int BN, bool merge, const CUtensorMap &tw, const PartMaps &twp,
                           const CUtensorMap &th, const FmmsParams &p, cudaStream_t stream);
 cudaError_t launch_flat_pair(int BN, const CUtensorMap &tw, const PartMaps &twp,
                              const CUtensorMap &th, const FmmsParams &p, cudaStream_t stream);
@@ -36,7 +36,7 @@ cudaError_t pair_units_grouped(int BN, int *units);
 
 // The fused kernel in mode kModeFlat / kModeGrouped / kModeLogits with batch
 // tile BN, grid p.num_ctas x kThreads threads.
-cudaError_t launch_fmms(int mode, int BN, const CUtensorMap &tw, const PartMaps &twp,
+cudaError_t launch_fmms(int mode, int BN, bool merge, const CUtensorMap &tw, const PartMaps &twp,
                         const CUtensorMap &th, const FmmsParams &p, cudaStream_t stream);
 
 // The flat or grouped kernel on CTA pairs (clusters of two, tcgen05
