@@ -433,7 +433,10 @@ fs_status fs_set_partial_merge(int policy);
  * max_tiles rows of int32 [5] = (tile start, first valid token, end of valid
  * tokens, partial slot, last-tile-of-segment flag) for CTA `cta` and returns
  * the count in *ntiles.  Tiles are 128 tokens; a CTA's range is a multiple
- * of 8 tokens (except at V); a tile never crosses a group boundary. */
+ * of 8 tokens (except at V); a tile never crosses a group boundary.  (With
+ * merged partial tiles, fs_set_partial_merge, the kernel multiplies an 8-row
+ * partial tile in the same pipeline stages as the tile after it; the tiles
+ * and slots listed here stay the same.) */
 fs_status fs_plan_tiles(int V, int G, int num_sms, int cta, int32_t *tiles,
                         int max_tiles, int *ntiles, int *num_ctas_out);
 
