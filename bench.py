@@ -411,7 +411,9 @@ def run_gpu(args, world, rank, local):
         "clocks": sampler.summary(),
     }
 
-    if rank == 0 and not args.no_sweep:
+    # The single-GPU characterisation (batch sweep, other modes) runs at N=1
+    # only: at N > 1 it would hold the other GPUs idle while rank 0 works.
+    if rank == 0 and world == 1 and not args.no_sweep:
         result["sweep"] = sweep(torch, binding, synth, W, wl, dev, stream, peaks, peak_kind)
         result["grouped_masked"] = grouped_points(torch, binding, synth, dev, stream, peaks,
                                                   peak_kind, W)
