@@ -33,6 +33,10 @@
 //  * flat mode: every improvement of a row's maximum is published with one
 //    atomicMax of a packed (score, token) key; the last CTA to finish (atomic
 //    ticket, no waiting) decodes the tokens and re-zeroes the keys;
+//  * a CTA range's 8-row partial tile either runs as a tile of its own or
+//    (MERGE variant) rides along with the first whole tile: its rows get a
+//    1 KB slot per stage and a second MMA into an accumulator of its own,
+//    sharing the H loads;
 //  * grouped mode: per (segment, row) partial (max key, lse pieces) for the
 //    Group-Gumbel-Max merge kernel;
 //  * logits mode: raw fp32 logits to HBM for the unfused measurement path.
@@ -445,7 +449,9 @@ __device__ __forceinline__ void tp_exchange(const FmmsParams &p, int etid, int *
 // ---------------------------------------------------------------------------
 
 // Bytes of W a CTA loads per 64-wide K sub-block for `rows` rows from the
-// tile start (whole tile: one 128-row box; otherwise 8-row boxes).
+// tile start: 16 KB for a whole tile (one 128-row box, also for a tile cut
+// short by fewer than 8 rows), else one kilobyte per 8-row granule (boxes of
+// 64, 32, 16 and 8 rows).
 __device__ __forceinline__ uint32_t w_sub_bytes(int rows) {
   if (rows <= 0) return 0u;
   if (rows >= kTileM) return static_cast<uint32_t>(kTileM * kBlockK * 2);
