@@ -385,7 +385,7 @@ fs_status run_locked(int mode, const void *H, const void *W, int B, int d, int V
     p.row_seeds = row_seeds;
     p.mask = mask;
     p.mask_words = ((shard.V_total > 0 ? shard.V_total : V) + 31) / 32;
-    p.out_idx = out_idx + static_cast<size_t>(b0) * S;
+    p.out_idx = out_idx ? out_idx + static_cast<size_t>(b0) * S : nullptr;
     p.keys = w.keys;
     p.ticket = w.ticket;
     p.err = w.err;
@@ -681,8 +681,7 @@ fs_status fs_sample_tp(const void *H, const void *W_shard, int B, int d, int V_s
                        const uint64_t *row_seeds, uint32_t step, const uint32_t *mask_bits,
                        void *const *areas, int world, uint32_t seq, void *workspace,
                        size_t workspace_bytes, fs_stream_t stream) {
-  static int32_t unused;  // the tokens go to the exchange areas
-  fs_status s = validate(H, W_shard, B, d, V_shard, temperature, &unused);
+  fs_status s = validate(H, W_shard, B, d, V_shard, temperature, areas);  // tokens go to the areas
   if (s != FS_OK) return s;
   if (B > fmms::kMaxBN) return FS_ERR_UNSUPPORTED;
   if (vocab_offset < 0 || (vocab_offset % fmms::kGranule) != 0 || V_total < 1 ||
@@ -700,7 +699,7 @@ fs_status fs_sample_tp(const void *H, const void *W_shard, int B, int d, int V_s
   opts.tp_areas = areas;
   std::lock_guard<std::mutex> lock(g_mu);
   return run_locked(fmms::kModeFlat, H, W_shard, B, d, V_shard, 1, temperature, seed, row_seeds,
-                    step, mask_bits, &unused, nullptr, nullptr, workspace, workspace_bytes,
+                    step, mask_bits, nullptr, nullptr, nullptr, workspace, workspace_bytes,
                     static_cast<cudaStream_t>(stream), opts);
 }
 
