@@ -312,6 +312,39 @@ def cpu_baseline(H, W, wl, B, rs, budget_s=12.0, max_rows=64):
             "seconds": round(sum(times), 2)}
 
 
+def oracle_per_workload(slice_rows=8192, reps=3):
+    """The oracle timed on this host's cores for one row of every workload:
+    `reps` rows over a vocabulary slice of at most `slice_rows` tokens (the
+    whole head for the tiny one), scaled by V / slice to a full-vocabulary
+    row, which is one B=1 call."""
+    import numpy as np
+    import oracle
+    from lm_head_exact_fmms_b200 import synth
+    out = []
+    for name, wl in synth.WORKLOADS.items():
+        Vs = min(wl.V, slice_rows)
+        Ws = synth.make_weight(Vs, wl.d, wl.w_std)
+        H = synth.make_hidden(reps, wl.d)
+        rs = synth.make_row_seeds(reps) if wl.per_row_seeds else None
+        mask = synth.make_mask(reps, Vs, wl.mask_allowed) if wl.groups else None
+        times = []
+        for r in range(reps):
+            rows = np.array([r], dtype=np.int32)
+            t0 = time.perf_counter()
+            if wl.groups:
+                oracle.sample_grouped(H, Ws, wl.groups, T=wl.temperature, mask=mask, rows=rows)
+            else:
+                oracle.sample(H, Ws, T=wl.temperature, row_seeds=rs, rows=rows)
+            times.append(time.perf_counter() - t0)
+        per_row = sorted(times)[len(times) // 2] * wl.V / Vs
+        out.append({"workload": name, "d": wl.d, "V": wl.V,
+                    "us_per_row": round(per_row * 1e6, 1),
+                    "sample": "median of %d rows x %d-token slice, scaled by V/%d"
+                              % (reps, Vs, Vs)})
+    return {"cores": oracle.num_threads(), "cpu": cpu_model(), "kind": "oracle",
+            "points": out}
+
+
 def run_gpu(args, world, rank, local):
     import torch
 
@@ -427,8 +460,11 @@ def run_gpu(args, world, rank, local):
         result["multi_sample"] = multi_point(torch, binding, synth, W, wl, dev, stream, B)
         result["cuda_graph"] = graph_point(torch, binding, synth, W, wl, dev, B)
         result["top_k"] = topk_point(torch, binding, synth, W, wl, dev, stream, B)
+        result["tiny"] = tiny_point(torch, binding, synth, dev, stream)
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not grouped:
         result["cpu_baseline"] = cpu_baseline(H, W, wl, B, rs)
+        if not args.no_sweep:
+            result["cpu_baseline"]["per_workload"] = oracle_per_workload()
     if fused_tp:
         exchange.close()  # every rank, after its last call
     return result
@@ -548,6 +584,55 @@ def graph_point(torch, binding, synth, W, wl, dev, B, calls=10, replays=30):
         return {"B": B, "us_per_call": round(us, 3), "calls_per_graph": calls}
     except Exception as exc:   # report, do not break the bench line
         return {"B": B, "us_per_call": None, "error": str(exc)[:200]}
+
+
+def tiny_point(torch, binding, synth, dev, stream, copies=64, steps=640, graph_calls=64,
+               replays=10):
+    """The tiny head (d=256, V=4096, 2 MiB of W): launch latency, not
+    bandwidth.  Each call reads the next of `copies` distinct W tensors
+    (128 MiB in all, above the 126 MB L2), so no call finds its W in L2.
+    Reported per call through the stream and inside a CUDA graph."""
+    wl = synth.WORKLOADS["tiny"]
+    B = wl.batches[0]
+    try:
+        Ws = [synth.make_weight(wl.V, wl.d, wl.w_std, seed=1234 + c, device=dev)
+              for c in range(copies)]
+        H = synth.make_hidden(B, wl.d, device=dev)
+        out = torch.empty(B, dtype=torch.int32, device=dev)
+        ws = torch.zeros(binding.fs_workspace_bytes(B, wl.V, 0), dtype=torch.uint8, device=dev)
+
+        def step(i):
+            binding.fs_sample_ex(H, Ws[i % copies], temperature=wl.temperature, seed=0, step=i,
+                                 out_idx=out, workspace=ws, stream=stream)
+
+        region_ms, per = time_calls(step, steps, 3 * copies, stream)
+        res = {"workload": "tiny head d=%d V=%d B=%d, %d rotating W copies (%d MiB)"
+                           % (wl.d, wl.V, B, copies, copies * wl.V * wl.d * 2 >> 20),
+               "us_per_call": round(region_ms * 1e3 / steps, 3),
+               "kernel_us_p10_p50_p90": [round(x, 3) for x in percentiles(per)]}
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            for i in range(graph_calls):
+                binding.fs_sample_ex(H, Ws[i % copies], temperature=wl.temperature, seed=0,
+                                     step=i, out_idx=out, workspace=ws, stream=s)
+        torch.cuda.synchronize()
+        g.replay()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(replays):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        res["graph_us_per_call"] = round(e0.elapsed_time(e1) * 1e3 / (replays * graph_calls), 3)
+        del g
+        return res
+    except Exception as exc:   # report, do not break the bench line
+        return {"us_per_call": None, "error": str(exc)[:200]}
 
 
 def topk_point(torch, binding, synth, W, wl, dev, stream, B, K=50, steps=100):
