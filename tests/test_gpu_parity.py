@@ -110,12 +110,33 @@ def test_gumbel_transform_accuracy(dev, oracle):
     r = gumbel_rs()
     ref = oracle.gumbel(r)
     got = binding.fs_gumbel(torch.from_numpy(r.view(np.int32)).to(dev)).cpu().numpy()
+    gumbel_check_chunk(r, got, ref)
+
+
+
+def gumbel_check_chunk(r, got, ref):
+    """Asserts the transform's bound on one chunk of increasing words."""
     assert np.all(np.isfinite(got))
     ulp = np.spacing(np.abs(ref).astype(np.float32)).astype(np.float64)
     tol = GUMBEL_ULPS * ulp + GUMBEL_ABS
     err = np.abs(got.astype(np.float64) - ref)
-    assert np.all(err <= tol), ((err / ulp).max(), err.max())
+    assert np.all(err <= tol), (int(r[np.argmax(err / tol)]), (err / ulp).max(), err.max())
     assert np.all(np.diff(got.astype(np.float64)) >= -2 * tol[1:])
+    return float((err / ulp).max())
+
+
+def test_gumbel_transform_stratified_2_27(dev, oracle):
+    """The same bound on 2^27 words, one drawn from every aligned block of 32
+    (1.3e8 of the 2^32 inputs, every part of the range), in 2^24-word
+    chunks."""
+    rng = np.random.default_rng(20260)
+    n_all, chunk = 1 << 27, 1 << 24
+    for c0 in range(0, n_all, chunk):
+        base = np.arange(c0, c0 + chunk, dtype=np.uint64) << np.uint64(5)
+        r = (base + rng.integers(0, 32, size=chunk, dtype=np.uint64)).astype(np.uint32)
+        ref = oracle.gumbel(r)
+        got = binding.fs_gumbel(torch.from_numpy(r.view(np.int32)).to(dev)).cpu().numpy()
+        gumbel_check_chunk(r, got, ref)
 
 
 # ------------------------------------------------------------ flat sampling
