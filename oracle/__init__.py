@@ -38,6 +38,8 @@ def _load():
     lib = ctypes.CDLL(path)
     lib.oracle_philox4x32_10.argtypes = [_u32p, _u32p, _u32p]
     lib.oracle_philox_batch.argtypes = [_u32p, _u32p, _u32p, ctypes.c_int64]
+    lib.oracle_philox_digest.argtypes = [ctypes.c_uint32] * 4 + [ctypes.c_uint64, ctypes.c_int64]
+    lib.oracle_philox_digest.restype = ctypes.c_uint64
     lib.oracle_noise_word.argtypes = [ctypes.c_uint64, ctypes.c_uint32, ctypes.c_uint32,
                                       ctypes.c_uint32, ctypes.c_uint32]
     lib.oracle_noise_word.restype = ctypes.c_uint32
@@ -97,6 +99,14 @@ def philox4x32_10(ctr, key):
     n = ctr.size // 4
     lib.oracle_philox_batch(_ptr(ctr, _u32p), _ptr(key, _u32p), _ptr(out, _u32p), n)
     return out
+
+
+def philox_digest(ctr0, seed, n) -> int:
+    """Digest of the Philox words of the n counters (ctr0[0] + i mod 2^32,
+    ctr0[1], ctr0[2], ctr0[3]) under `seed`: sum of word j of counter i times
+    (4 i + j + 1), mod 2^64."""
+    c = [int(x) & 0xFFFFFFFF for x in ctr0]
+    return int(_load().oracle_philox_digest(c[0], c[1], c[2], c[3], int(seed) % (1 << 64), int(n)))
 
 
 def noise_word(seed, step, row, index, tag=0) -> int:

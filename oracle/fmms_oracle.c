@@ -98,6 +98,26 @@ void oracle_philox_batch(const uint32_t *ctrs, const uint32_t *keys,
     oracle_philox4x32_10(ctrs + 4 * i, keys + 2 * i, outs + 4 * i);
 }
 
+/* A 64-bit digest of the Philox words of the n consecutive counters
+ * (c0 + i mod 2^32, c1, c2, c3), i = 0..n-1, under the key of `seed`:
+ * the sum over i and j of word j of counter i times (4 i + j + 1), mod 2^64.
+ * It lets a test compare two Philox implementations on billions of counters
+ * without storing their words: for n <= 2^28 every weight is below 2^30, so
+ * any single differing word changes the digest. */
+uint64_t oracle_philox_digest(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3,
+                              uint64_t seed, int64_t n) {
+  const uint32_t key[2] = {(uint32_t)(seed & 0xFFFFFFFFu), (uint32_t)(seed >> 32)};
+  uint64_t total = 0;
+#pragma omp parallel for schedule(static) reduction(+ : total)
+  for (int64_t i = 0; i < n; ++i) {
+    const uint32_t ctr[4] = {c0 + (uint32_t)i, c1, c2, c3};
+    uint32_t out[4];
+    oracle_philox4x32_10(ctr, key, out);
+    for (int j = 0; j < 4; ++j) total += (uint64_t)out[j] * (uint64_t)(4 * i + j + 1);
+  }
+  return total;
+}
+
 /* The 32-bit noise word for (seed, step, row, index, tag). */
 uint32_t oracle_noise_word(uint64_t seed, uint32_t step, uint32_t row,
                            uint32_t index, uint32_t tag) {

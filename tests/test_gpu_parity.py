@@ -86,6 +86,45 @@ def test_philox_bitwise_sequential_counters(dev, oracle):
         del t_ctr, t_key
 
 
+def signed32(x):
+    """int64 tensor of u32 values -> the same bit patterns as int32."""
+    return (x - ((x >> 31) & 1) * (1 << 32)).to(torch.int32)
+
+
+def device_philox_digest(dev, ctr0, seed, n):
+    """The oracle's Philox digest computed from the device Philox: counters
+    (ctr0[0] + i mod 2^32, ctr0[1], ctr0[2], ctr0[3]), the sum of word j of
+    counter i times (4 i + j + 1) mod 2^64, summed as 32-bit halves so that
+    no int64 sum overflows."""
+    i = torch.arange(n, dtype=torch.int64, device=dev)
+    ctr = torch.empty(n, 4, dtype=torch.int64, device=dev)
+    ctr[:, 0] = (i + int(ctr0[0])) & 0xFFFFFFFF
+    for j in range(1, 4):
+        ctr[:, j] = int(ctr0[j]) & 0xFFFFFFFF
+    key = torch.tensor([seed & 0xFFFFFFFF, seed >> 32], dtype=torch.int64, device=dev)
+    key = signed32(key).expand(n, 2).contiguous()
+    words = binding.fs_philox4x32_10(signed32(ctr), key).to(torch.int64) & 0xFFFFFFFF
+    del ctr, key
+    prod = words * torch.arange(1, 4 * n + 1, dtype=torch.int64, device=dev).view(n, 4)
+    lo = int((prod & 0xFFFFFFFF).sum())
+    hi = int((prod >> 32).sum())
+    return ((hi << 32) + lo) % (1 << 64)
+
+
+def test_philox_digest_2_30_counters(dev, oracle):
+    """2^30 counters (64 runs of 2^24 consecutive ones: word 0, the token
+    index / 4, covers [0, 2^30) -- every token index below 2^32 -- under
+    varied row, step, tag and key): the device Philox and the oracle's agree
+    on each run's digest, in which any single differing word would show."""
+    rng = np.random.default_rng(2030)
+    n = 1 << 24
+    for k in range(64):
+        ctr0 = (k * n, (k * 2654435761) & 0xFFFFFFFF, (k * 0x85EBCA6B) & 0xFFFFFFFF, k % 3)
+        seed = int(rng.integers(0, 2 ** 63)) * 2 + (k & 1)
+        assert device_philox_digest(dev, ctr0, seed, n) == oracle.philox_digest(ctr0, seed, n), \
+            (k, ctr0, seed)
+
+
 def gumbel_rs():
     lo = np.arange(0, 1 << 20, dtype=np.uint64)
     hi = np.arange((1 << 32) - (1 << 20), 1 << 32, dtype=np.uint64)

@@ -113,6 +113,26 @@ def test_philox_bit_balance_and_bytes(oracle):
     assert len(np.unique(out)) > 0.999 * out.size
 
 
+
+def test_philox_digest_definition(oracle):
+    """The digest helper equals its definition written out over the oracle's
+    own words (word 0 of the counter wrapping past 2^32), and a change of one
+    word in one counter changes it."""
+    n = 5000
+    c0 = (0xFFFFFFFF - 1234, 77, 0xDEADBEEF, 2)
+    seed = 0x0123456789ABCDEF
+    ctrs = np.empty((n, 4), dtype=np.uint32)
+    ctrs[:, 0] = (np.arange(n, dtype=np.uint64) + c0[0]).astype(np.uint32)
+    ctrs[:, 1:] = c0[1:]
+    words = oracle.philox4x32_10(ctrs, np.array([seed & 0xFFFFFFFF, seed >> 32], dtype=np.uint32))
+    weights = np.arange(1, 4 * n + 1, dtype=object).reshape(n, 4)
+    want = int((words.astype(object) * weights).sum()) % (1 << 64)
+    assert oracle.philox_digest(c0, seed, n) == want
+    assert oracle.philox_digest(c0, seed ^ 1, n) != want
+    assert oracle.philox_digest((c0[0], c0[1], c0[2], 3), seed, n) != want
+    assert oracle.philox_digest(c0, seed, n - 1) != want
+
+
 # --------------------------------------------------------------------------
 # Gumbel transform g(r) = -log(-log((r+1)/(2^32+1)))
 # --------------------------------------------------------------------------
