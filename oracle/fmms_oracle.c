@@ -484,14 +484,8 @@ void oracle_histogram(const uint16_t *H, const uint16_t *W, int B, int d,
 #pragma omp for schedule(static)
     for (int64_t n = 0; n < nsteps; ++n) {
       uint32_t step = step0 + (uint32_t)n;
-      for (int v = 0; v < V; ++v) {
-        if (!token_allowed(mask, V, b, v)) {
-          s[v] = -INFINITY;
-        } else {
-          uint32_t r = oracle_noise_word(key, step, (uint32_t)b, (uint32_t)v, 0u);
-          s[v] = l[v] / T + oracle_gumbel_from_u32(r);
-        }
-      }
+      /* the samplers' own scores (the nested parallel loop runs on this thread) */
+      scores_from_logits(l, V, T, key, step, b, mask, s);
       int pick;
       if (G <= 0) {
         pick = argmax_scan(s, 0, V, NULL, NULL);

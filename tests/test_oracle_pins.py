@@ -245,6 +245,32 @@ def _chi2_pvalue(counts, probs):
     return stats.chi2.sf(chi2, len(obs_b) - 1)
 
 
+@pytest.mark.parametrize("G", [0, 3])
+def test_histogram_counts_the_sampler_draws(oracle, G):
+    """The draw-counting helper that the distribution pins use returns the
+    bincount of the samplers' own tokens over the same steps (flat, and
+    grouped with uneven groups), masked tokens and row seeds included -- so
+    what those pins show about it holds for the samplers."""
+    V, d, B, row, T, N, step0 = 61, 32, 3, 1, 0.8, 300, 100
+    H = synth.make_hidden(B, d, seed=131)
+    W = synth.make_weight(V, d, 0.35, seed=132)
+    rs = synth.make_row_seeds(B)
+    allowed = torch.from_numpy(np.random.default_rng(133).random((B, V)) < 0.6)
+    mask = synth.mask_from_bool(allowed)
+    counts = oracle.histogram(H, W, row=row, nsteps=N, G=G, T=T, row_seeds=rs, mask=mask,
+                              step0=step0)
+    rows = np.array([row], dtype=np.int32)
+    want = np.zeros(V + 1, dtype=np.int64)
+    for step in range(step0, step0 + N):
+        if G:
+            idx, _, _ = oracle.sample_grouped(H, W, G, T=T, row_seeds=rs, step=step, mask=mask,
+                                              rows=rows)
+        else:
+            idx, _, _ = oracle.sample(H, W, T=T, row_seeds=rs, step=step, mask=mask, rows=rows)
+        want[V if idx[0] < 0 else idx[0]] += 1
+    assert np.array_equal(counts, want)
+
+
 @pytest.mark.parametrize("T", [0.7, 1.0, 2.0])
 def test_gumbel_max_matches_softmax(oracle, T):
     V, d, N = 64, 32, 400_000
@@ -408,6 +434,53 @@ def test_grouped_matches_softmax(oracle, G):
     p = _softmax(oracle.logits(H, W)[0] / T)
     assert counts[V] == 0
     assert _chi2_pvalue(counts[:V], p) > 1e-3
+
+
+def _two_sample_pvalue(a, b, min_count=10):
+    """Chi-square test that two count vectors come from one distribution;
+    bins with fewer than `min_count` draws in total are pooled."""
+    from scipy import stats
+    keep = (a + b) >= min_count
+    table = [np.append(a[keep], a[~keep].sum()), np.append(b[keep], b[~keep].sum())]
+    table = np.array(table)
+    table = table[:, table.sum(axis=0) > 0]
+    return stats.chi2_contingency(table, correction=False)[1]
+
+
+@pytest.mark.parametrize("G", [3, 8])
+def test_grouped_and_flat_draws_agree(oracle, G):
+    """Grouped draws and flat draws, with independent noise, follow one
+    distribution (two-sample chi-square); the same test tells apart flat
+    draws at two temperatures."""
+    V, d, N, T = 64, 32, 200_000, 1.3
+    H = synth.make_hidden(1, d, seed=93)
+    W = synth.make_weight(V, d, 0.35, seed=94)
+    flat = oracle.histogram(H, W, row=0, nsteps=N, T=T, seed=13)[:V]
+    grouped = oracle.histogram(H, W, row=0, nsteps=N, G=G, T=T, seed=14)[:V]
+    assert _two_sample_pvalue(flat, grouped) > 1e-3
+    other_T = oracle.histogram(H, W, row=0, nsteps=N, T=1.0, seed=15)[:V]
+    assert _two_sample_pvalue(flat, other_T) < 1e-6
+
+
+def test_constant_rows_sample_the_noise_argmax(oracle):
+    """With every row of W equal, all logits of a row are equal, so the token
+    is the allowed index of the largest Gumbel value alone: the sampler's
+    noise must be word v&3 of Philox(row seed, (v>>2, row, step, 0)), the
+    layout pinned above, and ties go to the smaller index."""
+    V, d, B = 1000, 16, 4
+    H = synth.make_hidden(B, d, seed=121)
+    w = synth.make_weight(1, d, 0.5, seed=122)
+    W = w.expand(V, d).contiguous()
+    rs = synth.make_row_seeds(B)
+    allowed = torch.from_numpy(np.random.default_rng(123).random((B, V)) < 0.5)
+    mask = synth.mask_from_bool(allowed)
+    for step in (0, 1, 77):
+        idx, _, _ = oracle.sample(H, W, T=0.9, row_seeds=rs, step=step, mask=mask)
+        for b in range(B):
+            words = np.array([oracle.noise_word(int(rs[b]), step, b, v) for v in range(V)],
+                             dtype=np.uint32)
+            g = np.where(allowed[b].numpy(), oracle.gumbel(words), -np.inf)
+            assert idx[b] == int(np.argmax(g)), (step, b)
 
 
 def test_grouped_masked_groups(oracle):
