@@ -16,6 +16,8 @@ Two ways to exchange the keys:
   * tp_sample: an int64 MAX all-reduce of 8 bytes per row through
     torch.distributed (NCCL) after the kernel, then a decode kernel.
 """
+import time
+
 import torch
 import torch.distributed as dist
 
@@ -59,13 +61,70 @@ def exchange_handles(handle, group=None):
     return out
 
 
+class PeerLost(RuntimeError):
+    """A rank of the group did not reach a call in time, or left the group."""
+
+    def __init__(self, seq, missing, left):
+        self.seq, self.missing, self.left = seq, sorted(missing), sorted(left)
+        super().__init__("call %d: rank(s) %s did not check in%s" % (
+            seq, self.missing, (" (left the group: %s)" % self.left) if self.left else ""))
+
+
+class PeerMonitor:
+    """Host-side liveness of the ranks of a group, checked before each launch
+    whose completion depends on the peers (the fused exchange's kernel and
+    stream wait): every rank posts the number of the call it is about to
+    launch in a key-value store (a torch.distributed Store) and waits, for at
+    most `timeout_s`, until every other rank has posted it.  A rank that
+    raised, exited or never arrived is reported here, as PeerLost, before
+    this rank enqueues anything that would wait for it; a rank that leaves on
+    purpose calls leave(), which the others see within one poll interval.
+    Each rank keeps one key per call alive at a time."""
+
+    def __init__(self, store, rank, world, timeout_s=10.0, poll_s=0.05, prefix="fmms/peers"):
+        self.store, self.rank, self.world = store, rank, world
+        self.timeout_s, self.poll_s, self.prefix = timeout_s, poll_s, prefix
+        self._posted = None
+
+    def _key(self, seq, r):
+        return "%s/%d/%d" % (self.prefix, seq, r)
+
+    def _left_key(self, r):
+        return "%s/left/%d" % (self.prefix, r)
+
+    def check_in(self, seq):
+        """Posts call `seq` and returns once every rank has posted it;
+        raises PeerLost otherwise."""
+        self.store.set(self._key(seq, self.rank), b"1")
+        others = [r for r in range(self.world) if r != self.rank]
+        deadline = time.monotonic() + self.timeout_s
+        pending = list(others)
+        while True:
+            pending = [r for r in pending if not self.store.check([self._key(seq, r)])]
+            if not pending:
+                break
+            left = [r for r in pending if self.store.check([self._left_key(r)])]
+            if left or time.monotonic() >= deadline:
+                raise PeerLost(seq, pending, left)
+            time.sleep(self.poll_s)
+        # Every rank has posted `seq`, so none still waits for call seq-1.
+        if self._posted is not None:
+            self.store.delete_key(self._key(self._posted, self.rank))
+        self._posted = seq
+
+    def leave(self):
+        """Tells the other ranks that this one takes no further calls."""
+        self.store.set(self._left_key(self.rank), b"1")
+
+
 class FusedExchange:
     """The exchange areas of a process group for fs_sample_tp: this rank's
     own area and its peers', mapped here by CUDA IPC.  Every rank calls
     sample() in the same order (the call sequence number is kept here)."""
 
-    def __init__(self, group=None):
+    def __init__(self, group=None, monitor=None):
         self.group = group
+        self.monitor = monitor    # an optional PeerMonitor, checked before every call
         self.rank = dist.get_rank(group)
         self.world = dist.get_world_size(group)
         self.mine = binding.fs_tp_area_create()
@@ -83,7 +142,11 @@ class FusedExchange:
 
     def sample(self, H, W_shard, vocab_offset, V_total, temperature=1.0, seed=0, row_seeds=None,
                step=0, mask_bits=None, out_idx=None, workspace=None, stream=None):
-        """Samples B <= 256 rows of the sharded head; every rank gets all tokens."""
+        """Samples B <= 256 rows of the sharded head; every rank gets all tokens.
+        With a monitor, raises PeerLost (having enqueued nothing) when a peer
+        did not reach this call."""
+        if self.monitor is not None:
+            self.monitor.check_in(self.seq)
         binding.fs_sample_tp(H, W_shard, vocab_offset, V_total, self.areas, self.seq, temperature,
                              seed, row_seeds, step, mask_bits, workspace=workspace, stream=stream)
         out = binding.fs_tp_wait(self.mine, H.shape[0], self.seq, out_idx, device=H.device,

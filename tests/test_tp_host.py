@@ -6,8 +6,10 @@ the documented packed key (order-preserving score bits << 32 | ~token, then
 XOR 2^63 so that signed order is key order), the ranks reduce with an int64
 MAX all-reduce, and the decoded token must equal the oracle's flat sample
 (abstract: argmax decomposes over a partition)."""
+import datetime
 import os
 import socket
+import time
 
 import numpy as np
 import pytest
@@ -135,3 +137,124 @@ def test_exchange_handles_in_rank_order():
     want = [bytes([r + 1]) * 64 for r in range(world)]
     for r in range(world):
         assert list(results[r]) == want
+
+
+# ------------------------------------------------ failure detection on the host
+def _monitor_rank(rank, world, port, plan, results):
+    """Runs six calls' check-ins; `plan[rank]` = (what, at_call) makes this
+    rank exit without a word, raise, or leave the group before that call."""
+    import torch.distributed as dist
+    from lm_head_exact_fmms_b200.tp import PeerLost, PeerMonitor
+    store = dist.TCPStore("127.0.0.1", port, None, False, timeout=datetime.timedelta(seconds=30))
+    mon = PeerMonitor(store, rank, world, timeout_s=3.0)
+    what, at = plan.get(rank, ("ok", -1))
+    log = []
+    for seq in range(6):
+        if seq == at:
+            results[rank] = log
+            if what == "exit":
+                os._exit(0)
+            if what == "raise":
+                raise RuntimeError("planted failure on rank %d" % rank)
+            if what == "leave":
+                mon.leave()
+                return
+        t0 = time.monotonic()
+        try:
+            mon.check_in(seq)
+        except PeerLost as e:
+            log.append(("lost", e.seq, e.missing, e.left, time.monotonic() - t0))
+            break
+        log.append(("ok", seq))
+    results[rank] = log
+
+
+def _run_monitor(world, plan):
+    import torch.distributed as dist
+    server = dist.TCPStore("127.0.0.1", 0, None, True, timeout=datetime.timedelta(seconds=30),
+                           wait_for_workers=False)
+    ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    results = mgr.dict()
+    procs = [ctx.Process(target=_monitor_rank, args=(r, world, server.port, plan, results))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+    codes = [p.exitcode for p in procs]
+    out = {r: list(results.get(r, [])) for r in range(world)}
+    return server, codes, out
+
+
+def test_peer_monitor_all_ranks_present():
+    """Three ranks through six calls: every check-in passes, and each rank
+    keeps only its latest call's key in the store."""
+    server, codes, out = _run_monitor(3, {})
+    assert codes == [0, 0, 0]
+    for r in range(3):
+        assert out[r] == [("ok", s) for s in range(6)]
+    assert server.num_keys() <= 3 + 1   # one live key per rank (+ the store's own counter)
+
+
+@pytest.mark.parametrize("what", ["exit", "raise"])
+def test_peer_monitor_reports_a_rank_that_died(what):
+    """A rank that exits without a word or raises before call 2: the others
+    get PeerLost for call 2, naming it, after the 3 s limit and before
+    launching anything."""
+    _, codes, out = _run_monitor(3, {2: (what, 2)})
+    assert codes[:2] == [0, 0] and codes[2] == (0 if what == "exit" else 1)
+    for r in (0, 1):
+        assert out[r][:2] == [("ok", 0), ("ok", 1)]
+        kind, seq, missing, left, waited = out[r][2]
+        assert (kind, seq, missing, left) == ("lost", 2, [2], [])
+        assert 2.9 <= waited < 30
+
+
+def test_peer_monitor_sees_a_leave_at_once():
+    """A rank that leaves on purpose before call 3 is reported within a poll
+    interval or so, not after the time limit."""
+    _, codes, out = _run_monitor(2, {1: ("leave", 3)})
+    assert codes == [0, 0]
+    assert out[1] == [("ok", 0), ("ok", 1), ("ok", 2)]
+    kind, seq, missing, left, waited = out[0][3]
+    assert (kind, seq, missing, left) == ("lost", 3, [1], [1])
+    assert waited < 2.0
+
+
+def _collective_rank(rank, world, port, results):
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=3))
+    keys = torch.full((4,), rank, dtype=torch.int64)
+    reduce_keys(keys)                                  # call 0: both ranks
+    if rank == 1:
+        time.sleep(8)                                  # alive, but skips call 1
+        results[rank] = "skipped"
+        return
+    t0 = time.monotonic()
+    try:
+        reduce_keys(keys)
+        results[rank] = "returned"
+    except RuntimeError:
+        results[rank] = ("error", time.monotonic() - t0)
+
+
+def test_key_all_reduce_ends_with_an_error_when_a_peer_skips_it():
+    """The all-reduce exchange: a rank that is alive but never joins call 1
+    makes the other rank's collective end with an error after the process
+    group's 3 s timeout, not hang."""
+    ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    results = mgr.dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_collective_rank, args=(r, 2, port, results)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+    assert results[1] == "skipped"
+    kind, waited = results[0]
+    assert kind == "error" and waited < 30
