@@ -408,7 +408,9 @@ def run_gpu(args, world, rank, local):
     nbytes, flops = algorithmic(B, wl.d, wl.V, mask is not None)
     # fused kernel per 256 rows, plus the group merge (grouped) or the decode (tp)
     fused_tp = tp and not (args.tp_nccl or B > 256)
-    launches_per_call = (B + 255) // 256 * (2 if grouped else 1) + (1 if tp and not fused_tp else 0)
+    # tensor-parallel: + the token decode after the all-reduce, or the bounded
+    # wait that copies the exchanged tokens
+    launches_per_call = (B + 255) // 256 * (2 if grouped else 1) + (1 if tp else 0)
     if tp:
         # each rank streams its shard; the roofline below is per rank
         nbytes = nbytes * W.shape[0] // wl.V

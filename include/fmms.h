@@ -226,14 +226,18 @@ fs_status fs_keys_to_tokens(const int64_t *keys, int B, int32_t *out_idx,
  *      (areas[own rank] = mine).  Every rank uses the same order.
  *   2. call number seq = 0, 1, 2, ... (the same on every rank):
  *      fs_sample_tp(..., areas, world, seq, ...) then
- *      fs_tp_wait(mine, B, seq, out_idx, stream) on the same stream; out_idx
- *      holds the tokens once the stream gets there.
+ *      fs_tp_wait(mine, B, seq, out_idx, timeout_us, stream) on the same
+ *      stream; out_idx holds the tokens once the stream gets there.
  *   3. at the end: fs_ipc_close on the peers' areas, fs_tp_area_destroy.
  * A rank must not issue call seq + 1 on a stream that has not passed its
  * fs_tp_wait of call seq (the alternate halves of the area rely on it).
  * If any rank's kernel records a device error, it still completes the
  * exchange; every rank then gets -1 for every row of that call and
- * fs_tp_failed reports the call.  Sequence numbers wrap after 2^32 calls. */
+ * fs_tp_failed reports the call.  If a peer never completes a call (its
+ * process died, say), this rank's fs_tp_wait gives up after its time limit,
+ * with the same -1 tokens and fs_tp_failed report; the areas are then in an
+ * unknown state and must be recreated on every rank before further calls.
+ * Sequence numbers wrap after 2^32 calls. */
 #define FS_IPC_HANDLE_BYTES 64
 
 /* Bytes of one exchange area (fixed; up to 256 rows per call). */
@@ -265,15 +269,17 @@ fs_status fs_sample_tp(const void *H, const void *W_shard, int B, int d,
                        uint32_t seq, void *workspace, size_t workspace_bytes,
                        fs_stream_t stream);
 
-/* Makes `stream` wait (a stream memory operation, no kernel) until call
- * `seq` has been decoded into this rank's area `area`, then copies its B
- * tokens to out_idx (device int32 [B]).  FS_ERR_UNSUPPORTED when the device
- * has no stream memory operations. */
+/* Enqueues on `stream` one small kernel that waits until call `seq` has
+ * been decoded into this rank's area `area` (the flag the completing rank
+ * stores with release semantics at system scope), for at most timeout_us
+ * microseconds (1 .. 60,000,000, else FS_ERR_INVALID_ARG), then copies the
+ * call's B <= 256 tokens to out_idx (device int32 [B]).  If the limit
+ * passes first, every token is -1 and fs_tp_failed reports seq. */
 fs_status fs_tp_wait(const void *area, int B, uint32_t seq, int32_t *out_idx,
-                     fs_stream_t stream);
+                     uint32_t timeout_us, fs_stream_t stream);
 
 /* Synchronous: seq + 1 of the last call decoded with a device error in
- * `area` (0: none). */
+ * `area`, or whose fs_tp_wait on `area` ran out of time (0: none). */
 fs_status fs_tp_failed(const void *area, uint32_t *failed);
 
 /* Top-k sampling (readus.org page, "Top-K and masking": a fast prefilter

@@ -86,7 +86,7 @@ def load_library():
     lib.fs_ipc_close.argtypes = [vp]
     lib.fs_sample_tp.argtypes = common + [i32, i32, f32, u64, vp, u32, vp, vp, i32, u32, vp, sz,
                                           vp]
-    lib.fs_tp_wait.argtypes = [vp, i32, u32, vp, vp]
+    lib.fs_tp_wait.argtypes = [vp, i32, u32, vp, u32, vp]
     lib.fs_tp_failed.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
     lib.fs_test_stall_loads.argtypes = [i32]
     lib.fs_set_partial_merge.argtypes = [i32]
@@ -418,13 +418,14 @@ def fs_sample_tp(H, W_shard, vocab_offset, V_total, areas, seq, temperature=1.0,
                             _ptr(workspace), ws_bytes, _stream(stream)), "fs_sample_tp")
 
 
-def fs_tp_wait(area, B, seq, out_idx=None, device=None, stream=None):
-    """Orders the stream after call `seq`'s tokens reached `area`; returns them."""
+def fs_tp_wait(area, B, seq, out_idx=None, device=None, stream=None, timeout_us=10_000_000):
+    """Tokens of call `seq` once they reach `area`, waiting on the stream for
+    at most timeout_us (then -1 tokens, and fs_tp_failed reports the call)."""
     lib = load_library()
     dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
     out_idx = _out(out_idx, B, dev)
     _check(lib.fs_tp_wait(ctypes.c_void_p(area), int(B), int(seq) & 0xFFFFFFFF, _ptr(out_idx),
-                          _stream(stream)), "fs_tp_wait")
+                          int(timeout_us), _stream(stream)), "fs_tp_wait")
     return out_idx
 
 

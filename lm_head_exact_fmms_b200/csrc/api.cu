@@ -110,22 +110,6 @@ StreamWriteValue32Fn write_value_fn() {
   return fn;
 }
 
-using StreamWaitValue32Fn = CUresult (*)(CUstream, CUdeviceptr, cuuint32_t, unsigned int);
-
-StreamWaitValue32Fn wait_value_fn() {
-  static StreamWaitValue32Fn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void *p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuStreamWaitValue32", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<StreamWaitValue32Fn>(p);
-  });
-  return fn;
-}
-
 EncodeTiledFn encode_fn() {
   static EncodeTiledFn fn = nullptr;
   static std::once_flag once;
@@ -629,6 +613,9 @@ fs_status fs_sample_shard_keys(const void *H, const void *W_shard, int B, int d,
 }
 
 // ------------------------------------------- fused vocabulary-parallel exchange
+// Longest wait fs_tp_wait accepts: one minute.
+constexpr uint32_t kMaxTpWaitUs = 60u * 1000u * 1000u;
+
 size_t fs_tp_area_bytes(void) { return fmms::kTpAreaBytes; }
 
 fs_status fs_tp_area_create(void **area) {
@@ -704,20 +691,18 @@ fs_status fs_sample_tp(const void *H, const void *W_shard, int B, int d, int V_s
 }
 
 fs_status fs_tp_wait(const void *area, int B, uint32_t seq, int32_t *out_idx,
-                     fs_stream_t stream) {
-  if (area == nullptr || out_idx == nullptr || B < 1 || B > fmms::kMaxBN)
+                     uint32_t timeout_us, fs_stream_t stream) {
+  if (area == nullptr || out_idx == nullptr || B < 1 || B > fmms::kMaxBN || timeout_us < 1 ||
+      timeout_us > kMaxTpWaitUs)
     return FS_ERR_INVALID_ARG;
-  const StreamWaitValue32Fn wait = wait_value_fn();
-  if (wait == nullptr) return FS_ERR_UNSUPPORTED;
-  const fmms::TpArea *a = static_cast<const fmms::TpArea *>(area);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (wait(reinterpret_cast<CUstream>(st), reinterpret_cast<CUdeviceptr>(&a->flag), seq + 1u,
-           CU_STREAM_WAIT_VALUE_GEQ) != CUDA_SUCCESS)
-    return FS_ERR_CUDA;
-  if (cudaMemcpyAsync(out_idx, a->tokens[seq & 1u], static_cast<size_t>(B) * 4,
-                      cudaMemcpyDeviceToDevice, st) != cudaSuccess)
-    return FS_ERR_CUDA;
-  return FS_OK;
+  DeviceState *st = nullptr;
+  fs_status s = get_device(&st);
+  if (s != FS_OK) return s;
+  return fmms::launch_tp_wait(static_cast<fmms::TpArea *>(const_cast<void *>(area)), B, seq,
+                              out_idx, timeout_us, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? FS_OK
+             : FS_ERR_CUDA;
 }
 
 fs_status fs_tp_failed(const void *area, uint32_t *failed) {

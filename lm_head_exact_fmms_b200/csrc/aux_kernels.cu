@@ -3,6 +3,7 @@
 //    page, "Group Gumbel Max": pick a group with Gumbel noise on the group
 //    log-masses, then take the sample inside the winning group);
 //  * the second kernel of the unfused mode, sampling from fp32 logits in HBM;
+//  * the bounded wait of the tensor-parallel exchange;
 //  * test kernels exposing the device Philox and Gumbel primitives.
 #include <cuda_runtime.h>
 #include <math.h>
@@ -897,6 +898,79 @@ cudaError_t launch_keys_to_tokens(const long long *keys, int B, int32_t *out_idx
                                   cudaStream_t stream) {
   return launch_dependent(keys_to_tokens_kernel, dim3((B + 255) / 256), dim3(256), stream, keys, B,
                           out_idx);
+}
+
+// ---------------------------------------------------------------------------
+// Tensor-parallel exchange: this rank's wait for a call's tokens.
+// ---------------------------------------------------------------------------
+// Acquire load at system scope (a word another GPU stores with release
+// semantics after the data it guards), a relaxed load of a guarded word, and
+// the GPU's global nanosecond timer.
+__device__ __forceinline__ uint32_t ld_acquire_sys(const uint32_t *addr) {
+  uint32_t v;
+  asm volatile("ld.acquire.sys.global.u32 %0, [%1];" : "=r"(v) : "l"(addr) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ int32_t ld_relaxed_sys(const int32_t *addr) {
+  int32_t v;
+  asm volatile("ld.relaxed.sys.global.b32 %0, [%1];" : "=r"(v) : "l"(addr) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ unsigned long long global_time_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// One block, launched after this rank's sampling kernel.  Thread 0 polls the
+// area's flag -- stored with release semantics at system scope, after the
+// tokens, by whichever rank's last CTA completed the area -- until it reaches
+// seq + 1 (compared modulo 2^32) or the time limit passes; every poll sleeps
+// a little, and the number of polls is capped as well.  Then the block copies
+// the tokens of the call's half of the area, or, if the limit passed, writes
+// -1 for every row and marks the call failed in the area.
+__global__ void __launch_bounds__(256) tp_wait_kernel(TpArea *area, int B, uint32_t seq,
+                                                      int32_t *out_idx,
+                                                      unsigned long long limit_ns,
+                                                      unsigned long long max_polls) {
+  __shared__ int late;
+  const uint32_t want = seq + 1u;
+  if (threadIdx.x == 0) {
+    const unsigned long long t0 = global_time_ns();
+    int timed_out = 0;
+    unsigned nap = 32;
+    for (unsigned long long n = 0;; ++n) {
+      if (static_cast<int32_t>(ld_acquire_sys(&area->flag) - want) >= 0) break;
+      if (n >= max_polls || global_time_ns() - t0 >= limit_ns) {
+        timed_out = 1;
+        break;
+      }
+      __nanosleep(nap);
+      if (nap < 1024) nap *= 2;
+    }
+    late = timed_out;
+  }
+  __syncthreads();
+  const int half = static_cast<int>(seq & 1u);
+  for (int b = threadIdx.x; b < B; b += blockDim.x) {
+    if (late) {
+      out_idx[b] = -1;
+    } else {
+      (void)ld_acquire_sys(&area->flag);  // orders this thread's token load after the flag
+      out_idx[b] = ld_relaxed_sys(&area->tokens[half][b]);
+    }
+  }
+  if (late && threadIdx.x == 0) atomicExch(&area->failed, want);
+}
+
+cudaError_t launch_tp_wait(TpArea *area, int B, uint32_t seq, int32_t *out_idx,
+                           uint32_t timeout_us, cudaStream_t stream) {
+  const unsigned long long limit_ns = 1000ull * timeout_us;
+  const unsigned long long max_polls = 64ull * timeout_us + 4096ull;
+  tp_wait_kernel<<<1, 256, 0, stream>>>(area, B, seq, out_idx, limit_ns, max_polls);
+  return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------------------

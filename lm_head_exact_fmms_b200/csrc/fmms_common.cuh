@@ -215,8 +215,8 @@ enum Mode { kModeFlat = 0, kModeGrouped = 1, kModeLogits = 2 };
 // every area's keys to its rows' packed maxima, then counts itself in every
 // area's arrivals; the arrival that completes an area decodes its keys into
 // its tokens, clears the keys and the count, and sets its flag to seq + 1.
-// No kernel waits for another: the stream that needs the tokens waits on the
-// flag (a stream memory operation).
+// No sampling kernel waits for another: the stream that needs the tokens runs
+// a small kernel that polls the flag, for a bounded time, and copies them.
 constexpr int kMaxTpWorld = 16;
 struct TpArea {
   unsigned int arrivals[2];  // ranks counted in, per parity

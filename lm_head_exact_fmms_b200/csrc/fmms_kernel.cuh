@@ -935,7 +935,7 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
     // decodes the keys and re-zeroes them for the next call.  With the fused
     // exchange an aborted CTA counts itself too (in the ticket's high half),
     // so that the exchange still completes, marked as failed, and no peer's
-    // stream waits forever.
+    // wait for the tokens runs into its time limit.
     __threadfence();
     sm100::epi_sync(kEpiThreads);
     if (etid == 0) {

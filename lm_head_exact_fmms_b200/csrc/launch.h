@@ -91,6 +91,11 @@ cudaError_t launch_merge_summaries(const void *summaries, int G, int B, uint64_t
                                    const uint64_t *row_seeds, uint32_t step, int32_t *out_idx,
                                    cudaStream_t stream);
 
+// Waits, at most timeout_us, for call `seq` of this rank's exchange area and
+// copies its tokens (or writes -1 and marks the call failed).
+cudaError_t launch_tp_wait(TpArea *area, int B, uint32_t seq, int32_t *out_idx,
+                           uint32_t timeout_us, cudaStream_t stream);
+
 // Decodes packed keys (XOR 2^63, as fs_sample_shard_keys writes them) to tokens.
 cudaError_t launch_keys_to_tokens(const long long *keys, int B, int32_t *out_idx,
                                   cudaStream_t stream);

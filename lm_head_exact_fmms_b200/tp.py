@@ -122,9 +122,10 @@ class FusedExchange:
     own area and its peers', mapped here by CUDA IPC.  Every rank calls
     sample() in the same order (the call sequence number is kept here)."""
 
-    def __init__(self, group=None, monitor=None):
+    def __init__(self, group=None, monitor=None, timeout_us=10_000_000):
         self.group = group
         self.monitor = monitor    # an optional PeerMonitor, checked before every call
+        self.timeout_us = timeout_us  # limit of each call's wait for its tokens
         self.rank = dist.get_rank(group)
         self.world = dist.get_world_size(group)
         self.mine = binding.fs_tp_area_create()
@@ -150,7 +151,7 @@ class FusedExchange:
         binding.fs_sample_tp(H, W_shard, vocab_offset, V_total, self.areas, self.seq, temperature,
                              seed, row_seeds, step, mask_bits, workspace=workspace, stream=stream)
         out = binding.fs_tp_wait(self.mine, H.shape[0], self.seq, out_idx, device=H.device,
-                                 stream=stream)
+                                 stream=stream, timeout_us=self.timeout_us)
         self.seq += 1
         return out
 

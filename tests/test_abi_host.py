@@ -141,9 +141,12 @@ def test_fused_exchange_validation(lib):
     assert tp(table=None) == 1
     assert tp(world=0) == 1 and tp(world=17) == 1
     assert tp(table=odd) == 1                 # areas are 256-byte aligned
-    assert lib.fs_tp_wait(None, 4, 0, FAKE, None) == 1
-    assert lib.fs_tp_wait(FAKE, 0, 0, FAKE, None) == 1
-    assert lib.fs_tp_wait(FAKE, 257, 0, FAKE, None) == 1
+    assert lib.fs_tp_wait(None, 4, 0, FAKE, 1000, None) == 1
+    assert lib.fs_tp_wait(FAKE, 0, 0, FAKE, 1000, None) == 1
+    assert lib.fs_tp_wait(FAKE, 257, 0, FAKE, 1000, None) == 1
+    assert lib.fs_tp_wait(FAKE, 4, 0, None, 1000, None) == 1
+    assert lib.fs_tp_wait(FAKE, 4, 0, FAKE, 0, None) == 1            # no time to wait
+    assert lib.fs_tp_wait(FAKE, 4, 0, FAKE, 60_000_001, None) == 1   # longer than a minute
     assert lib.fs_ipc_handle(None, None) == 1
     assert lib.fs_ipc_open(None, None) == 1
     assert lib.fs_tp_area_create(None) == 1

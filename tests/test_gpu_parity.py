@@ -613,6 +613,41 @@ def test_fused_exchange_marks_a_failed_call(dev):
         ex.close()
 
 
+
+def test_exchange_wait_runs_out_when_no_rank_completes_the_call(dev):
+    """A wait on a call that no rank ever ran (the flag nothing sets, as when
+    a peer's process died): the wait kernel gives up after its 0.2 s limit,
+    the tokens read -1, the area reports the call, and the context goes on
+    working -- a fresh exchange right after it is correct."""
+    import time
+
+    from lm_head_exact_fmms_b200.tp import LocalExchange, shard_bounds
+    area = binding.fs_tp_area_create()
+    try:
+        torch.cuda.synchronize()
+        t0 = time.monotonic()
+        out = binding.fs_tp_wait(area, 40, 6, device=dev, timeout_us=200_000)
+        torch.cuda.synchronize()
+        waited = time.monotonic() - t0
+        assert (out == -1).all()
+        assert binding.fs_tp_failed(area) == 7
+        assert 0.19 <= waited < 10.0
+    finally:
+        binding.fs_tp_area_destroy(area)
+    world, B, d, V = 2, 24, 64, 5000
+    H, W, Hd, Wd = rand_inputs(B, d, V, seed=93)
+    shards = [(Wd[lo:hi].contiguous(), lo) for lo, hi in shard_bounds(V, world)]
+    ex = LocalExchange(world)
+    try:
+        outs = ex.sample(Hd, shards, V, temperature=0.8, seed=4, step=1)
+        ref = binding.fs_sample_ex(Hd, Wd, temperature=0.8, seed=4, step=1)
+        for o in outs:
+            assert torch.equal(o, ref)
+        assert [binding.fs_tp_failed(a) for a in ex.areas] == [0] * world
+    finally:
+        ex.close()
+
+
 # ----------------------------------------------------- several samples per row
 @pytest.mark.parametrize("B,d,V,S", [(1, 64, 4096, 8), (17, 96, 3001, 3), (64, 128, 9000, 4),
                                      (300, 64, 2048, 2)])
