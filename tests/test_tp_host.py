@@ -258,3 +258,89 @@ def test_key_all_reduce_ends_with_an_error_when_a_peer_skips_it():
     assert results[1] == "skipped"
     kind, waited = results[0]
     assert kind == "error" and waited < 30
+
+
+class _FakeBinding:
+    """Records the exchange's library calls (no GPU): areas are integers."""
+
+    def __init__(self, rank, log):
+        self.rank, self.log = rank, log
+
+    def fs_tp_area_create(self):
+        return 1000 + self.rank
+
+    def fs_ipc_handle(self, area):
+        return bytes([area - 1000 + 1]) * 64
+
+    def fs_ipc_open(self, handle):
+        return 2000 + handle[0] - 1
+
+    def fs_ipc_close(self, area):
+        self.log.append(("ipc_close", area))
+
+    def fs_tp_area_destroy(self, area):
+        self.log.append(("destroy", area))
+
+    def fs_sample_tp(self, H, W, off, V, areas, seq, *args, **kw):
+        self.log.append(("sample", seq, tuple(areas)))
+
+    def fs_tp_wait(self, area, B, seq, out_idx=None, device=None, stream=None, timeout_us=None):
+        self.log.append(("wait", seq, area, timeout_us))
+        return out_idx
+
+
+def _fused_host_rank(rank, world, port, store_port, results):
+    import torch.distributed as dist
+    from lm_head_exact_fmms_b200 import tp
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=20))
+    log = []
+    tp.binding = _FakeBinding(rank, log)
+    torch.cuda.synchronize = lambda *a, **k: None     # no device here
+    store = dist.TCPStore("127.0.0.1", store_port, None, False,
+                          timeout=datetime.timedelta(seconds=30))
+    ex = tp.FusedExchange(monitor=tp.PeerMonitor(store, rank, world, timeout_s=2.0),
+                          timeout_us=123_456)
+    H = torch.zeros(4, 8)
+    outcome = "done"
+    for call in range(4):
+        if rank == 1 and call == 2:
+            results[rank] = (log, "exited")
+            os._exit(0)                                  # dies between calls, without a word
+        try:
+            ex.sample(H, None, 0, 100, out_idx=torch.zeros(4, dtype=torch.int32))
+        except tp.PeerLost as e:
+            outcome = ("lost", e.seq, e.missing)
+            break
+    results[rank] = (log, outcome, ex.areas)
+
+
+def test_fused_exchange_stops_before_launching_when_a_peer_died():
+    """FusedExchange on two gloo ranks with the library calls recorded: the
+    areas are the own one plus the peers' opened handles, in rank order; each
+    call checks in, samples with the call number and waits with the given
+    limit; when rank 1 dies before call 2, rank 0 gets PeerLost for call 2
+    and has enqueued nothing for it."""
+    import torch.distributed as dist
+    server = dist.TCPStore("127.0.0.1", 0, None, True, timeout=datetime.timedelta(seconds=30),
+                           wait_for_workers=False)
+    ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    results = mgr.dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_fused_host_rank, args=(r, 2, port, server.port, results))
+             for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+    assert [p.exitcode for p in procs] == [0, 0]
+    log0, outcome0, areas0 = results[0]
+    assert areas0 == [1000, 2001]                        # own area, then rank 1's opened handle
+    assert outcome0 == ("lost", 2, [1])
+    assert log0 == [("sample", 0, (1000, 2001)), ("wait", 0, 1000, 123_456),
+                    ("sample", 1, (1000, 2001)), ("wait", 1, 1000, 123_456)]
+    log1, outcome1 = results[1]
+    assert outcome1 == "exited" and [e[1] for e in log1 if e[0] == "sample"] == [0, 1]
