@@ -434,8 +434,8 @@ fs_status fs_set_partial_merge(int policy);
 /* ---- Host-only schedule query (no GPU needed) ---- */
 
 /* The vocabulary schedule of the fused kernel for V tokens, G groups
- * (0 or 1: flat) and `num_ctas` persistent CTAs (0: the value the library
- * would launch on `num_sms` SMs, returned in *num_ctas_out).  Writes up to
+ * (0 or 1: flat) on `num_sms` SMs (the number of persistent CTAs it
+ * launches is returned in *num_ctas_out if not NULL).  Writes up to
  * max_tiles rows of int32 [5] = (tile start, first valid token, end of valid
  * tokens, partial slot, last-tile-of-segment flag) for CTA `cta` and returns
  * the count in *ntiles.  Tiles are 128 tokens; a CTA's range is a multiple
@@ -445,6 +445,18 @@ fs_status fs_set_partial_merge(int policy);
  * and slots listed here stay the same.) */
 fs_status fs_plan_tiles(int V, int G, int num_sms, int cta, int32_t *tiles,
                         int max_tiles, int *ntiles, int *num_ctas_out);
+
+/* The same schedule as the kernel variant with merged partial tiles runs it
+ * (single-CTA launches of at most 64 rows; fs_set_partial_merge): rows of
+ * int32 [8] = the five columns above, then (partial start, first valid
+ * token, end of valid tokens) of the 8-row partial tile multiplied in the
+ * same stages as this tile, or (-1, 0, 0) for none.  Expanding every merged
+ * partial into a tile of its own, just before its tile and with the same
+ * slot, gives fs_plan_tiles' list.  *merges (if not NULL) = 1 when the
+ * automatic choice runs this variant for the split (at least one CTA in ten
+ * starts a segment with an 8-row partial tile), else 0. */
+fs_status fs_plan_tiles_merged(int V, int G, int num_sms, int cta, int32_t *tiles,
+                               int max_tiles, int *ntiles, int *merges);
 
 /* The CTAs whose vocabulary range meets group g (0 <= g < G), as the grouped
  * merge kernel enumerates them: [*first, *last].  Host-only. */

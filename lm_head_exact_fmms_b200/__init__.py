@@ -13,7 +13,7 @@ _BINDING_NAMES = ("FmmsError", "fs_sample", "fs_sample_ex", "fs_sample_grouped",
                   "fs_test_stalled_sample", "fs_sample_shard_keys", "fs_keys_to_tokens",
                   "fs_sample_multi", "fs_workspace_bytes_multi", "fs_summarize_group",
                   "fs_merge_groups", "fs_workspace_bytes_summary", "fs_sample_topk",
-                  "fs_set_cta_pairs", "fs_set_partial_merge")
+                  "fs_set_cta_pairs", "fs_set_partial_merge", "fs_plan_tiles_merged")
 
 
 def __getattr__(name):

@@ -26,7 +26,8 @@ EXPORTED = ("fs_sample", "fs_sample_ex", "fs_sample_grouped", "fs_sample_unfused
             "fs_summarize_group", "fs_merge_groups", "fs_workspace_bytes_summary",
             "fs_sample_topk", "fs_set_cta_pairs", "fs_tp_area_bytes", "fs_tp_area_create",
             "fs_tp_area_destroy", "fs_ipc_handle", "fs_ipc_open", "fs_ipc_close", "fs_sample_tp",
-            "fs_tp_wait", "fs_tp_failed", "fs_test_stall_loads", "fs_set_partial_merge")
+            "fs_tp_wait", "fs_tp_failed", "fs_test_stall_loads", "fs_set_partial_merge",
+            "fs_plan_tiles_merged")
 
 FS_IPC_HANDLE_BYTES = 64
 
@@ -101,6 +102,8 @@ def load_library():
                                   ctypes.POINTER(ctypes.c_int)]
     lib.fs_plan_group_ctas.argtypes = [i32, i32, i32, i32, ctypes.POINTER(ctypes.c_int),
                                        ctypes.POINTER(ctypes.c_int)]
+    lib.fs_plan_tiles_merged.argtypes = [i32, i32, i32, i32, vp, i32,
+                                         ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
     for name in EXPORTED:
         if name not in ("fs_workspace_bytes", "fs_workspace_bytes_multi",
                         "fs_workspace_bytes_summary", "fs_status_string", "fs_tp_area_bytes"):
@@ -287,6 +290,21 @@ def fs_plan_tiles(V, G, num_sms, cta, max_tiles=4096):
                              buf.ctypes.data_as(ctypes.c_void_p), max_tiles, ctypes.byref(n),
                              ctypes.byref(nc)), "fs_plan_tiles")
     return buf[: min(n.value, max_tiles)].copy(), nc.value
+
+
+def fs_plan_tiles_merged(V, G, num_sms, cta, max_tiles=4096):
+    """Host-only query of the merged-partial schedule: (tiles int32 [n, 8],
+    whether the automatic choice merges for this split)."""
+    import numpy as np
+    lib = load_library()
+    buf = np.zeros((max_tiles, 8), dtype=np.int32)
+    n = ctypes.c_int(0)
+    merges = ctypes.c_int(0)
+    _check(lib.fs_plan_tiles_merged(int(V), int(G), int(num_sms), int(cta),
+                                    buf.ctypes.data_as(ctypes.c_void_p), max_tiles,
+                                    ctypes.byref(n), ctypes.byref(merges)),
+           "fs_plan_tiles_merged")
+    return buf[: min(n.value, max_tiles)].copy(), bool(merges.value)
 
 
 def plan_num_ctas(V, G, num_sms):

@@ -278,18 +278,9 @@ struct ShardOpts {
 // Whether the kernel variant with merged 8-row partial tiles pays for this
 // vocabulary split: at least one CTA in ten starts a segment with an 8-row
 // partial tile (the Qwen3 heads: 48 of 148).  Elsewhere its extra slot per
-// stage only costs ring space.  Remembers the last few answers.
-bool merge_partials(const Schedule &sch) {
-  if (g_merge_policy >= 0) return g_merge_policy == 1;
-  struct Entry {
-    int V, G, num_ctas;
-    bool merge;
-  };
-  static Entry memo[8];
-  static int memo_next = 0, memo_used = 0;
-  for (int i = 0; i < memo_used; ++i)
-    if (memo[i].V == sch.V && memo[i].G == sch.G && memo[i].num_ctas == sch.num_ctas)
-      return memo[i].merge;
+// stage only costs ring space.  merge_partials applies the policy switch and
+// remembers the last few answers.
+bool merge_rule(const Schedule &sch) {
   int with = 0;
   for (int c = 0; c < sch.num_ctas; ++c) {
     fmms::TileIter it(sch, c, 1);
@@ -301,7 +292,21 @@ bool merge_partials(const Schedule &sch) {
       }
     }
   }
-  const bool merge = with * 10 >= sch.num_ctas;
+  return with * 10 >= sch.num_ctas;
+}
+
+bool merge_partials(const Schedule &sch) {
+  if (g_merge_policy >= 0) return g_merge_policy == 1;
+  struct Entry {
+    int V, G, num_ctas;
+    bool merge;
+  };
+  static Entry memo[8];
+  static int memo_next = 0, memo_used = 0;
+  for (int i = 0; i < memo_used; ++i)
+    if (memo[i].V == sch.V && memo[i].G == sch.G && memo[i].num_ctas == sch.num_ctas)
+      return memo[i].merge;
+  const bool merge = merge_rule(sch);
   memo[memo_next] = Entry{sch.V, sch.G, sch.num_ctas, merge};
   memo_next = (memo_next + 1) % 8;
   if (memo_used < 8) ++memo_used;
@@ -901,6 +906,26 @@ fs_status fs_plan_tiles(int V, int G, int num_sms, int cta, int32_t *tiles, int 
       tiles[5 * n + 2] = t.hi;
       tiles[5 * n + 3] = t.slot;
       tiles[5 * n + 4] = t.last;
+    }
+    ++n;
+  }
+  *ntiles = n;
+  return FS_OK;
+}
+
+fs_status fs_plan_tiles_merged(int V, int G, int num_sms, int cta, int32_t *tiles,
+                               int max_tiles, int *ntiles, int *merges) {
+  if (V < 1 || G < 0 || G > V || num_sms < 1 || !ntiles) return FS_ERR_INVALID_ARG;
+  const Schedule sch = fmms::make_schedule(V, G, num_sms);
+  if (merges) *merges = merge_rule(sch) ? 1 : 0;
+  if (cta < 0 || cta >= sch.num_ctas) return FS_ERR_INVALID_ARG;
+  fmms::TileIter it(sch, cta, 1);
+  fmms::Tile t;
+  int n = 0;
+  while (it.next(t)) {
+    if (tiles && n < max_tiles) {
+      const int32_t row[8] = {t.start, t.lo, t.hi, t.slot, t.last, t.pstart, t.plo, t.phi};
+      memcpy(tiles + 8 * n, row, sizeof row);
     }
     ++n;
   }

@@ -119,6 +119,48 @@ def test_schedule_covers_vocab_once(lib, V, G, sms):
             assert met == list(range(first, last + 1))
 
 
+@pytest.mark.parametrize("V,G,sms", [
+    (151936, 0, 148), (151936, 8, 148), (151937, 8, 148), (128256, 0, 148), (4097, 5, 148),
+    (5003, 7, 13), (100000, 97, 148), (12, 3, 148), (1000, 1000, 148),
+])
+def test_merged_schedule_is_the_schedule_with_pairs_fused(lib, V, G, sms):
+    """The schedule of the merged-partial kernel variant: expanding each merged
+    8-row partial into a tile of its own, just before its tile and with its
+    slot, gives exactly the plain schedule; a merged partial is an 8-row tile
+    directly followed by a whole tile of the same segment."""
+    nc, per_cta = _all_tiles(V, G, sms)
+    merged_ctas = 0
+    for c in range(nc):
+        merged, _ = binding.fs_plan_tiles_merged(V, G, sms, c)
+        expanded = []
+        any_merged = False
+        for start, lo, hi, slot, last, pstart, plo, phi in merged:
+            if pstart >= 0:
+                any_merged = True
+                assert pstart + 8 == start and pstart <= plo < phi <= pstart + 8
+                assert hi - lo == 128 or last == 1
+                expanded.append((pstart, plo, phi, slot, 0))
+            else:
+                assert (plo, phi) == (0, 0)
+            expanded.append((start, lo, hi, slot, last))
+        assert [tuple(t) for t in per_cta[c]] == expanded
+        merged_ctas += any_merged
+    _, merges = binding.fs_plan_tiles_merged(V, G, sms, 0)
+    assert merges == (merged_ctas * 10 >= nc)
+
+
+def test_merge_choice_on_the_benchmarked_heads(lib):
+    """The automatic choice: 48 of the 148 CTAs of a 151936-token head start
+    with an 8-row partial tile, so it merges; the 128256-token head has none
+    worth it."""
+    _, nc = binding.fs_plan_tiles(151936, 0, 148, 0)
+    with_partial = sum(bool((binding.fs_plan_tiles_merged(151936, 0, 148, c)[0][:, 5] >= 0).any())
+                       for c in range(nc))
+    assert (nc, with_partial) == (148, 48)
+    assert binding.fs_plan_tiles_merged(151936, 0, 148, 0)[1] is True
+    assert binding.fs_plan_tiles_merged(128256, 0, 148, 0)[1] is False
+
+
 def test_flagship_schedule_balance(lib):
     """Qwen3 heads: 148 CTAs stream 1026-1027 rows each (8.02 tiles), not 8 or 9 tiles."""
     nc, per_cta = _all_tiles(151936, 0, 148)
