@@ -10,11 +10,11 @@ touched.  This shows the pins are tight enough that an error of these kinds
 anywhere in the oracle's arithmetic would not go unnoticed.
 
 Not covered, on purpose: the smallest-index rule of the oracle's argmax scan
-(perturbed scores of distinct tokens tie with probability about 2^-32 per
-pair, so no pin on random inputs can see it; the GPU tests plant exact ties
-in the top-k selection instead) and the choice of counter tag for the group
-noise (a reading of the pages, not arithmetic; the grouped GPU parity tests
-compare the tag bit for bit).
+over perturbed scores (distinct tokens' scores tie with probability about
+2^-32 per pair, so no pin on random inputs can see it; ties of logits, which
+do occur, are pinned through top-k with every logit tied) and the choice of
+counter tag for the group noise (a reading of the pages, not arithmetic; the
+grouped GPU parity tests compare the tag bit for bit).
 """
 import importlib.util
 import os
@@ -90,6 +90,10 @@ MUTANTS = [
      "2u * (uint32_t)k, mask, s);",
      "0u * (uint32_t)k, mask, s);",
      "test_multi_samples_are_softmax_draws", {}),
+    ("topk_ties_toward_the_larger_index",
+     "return (x->v < y->v) ? -1 : (x->v > y->v);",
+     "return (x->v > y->v) ? -1 : (x->v < y->v);",
+     "test_topk_all_logits_tied_keeps_the_smallest_indices", {}),
     ("topk_keeps_smallest_logits",
      "if (x->l > y->l) return -1;\n  if (x->l < y->l) return 1;",
      "if (x->l < y->l) return -1;\n  if (x->l > y->l) return 1;",

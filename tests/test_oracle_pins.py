@@ -580,6 +580,24 @@ def test_topk_respects_mask_and_set(oracle):
             assert idx[b] in top
 
 
+def test_topk_all_logits_tied_keeps_the_smallest_indices(oracle):
+    """Every W row equal, so every logit of a row ties: the k candidates are
+    the k smallest allowed indices, and the token is the largest Gumbel value
+    among them (noise from the separately pinned noise-word function)."""
+    V, d, B, K = 300, 16, 3, 37
+    H = synth.make_hidden(B, d, seed=161)
+    W = synth.make_weight(1, d, 0.5, seed=162).expand(V, d).contiguous()
+    allowed = torch.from_numpy(np.random.default_rng(163).random((B, V)) < 0.7)
+    mask = synth.mask_from_bool(allowed)
+    for step in (0, 9):
+        idx, _, _ = oracle.sample_topk(H, W, K, T=1.1, seed=77, step=step, mask=mask)
+        for b in range(B):
+            cand = np.flatnonzero(allowed[b].numpy())[:K]
+            words = np.array([oracle.noise_word(77, step, b, int(v)) for v in cand],
+                             dtype=np.uint32)
+            assert idx[b] == int(cand[np.argmax(oracle.gumbel(words))]), (step, b)
+
+
 def test_topk_matches_truncated_softmax(oracle):
     V, d, K, N, T = 64, 32, 9, 200_000, 1.1
     H = synth.make_hidden(1, d, seed=161)
