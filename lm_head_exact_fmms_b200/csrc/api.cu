@@ -54,18 +54,20 @@ struct DeviceState {
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
+// The device attributes are read once per device, also when the first calls
+// come from several threads at once (not every entry point holds g_mu).
+std::once_flag g_dev_once[kMaxDevices];
 
 fs_status get_device(DeviceState **out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FS_ERR_CUDA;
   DeviceState &st = g_dev[dev];
-  if (!st.init) {
-    if (cudaDeviceGetAttribute(&st.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      return FS_ERR_CUDA;
-    if (cudaDeviceGetAttribute(&st.cc_major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
-      return FS_ERR_CUDA;
-    st.init = true;
-  }
+  std::call_once(g_dev_once[dev], [&st, dev] {
+    st.init = cudaDeviceGetAttribute(&st.sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+              cudaDeviceGetAttribute(&st.cc_major, cudaDevAttrComputeCapabilityMajor, dev) ==
+                  cudaSuccess;
+  });
+  if (!st.init) return FS_ERR_CUDA;
   if (st.cc_major != 10) return FS_ERR_UNSUPPORTED;  // built for sm_100a only
   *out = &st;
   return FS_OK;
