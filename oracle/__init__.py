@@ -52,6 +52,9 @@ def _load():
                    _i32p, ctypes.c_int]
     lib.oracle_scores.argtypes = common + sample_args + [_f64p]
     lib.oracle_sample.argtypes = common + sample_args + [_i32p, _f64p, _f64p]
+    lib.oracle_sample_steps.argtypes = common + [ctypes.c_double, ctypes.c_uint64, _u64p,
+                                                 ctypes.c_uint32, ctypes.c_int, _u32p, _i32p,
+                                                 _f64p, _f64p]
     lib.oracle_sample_grouped.argtypes = common + [ctypes.c_int] + sample_args + [_i32p, _f64p, _f64p]
     lib.oracle_sample_multi.argtypes = common + [ctypes.c_int] + sample_args + [_i32p, _f64p, _f64p]
     lib.oracle_sample_topk.argtypes = common + [ctypes.c_int] + sample_args + [_i32p, _f64p, _f64p]
@@ -175,6 +178,21 @@ def sample(H, W, T=1.0, seed=0, row_seeds=None, step=0, mask=None, rows=None):
     lib.oracle_sample(_ptr(H16, _u16p), _ptr(W16, _u16p), B, d, V, float(T), int(seed),
                       _ptr(rs, _u64p), int(step), _ptr(mk, _u32p), _ptr(rows, _i32p), rows.size,
                       _ptr(idx, _i32p), _ptr(best, _f64p), _ptr(second, _f64p))
+    return idx, best, second
+
+
+def sample_steps(H, W, nsteps, T=1.0, seed=0, row_seeds=None, step0=0, mask=None):
+    """Flat FMMS sample of every row at steps step0 .. step0+nsteps-1 (the
+    logits computed once).  Returns (idx int32 [nsteps, B], best, second f64
+    [nsteps, B]), equal to `sample` called at each step."""
+    lib = _load()
+    H16, W16, B, d, V, rs, mk, _ = _sample_common(H, W, T, seed, row_seeds, step0, mask, None)
+    idx = np.empty((nsteps, B), dtype=np.int32)
+    best = np.empty((nsteps, B), dtype=np.float64)
+    second = np.empty((nsteps, B), dtype=np.float64)
+    lib.oracle_sample_steps(_ptr(H16, _u16p), _ptr(W16, _u16p), B, d, V, float(T), int(seed),
+                            _ptr(rs, _u64p), int(step0), int(nsteps), _ptr(mk, _u32p),
+                            _ptr(idx, _i32p), _ptr(best, _f64p), _ptr(second, _f64p))
     return idx, best, second
 
 

@@ -286,6 +286,38 @@ void oracle_sample(const uint16_t *H, const uint16_t *W, int B, int d, int V,
   free(l);
 }
 
+/* Flat sampling of every row at each of the steps step0 .. step0+nsteps-1:
+ * the same result as oracle_sample called once per step, with the logits
+ * (which do not depend on the step) computed once.  out_idx[n*B + b],
+ * out_best / out_second likewise.  Parallel over (step, row) pairs; each
+ * pair's scores and argmax run on one thread. */
+void oracle_sample_steps(const uint16_t *H, const uint16_t *W, int B, int d,
+                         int V, double T, uint64_t seed,
+                         const uint64_t *row_seeds, uint32_t step0,
+                         int nsteps, const uint32_t *mask, int32_t *out_idx,
+                         double *out_best, double *out_second) {
+  double *l = (double *)malloc(sizeof(double) * (size_t)B * (size_t)V);
+  for (int b = 0; b < B; ++b)
+    logits_row(H + (int64_t)b * d, W, d, V, l + (int64_t)b * V);
+#pragma omp parallel
+  {
+    double *s = (double *)malloc(sizeof(double) * (size_t)V);
+#pragma omp for schedule(static)
+    for (int64_t i = 0; i < (int64_t)nsteps * B; ++i) {
+      const int n = (int)(i / B), b = (int)(i % B);
+      /* the nested parallel loop of the scores runs on this thread */
+      scores_from_logits(l + (int64_t)b * V, V, T, row_key(seed, row_seeds, b),
+                         step0 + (uint32_t)n, b, mask, s);
+      double b1, b2;
+      out_idx[i] = argmax_scan(s, 0, V, &b1, &b2);
+      if (out_best) out_best[i] = b1;
+      if (out_second) out_second[i] = b2;
+    }
+    free(s);
+  }
+  free(l);
+}
+
 /* Several samples per row: sample k draws with token-noise tag 2k, so the
  * samples are independent draws from the same softmax and sample 0 is the
  * single-sample result.  out_idx[i*S + k], out_best / out_second likewise

@@ -379,6 +379,7 @@ def test_mismatch_rate_bound(dev, oracle):
     assert mism / total < 1e-4, (mism, total)
 
 
+
 # --------------------------------------------------------- grouped sampling
 @pytest.mark.parametrize("G,masked", [(1, False), (2, False), (3, True), (8, True), (64, False),
                                       (1000, True)])

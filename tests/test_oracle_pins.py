@@ -505,6 +505,24 @@ def test_grouped_masked_groups(oracle):
 # Reproducibility (readus.org page, seed management)
 # --------------------------------------------------------------------------
 
+def test_sample_steps_equals_one_call_per_step(oracle):
+    """The many-steps helper (logits computed once) returns, bit for bit, what
+    one sampling call per step returns, masks and row seeds included."""
+    V, d, B, n0, N = 333, 48, 7, 1000, 6
+    H = synth.make_hidden(B, d, seed=171)
+    W = synth.make_weight(V, d, 0.3, seed=172)
+    rs = synth.make_row_seeds(B)
+    allowed = torch.from_numpy(np.random.default_rng(173).random((B, V)) < 0.4)
+    allowed[3] = False
+    mask = synth.mask_from_bool(allowed)
+    idx, best, second = oracle.sample_steps(H, W, N, T=0.6, row_seeds=rs, step0=n0, mask=mask)
+    for n in range(N):
+        i1, b1, s1 = oracle.sample(H, W, T=0.6, row_seeds=rs, step=n0 + n, mask=mask)
+        assert np.array_equal(idx[n], i1) and np.array_equal(best[n], b1)
+        assert np.array_equal(second[n], s1)
+    assert np.all(idx[:, 3] == -1)
+
+
 def test_same_seed_same_tokens_and_steps_differ(oracle):
     V, d, B = 500, 64, 32
     H = synth.make_hidden(B, d, seed=111)
