@@ -13,6 +13,7 @@ Under torchrun each rank runs an independent replica (the path has no
 data-path exchange at one GPU per replica); timings are the max over ranks.
 """
 import argparse
+import contextlib
 import hashlib
 import json
 import os
@@ -171,6 +172,28 @@ class ClockSampler:
         med = s[len(s) // 2] if s else None
         return {"sm_mhz": med, "sm_max_mhz": self.max_mhz,
                 "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(s)}
+
+
+@contextlib.contextmanager
+def nvtx(name):
+    """An NVTX range around a benchmark section, so that a profiler's
+    timeline shows which section a kernel belongs to; nothing happens if
+    NVTX is unavailable.  Pushed and popped once per section, outside the
+    per-step loop."""
+    try:
+        import torch
+        torch.cuda.nvtx.range_push(name)
+        pushed = True
+    except Exception:
+        pushed = False
+    try:
+        yield
+    finally:
+        if pushed:
+            try:
+                torch.cuda.nvtx.range_pop()
+            except Exception:
+                pass
 
 
 def dist_setup():
@@ -400,7 +423,8 @@ def run_gpu(args, world, rank, local):
                                  mask_bits=mask, out_idx=out, workspace=ws, stream=stream)
 
     sampler = ClockSampler(local)
-    region_ms, per_call = time_calls(step, args.steps, args.warmup, stream, world, sampler)
+    with nvtx("fmms: timed steps"):
+        region_ms, per_call = time_calls(step, args.steps, args.warmup, stream, world, sampler)
     region_ms = max_over_ranks(region_ms, world)
     kernel_us = sum(per_call) / len(per_call)
     kernel_us = max_over_ranks(kernel_us, world)
@@ -429,7 +453,8 @@ def run_gpu(args, world, rank, local):
             H.copy_(Hh, non_blocking=True)
             step(i)
             Oh.copy_(out, non_blocking=True)
-    e2e_ms, _ = time_calls(step_host, args.steps, args.warmup, stream, world)
+    with nvtx("fmms: end-to-end steps (host buffers)"):
+        e2e_ms, _ = time_calls(step_host, args.steps, args.warmup, stream, world)
     e2e_ms = max_over_ranks(e2e_ms, world)
 
     result = {
@@ -455,14 +480,21 @@ def run_gpu(args, world, rank, local):
     # The single-GPU characterisation (batch sweep, other modes) runs at N=1
     # only: at N > 1 it would hold the other GPUs idle while rank 0 works.
     if rank == 0 and world == 1 and not args.no_sweep:
-        result["sweep"] = sweep(torch, binding, synth, W, wl, dev, stream, peaks, peak_kind)
-        result["grouped_masked"] = grouped_points(torch, binding, synth, dev, stream, peaks,
-                                                  peak_kind, W)
-        result["unfused"] = unfused_point(torch, binding, synth, W, wl, dev, stream, B)
-        result["multi_sample"] = multi_point(torch, binding, synth, W, wl, dev, stream, B)
-        result["cuda_graph"] = graph_point(torch, binding, synth, W, wl, dev, B)
-        result["top_k"] = topk_point(torch, binding, synth, W, wl, dev, stream, B)
-        result["tiny"] = tiny_point(torch, binding, synth, dev, stream)
+        with nvtx("fmms: batch sweep"):
+            result["sweep"] = sweep(torch, binding, synth, W, wl, dev, stream, peaks, peak_kind)
+        with nvtx("fmms: grouped + masked"):
+            result["grouped_masked"] = grouped_points(torch, binding, synth, dev, stream, peaks,
+                                                      peak_kind, W)
+        with nvtx("fmms: unfused"):
+            result["unfused"] = unfused_point(torch, binding, synth, W, wl, dev, stream, B)
+        with nvtx("fmms: several samples per row"):
+            result["multi_sample"] = multi_point(torch, binding, synth, W, wl, dev, stream, B)
+        with nvtx("fmms: CUDA graph"):
+            result["cuda_graph"] = graph_point(torch, binding, synth, W, wl, dev, B)
+        with nvtx("fmms: top-k"):
+            result["top_k"] = topk_point(torch, binding, synth, W, wl, dev, stream, B)
+        with nvtx("fmms: tiny head"):
+            result["tiny"] = tiny_point(torch, binding, synth, dev, stream)
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not grouped:
         result["cpu_baseline"] = cpu_baseline(H, W, wl, B, rs)
         if not args.no_sweep:

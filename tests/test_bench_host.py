@@ -86,3 +86,14 @@ def test_reference_arm_prints_the_contract_line():
     assert r["e2e"] == {"value": r["value"], "unit": bench.UNIT, "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
     assert r["config"]["V"] == 4096 and r["config"]["d"] == 256
+
+
+def test_nvtx_sections_are_transparent():
+    """The NVTX section wrapper runs its body and lets its exceptions through."""
+    ran = []
+    with bench.nvtx("section"):
+        ran.append(1)
+    with pytest.raises(KeyError):
+        with bench.nvtx("failing section"):
+            raise KeyError("k")
+    assert ran == [1]
