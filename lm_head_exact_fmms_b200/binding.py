@@ -235,12 +235,17 @@ def fs_sample_host(H_host, W, temperature=1.0, seed=0, row_seeds=None, step=0, m
         raise ValueError("H_host must be a contiguous CPU bfloat16 tensor")
     if W.dtype != torch.bfloat16 or not W.is_cuda or not W.is_contiguous():
         raise ValueError("W must be a contiguous CUDA bfloat16 tensor")
+    if H_host.dim() != 2 or W.dim() != 2 or H_host.shape[1] != W.shape[1]:
+        raise ValueError("H_host must be [B, d] and W [V, d]")
     B, d = H_host.shape
     V = W.shape[0]
     row_seeds = _opt_dev(row_seeds, torch.int64, B, "row_seeds", W.device)
     mask_bits = _opt_dev(mask_bits, torch.int32, B * ((V + 31) // 32), "mask_bits", W.device)
     if out_idx_host is None:
         out_idx_host = torch.empty(B, dtype=torch.int32, pin_memory=True)
+    elif (out_idx_host.dtype != torch.int32 or out_idx_host.is_cuda
+          or not out_idx_host.is_contiguous() or out_idx_host.numel() < B):
+        raise ValueError("out_idx_host must be a contiguous CPU int32 tensor of at least B elements")
     _check(lib.fs_sample_host(_ptr(H_host), _ptr(W), B, d, V, float(temperature), _seed(seed),
                               _ptr(row_seeds), int(step), _ptr(mask_bits), _ptr(out_idx_host),
                               _stream(stream)), "fs_sample_host")

@@ -8,6 +8,7 @@ import re
 
 import numpy as np
 import pytest
+import torch
 
 from lm_head_exact_fmms_b200 import binding
 
@@ -196,3 +197,32 @@ def test_fused_exchange_validation(lib):
     # the area holds two halves of 256 keys and 256 tokens plus its header
     assert binding.fs_tp_area_bytes() >= 2 * 256 * (8 + 4) + 32
     assert binding.fs_tp_area_bytes() % 256 == 0
+
+
+class _DeviceTensorStandIn:
+    """Just enough of a CUDA bf16 tensor for the binding's argument checks."""
+    dtype = torch.bfloat16
+    is_cuda = True
+    device = torch.device("cuda", 0)
+
+    def __init__(self, *shape):
+        self.shape = shape
+
+    def dim(self):
+        return len(self.shape)
+
+    def is_contiguous(self):
+        return True
+
+
+def test_host_entry_binding_rejects_mismatched_operands(lib):
+    """fs_sample_host's binding refuses, before any library call, a W whose
+    inner dimension differs from H's (the C ABI cannot see W's real shape,
+    and the kernel would read past its end) and an unusable token buffer."""
+    H = torch.zeros(4, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match=r"\[B, d\]"):
+        binding.fs_sample_host(H, _DeviceTensorStandIn(100, 32))
+    for bad in (torch.zeros(4, dtype=torch.int64), torch.zeros(3, dtype=torch.int32),
+                torch.zeros(8, dtype=torch.int32)[::2]):
+        with pytest.raises(ValueError, match="out_idx_host"):
+            binding.fs_sample_host(H, _DeviceTensorStandIn(100, 64), out_idx_host=bad)
