@@ -157,7 +157,10 @@ class FusedExchange:
 
     def close(self):
         """Unmaps the peers' areas and frees this rank's, once every rank is
-        done with the exchange."""
+        done with the exchange.  With a monitor, first tells the peers that
+        this rank takes no further calls."""
+        if self.monitor is not None:
+            self.monitor.leave()
         torch.cuda.synchronize()
         dist.barrier(group=self.group)
         for a in self._opened:
