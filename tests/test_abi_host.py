@@ -226,3 +226,47 @@ def test_host_entry_binding_rejects_mismatched_operands(lib):
                 torch.zeros(8, dtype=torch.int32)[::2]):
         with pytest.raises(ValueError, match="out_idx_host"):
             binding.fs_sample_host(H, _DeviceTensorStandIn(100, 64), out_idx_host=bad)
+
+
+C_CALLER = r"""
+#include <stdio.h>
+#include "fmms.h"
+int main(void) {
+  int32_t tiles[8 * 64];
+  int n = 0, nc = 0, merges = -1;
+  if (fs_plan_tiles(151936, 0, 148, 5, tiles, 64, &n, &nc) != FS_OK) return 1;
+  printf("plain %d %d %d %d\n", n, nc, tiles[0], tiles[2]);
+  if (fs_plan_tiles_merged(151936, 0, 148, 5, tiles, 64, &n, &merges) != FS_OK) return 2;
+  printf("merged %d %d %d\n", n, merges, tiles[5]);
+  printf("area %zu\n", fs_tp_area_bytes());
+  printf("status %d %s\n",
+         (int)fs_sample(NULL, NULL, 1, 64, 100, 1.0f, 0, 0, NULL, NULL, NULL),
+         fs_status_string(FS_ERR_INVALID_ARG));
+  return 0;
+}
+"""
+
+
+def test_c_program_links_and_calls_the_abi(lib):
+    """A plain C99 program that includes only include/fmms.h links against
+    libfmms.so and gets, from host-only calls, what the Python binding gets."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    work = os.path.join(ROOT, "_build", "c_abi")
+    os.makedirs(work, exist_ok=True)
+    src, exe = os.path.join(work, "caller.c"), os.path.join(work, "caller")
+    with open(src, "w") as f:
+        f.write(C_CALLER)
+    libdir = os.path.dirname(binding.library_path())
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), src,
+                    "-L", libdir, "-lfmms", "-Wl,-rpath," + libdir, "-o", exe], check=True)
+    out = subprocess.run([exe], capture_output=True, text=True, timeout=120, check=True).stdout
+    lines = dict(line.split(" ", 1) for line in out.strip().splitlines())
+    tiles, nc = binding.fs_plan_tiles(151936, 0, 148, 5)
+    assert lines["plain"].split() == [str(len(tiles)), str(nc), str(tiles[0][0]), str(tiles[0][2])]
+    merged, merges = binding.fs_plan_tiles_merged(151936, 0, 148, 5)
+    assert lines["merged"].split() == [str(len(merged)), str(int(merges)), str(merged[0][5])]
+    assert int(lines["area"]) == binding.fs_tp_area_bytes()
+    assert lines["status"] == "1 FS_ERR_INVALID_ARG"
