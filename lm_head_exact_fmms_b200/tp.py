@@ -117,12 +117,24 @@ class PeerMonitor:
         self.store.set(self._left_key(self.rank), b"1")
 
 
+# Default limit of each fused call's wait for its tokens.  The sampling
+# kernel's own bounded waits give up after 2e9 SM cycles (about 1.0 s at the
+# top clock, 1.7 s at the 1.2 GHz a power-capped board can fall to), and a
+# call whose kernel gave up still completes the exchange, marked as failed;
+# 3 s keeps that report ahead of the wait's own limit while a peer that died
+# with its kernel in flight stalls this rank's stream for seconds, not tens
+# of seconds.
+DEFAULT_WAIT_US = 3_000_000
+
+
 class FusedExchange:
     """The exchange areas of a process group for fs_sample_tp: this rank's
     own area and its peers', mapped here by CUDA IPC.  Every rank calls
-    sample() in the same order (the call sequence number is kept here)."""
+    sample() in the same order (the call sequence number is kept here).
+    timeout_us: the limit of each call's wait for its tokens (after it, the
+    tokens read -1 and fs_tp_failed names the call)."""
 
-    def __init__(self, group=None, monitor=None, timeout_us=10_000_000):
+    def __init__(self, group=None, monitor=None, timeout_us=DEFAULT_WAIT_US):
         self.group = group
         self.monitor = monitor    # an optional PeerMonitor, checked before every call
         self.timeout_us = timeout_us  # limit of each call's wait for its tokens

@@ -61,6 +61,8 @@ def _load():
     lib.oracle_histogram.argtypes = common + [ctypes.c_int, ctypes.c_double, ctypes.c_uint64, _u64p,
                                               ctypes.c_int, _u32p, ctypes.c_uint32, ctypes.c_int64,
                                               _i64p]
+    lib.oracle_argmax.argtypes = [_f64p, ctypes.c_int, _f64p, _f64p]
+    lib.oracle_argmax.restype = ctypes.c_int
     lib.oracle_num_threads.restype = ctypes.c_int
     _lib = lib
     return lib
@@ -123,6 +125,18 @@ def gumbel(r):
     out = np.empty(r.shape, dtype=np.float64)
     lib.oracle_gumbel_batch(_ptr(r, _u32p), _ptr(out, _f64p), r.size)
     return out
+
+
+def argmax(s):
+    """The samplers' argmax scan over a 1-D fp64 score array: returns (index,
+    best, second); -inf entries (masked tokens) never win, the smallest index
+    wins ties, and the index is -1 when every entry is -inf."""
+    lib = _load()
+    s = np.ascontiguousarray(s, dtype=np.float64)
+    b1 = ctypes.c_double()
+    b2 = ctypes.c_double()
+    i = lib.oracle_argmax(_ptr(s, _f64p), int(s.size), ctypes.byref(b1), ctypes.byref(b2))
+    return int(i), b1.value, b2.value
 
 
 def _rows(rows, B):

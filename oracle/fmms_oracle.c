@@ -262,6 +262,12 @@ static int argmax_scan(const double *s, int lo, int hi, double *best,
   return arg;
 }
 
+/* Test entry point: the samplers' argmax scan over s[0, n), with its
+ * best and second-best score (NULL pointers allowed). */
+int oracle_argmax(const double *s, int n, double *best, double *second) {
+  return argmax_scan(s, 0, n, best, second);
+}
+
 /* Flat FMMS sampling of the listed rows.
  * out_idx[i]   = sampled token of row rows[i] (or -1)
  * out_best[i]  = its perturbed score, out_second[i] = runner-up score. */

@@ -9,12 +9,12 @@ test_oracle_pins.py against it: the pin must fail.  The real oracle is never
 touched.  This shows the pins are tight enough that an error of these kinds
 anywhere in the oracle's arithmetic would not go unnoticed.
 
-Not covered, on purpose: the smallest-index rule of the oracle's argmax scan
-over perturbed scores (distinct tokens' scores tie with probability about
-2^-32 per pair, so no pin on random inputs can see it; ties of logits, which
-do occur, are pinned through top-k with every logit tied) and the choice of
-counter tag for the group noise (a reading of the pages, not arithmetic; the
-grouped GPU parity tests compare the tag bit for bit).
+The smallest-index rule of the argmax scan is pinned on planted exact ties
+through the oracle's argmax test entry point (perturbed scores of distinct
+tokens tie with probability about 2^-32 per pair, so random sampler inputs
+cannot show it).  Not covered, on purpose: the choice of counter tag for the
+group noise (a reading of the pages, not arithmetic; the grouped GPU parity
+tests compare the tag bit for bit).
 """
 import importlib.util
 import os
@@ -90,6 +90,14 @@ MUTANTS = [
      "2u * (uint32_t)k, mask, s);",
      "0u * (uint32_t)k, mask, s);",
      "test_multi_samples_are_softmax_draws", {}),
+    ("argmax_ties_toward_the_larger_index",
+     "if (arg < 0 || s[v] > b1) {\n      b2 = b1;",
+     "if (arg < 0 || s[v] >= b1) {\n      b2 = b1;",
+     "test_oracle_argmax_scan_ties_to_the_smallest_index", {}),
+    ("argmax_second_best_dropped",
+     "} else if (s[v] > b2) {\n      b2 = s[v];\n    }\n  }\n  if (best) *best = b1;",
+     "}\n  }\n  if (best) *best = b1;",
+     "test_oracle_argmax_scan_ties_to_the_smallest_index", {}),
     ("topk_ties_toward_the_larger_index",
      "return (x->v < y->v) ? -1 : (x->v > y->v);",
      "return (x->v > y->v) ? -1 : (x->v < y->v);",

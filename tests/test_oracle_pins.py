@@ -385,6 +385,30 @@ def test_tie_rule_smallest_index():
         assert _reduce_parts(s, parts) == 1
 
 
+def test_oracle_argmax_scan_ties_to_the_smallest_index(oracle):
+    """The oracle's own argmax scan (the one every sampler runs) on scores
+    drawn from a handful of values, so exact ties are everywhere, with -inf
+    (masked) entries mixed in: the index is numpy's argmax, whose documented
+    rule is the first occurrence of the maximum; the best score is the
+    maximum and the second-best is the second entry of the sorted finite
+    scores (equal to the best on a tie); all -inf gives -1."""
+    rng = np.random.default_rng(12)
+    for n in (1, 2, 3, 7, 64, 1000):
+        for _ in range(200):
+            s = rng.integers(0, 4, size=n).astype(np.float64) - 1.5
+            s[rng.random(n) < 0.3] = -np.inf
+            idx, best, second = oracle.argmax(s)
+            fin = np.sort(s[np.isfinite(s)])
+            if fin.size == 0:
+                assert idx == -1 and best == -np.inf and second == -np.inf
+                continue
+            assert idx == int(np.argmax(s)), (s, idx)
+            assert best == fin[-1]
+            assert second == (fin[-2] if fin.size > 1 else -np.inf)
+    assert oracle.argmax(np.array([2.0, 5.0, 5.0, 5.0]))[0] == 1
+    assert oracle.argmax(np.full(9, -np.inf))[0] == -1
+
+
 # --------------------------------------------------------------------------
 # Group-Gumbel-Max
 # --------------------------------------------------------------------------

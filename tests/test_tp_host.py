@@ -301,8 +301,8 @@ def _fused_host_rank(rank, world, port, store_port, results):
     torch.cuda.synchronize = lambda *a, **k: None     # no device here
     store = dist.TCPStore("127.0.0.1", store_port, None, False,
                           timeout=datetime.timedelta(seconds=30))
-    ex = tp.FusedExchange(monitor=tp.PeerMonitor(store, rank, world, timeout_s=2.0),
-                          timeout_us=123_456)
+    kw = {} if rank == 1 else {"timeout_us": 123_456}   # rank 1 keeps the default limit
+    ex = tp.FusedExchange(monitor=tp.PeerMonitor(store, rank, world, timeout_s=2.0), **kw)
     H = torch.zeros(4, 8)
     outcome = "done"
     for call in range(4):
@@ -344,3 +344,6 @@ def test_fused_exchange_stops_before_launching_when_a_peer_died():
                     ("sample", 1, (1000, 2001)), ("wait", 1, 1000, 123_456)]
     log1, outcome1 = results[1]
     assert outcome1 == "exited" and [e[1] for e in log1 if e[0] == "sample"] == [0, 1]
+    from lm_head_exact_fmms_b200 import tp
+    assert tp.DEFAULT_WAIT_US == 3_000_000
+    assert [e[3] for e in log1 if e[0] == "wait"] == [tp.DEFAULT_WAIT_US] * 2
