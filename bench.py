@@ -234,20 +234,41 @@ def algorithmic(B, d, V, masked):
     return nbytes, 2.0 * B * V * d
 
 
-def roofline(B, d, V, masked, kernel_us, peaks, peak_kind, traffic):
+# A timed region at least this long runs at the board's power limit, so its
+# tensor roofline is the sustained bf16 peak; a shorter one (a kernel timed
+# in isolation, back to back for milliseconds) takes the burst peak.
+SUSTAINED_REGION_S = 1.0
+
+
+def regime_of(region_s):
+    return "sustained" if region_s >= SUSTAINED_REGION_S else "burst"
+
+
+def roofline(B, d, V, masked, kernel_us, peaks, peak_kind, traffic, regime="burst"):
+    """Roofline of one call: the bound is the larger of (algorithmic bytes /
+    measured copy bandwidth) and (flops / measured bf16 peak of the regime:
+    burst for a short region, sustained for one of seconds at the power
+    limit).  `fracs` carries the achieved rate against every peak, so a point
+    near the ridge shows both."""
     nbytes, flops = algorithmic(B, d, V, masked)
+    tc_key = "bf16_tflops_sustained" if regime == "sustained" else "bf16_tflops"
     t_mem = nbytes / (peaks["hbm_gbs"] * 1e9)
-    t_tc = flops / (peaks["bf16_tflops_sustained"] * 1e12)
+    t_tc = flops / (peaks[tc_key] * 1e12)
+    gbs = nbytes / (kernel_us * 1e-6) / 1e9
+    tfs = flops / (kernel_us * 1e-6) / 1e12
     if t_mem >= t_tc:
-        achieved = nbytes / (kernel_us * 1e-6) / 1e9
-        r = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+        r = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
     else:
-        achieved = flops / (kernel_us * 1e-6) / 1e12
-        r = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops_sustained"],
-             "unit": "TFLOP/s"}
+        r = {"bound": "tensor", "achieved": tfs, "peak": peaks[tc_key], "unit": "TFLOP/s"}
     r["frac"] = r["achieved"] / r["peak"]
     r["traffic"] = traffic
-    r["peak_source"] = "%s (MEASURED_PEAKS.json)" % peak_kind if peak_kind == "measured" else "fallback"
+    r["regime"] = regime
+    r["peak_source"] = ("%s %s (MEASURED_PEAKS.json)" % (peak_kind, tc_key if r["bound"] == "tensor"
+                                                        else "hbm_gbs")
+                        if peak_kind == "measured" else "fallback")
+    r["fracs"] = {"hbm": round(gbs / peaks["hbm_gbs"], 4),
+                  "tensor_burst": round(tfs / peaks["bf16_tflops"], 4),
+                  "tensor_sustained": round(tfs / peaks["bf16_tflops_sustained"], 4)}
     r["algorithmic_bytes"] = nbytes
     r["algorithmic_flops"] = flops
     return r
@@ -422,7 +443,7 @@ def run_gpu(args, world, rank, local):
             binding.fs_sample_ex(H, W, temperature=wl.temperature, seed=0, row_seeds=rs, step=i,
                                  mask_bits=mask, out_idx=out, workspace=ws, stream=stream)
 
-    sampler = ClockSampler(local)
+    sampler = ClockSampler(local, period=0.002)
     with nvtx("fmms: timed steps"):
         region_ms, per_call = time_calls(step, args.steps, args.warmup, stream, world, sampler)
     region_ms = max_over_ranks(region_ms, world)
@@ -469,7 +490,8 @@ def run_gpu(args, world, rank, local):
         "hbm_gbs_per_gpu": round(nbytes / (us_per_call * 1e-6) / 1e9, 1),
         "kernel_us": round(kernel_us, 3),
         "roofline": roofline(B, wl.d, W.shape[0], mask is not None, kernel_us, peaks, peak_kind,
-                             None if tp else committed_traffic("%s/B%d" % (wl.name, B))),
+                             None if tp else committed_traffic("%s/B%d" % (wl.name, B)),
+                             regime_of(region_ms * 1e-3)),
         "e2e": {"value": round(e2e_ms * 1e3 / args.steps, 3), "unit": UNIT,
                 "h2d_bytes_per_step": B * wl.d * 2, "d2h_bytes_per_step": B * 4,
                 "entry_point": "fs_sample_host (pinned host H in, host tokens out)"},
@@ -481,7 +503,23 @@ def run_gpu(args, world, rank, local):
     # only: at N > 1 it would hold the other GPUs idle while rank 0 works.
     if rank == 0 and world == 1 and not args.no_sweep:
         with nvtx("fmms: batch sweep"):
-            result["sweep"] = sweep(torch, binding, synth, W, wl, dev, stream, peaks, peak_kind)
+            result["sweep"] = sweep(torch, binding, synth, W, wl, dev, stream, peaks, peak_kind,
+                                    compare_single=True)
+        with nvtx("fmms: sustained decode"):
+            result["sustained"] = sustained_point(torch, binding, synth, W, wl, dev, stream, peaks,
+                                                  peak_kind, local)
+        # The other LM-head shapes, each at its own batch sizes.
+        result["sweeps"] = {}
+        for other in ("qwen3-1.7b", "large"):
+            owl = synth.WORKLOADS[other]
+            with nvtx("fmms: batch sweep, %s head" % other):
+                Wo = synth.make_weight(owl.V, owl.d, owl.w_std, device=dev)
+                result["sweeps"][other] = {
+                    "workload": "%s LM head d=%d V=%d T=%g, fused fs_sample_ex"
+                                % (other, owl.d, owl.V, owl.temperature),
+                    "points": sweep(torch, binding, synth, Wo, owl, dev, stream, peaks, peak_kind)}
+                del Wo
+                torch.cuda.empty_cache()
         with nvtx("fmms: grouped + masked"):
             result["grouped_masked"] = grouped_points(torch, binding, synth, dev, stream, peaks,
                                                       peak_kind, W)
@@ -504,7 +542,10 @@ def run_gpu(args, world, rank, local):
     return result
 
 
-def sweep(torch, binding, synth, W, wl, dev, stream, peaks, peak_kind, steps=200, warmup=10):
+def sweep(torch, binding, synth, W, wl, dev, stream, peaks, peak_kind, steps=200, warmup=10,
+          compare_single=False):
+    """Each of the workload's batch sizes, `steps` back-to-back calls after a
+    one-second idle: a short region, so the burst tensor peak applies."""
     rows = []
     for B in wl.batches:
         H = synth.make_hidden(B, wl.d, device=dev)
@@ -518,16 +559,17 @@ def sweep(torch, binding, synth, W, wl, dev, stream, peaks, peak_kind, steps=200
         region_ms, per = time_calls(step, steps, warmup, stream)
         kus = sum(per) / len(per)
         rf = roofline(B, wl.d, wl.V, False, kus, peaks, peak_kind,
-                      committed_traffic("%s/B%d" % (wl.name, B)))
+                      committed_traffic("%s/B%d" % (wl.name, B)), regime_of(region_ms * 1e-3))
         row = {"B": B, "us_per_call": round(region_ms * 1e3 / steps, 3),
                "kernel_us": round(kus, 3),
                "kernel_us_p10_p50_p90": [round(x, 3) for x in percentiles(per)],
                "bound": rf["bound"],
                "achieved": round(rf["achieved"], 1), "unit": rf["unit"],
-               "frac": round(rf["frac"], 4),
+               "frac": round(rf["frac"], 4), "fracs": rf["fracs"], "regime": rf["regime"],
+               "traffic": rf["traffic"],
                # the library's automatic choice: CTA pairs above 64 rows per launch
-               "cta_pairs": B > 64}
-        if B > 64:
+               "cta_pairs": binding.fs_uses_cta_pairs(B)}
+        if compare_single and row["cta_pairs"]:
             # the same call on the single-CTA kernel, for comparison
             binding.fs_set_cta_pairs(0)
             try:
@@ -537,6 +579,37 @@ def sweep(torch, binding, synth, W, wl, dev, stream, peaks, peak_kind, steps=200
             row["single_cta_kernel_us"] = round(sum(per1) / len(per1), 3)
         rows.append(row)
     return rows
+
+
+def sustained_point(torch, binding, synth, W, wl, dev, stream, peaks, peak_kind, local, B=64,
+                    seconds=2.5):
+    """The decode regime: B=64 calls back to back for `seconds` (the board
+    sits at its power limit and the SM clock gives way), with the clocks
+    sampled throughout.  Reports the kernel time, the median SM clock, the
+    kernel time in clock cycles (time x median MHz) and the roofline against
+    the copy bandwidth."""
+    H = synth.make_hidden(B, wl.d, device=dev)
+    rs = synth.make_row_seeds(B, device=dev) if wl.per_row_seeds else None
+    out = torch.empty(B, dtype=torch.int32, device=dev)
+
+    def step(i):
+        binding.fs_sample_ex(H, W, temperature=wl.temperature, seed=0, row_seeds=rs, step=i,
+                             out_idx=out, stream=stream)
+
+    calls = max(100, int(seconds / 200e-6))
+    sampler = ClockSampler(local, period=0.01)
+    region_ms, per = time_calls(step, calls, 20, stream, sampler=sampler)
+    kus = sum(per) / len(per)
+    clk = sampler.summary()
+    rf = roofline(B, wl.d, wl.V, False, kus, peaks, peak_kind, None, regime_of(region_ms * 1e-3))
+    return {"B": B, "calls": calls, "region_s": round(region_ms * 1e-3, 3),
+            "us_per_call": round(region_ms * 1e3 / calls, 3), "kernel_us": round(kus, 3),
+            "kernel_us_p10_p50_p90": [round(x, 3) for x in percentiles(per)],
+            "sm_mhz_median": clk["sm_mhz"], "clock_samples": clk["samples"],
+            "reasons": clk["reasons"],
+            "kcycles_per_call": round(kus * clk["sm_mhz"] / 1e3, 1) if clk["sm_mhz"] else None,
+            "bound": rf["bound"], "achieved": round(rf["achieved"], 1), "unit": rf["unit"],
+            "frac": round(rf["frac"], 4), "regime": rf["regime"]}
 
 
 def grouped_points(torch, binding, synth, dev, stream, peaks, peak_kind, W8, steps=100):
@@ -556,11 +629,13 @@ def grouped_points(torch, binding, synth, dev, stream, peaks, peak_kind, W8, ste
 
         region_ms, _ = time_calls(step, steps, 10, stream)
         us = region_ms * 1e3 / steps
-        rf = roofline(B, wl.d, wl.V, True, us, peaks, peak_kind, None)
+        rf = roofline(B, wl.d, wl.V, True, us, peaks, peak_kind,
+                      committed_traffic("%s/B%d" % (wl.name, B)), regime_of(region_ms * 1e-3))
         rows.append({"B": B, "us_per_call": round(us, 3), "bound": rf["bound"],
                      "achieved": round(rf["achieved"], 1), "unit": rf["unit"],
-                     "frac": round(rf["frac"], 4),
-                     "launches_per_call": 2 * ((B + 255) // 256)})
+                     "frac": round(rf["frac"], 4), "fracs": rf["fracs"], "regime": rf["regime"],
+                     "traffic": rf["traffic"],
+                     "launches_per_call": 2 * binding.fs_fused_launches(B, "grouped")})
     return {"workload": "grouped-masked d=%d V=%d G=%d, 50%% mask, T=%g (fused kernel + merge)"
                         % (wl.d, wl.V, wl.groups, wl.temperature), "points": rows}
 

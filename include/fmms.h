@@ -340,14 +340,27 @@ fs_status fs_sample_host(const void *H_host, const void *W, int B, int d,
  * (split the batch into several calls).  The first call on each device
  * looks up the array's device address and may load the library's device
  * code; make that first call before any stream capture.  Each call clears
- * the array on `stream` before using it, and every call on a device shares
- * the same array: calls that overlap on the GPU (different streams or
- * threads) race, so the caller must order them. */
+ * the array's ticket and keys on `stream` before using them, and every call
+ * on a device shares the same array: calls that overlap on the GPU
+ * (different streams or threads) race, so the caller must order them.
+ * Device-side errors: a kernel that gave up on a bounded wait records
+ * FS_ERR_DEVICE_TIMEOUT in the array's own status word (not in any
+ * workspace; fs_device_status does not see it) and leaves out_idx
+ * unwritten; the word keeps it across later calls until fs_noalloc_status
+ * reads and clears it. */
 fs_status fs_sample_noalloc(const void *H, const void *W, int B, int d, int V,
                             float temperature, uint64_t seed,
                             const uint64_t *row_seeds, uint32_t step,
                             const uint32_t *mask_bits, int32_t *out_idx,
                             fs_stream_t stream);
+
+/* Reads (synchronously, after `stream` drains) and clears the status word of
+ * fs_sample_noalloc's fixed array on the current device: FS_OK, or
+ * FS_ERR_DEVICE_TIMEOUT when a call since the last read gave up on a bounded
+ * wait (its tokens were not written); FS_OK too before the first call.
+ * Allocates nothing; like fs_sample_noalloc, it must not overlap such a call
+ * on the GPU.  The paper has no counterpart for this entry point. */
+fs_status fs_noalloc_status(fs_stream_t stream);
 
 /* Bytes of caller workspace needed by the calls above for these sizes on the
  * current device (G = 0 or 1 for flat sampling).  Returns 0 on invalid sizes. */
@@ -363,7 +376,8 @@ size_t fs_workspace_bytes_summary(int B, int V_g);
 /* Reads (synchronously, after the stream drains) and clears the device-side
  * status word of a workspace (NULL = the library-owned one on the current
  * device).  Returns FS_OK or FS_ERR_DEVICE_TIMEOUT; after a timeout the
- * workspace is zero-filled again so it can be reused. */
+ * workspace is zero-filled again so it can be reused.  fs_sample_noalloc
+ * keeps its status in its own array: read it with fs_noalloc_status. */
 fs_status fs_device_status(void *workspace, size_t workspace_bytes,
                            fs_stream_t stream);
 
@@ -401,6 +415,17 @@ fs_status fs_test_stalled_sample(const void *H, const void *W, int B, int d,
                                  int V, int32_t *out_idx, void *workspace,
                                  size_t workspace_bytes, fs_stream_t stream);
 
+/* Host-side fault injection for failure-detection tests (nothing is done to
+ * the GPU).  kind 1 ("alloc"): every device allocation the library would
+ * make fails; kind 2 ("launch"): every call that would enqueue work on a
+ * stream fails; either way the call returns FS_ERR_CUDA before it touches
+ * the GPU, and the library stays usable once the kind is back to 0 (none).
+ * The initial kind comes from the environment variable FS_FAULT ("alloc" or
+ * "launch"; anything else is none), read at the first call.  kind -1 leaves
+ * the setting as it is; *previous (if not NULL) receives the kind in force
+ * before the call.  Process-wide.  FS_ERR_INVALID_ARG for kind < -1 or > 2. */
+fs_status fs_test_inject_fault(int kind, int *previous);
+
 /* ---- Kernel choice ---- */
 
 /* Whether flat-mode calls (fs_sample, fs_sample_ex, fs_sample_host,
@@ -410,8 +435,9 @@ fs_status fs_test_stalled_sample(const void *H, const void *W, int B, int d,
  * (tcgen05 cta_group::2), each SM staging 128 rows of W and half of the batch
  * rows of H per pipeline stage.  This is a B200 design choice, not part of
  * the method: the results are the same either way (tokens bit for bit).
- * policy: -1 automatic (the default: pairs for launches of more than 64
- * batch rows), 0 never, 1 always.  Process-wide; applies to calls made after
+ * policy: -1 automatic (the default: pairs for launches whose batch tile,
+ * the row count rounded up to a multiple of 16, is 128 or more, i.e. from
+ * 113 rows per launch; fs_plan_batch reports the choice), 0 never, 1 always.  Process-wide; applies to calls made after
  * it returns.  FS_ERR_INVALID_ARG for any other value.  When the device
  * cannot co-schedule a pair, the single-CTA kernel runs.  The unfused
  * measurement path (fs_sample_unfused, fs_sample_topk) always runs on single
@@ -457,6 +483,15 @@ fs_status fs_plan_tiles(int V, int G, int num_sms, int cta, int32_t *tiles,
  * starts a segment with an 8-row partial tile), else 0. */
 fs_status fs_plan_tiles_merged(int V, int G, int num_sms, int cta, int32_t *tiles,
                                int max_tiles, int *ntiles, int *merges);
+
+/* How a call of B rows is launched: *launches = fused-kernel launches (one
+ * per 256 rows), *batch_tile = the first launch's batch tile (MMA N: the
+ * row count rounded up to a multiple of 16, at most 256), *cta_pairs = 1 when
+ * the current fs_set_cta_pairs policy runs it on CTA pairs (on a device
+ * that can co-schedule them), else 0.  kind: 0 flat (fs_sample and the
+ * other flat-mode calls), 1 grouped, 2 unfused / top-k (logits mode, single
+ * CTAs).  Output pointers other than `launches` may be NULL.  Host-only. */
+fs_status fs_plan_batch(int B, int kind, int *launches, int *batch_tile, int *cta_pairs);
 
 /* The CTAs whose vocabulary range meets group g (0 <= g < G), as the grouped
  * merge kernel enumerates them: [*first, *last].  Host-only. */

@@ -27,7 +27,8 @@ EXPORTED = ("fs_sample", "fs_sample_ex", "fs_sample_grouped", "fs_sample_unfused
             "fs_sample_topk", "fs_set_cta_pairs", "fs_tp_area_bytes", "fs_tp_area_create",
             "fs_tp_area_destroy", "fs_ipc_handle", "fs_ipc_open", "fs_ipc_close", "fs_sample_tp",
             "fs_tp_wait", "fs_tp_failed", "fs_test_stall_loads", "fs_set_partial_merge",
-            "fs_plan_tiles_merged")
+            "fs_plan_tiles_merged", "fs_plan_batch", "fs_noalloc_status",
+            "fs_test_inject_fault")
 
 FS_IPC_HANDLE_BYTES = 64
 
@@ -104,6 +105,10 @@ def load_library():
                                        ctypes.POINTER(ctypes.c_int)]
     lib.fs_plan_tiles_merged.argtypes = [i32, i32, i32, i32, vp, i32,
                                          ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
+    lib.fs_plan_batch.argtypes = [i32, i32, ctypes.POINTER(ctypes.c_int),
+                                  ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
+    lib.fs_noalloc_status.argtypes = [vp]
+    lib.fs_test_inject_fault.argtypes = [i32, ctypes.POINTER(ctypes.c_int)]
     for name in EXPORTED:
         if name not in ("fs_workspace_bytes", "fs_workspace_bytes_multi",
                         "fs_workspace_bytes_summary", "fs_status_string", "fs_tp_area_bytes"):
@@ -312,6 +317,27 @@ def fs_plan_tiles_merged(V, G, num_sms, cta, max_tiles=4096):
     return buf[: min(n.value, max_tiles)].copy(), bool(merges.value)
 
 
+_PLAN_KINDS = {"flat": 0, "grouped": 1, "logits": 2}
+
+
+def fs_plan_batch(B, kind="flat"):
+    """Host-only query of how a call of B rows launches: (fused launches,
+    first launch's batch tile, 1 if the current policy runs it on CTA pairs)."""
+    lib = load_library()
+    n, bn, pairs = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
+    _check(lib.fs_plan_batch(int(B), _PLAN_KINDS[kind], ctypes.byref(n), ctypes.byref(bn),
+                             ctypes.byref(pairs)), "fs_plan_batch")
+    return n.value, bn.value, pairs.value
+
+
+def fs_uses_cta_pairs(B, kind="flat"):
+    return bool(fs_plan_batch(B, kind)[2])
+
+
+def fs_fused_launches(B, kind="flat"):
+    return fs_plan_batch(B, kind)[0]
+
+
 def plan_num_ctas(V, G, num_sms):
     lib = load_library()
     n = ctypes.c_int(0)
@@ -345,6 +371,25 @@ def fs_sample_noalloc(H, W, temperature=1.0, seed=0, row_seeds=None, step=0, mas
                                  _ptr(row_seeds), int(step), _ptr(mask_bits), _ptr(out_idx),
                                  _stream(stream)), "fs_sample_noalloc")
     return out_idx
+
+
+def fs_noalloc_status(stream=None):
+    """Reads and clears the status word of fs_sample_noalloc's fixed array:
+    0 (FS_OK) or 5 (FS_ERR_DEVICE_TIMEOUT: a call gave up on a bounded wait)."""
+    return int(load_library().fs_noalloc_status(_stream(stream)))
+
+
+FAULT_KINDS = {"none": 0, "alloc": 1, "launch": 2}
+
+
+def fs_test_inject_fault(kind=None):
+    """Sets the host-side fault injection ("none", "alloc" or "launch"; None
+    leaves it unchanged) and returns the kind in force before the call."""
+    lib = load_library()
+    prev = ctypes.c_int(0)
+    k = -1 if kind is None else FAULT_KINDS[kind]
+    _check(lib.fs_test_inject_fault(k, ctypes.byref(prev)), "fs_test_inject_fault")
+    return {v: n for n, v in FAULT_KINDS.items()}[prev.value]
 
 
 def fs_test_stalled_sample(H, W, workspace, out_idx=None, stream=None):

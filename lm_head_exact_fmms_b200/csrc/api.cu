@@ -5,8 +5,10 @@
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "fmms.h"
@@ -73,9 +75,32 @@ fs_status get_device(DeviceState **out) {
   return FS_OK;
 }
 
+// Host-side fault injection for failure-detection tests.  FS_FAULT=alloc
+// makes every device allocation the library would make fail, FS_FAULT=launch
+// every call that would enqueue work; such a call returns FS_ERR_CUDA before
+// it touches the GPU.  The environment is read once; fs_test_inject_fault
+// overrides it.
+constexpr int kFaultNone = 0, kFaultAlloc = 1, kFaultLaunch = 2;
+std::atomic<int> g_fault{-1};  // -1: environment not read yet
+
+int fault_mode() {
+  int f = g_fault.load(std::memory_order_relaxed);
+  if (f >= 0) return f;
+  const char *e = getenv("FS_FAULT");
+  f = kFaultNone;
+  if (e != nullptr && strcmp(e, "alloc") == 0) f = kFaultAlloc;
+  if (e != nullptr && strcmp(e, "launch") == 0) f = kFaultLaunch;
+  int expect = -1;
+  g_fault.compare_exchange_strong(expect, f);
+  return g_fault.load(std::memory_order_relaxed);
+}
+
+bool launch_fault() { return fault_mode() == kFaultLaunch; }
+
 // Grows a library-owned device buffer; new memory is zero-filled.
 fs_status grow(void **buf, size_t *have, size_t need) {
   if (*have >= need) return FS_OK;
+  if (fault_mode() == kFaultAlloc) return FS_ERR_CUDA;
   if (*buf) {
     cudaDeviceSynchronize();
     cudaFree(*buf);
@@ -336,6 +361,7 @@ fs_status run_locked(int mode, const void *H, const void *W, int B, int d, int V
                      const uint32_t *mask, int32_t *out_idx, fs_group_summary *summary,
                      float *logits, void *ws, size_t ws_bytes, cudaStream_t stream,
                      const ShardOpts &shard) {
+  if (launch_fault()) return FS_ERR_CUDA;
   DeviceState *st = nullptr;
   fs_status s = get_device(&st);
   if (s != FS_OK) return s;
@@ -509,6 +535,7 @@ fs_status fs_sample_host(const void *H_host, const void *W, int B, int d, int V,
   if (B < 1 || V < 1 || d < 8 || (d % 8) != 0) return FS_ERR_INVALID_ARG;
   if (!(temperature > 0.f) || !isfinite(temperature) || !W || !aligned16(W))
     return FS_ERR_INVALID_ARG;
+  if (launch_fault()) return FS_ERR_CUDA;
   cudaStream_t st_ = static_cast<cudaStream_t>(stream);
   std::lock_guard<std::mutex> lock(g_mu);
   DeviceState *st = nullptr;
@@ -631,6 +658,7 @@ fs_status fs_tp_area_create(void **area) {
   fs_status s = get_device(&st);
   if (s != FS_OK) return s;
   *area = nullptr;
+  if (fault_mode() == kFaultAlloc) return FS_ERR_CUDA;
   if (cudaMalloc(area, fmms::kTpAreaBytes) != cudaSuccess) return FS_ERR_CUDA;
   if (cudaMemset(*area, 0, fmms::kTpAreaBytes) != cudaSuccess ||
       cudaDeviceSynchronize() != cudaSuccess) {
@@ -702,6 +730,7 @@ fs_status fs_tp_wait(const void *area, int B, uint32_t seq, int32_t *out_idx,
   if (area == nullptr || out_idx == nullptr || B < 1 || B > fmms::kMaxBN || timeout_us < 1 ||
       timeout_us > kMaxTpWaitUs)
     return FS_ERR_INVALID_ARG;
+  if (launch_fault()) return FS_ERR_CUDA;
   DeviceState *st = nullptr;
   fs_status s = get_device(&st);
   if (s != FS_OK) return s;
@@ -746,6 +775,7 @@ size_t fs_workspace_bytes_multi(int B, int V, int num_samples) {
 
 fs_status fs_keys_to_tokens(const int64_t *keys, int B, int32_t *out_idx, fs_stream_t stream) {
   if (!keys || !out_idx || B < 1) return FS_ERR_INVALID_ARG;
+  if (launch_fault()) return FS_ERR_CUDA;
   DeviceState *st = nullptr;
   fs_status s = get_device(&st);
   if (s != FS_OK) return s;
@@ -814,6 +844,7 @@ fs_status fs_merge_groups(const fs_group_summary *summaries, int G, int B, uint6
                           const uint64_t *row_seeds, uint32_t step, int32_t *out_idx,
                           fs_stream_t stream) {
   if (!summaries || !out_idx || G < 1 || B < 1) return FS_ERR_INVALID_ARG;
+  if (launch_fault()) return FS_ERR_CUDA;
   DeviceState *st = nullptr;
   fs_status s = get_device(&st);
   if (s != FS_OK) return s;
@@ -860,6 +891,7 @@ const char *fs_status_string(fs_status status) {
 fs_status fs_philox4x32_10(const uint32_t *ctr, const uint32_t *key, uint32_t *out, int64_t n,
                            fs_stream_t stream) {
   if (n < 0 || (n > 0 && (!ctr || !key || !out))) return FS_ERR_INVALID_ARG;
+  if (launch_fault()) return FS_ERR_CUDA;
   DeviceState *st = nullptr;
   fs_status s = get_device(&st);
   if (s != FS_OK) return s;
@@ -870,6 +902,7 @@ fs_status fs_philox4x32_10(const uint32_t *ctr, const uint32_t *key, uint32_t *o
 
 fs_status fs_gumbel(const uint32_t *r, float *g, int64_t n, fs_stream_t stream) {
   if (n < 0 || (n > 0 && (!r || !g))) return FS_ERR_INVALID_ARG;
+  if (launch_fault()) return FS_ERR_CUDA;
   DeviceState *st = nullptr;
   fs_status s = get_device(&st);
   if (s != FS_OK) return s;
@@ -882,6 +915,14 @@ fs_status fs_set_partial_merge(int policy) {
   if (policy < -1 || policy > 1) return FS_ERR_INVALID_ARG;
   std::lock_guard<std::mutex> lock(g_mu);
   g_merge_policy = policy;
+  return FS_OK;
+}
+
+fs_status fs_test_inject_fault(int kind, int *previous) {
+  if (kind < -1 || kind > kFaultLaunch) return FS_ERR_INVALID_ARG;
+  const int before = fault_mode();
+  if (previous) *previous = before;
+  if (kind >= 0) g_fault.store(kind, std::memory_order_relaxed);
   return FS_OK;
 }
 
@@ -935,6 +976,20 @@ fs_status fs_plan_tiles_merged(int V, int G, int num_sms, int cta, int32_t *tile
   return FS_OK;
 }
 
+fs_status fs_plan_batch(int B, int kind, int *launches, int *batch_tile, int *cta_pairs) {
+  if (B < 1 || kind < 0 || kind > 2 || !launches) return FS_ERR_INVALID_ARG;
+  const int mode = kind == 1 ? fmms::kModeGrouped : kind == 2 ? fmms::kModeLogits : fmms::kModeFlat;
+  const int first = fmms::imin(fmms::kMaxBN, B);
+  const int BN = fmms::fmms_batch_tile(first);
+  *launches = (B + fmms::kMaxBN - 1) / fmms::kMaxBN;
+  if (batch_tile) *batch_tile = BN;
+  if (cta_pairs) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    *cta_pairs = use_pairs(mode, BN) ? 1 : 0;
+  }
+  return FS_OK;
+}
+
 fs_status fs_plan_group_ctas(int V, int G, int num_sms, int g, int *first, int *last) {
   if (V < 1 || G < 1 || G > V || num_sms < 1 || g < 0 || g >= G || !first || !last)
     return FS_ERR_INVALID_ARG;
@@ -984,8 +1039,33 @@ extern "C" fs_status fs_sample_noalloc(const void *H, const void *W, int B, int 
     }
     scratch = g_noalloc_addr[dev];
   }
+  // Everything after the status word starts at zero (the ticket and keys are
+  // left zeroed by a completed call, but not by one that gave up on a
+  // bounded wait); the status word keeps a recorded timeout until
+  // fs_noalloc_status reads and clears it.
+  if (launch_fault()) return FS_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(scratch, 0, kNoAllocScratchBytes, st) != cudaSuccess) return FS_ERR_CUDA;
+  if (cudaMemsetAsync(static_cast<char *>(scratch) + 4, 0, kNoAllocScratchBytes - 4, st) !=
+      cudaSuccess)
+    return FS_ERR_CUDA;
   return run(fmms::kModeFlat, H, W, B, d, V, 1, temperature, seed, row_seeds, step, mask_bits,
              out_idx, nullptr, nullptr, scratch, kNoAllocScratchBytes, st);
+}
+
+extern "C" fs_status fs_noalloc_status(fs_stream_t stream) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FS_ERR_CUDA;
+  void *scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    scratch = g_noalloc_addr[dev];
+  }
+  if (scratch == nullptr) return FS_OK;  // no call on this device yet
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FS_ERR_CUDA;
+  int err = 0;
+  if (cudaMemcpy(&err, scratch, sizeof err, cudaMemcpyDeviceToHost) != cudaSuccess)
+    return FS_ERR_CUDA;
+  if (err == 0) return FS_OK;
+  if (cudaMemset(scratch, 0, kNoAllocScratchBytes) != cudaSuccess) return FS_ERR_CUDA;
+  return FS_ERR_DEVICE_TIMEOUT;
 }

@@ -72,6 +72,73 @@ def test_grouped_and_unfused_validation(lib):
     assert lib.fs_gumbel(None, None, -1, None) == 1
 
 
+@pytest.mark.parametrize("B,kind,want", [
+    (1, "flat", (1, 16, 0)), (16, "flat", (1, 16, 0)), (17, "flat", (1, 32, 0)),
+    (64, "flat", (1, 64, 0)), (112, "flat", (1, 112, 0)), (113, "flat", (1, 128, 1)),
+    (200, "flat", (1, 208, 1)), (256, "flat", (1, 256, 1)), (257, "flat", (2, 256, 1)),
+    (1, "grouped", (1, 16, 0)), (512, "grouped", (2, 256, 1)), (100, "grouped", (1, 112, 0)),
+    (256, "logits", (1, 256, 0)), (300, "logits", (2, 256, 0)),
+])
+def test_plan_batch_automatic_choice(lib, B, kind, want):
+    """The launch plan of a call: one fused launch per 256 rows, the batch
+    tile rounded up to 16 rows, and CTA pairs (automatic policy) from a
+    128-row tile up, never in logits mode."""
+    binding.fs_set_cta_pairs(-1)
+    assert binding.fs_plan_batch(B, kind) == want
+
+
+def test_plan_batch_follows_the_pair_policy(lib):
+    try:
+        binding.fs_set_cta_pairs(0)
+        assert binding.fs_plan_batch(256)[2] == 0
+        binding.fs_set_cta_pairs(1)
+        assert binding.fs_plan_batch(1)[2] == 1 and binding.fs_plan_batch(1, "grouped")[2] == 1
+        assert binding.fs_plan_batch(1, "logits")[2] == 0
+    finally:
+        binding.fs_set_cta_pairs(-1)
+    n = ctypes.c_int(0)
+    assert lib.fs_plan_batch(0, 0, ctypes.byref(n), None, None) == 1
+    assert lib.fs_plan_batch(4, 3, ctypes.byref(n), None, None) == 1
+    assert lib.fs_plan_batch(4, 0, None, None, None) == 1
+
+
+def test_fault_injection_switch(lib):
+    """fs_test_inject_fault sets and reports the kind; invalid kinds are
+    refused; with "launch" set a sampling call with valid arguments fails with
+    FS_ERR_CUDA before touching any device."""
+    assert binding.fs_test_inject_fault("launch") == "none"
+    try:
+        assert binding.fs_test_inject_fault() == "launch"
+        assert _sample(lib) == 3
+        assert lib.fs_sample_noalloc(FAKE, FAKE, 4, 64, 100, 1.0, 0, None, 0, None, FAKE,
+                                     None) == 3
+        assert binding.fs_test_inject_fault("alloc") == "launch"
+        area = ctypes.c_void_p(0)
+        assert lib.fs_tp_area_create(ctypes.byref(area)) in (2, 3)
+        assert area.value is None
+    finally:
+        binding.fs_test_inject_fault("none")
+    prev = ctypes.c_int(0)
+    assert lib.fs_test_inject_fault(3, ctypes.byref(prev)) == 1
+    assert lib.fs_test_inject_fault(-2, None) == 1
+
+
+@pytest.mark.parametrize("env,kind", [("alloc", "alloc"), ("launch", "launch"), ("", "none"),
+                                      ("bogus", "none")])
+def test_fault_injection_reads_the_environment(env, kind):
+    """FS_FAULT sets the initial kind, read at the first call (a fresh
+    process per value)."""
+    import subprocess
+    import sys
+    code = ("from lm_head_exact_fmms_b200 import binding; "
+            "print(binding.fs_test_inject_fault())")
+    envd = dict(os.environ, FS_FAULT=env)
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True,
+                         env=envd, cwd=ROOT, timeout=300)
+    assert out.returncode == 0, out.stderr[-1000:]
+    assert out.stdout.strip().splitlines()[-1] == kind
+
+
 def _all_tiles(V, G, sms):
     _, nc = binding.fs_plan_tiles(V, G, sms, 0)
     return nc, [binding.fs_plan_tiles(V, G, sms, c)[0] for c in range(nc)]

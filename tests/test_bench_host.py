@@ -42,9 +42,23 @@ def test_roofline_picks_the_larger_bound():
     assert r["traffic"] == 123
     t = bench.roofline(256, 4096, 151936, False, 340.0, PEAKS, "measured", None)
     assert t["bound"] == "tensor" and t["unit"] == "TFLOP/s"
-    assert t["peak"] == PEAKS["bf16_tflops_sustained"]
+    assert t["regime"] == "burst" and t["peak"] == PEAKS["bf16_tflops"]
     assert t["achieved"] == pytest.approx(2 * 256 * 151936 * 4096 / 340e-6 / 1e12)
     assert t["traffic"] is None
+    assert t["fracs"]["tensor_burst"] == pytest.approx(t["achieved"] / PEAKS["bf16_tflops"], abs=1e-4)
+    assert t["fracs"]["tensor_sustained"] == pytest.approx(
+        t["achieved"] / PEAKS["bf16_tflops_sustained"], abs=1e-4)
+    u = bench.roofline(256, 4096, 151936, False, 340.0, PEAKS, "measured", None, "sustained")
+    assert u["regime"] == "sustained" and u["peak"] == PEAKS["bf16_tflops_sustained"]
+
+
+def test_regime_follows_the_region_length():
+    """A region of a second or more runs at the board's power limit (the
+    sustained bf16 peak); shorter ones take the burst peak."""
+    assert bench.regime_of(0.004) == "burst"
+    assert bench.regime_of(0.999) == "burst"
+    assert bench.regime_of(1.0) == "sustained"
+    assert bench.regime_of(2.5) == "sustained"
 
 
 def test_percentiles_and_median():

@@ -48,3 +48,55 @@ def test_wait_timeout_is_reported_and_context_survives(dev, oracle):
     bad = got.cpu().numpy() != idx
     assert not np.any(bad & ((best - second) > 2e-3 * (1 + np.abs(best))))
     assert binding.fs_device_status(ws) == 0
+
+
+def test_injected_host_faults_leave_the_library_usable(dev, oracle):
+    """Host-side fault injection (fs_test_inject_fault, or FS_FAULT in the
+    environment): with "launch" every sampling call fails with FS_ERR_CUDA
+    and enqueues nothing (the output keeps its sentinel); with "alloc" every
+    call that needs new device memory fails the same way; once cleared, the
+    same calls on the same context sample the oracle's tokens."""
+    B, d, V = 16, 64, 3001
+    H = synth.make_hidden(B, d, seed=30)
+    W = synth.make_weight(V, d, 0.125, seed=31)
+    Hd, Wd = H.to(dev), W.to(dev)
+    out = torch.full((B,), -7, dtype=torch.int32, device=dev)
+    keys = torch.zeros(B, dtype=torch.int64, device=dev)
+    torch.cuda.synchronize()
+    binding.fs_test_inject_fault("launch")
+    try:
+        for call in (lambda: binding.fs_sample_ex(Hd, Wd, seed=2, step=1, out_idx=out),
+                     lambda: binding.fs_sample_grouped(Hd, Wd, 4, seed=2, step=1, out_idx=out),
+                     lambda: binding.fs_sample_noalloc(Hd, Wd, seed=2, step=1, out_idx=out),
+                     lambda: binding.fs_keys_to_tokens(keys, out_idx=out)):
+            with pytest.raises(binding.FmmsError) as err:
+                call()
+            assert err.value.status == 3                          # FS_ERR_CUDA
+    finally:
+        binding.fs_test_inject_fault("none")
+    torch.cuda.synchronize()
+    assert (out == -7).all()                                       # nothing ran
+    # 4 MiB of H: more than any host-entry staging buffer the other tests grew
+    Hh = synth.make_hidden(64, 32768, seed=32).pin_memory()
+    W2 = synth.make_weight(64, 32768, 0.01, seed=33).to(dev)
+    binding.fs_test_inject_fault("alloc")
+    try:
+        with pytest.raises(binding.FmmsError) as err:
+            binding.fs_tp_area_create()
+        assert err.value.status == 3
+        with pytest.raises(binding.FmmsError) as err:
+            binding.fs_sample_host(Hh, W2, seed=1)
+        assert err.value.status == 3
+    finally:
+        binding.fs_test_inject_fault("none")
+    got = binding.fs_sample_ex(Hd, Wd, seed=2, step=1, out_idx=out)
+    torch.cuda.synchronize()
+    idx, best, second = oracle.sample(H, W, T=1.0, seed=2, step=1)
+    bad = got.cpu().numpy() != idx
+    assert not np.any(bad & ((best - second) > 2e-3 * (1 + np.abs(best))))
+    host = binding.fs_sample_host(Hh, W2, seed=1)
+    ref = binding.fs_sample(Hh.to(dev), W2, seed=1)
+    torch.cuda.synchronize()
+    assert torch.equal(host.to(dev), ref)
+    area = binding.fs_tp_area_create()
+    binding.fs_tp_area_destroy(area)

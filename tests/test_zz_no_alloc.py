@@ -6,8 +6,10 @@ plug-in only its inputs and outputs.  Instead of a workspace it uses a fixed
 scratch array inside the library.  This test calls it through the C ABI twice
 in a row and compares each result with the regular entry point's tokens for
 the same inputs (the kernels are the same, so the tokens must be identical),
-then checks that a batch above its 256-row limit is refused.  It lives in its
-own file so that pytest collects it last.
+then checks that a batch above its 256-row limit is refused and that a call
+whose kernel gave up on a bounded wait is reported by fs_noalloc_status (the
+array's own status word, which later calls keep until it is read).  It lives
+in its own file so that pytest collects it last.
 """
 import pytest
 import torch
@@ -27,8 +29,11 @@ def dev():
     return torch.device("cuda:0")
 
 
-def test_noalloc_matches_fs_sample_ex_on_two_calls(dev):
-    B, d, V = 96, 256, 20011
+@pytest.mark.parametrize("B", [1, 2, 96, 256])
+def test_noalloc_matches_fs_sample_ex_on_two_calls(dev, B):
+    """1 and 2 rows, 96 rows (single CTAs) and 256 rows (CTA pairs, whose
+    ticket counts both CTAs of every pair)."""
+    d, V = 256, 20011
     H = synth.make_hidden(B, d, device="cpu", seed=7).to(dev)
     W = synth.make_weight(V, d, 1.0 / 16.0, device="cpu", seed=8).to(dev)
     seeds = synth.make_row_seeds(B).to(dev)
@@ -52,3 +57,29 @@ def test_noalloc_refuses_batches_above_its_limit(dev):
     with pytest.raises(binding.FmmsError) as err:
         binding.fs_sample_noalloc(H, W)
     assert err.value.status == 2   # FS_ERR_UNSUPPORTED
+
+
+def test_noalloc_reports_a_kernel_that_gave_up(dev):
+    """With the failure-detection switch on, the load warp issues nothing and
+    the kernel's bounded waits run out (about a second): fs_noalloc_status
+    then reports FS_ERR_DEVICE_TIMEOUT, also after a later good call, and
+    reads 0 once cleared; the calls after it match fs_sample_ex again."""
+    B, d, V = 24, 128, 5003
+    H = synth.make_hidden(B, d, device="cpu", seed=12).to(dev)
+    W = synth.make_weight(V, d, 0.125, device="cpu", seed=13).to(dev)
+    assert binding.fs_noalloc_status() == 0
+    binding.fs_test_stall_loads(True)
+    try:
+        binding.fs_sample_noalloc(H, W, temperature=0.9, seed=5, step=0)
+    finally:
+        binding.fs_test_stall_loads(False)
+    ref = binding.fs_sample_ex(H, W, temperature=0.9, seed=5, step=1)
+    got = binding.fs_sample_noalloc(H, W, temperature=0.9, seed=5, step=1)
+    torch.cuda.synchronize()
+    assert torch.equal(got, ref)
+    assert binding.fs_noalloc_status() == 5    # FS_ERR_DEVICE_TIMEOUT, kept until read
+    assert binding.fs_noalloc_status() == 0
+    again = binding.fs_sample_noalloc(H, W, temperature=0.9, seed=5, step=1)
+    torch.cuda.synchronize()
+    assert torch.equal(again, ref)
+    assert binding.fs_noalloc_status() == 0
