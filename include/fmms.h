@@ -77,7 +77,9 @@ typedef enum {
   FS_ERR_UNSUPPORTED = 2,    /* no sm_100 device, or a shape outside the supported range */
   FS_ERR_CUDA = 3,           /* a CUDA runtime/driver call or a launch failed */
   FS_ERR_WORKSPACE = 4,      /* the workspace is too small or misaligned */
-  FS_ERR_DEVICE_TIMEOUT = 5  /* a kernel gave up on a bounded wait (see fs_device_status) */
+  FS_ERR_DEVICE_TIMEOUT = 5, /* a kernel gave up on a bounded wait (see fs_device_status) */
+  FS_ERR_DEVICE_BOUNDS = 6   /* debug build only: a device-side bounds check failed and the
+                                access was skipped (see fs_device_status) */
 } fs_status;
 
 /* A cudaStream_t, passed without the CUDA headers. */

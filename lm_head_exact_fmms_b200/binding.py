@@ -11,11 +11,14 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-_LIB_PATH = os.path.join(_HERE, "libfmms.so")
+# FMMS_LIBRARY=debug selects the debug build (device-side bounds checks that
+# report FS_ERR_DEVICE_BOUNDS through fs_device_status).
+_LIB_PATH = os.path.join(_HERE, "libfmms_debug.so" if os.environ.get("FMMS_LIBRARY") == "debug"
+                         else "libfmms.so")
 
 FS_OK = 0
 _STATUS = {0: "FS_OK", 1: "FS_ERR_INVALID_ARG", 2: "FS_ERR_UNSUPPORTED", 3: "FS_ERR_CUDA",
-           4: "FS_ERR_WORKSPACE", 5: "FS_ERR_DEVICE_TIMEOUT"}
+           4: "FS_ERR_WORKSPACE", 5: "FS_ERR_DEVICE_TIMEOUT", 6: "FS_ERR_DEVICE_BOUNDS"}
 
 # Every symbol include/fmms.h declares.
 EXPORTED = ("fs_sample", "fs_sample_ex", "fs_sample_grouped", "fs_sample_unfused",

@@ -420,6 +420,17 @@ fs_status run_locked(int mode, const void *H, const void *W, int B, int d, int V
     p.tp_seq = shard.tp_seq;
     for (int r = 0; r < shard.tp_world; ++r)
       p.tp_area[r] = static_cast<fmms::TpArea *>(shard.tp_areas[r]);
+    {
+      const long long rows = fmms::imin(B, fmms::kMaxBN);
+      p.rows_total = B;
+      p.keys_cap = grouped ? fmms::kWsKeysRegion / 8 : S * fmms::kMaxBN;
+      p.partials_cap = fmms::ws_partials_bytes(B, sch.G, sch.num_ctas) /
+                       static_cast<long long>(sizeof(fmms::GroupPartial));
+      p.gkeys_cap = fmms::ws_gkeys_bytes(B, sch.G) / 8;
+      p.out_cap = Bc * S;
+      p.logits_cap = static_cast<long long>(Bc) * V;
+      (void)rows;
+    }
     const int pair_units_used = pair ? fmms::make_schedule(V, sch.G, units).num_ctas : 0;
     if (pair) {
       p.num_ctas = 2 * pair_units_used;
@@ -446,6 +457,10 @@ fs_status run_locked(int mode, const void *H, const void *W, int B, int d, int V
       m.step = step;
       m.out_idx = out_idx ? out_idx + b0 : nullptr;
       m.summary = summary ? static_cast<void *>(summary + static_cast<size_t>(b0) * sch.G) : nullptr;
+      m.err = w.err;
+      m.partials_cap = p.partials_cap;
+      m.gkeys_cap = p.gkeys_cap;
+      m.rows_total = B;
       if (fmms::launch_group_merge(m, stream) != cudaSuccess) return FS_ERR_CUDA;
     } else if (mode == fmms::kModeLogits) {
       fmms::SampleLogitsParams sp;
@@ -463,6 +478,8 @@ fs_status run_locked(int mode, const void *H, const void *W, int B, int d, int V
       sp.ticket = w.ticket;
       sp.out_idx = out_idx + b0;
       sp.num_sms = st->sms;
+      sp.err = w.err;
+      sp.rows_total = B;
       cudaError_t e;
       if (shard.top_k > 0) {
         s = grow(&st->topk_scratch, &st->topk_scratch_bytes,
@@ -873,7 +890,7 @@ fs_status fs_device_status(void *workspace, size_t workspace_bytes, fs_stream_t 
   if (cudaMemcpy(&err, ws, sizeof err, cudaMemcpyDeviceToHost) != cudaSuccess) return FS_ERR_CUDA;
   if (err == 0) return FS_OK;
   if (cudaMemset(ws, 0, bytes) != cudaSuccess) return FS_ERR_CUDA;
-  return FS_ERR_DEVICE_TIMEOUT;
+  return err == fmms::kErrBounds ? FS_ERR_DEVICE_BOUNDS : FS_ERR_DEVICE_TIMEOUT;
 }
 
 const char *fs_status_string(fs_status status) {
@@ -884,6 +901,7 @@ const char *fs_status_string(fs_status status) {
     case FS_ERR_CUDA: return "FS_ERR_CUDA";
     case FS_ERR_WORKSPACE: return "FS_ERR_WORKSPACE";
     case FS_ERR_DEVICE_TIMEOUT: return "FS_ERR_DEVICE_TIMEOUT";
+    case FS_ERR_DEVICE_BOUNDS: return "FS_ERR_DEVICE_BOUNDS";
   }
   return "FS_ERR_UNKNOWN";
 }
@@ -1067,5 +1085,5 @@ extern "C" fs_status fs_noalloc_status(fs_stream_t stream) {
     return FS_ERR_CUDA;
   if (err == 0) return FS_OK;
   if (cudaMemset(scratch, 0, kNoAllocScratchBytes) != cudaSuccess) return FS_ERR_CUDA;
-  return FS_ERR_DEVICE_TIMEOUT;
+  return err == fmms::kErrBounds ? FS_ERR_DEVICE_BOUNDS : FS_ERR_DEVICE_TIMEOUT;
 }

@@ -57,7 +57,8 @@ __global__ void __launch_bounds__(128) group_merge_kernel(const MergeParams m) {
   sch.ngran = m.ngran;
   sch.tile_rows = kTileM;
   const uint32_t bg = static_cast<uint32_t>(m.b_off + b);
-  const uint64_t k64 = m.row_seeds ? m.row_seeds[bg] : m.seed;
+  const uint64_t k64 =
+      (m.row_seeds && FS_IN_BOUNDS(m.err, bg, m.rows_total)) ? m.row_seeds[bg] : m.seed;
   fs_group_summary *summary = static_cast<fs_group_summary *>(m.summary);
 
   float best_key = -INFINITY;
@@ -82,8 +83,12 @@ __global__ void __launch_bounds__(128) group_merge_kernel(const MergeParams m) {
     for (int i0 = 0; i0 < nslots; i0 += 8) {
       GroupPartial gp[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
-        if (i0 + j < nslots) gp[j] = m.partials[slot_of(i0 + j) * m.B + b];
+      for (int j = 0; j < 8; ++j) {
+        gp[j] = GroupPartial{0ull, -INFINITY, 0.f};
+        if (i0 + j < nslots &&
+            FS_IN_BOUNDS(m.err, static_cast<long long>(slot_of(i0 + j)) * m.B + b, m.partials_cap))
+          gp[j] = m.partials[slot_of(i0 + j) * m.B + b];
+      }
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         if (i0 + j >= nslots) break;
@@ -101,8 +106,11 @@ __global__ void __launch_bounds__(128) group_merge_kernel(const MergeParams m) {
       }
     }
     for (int i = 0; i < nslots; ++i)  // leave the workspace zeroed
-      m.partials[slot_of(i) * m.B + b] = GroupPartial{0ull, 0.f, 0.f};
-    if (m.gkeys != nullptr) m.gkeys[static_cast<size_t>(g) * m.B + b] = 0ull;  // left zeroed
+      if (FS_IN_BOUNDS(m.err, static_cast<long long>(slot_of(i)) * m.B + b, m.partials_cap))
+        m.partials[slot_of(i) * m.B + b] = GroupPartial{0ull, 0.f, 0.f};
+    if (m.gkeys != nullptr &&
+        FS_IN_BOUNDS(m.err, static_cast<long long>(g) * m.B + b, m.gkeys_cap))
+      m.gkeys[static_cast<size_t>(g) * m.B + b] = 0ull;  // left zeroed
     const float lse = (M == -INFINITY) ? -INFINITY : M + logf(S);
     if (summary != nullptr) {
       fs_group_summary gs;
@@ -200,7 +208,8 @@ __global__ void __launch_bounds__(256) sample_logits_kernel(const SampleLogitsPa
   sm100::grid_dependency_wait();  // the logits
   const int b = blockIdx.y;
   const uint32_t bg = static_cast<uint32_t>(s.b_off + b);
-  const uint64_t k64 = s.row_seeds ? s.row_seeds[bg] : s.seed;
+  const uint64_t k64 =
+      (s.row_seeds && FS_IN_BOUNDS(s.err, bg, s.rows_total)) ? s.row_seeds[bg] : s.seed;
   const float *row = s.logits + static_cast<size_t>(b) * s.V;
   const int nquads = (s.V + 3) / 4;
   const bool vec = (s.V & 3) == 0;
@@ -222,7 +231,9 @@ __global__ void __launch_bounds__(256) sample_logits_kernel(const SampleLogitsPa
       for (int m = 0; m < 4; ++m) l[m] = (v0 + m < s.V) ? row[v0 + m] : 0.f;
     }
     uint32_t mword = 0xFFFFFFFFu;
-    if (s.mask) mword = s.mask[static_cast<size_t>(bg) * s.mask_words + (v0 >> 5)];
+    if (s.mask && FS_IN_BOUNDS(s.err, bg, s.rows_total) &&
+        FS_IN_BOUNDS(s.err, v0 >> 5, s.mask_words))
+      mword = s.mask[static_cast<size_t>(bg) * s.mask_words + (v0 >> 5)];
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
       const int v = v0 + m;
@@ -244,7 +255,8 @@ __global__ void __launch_bounds__(256) sample_logits_kernel(const SampleLogitsPa
   if (threadIdx.x == 0) {
     uint64_t r = 0ull;
     for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) r = warp_best[i] > r ? warp_best[i] : r;
-    if (key_valid(r)) atomicMax(s.keys + b, static_cast<unsigned long long>(r));
+    if (key_valid(r) && FS_IN_BOUNDS(s.err, b, kMaxBN))
+      atomicMax(s.keys + b, static_cast<unsigned long long>(r));
     __threadfence();
     const unsigned total = gridDim.x * gridDim.y;
     is_last = (atomicAdd(s.ticket, 1u) == total - 1) ? 1 : 0;
@@ -253,7 +265,7 @@ __global__ void __launch_bounds__(256) sample_logits_kernel(const SampleLogitsPa
   if (is_last) {
     __threadfence();
     for (int r = threadIdx.x; r < s.B; r += blockDim.x)
-      s.out_idx[r] = key_token(atomicExch(s.keys + r, 0ull));
+      if (FS_IN_BOUNDS(s.err, r, kMaxBN)) s.out_idx[r] = key_token(atomicExch(s.keys + r, 0ull));
     if (threadIdx.x == 0) atomicExch(s.ticket, 0u);
   }
 }
@@ -438,7 +450,8 @@ __device__ __forceinline__ uint32_t topk_load(const SampleLogitsParams &s, const
     }
   }
   if (s.mask != nullptr && v0 < hi)  // 16 tokens from a multiple of 16 lie in one mask word
-    okm &= s.mask[static_cast<size_t>(bg) * s.mask_words + (v0 >> 5)] >> (v0 & 31);
+    if (FS_IN_BOUNDS(s.err, bg, s.rows_total) && FS_IN_BOUNDS(s.err, v0 >> 5, s.mask_words))
+      okm &= s.mask[static_cast<size_t>(bg) * s.mask_words + (v0 >> 5)] >> (v0 & 31);
 #pragma unroll
   for (int i = 0; i < kTopkItems; ++i) key[i] = order_bits(key[i]);
   return okm;
@@ -805,7 +818,8 @@ __global__ void __launch_bounds__(kTopkThreads) topk_row_kernel(const TopkArgs a
     }
   }
 
-  const uint64_t k64 = s.row_seeds ? s.row_seeds[bg] : s.seed;
+  const uint64_t k64 =
+      (s.row_seeds && FS_IN_BOUNDS(s.err, bg, s.rows_total)) ? s.row_seeds[bg] : s.seed;
   uint64_t best = 0ull;
   // Ranking: G consecutive lanes share an entry (G = 1024 / n rounded down to
   // a power of two, at most 32), each counting over every G-th entry.

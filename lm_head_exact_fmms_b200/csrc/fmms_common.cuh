@@ -33,6 +33,26 @@ FS_HD int imin(int a, int b) { return a < b ? a : b; }
 FS_HD int imax(int a, int b) { return a > b ? a : b; }
 
 // ---------------------------------------------------------------------------
+// Debug build (compiled with -DFS_DEBUG, libfmms_debug.so): device-side bounds
+// checks on the kernels' global, shared and tensor memory indices.  A check
+// that fails records kErrBounds in the call's status word (the first error
+// recorded wins) and the access is skipped; nothing traps, so the context
+// stays usable and the host reads the error with fs_device_status.  In the
+// release build every check is the constant true and compiles away.
+// ---------------------------------------------------------------------------
+constexpr int kErrBounds = 6;
+#if defined(FS_DEBUG) && defined(__CUDACC__)
+__device__ __forceinline__ bool dbg_in_bounds(int *err, long long i, long long n) {
+  if (i >= 0 && i < n) return true;
+  if (err != nullptr) atomicCAS(err, 0, kErrBounds);
+  return false;
+}
+#define FS_IN_BOUNDS(err, i, n) ::fmms::dbg_in_bounds((err), (long long)(i), (long long)(n))
+#else
+#define FS_IN_BOUNDS(err, i, n) true
+#endif
+
+// ---------------------------------------------------------------------------
 // Split-V schedule.  The vocabulary is cut into ceil(V/8) granules; CTA c of
 // num_ctas owns granules [floor(c n / C), floor((c+1) n / C)), so every CTA
 // streams the same number of W rows to within one granule.  Group g of G
@@ -266,6 +286,16 @@ struct FmmsParams {
   int tp_world;
   uint32_t tp_seq;
   TpArea *tp_area[kMaxTpWorld];
+  // Extents the debug build's bounds checks compare against (entries, not
+  // bytes): rows of row_seeds and mask (the whole call), packed keys in the
+  // workspace, partial records and published group maxima, and tokens (or
+  // keys) and logits this launch may write.
+  int rows_total;
+  int keys_cap;
+  long long partials_cap;
+  long long gkeys_cap;
+  int out_cap;
+  long long logits_cap;
 };
 
 // Workspace layout (bytes), fixed so that calls of different kinds can share

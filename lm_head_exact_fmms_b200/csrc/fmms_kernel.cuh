@@ -245,7 +245,8 @@ __device__ __forceinline__ void chunk_noise(const FmmsParams &p, int v, int col0
     const int colp = col0 + 4 * q4 + (lane & 3);  // column of this lane's Philox call
     const uint32_t bg = static_cast<uint32_t>(p.b_off + colp);
     uint64_t k64 = p.seed;
-    if (p.row_seeds != nullptr && colp < p.B) k64 = __ldg(p.row_seeds + bg);
+    if (p.row_seeds != nullptr && colp < p.B && FS_IN_BOUNDS(p.err, bg, p.rows_total))
+      k64 = __ldg(p.row_seeds + bg);
     const Philox4 ph = philox4x32_10(static_cast<uint32_t>(v) >> 2, bg, p.step, tag,
                                      static_cast<uint32_t>(k64), static_cast<uint32_t>(k64 >> 32));
     uint32_t w[4] = {ph.w0, ph.w1, ph.w2, ph.w3};
@@ -282,7 +283,7 @@ __device__ __forceinline__ uint32_t chunk_allowed(const FmmsParams &p, int v, bo
   if (p.mask == nullptr) return v_ok ? in_range : 0u;
   const int v0 = v - lane;  // token of lane 0 (a multiple of 8)
   uint32_t rowbits = 0u;
-  if (lane < CW && lane < n) {
+  if (lane < CW && lane < n && FS_IN_BOUNDS(p.err, p.b_off + col0 + lane, p.rows_total)) {
     const uint32_t *row = p.mask + static_cast<size_t>(p.b_off + col0 + lane) * p.mask_words;
     const int w0 = v0 >> 5;
     const int sh = v0 & 31;
@@ -481,8 +482,8 @@ __device__ __forceinline__ void issue_h(const CUtensorMap *th, const FmmsParams 
 
 // TMA producer (one thread).  In pair mode both CTAs load their own half of
 // every stage (128 W rows, BN/2 H rows) and count the bytes on the even
-// CTA's full barrier; the even CTA also hands each freed stage on to the odd
-// CTA, whose MMA reads happen in the even CTA's tcgen05 pipeline.
+// CTA's full barrier; a freed stage is signalled to both CTAs by the even
+// CTA's MMA commit (multicast to the pair).
 template <int BN, int MODE, bool PAIR, bool MERGE = false>
 __device__ __forceinline__ void role_producer(const CUtensorMap *tw, const PartMaps *twp,
                                               const CUtensorMap *th, const FmmsParams &p,
@@ -535,8 +536,6 @@ __device__ __forceinline__ void role_producer(const CUtensorMap *tw, const PartM
         ok = false;
         break;
       }
-      if (PAIR && rank == 0 && issued >= C::kStages)
-        sm100::mbar_arrive_cluster(sm100::cluster_addr(&empty[stage], 1));
       uint8_t *sp0 = stages + stage * C::kStageBytes;
       uint8_t *sw0 = sp0 + C::kOffW;
       if (!PAIR || rank == 0) sm100::mbar_arrive_expect_tx(&full[stage], bytes);
@@ -658,6 +657,8 @@ __device__ __forceinline__ void role_mma(const FmmsParams &p, const Schedule &sc
   int buf = 0;
   uint32_t acc_phase = 0;
   bool ok = true;
+  const uint32_t stage_lo = sm100::desc_lo(sm100::smem_addr(stages));
+  const uint32_t desc_hi = sm100::kDescHi;
   while (ok && it.next(tile)) {
     // A merged partial takes the next accumulator too.
     const bool merged = C::kMerge && tile.pstart >= 0;
@@ -677,21 +678,36 @@ __device__ __forceinline__ void role_mma(const FmmsParams &p, const Schedule &sc
       }
       sm100::tc_fence_after();
       const int nsub = imin(C::kSub, p.nk - ks * C::kSub);
-      const uint32_t p_addr = sm100::smem_addr(stages + stage * C::kStageBytes);
-      const uint32_t a_addr = p_addr + C::kOffW;
-      const uint32_t b_addr = p_addr + C::kOffH;
+      // Descriptor low words of this stage's operands; each MMA below adds a
+      // compile-time offset (in 16-byte units) to them.
+      const uint32_t p_lo = stage_lo + static_cast<uint32_t>(stage * (C::kStageBytes >> 4));
+      const uint32_t a_lo = p_lo + (C::kOffW >> 4);
+      const uint32_t b_lo = p_lo + (C::kOffH >> 4);
+      if (nsub == C::kSub) {
+        // A full stage: every K step unrolled, only the tile's first MMA
+        // overwrites the accumulator.
 #pragma unroll
-      for (int j = 0; j < C::kSub; ++j) {
-        if (j >= nsub) break;
+        for (int j = 0; j < C::kSub; ++j) {
 #pragma unroll
-        for (int kk = 0; kk < kBlockK / 16; ++kk) {
-          const uint64_t da = sm100::smem_desc_sw128(a_addr + j * C::kSubW + kk * 32);
-          const uint64_t db = sm100::smem_desc_sw128(b_addr + j * C::kSubH + kk * 32);
-          const uint32_t acc = (ks | j | kk) != 0 ? 1u : 0u;
-          if constexpr (PAIR) {
-            sm100::mma_bf16_ss_pair(d_tmem, da, db, C::kIdesc, acc);
-          } else {
-            sm100::mma_bf16_ss(d_tmem, da, db, C::kIdesc, acc);
+          for (int kk = 0; kk < kBlockK / 16; ++kk) {
+            const uint32_t acc = (j | kk) != 0 ? 1u : (ks != 0 ? 1u : 0u);
+            sm100::mma_bf16_lo<PAIR>(d_tmem, a_lo + ((j * C::kSubW + kk * 32) >> 4),
+                                     b_lo + ((j * C::kSubH + kk * 32) >> 4), desc_hi, C::kIdesc,
+                                     acc);
+          }
+        }
+      } else {
+        // The tile's last stage, partly filled when d is not a multiple of
+        // the stage's K extent.
+#pragma unroll
+        for (int j = 0; j < C::kSub; ++j) {
+          if (j >= nsub) break;
+#pragma unroll
+          for (int kk = 0; kk < kBlockK / 16; ++kk) {
+            const uint32_t acc = (ks | j | kk) != 0 ? 1u : 0u;
+            sm100::mma_bf16_lo<PAIR>(d_tmem, a_lo + ((j * C::kSubW + kk * 32) >> 4),
+                                     b_lo + ((j * C::kSubH + kk * 32) >> 4), desc_hi, C::kIdesc,
+                                     acc);
           }
         }
       }
@@ -705,16 +721,16 @@ __device__ __forceinline__ void role_mma(const FmmsParams &p, const Schedule &sc
             if (j >= nsub) break;
 #pragma unroll
             for (int kk = 0; kk < kBlockK / 16; ++kk) {
-              const uint64_t dp = sm100::smem_desc_sw128(p_addr + j * C::kSubP + kk * 32);
-              const uint64_t db = sm100::smem_desc_sw128(b_addr + j * C::kSubH + kk * 32);
-              sm100::mma_bf16_ss(d_tmem2, dp, db, C::kIdesc, (ks | j | kk) != 0 ? 1u : 0u);
+              sm100::mma_bf16_lo<false>(d_tmem2, p_lo + ((j * C::kSubP + kk * 32) >> 4),
+                                        b_lo + ((j * C::kSubH + kk * 32) >> 4), desc_hi,
+                                        C::kIdesc, (ks | j | kk) != 0 ? 1u : 0u);
             }
           }
         }
       }
-      // Frees the stage once these MMAs finish.
+      // Frees the stage (in both CTAs of a pair) once these MMAs finish.
       if constexpr (PAIR) {
-        sm100::mma_commit_pair(&empty[stage]);
+        sm100::mma_commit_pair_both(&empty[stage]);
       } else {
         sm100::mma_commit(&empty[stage]);
       }
@@ -724,9 +740,9 @@ __device__ __forceinline__ void role_mma(const FmmsParams &p, const Schedule &sc
       }
     }
     if (!ok) break;
-    // Accumulator ready for the epilogue.
+    // Accumulator ready for the epilogue (of both CTAs of a pair).
     if constexpr (PAIR) {
-      sm100::mma_commit_pair(&acc_full[buf]);
+      sm100::mma_commit_pair_both(&acc_full[buf]);
     } else {
       sm100::mma_commit(&acc_full[buf]);
       if (merged) sm100::mma_commit(&acc_full[buf2]);
@@ -750,9 +766,9 @@ __device__ __forceinline__ void role_mma(const FmmsParams &p, const Schedule &sc
 }
 
 // Epilogue warps.  In pair mode each CTA drains its own 128 accumulator rows
-// (its half of the pair tile); the even CTA hands every filled accumulator on
-// to the odd CTA, and the odd CTA's warps release it on the even CTA's
-// barrier, where the MMAs are issued.
+// (its half of the pair tile); the even CTA's MMA commit signals a filled
+// accumulator to both CTAs, and the odd CTA's warps release it on the even
+// CTA's barrier, where the MMAs are issued.
 template <int BN, int MODE, bool PAIR, bool MERGE = false>
 __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedule &sch,
                                               uint32_t tmem_base, uint64_t *acc_full,
@@ -794,8 +810,6 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
     const bool got = aborted ? false : sm100::wait_bounded<PAIR>(&acc_full[buf], phase, abort_flag, p.err);
     aborted = __any_sync(0xffffffffu, !got);
     if (!aborted) {
-      if (PAIR && rank == 0 && warp == 2 && lane == 0)
-        sm100::mbar_arrive_cluster(sm100::cluster_addr(&acc_full[buf], 1));
       sm100::tc_fence_after();
       const Tile mine = PAIR ? pair_half(cur, rank) : cur;
       const int v = mine.start + 32 * q + lane;           // row of W in this launch
@@ -810,6 +824,7 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
         const int col0 = k * CW;
         if (col0 >= p.B) continue;  // warp-uniform
         uint32_t acc[CW];
+        if (!FS_IN_BOUNDS(p.err, buf * BN + col0 + CW - 1, C::kTmemCols)) continue;  // warp-uniform
         if constexpr (CW == 32) {
           sm100::tmem_ld_32(tbase + col0, acc);
         } else {
@@ -822,7 +837,9 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
             const int ncol = imin(CW, p.B - col0);
 #pragma unroll
             for (int j = 0; j < CW; ++j) {
-              if (j < ncol) *dst = __uint_as_float(acc[j]);
+              if (j < ncol &&
+                  FS_IN_BOUNDS(p.err, static_cast<long long>(col0 + j) * p.V + v, p.logits_cap))
+                *dst = __uint_as_float(acc[j]);
               dst += p.V;
             }
           }
@@ -839,7 +856,8 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
 #pragma unroll 1
             for (int smp = 0; smp < p.num_samples; ++smp) {
               unsigned long long *kp = p.keys + smp * kMaxBN + c;
-              const uint64_t pub = c < p.B ? ld_key(kp) : 0ull;  // in flight during Philox
+              const bool kin = c < p.B && FS_IN_BOUNDS(p.err, smp * kMaxBN + c, p.keys_cap);
+              const uint64_t pub = kin ? ld_key(kp) : 0ull;  // in flight during Philox
               uint32_t words[CW];
               chunk_noise<CW>(p, vg, col0, lane, 2u * static_cast<uint32_t>(smp), words);
               if (chunk_any_candidate<CW>(acc, words, p, in_range, 0ull, pub, lane)) {
@@ -849,18 +867,20 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
                 }
                 uint64_t cbest = 0ull;
                 chunk_keys<CW>(acc, words, p, vg, allowed, lane, cbest);
-                if ((lane & 1) == 0 && c < p.B && key_valid(cbest) && cbest > pub)
+                if ((lane & 1) == 0 && kin && key_valid(cbest) && cbest > pub)
                   atomicMax(kp, static_cast<unsigned long long>(cbest));
               }
             }
           } else {
+            const long long gki = static_cast<long long>(tile.slot - unit) * p.B + c;
             unsigned long long *gk =
-                p.gkeys ? p.gkeys + static_cast<size_t>(tile.slot - unit) * p.B + c : nullptr;
+                (p.gkeys && (c >= p.B || FS_IN_BOUNDS(p.err, gki, p.gkeys_cap))) ? p.gkeys + gki
+                                                                              : nullptr;
             const uint64_t pub = (gk != nullptr && c < p.B) ? ld_key(gk) : 0ull;
             const uint32_t allowed = chunk_allowed<CW>(p, vg, v_ok, col0, lane);
             uint32_t words[CW];
             chunk_noise<CW>(p, vg, col0, lane, 0u, words);
-            const int si = q * BN + c;  // this lane's (quarter, column) state
+            const int si = FS_IN_BOUNDS(p.err, q * BN + c, 4 * BN) ? q * BN + c : 0;  // this lane's (quarter, column) state
             float m_run = comb_m[si], s_run = comb_s[si];
             uint64_t best = comb_key[si];
             chunk_lse2<CW>(acc, c1, allowed, comb_m + q * BN + col0, lane, m_run, s_run);
@@ -917,7 +937,8 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
             comb_m[qq * BN + b] = -INFINITY;
             comb_s[qq * BN + b] = 0.f;
           }
-          if (b < p.B && !*abort_flag) {
+          if (b < p.B && !*abort_flag &&
+              FS_IN_BOUNDS(p.err, static_cast<long long>(slot) * p.B + b, p.partials_cap)) {
             GroupPartial gp;
             gp.key = kb;
             gp.m = m * 0.69314718055994531f;  // base-2 maximum back to natural units
@@ -961,6 +982,9 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
       for (int i = etid; i < total; i += kEpiThreads) {
         const int b = i / p.num_samples;
         const int smp = i - b * p.num_samples;
+        if (!FS_IN_BOUNDS(p.err, smp * kMaxBN + b, p.keys_cap) ||
+            !FS_IN_BOUNDS(p.err, i, p.out_cap))
+          continue;
         const unsigned long long kb = atomicExch(p.keys + smp * kMaxBN + b, 0ull);
         if (p.out_keys != nullptr)
           p.out_keys[i] = static_cast<long long>(kb ^ 0x8000000000000000ull);  // signed order

@@ -58,6 +58,11 @@ struct MergeParams {
   uint32_t step;
   int32_t *out_idx;              // [B], offset to this launch
   void *summary;                 // fs_group_summary [B][G] offset to this launch, or null
+  // Debug-build bounds checks (entries): the status word, the partial records
+  // and published maxima in the workspace, rows of row_seeds.
+  int *err;
+  long long partials_cap, gkeys_cap;
+  int rows_total;
 };
 cudaError_t launch_group_merge(const MergeParams &m, cudaStream_t stream);
 
@@ -75,6 +80,8 @@ struct SampleLogitsParams {
   unsigned int *ticket;
   int32_t *out_idx;
   int num_sms;
+  int *err;                      // status word (debug-build bounds checks)
+  int rows_total;                // rows of row_seeds and mask (the whole call)
 };
 cudaError_t launch_sample_logits(const SampleLogitsParams &s, cudaStream_t stream);
 

@@ -253,6 +253,43 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
   return desc;
 }
 
+// The same descriptor as two 32-bit words: the low word holds the start
+// address >> 4 (bits 0-13) and the leading byte offset (16-29); the high word
+// (stride byte offset, version, layout) is the same for every operand here.
+// The MMA loop computes each stage's low words once and adds compile-time
+// offsets per K step, so one tcgen05.mma costs the issuing thread two adds.
+constexpr uint32_t kDescHi = (1024u >> 4) | (1u << 14) | (2u << 29);
+__device__ __forceinline__ uint32_t desc_lo(uint32_t saddr) {
+  return ((saddr >> 4) & 0x3FFFu) | (1u << 16);
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, bf16 inputs, fp32 accumulate, with the
+// operands given as descriptor low words and the shared high word;
+// cta_group::2 when PAIR (issued by the even CTA of the pair).
+template <bool PAIR>
+__device__ __forceinline__ void mma_bf16_lo(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo,
+                                            uint32_t hi, uint32_t idesc, uint32_t accumulate) {
+  if constexpr (PAIR) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+        "mov.b64 da, {%1, %3};\n\t"
+        "mov.b64 db, {%2, %3};\n\t"
+        "setp.ne.b32 p, %5, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], da, db, %4, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_lo), "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+        "mov.b64 da, {%1, %3};\n\t"
+        "mov.b64 db, {%2, %3};\n\t"
+        "setp.ne.b32 p, %5, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %4, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_lo), "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate)
+        : "memory");
+  }
+}
+
 // Instruction descriptor of kind::f16 with bf16 A and B (both K-major) and an
 // fp32 accumulator:
 //   bits 4-5 D format (1 = f32), 7-9 A format (1 = bf16), 10-12 B format
@@ -289,14 +326,14 @@ __device__ __forceinline__ void cluster_sync() {
 }
 
 // One arrival on an mbarrier of another CTA of the cluster, with relaxed
-// semantics.  Every such arrival in the pair kernel reports the completion
-// of asynchronous work that the arriving thread has already observed (an MMA
-// commit seen through an acquire wait, or tensor-memory loads finished by
-// tcgen05.wait::ld); no ordinary memory write of the arriving thread has to
-// become visible to the other CTA.  A release at cluster scope is not needed,
-// and it is costly here: it stalls the issuing thread while that thread's
-// TMA loads are in flight (about a microsecond per pipeline stage, measured),
-// which halved the pair kernel's streaming rate.
+// semantics.  The pair kernel's one such arrival (the odd CTA's epilogue
+// releasing an accumulator on the even CTA's barrier) reports tensor-memory
+// loads already finished by tcgen05.wait::ld; no ordinary memory write of
+// the arriving thread has to become visible to the other CTA.  A release at
+// cluster scope is not needed, and it is costly: used for the stage hand-off
+// an earlier version of the kernel made this way, it stalled the issuing
+// thread while its TMA loads were in flight (about a microsecond per
+// pipeline stage, measured), which halved the pair kernel's streaming rate.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
   asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar)
                : "memory");
@@ -355,6 +392,20 @@ __device__ __forceinline__ void mma_commit_pair(uint64_t *bar) {
   asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                    smem_addr(bar))
                : "memory");
+}
+
+// Arrives once on `bar` in BOTH CTAs of the pair (the same shared-memory
+// offset in each) when every pair MMA this thread issued so far has
+// completed.  Used for the stage and accumulator barriers that both CTAs
+// wait on, so the odd CTA hears of a freed stage or a filled accumulator
+// straight from the tensor cores instead of through the even CTA's threads.
+__device__ __forceinline__ void mma_commit_pair_both(uint64_t *bar) {
+  const uint16_t cta_mask = 3;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(smem_addr(bar)),
+      "h"(cta_mask)
+      : "memory");
 }
 
 // Programmatic dependent launch: a kernel launched with the

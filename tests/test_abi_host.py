@@ -337,3 +337,16 @@ def test_c_program_links_and_calls_the_abi(lib):
     assert lines["merged"].split() == [str(len(merged)), str(int(merges)), str(merged[0][5])]
     assert int(lines["area"]) == binding.fs_tp_area_bytes()
     assert lines["status"] == "1 FS_ERR_INVALID_ARG"
+
+
+def test_debug_build_exports_the_same_symbols():
+    """libfmms_debug.so (device-side bounds checks, selected with
+    FMMS_LIBRARY=debug) exports every symbol the header declares."""
+    from lm_head_exact_fmms_b200 import build
+    path = build.build(debug=True)
+    dbg = ctypes.CDLL(path)
+    for name in declared_functions():
+        assert hasattr(dbg, name), name
+    assert dbg.fs_status_string is not None
+    dbg.fs_status_string.restype = ctypes.c_char_p
+    assert dbg.fs_status_string(6) == b"FS_ERR_DEVICE_BOUNDS"
