@@ -505,6 +505,8 @@ def run_gpu(args, world, rank, local):
         with nvtx("fmms: batch sweep"):
             result["sweep"] = sweep(torch, binding, synth, W, wl, dev, stream, peaks, peak_kind,
                                     compare_single=True)
+        with nvtx("fmms: library GEMM for context"):
+            result["library_gemm"] = library_gemm_points(torch, synth, W, wl, dev)
         with nvtx("fmms: sustained decode"):
             result["sustained"] = sustained_point(torch, binding, synth, W, wl, dev, stream, peaks,
                                                   peak_kind, local)
@@ -579,6 +581,20 @@ def sweep(torch, binding, synth, W, wl, dev, stream, peaks, peak_kind, steps=200
             row["single_cta_kernel_us"] = round(sum(per1) / len(per1), 3)
         rows.append(row)
     return rows
+
+
+def library_gemm_points(torch, synth, W, wl, dev, batches=(64, 128, 256), steps=100):
+    """For context only: the logits GEMM alone, H W^T in bf16 through torch
+    (cuBLAS), which writes B x V bf16 logits and samples nothing."""
+    rows = []
+    for B in batches:
+        H = synth.make_hidden(B, wl.d, device=dev)
+        out = torch.empty(B, wl.V, dtype=torch.bfloat16, device=dev)
+        region_ms, _ = time_calls(lambda i: torch.matmul(H, W.t(), out=out), steps, 10,
+                                  torch.cuda.current_stream())
+        rows.append({"B": B, "us_per_call": round(region_ms * 1e3 / steps, 3)})
+    return {"what": "torch.matmul(H, W.T) bf16 -> bf16 logits [B, V] (cuBLAS), no sampling",
+            "points": rows}
 
 
 def sustained_point(torch, binding, synth, W, wl, dev, stream, peaks, peak_kind, local, B=64,

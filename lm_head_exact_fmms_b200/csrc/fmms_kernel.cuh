@@ -67,21 +67,29 @@ constexpr int kSmemBudget = 232448 - 1024 - 256;
 // sub-blocks per stage win (fewer handshakes per byte, 128 B more of each W
 // row per sub-block).  So: among 1..4 sub-blocks with at least three stages
 // (at most ten), the most W bytes in flight, ties to more sub-blocks.
-// E.g. single CTAs: 4 x 3 stages at 16 batch rows, 2 x 5 at 32, 3 x 3 at 64;
-// CTA pairs: 3 x 3 at 128 rows (64 H rows per CTA), 1 x 7 at 256.
+// E.g. single CTAs: 4 x 3 stages at 16 batch rows, 2 x 5 at 32, 3 x 3 at 64.
+// CTA pairs at 224 rows and more run tensor-bound, where the MMAs of a stage
+// hold it longer and fewer, larger stages pay more: there a choice with one
+// sub-block less in flight still counts as a tie (`slack`), so 256 rows take
+// 2 x 3 instead of 1 x 7 (measured: B=256 on the Qwen3-8B head 322 -> 305 us,
+// on the d=8192 head 504 -> 483 us; 1 x 7 and 3 x 2 both slower).  Below 224
+// rows the plain rule measured best (pairs: 3 x 3 at 128 rows, 64 H rows per
+// CTA; 2 x 4 at 160 and 192).
 constexpr int kMaxStages = 10;
 constexpr int stages_for(int ksub, int h_rows, int comb_bytes, int p_bytes) {
   const int fit = (kSmemBudget - comb_bytes) / (ksub * ((kTileM + h_rows) * kBlockK * 2 + p_bytes));
   return fit < kMaxStages ? fit : kMaxStages;
 }
-constexpr int ksub_for(int h_rows, int comb_bytes, int p_bytes) {
-  int best = 1, best_bytes = 0;
+constexpr int ksub_for(int h_rows, int comb_bytes, int p_bytes, int slack = 0) {
+  int best_bytes = 0;
   for (int k = 1; k <= 4; ++k) {
     const int st = stages_for(k, h_rows, comb_bytes, p_bytes);
-    if (st >= 3 && st * k >= best_bytes) {
-      best = k;
-      best_bytes = st * k;
-    }
+    if (st >= 3 && st * k > best_bytes) best_bytes = st * k;
+  }
+  int best = 1;
+  for (int k = 1; k <= 4; ++k) {
+    const int st = stages_for(k, h_rows, comb_bytes, p_bytes);
+    if (st >= 3 && st * k >= best_bytes - slack) best = k;
   }
   return best;
 }
@@ -108,7 +116,8 @@ struct KCfg {
   // d=8192 head ran 3-4 % slower with it.
   static constexpr bool kMerge = MERGE && !PAIR && BN <= 64;
   static constexpr int kSubP = kMerge ? kGranule * kBlockK * 2 : 0;  // 1 KB per sub-block
-  static constexpr int kSub = ksub_for(kHRows, kCombBytes, kSubP);  // 64-wide K blocks per stage
+  static constexpr int kSub =
+      ksub_for(kHRows, kCombBytes, kSubP, PAIR && BN >= 224 ? 1 : 0);  // 64-wide K blocks per stage
   static constexpr int kSubW = kTileM * kBlockK * 2;    // 16 KB of W per sub-block
   static constexpr int kSubH = kHRows * kBlockK * 2;    // this CTA's H rows per sub-block
   static constexpr int kStageP = kSub * kSubP;
