@@ -446,6 +446,19 @@ fs_status fs_test_inject_fault(int kind, int *previous);
  * CTAs. */
 fs_status fs_set_cta_pairs(int policy);
 
+/* Whether the fused kernel is launched as a programmatic dependent of the
+ * kernel ahead of it in the stream (CUDA programmatic dependent launch):
+ * on (1, the default), for launches whose batch tile is at most 128 rows
+ * (where W streaming sets the time), back-to-back calls overlap, the next
+ * kernel's CTAs starting on the SMs the previous one has left and streaming
+ * W at once, while its loads of H and every access to the workspace wait
+ * until the previous kernel has completed (H may be that kernel's output);
+ * larger tiles, tensor-bound, run in plain order.  Off (0): plain stream
+ * order for every launch.  The tokens are the same either way (bit for bit).  A
+ * B200 scheduling choice, not part of the method.  Process-wide; applies to
+ * calls made after it returns.  FS_ERR_INVALID_ARG for any other value. */
+fs_status fs_set_programmatic_launch(int on);
+
 /* Kernel choice for single-CTA launches of up to 64 batch rows: a CTA whose
  * vocabulary range starts with an 8-row partial tile can either run it as a
  * tile of its own (which streams all of H again for 8 rows of W) or multiply

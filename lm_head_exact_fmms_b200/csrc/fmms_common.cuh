@@ -286,6 +286,9 @@ struct FmmsParams {
   int tp_world;
   uint32_t tp_seq;
   TpArea *tp_area[kMaxTpWorld];
+  // 1: launched as a programmatic dependent of the grid ahead in the stream
+  // (may start before it ends; H loads and workspace accesses wait for it).
+  int pdl;
   // Extents the debug build's bounds checks compare against (entries, not
   // bytes): rows of row_seeds and mask (the whole call), packed keys in the
   // workspace, partial records and published group maxima, and tokens (or

@@ -507,12 +507,31 @@ __device__ __forceinline__ void role_producer(const CUtensorMap *tw, const PartM
   int stage = 0;
   uint32_t phase = 0;
   long long issued = 0;
-  int h_chunks_ready = -1;  // chunks of H known to have arrived (h_ready mode)
-  // h_ready mode: stages whose W loads went out while the copy of H was still
-  // in flight; their H loads follow once it has landed, so the ring fills
-  // with W during the copy instead of stopping at the first stage.
+  // The H loads are gated in two cases: with a programmatic launch (p.pdl)
+  // until the grid ahead in the stream has completed (H may be its output),
+  // and in fs_sample_host (p.h_ready) until the copy of H from the host has
+  // landed.  While the gate is closed, a stage's W loads go out at once and
+  // its H loads are deferred as long as free stages remain, so the ring fills
+  // with W meanwhile instead of stopping at the first stage.
+  bool dep_pending = p.pdl != 0;
+  int h_chunks_ready =  // chunks of H known to be loadable
+      (p.h_ready != nullptr || dep_pending) ? -1 : 0x7FFFFFFF;
   int pend_stage[C::kStages], pend_sub0[C::kStages], pend_nsub[C::kStages];
   int npend = 0, pend_need = 0;
+  // Opens the gate up to H chunk `need`: false if the copy of H did not land
+  // within the wait limit.
+  auto open_gate = [&](int need) -> bool {
+    if (dep_pending) {
+      sm100::grid_dependency_wait();
+      dep_pending = false;
+    }
+    if (p.h_ready == nullptr) {
+      h_chunks_ready = 0x7FFFFFFF;
+      return true;
+    }
+    h_chunks_ready = need;
+    return sm100::wait_flag_bounded(p.h_ready + need, p.h_epoch, abort_flag, p.err);
+  };
   bool ok = p.test_no_loads == 0;
   while (ok && it.next(tile)) {
     const bool merged = C::kMerge && tile.pstart >= 0;
@@ -586,34 +605,32 @@ __device__ __forceinline__ void role_producer(const CUtensorMap *tw, const PartM
           }
         }
       }
-      // H still arriving from the host: until the chunk this stage ends in
-      // is known to have landed, defer the stage's H loads while free stages
-      // remain; then wait for it and issue every deferred H load.
+      // Gate closed for the chunk of H this stage ends in: defer the stage's
+      // H loads while free stages remain; then open it (wait) and issue every
+      // deferred H load.  (The grid dependency cannot be polled, so with
+      // p.pdl the gate opens once the ring is full or the CTA's stages end.)
       bool h_now = true;
-      if (p.h_ready != nullptr) {
-        const int need = (sub0 + nsub - 1) / p.h_chunk_subs;
-        if (need > h_chunks_ready) {
-          pend_stage[npend] = stage;
-          pend_sub0[npend] = sub0;
-          pend_nsub[npend] = nsub;
-          pend_need = need;
-          ++npend;
-          h_now = false;
-          if (npend == C::kStages || sm100::flag_is(p.h_ready + need, p.h_epoch)) {
-            const bool landed =
-                sm100::wait_flag_bounded(p.h_ready + need, p.h_epoch, abort_flag, p.err);
-            h_chunks_ready = need;
-            // After a timeout too: the loads stay in bounds, and completing
-            // the stages lets the drain below account for every copy.
-            for (int q = 0; q < npend; ++q)
-              issue_h<BN, MODE, PAIR, MERGE>(th, p, stages, full, pend_stage[q], pend_sub0[q],
-                                      pend_nsub[q], rank, pol_h);
-            npend = 0;
-            if (!landed) {
-              ok = false;
-              ++issued;
-              break;
-            }
+      const int need = p.h_ready != nullptr ? (sub0 + nsub - 1) / p.h_chunk_subs : 0;
+      if (need > h_chunks_ready) {
+        pend_stage[npend] = stage;
+        pend_sub0[npend] = sub0;
+        pend_nsub[npend] = nsub;
+        pend_need = need;
+        ++npend;
+        h_now = false;
+        if (npend == C::kStages ||
+            (!dep_pending && sm100::flag_is(p.h_ready + need, p.h_epoch))) {
+          const bool landed = open_gate(need);
+          // After a timeout too: the loads stay in bounds, and completing
+          // the stages lets the drain below account for every copy.
+          for (int q = 0; q < npend; ++q)
+            issue_h<BN, MODE, PAIR, MERGE>(th, p, stages, full, pend_stage[q], pend_sub0[q],
+                                           pend_nsub[q], rank, pol_h);
+          npend = 0;
+          if (!landed) {
+            ok = false;
+            ++issued;
+            break;
           }
         }
       }
@@ -627,7 +644,7 @@ __device__ __forceinline__ void role_producer(const CUtensorMap *tw, const PartM
   }
   if (ok && npend > 0) {
     // The CTA's last stages are still waiting for H (a range shorter than the ring).
-    const bool landed = sm100::wait_flag_bounded(p.h_ready + pend_need, p.h_epoch, abort_flag, p.err);
+    const bool landed = open_gate(pend_need);
     for (int q = 0; q < npend; ++q)
       issue_h<BN, MODE, PAIR, MERGE>(th, p, stages, full, pend_stage[q], pend_sub0[q], pend_nsub[q], rank,
                               pol_h);
@@ -792,6 +809,10 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
   const float c1 = p.inv_temp * 1.4426950408889634f;  // log2(e) / T: base-2 log-sum-exp
   const int etid = (warp - 2) * 32 + lane;
   const bool has_chunks = h < C::kChunks;
+  // A programmatic launch may start while the grid ahead in the stream (the
+  // previous call, which shares the workspace) finishes: touch no global
+  // memory before it has completed.  Returns at once otherwise.
+  if (p.pdl) sm100::grid_dependency_wait();
 
   // Grouped mode: the running (best key, max, sum) of each (lane quarter,
   // column) over the current segment live in shared memory, [4][BN] each,
@@ -1120,6 +1141,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------------------
 // Host launchers
 // ---------------------------------------------------------------------------
+// p.pdl: launched with programmatic stream serialization, so the kernel may
+// start while the kernel ahead of it in the stream finishes (that kernel's
+// CTAs signal launch_dependents once their work is done); it streams W at
+// once and waits for the grid dependency before it loads H or touches the
+// workspace.
 template <int BN, int MODE, bool MERGE = false>
 cudaError_t launch_t(const CUtensorMap &tw, const PartMaps &twp, const CUtensorMap &th,
                             const FmmsParams &p, cudaStream_t stream) {
@@ -1128,14 +1154,25 @@ cudaError_t launch_t(const CUtensorMap &tw, const PartMaps &twp, const CUtensorM
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  kern<<<p.num_ctas, kThreads, C::kSmemBytes, stream>>>(tw, twp, th, p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(p.num_ctas), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = p.pdl ? 1 : 0;
+  e = cudaLaunchKernelEx(&cfg, kern, tw, twp, th, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 // Pair kernels: clusters of two CTAs, p.num_ctas = 2 x schedule units.
 template <int BN, int MODE>
 cudaLaunchConfig_t pair_config(int num_ctas, cudaStream_t stream,
-                                      cudaLaunchAttribute *attr) {
+                                      cudaLaunchAttribute *attr, bool pdl = false) {
   using C = KCfg<BN, MODE, true>;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(num_ctas), 1, 1);
@@ -1146,8 +1183,10 @@ cudaLaunchConfig_t pair_config(int num_ctas, cudaStream_t stream,
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl ? 2 : 1;
   return cfg;
 }
 
@@ -1158,7 +1197,7 @@ cudaError_t pair_units_t(int *units) {
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   cudaLaunchConfig_t cfg = pair_config<BN, MODE>(2, nullptr, attr);
   int n = 0;
   e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
@@ -1176,8 +1215,8 @@ cudaError_t launch_pair_t(const CUtensorMap &tw, const PartMaps &twp,
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  cudaLaunchAttribute attr[1];
-  cudaLaunchConfig_t cfg = pair_config<BN, MODE>(p.num_ctas, stream, attr);
+  cudaLaunchAttribute attr[2];
+  cudaLaunchConfig_t cfg = pair_config<BN, MODE>(p.num_ctas, stream, attr, p.pdl != 0);
   e = cudaLaunchKernelEx(&cfg, kern, tw, twp, th, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

@@ -350,3 +350,10 @@ def test_debug_build_exports_the_same_symbols():
     assert dbg.fs_status_string is not None
     dbg.fs_status_string.restype = ctypes.c_char_p
     assert dbg.fs_status_string(6) == b"FS_ERR_DEVICE_BOUNDS"
+
+
+def test_programmatic_launch_switch_validates(lib):
+    assert lib.fs_set_programmatic_launch(2) == 1
+    assert lib.fs_set_programmatic_launch(-1) == 1
+    assert lib.fs_set_programmatic_launch(0) == 0
+    assert lib.fs_set_programmatic_launch(1) == 0

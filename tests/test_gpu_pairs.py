@@ -285,3 +285,45 @@ def test_partial_last_stage(dev, oracle, B, d):
     for b in np.flatnonzero(tok != idx):
         scale = TIE_REL * (1 + abs(summ[b, :, 0].max()))
         assert margin[b, 0] <= scale or margin[b, 1] <= scale, (b, tok[b], idx[b])
+
+
+def test_programmatic_launch_back_to_back_equals_plain_order(dev, oracle):
+    """Back-to-back calls on one stream with no synchronisation between them,
+    sharing the library workspace -- flat calls of several batch sizes (single
+    CTAs and CTA pairs), grouped calls (fused kernel + merge) and several
+    samples per row, interleaved -- give the same tokens bit for bit with the
+    fused kernel launched as a programmatic dependent of the kernel ahead
+    (its workspace accesses and H loads waiting for it) as in plain stream
+    order, and match the oracle."""
+    d, V = 256, 20011
+    W = synth.make_weight(V, d, 1.0 / 16.0, device="cpu", seed=77)
+    Wd = W.cuda()
+    Bs = [1, 64, 130, 256, 17, 200]
+    Hs = {B: synth.make_hidden(B, d, device="cpu", seed=78 + B) for B in Bs}
+    Hd = {B: h.cuda() for B, h in Hs.items()}
+
+    def run():
+        outs = []
+        for step in range(4):
+            for B in Bs:
+                outs.append(binding.fs_sample(Hd[B], Wd, temperature=0.9, seed=5, step=step))
+            outs.append(binding.fs_sample_grouped(Hd[130], Wd, 5, temperature=0.9, seed=5,
+                                                  step=step))
+            outs.append(binding.fs_sample_multi(Hd[64], Wd, 3, temperature=0.9, seed=5,
+                                                step=step))
+        torch.cuda.synchronize()
+        return outs
+    try:
+        binding.fs_set_programmatic_launch(0)
+        plain = run()
+        binding.fs_set_programmatic_launch(1)
+        pdl = run()
+    finally:
+        binding.fs_set_programmatic_launch(1)
+    for a, b in zip(plain, pdl):
+        assert torch.equal(a, b)
+    for step in range(4):
+        for i, B in enumerate(Bs):
+            got = pdl[step * (len(Bs) + 2) + i].cpu().numpy()
+            assert_parity(got, *oracle.sample(Hs[B], W, T=0.9, seed=5, step=step),
+                          "B=%d step %d" % (B, step))
