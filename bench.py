@@ -275,19 +275,25 @@ def roofline(B, d, V, masked, kernel_us, peaks, peak_kind, traffic, regime="burs
 
 
 # ------------------------------------------------------------ the GPU arm
-def time_calls(fn, steps, warmup, stream, world=1, sampler=None, cooldown_s=1.0):
+def time_calls(fn, steps, warmup, stream, world=1, sampler=None, cooldown_s=1.0, per_call=True):
     """Times exactly `steps` calls after `warmup` untimed ones.  Returns
-    (region ms, per-call event durations in us).  A short idle period first
-    lets the clocks recover from the power limit a previous heavy section may
-    have left them at."""
+    (region ms, per-call event durations in us, or None without per_call).
+    Events recorded between the calls keep each kernel from overlapping the
+    one before it (a programmatic dependent launch overlaps only kernels
+    adjacent in the stream), so the region that gives the throughput is
+    timed without them (per_call=False) and the per-call percentiles come
+    from a pass of their own.  A short idle period first lets the clocks
+    recover from the power limit a previous heavy section may have left them
+    at."""
     import torch
     torch.cuda.synchronize()
     time.sleep(cooldown_s)
     for i in range(warmup):
         fn(i)
     torch.cuda.synchronize()
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    n_ev = steps if per_call else 0
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
     r0 = torch.cuda.Event(enable_timing=True)
     r1 = torch.cuda.Event(enable_timing=True)
     barrier(world)
@@ -296,9 +302,11 @@ def time_calls(fn, steps, warmup, stream, world=1, sampler=None, cooldown_s=1.0)
         sampler.start()
     r0.record(stream)
     for i in range(steps):
-        starts[i].record(stream)
+        if per_call:
+            starts[i].record(stream)
         fn(warmup + i)
-        ends[i].record(stream)
+        if per_call:
+            ends[i].record(stream)
     r1.record(stream)
     while not r1.query():     # poll (releasing the GIL) so the clock sampler keeps running
         time.sleep(0.0005)
@@ -306,7 +314,7 @@ def time_calls(fn, steps, warmup, stream, world=1, sampler=None, cooldown_s=1.0)
     barrier(world)
     if sampler:
         sampler.stop()
-    per = [s.elapsed_time(e) * 1e3 for s, e in zip(starts, ends)]
+    per = [s.elapsed_time(e) * 1e3 for s, e in zip(starts, ends)] if per_call else None
     return r0.elapsed_time(r1), per
 
 
@@ -445,10 +453,9 @@ def run_gpu(args, world, rank, local):
 
     sampler = ClockSampler(local, period=0.002)
     with nvtx("fmms: timed steps"):
-        region_ms, per_call = time_calls(step, args.steps, args.warmup, stream, world, sampler)
+        region_ms, _ = time_calls(step, args.steps, args.warmup, stream, world, sampler,
+                                  per_call=False)
     region_ms = max_over_ranks(region_ms, world)
-    kernel_us = sum(per_call) / len(per_call)
-    kernel_us = max_over_ranks(kernel_us, world)
     us_per_call = region_ms * 1e3 / args.steps
     nbytes, flops = algorithmic(B, wl.d, wl.V, mask is not None)
     # fused kernel per 256 rows, plus the group merge (grouped) or the decode (tp)
@@ -456,6 +463,11 @@ def run_gpu(args, world, rank, local):
     # tensor-parallel: + the token decode after the all-reduce, or the bounded
     # wait that copies the exchanged tokens
     launches_per_call = (B + 255) // 256 * (2 if grouped else 1) + (1 if tp else 0)
+    # The fused kernel's average time per launch over the timed region (the
+    # stream holds nothing else in flat mode; with a merge or exchange kernel
+    # per call this is the call's time divided by its fused launches).
+    fused_launches = (B + 255) // 256
+    kernel_us = us_per_call / fused_launches
     if tp:
         # each rank streams its shard; the roofline below is per rank
         nbytes = nbytes * W.shape[0] // wl.V
@@ -475,7 +487,7 @@ def run_gpu(args, world, rank, local):
             step(i)
             Oh.copy_(out, non_blocking=True)
     with nvtx("fmms: end-to-end steps (host buffers)"):
-        e2e_ms, _ = time_calls(step_host, args.steps, args.warmup, stream, world)
+        e2e_ms, _ = time_calls(step_host, args.steps, args.warmup, stream, world, per_call=False)
     e2e_ms = max_over_ranks(e2e_ms, world)
 
     result = {
@@ -558,13 +570,15 @@ def sweep(torch, binding, synth, W, wl, dev, stream, peaks, peak_kind, steps=200
             binding.fs_sample_ex(H, W, temperature=wl.temperature, seed=0, row_seeds=rs, step=i,
                                  out_idx=out, stream=stream)
 
-        region_ms, per = time_calls(step, steps, warmup, stream)
-        kus = sum(per) / len(per)
+        region_ms, _ = time_calls(step, steps, warmup, stream, per_call=False)
+        _, per = time_calls(step, steps, warmup, stream, cooldown_s=0.2)
+        kus = region_ms * 1e3 / steps / binding.fs_fused_launches(B)
         rf = roofline(B, wl.d, wl.V, False, kus, peaks, peak_kind,
                       committed_traffic("%s/B%d" % (wl.name, B)), regime_of(region_ms * 1e-3))
         row = {"B": B, "us_per_call": round(region_ms * 1e3 / steps, 3),
                "kernel_us": round(kus, 3),
-               "kernel_us_p10_p50_p90": [round(x, 3) for x in percentiles(per)],
+               # per call with an event on each side (no overlap with the call before)
+               "event_us_p10_p50_p90": [round(x, 3) for x in percentiles(per)],
                "bound": rf["bound"],
                "achieved": round(rf["achieved"], 1), "unit": rf["unit"],
                "frac": round(rf["frac"], 4), "fracs": rf["fracs"], "regime": rf["regime"],
@@ -575,10 +589,10 @@ def sweep(torch, binding, synth, W, wl, dev, stream, peaks, peak_kind, steps=200
             # the same call on the single-CTA kernel, for comparison
             binding.fs_set_cta_pairs(0)
             try:
-                _, per1 = time_calls(step, steps, warmup, stream)
+                r1, _ = time_calls(step, steps, warmup, stream, per_call=False)
             finally:
                 binding.fs_set_cta_pairs(-1)
-            row["single_cta_kernel_us"] = round(sum(per1) / len(per1), 3)
+            row["single_cta_kernel_us"] = round(r1 * 1e3 / steps, 3)
         rows.append(row)
     return rows
 
@@ -591,7 +605,7 @@ def library_gemm_points(torch, synth, W, wl, dev, batches=(64, 128, 256), steps=
         H = synth.make_hidden(B, wl.d, device=dev)
         out = torch.empty(B, wl.V, dtype=torch.bfloat16, device=dev)
         region_ms, _ = time_calls(lambda i: torch.matmul(H, W.t(), out=out), steps, 10,
-                                  torch.cuda.current_stream())
+                                  torch.cuda.current_stream(), per_call=False)
         rows.append({"B": B, "us_per_call": round(region_ms * 1e3 / steps, 3)})
     return {"what": "torch.matmul(H, W.T) bf16 -> bf16 logits [B, V] (cuBLAS), no sampling",
             "points": rows}
@@ -614,13 +628,12 @@ def sustained_point(torch, binding, synth, W, wl, dev, stream, peaks, peak_kind,
 
     calls = max(100, int(seconds / 200e-6))
     sampler = ClockSampler(local, period=0.01)
-    region_ms, per = time_calls(step, calls, 20, stream, sampler=sampler)
-    kus = sum(per) / len(per)
+    region_ms, _ = time_calls(step, calls, 20, stream, sampler=sampler, per_call=False)
+    kus = region_ms * 1e3 / calls
     clk = sampler.summary()
     rf = roofline(B, wl.d, wl.V, False, kus, peaks, peak_kind, None, regime_of(region_ms * 1e-3))
     return {"B": B, "calls": calls, "region_s": round(region_ms * 1e-3, 3),
             "us_per_call": round(region_ms * 1e3 / calls, 3), "kernel_us": round(kus, 3),
-            "kernel_us_p10_p50_p90": [round(x, 3) for x in percentiles(per)],
             "sm_mhz_median": clk["sm_mhz"], "clock_samples": clk["samples"],
             "reasons": clk["reasons"],
             "kcycles_per_call": round(kus * clk["sm_mhz"] / 1e3, 1) if clk["sm_mhz"] else None,
@@ -643,7 +656,7 @@ def grouped_points(torch, binding, synth, dev, stream, peaks, peak_kind, W8, ste
             binding.fs_sample_grouped(H, W, wl.groups, temperature=wl.temperature, seed=0, step=i,
                                       mask_bits=mask, out_idx=out, stream=stream)
 
-        region_ms, _ = time_calls(step, steps, 10, stream)
+        region_ms, _ = time_calls(step, steps, 10, stream, per_call=False)
         us = region_ms * 1e3 / steps
         rf = roofline(B, wl.d, wl.V, True, us, peaks, peak_kind,
                       committed_traffic("%s/B%d" % (wl.name, B)), regime_of(region_ms * 1e-3))
@@ -667,7 +680,7 @@ def multi_point(torch, binding, synth, W, wl, dev, stream, B, S=4, steps=100):
         binding.fs_sample_multi(H, W, S, temperature=wl.temperature, seed=0, row_seeds=rs, step=i,
                                 out_idx=out, workspace=ws, stream=stream)
 
-    region_ms, _ = time_calls(step, steps, 10, stream)
+    region_ms, _ = time_calls(step, steps, 10, stream, per_call=False)
     return {"B": B, "num_samples": S, "us_per_call": round(region_ms * 1e3 / steps, 3),
             "samples_per_s": round(B * S / (region_ms * 1e-3 / steps), 1)}
 
@@ -730,11 +743,12 @@ def tiny_point(torch, binding, synth, dev, stream, copies=64, steps=640, graph_c
             binding.fs_sample_ex(H, Ws[i % copies], temperature=wl.temperature, seed=0, step=i,
                                  out_idx=out, workspace=ws, stream=stream)
 
-        region_ms, per = time_calls(step, steps, 3 * copies, stream)
+        region_ms, _ = time_calls(step, steps, 3 * copies, stream, per_call=False)
+        _, per = time_calls(step, steps, 3 * copies, stream, cooldown_s=0.2)
         res = {"workload": "tiny head d=%d V=%d B=%d, %d rotating W copies (%d MiB)"
                            % (wl.d, wl.V, B, copies, copies * wl.V * wl.d * 2 >> 20),
                "us_per_call": round(region_ms * 1e3 / steps, 3),
-               "kernel_us_p10_p50_p90": [round(x, 3) for x in percentiles(per)]}
+               "event_us_p10_p50_p90": [round(x, 3) for x in percentiles(per)]}
         s = torch.cuda.Stream()
         s.wait_stream(torch.cuda.current_stream())
         torch.cuda.synchronize()
@@ -772,7 +786,7 @@ def topk_point(torch, binding, synth, W, wl, dev, stream, B, K=50, steps=100):
         binding.fs_sample_topk(H, W, K, temperature=wl.temperature, seed=0, row_seeds=rs, step=i,
                                out_idx=out, logits=logits, stream=stream)
 
-    region_ms, _ = time_calls(step, steps, 10, stream)
+    region_ms, _ = time_calls(step, steps, 10, stream, per_call=False)
     return {"B": B, "K": K, "us_per_call": round(region_ms * 1e3 / steps, 3),
             "launches_per_call": 3 * ((B + 255) // 256)}
 
@@ -787,7 +801,7 @@ def unfused_point(torch, binding, synth, W, wl, dev, stream, B, steps=100):
         binding.fs_sample_unfused(H, W, temperature=wl.temperature, seed=0, row_seeds=rs, step=i,
                                   out_idx=out, logits=logits, stream=stream)
 
-    region_ms, _ = time_calls(step, steps, 10, stream)
+    region_ms, _ = time_calls(step, steps, 10, stream, per_call=False)
     return {"us_per_call": round(region_ms * 1e3 / steps, 3),
             "extra_hbm_bytes_per_call": 2 * B * wl.V * 4,
             "note": "matmul writes fp32 logits [B,V], a second kernel reads them back"}
