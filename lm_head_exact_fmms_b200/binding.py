@@ -31,7 +31,7 @@ EXPORTED = ("fs_sample", "fs_sample_ex", "fs_sample_grouped", "fs_sample_unfused
             "fs_tp_area_destroy", "fs_ipc_handle", "fs_ipc_open", "fs_ipc_close", "fs_sample_tp",
             "fs_tp_wait", "fs_tp_failed", "fs_test_stall_loads", "fs_set_partial_merge",
             "fs_plan_tiles_merged", "fs_plan_batch", "fs_noalloc_status",
-            "fs_test_inject_fault", "fs_set_programmatic_launch")
+            "fs_test_inject_fault", "fs_set_programmatic_launch", "fs_get_policies")
 
 FS_IPC_HANDLE_BYTES = 64
 
@@ -113,6 +113,7 @@ def load_library():
     lib.fs_noalloc_status.argtypes = [vp]
     lib.fs_test_inject_fault.argtypes = [i32, ctypes.POINTER(ctypes.c_int)]
     lib.fs_set_programmatic_launch.argtypes = [i32]
+    lib.fs_get_policies.argtypes = [ctypes.POINTER(ctypes.c_int)] * 4
     for name in EXPORTED:
         if name not in ("fs_workspace_bytes", "fs_workspace_bytes_multi",
                         "fs_workspace_bytes_summary", "fs_status_string", "fs_tp_area_bytes"):
@@ -418,6 +419,15 @@ def fs_set_programmatic_launch(on):
     """1: launch the fused kernel as a programmatic dependent of the kernel
     ahead of it in the stream (the default); 0: plain stream order."""
     _check(load_library().fs_set_programmatic_launch(int(on)), "fs_set_programmatic_launch")
+
+
+def fs_get_policies():
+    """The execution-path choices in force (FS_FORCE_PATH, then the fs_set_*
+    calls): {"cta_pairs", "partial_merge", "programmatic", "unfused"}."""
+    v = [ctypes.c_int(0) for _ in range(4)]
+    _check(load_library().fs_get_policies(*[ctypes.byref(x) for x in v]), "fs_get_policies")
+    return dict(zip(("cta_pairs", "partial_merge", "programmatic", "unfused"),
+                    (x.value for x in v)))
 
 
 def fs_sample_shard_keys(H, W_shard, vocab_offset, V_total, temperature=1.0, seed=0,

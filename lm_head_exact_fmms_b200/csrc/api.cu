@@ -32,6 +32,8 @@ struct DeviceState {
   void *o_stage = nullptr;  // fs_sample_host: device tokens
   size_t o_stage_bytes = 0;
   void *topk_scratch = nullptr;  // fs_sample_topk: per-block candidate lists and counts
+  void *forced_logits = nullptr;  // FS_FORCE_PATH=unfused: fp32 logits of flat calls
+  size_t forced_logits_bytes = 0;
   size_t topk_scratch_bytes = 0;
   // fs_sample_host: H is copied on copy_stream while the kernel already
   // streams W; h_flags[k] takes the call's epoch once the copy into
@@ -265,6 +267,40 @@ int g_pdl_policy = 1;
 // fs_set_partial_merge: -1 automatic, 0 never, 1 always (single CTAs, <= 64 rows).
 int g_merge_policy = -1;
 
+// FS_FORCE_PATH (environment, read once at the first sampling call): a
+// comma-separated list that sets the initial execution-path choices for A/B
+// runs without code changes -- "unfused" (flat single-sample calls fs_sample
+// and fs_sample_ex run the two-kernel measurement mode: fp32 logits through
+// HBM, then the sampling kernel) or "fused"; "pairs" or "single" (as
+// fs_set_cta_pairs(1 / 0)); "merge" or "nomerge" (fs_set_partial_merge);
+// "plain" or "programmatic" (fs_set_programmatic_launch).  Unknown words are
+// ignored.  The fs_set_* calls still override it afterwards.
+bool g_force_unfused = false;
+std::once_flag g_force_once;
+
+void read_force_path() {
+  std::call_once(g_force_once, [] {
+    const char *e = getenv("FS_FORCE_PATH");
+    if (e == nullptr) return;
+    const char *p = e;
+    while (*p) {
+      const char *q = p;
+      while (*q && *q != ',') ++q;
+      const size_t n = static_cast<size_t>(q - p);
+      auto is = [&](const char *w) { return strlen(w) == n && strncmp(p, w, n) == 0; };
+      if (is("unfused")) g_force_unfused = true;
+      if (is("fused")) g_force_unfused = false;
+      if (is("pairs")) g_pair_policy = 1;
+      if (is("single")) g_pair_policy = 0;
+      if (is("merge")) g_merge_policy = 1;
+      if (is("nomerge")) g_merge_policy = 0;
+      if (is("plain")) g_pdl_policy = 0;
+      if (is("programmatic")) g_pdl_policy = 1;
+      p = *q ? q + 1 : q;
+    }
+  });
+}
+
 int bn_index(int BN) { return BN / 16 - 1; }
 
 // CTA pairs of the BN pair kernel of `mode` that fit on the device at once
@@ -355,6 +391,7 @@ fs_status run(int mode, const void *H, const void *W, int B, int d, int V, int G
               uint64_t seed, const uint64_t *row_seeds, uint32_t step, const uint32_t *mask,
               int32_t *out_idx, fs_group_summary *summary, float *logits, void *ws,
               size_t ws_bytes, cudaStream_t stream) {
+  read_force_path();
   std::lock_guard<std::mutex> lock(g_mu);
   return run_locked(mode, H, W, B, d, V, G, T, seed, row_seeds, step, mask, out_idx, summary,
                     logits, ws, ws_bytes, stream);
@@ -509,13 +546,38 @@ fs_status run_locked(int mode, const void *H, const void *W, int B, int d, int V
 
 extern "C" {
 
+namespace {
+// A flat single-sample call: the fused kernel, or with FS_FORCE_PATH=unfused
+// the two-kernel mode with a library-owned logits buffer (same tokens).
+fs_status run_flat(const void *H, const void *W, int B, int d, int V, float T, uint64_t seed,
+                   const uint64_t *row_seeds, uint32_t step, const uint32_t *mask,
+                   int32_t *out_idx, void *ws, size_t ws_bytes, cudaStream_t stream) {
+  read_force_path();
+  if (!g_force_unfused)
+    return run(fmms::kModeFlat, H, W, B, d, V, 1, T, seed, row_seeds, step, mask, out_idx,
+               nullptr, nullptr, ws, ws_bytes, stream);
+  if (launch_fault()) return FS_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState *st = nullptr;
+  fs_status s = get_device(&st);
+  if (s != FS_OK) return s;
+  const size_t bytes = static_cast<size_t>(B) * V * sizeof(float);
+  if ((s = grow(&st->forced_logits, &st->forced_logits_bytes, bytes)) != FS_OK) return s;
+  ShardOpts o;
+  s = run_locked(fmms::kModeLogits, H, W, B, d, V, 1, T, seed, row_seeds, step, mask, out_idx,
+                 nullptr, static_cast<float *>(st->forced_logits), ws, ws_bytes, stream, o);
+  if (s != FS_OK) return s;
+  return FS_OK;
+}
+}  // namespace
+
 fs_status fs_sample(const void *H, const void *W, int B, int d, int V, float temperature,
                     uint64_t seed, uint32_t step, const uint32_t *mask_bits, int32_t *out_idx,
                     fs_stream_t stream) {
   fs_status s = validate(H, W, B, d, V, temperature, out_idx);
   if (s != FS_OK) return s;
-  return run(fmms::kModeFlat, H, W, B, d, V, 1, temperature, seed, nullptr, step, mask_bits,
-             out_idx, nullptr, nullptr, nullptr, 0, static_cast<cudaStream_t>(stream));
+  return run_flat(H, W, B, d, V, temperature, seed, nullptr, step, mask_bits, out_idx, nullptr,
+                  0, static_cast<cudaStream_t>(stream));
 }
 
 fs_status fs_sample_ex(const void *H, const void *W, int B, int d, int V, float temperature,
@@ -524,9 +586,8 @@ fs_status fs_sample_ex(const void *H, const void *W, int B, int d, int V, float 
                        size_t workspace_bytes, fs_stream_t stream) {
   fs_status s = validate(H, W, B, d, V, temperature, out_idx);
   if (s != FS_OK) return s;
-  return run(fmms::kModeFlat, H, W, B, d, V, 1, temperature, seed, row_seeds, step, mask_bits,
-             out_idx, nullptr, nullptr, workspace, workspace_bytes,
-             static_cast<cudaStream_t>(stream));
+  return run_flat(H, W, B, d, V, temperature, seed, row_seeds, step, mask_bits, out_idx,
+                  workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
 fs_status fs_sample_grouped(const void *H, const void *W, int B, int d, int V, int G,
@@ -941,6 +1002,7 @@ fs_status fs_gumbel(const uint32_t *r, float *g, int64_t n, fs_stream_t stream) 
 
 fs_status fs_set_partial_merge(int policy) {
   if (policy < -1 || policy > 1) return FS_ERR_INVALID_ARG;
+  read_force_path();
   std::lock_guard<std::mutex> lock(g_mu);
   g_merge_policy = policy;
   return FS_OK;
@@ -954,8 +1016,20 @@ fs_status fs_test_inject_fault(int kind, int *previous) {
   return FS_OK;
 }
 
+fs_status fs_get_policies(int *cta_pairs, int *partial_merge, int *programmatic,
+                          int *unfused) {
+  read_force_path();
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (cta_pairs) *cta_pairs = g_pair_policy;
+  if (partial_merge) *partial_merge = g_merge_policy;
+  if (programmatic) *programmatic = g_pdl_policy;
+  if (unfused) *unfused = g_force_unfused ? 1 : 0;
+  return FS_OK;
+}
+
 fs_status fs_set_programmatic_launch(int on) {
   if (on < 0 || on > 1) return FS_ERR_INVALID_ARG;
+  read_force_path();
   std::lock_guard<std::mutex> lock(g_mu);
   g_pdl_policy = on;
   return FS_OK;
@@ -963,6 +1037,7 @@ fs_status fs_set_programmatic_launch(int on) {
 
 fs_status fs_set_cta_pairs(int policy) {
   if (policy < -1 || policy > 1) return FS_ERR_INVALID_ARG;
+  read_force_path();
   std::lock_guard<std::mutex> lock(g_mu);
   g_pair_policy = policy;
   return FS_OK;
@@ -1013,6 +1088,7 @@ fs_status fs_plan_tiles_merged(int V, int G, int num_sms, int cta, int32_t *tile
 
 fs_status fs_plan_batch(int B, int kind, int *launches, int *batch_tile, int *cta_pairs) {
   if (B < 1 || kind < 0 || kind > 2 || !launches) return FS_ERR_INVALID_ARG;
+  read_force_path();
   const int mode = kind == 1 ? fmms::kModeGrouped : kind == 2 ? fmms::kModeLogits : fmms::kModeFlat;
   const int first = fmms::imin(fmms::kMaxBN, B);
   const int BN = fmms::fmms_batch_tile(first);

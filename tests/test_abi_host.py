@@ -357,3 +357,41 @@ def test_programmatic_launch_switch_validates(lib):
     assert lib.fs_set_programmatic_launch(-1) == 1
     assert lib.fs_set_programmatic_launch(0) == 0
     assert lib.fs_set_programmatic_launch(1) == 0
+
+
+@pytest.mark.parametrize("env,want,pairs256", [
+    (None, {"cta_pairs": -1, "partial_merge": -1, "programmatic": 1, "unfused": 0}, 1),
+    ("single,nomerge,plain,unfused",
+     {"cta_pairs": 0, "partial_merge": 0, "programmatic": 0, "unfused": 1}, 0),
+    ("pairs,merge,bogus,fused", {"cta_pairs": 1, "partial_merge": 1, "programmatic": 1,
+                                 "unfused": 0}, 1),
+])
+def test_force_path_environment(env, want, pairs256):
+    """FS_FORCE_PATH sets the initial execution-path choices (read once, in a
+    fresh process per value); fs_plan_batch follows them."""
+    import subprocess
+    import sys
+    code = ("from lm_head_exact_fmms_b200 import binding; import json; "
+            "print(json.dumps([binding.fs_get_policies(), binding.fs_plan_batch(256)[2]]))")
+    envd = dict(os.environ)
+    envd.pop("FS_FORCE_PATH", None)
+    if env is not None:
+        envd["FS_FORCE_PATH"] = env
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True,
+                         env=envd, cwd=ROOT, timeout=300)
+    assert out.returncode == 0, out.stderr[-1000:]
+    import json
+    pol, pairs = json.loads(out.stdout.strip().splitlines()[-1])
+    assert pol == want and pairs == pairs256
+
+
+def test_setters_override_the_environment():
+    import subprocess
+    import sys
+    code = ("from lm_head_exact_fmms_b200 import binding; binding.fs_set_cta_pairs(1); "
+            "print(binding.fs_get_policies()['cta_pairs'])")
+    envd = dict(os.environ, FS_FORCE_PATH="single")
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True,
+                         env=envd, cwd=ROOT, timeout=300)
+    assert out.returncode == 0, out.stderr[-1000:]
+    assert out.stdout.strip().splitlines()[-1] == "1"

@@ -100,3 +100,50 @@ def test_injected_host_faults_leave_the_library_usable(dev, oracle):
     assert torch.equal(host.to(dev), ref)
     area = binding.fs_tp_area_create()
     binding.fs_tp_area_destroy(area)
+
+
+def test_forced_unfused_path_gives_the_fused_tokens(dev, oracle):
+    """FS_FORCE_PATH=unfused (a child process): fs_sample_ex runs the two-kernel
+    mode (fp32 logits through HBM, then the sampler) and returns the tokens
+    of the fused kernel bit for bit, for one and for two 256-row launches, with
+    mask and row seeds; the tokens match the oracle."""
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    shapes = [(5, 128, 3001), (300, 64, 2048)]
+    code = """
+import json, sys, torch
+sys.path.insert(0, %r)
+from lm_head_exact_fmms_b200 import binding, synth
+assert binding.fs_get_policies()["unfused"] == 1
+res = []
+for B, d, V in %r:
+    H = synth.make_hidden(B, d, seed=B).cuda()
+    W = synth.make_weight(V, d, 0.125, seed=V).cuda()
+    rs = synth.make_row_seeds(B).cuda()
+    mask = synth.make_mask(B, V, 0.5, seed=3).cuda()
+    t = binding.fs_sample_ex(H, W, temperature=0.8, seed=2, row_seeds=rs, step=4, mask_bits=mask)
+    torch.cuda.synchronize()
+    assert binding.fs_device_status(None) == 0
+    res.append(t.cpu().tolist())
+print(json.dumps(res))
+""" % (root, shapes)
+    env = dict(os.environ, FS_FORCE_PATH="unfused")
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, env=env,
+                         cwd=root, timeout=600)
+    assert out.returncode == 0, out.stdout[-2000:] + out.stderr[-2000:]
+    forced = json.loads(out.stdout.strip().splitlines()[-1])
+    for (B, d, V), toks in zip(shapes, forced):
+        H = synth.make_hidden(B, d, seed=B)
+        W = synth.make_weight(V, d, 0.125, seed=V)
+        rs = synth.make_row_seeds(B)
+        mask = synth.make_mask(B, V, 0.5, seed=3)
+        fused = binding.fs_sample_ex(H.to(dev), W.to(dev), temperature=0.8, seed=2,
+                                     row_seeds=rs.to(dev), step=4, mask_bits=mask.to(dev))
+        torch.cuda.synchronize()
+        assert fused.cpu().tolist() == toks, (B, d, V)
+        idx, best, second = oracle.sample(H, W, T=0.8, seed=2, row_seeds=rs, step=4, mask=mask)
+        bad = np.asarray(toks) != idx
+        assert not np.any(bad & ((best - second) > 2e-3 * (1 + np.abs(best))))
