@@ -124,16 +124,19 @@ class ClockSampler:
             getattr(n, "nvmlDeviceGetCurrentClocksThrottleReasons")
         return fn(self._h)
 
+    def _sample(self):
+        try:
+            self.samples.append(self._nvml.nvmlDeviceGetClockInfo(self._h, self._nvml.NVML_CLOCK_SM))
+            bits = self._reasons()
+            for b, name in self.REASONS.items():
+                if bits & b:
+                    self.reasons.add(name)
+        except Exception:
+            pass
+
     def _run(self):
         while not self._stop.is_set():
-            try:
-                self.samples.append(self._nvml.nvmlDeviceGetClockInfo(self._h, self._nvml.NVML_CLOCK_SM))
-                bits = self._reasons()
-                for b, name in self.REASONS.items():
-                    if bits & b:
-                        self.reasons.add(name)
-            except Exception:
-                pass
+            self._sample()
             time.sleep(self.period)
 
     def start(self):
@@ -451,7 +454,7 @@ def run_gpu(args, world, rank, local):
             binding.fs_sample_ex(H, W, temperature=wl.temperature, seed=0, row_seeds=rs, step=i,
                                  mask_bits=mask, out_idx=out, workspace=ws, stream=stream)
 
-    sampler = ClockSampler(local, period=0.002)
+    sampler = ClockSampler(local, period=0.0005)
     with nvtx("fmms: timed steps"):
         region_ms, _ = time_calls(step, args.steps, args.warmup, stream, world, sampler,
                                   per_call=False)
