@@ -1,6 +1,7 @@
 """Every row of the LM-head workloads at full size against the CPU oracle, in
-the launch configuration the benchmark times (CTA pairs above 64 rows,
-several 256-row launches for B=512): 1,664 rows in all, over several steps.
+the launch configuration the benchmark times (CTA pairs from 113 rows,
+several 256-row launches for B=512, flat steps issued back to back): 1,664 rows in all,
+over several steps.
 Same tolerance as test_gpu_parity: a token may differ from the oracle's only
 at a near tie of the oracle's two best perturbed scores; at most one such row
 is allowed here (the expected count is about 0.02).  (Runs for about a
@@ -44,7 +45,14 @@ def test_every_row_of_full_size_workloads(dev, oracle):
                     assert margin[b, 0] <= scale or margin[b, 1] <= scale, (name, step, b)
                 mism += int(bad.sum())
             else:
-                got = binding.fs_sample_ex(Hd, Wd, **kw).cpu().numpy()
+                # The steps go out back to back with no synchronisation (each
+                # launch of up to 128 rows a programmatic dependent of the one
+                # before, as in the benchmark) and are checked afterwards.
+                if step == 0:
+                    outs = [binding.fs_sample_ex(Hd, Wd, **dict(kw, step=s))
+                            for s in range(steps)]
+                    torch.cuda.synchronize()
+                got = outs[step].cpu().numpy()
                 idx, best, second = oracle.sample(H, W, T=wl.temperature, seed=11,
                                                   row_seeds=rs, step=step, mask=mask)
                 mism += assert_parity(got, idx, best, second, "%s B=%d step %d" % (name, B, step))
