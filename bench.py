@@ -586,7 +586,7 @@ def sweep(torch, binding, synth, W, wl, dev, stream, peaks, peak_kind, steps=200
                "achieved": round(rf["achieved"], 1), "unit": rf["unit"],
                "frac": round(rf["frac"], 4), "fracs": rf["fracs"], "regime": rf["regime"],
                "traffic": rf["traffic"],
-               # the library's automatic choice: CTA pairs above 64 rows per launch
+               # the library's automatic choice (fs_plan_batch): CTA pairs from a 112-row tile
                "cta_pairs": binding.fs_uses_cta_pairs(B)}
         if compare_single and row["cta_pairs"]:
             # the same call on the single-CTA kernel, for comparison

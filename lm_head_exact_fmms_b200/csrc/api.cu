@@ -318,13 +318,15 @@ int pair_units(DeviceState *st, int mode, int BN) {
   return u;
 }
 
-// Flat and grouped calls with a batch tile of 128 or more rows run on CTA
+// Flat and grouped calls with a batch tile of 112 or more rows run on CTA
 // pairs: each SM then stages half of H per stage, which halves the batch
 // operand's L2 traffic and the MMA issues per byte of W where the tensor
-// cores are busy.
+// cores are busy.  Measured (200 back-to-back calls, single CTAs / pairs):
+// Qwen3-8B head B=96 208.8 / 212.4 us, B=112 239.3 / 218.6 us, B=128
+// 248.9 / 226.9 us; Qwen3-1.7B head B=96 110.7 / 110.5, B=112 126.9 / 113.6.
 bool use_pairs(int mode, int BN) {
   if (mode == fmms::kModeLogits || g_pair_policy == 0) return false;
-  return g_pair_policy == 1 || BN >= 128;
+  return g_pair_policy == 1 || BN >= 112;
 }
 
 // Options of vocabulary-shard and multi-sample calls.

@@ -74,15 +74,17 @@ def test_grouped_and_unfused_validation(lib):
 
 @pytest.mark.parametrize("B,kind,want", [
     (1, "flat", (1, 16, 0)), (16, "flat", (1, 16, 0)), (17, "flat", (1, 32, 0)),
-    (64, "flat", (1, 64, 0)), (112, "flat", (1, 112, 0)), (113, "flat", (1, 128, 1)),
+    (64, "flat", (1, 64, 0)), (96, "flat", (1, 96, 0)), (97, "flat", (1, 112, 1)),
+    (112, "flat", (1, 112, 1)), (113, "flat", (1, 128, 1)),
     (200, "flat", (1, 208, 1)), (256, "flat", (1, 256, 1)), (257, "flat", (2, 256, 1)),
-    (1, "grouped", (1, 16, 0)), (512, "grouped", (2, 256, 1)), (100, "grouped", (1, 112, 0)),
+    (1, "grouped", (1, 16, 0)), (512, "grouped", (2, 256, 1)), (100, "grouped", (1, 112, 1)),
+    (90, "grouped", (1, 96, 0)),
     (256, "logits", (1, 256, 0)), (300, "logits", (2, 256, 0)),
 ])
 def test_plan_batch_automatic_choice(lib, B, kind, want):
     """The launch plan of a call: one fused launch per 256 rows, the batch
     tile rounded up to 16 rows, and CTA pairs (automatic policy) from a
-    128-row tile up, never in logits mode."""
+    112-row tile up, never in logits mode."""
     binding.fs_set_cta_pairs(-1)
     assert binding.fs_plan_batch(B, kind) == want
 

@@ -1,5 +1,5 @@
 """Every row of the LM-head workloads at full size against the CPU oracle, in
-the launch configuration the benchmark times (CTA pairs from 113 rows,
+the launch configuration the benchmark times (CTA pairs from 97 rows,
 several 256-row launches for B=512, flat steps issued back to back): 1,664 rows in all,
 over several steps.
 Same tolerance as test_gpu_parity: a token may differ from the oracle's only
