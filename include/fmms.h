@@ -439,8 +439,9 @@ fs_status fs_test_inject_fault(int kind, int *previous);
  * the method: the results are the same either way (tokens bit for bit).
  * policy: -1 automatic (the default: pairs for launches whose batch tile,
  * the row count rounded up to a multiple of 16, is 112 or more, i.e. from
- * 97 rows per launch; fs_plan_batch reports the choice), 0 never, 1 always.  Process-wide; applies to calls made after
- * it returns.  FS_ERR_INVALID_ARG for any other value.  When the device
+ * 97 rows per launch; fs_plan_batch reports the choice), 0 never, 1 always.
+ * Process-wide; applies to calls made after it returns.  FS_ERR_INVALID_ARG
+ * for any other value.  When the device
  * cannot co-schedule a pair, the single-CTA kernel runs.  The unfused
  * measurement path (fs_sample_unfused, fs_sample_topk) always runs on single
  * CTAs. */

@@ -910,7 +910,8 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
             const uint32_t allowed = chunk_allowed<CW>(p, vg, v_ok, col0, lane);
             uint32_t words[CW];
             chunk_noise<CW>(p, vg, col0, lane, 0u, words);
-            const int si = FS_IN_BOUNDS(p.err, q * BN + c, 4 * BN) ? q * BN + c : 0;  // this lane's (quarter, column) state
+            // this lane's (quarter, column) state
+            const int si = FS_IN_BOUNDS(p.err, q * BN + c, 4 * BN) ? q * BN + c : 0;
             float m_run = comb_m[si], s_run = comb_s[si];
             uint64_t best = comb_key[si];
             chunk_lse2<CW>(acc, c1, allowed, comb_m + q * BN + col0, lane, m_run, s_run);
