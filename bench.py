@@ -454,7 +454,8 @@ def run_gpu(args, world, rank, local):
             binding.fs_sample_ex(H, W, temperature=wl.temperature, seed=0, row_seeds=rs, step=i,
                                  mask_bits=mask, out_idx=out, workspace=ws, stream=stream)
 
-    sampler = ClockSampler(local, period=0.0)  # as fast as NVML answers: the region lasts milliseconds
+    # As fast as NVML answers while the region lasts milliseconds; every 5 ms for long runs.
+    sampler = ClockSampler(local, period=0.0 if args.steps <= 200 else 0.005)
     with nvtx("fmms: timed steps"):
         region_ms, _ = time_calls(step, args.steps, args.warmup, stream, world, sampler,
                                   per_call=False)
