@@ -194,6 +194,8 @@ def test_tiny_workload_matches_golden(dev, oracle):
     (128, 8, 300), (200, 96, 5000), (256, 256, 4096), (257, 64, 2048), (300, 40, 64),
     (16, 64, 1), (16, 64, 7), (33, 64, 8), (2, 64, 9), (5, 512, 127), (5, 512, 128),
     (4, 72, 1183),
+    # either side of the automatic CTA-pair threshold (a 112-row batch tile)
+    (96, 128, 3001), (97, 128, 3001), (112, 64, 10007),
 ])
 def test_flat_parity_shapes(dev, oracle, B, d, V):
     H, W, Hd, Wd = rand_inputs(B, d, V, seed=B * 1000 + V)
