@@ -105,6 +105,8 @@ class ClockSampler:
     def __init__(self, index, period=0.01):
         self.index, self.period = index, period
         self.samples, self.reasons = [], set()
+        self.stamped = []          # (host time, SM MHz, reason bits) of every NVML sample
+        self.window = None         # (t0, t1): keep only samples taken inside it
         self.max_mhz = None
         self._stop = threading.Event()
         self._thread = None
@@ -126,11 +128,9 @@ class ClockSampler:
 
     def _sample(self):
         try:
-            self.samples.append(self._nvml.nvmlDeviceGetClockInfo(self._h, self._nvml.NVML_CLOCK_SM))
+            mhz = self._nvml.nvmlDeviceGetClockInfo(self._h, self._nvml.NVML_CLOCK_SM)
             bits = self._reasons()
-            for b, name in self.REASONS.items():
-                if bits & b:
-                    self.reasons.add(name)
+            self.stamped.append((time.perf_counter(), mhz, bits))
         except Exception:
             pass
 
@@ -170,7 +170,26 @@ class ClockSampler:
                 except Exception:
                     pass
 
+    def set_window(self, t0, t1):
+        """Keep only the samples taken between host times t0 and t1 (the
+        timed region: the sampler may start earlier, during the warm-up, so
+        that it is already answering when a region of milliseconds begins)."""
+        self.window = (t0, t1)
+
+    def _collect(self):
+        if self._nvml is None:
+            return
+        t0, t1 = self.window if self.window is not None else (-1e30, 1e30)
+        self.samples = [m for t, m, _ in self.stamped if t0 <= t <= t1]
+        self.reasons = set()
+        for t, _, bits in self.stamped:
+            if t0 <= t <= t1:
+                for b, name in self.REASONS.items():
+                    if bits & b:
+                        self.reasons.add(name)
+
     def summary(self):
+        self._collect()
         s = sorted(self.samples)
         med = s[len(s) // 2] if s else None
         return {"sm_mhz": med, "sm_max_mhz": self.max_mhz,
@@ -291,6 +310,8 @@ def time_calls(fn, steps, warmup, stream, world=1, sampler=None, cooldown_s=1.0,
     import torch
     torch.cuda.synchronize()
     time.sleep(cooldown_s)
+    if sampler:
+        sampler.start()  # answering by the time the region starts; samples outside it are dropped
     for i in range(warmup):
         fn(i)
     torch.cuda.synchronize()
@@ -301,8 +322,7 @@ def time_calls(fn, steps, warmup, stream, world=1, sampler=None, cooldown_s=1.0,
     r1 = torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
-    if sampler:
-        sampler.start()
+    t_host0 = time.perf_counter()
     r0.record(stream)
     for i in range(steps):
         if per_call:
@@ -314,9 +334,11 @@ def time_calls(fn, steps, warmup, stream, world=1, sampler=None, cooldown_s=1.0,
     while not r1.query():     # poll (releasing the GIL) so the clock sampler keeps running
         time.sleep(0.0005)
     torch.cuda.synchronize()
+    t_host1 = time.perf_counter()
     barrier(world)
     if sampler:
         sampler.stop()
+        sampler.set_window(t_host0, t_host1)
     per = [s.elapsed_time(e) * 1e3 for s, e in zip(starts, ends)] if per_call else None
     return r0.elapsed_time(r1), per
 

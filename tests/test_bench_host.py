@@ -111,3 +111,16 @@ def test_nvtx_sections_are_transparent():
         with bench.nvtx("failing section"):
             raise KeyError("k")
     assert ran == [1]
+
+
+def test_clock_sampler_keeps_only_samples_inside_the_region():
+    """The sampler starts before the warm-up; the summary counts only samples
+    stamped inside the timed region's host window, and their reasons."""
+    s = bench.ClockSampler(0)
+    s._nvml = object()          # as if NVML answered (no GPU here)
+    s.max_mhz = 1965
+    s.stamped = [(0.5, 1965, 0x1), (1.0, 1500, 0x4), (1.5, 1480, 0x4), (2.5, 1965, 0x8)]
+    s.set_window(0.9, 2.0)
+    r = s.summary()
+    assert r["samples"] == 2 and r["sm_mhz"] in (1480, 1500)
+    assert r["reasons"] == ["sw_power_cap"] and r["sm_max_mhz"] == 1965
