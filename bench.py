@@ -563,6 +563,8 @@ def run_gpu(args, world, rank, local):
         with nvtx("fmms: grouped + masked"):
             result["grouped_masked"] = grouped_points(torch, binding, synth, dev, stream, peaks,
                                                       peak_kind, W)
+        with nvtx("fmms: online grouped"):
+            result["online_grouped"] = online_grouped_point(torch, binding, synth, dev, stream, W)
         with nvtx("fmms: unfused"):
             result["unfused"] = unfused_point(torch, binding, synth, W, wl, dev, stream, B)
         with nvtx("fmms: several samples per row"):
@@ -693,6 +695,40 @@ def grouped_points(torch, binding, synth, dev, stream, peaks, peak_kind, W8, ste
                      "launches_per_call": 2 * binding.fs_fused_launches(B, "grouped")})
     return {"workload": "grouped-masked d=%d V=%d G=%d, 50%% mask, T=%g (fused kernel + merge)"
                         % (wl.d, wl.V, wl.groups, wl.temperature), "points": rows}
+
+
+def online_grouped_point(torch, binding, synth, dev, stream, W8, B=64, steps=100):
+    """Online grouped sampling on the grouped + masked head: each of the G
+    groups summarised by its own call on its slice of W (as when only one
+    group's weights are on chip at a time), then the summaries merged."""
+    wl = synth.WORKLOADS["grouped-masked"]
+    W = W8 if (W8.shape[0] == wl.V and W8.shape[1] == wl.d) else \
+        synth.make_weight(wl.V, wl.d, wl.w_std, device=dev)
+    G = wl.groups
+    bounds = [(g * wl.V) // G for g in range(G + 1)]
+    if any(b % 8 for b in bounds):
+        return {"B": B, "us_per_call": None, "error": "group boundaries not multiples of 8"}
+    H = synth.make_hidden(B, wl.d, device=dev)
+    mask = synth.make_mask(B, wl.V, wl.mask_allowed).to(dev)
+    summ = torch.empty(G, B, 3, dtype=torch.float32, device=dev)
+    out = torch.empty(B, dtype=torch.int32, device=dev)
+    slices = [W[bounds[g]:bounds[g + 1]] for g in range(G)]  # contiguous row ranges
+    ws = torch.zeros(binding.fs_workspace_bytes_summary(B, max(b1 - b0 for b0, b1 in
+                                                              zip(bounds, bounds[1:]))),
+                     dtype=torch.uint8, device=dev)
+
+    def step(i):
+        for g in range(G):
+            binding.fs_summarize_group(H, slices[g], bounds[g], wl.V, temperature=wl.temperature,
+                                       seed=0, step=i, mask_bits=mask, out_summary=summ[g],
+                                       workspace=ws, stream=stream)
+        binding.fs_merge_groups(summ, seed=0, step=i, out_idx=out, stream=stream)
+
+    region_ms, _ = time_calls(step, steps, 10, stream, per_call=False)
+    return {"B": B, "groups": G, "us_per_call": round(region_ms * 1e3 / steps, 3),
+            "launches_per_call": 2 * G + 1,
+            "note": "one fs_summarize_group per group (fused kernel + summary merge) and one "
+                    "fs_merge_groups"}
 
 
 def multi_point(torch, binding, synth, W, wl, dev, stream, B, S=4, steps=100):

@@ -43,9 +43,15 @@ static cudaError_t launch_dependent(void (*kern)(KArgs...), dim3 grid, dim3 bloc
 }
 
 // ---------------------------------------------------------------------------
-// Group merge: one warp per row; lanes stride over the groups.
+// Group merge: one warp per row; lanes stride over the groups, or with at
+// most four groups teams of lanes share each group's partials.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(128) group_merge_kernel(const MergeParams m) {
+  // The kernel after this one may start launching now: a fused sampling
+  // kernel launched as a programmatic dependent streams W meanwhile and
+  // waits for this grid to complete before it loads H or touches the
+  // workspace or the outputs this grid writes.
+  sm100::launch_dependents();
   sm100::grid_dependency_wait();  // the fused kernel's partials
   const int b = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
   const int lane = threadIdx.x & 31;
@@ -64,34 +70,46 @@ __global__ void __launch_bounds__(128) group_merge_kernel(const MergeParams m) {
   float best_key = -INFINITY;
   int best_g = -1;
   unsigned long long best_tok = 0ull;
-  for (int g = lane; g < m.G; g += 32) {
-    const int lo = group_begin(g, m.V, m.G);
-    const int hi = group_begin(g + 1, m.V, m.G);
-    const int c_first = cta_of(lo, sch);
-    const int c_last = cta_of(hi - 1, sch);
+  // With few groups a team of lanes shares one group's partials (a group of
+  // a single-group call spans every CTA: 148 slots a row), else each lane
+  // takes whole groups.  Teams are aligned runs of `team` lanes.
+  const int team = m.G == 1 ? 32 : m.G == 2 ? 16 : m.G <= 4 ? 8 : 1;
+  const int member = lane & (team - 1);
+  const int nteams = 32 / team;
+  for (int g0 = 0; g0 < m.G; g0 += nteams) {  // warp-uniform
+    const int g = g0 + lane / team;
+    const bool gok = g < m.G;
     unsigned long long kmax = 0ull;
     float M = -INFINITY, S = 0.f;
     // The group's partials: slots c + g for its CTAs c (2 (c + g) and
-    // 2 (c + g) + 1 for CTA pairs c).  Loads go out eight at a time, and the
-    // slots are zeroed only after all are read, so the loads overlap.
+    // 2 (c + g) + 1 for CTA pairs c).  A member takes slots member,
+    // member + team, ...; loads go out eight at a time, and the slots are
+    // zeroed only after all are read, so the loads overlap.
+    int c_first = 0, nslots = 0;
     const int per_unit = m.pair ? 2 : 1;
-    const int nslots = (c_last - c_first + 1) * per_unit;
+    if (gok) {
+      const int lo = group_begin(g, m.V, m.G);
+      const int hi = group_begin(g + 1, m.V, m.G);
+      c_first = cta_of(lo, sch);
+      nslots = (cta_of(hi - 1, sch) - c_first + 1) * per_unit;
+    }
     auto slot_of = [&](int i) -> size_t {
       const int u = c_first * per_unit + i;
       return m.pair ? 2 * static_cast<size_t>(u / 2 + g) + (u & 1) : static_cast<size_t>(u + g);
     };
-    for (int i0 = 0; i0 < nslots; i0 += 8) {
+    for (int i0 = member; i0 < nslots; i0 += 8 * team) {
       GroupPartial gp[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
+        const int i = i0 + j * team;
         gp[j] = GroupPartial{0ull, -INFINITY, 0.f};
-        if (i0 + j < nslots &&
-            FS_IN_BOUNDS(m.err, static_cast<long long>(slot_of(i0 + j)) * m.B + b, m.partials_cap))
-          gp[j] = m.partials[slot_of(i0 + j) * m.B + b];
+        if (i < nslots &&
+            FS_IN_BOUNDS(m.err, static_cast<long long>(slot_of(i)) * m.B + b, m.partials_cap))
+          gp[j] = m.partials[slot_of(i) * m.B + b];
       }
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        if (i0 + j >= nslots) break;
+        if (i0 + j * team >= nslots) break;
         kmax = gp[j].key > kmax ? gp[j].key : kmax;
         if (gp[j].m != -INFINITY) {
           if (M == -INFINITY) {
@@ -105,9 +123,27 @@ __global__ void __launch_bounds__(128) group_merge_kernel(const MergeParams m) {
         }
       }
     }
-    for (int i = 0; i < nslots; ++i)  // leave the workspace zeroed
+    for (int i = member; i < nslots; i += team)  // leave the workspace zeroed
       if (FS_IN_BOUNDS(m.err, static_cast<long long>(slot_of(i)) * m.B + b, m.partials_cap))
         m.partials[slot_of(i) * m.B + b] = GroupPartial{0ull, 0.f, 0.f};
+    // Team reduction: the maximum key and the merged (max, sum) pair.
+    for (int off = team / 2; off >= 1; off >>= 1) {
+      const unsigned long long ko = __shfl_xor_sync(0xffffffffu, kmax, off);
+      const float Mo = __shfl_xor_sync(0xffffffffu, M, off);
+      const float So = __shfl_xor_sync(0xffffffffu, S, off);
+      kmax = ko > kmax ? ko : kmax;
+      if (Mo != -INFINITY) {
+        if (M == -INFINITY) {
+          M = Mo;
+          S = So;
+        } else {
+          const float mx = fmaxf(M, Mo);
+          S = S * expf(M - mx) + So * expf(Mo - mx);
+          M = mx;
+        }
+      }
+    }
+    if (!gok || member != 0) continue;
     if (m.gkeys != nullptr &&
         FS_IN_BOUNDS(m.err, static_cast<long long>(g) * m.B + b, m.gkeys_cap))
       m.gkeys[static_cast<size_t>(g) * m.B + b] = 0ull;  // left zeroed
@@ -139,8 +175,9 @@ __global__ void __launch_bounds__(128) group_merge_kernel(const MergeParams m) {
     packed = o > packed ? o : packed;
   }
   const int gwin = key_token(packed);
+  // group g was taken by the first lane of team g mod nteams
   const unsigned long long tok =
-      __shfl_sync(0xffffffffu, best_tok, gwin < 0 ? 0 : (gwin & 31));
+      __shfl_sync(0xffffffffu, best_tok, gwin < 0 ? 0 : (gwin % nteams) * team);
   if (lane == 0 && m.out_idx != nullptr) m.out_idx[b] = gwin < 0 ? -1 : key_token(tok);
 }
 
@@ -149,6 +186,11 @@ __global__ void __launch_bounds__(128) group_merge_kernel(const MergeParams m) {
 __global__ void __launch_bounds__(128)
     merge_summaries_kernel(const fs_group_summary *summaries, int G, int B, uint64_t seed,
                            const uint64_t *row_seeds, uint32_t step, int32_t *out_idx) {
+  // The kernel after this one may start launching now: a fused sampling
+  // kernel launched as a programmatic dependent streams W meanwhile and
+  // waits for this grid to complete before it loads H or touches the
+  // workspace or the outputs this grid writes.
+  sm100::launch_dependents();
   sm100::grid_dependency_wait();
   const int b = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
   const int lane = threadIdx.x & 31;
@@ -205,6 +247,11 @@ cudaError_t launch_group_merge(const MergeParams &m, cudaStream_t stream) {
 // block decodes.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) sample_logits_kernel(const SampleLogitsParams s) {
+  // The kernel after this one may start launching now: a fused sampling
+  // kernel launched as a programmatic dependent streams W meanwhile and
+  // waits for this grid to complete before it loads H or touches the
+  // workspace or the outputs this grid writes.
+  sm100::launch_dependents();
   sm100::grid_dependency_wait();  // the logits
   const int b = blockIdx.y;
   const uint32_t bg = static_cast<uint32_t>(s.b_off + b);
@@ -720,6 +767,11 @@ __global__ void __launch_bounds__(kTopkThreads) topk_row_kernel(const TopkArgs a
   __shared__ unsigned int t0;
   __shared__ unsigned long long small[kTopkRowSmall];
   extern __shared__ unsigned long long kept[];  // kTopkRowCap entries
+  // The kernel after this one may start launching now: a fused sampling
+  // kernel launched as a programmatic dependent streams W meanwhile and
+  // waits for this grid to complete before it loads H or touches the
+  // workspace or the outputs this grid writes.
+  sm100::launch_dependents();
   sm100::grid_dependency_wait();  // the candidate lists
   const int b = blockIdx.x;
   const int lane = threadIdx.x & 31;
@@ -903,6 +955,11 @@ cudaError_t launch_topk_sample(const SampleLogitsParams &s, int K, void *scratch
 // Vocabulary shards: tokens from the reduced keys.
 // ---------------------------------------------------------------------------
 __global__ void keys_to_tokens_kernel(const long long *keys, int B, int32_t *out_idx) {
+  // The kernel after this one may start launching now: a fused sampling
+  // kernel launched as a programmatic dependent streams W meanwhile and
+  // waits for this grid to complete before it loads H or touches the
+  // workspace or the outputs this grid writes.
+  sm100::launch_dependents();
   sm100::grid_dependency_wait();  // the reduced keys
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b < B) out_idx[b] = key_token(static_cast<uint64_t>(keys[b]) ^ 0x8000000000000000ull);

@@ -196,10 +196,13 @@ def test_pairs_grouped(dev, oracle, B, d, V, G, masked):
     assert np.allclose(l0[fin], l1[fin], rtol=1e-6, atol=1e-5)
     idx, o_summ, margin = oracle.sample_grouped(H, W, G, T=0.8, seed=12, step=2, mask=mask)
     got = t1.cpu().numpy()
-    for b in np.flatnonzero(got != idx):
-        scale = TIE_REL * (1 + abs(o_summ[b, :, 0].max()))
-        assert margin[b, 0] <= scale or margin[b, 1] <= scale, (b, got[b], idx[b])
-    assert (t0.cpu().numpy() == got).mean() > 0.99
+    # Both kernels' tokens follow the oracle; where they differ from it (or
+    # from each other, the log-sum-exps being merged in another order), the
+    # oracle's group keys or the chosen group's top two scores are a near tie.
+    for name, toks in (("single", t0.cpu().numpy()), ("pair", got)):
+        for b in np.flatnonzero(toks != idx):
+            scale = TIE_REL * (1 + abs(o_summ[b, :, 0].max()))
+            assert margin[b, 0] <= scale or margin[b, 1] <= scale, (name, b, toks[b], idx[b])
     if G == 1:
         flat = with_policy(1, lambda: binding.fs_sample_ex(Hd, Wd, temperature=0.8, seed=12,
                                                            step=2, mask_bits=md))
@@ -217,14 +220,16 @@ def test_pairs_grouped_full_size_head(dev, oracle):
     single, pair = both(lambda: binding.fs_sample_grouped(Hd, Wd, wl.groups,
                                                           temperature=wl.temperature, seed=0,
                                                           step=0, mask_bits=mask.to(dev)))
-    assert (single == pair).float().mean().item() > 0.99
-    rows = np.array([0, 255, 256, B - 1], dtype=np.int32)
+    s_np, p_np = single.cpu().numpy(), pair.cpu().numpy()
+    # sampled rows (launch edges) and every row where the two kernels differ
+    rows = np.union1d([0, 255, 256, B - 1], np.flatnonzero(s_np != p_np)).astype(np.int32)
+    assert rows.size <= 4 + 5   # differences only at rare near ties
     idx, summ, margin = oracle.sample_grouped(Hd.cpu(), Wd.cpu(), wl.groups, T=wl.temperature,
                                               seed=0, step=0, mask=mask, rows=rows)
-    got = pair.cpu().numpy()[rows]
-    for i in np.flatnonzero(got != idx):
-        scale = TIE_REL * (1 + abs(summ[i, :, 0].max()))
-        assert margin[i, 0] <= scale or margin[i, 1] <= scale, (rows[i], got[i], idx[i])
+    for name, toks in (("single", s_np[rows]), ("pair", p_np[rows])):
+        for i in np.flatnonzero(toks != idx):
+            scale = TIE_REL * (1 + abs(summ[i, :, 0].max()))
+            assert margin[i, 0] <= scale or margin[i, 1] <= scale, (name, rows[i], toks[i], idx[i])
     del Wd, Hd
     torch.cuda.empty_cache()
 
