@@ -98,6 +98,10 @@ MUTANTS = [
      "} else if (s[v] > b2) {\n      b2 = s[v];\n    }\n  }\n  if (best) *best = b1;",
      "}\n  }\n  if (best) *best = b1;",
      "test_oracle_argmax_scan_ties_to_the_smallest_index", {}),
+    ("grouped_within_margin_from_the_wrong_scores",
+     "out_margin[2 * i + 1] = (gstar < 0) ? INFINITY : in1 - in2;",
+     "out_margin[2 * i + 1] = (gstar < 0) ? INFINITY : in1 - k2;",
+     "test_grouped_summary_and_margins_match_the_scores", {"G": 3}),
     ("topk_ties_toward_the_larger_index",
      "return (x->v < y->v) ? -1 : (x->v > y->v);",
      "return (x->v > y->v) ? -1 : (x->v < y->v);",

@@ -451,6 +451,49 @@ def test_grouped_summary_identities(oracle, G):
         assert best_v == flat[b]
 
 
+@pytest.mark.parametrize("G", [1, 2, 3, 8])
+def test_grouped_summary_and_margins_match_the_scores(oracle, G):
+    """The grouped sampler's per-group (max score, argmax) and its margins,
+    which the GPU tests' tie rule relies on, against the separately pinned
+    perturbed scores: each group's maximum and first maximiser over its range;
+    the token lies in a group; the within-group margin is the gap between the
+    top two scores of the token's group (+inf with one allowed token); the
+    group-key margin is positive, and +inf with a single group."""
+    V, d, B, T = 211, 24, 12, 0.9
+    H = synth.make_hidden(B, d, seed=91)
+    W = synth.make_weight(V, d, 0.5, seed=92)
+    allowed = torch.rand(B, V, generator=torch.Generator().manual_seed(5)) < 0.5
+    allowed[1] = False
+    allowed[2] = False
+    allowed[2, 17] = True
+    mask = synth.mask_from_bool(allowed)
+    rs = synth.make_row_seeds(B)
+    idx, summ, margin = oracle.sample_grouped(H, W, G, T=T, seed=6, row_seeds=rs, step=3,
+                                              mask=mask)
+    sc = oracle.scores(H, W, T=T, seed=6, row_seeds=rs, step=3, mask=mask)
+    for b in range(B):
+        for g in range(G):
+            lo, hi = (g * V) // G, ((g + 1) * V) // G
+            seg = sc[b, lo:hi]
+            if np.isfinite(seg).any():
+                assert summ[b, g, 0] == seg.max()
+                assert int(summ[b, g, 1]) == lo + int(np.argmax(seg))
+            else:
+                assert summ[b, g, 0] == -np.inf and int(summ[b, g, 1]) == -1
+        if idx[b] < 0:
+            assert not np.isfinite(sc[b]).any()
+            continue
+        g = next(g for g in range(G) if (g * V) // G <= idx[b] < ((g + 1) * V) // G)
+        assert idx[b] == int(summ[b, g, 1])
+        seg = np.sort(sc[b, (g * V) // G:((g + 1) * V) // G])
+        want = seg[-1] - seg[-2] if np.isfinite(seg[-2]) else np.inf
+        assert margin[b, 1] == want
+        assert margin[b, 0] > 0
+        if G == 1:
+            assert margin[b, 0] == np.inf
+    assert idx[1] == -1 and idx[2] == 17
+
+
 @pytest.mark.parametrize("G", [2, 3, 8, 64])
 def test_grouped_matches_softmax(oracle, G):
     V, d, N, T = 64, 32, 200_000, 1.3
