@@ -613,9 +613,10 @@ def test_multi_sample_first_is_single_sample(oracle):
     B, d, V = 12, 32, 300
     H = synth.make_hidden(B, d, seed=121)
     W = synth.make_weight(V, d, 0.5, seed=122)
-    single, b1, _ = oracle.sample(H, W, T=0.8, seed=5, step=3)
-    multi, mb, _ = oracle.sample_multi(H, W, 6, T=0.8, seed=5, step=3)
+    single, b1, s1 = oracle.sample(H, W, T=0.8, seed=5, step=3)
+    multi, mb, ms = oracle.sample_multi(H, W, 6, T=0.8, seed=5, step=3)
     assert np.array_equal(multi[:, 0], single) and np.array_equal(mb[:, 0], b1)
+    assert np.array_equal(ms[:, 0], s1)      # the runner-up the tie rule uses, too
     # the samples use distinct noise: they are not all equal
     assert (multi != multi[:, :1]).any()
 
@@ -642,10 +643,11 @@ def test_topk_degenerate_cases(oracle):
     H = synth.make_hidden(B, d, seed=141)
     W = synth.make_weight(V, d, 0.5, seed=142)
     for step in range(4):
-        flat, fb, _ = oracle.sample(H, W, T=0.9, seed=2, step=step)
-        all_k, ab, _ = oracle.sample_topk(H, W, V, T=0.9, seed=2, step=step)
+        flat, fb, fs = oracle.sample(H, W, T=0.9, seed=2, step=step)
+        all_k, ab, asec = oracle.sample_topk(H, W, V, T=0.9, seed=2, step=step)
         more, _, _ = oracle.sample_topk(H, W, 10 * V, T=0.9, seed=2, step=step)
         assert np.array_equal(all_k, flat) and np.array_equal(ab, fb) and np.array_equal(more, flat)
+        assert np.array_equal(asec, fs)     # the runner-up the tie rule uses, too
         one, _, _ = oracle.sample_topk(H, W, 1, T=0.9, seed=2, step=step)
         assert np.array_equal(one, np.argmax(oracle.logits(H, W), axis=1))   # greedy
 
