@@ -462,18 +462,21 @@ fs_status fs_set_programmatic_launch(int on);
 
 /* The execution-path choices in force: *cta_pairs and *partial_merge (-1
  * automatic, 0 never, 1 always, as set by fs_set_cta_pairs and
- * fs_set_partial_merge), *programmatic (fs_set_programmatic_launch) and
- * *unfused (1 when flat single-sample calls run the unfused two-kernel mode).
- * The initial choices come from the environment variable FS_FORCE_PATH, read
- * once at the first call that uses them: a comma-separated list of
- * "unfused" or "fused" (fs_sample and fs_sample_ex run the measurement mode of
- * fs_sample_unfused, fp32 logits through HBM in a library-owned buffer, or
- * the fused kernel; same tokens), "pairs" or "single", "merge" or "nomerge",
+ * fs_set_partial_merge), *programmatic (fs_set_programmatic_launch),
+ * *unfused (1 when flat single-sample calls run the unfused two-kernel mode)
+ * and *two_kernel_reduce (1 when flat calls leave the per-row maxima to a
+ * second, decoding kernel instead of the fused kernel's last CTA; the fused
+ * tensor-parallel exchange always uses the last CTA).  The initial choices
+ * come from the environment variable FS_FORCE_PATH, read once at the first
+ * call that uses them: a comma-separated list of "unfused" or "fused"
+ * (fs_sample and fs_sample_ex run the measurement mode of fs_sample_unfused,
+ * fp32 logits through HBM in a library-owned buffer, or the fused kernel),
+ * "twokernel" or "lastcta", "pairs" or "single", "merge" or "nomerge",
  * "plain" or "programmatic"; unknown words are ignored, and the fs_set_*
- * calls override it afterwards.  For A/B runs without code changes.
- * Host-only; NULL pointers are skipped. */
+ * calls override it afterwards.  Every choice gives the same tokens.  For A/B
+ * runs without code changes.  Host-only; NULL pointers are skipped. */
 fs_status fs_get_policies(int *cta_pairs, int *partial_merge, int *programmatic,
-                          int *unfused);
+                          int *unfused, int *two_kernel_reduce);
 
 /* Kernel choice for single-CTA launches of up to 64 batch rows: a CTA whose
  * vocabulary range starts with an 8-row partial tile can either run it as a

@@ -113,7 +113,7 @@ def load_library():
     lib.fs_noalloc_status.argtypes = [vp]
     lib.fs_test_inject_fault.argtypes = [i32, ctypes.POINTER(ctypes.c_int)]
     lib.fs_set_programmatic_launch.argtypes = [i32]
-    lib.fs_get_policies.argtypes = [ctypes.POINTER(ctypes.c_int)] * 4
+    lib.fs_get_policies.argtypes = [ctypes.POINTER(ctypes.c_int)] * 5
     for name in EXPORTED:
         if name not in ("fs_workspace_bytes", "fs_workspace_bytes_multi",
                         "fs_workspace_bytes_summary", "fs_status_string", "fs_tp_area_bytes"):
@@ -423,11 +423,12 @@ def fs_set_programmatic_launch(on):
 
 def fs_get_policies():
     """The execution-path choices in force (FS_FORCE_PATH, then the fs_set_*
-    calls): {"cta_pairs", "partial_merge", "programmatic", "unfused"}."""
-    v = [ctypes.c_int(0) for _ in range(4)]
+    calls): {"cta_pairs", "partial_merge", "programmatic", "unfused",
+    "two_kernel_reduce"}."""
+    v = [ctypes.c_int(0) for _ in range(5)]
     _check(load_library().fs_get_policies(*[ctypes.byref(x) for x in v]), "fs_get_policies")
-    return dict(zip(("cta_pairs", "partial_merge", "programmatic", "unfused"),
-                    (x.value for x in v)))
+    return dict(zip(("cta_pairs", "partial_merge", "programmatic", "unfused",
+                     "two_kernel_reduce"), (x.value for x in v)))
 
 
 def fs_sample_shard_keys(H, W_shard, vocab_offset, V_total, temperature=1.0, seed=0,

@@ -273,9 +273,12 @@ int g_merge_policy = -1;
 // and fs_sample_ex run the two-kernel measurement mode: fp32 logits through
 // HBM, then the sampling kernel) or "fused"; "pairs" or "single" (as
 // fs_set_cta_pairs(1 / 0)); "merge" or "nomerge" (fs_set_partial_merge);
-// "plain" or "programmatic" (fs_set_programmatic_launch).  Unknown words are
-// ignored.  The fs_set_* calls still override it afterwards.
+// "plain" or "programmatic" (fs_set_programmatic_launch); "twokernel" or
+// "lastcta" (flat calls reduce the per-row maxima in a second kernel, or in
+// the fused kernel's last CTA).  Unknown words are ignored.  The fs_set_*
+// calls still override it afterwards.
 bool g_force_unfused = false;
+bool g_two_kernel_reduce = false;
 std::once_flag g_force_once;
 
 void read_force_path() {
@@ -294,6 +297,8 @@ void read_force_path() {
       if (is("single")) g_pair_policy = 0;
       if (is("merge")) g_merge_policy = 1;
       if (is("nomerge")) g_merge_policy = 0;
+      if (is("twokernel")) g_two_kernel_reduce = true;
+      if (is("lastcta")) g_two_kernel_reduce = false;
       if (is("plain")) g_pdl_policy = 0;
       if (is("programmatic")) g_pdl_policy = 1;
       p = *q ? q + 1 : q;
@@ -459,6 +464,10 @@ fs_status run_locked(int mode, const void *H, const void *W, int B, int d, int V
     // head 13-16 -> 12.4 us); at 256 rows, tensor-bound, the overlap
     // measured 2-3 % slower.
     p.pdl = (g_pdl_policy != 0 && BN <= 128) ? 1 : 0;
+    // The two-kernel reduction applies to flat launches that end in tokens
+    // or keys of this device (not the fused exchange).
+    const bool two_kernel = g_two_kernel_reduce && mode == fmms::kModeFlat && shard.tp_world == 0;
+    p.no_ticket = two_kernel ? 1 : 0;
     p.vocab_offset = shard.vocab_offset;
     p.out_keys = shard.out_keys ? shard.out_keys + static_cast<size_t>(b0) * S : nullptr;
     p.num_samples = S;
@@ -490,7 +499,11 @@ fs_status run_locked(int mode, const void *H, const void *W, int B, int d, int V
         return FS_ERR_CUDA;
     }
 
-    if (mode == fmms::kModeGrouped) {
+    if (two_kernel) {
+      if (fmms::launch_decode_published(w.keys, Bc, S, p.out_idx, p.out_keys, w.err, p.keys_cap,
+                                        stream) != cudaSuccess)
+        return FS_ERR_CUDA;
+    } else if (mode == fmms::kModeGrouped) {
       fmms::MergeParams m;
       m.partials = w.partials;
       m.gkeys = w.gkeys;
@@ -1019,13 +1032,14 @@ fs_status fs_test_inject_fault(int kind, int *previous) {
 }
 
 fs_status fs_get_policies(int *cta_pairs, int *partial_merge, int *programmatic,
-                          int *unfused) {
+                          int *unfused, int *two_kernel_reduce) {
   read_force_path();
   std::lock_guard<std::mutex> lock(g_mu);
   if (cta_pairs) *cta_pairs = g_pair_policy;
   if (partial_merge) *partial_merge = g_merge_policy;
   if (programmatic) *programmatic = g_pdl_policy;
   if (unfused) *unfused = g_force_unfused ? 1 : 0;
+  if (two_kernel_reduce) *two_kernel_reduce = g_two_kernel_reduce ? 1 : 0;
   return FS_OK;
 }
 

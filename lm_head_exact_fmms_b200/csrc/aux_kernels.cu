@@ -952,6 +952,34 @@ cudaError_t launch_topk_sample(const SampleLogitsParams &s, int K, void *scratch
                                a);
 }
 // ---------------------------------------------------------------------------
+// Two-kernel reduction (an A/B alternative to the last CTA's ticket): one
+// thread per (row, sample) reads the published maximum and re-zeroes it.
+// ---------------------------------------------------------------------------
+__global__ void decode_published_kernel(unsigned long long *keys, int B, int S, int32_t *out_idx,
+                                        long long *out_keys, int *err, int keys_cap) {
+  sm100::launch_dependents();
+  sm100::grid_dependency_wait();  // the fused kernel's published keys
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= B * S) return;
+  const int b = i / S;
+  const int smp = i - b * S;
+  if (!FS_IN_BOUNDS(err, smp * kMaxBN + b, keys_cap)) return;
+  const unsigned long long kb = atomicExch(keys + smp * kMaxBN + b, 0ull);
+  if (out_keys != nullptr)
+    out_keys[i] = static_cast<long long>(kb ^ 0x8000000000000000ull);  // signed order
+  else
+    out_idx[i] = key_token(kb);
+}
+
+cudaError_t launch_decode_published(unsigned long long *keys, int B, int num_samples,
+                                    int32_t *out_idx, long long *out_keys, int *err,
+                                    int keys_cap, cudaStream_t stream) {
+  const int n = B * num_samples;
+  return launch_dependent(decode_published_kernel, dim3((n + 255) / 256), dim3(256), stream, keys,
+                          B, num_samples, out_idx, out_keys, err, keys_cap);
+}
+
+// ---------------------------------------------------------------------------
 // Vocabulary shards: tokens from the reduced keys.
 // ---------------------------------------------------------------------------
 __global__ void keys_to_tokens_kernel(const long long *keys, int B, int32_t *out_idx) {

@@ -289,6 +289,9 @@ struct FmmsParams {
   // 1: launched as a programmatic dependent of the grid ahead in the stream
   // (may start before it ends; H loads and workspace accesses wait for it).
   int pdl;
+  // Flat mode: 1 leaves the published keys for a second kernel to decode
+  // (the two-kernel reduction, an A/B alternative to the last-CTA ticket).
+  int no_ticket;
   // Extents the debug build's bounds checks compare against (entries, not
   // bytes): rows of row_seeds and mask (the whole call), packed keys in the
   // workspace, partial records and published group maxima, and tokens (or

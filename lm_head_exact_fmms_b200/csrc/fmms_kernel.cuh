@@ -982,6 +982,7 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
     }
   }
 
+  if (MODE == kModeFlat && p.no_ticket) return;  // a second kernel decodes the keys
   if constexpr (MODE == kModeFlat) {
     // Every maximum is already published; take a ticket, and the last CTA
     // decodes the keys and re-zeroes them for the next call.  With the fused

@@ -103,6 +103,13 @@ cudaError_t launch_merge_summaries(const void *summaries, int G, int B, uint64_t
 cudaError_t launch_tp_wait(TpArea *area, int B, uint32_t seq, int32_t *out_idx,
                            uint32_t timeout_us, cudaStream_t stream);
 
+// The two-kernel reduction: decodes the fused kernel's published keys
+// [sample][kMaxBN rows] of this launch's B rows into tokens (or, with
+// out_keys, packed keys XOR 2^63) and re-zeroes them for the next call.
+cudaError_t launch_decode_published(unsigned long long *keys, int B, int num_samples,
+                                    int32_t *out_idx, long long *out_keys, int *err,
+                                    int keys_cap, cudaStream_t stream);
+
 // Decodes packed keys (XOR 2^63, as fs_sample_shard_keys writes them) to tokens.
 cudaError_t launch_keys_to_tokens(const long long *keys, int B, int32_t *out_idx,
                                   cudaStream_t stream);

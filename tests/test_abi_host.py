@@ -362,11 +362,14 @@ def test_programmatic_launch_switch_validates(lib):
 
 
 @pytest.mark.parametrize("env,want,pairs256", [
-    (None, {"cta_pairs": -1, "partial_merge": -1, "programmatic": 1, "unfused": 0}, 1),
-    ("single,nomerge,plain,unfused",
-     {"cta_pairs": 0, "partial_merge": 0, "programmatic": 0, "unfused": 1}, 0),
-    ("pairs,merge,bogus,fused", {"cta_pairs": 1, "partial_merge": 1, "programmatic": 1,
-                                 "unfused": 0}, 1),
+    (None, {"cta_pairs": -1, "partial_merge": -1, "programmatic": 1, "unfused": 0,
+            "two_kernel_reduce": 0}, 1),
+    ("single,nomerge,plain,unfused,twokernel",
+     {"cta_pairs": 0, "partial_merge": 0, "programmatic": 0, "unfused": 1,
+      "two_kernel_reduce": 1}, 0),
+    ("pairs,merge,bogus,fused,twokernel,lastcta",
+     {"cta_pairs": 1, "partial_merge": 1, "programmatic": 1, "unfused": 0,
+      "two_kernel_reduce": 0}, 1),
 ])
 def test_force_path_environment(env, want, pairs256):
     """FS_FORCE_PATH sets the initial execution-path choices (read once, in a

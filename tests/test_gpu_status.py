@@ -147,3 +147,45 @@ print(json.dumps(res))
         idx, best, second = oracle.sample(H, W, T=0.8, seed=2, row_seeds=rs, step=4, mask=mask)
         bad = np.asarray(toks) != idx
         assert not np.any(bad & ((best - second) > 2e-3 * (1 + np.abs(best))))
+
+
+def test_two_kernel_reduction_gives_the_last_cta_tokens(dev, oracle):
+    """FS_FORCE_PATH=twokernel (a child process): flat calls leave the per-row
+    maxima for a second, decoding kernel instead of the fused kernel's last
+    CTA; single- and several-sample calls, one and two 256-row launches, and
+    shard keys give the default path's results bit for bit."""
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+    def runs(binding, synth, torch):
+        out = []
+        for B, d, V in [(5, 128, 3001), (300, 64, 2048)]:
+            H = synth.make_hidden(B, d, seed=B).cuda()
+            W = synth.make_weight(V, d, 0.125, seed=V).cuda()
+            rs = synth.make_row_seeds(B).cuda()
+            t = binding.fs_sample_ex(H, W, temperature=0.8, seed=2, row_seeds=rs, step=4)
+            m = binding.fs_sample_multi(H, W, 3, temperature=0.8, seed=2, step=4)
+            k = binding.fs_sample_shard_keys(H, W[:1024].contiguous(), 0, V, temperature=0.8,
+                                             seed=2, step=4)
+            torch.cuda.synchronize()
+            assert binding.fs_device_status(None) == 0
+            out.append([t.cpu().tolist(), m.cpu().tolist(), k.cpu().tolist()])
+        return out
+
+    import inspect
+    import textwrap
+    src = textwrap.dedent(inspect.getsource(runs))
+    code = "import json, sys, torch\nsys.path.insert(0, %r)\n" % root + \
+        "from lm_head_exact_fmms_b200 import binding, synth\n" + src + \
+        "assert binding.fs_get_policies()['two_kernel_reduce'] == 1\n" + \
+        "print(json.dumps(runs(binding, synth, torch)))\n"
+    env = dict(os.environ, FS_FORCE_PATH="twokernel")
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, env=env,
+                         cwd=root, timeout=600)
+    assert out.returncode == 0, out.stdout[-2000:] + out.stderr[-2000:]
+    forced = json.loads(out.stdout.strip().splitlines()[-1])
+    assert binding.fs_get_policies()["two_kernel_reduce"] == 0
+    assert runs(binding, synth, torch) == forced
