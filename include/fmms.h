@@ -359,7 +359,9 @@ fs_status fs_sample_noalloc(const void *H, const void *W, int B, int d, int V,
 /* Reads (synchronously, after `stream` drains) and clears the status word of
  * fs_sample_noalloc's fixed array on the current device: FS_OK, or
  * FS_ERR_DEVICE_TIMEOUT when a call since the last read gave up on a bounded
- * wait (its tokens were not written); FS_OK too before the first call.
+ * wait (its tokens were not written), or in the debug build
+ * FS_ERR_DEVICE_BOUNDS when a bounds check failed; FS_OK too before the
+ * first call.
  * Allocates nothing; like fs_sample_noalloc, it must not overlap such a call
  * on the GPU.  The paper has no counterpart for this entry point. */
 fs_status fs_noalloc_status(fs_stream_t stream);
@@ -377,8 +379,9 @@ size_t fs_workspace_bytes_summary(int B, int V_g);
 
 /* Reads (synchronously, after the stream drains) and clears the device-side
  * status word of a workspace (NULL = the library-owned one on the current
- * device).  Returns FS_OK or FS_ERR_DEVICE_TIMEOUT; after a timeout the
- * workspace is zero-filled again so it can be reused.  fs_sample_noalloc
+ * device).  Returns FS_OK, FS_ERR_DEVICE_TIMEOUT, or (debug build only)
+ * FS_ERR_DEVICE_BOUNDS; after either error the workspace is zero-filled again
+ * so it can be reused.  fs_sample_noalloc
  * keeps its status in its own array: read it with fs_noalloc_status. */
 fs_status fs_device_status(void *workspace, size_t workspace_bytes,
                            fs_stream_t stream);
