@@ -127,12 +127,22 @@ class ClockSampler:
         return fn(self._h)
 
     def _sample(self):
+        # Stamped at the midpoint of the two queries: on some hosts a query
+        # takes milliseconds, as long as a whole short timed region.
         try:
+            t = time.perf_counter()
             mhz = self._nvml.nvmlDeviceGetClockInfo(self._h, self._nvml.NVML_CLOCK_SM)
             bits = self._reasons()
-            self.stamped.append((time.perf_counter(), mhz, bits))
+            self.stamped.append((0.5 * (t + time.perf_counter()), mhz, bits))
         except Exception:
             pass
+
+    def sample_now(self):
+        """One sample from the calling thread (the host polls the GPU with
+        it while a timed region drains, so even a region of a few
+        milliseconds holds samples)."""
+        if self._nvml is not None:
+            self._sample()
 
     def _run(self):
         while not self._stop.is_set():
@@ -331,8 +341,11 @@ def time_calls(fn, steps, warmup, stream, world=1, sampler=None, cooldown_s=1.0,
         if per_call:
             ends[i].record(stream)
     r1.record(stream)
-    while not r1.query():     # poll (releasing the GIL) so the clock sampler keeps running
-        time.sleep(0.0005)
+    while not r1.query():     # poll, sampling the clocks while the queued calls run
+        if sampler:
+            sampler.sample_now()
+        else:
+            time.sleep(0.0005)
     torch.cuda.synchronize()
     t_host1 = time.perf_counter()
     barrier(world)

@@ -124,3 +124,40 @@ def test_clock_sampler_keeps_only_samples_inside_the_region():
     r = s.summary()
     assert r["samples"] == 2 and r["sm_mhz"] in (1480, 1500)
     assert r["reasons"] == ["sw_power_cap"] and r["sm_max_mhz"] == 1965
+
+
+def test_clock_sampler_samples_from_the_polling_thread():
+    """sample_now() queries from the calling thread and stamps the sample at
+    the middle of its queries, so a region shorter than one query of a slow
+    NVML still holds the sample taken while it drained."""
+    import types
+    import time as _time
+
+    calls = []
+
+    def clock(h, which):
+        calls.append("clock")
+        _time.sleep(0.002)
+        return 1700
+
+    def reasons(h):
+        calls.append("reasons")
+        _time.sleep(0.002)
+        return 0x4
+
+    s = bench.ClockSampler(0)
+    s._nvml = types.SimpleNamespace(nvmlDeviceGetClockInfo=clock, NVML_CLOCK_SM=1,
+                                    nvmlDeviceGetCurrentClocksEventReasons=reasons)
+    s._h = None
+    s.max_mhz = 1965
+    t0 = _time.perf_counter()
+    s.sample_now()
+    t1 = _time.perf_counter()
+    assert calls == ["clock", "reasons"] and len(s.stamped) == 1
+    t, mhz, bits = s.stamped[0]
+    assert t0 < t < t1 and mhz == 1700 and bits == 0x4
+    # A window that opens after the first query began and closes before
+    # the last one ended still keeps it.
+    s.set_window(t0 + 0.001, t1 - 0.001)
+    r = s.summary()
+    assert r["samples"] == 1 and r["sm_mhz"] == 1700 and r["reasons"] == ["sw_power_cap"]
