@@ -137,17 +137,27 @@ class ClockSampler:
         except Exception:
             pass
 
+    MIN_INTERVAL_S = 0.0005  # at most 2,000 queries a second from the polling loop
+
     def sample_now(self):
         """One sample from the calling thread (the host polls the GPU with
         it while a timed region drains, so even a region of a few
-        milliseconds holds samples)."""
-        if self._nvml is not None:
-            self._sample()
+        milliseconds holds samples), at most one per MIN_INTERVAL_S; in
+        between it only sleeps, so a long region does not keep the driver
+        busy with queries."""
+        if self._nvml is None:
+            time.sleep(self.MIN_INTERVAL_S)
+            return
+        last = self.stamped[-1][0] if self.stamped else -1e30
+        if time.perf_counter() - last < self.MIN_INTERVAL_S:
+            time.sleep(0.0002)
+            return
+        self._sample()
 
     def _run(self):
         while not self._stop.is_set():
             self._sample()
-            time.sleep(self.period)
+            time.sleep(max(self.period, self.MIN_INTERVAL_S))
 
     def start(self):
         if self._nvml is not None:
@@ -489,7 +499,8 @@ def run_gpu(args, world, rank, local):
             binding.fs_sample_ex(H, W, temperature=wl.temperature, seed=0, row_seeds=rs, step=i,
                                  mask_bits=mask, out_idx=out, workspace=ws, stream=stream)
 
-    # As fast as NVML answers while the region lasts milliseconds; every 5 ms for long runs.
+    # Every 0.5 ms while the region lasts milliseconds; every 5 ms for long runs (the host's
+    # polling loop adds samples at up to the same 0.5 ms rate).
     sampler = ClockSampler(local, period=0.0 if args.steps <= 200 else 0.005)
     with nvtx("fmms: timed steps"):
         region_ms, _ = time_calls(step, args.steps, args.warmup, stream, world, sampler,

@@ -468,6 +468,23 @@ __device__ __forceinline__ uint32_t w_sub_bytes(int rows) {
   return static_cast<uint32_t>((rows + kGranule - 1) / kGranule) * 1024u;
 }
 
+// Transposed pair tiles.  On a CTA pair with a 256-row batch tile, a tile of
+// at most 240 vocabulary rows (a segment's partial tile) runs as logits^T:
+// A = the pair's 256 batch rows of H (each CTA's 128, already staged), B =
+// the tile's rows of W rounded up to n = a multiple of 16, n / 2 from each
+// CTA, so the MMA costs n / 256 of a whole tile's instead of all of it.
+// Accumulator lane = batch row, column j = vocabulary row tile.start + j.
+// Returns n, or 0 for a tile that runs as usual.
+template <int BN, bool PAIR>
+__device__ __forceinline__ int transposed_cols(const Tile &t) {
+  if constexpr (!PAIR || BN != 2 * kTileM) {
+    return 0;
+  } else {
+    const int n = (t.hi - t.start + 15) & ~15;
+    return n < BN ? n : 0;
+  }
+}
+
 // The H loads of one stage (this CTA's rows of the batch operand).
 template <int BN, int MODE, bool PAIR, bool MERGE = false>
 __device__ __forceinline__ void issue_h(const CUtensorMap *th, const FmmsParams &p,
@@ -535,7 +552,12 @@ __device__ __forceinline__ void role_producer(const CUtensorMap *tw, const PartM
   bool ok = p.test_no_loads == 0;
   while (ok && it.next(tile)) {
     const bool merged = C::kMerge && tile.pstart >= 0;
-    const Tile mine = PAIR ? pair_half(tile, rank) : tile;
+    const int tn = transposed_cols<BN, PAIR>(tile);
+    Tile mine = PAIR ? pair_half(tile, rank) : tile;
+    if (tn != 0) {  // each CTA of the pair: n / 2 rows from tile.start + rank n / 2
+      mine.start = tile.start + rank * (tn / 2);
+      mine.hi = mine.start + tn / 2;
+    }
     const int rows = mine.hi - mine.start;
     const int nbox8 = rows > 0 ? (rows + kGranule - 1) / kGranule : 0;
     // 16 granules (a tile cut short by fewer than 8 rows at the end of a
@@ -553,7 +575,7 @@ __device__ __forceinline__ void role_producer(const CUtensorMap *tw, const PartM
     uint32_t sub_bytes = w_sub_bytes(rows) + C::kSubH + (merged ? C::kSubP : 0u);  // this CTA's
     if (PAIR) {
       const Tile other = pair_half(tile, 1 - rank);
-      sub_bytes += w_sub_bytes(other.hi - other.start) + C::kSubH;
+      sub_bytes += (tn != 0 ? w_sub_bytes(tn / 2) : w_sub_bytes(other.hi - other.start)) + C::kSubH;
     }
     const int nks = (p.nk + C::kSub - 1) / C::kSub;
     for (int ks = 0; ks < nks; ++ks) {
@@ -696,6 +718,11 @@ __device__ __forceinline__ void role_mma(const FmmsParams &p, const Schedule &sc
     sm100::tc_fence_after();
     const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
     const uint32_t d_tmem2 = tmem_base + static_cast<uint32_t>(buf2 * BN);
+    // A transposed tile swaps the operands (H sub-blocks and W sub-blocks have
+    // the same size there) and multiplies 256 x n.
+    const int tn = transposed_cols<BN, PAIR>(tile);
+    static_assert(!PAIR || BN != 2 * kTileM || C::kSubH == C::kSubW, "transposed operand strides");
+    const uint32_t idesc = tn != 0 ? sm100::idesc_bf16_f32(2 * kTileM, tn) : C::kIdesc;
     const int nks = (p.nk + C::kSub - 1) / C::kSub;
     for (int ks = 0; ks < nks; ++ks) {
       if (!sm100::wait_bounded<PAIR>(&full[stage], phase, abort_flag, p.err)) {
@@ -707,8 +734,10 @@ __device__ __forceinline__ void role_mma(const FmmsParams &p, const Schedule &sc
       // Descriptor low words of this stage's operands; each MMA below adds a
       // compile-time offset (in 16-byte units) to them.
       const uint32_t p_lo = stage_lo + static_cast<uint32_t>(stage * (C::kStageBytes >> 4));
-      const uint32_t a_lo = p_lo + (C::kOffW >> 4);
-      const uint32_t b_lo = p_lo + (C::kOffH >> 4);
+      const uint32_t w_lo = p_lo + (C::kOffW >> 4);
+      const uint32_t h_lo = p_lo + (C::kOffH >> 4);
+      const uint32_t a_lo = tn != 0 ? h_lo : w_lo;
+      const uint32_t b_lo = tn != 0 ? w_lo : h_lo;
       if (nsub == C::kSub) {
         // A full stage: every K step unrolled, only the tile's first MMA
         // overwrites the accumulator.
@@ -718,8 +747,7 @@ __device__ __forceinline__ void role_mma(const FmmsParams &p, const Schedule &sc
           for (int kk = 0; kk < kBlockK / 16; ++kk) {
             const uint32_t acc = (j | kk) != 0 ? 1u : (ks != 0 ? 1u : 0u);
             sm100::mma_bf16_lo<PAIR>(d_tmem, a_lo + ((j * C::kSubW + kk * 32) >> 4),
-                                     b_lo + ((j * C::kSubH + kk * 32) >> 4), desc_hi, C::kIdesc,
-                                     acc);
+                                     b_lo + ((j * C::kSubH + kk * 32) >> 4), desc_hi, idesc, acc);
           }
         }
       } else {
@@ -732,8 +760,7 @@ __device__ __forceinline__ void role_mma(const FmmsParams &p, const Schedule &sc
           for (int kk = 0; kk < kBlockK / 16; ++kk) {
             const uint32_t acc = (ks | j | kk) != 0 ? 1u : 0u;
             sm100::mma_bf16_lo<PAIR>(d_tmem, a_lo + ((j * C::kSubW + kk * 32) >> 4),
-                                     b_lo + ((j * C::kSubH + kk * 32) >> 4), desc_hi, C::kIdesc,
-                                     acc);
+                                     b_lo + ((j * C::kSubH + kk * 32) >> 4), desc_hi, idesc, acc);
           }
         }
       }
@@ -791,6 +818,217 @@ __device__ __forceinline__ void role_mma(const FmmsParams &p, const Schedule &sc
   }
 }
 
+// Mask bits of row b (of this launch) for the 4 tokens from vg0 (a multiple
+// of 4, so they lie in one mask word): bit m for token vg0 + m; all set
+// without a mask.
+__device__ __forceinline__ uint32_t row_mask4(const FmmsParams &p, int b, int vg0) {
+  if (p.mask == nullptr) return 0xFu;
+  const int w = vg0 >> 5;
+  if (!FS_IN_BOUNDS(p.err, p.b_off + b, p.rows_total) || w >= p.mask_words) return 0u;
+  return (__ldg(p.mask + static_cast<size_t>(p.b_off + b) * p.mask_words + w) >> (vg0 & 31)) & 0xFu;
+}
+
+// The Philox key of row b: its own seed, or the call's.
+__device__ __forceinline__ uint64_t row_key64(const FmmsParams &p, int b) {
+  const uint32_t bg = static_cast<uint32_t>(p.b_off + b);
+  if (p.row_seeds != nullptr && FS_IN_BOUNDS(p.err, bg, p.rows_total)) return __ldg(p.row_seeds + bg);
+  return p.seed;
+}
+
+// Best packed key of row b over the 4 tokens from vg0 (a multiple of 4) whose
+// bit is set in `allowed`, with noise tag `tag`: one Philox call, whose word
+// m is token vg0 + m's (the words chunk_noise hands out).  The filter of
+// chunk_any_candidate comes first: only when some element's upper bound
+// reaches the score of `thr_key` (computed exactly) are the exact scores
+// computed.  0 when none passes.
+__device__ __forceinline__ uint64_t row_best4(const uint32_t (&acc)[4], const FmmsParams &p, int b,
+                                              int vg0, uint32_t tag, uint64_t k64,
+                                              uint32_t allowed, uint64_t thr_key) {
+  const Philox4 ph = philox4x32_10(static_cast<uint32_t>(vg0) >> 2, static_cast<uint32_t>(p.b_off + b),
+                                   p.step, tag, static_cast<uint32_t>(k64),
+                                   static_cast<uint32_t>(k64 >> 32));
+  const uint32_t w[4] = {ph.w0, ph.w1, ph.w2, ph.w3};
+  const float thr = key_valid(thr_key) ? __uint_as_float(key_score_bits(thr_key)) : -INFINITY;
+  bool any = false;
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const float ub = fmaf(__uint_as_float(acc[m]), p.inv_temp, gumbel_upper_bound(w[m]));
+    any = any || (((allowed >> m) & 1u) && ub >= thr);
+  }
+  if (!any) return 0ull;
+  uint64_t best = 0ull;
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    if (!((allowed >> m) & 1u)) continue;
+    const float sc = fmaf(__uint_as_float(acc[m]), p.inv_temp, gumbel_from_u32(w[m]));
+    const uint64_t key = pack_key(__float_as_uint(sc), vg0 + m);
+    best = key > best ? key : best;
+  }
+  return best;
+}
+
+// Mask bits of row b (of this launch) for the 16 tokens from vg0 (a multiple
+// of 8): bit j for token vg0 + j; all set without a mask.
+__device__ __forceinline__ uint32_t row_mask16(const FmmsParams &p, int b, int vg0) {
+  if (p.mask == nullptr) return 0xFFFFu;
+  if (!FS_IN_BOUNDS(p.err, p.b_off + b, p.rows_total)) return 0u;
+  const uint32_t *row = p.mask + static_cast<size_t>(p.b_off + b) * p.mask_words;
+  const int w0 = vg0 >> 5;
+  const int sh = vg0 & 31;
+  const uint32_t lo = w0 < p.mask_words ? __ldg(row + w0) : 0u;
+  const uint32_t hi = (sh > 16 && w0 + 1 < p.mask_words) ? __ldg(row + w0 + 1) : 0u;
+  return (sh == 0 ? lo : ((lo >> sh) | (hi << (32 - sh)))) & 0xFFFFu;
+}
+
+// Best packed key of row b over the 16 tokens from vg0 (a multiple of 8)
+// whose bit is set in `allowed`, noise tag `tag`: the filter over all 16
+// first (four Philox calls, word m of call i for token vg0 + 4 i + m), then,
+// only when some upper bound reaches the score of `thr_key`, the exact scores
+// of the groups of four that hold an allowed token, their noise drawn again.
+// 0 when none passes.  The exact pass is a loop that is not unrolled: it
+// runs rarely, and indexing acc in it keeps acc in local memory there instead
+// of in registers that the hot path needs.
+__device__ __forceinline__ uint64_t row_best16(const uint32_t (&acc)[16], const FmmsParams &p,
+                                               int b, int vg0, uint32_t tag, uint64_t k64,
+                                               uint32_t allowed, uint64_t thr_key) {
+  const float thr = key_valid(thr_key) ? __uint_as_float(key_score_bits(thr_key)) : -INFINITY;
+  bool any = false;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const Philox4 ph = philox4x32_10((static_cast<uint32_t>(vg0) >> 2) + static_cast<uint32_t>(i),
+                                     static_cast<uint32_t>(p.b_off + b), p.step, tag,
+                                     static_cast<uint32_t>(k64), static_cast<uint32_t>(k64 >> 32));
+    const uint32_t w[4] = {ph.w0, ph.w1, ph.w2, ph.w3};
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const float ub = fmaf(__uint_as_float(acc[4 * i + m]), p.inv_temp, gumbel_upper_bound(w[m]));
+      any = any || (((allowed >> (4 * i + m)) & 1u) && ub >= thr);
+    }
+  }
+  if (!any) return 0ull;
+  uint64_t best = 0ull;
+#pragma unroll 1
+  for (int i = 0; i < 4; ++i) {
+    if (((allowed >> (4 * i)) & 0xFu) == 0u) continue;
+    const Philox4 ph = philox4x32_10((static_cast<uint32_t>(vg0) >> 2) + static_cast<uint32_t>(i),
+                                     static_cast<uint32_t>(p.b_off + b), p.step, tag,
+                                     static_cast<uint32_t>(k64), static_cast<uint32_t>(k64 >> 32));
+    const uint32_t w[4] = {ph.w0, ph.w1, ph.w2, ph.w3};
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int j = 4 * i + m;
+      if (!((allowed >> j) & 1u)) continue;
+      const float sc = fmaf(__uint_as_float(acc[j]), p.inv_temp, gumbel_from_u32(w[m]));
+      const uint64_t key = pack_key(__float_as_uint(sc), vg0 + j);
+      best = key > best ? key : best;
+    }
+  }
+  return best;
+}
+
+// Grouped-mode epilogue of a transposed pair tile (see transposed_cols): the
+// thread owns batch row b (its TMEM lane) and walks the tile's n columns in
+// 16-column chunks (h, h + 4, ... among the warps of its lane quarter), with
+// no exchange between lanes, and folds the row's (best key, max, sum) over the
+// tile into comb slot h of column b.  The tile is the first of its segment;
+// the caller synchronises the epilogue warps before the next tile reads the
+// slots.  (In this mode 16-column chunks ran faster than four-column ones.)
+template <int BN>
+__device__ __forceinline__ void epi_transposed_grouped(const FmmsParams &p, const Tile &t, int tn,
+                                                       uint32_t tbase, int b, int h, int unit,
+                                                       float c1, uint64_t *comb_key,
+                                                       float *comb_m, float *comb_s) {
+  constexpr int kWpq = kNumEpiWarps / 4;
+  const bool row_ok = b < p.B;
+  const uint64_t k64 = row_ok ? row_key64(p, b) : 0ull;
+  uint64_t g_best = 0ull;
+  float g_m = -INFINITY, g_s = 0.f;
+  unsigned long long *gk = nullptr;
+  const long long gki = static_cast<long long>(t.slot - unit) * p.B + b;
+  if (p.gkeys != nullptr && row_ok && FS_IN_BOUNDS(p.err, gki, p.gkeys_cap)) gk = p.gkeys + gki;
+  uint64_t g_pub = 0ull;
+  for (int col0 = 16 * h; col0 < tn; col0 += 16 * kWpq) {  // warp-uniform
+    uint32_t acc[16];
+    if (!FS_IN_BOUNDS(p.err, col0 + 15, BN)) continue;
+    sm100::tmem_ld_16(tbase + col0, acc);
+    sm100::tmem_wait_ld();
+    if (!row_ok) continue;
+    const int v0 = t.start + col0;
+    uint32_t in_range = 0u;
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (v0 + j >= t.lo && v0 + j < t.hi) in_range |= 1u << j;
+    if (in_range == 0u) continue;
+    const int vg0 = v0 + p.vocab_offset;
+    const uint32_t allowed = in_range & row_mask16(p, b, vg0);
+    // log-sum-exp pieces in base 2
+    float cm = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if ((allowed >> j) & 1u) cm = fmaxf(cm, __uint_as_float(acc[j]) * c1);
+    if (cm != -INFINITY) {
+      float cs = 0.f;
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        if ((allowed >> j) & 1u) cs += ex2_approx(__uint_as_float(acc[j]) * c1 - cm);
+      lse2_merge(g_m, g_s, cm, cs);
+    }
+    if (gk != nullptr && g_pub == 0ull) g_pub = ld_key(gk);
+    const uint64_t best =
+        row_best16(acc, p, b, vg0, 0u, k64, allowed, g_pub > g_best ? g_pub : g_best);
+    if (key_valid(best) && best > g_best) g_best = best;
+  }
+  if (row_ok) {
+    if (gk != nullptr && key_valid(g_best) && g_best > g_pub)
+      atomicMax(gk, static_cast<unsigned long long>(g_best));
+    const int si = h * BN + b;
+    if (g_best > comb_key[si]) comb_key[si] = g_best;
+    float m = comb_m[si], s = comb_s[si];
+    lse2_merge(m, s, g_m, g_s);
+    comb_m[si] = m;
+    comb_s[si] = s;
+  }
+}
+
+// Flat-mode epilogue of a transposed pair tile (see transposed_cols): the
+// thread owns batch row b (its TMEM lane) and walks the tile's n columns four
+// at a time, the warps of a lane quarter taking 16-column chunks in turn (h,
+// h + 4, ...), with no exchange between lanes; each sample's row maximum is
+// published at once.  Four columns at a time keep this cold path within a few
+// registers: it shares the kernel's register budget with the hot one.
+template <int BN>
+__device__ __forceinline__ void epi_transposed_flat(const FmmsParams &p, const Tile &t, int tn,
+                                                    uint32_t tbase, int b, int h) {
+  constexpr int kWpq = kNumEpiWarps / 4;
+  const bool row_ok = b < p.B;
+  const uint64_t k64 = row_ok ? row_key64(p, b) : 0ull;
+#pragma unroll 1
+  for (int c = 16 * h; c < tn; c += (c & 15) == 12 ? 16 * kWpq - 12 : 4) {  // warp-uniform
+    uint32_t acc[4];
+    if (!FS_IN_BOUNDS(p.err, c + 3, BN)) continue;
+    sm100::tmem_ld_4(tbase + c, acc);
+    sm100::tmem_wait_ld();
+    const int v0 = t.start + c;
+    uint32_t allowed = 0u;
+#pragma unroll
+    for (int m = 0; m < 4; ++m)
+      if (row_ok && v0 + m >= t.lo && v0 + m < t.hi) allowed |= 1u << m;
+    if (allowed == 0u) continue;
+    const int vg0 = v0 + p.vocab_offset;
+    allowed &= row_mask4(p, b, vg0);
+    if (allowed == 0u) continue;
+#pragma unroll 1
+    for (int smp = 0; smp < p.num_samples; ++smp) {
+      if (!FS_IN_BOUNDS(p.err, smp * kMaxBN + b, p.keys_cap)) continue;
+      unsigned long long *kp = p.keys + smp * kMaxBN + b;
+      const uint64_t pub = ld_key(kp);
+      const uint64_t best =
+          row_best4(acc, p, b, vg0, 2u * static_cast<uint32_t>(smp), k64, allowed, pub);
+      if (key_valid(best) && best > pub) atomicMax(kp, static_cast<unsigned long long>(best));
+    }
+  }
+}
+
 // Epilogue warps.  In pair mode each CTA drains its own 128 accumulator rows
 // (its half of the pair tile); the even CTA's MMA commit signals a filled
 // accumulator to both CTAs, and the odd CTA's warps release it on the even
@@ -839,7 +1077,20 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
     // warp-collective.
     const bool got = aborted ? false : sm100::wait_bounded<PAIR>(&acc_full[buf], phase, abort_flag, p.err);
     aborted = __any_sync(0xffffffffu, !got);
-    if (!aborted) {
+    const int tn = transposed_cols<BN, PAIR>(cur);
+    if (!aborted && tn != 0) {
+      sm100::tc_fence_after();
+      if constexpr (MODE != kModeLogits) {
+        const uint32_t tb =
+            tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(buf * BN);
+        const int b = rank * kTileM + 32 * q + lane;  // this thread's batch row
+        if constexpr (MODE == kModeGrouped) {
+          epi_transposed_grouped<BN>(p, cur, tn, tb, b, h, unit, c1, comb_key, comb_m, comb_s);
+        } else {
+          epi_transposed_flat<BN>(p, cur, tn, tb, b, h);
+        }
+      }
+    } else if (!aborted) {
       sm100::tc_fence_after();
       const Tile mine = PAIR ? pair_half(cur, rank) : cur;
       const int v = mine.start + 32 * q + lane;           // row of W in this launch
@@ -928,6 +1179,8 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
           }
         }
       }
+    }
+    if (!aborted) {
       sm100::tc_fence_before();
       __syncwarp();
       if (lane == 0) {
@@ -947,6 +1200,8 @@ __device__ __forceinline__ void role_epilogue(const FmmsParams &p, const Schedul
     run_acc(tile);
     // A merged partial comes as a second accumulator after its whole tile.
     if (C::kMerge && tile.pstart >= 0) run_acc(partial_of(tile));
+    // A transposed tile wrote other warps' slots of the segment's state.
+    if (MODE == kModeGrouped && transposed_cols<BN, PAIR>(tile) != 0) sm100::epi_sync(kEpiThreads);
 
     if constexpr (MODE == kModeGrouped) {
       if (tile.last) {
