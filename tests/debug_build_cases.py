@@ -6,7 +6,9 @@ check their global, shared and tensor-memory indices and record
 FS_ERR_DEVICE_BOUNDS in the status word instead of trapping.  For every shape
 (B in {1, 3, 17}, V in {1, 7, 129, 4097}, d in {8, 24}) and every kind of call
 (flat with mask and row seeds, on single CTAs and CTA pairs; grouped; several
-samples; unfused; top-k; vocabulary shards) the status word must read FS_OK
+samples; unfused; top-k; vocabulary shards), and for 250 and 256 rows (CTA
+pairs whose partial tiles run transposed; V up to 18952) with the flat,
+grouped, multi-sample and shard calls, the status word must read FS_OK
 and the tokens must match the oracle under the stated tie rule.  Prints one
 line per shape and exits non-zero on the first failure.
 """
@@ -103,6 +105,50 @@ def main():
                 parity(got.cpu().numpy(), *ref, what + " shards")
                 n += 1
                 print("ok", what, flush=True)
+    # 241-256 rows: CTA pairs with a 256-row batch tile, whose partial tiles
+    # run transposed (every unit's range is a single partial tile for the
+    # small vocabularies, an 8-row one beside whole tiles for V = 18952).
+    for V in (1, 7, 129, 4097, 18952):
+        for B in (250, 256):
+            d = 24
+            seed = 7000 + 10 * V + B
+            H = synth.make_hidden(B, d, seed=seed)
+            W = synth.make_weight(V, d, 0.5, seed=seed + 1)
+            Hd, Wd = H.to(dev), W.to(dev)
+            rs = synth.make_row_seeds(B)
+            mask = synth.make_mask(B, V, 0.5, seed=seed + 2)
+            rsd, md = rs.to(dev), mask.to(dev)
+            what = "B=%d d=%d V=%d" % (B, d, V)
+            assert binding.fs_uses_cta_pairs(B), what
+            ref = oracle.sample(H, W, T=0.9, seed=3, row_seeds=rs, step=1, mask=mask)
+            got = binding.fs_sample_ex(Hd, Wd, temperature=0.9, seed=3, row_seeds=rsd, step=1,
+                                       mask_bits=md)
+            status_ok(what + " flat")
+            parity(got.cpu().numpy(), *ref, what + " flat")
+            G = min(3, V)
+            g = binding.fs_sample_grouped(Hd, Wd, G, temperature=0.9, seed=3, row_seeds=rsd,
+                                          step=1, mask_bits=md)
+            status_ok(what + " grouped")
+            gi, gs, gm = oracle.sample_grouped(H, W, G, T=0.9, seed=3, row_seeds=rs, step=1,
+                                               mask=mask)
+            gg = g.cpu().numpy()
+            for b in np.flatnonzero(gg != gi):
+                scale = TIE_REL * (1 + abs(gs[b, :, 0].max()))
+                assert gm[b, 0] <= scale or gm[b, 1] <= scale, (what, "grouped", b)
+            got = binding.fs_sample_multi(Hd, Wd, 2, temperature=0.9, seed=3, row_seeds=rsd,
+                                          step=1, mask_bits=md)
+            status_ok(what + " multi")
+            parity(got.cpu().numpy(), *oracle.sample_multi(H, W, 2, T=0.9, seed=3, row_seeds=rs,
+                                                           step=1, mask=mask), what + " multi")
+            keys = [binding.fs_sample_shard_keys(Hd, Wd[lo:hi].contiguous(), lo, V,
+                                                 temperature=0.9, seed=3, row_seeds=rsd, step=1,
+                                                 mask_bits=md)
+                    for lo, hi in shard_bounds(V, 2) if hi > lo]
+            got = binding.fs_keys_to_tokens(torch.stack(keys).max(dim=0).values.contiguous())
+            status_ok(what + " shards")
+            parity(got.cpu().numpy(), *ref, what + " shards")
+            n += 1
+            print("ok", what, flush=True)
     print("debug build: %d shapes, every call FS_OK and oracle parity" % n, flush=True)
 
 
