@@ -572,6 +572,11 @@ def run_gpu(args, world, rank, local):
         with nvtx("fmms: sustained decode"):
             result["sustained"] = sustained_point(torch, binding, synth, W, wl, dev, stream, peaks,
                                                   peak_kind, local)
+        with nvtx("fmms: sustained large batch"):
+            # the tensor-bound batch over a long region, against the sustained bf16 peak
+            result["sustained_b256"] = sustained_point(torch, binding, synth, W, wl, dev, stream,
+                                                       peaks, peak_kind, local, B=256,
+                                                       est_us=300.0)
         # The other LM-head shapes, each at its own batch sizes.
         result["sweeps"] = {}
         for other in ("qwen3-1.7b", "large"):
@@ -664,12 +669,13 @@ def library_gemm_points(torch, synth, W, wl, dev, batches=(64, 128, 256), steps=
 
 
 def sustained_point(torch, binding, synth, W, wl, dev, stream, peaks, peak_kind, local, B=64,
-                    seconds=2.5):
-    """The decode regime: B=64 calls back to back for `seconds` (the board
-    sits at its power limit and the SM clock gives way), with the clocks
-    sampled throughout.  Reports the kernel time, the median SM clock, the
-    kernel time in clock cycles (time x median MHz) and the roofline against
-    the copy bandwidth."""
+                    seconds=2.5, est_us=200.0):
+    """A long run: calls of B rows back to back for about `seconds` (est_us:
+    the expected time per call; the board sits at its power limit and the SM
+    clock gives way), with the clocks sampled throughout.  Reports the kernel
+    time, the median SM clock, the kernel time in clock cycles (time x median
+    MHz) and the roofline of the sustained regime: the copy bandwidth, or
+    the sustained bf16 peak where the matmul bounds the call."""
     H = synth.make_hidden(B, wl.d, device=dev)
     rs = synth.make_row_seeds(B, device=dev) if wl.per_row_seeds else None
     out = torch.empty(B, dtype=torch.int32, device=dev)
@@ -678,7 +684,7 @@ def sustained_point(torch, binding, synth, W, wl, dev, stream, peaks, peak_kind,
         binding.fs_sample_ex(H, W, temperature=wl.temperature, seed=0, row_seeds=rs, step=i,
                              out_idx=out, stream=stream)
 
-    calls = max(100, int(seconds / 200e-6))
+    calls = max(100, int(seconds / (est_us * 1e-6)))
     sampler = ClockSampler(local, period=0.01)
     region_ms, _ = time_calls(step, calls, 20, stream, sampler=sampler, per_call=False)
     kus = region_ms * 1e3 / calls
@@ -690,7 +696,7 @@ def sustained_point(torch, binding, synth, W, wl, dev, stream, peaks, peak_kind,
             "reasons": clk["reasons"],
             "kcycles_per_call": round(kus * clk["sm_mhz"] / 1e3, 1) if clk["sm_mhz"] else None,
             "bound": rf["bound"], "achieved": round(rf["achieved"], 1), "unit": rf["unit"],
-            "frac": round(rf["frac"], 4), "regime": rf["regime"]}
+            "frac": round(rf["frac"], 4), "fracs": rf["fracs"], "regime": rf["regime"]}
 
 
 def grouped_points(torch, binding, synth, dev, stream, peaks, peak_kind, W8, steps=100):
