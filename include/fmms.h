@@ -438,7 +438,10 @@ fs_status fs_test_inject_fault(int kind, int *previous);
  * (fs_sample_grouped, fs_summarize_group) run the fused kernel on CTA pairs:
  * clusters of two CTAs on two SMs that share one M = 256 tensor-core MMA
  * (tcgen05 cta_group::2), each SM staging 128 rows of W and half of the batch
- * rows of H per pipeline stage.  This is a B200 design choice, not part of
+ * rows of H per pipeline stage.  On pairs with a 256-row batch tile, a
+ * partial tile of at most 240 vocabulary rows is multiplied transposed (the
+ * batch rows as the MMA's M operand), so that it costs its own width of MMA
+ * work rather than a whole tile's.  This is a B200 design choice, not part of
  * the method: the results are the same either way (tokens bit for bit).
  * policy: -1 automatic (the default: pairs for launches whose batch tile,
  * the row count rounded up to a multiple of 16, is 112 or more, i.e. from
