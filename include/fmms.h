@@ -505,7 +505,12 @@ fs_status fs_set_partial_merge(int policy);
  * max_tiles rows of int32 [5] = (tile start, first valid token, end of valid
  * tokens, partial slot, last-tile-of-segment flag) for CTA `cta` and returns
  * the count in *ntiles.  Tiles are 128 tokens; a CTA's range is a multiple
- * of 8 tokens (except at V); a tile never crosses a group boundary.  (With
+ * of 8 tokens (except at V); a tile never crosses a group boundary.  A launch
+ * on CTA pairs splits the vocabulary over its pair units in the same way
+ * (the query with num_sms = the number of units, 74 on a 148-SM device) and
+ * walks each segment in 256-token tiles, its partial tile first; with a
+ * 256-row batch tile a partial tile of at most 240 tokens is multiplied
+ * transposed (see fs_set_cta_pairs).  (With
  * merged partial tiles, fs_set_partial_merge, the kernel multiplies an 8-row
  * partial tile in the same pipeline stages as the tile after it; the tiles
  * and slots listed here stay the same.) */
